@@ -1,0 +1,452 @@
+"""Pins of the float64 oracle to facts fixed by the STAR-KV pages and by mathematics.
+
+Each test checks the oracle against something other than itself: a closed form,
+an identity the pages state, a brute-force enumeration, a library routine for a
+special case, or bytes derived by hand (tests/golden).  The last section plants
+plausible mistakes in the oracle and checks that these pins catch them.
+"""
+import copy
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+
+from oracle import starkv_oracle as O
+from synth import gen
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def small_spec(**kw):
+    base = dict(hidden=32, n_heads=2, n_kv_heads=2, head_dim=8, key_ranks=[3, 5], value_rank=6, dtype="f32")
+    base.update(kw)
+    return gen.LayerSpec(**base)
+
+
+# ---------------------------------------------------------------------------
+# Number formats
+# ---------------------------------------------------------------------------
+
+def test_bf16_round_matches_torch():
+    # Special case that reduces to a library routine: torch's float32 -> bfloat16 cast is RNE.
+    x = np.concatenate([gen.normals(gen.stream_key(5, 99), 20000) * 10.0 ** np.arange(-3, 3).repeat(20000 // 6 + 1)[:20000],
+                        np.array([0.0, -0.0, 1.0 + 2 ** -8, 1.0 + 3 * 2 ** -8, 1.0 + 2 ** -9])]).astype(np.float32)
+    ref = torch.from_numpy(x).to(torch.bfloat16).to(torch.float32).numpy()
+    np.testing.assert_array_equal(O.bf16_round(x), ref)
+
+
+def test_fp16_round_up_brute_force():
+    # Exhaustive: the answer is the smallest finite binary16 >= x.
+    halves = np.arange(0, 0x7C00, dtype=np.uint16).view(np.float16).astype(np.float32)  # +0 .. 65504, sorted
+    xs = np.concatenate([gen.uniforms(gen.stream_key(1, 98), 3000) * 70000.0 * (gen.uniforms(gen.stream_key(2, 98), 3000) ** 6),
+                         halves[::97].astype(np.float64), [1e-9, 6e-8, 65504.0]]).astype(np.float32)
+    xs = xs[xs <= 65504.0]
+    for x in xs:
+        want = halves[np.searchsorted(halves, x, side="left")]
+        assert np.float32(O.fp16_round_up(x)) == want, x
+
+
+# ---------------------------------------------------------------------------
+# Quantizer ("STAR-KV 阅读笔记" section 6.1)
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("bits", [3, 4])
+def test_quantizer_error_bound(bits):
+    z = (gen.normals(gen.stream_key(3, 97, bits), 32 * 500) * 3.0).astype(np.float32).reshape(500, 32)
+    for row in z:
+        s16, u = O.quantize_group(row, bits)
+        zh = O.dequantize_group(u, s16, bits)
+        assert np.all(np.abs(row - zh) <= float(s16) / 2 * (1 + 2 ** -20))
+        assert u.min() >= 1 and u.max() <= (1 << bits) - 1
+        # amax element maps to +-qmax or one below (scale rounded up)
+        assert float(s16) >= float(np.max(np.abs(row))) / ((1 << (bits - 1)) - 1)
+
+
+@pytest.mark.parametrize("bits", [3, 4])
+def test_quantizer_grid_ties_and_zero(bits):
+    qmax = (1 << (bits - 1)) - 1
+    s = np.float32(0.125)
+    grid = np.array([k * s for k in range(-qmax, qmax + 1)], dtype=np.float32)
+    s16, u = O.quantize_group(grid, bits)
+    assert float(s16) == 0.125
+    np.testing.assert_array_equal(u.astype(int) - (1 << (bits - 1)), np.arange(-qmax, qmax + 1))
+    # ties go to even: values (k + 1/2) s with amax fixing s = 0.125
+    ties = np.array([qmax * s] + [(k + 0.5) * s for k in range(-qmax, qmax)], dtype=np.float32)
+    s16, u = O.quantize_group(ties, bits)
+    q = u.astype(int)[1:] - (1 << (bits - 1))
+    for k, qq in zip(range(-qmax, qmax), q):
+        lo, hi = k, k + 1
+        assert qq == (lo if lo % 2 == 0 else hi)
+    s16, u = O.quantize_group(np.zeros(7, dtype=np.float32), bits)
+    assert float(s16) == 0.0 and np.all(u == (1 << (bits - 1)))
+    s16, u = O.quantize_group(np.array([-2.5], dtype=np.float32), bits)
+    assert int(u[0]) - (1 << (bits - 1)) == -qmax
+
+
+def test_groups_and_segments():
+    spec = gen.LayerSpec(hidden=1, n_heads=1, n_kv_heads=1, head_dim=128, key_ranks=[32], value_rank=1024,
+                         quantized=True)
+    g = O.groups(32, spec)
+    assert [(x.start, x.n, x.bits) for x in g] == [(0, 8, 4), (8, 24, 3)]
+    g = O.groups(1024, spec)
+    assert len(g) == 32 and sum(x.bits == 4 for x in g) == 8 and all(x.n == 32 for x in g)
+    g = O.groups(56, spec)  # n_hi = 14
+    assert [(x.start, x.n, x.bits) for x in g] == [(0, 14, 4), (14, 32, 3), (46, 10, 3)]
+
+
+# ---------------------------------------------------------------------------
+# Page format: hand-derived golden bytes
+# ---------------------------------------------------------------------------
+
+def _read_golden(name):
+    meta, hexes = {}, []
+    with open(os.path.join(GOLDEN, name)) as f:
+        for line in f:
+            if line.startswith("#") or not line.strip():
+                continue
+            k, *v = line.split()
+            if k == "hex":
+                hexes.append((int(v[0]), [int(x, 16) for x in v[1:]]))
+            else:
+                meta[k] = v
+    return meta, hexes
+
+
+def test_pack_block_golden_bytes():
+    meta, hexes = _read_golden("pack_r6_two_slots.txt")
+    r = int(meta["r"][0])
+    spec = gen.LayerSpec(hidden=1, n_heads=1, n_kv_heads=1, head_dim=8, key_ranks=[r], value_rank=r,
+                         quantized=True, top_fraction=float(meta["top_fraction"][0]))
+    Z = np.full((16, r), np.nan, dtype=np.float32)
+    Z[0] = [float(x) for x in meta["slot0"]]
+    Z[1] = [float(x) for x in meta["slot1"]]
+    blk = O.pack_block(Z, r, spec)
+    want = np.zeros(int(meta["bytes"][0]), dtype=np.uint8)
+    for off, bs in hexes:
+        want[off:off + len(bs)] = bs
+    np.testing.assert_array_equal(blk, want)
+
+
+def test_pack_roundtrip_and_layout():
+    spec = gen.config_spec(2)
+    offs, pb = O.page_layout(spec)
+    assert pb % 128 == 0 and all(o % 16 == 0 for o in offs)
+    # per-token algorithmic bytes: r=32 -> 8*4+24*3 bits + 2 scales = 17 B; r_v=1024 -> 480 B
+    assert O.latent_bytes_per_token(32, spec) == 17.0
+    assert O.latent_bytes_per_token(1024, spec) == 480.0
+    r = spec.key_ranks[0]
+    Z = (gen.normals(gen.stream_key(4, 96), 16 * r).reshape(16, r)).astype(np.float32)
+    blk = O.pack_block(Z, r, spec)
+    gs = O.groups(r, spec)
+    code_off = ((len(gs) * 16 * 2) + 15) // 16 * 16
+    for gi, g in enumerate(gs):
+        for slot in range(16):
+            s16, u = O.quantize_group(Z[slot, g.start:g.start + g.n], g.bits)
+            sb = blk[(gi * 16 + slot) * 2:(gi * 16 + slot) * 2 + 2].view(np.float16)[0]
+            assert sb == s16
+            for i in range(g.n):
+                assert O.read_bits(blk[code_off:], (slot * g.n + i) * g.bits, g.bits) == u[i]
+        code_off += (16 * g.n * g.bits // 8 + 15) // 16 * 16
+
+
+def test_unquantized_block_bf16_layout():
+    spec = gen.config_spec(1)
+    r = 24
+    Z = np.arange(16 * r, dtype=np.float32).reshape(16, r) / 7.0
+    blk = O.pack_block(Z, r, spec)
+    vals = blk[:16 * r * 2].view(np.uint16).astype(np.uint32) << 16
+    np.testing.assert_array_equal(vals.view(np.float32).reshape(16, r),
+                                  torch.from_numpy(Z).to(torch.bfloat16).float().numpy())
+
+
+def test_pool_page_table_permutation():
+    spec = small_spec(quantized=True, hadamard_block=32, key_ranks=[8, 12], value_rank=40)
+    T = 37
+    lat = [[gen.normals(gen.stream_key(9, 95, i), T * r).reshape(T, r).astype(np.float32)
+            for i, r in enumerate(spec.latent_widths)]]
+    pt1, n = gen.page_tables(1, [T], 16, extra_pages=2)
+    pt2, _ = gen.page_tables(2, [T], 16, extra_pages=2)
+    p1 = O.build_pool(spec, lat, pt1, n)
+    p2 = O.build_pool(spec, lat, pt2, n)
+    for j in range(3):
+        np.testing.assert_array_equal(p1[pt1[0][j]], p2[pt2[0][j]])
+    used = set(pt1[0][:3].tolist())
+    for p in range(n):
+        if p not in used:
+            assert not p1[p].any()
+    # the ragged last page: slots 5..15 of page 2 are zero in every latent block
+    offs, pb = O.page_layout(spec)
+    last = p1[pt1[0][2]]
+    for li, r in enumerate(spec.latent_widths):
+        Zs = [lat[0][li][t] if t < T else None for t in range(32, 48)]
+        rows = [None if z is None else [z] for z in Zs]
+        sub = gen.LayerSpec(**{**spec.__dict__, "key_ranks": [r], "n_kv_heads": 1})
+        ref = O.pack_block(np.stack([z if z is not None else np.full(r, np.nan, np.float32) for z in Zs]), r, spec)
+        np.testing.assert_array_equal(last[offs[li]:offs[li] + ref.size], ref)
+
+
+# ---------------------------------------------------------------------------
+# Rotation ("STAR-KV 阅读笔记" section 6.1)
+# ---------------------------------------------------------------------------
+
+def test_hadamard_golden_and_orthogonal():
+    rows = []
+    with open(os.path.join(GOLDEN, "hadamard_6.txt")) as f:
+        for line in f:
+            if line.startswith("#") or not line.strip():
+                continue
+            parts = line.split()
+            norm = float(parts[1])
+            rows.append([float(x) / norm for x in parts[3:]])
+    np.testing.assert_allclose(O.group_rotation(6), np.array(rows), atol=1e-15)
+    for n in (1, 2, 3, 6, 8, 18, 24, 32):
+        R = O.group_rotation(n)
+        np.testing.assert_allclose(R @ R.T, np.eye(n), atol=1e-13)
+        np.testing.assert_allclose(R, R.T, atol=0)
+        np.testing.assert_allclose(R @ R, np.eye(n), atol=1e-13)
+    # H32 entries are +-1/sqrt(32) and the first row is constant
+    R = O.group_rotation(32)
+    assert np.allclose(np.abs(R), 1 / math.sqrt(32)) and np.all(R[0] > 0)
+
+
+def test_absorbed_rotation_leaves_kv_unchanged():
+    spec = small_spec(quantized=True, hadamard_block=32, key_ranks=[20], n_kv_heads=1, n_heads=1, value_rank=40,
+                      head_dim=64, hidden=96)
+    f = gen.make_factors(spec, 3)
+    X = gen.hidden_states(3, 0, 0, 5, spec.hidden)
+    for A, B, r in ((f.A_k[0], f.B_k[0], 20), (f.A_v, f.B_v, 40)):
+        R = O.rotation(r, spec)
+        assert not np.allclose(R, np.eye(r))
+        Z = X @ A @ R                       # float64, before quantization
+        np.testing.assert_allclose(Z @ O.rotated_factor(B, R), X @ A @ B, atol=1e-12)
+
+
+# ---------------------------------------------------------------------------
+# Factors (generator) and decomposition facts ("STAR-KV 阅读笔记" sections 2.2, 5.2)
+# ---------------------------------------------------------------------------
+
+def test_factors_eckart_young_and_frames():
+    D, d, r = 48, 16, 5
+    U = gen.haar_frame(gen.stream_key(7, 94), D, d)
+    V = gen.haar_frame(gen.stream_key(8, 94), d, d)
+    assert np.abs(U.T @ U - np.eye(d)).max() < 1e-12
+    sig = gen.spectrum(d)
+    W = (U * sig) @ V.T
+    A, B = U[:, :r] * sig[:r], V[:, :r].T
+    assert abs(np.linalg.norm(W - A @ B) ** 2 - np.sum(sig[r:] ** 2)) < 1e-12
+    # Eckart-Young: the truncated SVD is the best rank-r approximation (compare with a library SVD)
+    s = np.linalg.svd(W, compute_uv=False)
+    np.testing.assert_allclose(s, sig, atol=1e-12)
+
+
+def test_joint_not_worse_than_headwise():
+    # Feasible-set inclusion ("STAR-KV 阅读笔记" section 5.2): best joint rank-R error <= head-wise.
+    D, d, H, R = 40, 8, 4, 12
+    W = gen.normals(gen.stream_key(11, 93), D * H * d).reshape(D, H * d)
+    s = np.linalg.svd(W, compute_uv=False)
+    joint = np.sum(s[R:] ** 2)
+    hd = sum(np.sum(np.linalg.svd(W[:, h * d:(h + 1) * d], compute_uv=False)[R // H:] ** 2) for h in range(H))
+    assert joint <= hd + 1e-12
+
+
+# ---------------------------------------------------------------------------
+# RoPE
+# ---------------------------------------------------------------------------
+
+def test_rope_closed_form_and_invariances():
+    d, theta = 8, 10000.0
+    e0 = np.eye(d)[0]
+    r = O.rope(e0, 1.0, theta)
+    np.testing.assert_allclose(r, [math.cos(1), 0, 0, 0, math.sin(1), 0, 0, 0], atol=1e-15)
+    e3 = np.eye(d)[3]
+    ang = 5.0 * theta ** (-2 * 3 / d)
+    np.testing.assert_allclose(O.rope(e3, 5.0, theta)[[3, 7]], [math.cos(ang), math.sin(ang)], atol=1e-15)
+    q = gen.normals(gen.stream_key(1, 92), d)
+    k = gen.normals(gen.stream_key(2, 92), d)
+    s1 = O.rope(q, 100, theta) @ O.rope(k, 37, theta)
+    s2 = O.rope(q, 1100, theta) @ O.rope(k, 1037, theta)
+    assert abs(s1 - s2) < 1e-12
+    assert abs(np.linalg.norm(O.rope(q, 12345, theta)) - np.linalg.norm(q)) < 1e-12
+
+
+# ---------------------------------------------------------------------------
+# Attention
+# ---------------------------------------------------------------------------
+
+def _unq_inputs(spec, T, seed=0):
+    f = gen.make_factors(spec, seed)
+    X = gen.hidden_states(seed, 0, 0, T, spec.hidden)
+    Z = [O.project(X, A, np.eye(A.shape[1])) for A in f.A_k] + [O.project(X, f.A_v, np.eye(spec.value_rank))]
+    Zh = [O.stored_values(z, z.shape[1], spec) for z in Z]
+    q = gen.queries(seed, 0, 1, spec.n_heads, spec.head_dim)[0, 0]
+    return f, X, Z, Zh, q
+
+
+def test_full_rank_equals_plain_attention():
+    # r = d with orthogonal factors: attention over latents equals attention computed from W directly.
+    spec = small_spec(key_ranks=[8, 8], value_rank=16, rope=True)
+    T = 9
+    f, X, Z, Zh, q = _unq_inputs(spec, T)
+    out = O.decode(spec, f, Zh, q, T - 1, T)
+    d = spec.head_dim
+    want = np.zeros(spec.hidden)
+    Wv = f.A_v @ f.B_v
+    for h in range(spec.n_heads):
+        K = X @ (f.A_k[h] @ f.B_k[h])
+        K = O.rope(K, np.arange(T), spec.rope_theta)
+        qh = O.rope(q[h], T - 1, spec.rope_theta)
+        s = K @ qh / math.sqrt(d)
+        p = np.exp(s - s.max()); p /= p.sum()
+        want += (p @ (X @ Wv)[:, h * d:(h + 1) * d]) @ f.W_o[h * d:(h + 1) * d]
+    np.testing.assert_allclose(out, want, rtol=1e-5, atol=1e-6)  # float32 rounding of latents only
+
+
+def test_reassociation_and_value_fusion():
+    spec = small_spec(key_ranks=[3, 5], value_rank=6, rope=False)
+    T = 11
+    f, X, Z, Zh, q = _unq_inputs(spec, T, seed=2)
+    out = O.decode(spec, f, Zh, q, T - 1, T)
+    d = spec.head_dim
+    alt = np.zeros(spec.hidden)
+    for h in range(spec.n_heads):
+        u = f.B_k[h] @ q[h]                      # re-associated query (q B^T)
+        s = (Zh[h] @ u) / math.sqrt(d)           # scores straight from the latents
+        p = np.exp(s - s.max()); p /= p.sum()
+        alt += (p @ Zh[-1]) @ O.fused_output_factor(spec, f, h)   # (P Z_v) M_h
+    np.testing.assert_allclose(out, alt, rtol=1e-12, atol=1e-13)
+
+
+def test_attention_special_cases():
+    spec = small_spec(rope=True)
+    d = spec.head_dim
+    f, X, Z, Zh, q = _unq_inputs(spec, 6, seed=4)
+    Bv = O.up_projections(spec, f)[-1]
+    # T = 1: output is v_0 W_o summed over heads
+    out = O.decode(spec, f, Zh, q, 0, 1)
+    V0 = Zh[-1][0] @ Bv
+    want = sum(V0[h * d:(h + 1) * d] @ f.W_o[h * d:(h + 1) * d] for h in range(spec.n_heads))
+    np.testing.assert_allclose(out, want, rtol=1e-12, atol=1e-13)
+    # identical keys (RoPE off): the average of the values
+    spec2 = small_spec(rope=False)
+    Zk = [np.repeat(z[:1], 6, axis=0) for z in Zh[:-1]]
+    out = O.decode(spec2, f, Zk + [Zh[-1]], q, 5, 6)
+    Vm = (Zh[-1] @ Bv).mean(axis=0)
+    want = sum(Vm[h * d:(h + 1) * d] @ f.W_o[h * d:(h + 1) * d] for h in range(spec.n_heads))
+    np.testing.assert_allclose(out, want, rtol=1e-12, atol=1e-13)
+    # one dominant score picks that value: per head, the query is the longest key scaled up
+    # (q . k_t = c k* . k_t < c |k*|^2 for every other, shorter key)
+    Ks = [Zh[h] @ f.B_k[h] for h in range(spec.n_heads)]
+    star = [int(np.argmax(np.linalg.norm(K, axis=1))) for K in Ks]
+    qbig = np.stack([Ks[h][star[h]] * 1e5 for h in range(spec.n_heads)])
+    out = O.decode(spec2, f, Zh, qbig, 5, 6)
+    V = Zh[-1] @ Bv
+    want = sum(V[star[h], h * d:(h + 1) * d] @ f.W_o[h * d:(h + 1) * d] for h in range(spec.n_heads))
+    np.testing.assert_allclose(out, want, rtol=1e-9, atol=1e-10)
+    # token permutation invariance when RoPE is off
+    perm = np.array([4, 0, 5, 2, 1, 3])
+    out1 = O.decode(spec2, f, Zh, q, 5, 6)
+    out2 = O.decode(spec2, f, [z[perm] for z in Zh], q, 5, 6)
+    np.testing.assert_allclose(out1, out2, rtol=1e-12, atol=1e-14)
+
+
+def test_brute_force_tiny():
+    # T = 2, d = 4, r = 1, one head, no RoPE: closed form p0 = 1 / (1 + exp(s1 - s0)).
+    spec = gen.LayerSpec(hidden=2, n_heads=1, n_kv_heads=1, head_dim=4, key_ranks=[1], value_rank=1, dtype="f32")
+    f = gen.LayerFactors(A_k=[None], B_k=[np.array([[1.0, 0, 0, 0]])], A_v=None,
+                         B_v=np.array([[0.0, 2.0, 0, 0]]), W_o=np.array([[1.0, 0], [0, 3.0], [0, 0], [0, 0]]))
+    Zh = [np.array([[2.0], [-1.0]]), np.array([[1.0], [5.0]])]
+    q = np.array([[1.5, 0, 0, 0]])
+    out = O.decode(spec, f, Zh, q, 1, 2)
+    s0, s1 = 1.5 * 2.0 / 2.0, 1.5 * -1.0 / 2.0
+    p0 = 1.0 / (1.0 + math.exp(s1 - s0))
+    v0, v1 = np.array([0, 2.0, 0, 0]), np.array([0, 10.0, 0, 0])
+    y = p0 * v0 + (1 - p0) * v1
+    np.testing.assert_allclose(out, [y[0], 3.0 * y[1]], rtol=1e-14)
+
+
+def test_prefill_is_causal():
+    spec = small_spec(rope=True)
+    f, X, Z, Zh, q = _unq_inputs(spec, 7, seed=6)
+    Q = gen.queries(6, 0, 1, spec.n_heads, spec.head_dim, n_pos=7)[0]
+    out = O.prefill(spec, f, Zh, Q, 0)
+    # query 0 sees only token 0
+    np.testing.assert_allclose(out[0], O.decode(spec, f, [z[:1] for z in Zh], Q[0], 0, 1), rtol=1e-13)
+    # changing future tokens does not change earlier outputs
+    Zh2 = [z.copy() for z in Zh]
+    for z in Zh2:
+        z[5:] += 3.0
+    out2 = O.prefill(spec, f, Zh2, Q, 0)
+    np.testing.assert_allclose(out[:5], out2[:5], rtol=1e-13)
+    assert not np.allclose(out[5:], out2[5:])
+
+
+def test_stored_values_fast_matches_loop():
+    spec = gen.config_spec(2)
+    Z = (gen.normals(gen.stream_key(12, 91), 40 * 1024).reshape(40, 1024) * 0.3).astype(np.float32)
+    np.testing.assert_array_equal(O.stored_values(Z, 1024, spec), O.stored_values_fast(Z, 1024, spec))
+    Z = Z[:, :56].copy()
+    np.testing.assert_array_equal(O.stored_values(Z, 56, spec), O.stored_values_fast(Z, 56, spec))
+
+
+# ---------------------------------------------------------------------------
+# Ledger ("STAR-KV 阅读笔记" sections 6.1 and 6.2; the arXiv abstract)
+# ---------------------------------------------------------------------------
+
+def test_ledger_numbers_from_the_pages():
+    assert abs(O.average_bits(0.2, 4, 3) - 3.2) < 1e-12
+    assert abs(O.average_bits(0.25, 4, 3) - 3.25) < 1e-12
+    assert abs(O.payload_reduction(0.25, 3.2) - 20.0) < 1e-12      # 75 % rank cut + 3.2 bit
+    assert abs(O.payload_reduction(0.40, 3.2) - 12.5) < 1e-12      # 60 % rank cut + 3.2 bit
+    assert abs(O.mixed_ledger(32, 3, 1 / 20) - 7.19) < 0.005        # 3 exempt layers of 32
+
+
+# ---------------------------------------------------------------------------
+# Planted mistakes: each plausible error in the oracle must fail a pin above.
+# ---------------------------------------------------------------------------
+
+def _fails(test_fn, monkeypatch, target, replacement, *args):
+    with monkeypatch.context() as m:
+        m.setattr(O, target, replacement)
+        with pytest.raises(AssertionError):
+            test_fn(*args)
+
+
+def test_planted_mistakes_are_caught(monkeypatch):
+    good_rope = O.rope
+
+    def rope_wrong_sign(x, pos, theta):
+        x = np.asarray(x, dtype=np.float64)
+        d = x.shape[-1]
+        half = d // 2
+        freq = theta ** (-2.0 * np.arange(half) / d)
+        ang = np.asarray(pos, dtype=np.float64)[..., None] * freq
+        c, s = np.cos(ang), np.sin(ang)
+        a, b = x[..., :half], x[..., half:]
+        return np.concatenate([a * c + b * s, b * c - a * s], axis=-1)
+    _fails(test_rope_closed_form_and_invariances, monkeypatch, "rope", rope_wrong_sign)
+
+    def quant_half_away(z, bits):
+        z = np.asarray(z, dtype=np.float32)
+        qmax = (1 << (bits - 1)) - 1
+        s16 = O.fp16_round_up(np.float32(np.max(np.abs(z)) / np.float32(qmax)))
+        q = np.clip(np.sign(z) * np.floor(np.abs(z / np.float32(s16)) + 0.5), -qmax, qmax).astype(np.int64)
+        return s16, (q + (1 << (bits - 1))).astype(np.uint8)
+    _fails(test_quantizer_grid_ties_and_zero, monkeypatch, "quantize_group", quant_half_away, 3)
+
+    def rot_unnormalised(n):
+        return O.group_rotation.__wrapped__(n) if hasattr(O.group_rotation, "__wrapped__") else \
+            np.kron(np.eye(1), O.sylvester(1 << (n.bit_length() - 1)))[:n, :n]
+    _fails(test_hadamard_golden_and_orthogonal, monkeypatch, "group_rotation", rot_unnormalised)
+
+    def up_no_transpose(spec, f):
+        out = [O.rotation(r, spec) @ f.B_k[h] * 1.0 for h, r in enumerate(spec.key_ranks)]
+        out.append(f.B_v[::-1].copy())    # plausible index mix-up of the value factor rows
+        return out
+    _fails(test_reassociation_and_value_fusion, monkeypatch, "up_projections", up_no_transpose)
+
+    def softmax_no_max(s):
+        e = np.exp(s)
+        return e / np.sum(e, axis=-1, keepdims=True) * 0.999
+    _fails(test_brute_force_tiny, monkeypatch, "softmax", softmax_no_max)
