@@ -1,0 +1,401 @@
+"""Benchmark: STAR-KV latent decode attention on B200.
+
+One step = the whole hot path for one batch: append one new token per sequence
+(projection from the hidden state, block Hadamard, 4/3-bit quantize, bit-pack
+into the paged cache) and one decode-attention step over the compressed cache
+(RoPE'd on-chip key scoring, joint-value contraction, combine, fused output
+factors).  Workload: LongChat-7B-shaped layer (32 heads, head_dim 128, hidden
+4096), ragged key ranks (mean 32), joint value rank 1024, block Hadamard 32,
+4/3-bit latents with fp16 group scales, 16-token pages, batch 16, context 32K.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Multi-GPU (torchrun): each rank runs an independent replica on its own
+sequences (the method has no cross-sequence exchange); value = all ranks'
+tokens / max-over-ranks time.  Prints one JSON line on rank 0.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "latent decode-attn tokens/s & HBM GB/s (% of ~8 TB/s) at ctx 4K-32K, 1 B200"
+WORKLOAD = dict(cfg=2, batch=16, ctx=32768)
+
+
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d.get("hbm_gbs", 6650.0), "measured"
+    return 6650.0, "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled during the timed region."""
+
+    FIELDS = "clocks.sm,clocks.max.sm,clocks_event_reasons.active,clocks_event_reasons.hw_slowdown," \
+             "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown," \
+             "clocks_event_reasons.sw_power_cap"
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                                          "-i", str(self.gpu), "-lms", "100"], stdout=subprocess.PIPE,
+                                         stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except (OSError, FileNotFoundError):
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.t.join(timeout=2)
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 7:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                mx.append(float(parts[1]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[3:7]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def dist_init():
+    import torch
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if ws > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(local)
+    return rank, ws, local
+
+
+def barrier(ws):
+    if ws > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(x: float, ws: int) -> float:
+    if ws == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ---------------------------------------------------------------------------
+# Our arm
+# ---------------------------------------------------------------------------
+
+def build_layer(seed_offset: int = 0):
+    """Seeded layer of the workload, loaded into the library."""
+    import numpy as np
+    import torch
+    from decode_attention_rank_b200 import starkv as lib
+    from synth import gen
+    spec = gen.config_spec(WORKLOAD["cfg"])
+    f = gen.make_factors(spec, gen.LAYER_SEED[WORKLOAD["cfg"]])
+
+    def t(x):
+        return torch.from_numpy(np.ascontiguousarray(x)).cuda().to(torch.bfloat16)
+    A_k = torch.cat([t(a).reshape(-1) for a in f.A_k])
+    B_k = torch.cat([t(b).reshape(-1) for b in f.B_k])
+    L = lib.load_factors(lib.LayerConfig.from_spec(spec), A_k, B_k, t(f.A_v), t(f.B_v), t(f.W_o))
+    torch.cuda.synchronize()
+    return spec, f, L
+
+
+def fill_cache(spec, f, L, B, T0, rank, ctx, tail_pages):
+    """Pool with B sequences of T0 tokens (T0 a multiple of 16), appended in
+    latent mode from seeded latents whose columns have the factor spectrum
+    (column j ~ N(0, sigma_j^2)).  Two page tables share the filled pages and
+    map the tail (positions >= T0) to disjoint zeroed pages, so the timed pass
+    and the end-to-end pass each append into fresh slots."""
+    import torch
+    pages_per_seq = (ctx + 15) // 16
+    head = T0 // 16
+    n_pages = B * pages_per_seq + B * tail_pages
+    g = torch.Generator(device="cuda")
+    g.manual_seed(1000 + rank)
+    perm = torch.randperm(n_pages, generator=g, device="cuda").to(torch.int32)
+    page_table = perm[:B * pages_per_seq].reshape(B, pages_per_seq).contiguous()
+    page_table_e2e = page_table.clone()
+    page_table_e2e[:, head:head + tail_pages] = perm[B * pages_per_seq:].reshape(B, tail_pages)
+    pool = torch.empty(n_pages * L.page_bytes, dtype=torch.uint8, device="cuda")
+    L.cache_init(pool, n_pages)
+    sig = torch.cat([torch.tensor(s[:r], dtype=torch.float32) for s, r in zip(f.sigma_k, spec.key_ranks)] +
+                    [torch.tensor(f.sigma_v[:spec.value_rank], dtype=torch.float32)]).cuda()
+    chunk = 4096
+    for b in range(B):
+        for c0 in range(0, T0, chunk):
+            n = min(chunk, T0 - c0)
+            z = torch.randn(n, L.latent_total, generator=g, device="cuda") * sig
+            seq = torch.full((n,), b, dtype=torch.int32, device="cuda")
+            pos = torch.arange(c0, c0 + n, dtype=torch.int32, device="cuda")
+            L.append(pool, n_pages, page_table, seq, pos, z, True)
+    torch.cuda.synchronize()
+    return pool, n_pages, page_table, page_table_e2e
+
+
+def decode_bytes(spec, L, B, ctx):
+    """Algorithmic HBM bytes of one decode step: cache + B'_k + M + q/out."""
+    return B * ctx * L.bytes_per_token + L.factor_bytes + B * (spec.n_heads * spec.head_dim + spec.hidden) * 2
+
+
+def cpu_baseline(sample_T: int):
+    """Time the float64 oracle on one sequence of the workload (host cores)."""
+    import numpy as np
+    sys.path.insert(0, os.path.join(ROOT, "tests"))
+    from harness import Case, queries
+    from synth import gen
+    c = Case(gen.config_spec(WORKLOAD["cfg"]), gen.LAYER_SEED[WORKLOAD["cfg"]])
+    Z = c.latents_direct(0, sample_T)
+    Zs = c.stored(Z)
+    q = queries(c, 1)[0, 0]
+    c.B_rot
+    t0 = time.perf_counter()
+    c.oracle_decode(Zs, q, sample_T - 1, sample_T)
+    dt = time.perf_counter() - t0
+    try:
+        from threadpoolctl import threadpool_info
+        cores = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
+    except Exception:
+        cores = os.cpu_count()
+    return dt, cores
+
+
+def run_ours(args, rank, ws, local):
+    import torch
+    B, ctx = WORKLOAD["batch"], WORKLOAD["ctx"]
+    K, W = args.steps, args.warmup
+    spec, f, L = build_layer()
+    tail_pages = (W + K + 15) // 16
+    T0 = ctx - 16 * tail_pages      # each step appends one token at T0 + i and decodes T0 + i + 1 tokens
+    pool, n_pages, page_table, page_table_e2e = fill_cache(spec, f, L, B, T0, rank, ctx, tail_pages)
+    dev = torch.device("cuda", torch.cuda.current_device())
+    stream = torch.cuda.current_stream()
+    g = torch.Generator(device="cuda")
+    g.manual_seed(77 + rank)
+    x_all = torch.randn(W + K, B, spec.hidden, generator=g, device=dev).to(torch.bfloat16)
+    q_all = (torch.randn(W + K, B, spec.n_heads, spec.head_dim, generator=g, device=dev) /
+             math.sqrt(spec.head_dim)).to(torch.bfloat16)
+    out = torch.empty(B, spec.hidden, dtype=torch.bfloat16, device=dev)
+    ws_dec = torch.empty(L.workspace_bytes(B, page_table.shape[1] * 16), dtype=torch.uint8, device=dev)
+    ws_app = torch.empty(max(L.append_workspace_bytes(B), 256), dtype=torch.uint8, device=dev)
+    seq_idx = torch.arange(B, dtype=torch.int32, device=dev)
+    lens = (torch.arange(W + K, dtype=torch.int32, device=dev)[:, None] + (T0 + 1)).repeat(1, B).contiguous()
+    pos_all = (lens - 1).contiguous()
+
+    def step(i, pt, ev=None):
+        L.append(pool, n_pages, pt, seq_idx, pos_all[i], x_all[i], False, workspace=ws_app)
+        if ev is not None:
+            ev[0].record(stream)
+        L.decode(pool, n_pages, pt, lens[i], q_all[i], out, ws_dec)
+        if ev is not None:
+            ev[1].record(stream)
+
+    for i in range(W):
+        step(i, page_table)
+    torch.cuda.synchronize()
+    barrier(ws)
+    clocks = ClockSampler(local)
+    clocks.start()
+    time.sleep(0.3)
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+    t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    barrier(ws)
+    t_start.record(stream)
+    for k in range(K):
+        step(W + k, page_table, evs[k])
+    t_end.record(stream)
+    torch.cuda.synchronize()
+    barrier(ws)
+    ms_total = t_start.elapsed_time(t_end)
+    dec_ms = sum(a.elapsed_time(b) for a, b in evs) / K
+    clk = clocks.stop()
+    assert L.sync_status() == 0, "device status word set during the benchmark"
+    ms_step = max_over_ranks(ms_total / K, ws)
+    dec_ms = max_over_ranks(dec_ms, ws)
+
+    # End to end through the C ABI with host buffers: every step copies its inputs
+    # (x, q, lengths, positions) from pinned host memory and reads the output back.
+    pin_x = x_all.cpu().pin_memory()
+    pin_q = q_all.cpu().pin_memory()
+    pin_len = lens.cpu().pin_memory()
+    pin_pos = pos_all.cpu().pin_memory()
+    pin_out = torch.empty(W + K, B, spec.hidden, dtype=torch.bfloat16).pin_memory()
+    x_d, q_d = torch.empty_like(x_all[0]), torch.empty_like(q_all[0])
+    len_d, pos_d = torch.empty_like(lens[0]), torch.empty_like(lens[0])
+
+    def e2e_step(i):
+        x_d.copy_(pin_x[i], non_blocking=True)
+        q_d.copy_(pin_q[i], non_blocking=True)
+        len_d.copy_(pin_len[i], non_blocking=True)
+        pos_d.copy_(pin_pos[i], non_blocking=True)
+        L.append(pool, n_pages, page_table_e2e, seq_idx, pos_d, x_d, False, workspace=ws_app)
+        L.decode(pool, n_pages, page_table_e2e, len_d, q_d, out, ws_dec)
+        pin_out[i].copy_(out, non_blocking=True)
+
+    for i in range(W):
+        e2e_step(i)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    barrier(ws)
+    e0.record(stream)
+    for k in range(K):
+        e2e_step(W + k)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1) / K, ws)
+    h2d = (x_d.numel() + q_d.numel()) * 2 + (len_d.numel() + pos_d.numel()) * 4
+    d2h = out.numel() * 2
+
+    peak, peak_kind = measured_peaks()
+    dbytes = decode_bytes(spec, L, B, T0 + W + K // 2)
+    achieved = dbytes / (dec_ms * 1e-3) / 1e9
+    tokens_per_s = B * ws / (ms_step * 1e-3)
+    res = {
+        "metric": METRIC,
+        "value": tokens_per_s,
+        "unit": "tokens/s",
+        "n_gpus": ws,
+        "steps": K,
+        "warmup": W,
+        "ms_per_step": ms_step,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "u3/u4 latent codes + fp16 scales, bf16 factors/q/out, fp32 accumulate",
+        "data": "synthetic (seeded latents with the factor spectrum; random-init factors)",
+        "config": {"workload": f"STAR-KV decode step: append 1 token/seq + decode, batch {B}, ctx ~{ctx} "
+                               f"(LongChat-7B-shaped layer: H 32, d 128, D 4096, R_k 1024, r_v 1024, "
+                               f"block Hadamard 32, 4/3-bit latents, 16-token pages)",
+                   "batch": B, "ctx": ctx, "ctx_range": [T0 + W + 1, T0 + W + K], "parallelism": f"replicas x{ws}",
+                   "l2": "inputs larger than L2 (cache %.0f MB + M %.0f MB)" % (B * ctx * L.bytes_per_token / 1e6,
+                                                                            L.factor_bytes / 1e6)},
+        "us_per_layer_step": ms_step * 1e3,
+        "decode_us": dec_ms * 1e3,
+        "roofline": {"bound": "hbm", "kernel": "starkv_decode_attn (all decode kernels of one call)",
+                     "achieved": achieved, "peak": peak, "peak_kind": peak_kind, "unit": "GB/s",
+                     "frac": achieved / peak, "traffic": None, "algorithmic_bytes": dbytes},
+        "e2e": {"value": B * ws / (e2e_ms * 1e-3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h},
+        "gpu_launches": K * 7,
+        "clocks": clk,
+    }
+    if rank == 0 and ws == 1 and not args.no_cpu_baseline:
+        dt, cores = cpu_baseline(ctx)
+        res["cpu_baseline"] = {"value": 1.0 / dt, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                               "sample": f"1 sequence of the batch at ctx {ctx}: float64 explicit K/V "
+                                         f"reconstruction + softmax attention + W_o ({dt:.1f} s)"}
+    return res
+
+
+def run_reference(args, rank, ws):
+    """The oracle, as it stands, on the host cores: one sequence per step."""
+    if rank != 0:
+        return None
+    B, ctx = WORKLOAD["batch"], WORKLOAD["ctx"]
+    K, W = args.steps, args.warmup
+    sys.path.insert(0, os.path.join(ROOT, "tests"))
+    from harness import Case, queries
+    from synth import gen
+    T = args.ref_ctx or ctx
+    c = Case(gen.config_spec(WORKLOAD["cfg"]), gen.LAYER_SEED[WORKLOAD["cfg"]])
+    c.B_rot
+    Zs = c.stored(c.latents_direct(0, T))
+    q = queries(c, 1)[0, 0]
+    for _ in range(W):
+        c.oracle_decode(Zs, q, T - 1, T)
+    t0 = time.perf_counter()
+    for _ in range(K):
+        c.oracle_decode(Zs, q, T - 1, T)
+    dt = (time.perf_counter() - t0) / K
+    try:
+        from threadpoolctl import threadpool_info
+        cores = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
+    except Exception:
+        cores = os.cpu_count()
+    v = 1.0 / dt
+    return {"metric": METRIC, "value": v, "unit": "tokens/s", "n_gpus": ws, "steps": K, "warmup": W,
+            "ms_per_step": dt * 1e3, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "f64", "data": "synthetic", "impl": "reference",
+            "config": {"workload": f"oracle decode of 1 sequence per step at ctx {T} (sample of batch {B})",
+                       "batch": 1, "ctx": T},
+            "cpu_baseline": {"value": v, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                             "sample": f"1 of {B} sequences per step at ctx {T}"},
+            "e2e": {"value": v, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--ref-ctx", type=int, default=0)
+    args = ap.parse_args()
+    if args.impl == "reference":
+        rank = int(os.environ.get("RANK", "0"))
+        ws = int(os.environ.get("WORLD_SIZE", "1"))
+        res = run_reference(args, rank, ws)
+        if res is not None:
+            print(json.dumps(res), flush=True)
+        return
+    rank, ws, local = dist_init()
+    res = run_ours(args, rank, ws, local)
+    if rank == 0:
+        print(json.dumps(res), flush=True)
+    if ws > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

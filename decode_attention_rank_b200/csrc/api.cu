@@ -1,0 +1,429 @@
+// Host side of the C ABI: argument checks, layer planning (page layout, group
+// tables), factor folding at load time, and kernel dispatch.
+#include <math.h>
+#include <stdio.h>
+#include <string.h>
+
+#include <algorithm>
+#include <string>
+
+#include "starkv_internal.cuh"
+
+namespace starkv {
+
+static thread_local std::string g_last_error;
+
+void set_error(const std::string& msg) { g_last_error = msg; }
+
+static size_t ru(size_t x, size_t m) { return (x + m - 1) / m * m; }
+
+// Channels of the high-precision segment: ceil(top_fraction * r) (reading notes
+// "STAR-KV 阅读笔记" section 6.1; the model card's top_fraction).
+static int n_high(int r, float top_fraction) {
+  return (int)ceil((double)top_fraction * (double)r - 1e-9);
+}
+
+}  // namespace starkv
+
+using namespace starkv;
+
+#define CHECK_ARG(cond, msg)            \
+  do {                                  \
+    if (!(cond)) {                      \
+      set_error(msg);                   \
+      return STARKV_ERR_ARG;            \
+    }                                   \
+  } while (0)
+
+#define CUDA_TRY(expr)                                                          \
+  do {                                                                          \
+    cudaError_t e_ = (expr);                                                    \
+    if (e_ != cudaSuccess) {                                                    \
+      set_error(std::string(#expr) + ": " + cudaGetErrorString(e_));           \
+      return STARKV_ERR_CUDA;                                                   \
+    }                                                                           \
+  } while (0)
+
+// Plan the page layout: latent blocks in order (keys per KV head, then values),
+// each a multiple of 16 bytes; a quantized block is the scale block
+// [group][slot] fp16 followed by one LSB-first code block per group.
+static starkv_status plan_layer(starkv_layer* L) {
+  const starkv_layer_config& c = L->cfg;
+  const int Hkv = c.n_kv_heads, d = c.head_dim;
+  const int es = c.dtype == STARKV_F32 ? 4 : 2;
+  std::vector<int> widths;
+  if (c.plain) {
+    for (int h = 0; h < Hkv; ++h) widths.push_back(d);
+    widths.push_back(Hkv * d);
+  } else {
+    for (int h = 0; h < Hkv; ++h) widths.push_back(L->key_ranks[h]);
+    widths.push_back(c.value_rank);
+  }
+  const bool quant = c.quantized && !c.plain;
+  size_t off = 0;
+  int ch = 0;
+  double bpt = 0;
+  L->lat.clear();
+  L->grp.clear();
+  for (size_t li = 0; li < widths.size(); ++li) {
+    LatentDesc ld{};
+    ld.width = widths[li];
+    ld.block_off = (int)off;
+    ld.ch_off = ch;
+    ld.group0 = (int)L->grp.size();
+    if (!quant) {
+      L->grp.push_back(GroupDesc{0, ld.width, 0, 0});
+      ld.n_groups = 1;
+      ld.scale_bytes = 0;
+      off += ru((size_t)kPage * ld.width * es, 16);
+      bpt += (double)ld.width * es;
+    } else {
+      const int nh = n_high(ld.width, c.top_fraction);
+      const int seg_start[2] = {0, nh}, seg_len[2] = {nh, ld.width - nh}, seg_bits[2] = {c.top_bits, c.bottom_bits};
+      std::vector<GroupDesc> gs;
+      for (int s = 0; s < 2; ++s)
+        for (int k = 0; k < seg_len[s]; k += c.group_size)
+          gs.push_back(GroupDesc{seg_start[s] + k, std::min(c.group_size, seg_len[s] - k), seg_bits[s], 0});
+      ld.n_groups = (int)gs.size();
+      ld.scale_bytes = (int)ru((size_t)gs.size() * kPage * 2, 16);
+      size_t boff = ld.scale_bytes;
+      for (auto& g : gs) {
+        g.code_off = (int)boff;
+        boff += ru((size_t)kPage * g.n * g.bits / 8, 16);
+        bpt += g.n * g.bits / 8.0 + 2.0;
+      }
+      for (auto& g : gs) L->grp.push_back(g);
+      off += boff;
+    }
+    ch += ld.width;
+    L->lat.push_back(ld);
+  }
+  L->page_bytes = ru(off, 128);
+  L->bytes_per_token = bpt;
+  LayerView& v = L->view;
+  v.D = c.hidden;
+  v.H = c.n_heads;
+  v.Hkv = Hkv;
+  v.d = d;
+  v.group_q = c.n_heads / Hkv;
+  v.L = (int)widths.size();
+  v.Ltot = ch;
+  v.Rk = ch - widths.back();
+  v.rv = widths.back();
+  v.wv = c.plain ? d : c.value_rank;
+  v.es = es;
+  v.dtype = c.dtype;
+  v.quantized = quant ? 1 : 0;
+  v.plain = c.plain ? 1 : 0;
+  v.rope = c.rope ? 1 : 0;
+  v.hadamard = (quant && c.hadamard_block) ? 1 : 0;
+  v.rope_log2_theta = (float)log2(c.rope_theta);
+  const float sc = c.softmax_scale > 0 ? c.softmax_scale : (float)(1.0 / sqrt((double)d));
+  v.scale_log2 = sc * kLog2e;
+  v.page_bytes = (long long)L->page_bytes;
+  L->key_off.assign(Hkv + 1, 0);
+  for (int h = 0; h < Hkv; ++h) L->key_off[h + 1] = L->key_off[h] + widths[h];
+  const size_t mel = c.dtype == STARKV_F32 ? 4 : 2;
+  L->factor_bytes = (c.plain ? 0 : (size_t)v.Rk * d * (c.dtype == STARKV_F32 ? 4 : 2)) +
+                    (size_t)c.hidden * c.n_heads * v.wv * mel;
+  return STARKV_OK;
+}
+
+static starkv_status check_config(const starkv_layer_config* c) {
+  CHECK_ARG(c != nullptr, "config is NULL");
+  CHECK_ARG(c->hidden > 0 && c->n_heads > 0 && c->n_kv_heads > 0 && c->head_dim > 0, "non-positive shape");
+  CHECK_ARG(c->n_heads % c->n_kv_heads == 0, "n_heads must be a multiple of n_kv_heads");
+  CHECK_ARG(c->head_dim % 2 == 0 && c->head_dim <= 256, "head_dim must be even and <= 256");
+  CHECK_ARG(c->dtype == STARKV_F32 || c->dtype == STARKV_BF16, "dtype must be STARKV_F32 or STARKV_BF16");
+  CHECK_ARG(c->page_size == 16, "page_size must be 16");
+  CHECK_ARG(c->n_heads <= 128, "n_heads must be <= 128");
+  if (!c->plain) {
+    CHECK_ARG(c->key_ranks != nullptr, "key_ranks is NULL");
+    for (int h = 0; h < c->n_kv_heads; ++h)
+      CHECK_ARG(c->key_ranks[h] >= 1 && c->key_ranks[h] <= c->head_dim, "key rank outside 1..head_dim");
+    CHECK_ARG(c->value_rank >= 1 && c->value_rank <= c->n_kv_heads * c->head_dim, "value_rank outside 1..H_kv*d");
+  }
+  if (c->quantized && !c->plain) {
+    CHECK_ARG(c->top_bits >= 2 && c->top_bits <= 8 && c->bottom_bits >= 2 && c->bottom_bits <= 8,
+              "code widths must be 2..8 bits");
+    CHECK_ARG(c->group_size >= 1 && c->group_size <= 32, "group_size must be 1..32");
+    CHECK_ARG(c->top_fraction >= 0.f && c->top_fraction <= 1.f, "top_fraction must be in [0, 1]");
+  }
+  if (c->hadamard_block) {
+    CHECK_ARG(c->quantized && !c->plain, "hadamard_block requires a quantized compressed layer");
+    CHECK_ARG(c->hadamard_block == c->group_size, "hadamard_block must equal group_size");
+  }
+  if (c->rope) CHECK_ARG(c->rope_theta > 1.0, "rope_theta must be > 1");
+  return STARKV_OK;
+}
+
+extern "C" {
+
+const char* starkv_status_string(starkv_status s) {
+  switch (s) {
+    case STARKV_OK: return "ok";
+    case STARKV_ERR_ARG: return "invalid argument";
+    case STARKV_ERR_UNSUPPORTED: return "unsupported";
+    case STARKV_ERR_OOM: return "out of device memory";
+    case STARKV_ERR_CUDA: return "CUDA error";
+    case STARKV_ERR_DEVICE: return "device status word set";
+    case STARKV_ERR_TIMEOUT: return "device wait timed out";
+    case STARKV_ERR_WORKSPACE: return "workspace too small";
+  }
+  return "unknown status";
+}
+
+const char* starkv_last_error(void) { return g_last_error.c_str(); }
+
+const char* starkv_version(void) { return "starkv-b200 0.1 (sm_100a)"; }
+
+void starkv_free_layer(starkv_layer* L) {
+  if (!L) return;
+  int cur = 0;
+  cudaGetDevice(&cur);
+  cudaSetDevice(L->device);
+  cudaFree(L->d_lat);
+  cudaFree(L->d_grp);
+  cudaFree(L->d_key_off);
+  cudaFree(L->A_T);
+  cudaFree(L->Bk);
+  cudaFree(L->M_T);
+  cudaFree(L->status);
+  cudaSetDevice(cur);
+  delete L;
+}
+
+starkv_status starkv_load_factors(const starkv_layer_config* cfg, const void* A_k, const void* B_k, const void* A_v,
+                                  const void* B_v, const void* W_o, starkv_stream_t stream, starkv_layer** out) {
+  set_error("");
+  CHECK_ARG(out != nullptr, "out is NULL");
+  *out = nullptr;
+  starkv_status st = check_config(cfg);
+  if (st != STARKV_OK) return st;
+  CHECK_ARG(A_k && A_v && W_o, "A_k, A_v and W_o must be non-NULL");
+  if (!cfg->plain) CHECK_ARG(B_k && B_v, "B_k and B_v must be non-NULL");
+  cudaStream_t s = (cudaStream_t)stream;
+  starkv_layer* L = new starkv_layer();
+  L->cfg = *cfg;
+  if (!cfg->plain) L->key_ranks.assign(cfg->key_ranks, cfg->key_ranks + cfg->n_kv_heads);
+  L->cfg.key_ranks = nullptr;
+  cudaGetDevice(&L->device);
+  plan_layer(L);
+  LayerView& v = L->view;
+  const int D = v.D, d = v.d, H = v.H;
+  const size_t es = cfg->dtype == STARKV_F32 ? 4 : 2;
+  auto fail = [&](starkv_status code, const char* what) {
+    set_error(std::string("load_factors: ") + what + ": " + cudaGetErrorString(cudaGetLastError()));
+    starkv_free_layer(L);
+    return code;
+  };
+  if (cudaMalloc(&L->d_lat, sizeof(LatentDesc) * L->lat.size()) != cudaSuccess ||
+      cudaMalloc(&L->d_grp, sizeof(GroupDesc) * L->grp.size()) != cudaSuccess ||
+      cudaMalloc(&L->d_key_off, sizeof(int) * L->key_off.size()) != cudaSuccess ||
+      cudaMalloc(&L->status, sizeof(uint32_t)) != cudaSuccess ||
+      cudaMalloc(&L->A_T, es * (size_t)v.Ltot * D) != cudaSuccess ||
+      cudaMalloc(&L->M_T, (cfg->dtype == STARKV_F32 ? 4 : 2) * (size_t)D * H * v.wv) != cudaSuccess)
+    return fail(STARKV_ERR_OOM, "cudaMalloc");
+  if (!cfg->plain && cudaMalloc(&L->Bk, sizeof(float) * (size_t)v.Rk * d) != cudaSuccess)
+    return fail(STARKV_ERR_OOM, "cudaMalloc");
+  v.lat = L->d_lat;
+  v.grp = L->d_grp;
+  v.status = L->status;
+  if (cudaMemcpyAsync(L->d_lat, L->lat.data(), sizeof(LatentDesc) * L->lat.size(), cudaMemcpyHostToDevice, s) ||
+      cudaMemcpyAsync(L->d_grp, L->grp.data(), sizeof(GroupDesc) * L->grp.size(), cudaMemcpyHostToDevice, s) ||
+      cudaMemcpyAsync(L->d_key_off, L->key_off.data(), sizeof(int) * L->key_off.size(), cudaMemcpyHostToDevice, s) ||
+      cudaMemsetAsync(L->status, 0, sizeof(uint32_t), s))
+    return fail(STARKV_ERR_CUDA, "upload tables");
+  // Projection rows A_T[ch][k] for every latent channel (keys, then values).
+  if (cfg->plain) {
+    if (launch_transpose_into(A_k, D, v.Rk, cfg->dtype, L->A_T, 0, D, s) ||
+        launch_transpose_into(A_v, D, v.rv, cfg->dtype, L->A_T, v.Rk, D, s))
+      return fail(STARKV_ERR_CUDA, "transpose W_k/W_v");
+  } else {
+    size_t elem_off = 0;
+    for (int h = 0; h < v.Hkv; ++h) {
+      const char* src = (const char*)A_k + elem_off * es;
+      if (launch_transpose_into(src, D, L->key_ranks[h], cfg->dtype, L->A_T, L->key_off[h], D, s))
+        return fail(STARKV_ERR_CUDA, "transpose A_k");
+      elem_off += (size_t)D * L->key_ranks[h];
+    }
+    if (launch_transpose_into(A_v, D, v.rv, cfg->dtype, L->A_T, v.Rk, D, s))
+      return fail(STARKV_ERR_CUDA, "transpose A_v");
+    // B'_k = R^T B_k per KV head (float32).
+    size_t boff = 0;
+    for (int h = 0; h < v.Hkv; ++h) {
+      const char* src = (const char*)B_k + boff * es;
+      if (launch_rotate_rows(L, src, cfg->dtype, h, d, L->Bk + (size_t)L->key_off[h] * d, s))
+        return fail(STARKV_ERR_CUDA, "rotate B_k");
+      boff += (size_t)L->key_ranks[h] * d;
+    }
+  }
+  // M_h = B'_v,kv(h) W_o,h, stored transposed as M_T [D][H * wv].
+  float* Bv_rot = nullptr;
+  if (!cfg->plain) {
+    if (cudaMalloc(&Bv_rot, sizeof(float) * (size_t)v.rv * v.Hkv * d) != cudaSuccess)
+      return fail(STARKV_ERR_OOM, "cudaMalloc");
+    if (launch_rotate_rows(L, B_v, cfg->dtype, v.Hkv, v.Hkv * d, Bv_rot, s)) {
+      cudaFree(Bv_rot);
+      return fail(STARKV_ERR_CUDA, "rotate B_v");
+    }
+  }
+  cudaError_t e = launch_fold_M(L, Bv_rot, W_o, s);
+  if (Bv_rot) {
+    cudaStreamSynchronize(s);
+    cudaFree(Bv_rot);
+  }
+  if (e != cudaSuccess) return fail(STARKV_ERR_CUDA, "fold M");
+  *out = L;
+  return STARKV_OK;
+}
+
+starkv_status starkv_layer_get_info(const starkv_layer* L, starkv_layer_info* info) {
+  CHECK_ARG(L && info, "NULL argument");
+  info->n_latents = L->view.L;
+  info->latent_total = L->view.Ltot;
+  info->key_rank_total = L->view.Rk;
+  info->page_bytes = L->page_bytes;
+  info->bytes_per_token = L->bytes_per_token;
+  info->factor_bytes = L->factor_bytes;
+  return STARKV_OK;
+}
+
+size_t starkv_page_bytes(const starkv_layer* L) { return L ? L->page_bytes : 0; }
+
+starkv_status starkv_cache_init(const starkv_layer* L, void* pool, int64_t n_pages, starkv_stream_t stream) {
+  set_error("");
+  CHECK_ARG(L && pool, "NULL argument");
+  CHECK_ARG(n_pages >= 0, "negative n_pages");
+  CHECK_ARG(((uintptr_t)pool & 15) == 0, "pool must be 16-byte aligned");
+  CUDA_TRY(cudaMemsetAsync(pool, 0, (size_t)n_pages * L->page_bytes, (cudaStream_t)stream));
+  return STARKV_OK;
+}
+
+size_t starkv_append_workspace_bytes(const starkv_layer* L, int n_tokens) {
+  if (!L || n_tokens <= 0) return 0;
+  return ru(sizeof(float) * (size_t)n_tokens * L->view.Ltot, 256);
+}
+
+starkv_status starkv_append(const starkv_layer* L, void* pool, int64_t n_pages, const int32_t* page_table,
+                            int n_seqs, int max_pages, int n_tokens, const int32_t* seq_idx, const int32_t* positions,
+                            const void* input, int input_is_latent, void* workspace, size_t ws_bytes,
+                            starkv_stream_t stream) {
+  set_error("");
+  CHECK_ARG(L != nullptr, "layer is NULL");
+  CHECK_ARG(n_tokens >= 0, "negative n_tokens");
+  if (n_tokens == 0) return STARKV_OK;
+  CHECK_ARG(pool && page_table && seq_idx && positions && input, "NULL buffer");
+  CHECK_ARG(((uintptr_t)pool & 15) == 0, "pool must be 16-byte aligned");
+  CHECK_ARG(n_pages > 0 && max_pages > 0 && n_seqs > 0, "empty pool or page table");
+  cudaStream_t s = (cudaStream_t)stream;
+  const float* z = (const float*)input;
+  if (!input_is_latent) {
+    const size_t need = starkv_append_workspace_bytes(L, n_tokens);
+    if (ws_bytes < need || workspace == nullptr) {
+      set_error("append workspace too small");
+      return STARKV_ERR_WORKSPACE;
+    }
+    CUDA_TRY(launch_project(L, input, n_tokens, (float*)workspace, s));
+    z = (const float*)workspace;
+  }
+  const int rotate = (!input_is_latent && L->view.hadamard) ? 1 : 0;
+  const int rope_keys = (!input_is_latent && L->view.plain && L->view.rope) ? 1 : 0;
+  CUDA_TRY(launch_pack(L, (uint8_t*)pool, n_pages, page_table, n_seqs, max_pages, n_tokens, seq_idx, positions, z,
+                       rotate, rope_keys, s));
+  return STARKV_OK;
+}
+
+size_t starkv_workspace_bytes(const starkv_layer* L, int batch, int max_ctx, int max_q) {
+  if (!L || batch <= 0) return 0;
+  if (max_q < 1) max_q = 1;
+  max_ctx = std::max(max_ctx, 1);
+  size_t need = decode_generic_ws_bytes(L, batch, max_ctx, false);
+  if (max_q > 1) {
+    const long long rows = std::min<long long>((long long)batch * max_q, 1 << 30);
+    need = std::max(need, ru(sizeof(int32_t) * 3 * (size_t)rows, 256) +
+                              decode_generic_ws_bytes(L, (int)rows, max_ctx, true));
+  }
+  return need;
+}
+
+starkv_status starkv_decode_attn(const starkv_layer* L, const void* pool, int64_t n_pages, const int32_t* page_table,
+                                 int max_pages, int batch, const int32_t* seq_lens, const int32_t* q_pos,
+                                 const void* q, void* out, void* workspace, size_t ws_bytes, starkv_stream_t stream) {
+  set_error("");
+  CHECK_ARG(L != nullptr, "layer is NULL");
+  CHECK_ARG(batch >= 0, "negative batch");
+  if (batch == 0) return STARKV_OK;
+  CHECK_ARG(pool && page_table && seq_lens && q && out, "NULL buffer");
+  CHECK_ARG(n_pages > 0 && max_pages > 0, "empty pool or page table");
+  const int max_len = max_pages * kPage;
+  const size_t need = decode_generic_ws_bytes(L, batch, max_len, false);
+  if (workspace == nullptr || ws_bytes < need) {
+    set_error("decode workspace too small: need " + std::to_string(need) + " bytes");
+    return STARKV_ERR_WORKSPACE;
+  }
+  RowInfo ri{nullptr, seq_lens, q_pos};
+  CUDA_TRY(launch_decode_generic(L, (const uint8_t*)pool, n_pages, page_table, max_pages, batch, ri, max_len, q, out,
+                                 workspace, ws_bytes, false, (cudaStream_t)stream));
+  return STARKV_OK;
+}
+
+starkv_status starkv_prefill_attn(const starkv_layer* L, const void* pool, int64_t n_pages, const int32_t* page_table,
+                                  int max_pages, int batch, const int32_t* q_start_host, const int32_t* q_len_host,
+                                  const void* q, void* out, void* workspace, size_t ws_bytes, starkv_stream_t stream) {
+  set_error("");
+  CHECK_ARG(L != nullptr, "layer is NULL");
+  CHECK_ARG(batch >= 0, "negative batch");
+  if (batch == 0) return STARKV_OK;
+  CHECK_ARG(pool && page_table && q_start_host && q_len_host && q && out, "NULL buffer");
+  CHECK_ARG(n_pages > 0 && max_pages > 0, "empty pool or page table");
+  std::vector<int32_t> tab;
+  int rows = 0, max_len = 0;
+  for (int b = 0; b < batch; ++b) {
+    CHECK_ARG(q_start_host[b] >= 0 && q_len_host[b] >= 0, "negative q_start or q_len");
+    CHECK_ARG((long long)q_start_host[b] + q_len_host[b] <= (long long)max_pages * kPage,
+              "queries beyond the page table");
+    rows += q_len_host[b];
+    max_len = std::max(max_len, q_start_host[b] + q_len_host[b]);
+  }
+  if (rows == 0) return STARKV_OK;
+  tab.resize(3 * (size_t)rows);
+  int r = 0;
+  for (int b = 0; b < batch; ++b)
+    for (int i = 0; i < q_len_host[b]; ++i, ++r) {
+      tab[r] = b;                                // sequence
+      tab[rows + r] = q_start_host[b] + i + 1;   // visible length
+      tab[2 * rows + r] = q_start_host[b] + i;   // RoPE position
+    }
+  const size_t tab_bytes = ru(sizeof(int32_t) * tab.size(), 256);
+  const size_t need = tab_bytes + decode_generic_ws_bytes(L, rows, max_len, true);
+  if (workspace == nullptr || ws_bytes < need) {
+    set_error("prefill workspace too small: need " + std::to_string(need) + " bytes");
+    return STARKV_ERR_WORKSPACE;
+  }
+  cudaStream_t s = (cudaStream_t)stream;
+  int32_t* dtab = (int32_t*)workspace;
+  CUDA_TRY(cudaMemcpyAsync(dtab, tab.data(), sizeof(int32_t) * tab.size(), cudaMemcpyHostToDevice, s));
+  RowInfo ri{dtab, dtab + rows, dtab + 2 * rows};
+  CUDA_TRY(launch_decode_generic(L, (const uint8_t*)pool, n_pages, page_table, max_pages, rows, ri, max_len, q, out,
+                                 (char*)workspace + tab_bytes, ws_bytes - tab_bytes, true, s));
+  // pageable host source: make sure the copy has consumed `tab` before it is freed
+  CUDA_TRY(cudaStreamSynchronize(s));
+  return STARKV_OK;
+}
+
+starkv_status starkv_sync_status(const starkv_layer* L, starkv_stream_t stream, uint32_t* bits) {
+  set_error("");
+  CHECK_ARG(L != nullptr, "layer is NULL");
+  uint32_t w = 0;
+  cudaStream_t s = (cudaStream_t)stream;
+  CUDA_TRY(cudaMemcpyAsync(&w, L->status, sizeof(w), cudaMemcpyDeviceToHost, s));
+  CUDA_TRY(cudaMemsetAsync(L->status, 0, sizeof(uint32_t), s));
+  CUDA_TRY(cudaStreamSynchronize(s));
+  if (bits) *bits = w;
+  if (w == 0) return STARKV_OK;
+  if (w == STARKV_DEV_TIMEOUT) return STARKV_ERR_TIMEOUT;
+  return STARKV_ERR_DEVICE;
+}
+
+}  // extern "C"

@@ -1,0 +1,152 @@
+// Load-time folding of a layer's factors (untimed; once per layer).
+//  - projection rows A_T[ch][k] = A[k][ch] for every latent channel;
+//  - rotated up-projections B' = R^T B, R the block-wise Hadamard of the
+//    latent ("STAR-KV 阅读笔记" section 6.1: the rotation is absorbed into the
+//    up projection);
+//  - value-side output fusion M_h = B'_v,kv(h) W_o,h (section 5.3), stored as
+//    M_T [D][H * wv], the operand layout of the output kernel.
+#include "starkv_internal.cuh"
+
+namespace starkv {
+
+template <typename T>
+__device__ __forceinline__ float ld_f(const T* p, size_t i);
+template <>
+__device__ __forceinline__ float ld_f<float>(const float* p, size_t i) { return p[i]; }
+template <>
+__device__ __forceinline__ float ld_f<__nv_bfloat16>(const __nv_bfloat16* p, size_t i) {
+  return __bfloat162float(p[i]);
+}
+
+template <typename T>
+__global__ void k_transpose_into(const T* __restrict__ src, int rows, int cols, T* __restrict__ dst, int dst_row0,
+                                 int dst_ld) {
+  __shared__ T tile[32][33];
+  const int c0 = blockIdx.x * 32, r0 = blockIdx.y * 32;
+  for (int i = threadIdx.y; i < 32; i += blockDim.y) {
+    const int r = r0 + i, c = c0 + threadIdx.x;
+    if (r < rows && c < cols) tile[i][threadIdx.x] = src[(size_t)r * cols + c];
+  }
+  __syncthreads();
+  for (int i = threadIdx.y; i < 32; i += blockDim.y) {
+    const int c = c0 + i, r = r0 + threadIdx.x;
+    if (r < rows && c < cols) dst[(size_t)(dst_row0 + c) * dst_ld + r] = tile[threadIdx.x][i];
+  }
+}
+
+cudaError_t launch_transpose_into(const void* src, int rows, int cols, int dtype, void* dst, int dst_row0,
+                                  int dst_ld, cudaStream_t s) {
+  dim3 grid((cols + 31) / 32, (rows + 31) / 32), block(32, 8);
+  if (dtype == STARKV_F32)
+    k_transpose_into<float><<<grid, block, 0, s>>>((const float*)src, rows, cols, (float*)dst, dst_row0, dst_ld);
+  else
+    k_transpose_into<__nv_bfloat16><<<grid, block, 0, s>>>((const __nv_bfloat16*)src, rows, cols,
+                                                           (__nv_bfloat16*)dst, dst_row0, dst_ld);
+  return cudaGetLastError();
+}
+
+// out[j][c] = sum_j' R[j][j'] B[j'][c] for the rows j of one latent; R is the
+// direct sum over groups of normalised Sylvester blocks (binary decomposition
+// of the group length, largest block first), or the identity.
+template <typename T>
+__global__ void k_rotate_rows(const T* __restrict__ B, int width, int cols, const GroupDesc* __restrict__ grp,
+                              int n_groups, int hadamard, float* __restrict__ out) {
+  const size_t idx = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (idx >= (size_t)width * cols) return;
+  const int j = (int)(idx / cols), c = (int)(idx % cols);
+  if (!hadamard) {
+    out[idx] = ld_f(B, idx);
+    return;
+  }
+  int gs = 0, gn = width;
+  for (int g = 0; g < n_groups; ++g)
+    if (j >= grp[g].start && j < grp[g].start + grp[g].n) {
+      gs = grp[g].start;
+      gn = grp[g].n;
+    }
+  const int o = j - gs;
+  int bs = 0, rem = gn, p = 1;
+  while (rem > 0) {
+    p = 1 << (31 - __clz(rem));
+    if (o < bs + p) break;
+    bs += p;
+    rem -= p;
+  }
+  double acc = 0.0;
+  for (int k = 0; k < p; ++k) {
+    const int sgn = __popc((o - bs) & k) & 1;
+    const double b = ld_f(B, (size_t)(gs + bs + k) * cols + c);
+    acc += sgn ? -b : b;
+  }
+  out[idx] = (float)(acc / sqrt((double)p));
+}
+
+cudaError_t launch_rotate_rows(const starkv_layer* L, const void* B, int dtype, int latent, int cols, float* out,
+                               cudaStream_t s) {
+  const LatentDesc& ld = L->lat[latent];
+  const size_t n = (size_t)ld.width * cols;
+  const int threads = 256;
+  const unsigned blocks = (unsigned)((n + threads - 1) / threads);
+  // group table of this latent, relative to the latent's channels
+  const GroupDesc* g = L->d_grp + ld.group0;
+  if (dtype == STARKV_F32)
+    k_rotate_rows<float><<<blocks, threads, 0, s>>>((const float*)B, ld.width, cols, g, ld.n_groups,
+                                                    L->view.hadamard, out);
+  else
+    k_rotate_rows<__nv_bfloat16><<<blocks, threads, 0, s>>>((const __nv_bfloat16*)B, ld.width, cols, g,
+                                                            ld.n_groups, L->view.hadamard, out);
+  return cudaGetLastError();
+}
+
+// M_T[n][h*wv + j] = sum_p Bsrc[j][kv(h)*d + p] * W_o[h*d + p][n], float32
+// accumulation; Bsrc = rotated B_v (joint layers) or the identity (plain
+// layers, wv = d).  64 x 64 output tiles, 256 threads, 4 x 4 per thread.
+template <typename T, typename TO>
+__global__ void k_fold_M(const float* __restrict__ Bsrc, int bsrc_ld, const T* __restrict__ Wo, int D, int d,
+                         int wv, int group_q, int H, TO* __restrict__ MT) {
+  __shared__ float As[16][64];
+  __shared__ float Ws[16][65];
+  const int h = blockIdx.z, kv = h / group_q;
+  const int j0 = blockIdx.y * 64, n0 = blockIdx.x * 64;
+  const int tx = threadIdx.x % 16, ty = threadIdx.x / 16;
+  float acc[4][4] = {};
+  for (int p0 = 0; p0 < d; p0 += 16) {
+    for (int i = threadIdx.x; i < 16 * 64; i += 256) {
+      const int pp = i / 64, jj = i % 64;
+      const int j = j0 + jj, p = p0 + pp;
+      float a = 0.f;
+      if (j < wv && p < d) a = Bsrc ? Bsrc[(size_t)j * bsrc_ld + kv * d + p] : (j == p ? 1.f : 0.f);
+      As[pp][jj] = a;
+      const int n = n0 + jj;
+      Ws[pp][jj] = (p < d && n < D) ? ld_f(Wo, (size_t)(h * d + p) * D + n) : 0.f;
+    }
+    __syncthreads();
+#pragma unroll
+    for (int pp = 0; pp < 16; ++pp)
+#pragma unroll
+      for (int a = 0; a < 4; ++a)
+#pragma unroll
+        for (int b = 0; b < 4; ++b) acc[a][b] += As[pp][ty * 4 + a] * Ws[pp][tx * 4 + b];
+    __syncthreads();
+  }
+  for (int a = 0; a < 4; ++a)
+    for (int b = 0; b < 4; ++b) {
+      const int j = j0 + ty * 4 + a, n = n0 + tx * 4 + b;
+      if (j < wv && n < D) MT[(size_t)n * H * wv + (size_t)h * wv + j] = (TO)acc[a][b];
+    }
+}
+
+cudaError_t launch_fold_M(const starkv_layer* L, const float* Bv_rot, const void* W_o, cudaStream_t s) {
+  const LayerView& v = L->view;
+  dim3 grid((v.D + 63) / 64, (v.wv + 63) / 64, v.H);
+  const int bld = v.Hkv * v.d;
+  if (v.dtype == STARKV_F32)
+    k_fold_M<float, float><<<grid, 256, 0, s>>>(Bv_rot, bld, (const float*)W_o, v.D, v.d, v.wv, v.group_q, v.H,
+                                                (float*)L->M_T);
+  else
+    k_fold_M<__nv_bfloat16, __half><<<grid, 256, 0, s>>>(Bv_rot, bld, (const __nv_bfloat16*)W_o, v.D, v.d, v.wv,
+                                                         v.group_q, v.H, (__half*)L->M_T);
+  return cudaGetLastError();
+}
+
+}  // namespace starkv

@@ -1,0 +1,115 @@
+// Internal definitions shared by the host API and the kernels of libstarkv.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <stdint.h>
+
+#include <string>
+#include <vector>
+
+#include "starkv.h"
+
+namespace starkv {
+
+// One quantization/rotation group of a latent (channels [start, start + n) at `bits`).
+struct GroupDesc {
+  int start;
+  int n;
+  int bits;      // 0 = unquantized latent (one group spanning the whole latent)
+  int code_off;  // byte offset of this group's code block inside the latent block
+};
+
+// One stored latent of a token: key latent of a KV head, or the value latent.
+struct LatentDesc {
+  int width;        // r
+  int block_off;    // byte offset of the latent block inside the page
+  int n_groups;
+  int group0;       // index of the first group in the group table
+  int ch_off;       // offset of this latent in the concatenated latent vector
+  int scale_bytes;  // bytes of the scale block (0 when unquantized)
+};
+
+constexpr int kPage = 16;
+
+// Device status bits (mirror of STARKV_DEV_* in the public header).
+constexpr uint32_t kBadPage = STARKV_DEV_BAD_PAGE;
+constexpr uint32_t kBadPos = STARKV_DEV_BAD_POSITION;
+constexpr uint32_t kScaleOvf = STARKV_DEV_SCALE_OVF;
+constexpr uint32_t kTimeout = STARKV_DEV_TIMEOUT;
+
+constexpr float kLog2e = 1.4426950408889634f;
+
+// Everything a kernel needs to read or write one layer's pages.
+struct LayerView {
+  int D, H, Hkv, d, group_q;  // group_q = H / Hkv
+  int L;                      // latents per token
+  int Ltot;                   // sum of widths
+  int Rk;                     // sum of key widths
+  int wv;                     // value width per query head: r_v (joint) or d (plain)
+  int rv;                     // width of the value latent (plain: Hkv*d)
+  int es;                     // element bytes of unquantized latents (4 or 2)
+  int dtype;                  // STARKV_F32 / STARKV_BF16
+  int quantized, plain, rope;
+  int hadamard;
+  float rope_log2_theta;      // log2(theta)
+  float scale_log2;           // softmax scale * log2(e)
+  long long page_bytes;
+  const LatentDesc* lat;      // device tables
+  const GroupDesc* grp;
+  uint32_t* status;
+};
+
+}  // namespace starkv
+
+struct starkv_layer {
+  starkv_layer_config cfg;
+  std::vector<int> key_ranks;
+  std::vector<starkv::LatentDesc> lat;
+  std::vector<starkv::GroupDesc> grp;
+  std::vector<int> key_off;     // prefix sums of key widths, size Hkv + 1
+  starkv::LayerView view;
+  size_t page_bytes = 0;
+  double bytes_per_token = 0;
+  size_t factor_bytes = 0;
+  int device = 0;
+  // device allocations owned by the layer
+  starkv::LatentDesc* d_lat = nullptr;
+  starkv::GroupDesc* d_grp = nullptr;
+  int* d_key_off = nullptr;
+  void* A_T = nullptr;          // [Ltot][D] dtype: projection rows (unrotated)
+  float* Bk = nullptr;          // [Rk][d] fp32: rotated key up-projections B' = R^T B
+  void* M_T = nullptr;          // [D][H * wv]: fp16 (bf16 layers) or fp32 (f32 layers)
+  uint32_t* status = nullptr;
+};
+
+namespace starkv {
+
+void set_error(const std::string& msg);
+
+// Kernel launchers (defined in the .cu files).
+cudaError_t launch_transpose_into(const void* src, int rows, int cols, int dtype, void* dst, int dst_row0,
+                                  int dst_ld, cudaStream_t s);
+cudaError_t launch_rotate_rows(const starkv_layer* L, const void* B, int dtype, int latent, int cols, float* out,
+                               cudaStream_t s);
+cudaError_t launch_fold_M(const starkv_layer* L, const float* Bv_rot, const void* W_o, cudaStream_t s);
+
+cudaError_t launch_project(const starkv_layer* L, const void* x, int n, float* z, cudaStream_t s);
+cudaError_t launch_pack(const starkv_layer* L, uint8_t* pool, long long n_pages, const int32_t* page_table,
+                        int n_seqs, int max_pages, int n, const int32_t* seq_idx, const int32_t* positions, const float* z,
+                        int rotate, int rope_keys, cudaStream_t s);
+
+// Generic decode path: rows are (sequence, query position, visible length) triples.
+struct RowInfo {
+  const int32_t* row_seq;   // [rows] sequence of each row, or null = identity
+  const int32_t* row_len;   // [rows] visible tokens (decode: seq_lens)
+  const int32_t* row_pos;   // [rows] RoPE position of the query, or null = len - 1
+};
+cudaError_t launch_decode_generic(const starkv_layer* L, const uint8_t* pool, long long n_pages,
+                                  const int32_t* page_table, int max_pages, int rows, RowInfo ri, int max_len,
+                                  const void* q, void* out, void* ws, size_t ws_bytes, bool prefill,
+                                  cudaStream_t s);
+size_t decode_generic_ws_bytes(const starkv_layer* L, int rows, int max_len, bool prefill);
+
+}  // namespace starkv

@@ -1,0 +1,65 @@
+"""The C ABI library on a machine without a GPU: it loads, exports every entry
+point declared in include/starkv.h, and rejects bad arguments on the host
+before touching CUDA."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def declared_symbols():
+    names = []
+    for h in sorted(os.listdir(os.path.join(ROOT, "include"))):
+        if h.endswith(".h"):
+            text = open(os.path.join(ROOT, "include", h)).read()
+            names += re.findall(r"STARKV_API\s+[\w\s\*]+?\b(starkv_\w+)\s*\(", text)
+    return names
+
+
+def test_library_exports_every_declared_symbol():
+    from decode_attention_rank_b200 import starkv as lib
+    names = declared_symbols()
+    assert len(names) >= 14
+    raw = lib.raw_lib()
+    for n in names:
+        assert hasattr(raw, n), n
+    assert set(lib.EXPORTED) <= set(names)
+
+
+def test_version_and_status_strings():
+    from decode_attention_rank_b200 import starkv as lib
+    assert "sm_100a" in lib.version()
+    raw = lib.raw_lib()
+    for code, text in lib.STATUS.items():
+        assert raw.starkv_status_string(code).decode() == text
+
+
+def test_host_validation_before_cuda():
+    from decode_attention_rank_b200 import starkv as lib
+    bad = [
+        dict(hidden=64, n_heads=3, n_kv_heads=2, head_dim=8, key_ranks=[4, 4], value_rank=8),    # H % Hkv
+        dict(hidden=64, n_heads=2, n_kv_heads=2, head_dim=7, key_ranks=[4, 4], value_rank=8),    # odd d
+        dict(hidden=64, n_heads=2, n_kv_heads=2, head_dim=8, key_ranks=[9, 4], value_rank=8),    # rank > d
+        dict(hidden=64, n_heads=2, n_kv_heads=2, head_dim=8, key_ranks=[4, 4], value_rank=17),   # r_v > Hkv d
+        dict(hidden=64, n_heads=2, n_kv_heads=2, head_dim=8, key_ranks=[4, 4], value_rank=8, page_size=8),
+        dict(hidden=64, n_heads=2, n_kv_heads=2, head_dim=8, key_ranks=[4, 4], value_rank=8, hadamard_block=32),
+        dict(hidden=64, n_heads=2, n_kv_heads=2, head_dim=8, key_ranks=[4, 4], value_rank=8, quantized=True,
+             top_bits=9),
+    ]
+    for kw in bad:
+        cfg = lib.LayerConfig(**kw)
+        with pytest.raises(lib.StarKVError) as e:
+            lib.load_factors(cfg, None, None, None, None, None, stream=0)
+        assert e.value.status == 1, kw
+    # null factors with a valid config are also rejected on the host
+    cfg = lib.LayerConfig(hidden=64, n_heads=2, n_kv_heads=2, head_dim=8, key_ranks=[4, 4], value_rank=8)
+    with pytest.raises(lib.StarKVError) as e:
+        lib.load_factors(cfg, None, None, None, None, None, stream=0)
+    assert e.value.status == 1
+    raw = lib.raw_lib()
+    assert raw.starkv_decode_attn(None, None, 0, None, 0, 1, None, None, None, None, None, 0, None) == 1
+    assert raw.starkv_append(None, None, 0, None, 0, 0, 1, None, None, None, 0, None, 0, None) == 1
+    assert raw.starkv_workspace_bytes(None, 1, 1, 1) == 0

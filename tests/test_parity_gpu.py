@@ -1,0 +1,192 @@
+"""GPU parity of the library against the float64 oracle, through the C ABI.
+
+Inputs are seeded (synth); the oracle never sees a value produced by the
+library.  Tolerances (attention outputs): relative L2 <= 3e-3 and
+max |err| <= 1e-2 * max |oracle|; packed pages: bit-exact.
+"""
+import functools
+
+import numpy as np
+import pytest
+import torch
+
+from oracle import starkv_oracle as O
+from synth import gen
+
+from harness import Case, GpuCache, check_close, queries, rel_l2
+
+pytestmark = pytest.mark.gpu
+
+
+@functools.lru_cache(maxsize=None)
+def case(cfg: int, quantized: bool = False, layer: int = 2) -> Case:
+    spec = gen.config_spec(cfg, quantized=quantized, layer=layer)
+    return Case(spec, gen.LAYER_SEED[cfg], layer if cfg == 4 else 0)
+
+
+def run_decode(c: Case, lens, peaky=1.0, use_hidden=True, check_pool=True, q_pos=None, page_seed=0):
+    """Fill a cache (latent mode), decode one query per sequence, compare with the oracle."""
+    L = c.load()
+    s = c.spec
+    cache = GpuCache(L, lens, seed=page_seed)
+    lat_all = []
+    for b, T in enumerate(lens):
+        if T == 0:
+            lat_all.append(None)
+            continue
+        if use_hidden:
+            X = c.hidden(b, T)
+            Z = c.latents_from_hidden(X, np.arange(T))
+        else:
+            Z = c.latents_direct(b, T)
+        lat_all.append(Z)
+        cache.append_latents(b, Z)
+    if check_pool:
+        pool = cache.pool_pages()
+        want = O.build_pool(s, [z for z in lat_all if z is not None],
+                            cache.page_table_np[[b for b, z in enumerate(lat_all) if z is not None]], cache.n_pages)
+        np.testing.assert_array_equal(pool, want)
+    B = len(lens)
+    q = queries(c, B, peaky)[:, 0]
+    qt = torch.from_numpy(q).cuda().to(torch.float32 if s.dtype == "f32" else torch.bfloat16)
+    out = torch.empty(B, s.hidden, device="cuda", dtype=qt.dtype)
+    ws = torch.empty(L.workspace_bytes(B, cache.page_table.shape[1] * 16), dtype=torch.uint8, device="cuda")
+    seq_lens = torch.tensor(lens, dtype=torch.int32, device="cuda")
+    qp = None if q_pos is None else torch.tensor(q_pos, dtype=torch.int32, device="cuda")
+    L.decode(cache.pool, cache.n_pages, cache.page_table, seq_lens, qt, out, ws, q_pos=qp)
+    torch.cuda.synchronize()
+    assert L.sync_status() == 0
+    got = out.to(torch.float64).cpu().numpy()
+    for b, T in enumerate(lens):
+        if T == 0:
+            assert np.all(got[b] == 0)
+            continue
+        Zs = c.stored(lat_all[b])
+        pos = (T - 1) if q_pos is None else q_pos[b]
+        want = c.oracle_decode(Zs, q[b], pos, T)
+        check_close(got[b], want, f"seq {b} (T={T})")
+    return got
+
+
+def test_cfg0_tiny_fp32():
+    run_decode(case(0), [256])
+
+
+def test_cfg0_ragged_and_empty():
+    run_decode(case(0), [1, 0, 37, 130])
+
+
+def test_cfg1_bf16_rope():
+    run_decode(case(1), [300, 17, 1])
+
+
+def test_cfg1_peaky():
+    # logits scaled up (std ~ 3) so attention is far from uniform
+    run_decode(case(1), [200, 129], peaky=25.0, check_pool=False)
+
+
+def test_cfg2_quantized_hadamard():
+    run_decode(case(2), [333, 64, 5])
+
+
+def test_cfg2_peaky_direct_latents():
+    run_decode(case(2), [257, 48], peaky=25.0, use_hidden=False)
+
+
+def test_cfg3_gqa_bf16():
+    run_decode(case(3), [200, 33, 96])
+
+
+def test_cfg3_gqa_quantized():
+    run_decode(case(3, quantized=True), [200, 33, 96])
+
+
+def test_cfg4_plain_layer():
+    run_decode(case(4, layer=0), [150, 31])
+
+
+def test_cfg4_compressed_layer():
+    run_decode(case(4, layer=2), [150, 31])
+
+
+def test_custom_query_positions():
+    run_decode(case(1), [100, 64], q_pos=[150, 5], check_pool=False)
+
+
+def test_page_table_permutation_invariance():
+    c = case(2)
+    a = run_decode(c, [90, 40], page_seed=1, check_pool=False)
+    b = run_decode(c, [90, 40], page_seed=7, check_pool=False)
+    np.testing.assert_array_equal(a, b)
+
+
+def test_hidden_mode_append_matches_oracle_projection():
+    """Append from hidden states: the kernel projects, rotates and quantizes.
+    Codes may differ from the oracle's float64 projection only at rounding
+    boundaries; the decoded output must still meet the attention tolerance."""
+    c = case(2)
+    s = c.spec
+    L = c.load()
+    T = 80
+    cache = GpuCache(L, [T])
+    X = c.hidden(0, T)
+    xt = torch.from_numpy(X).cuda().to(torch.bfloat16)
+    ws = torch.empty(L.append_workspace_bytes(T), dtype=torch.uint8, device="cuda")
+    seq = torch.zeros(T, dtype=torch.int32, device="cuda")
+    pos = torch.arange(T, dtype=torch.int32, device="cuda")
+    L.append(cache.pool, cache.n_pages, cache.page_table, seq, pos, xt, False, workspace=ws)
+    pool = cache.pool_pages()
+    Z = c.latents_from_hidden(X, np.arange(T))
+    want = O.build_pool(s, [Z], cache.page_table_np, cache.n_pages)
+    diff = np.count_nonzero(pool != want)
+    assert diff <= 0.01 * pool.size, diff
+    q = queries(c, 1)[:, 0]
+    qt = torch.from_numpy(q).cuda().to(torch.bfloat16)
+    out = torch.empty(1, s.hidden, device="cuda", dtype=torch.bfloat16)
+    wsd = torch.empty(L.workspace_bytes(1, cache.page_table.shape[1] * 16), dtype=torch.uint8, device="cuda")
+    L.decode(cache.pool, cache.n_pages, cache.page_table, torch.tensor([T], dtype=torch.int32, device="cuda"), qt, out,
+             wsd)
+    got = out.double().cpu().numpy()[0]
+    check_close(got, c.oracle_decode(c.stored(Z), q[0], T - 1, T), "hidden-mode append")
+
+
+def test_prefill_causal_small():
+    c = case(2)
+    s = c.spec
+    L = c.load()
+    T0, n = 40, 24            # 40 cached tokens, then 24 new queries (chunk of a prefill)
+    cache = GpuCache(L, [T0 + n])
+    Z = c.latents_direct(0, T0 + n)
+    cache.append_latents(0, Z)
+    Q = queries(c, 1, n_pos=n)[0]
+    qt = torch.from_numpy(Q).cuda().to(torch.bfloat16)
+    out = torch.empty(n, s.hidden, device="cuda", dtype=torch.bfloat16)
+    ws = torch.empty(L.workspace_bytes(1, T0 + n, n), dtype=torch.uint8, device="cuda")
+    L.prefill(cache.pool, cache.n_pages, cache.page_table, [T0], [n], qt, out, ws)
+    got = out.double().cpu().numpy()
+    want = O.prefill(s, c.f, c.stored(Z), Q, T0, c.B_rot)
+    for i in range(n):
+        check_close(got[i], want[i], f"prefill query {i}")
+
+
+def test_device_status_bad_page():
+    """An out-of-range page id is caught by the kernels (status word), not dereferenced."""
+    c = case(0)
+    L = c.load()
+    cache = GpuCache(L, [40])
+    cache.append_latents(0, c.latents_direct(0, 40))
+    torch.cuda.synchronize()
+    assert L.sync_status() == 0
+    bad = cache.page_table.clone()
+    bad[0, 1] = cache.n_pages + 5
+    q = torch.from_numpy(queries(c, 1)[:, 0]).cuda().float()
+    out = torch.empty(1, c.spec.hidden, device="cuda")
+    ws = torch.empty(L.workspace_bytes(1, bad.shape[1] * 16), dtype=torch.uint8, device="cuda")
+    L.decode(cache.pool, cache.n_pages, bad, torch.tensor([40], dtype=torch.int32, device="cuda"), q, out, ws)
+    assert L.sync_status() & 0x1
+    assert L.sync_status() == 0     # read-and-clear
+    # append to a position beyond the page table
+    z = torch.zeros(1, L.latent_total, device="cuda")
+    L.append(cache.pool, cache.n_pages, cache.page_table, torch.zeros(1, dtype=torch.int32, device="cuda"),
+             torch.tensor([cache.page_table.shape[1] * 16], dtype=torch.int32, device="cuda"), z, True)
+    assert L.sync_status() & 0x2
