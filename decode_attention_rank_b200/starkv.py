@@ -31,7 +31,8 @@ DEV_BAD_PAGE, DEV_BAD_POSITION, DEV_SCALE_OVF, DEV_TIMEOUT = 0x1, 0x2, 0x4, 0x8
 EXPORTED = ["starkv_load_factors", "starkv_free_layer", "starkv_layer_get_info", "starkv_page_bytes",
             "starkv_cache_init", "starkv_append", "starkv_append_workspace_bytes", "starkv_decode_attn",
             "starkv_prefill_attn", "starkv_workspace_bytes", "starkv_sync_status", "starkv_status_string",
-            "starkv_last_error", "starkv_version"]
+            "starkv_last_error", "starkv_version", "starkv_decode_attn_noalloc"]
+NOALLOC_SCRATCH_BYTES = 32 << 20
 
 
 class _Config(ctypes.Structure):
@@ -66,6 +67,8 @@ _lib.starkv_decode_attn.argtypes = [_vp, _vp, _i64, _i32p, ctypes.c_int, ctypes.
                                     _sz, _vp]
 _lib.starkv_prefill_attn.argtypes = [_vp, _vp, _i64, _i32p, ctypes.c_int, ctypes.c_int, _vp, _vp, _vp, _vp, _vp, _sz,
                                      _vp]
+_lib.starkv_decode_attn_noalloc.argtypes = [_vp, _vp, _i64, _i32p, ctypes.c_int, ctypes.c_int, _i32p, _i32p, _vp,
+                                            _vp, _vp]
 _lib.starkv_workspace_bytes.argtypes = [_vp, ctypes.c_int, ctypes.c_int, ctypes.c_int]
 _lib.starkv_workspace_bytes.restype = _sz
 _lib.starkv_sync_status.argtypes = [_vp, _vp, ctypes.POINTER(ctypes.c_uint32)]
@@ -196,6 +199,13 @@ class Layer:
                                        int(seq_lens.numel()), _ptr(seq_lens), _ptr(q_pos), _ptr(q), _ptr(out),
                                        _ptr(workspace), workspace.numel() * workspace.element_size(),
                                        _stream(stream)), "starkv_decode_attn")
+
+    def decode_noalloc(self, pool, n_pages: int, page_table, seq_lens, q, out, q_pos=None, stream=None) -> None:
+        """Decode without a workspace (scratch in the library's fixed device array)."""
+        _check(_lib.starkv_decode_attn_noalloc(self._h, _ptr(pool), n_pages, _ptr(page_table),
+                                               int(page_table.shape[1]), int(seq_lens.numel()), _ptr(seq_lens),
+                                               _ptr(q_pos), _ptr(q), _ptr(out), _stream(stream)),
+               "starkv_decode_attn_noalloc")
 
     def prefill(self, pool, n_pages: int, page_table, q_start: list, q_len: list, q, out, workspace,
                 stream=None) -> None:

@@ -219,6 +219,36 @@ STARKV_API size_t starkv_workspace_bytes(const starkv_layer* layer, int batch, i
  */
 STARKV_API starkv_status starkv_sync_status(const starkv_layer* layer, starkv_stream_t stream, uint32_t* bits);
 
+/*
+ * Decode attention without a caller-provided workspace.  The paper has no
+ * counterpart: this entry point exists for callers that cannot allocate
+ * device memory themselves — for example a plugin inside a serving engine
+ * whose allocator has already reserved the GPU's memory for its own pools,
+ * or a caller with no access to an allocator at all — and so cannot hand
+ * starkv_decode_attn a workspace buffer.
+ *
+ * Same arguments, results and error behaviour as starkv_decode_attn, minus
+ * the workspace.  The scratch lives in one fixed device array inside this
+ * library, STARKV_NOALLOC_SCRATCH_BYTES (32 MiB) on every GPU that loads the
+ * library, kept until the process exits.  The call returns
+ * STARKV_ERR_WORKSPACE, before any launch and with a message naming both
+ * sizes, when starkv_workspace_bytes(layer, batch, max_pages * 16, 1) exceeds
+ * that size.  It allocates nothing: no cudaMalloc, no cudaFree, no
+ * allocating library routine.
+ *
+ * The first call on each device looks up the array's device address (with
+ * that device current); make that first call before any stream capture.
+ * Every call on a device shares the one array and leaves its contents behind;
+ * each call writes every scratch element before reading it, so nothing needs
+ * to start at zero.  Calls whose work overlaps on the GPU (several streams,
+ * or several host threads) race on the array: serialise them.
+ */
+#define STARKV_NOALLOC_SCRATCH_BYTES ((size_t)32 << 20)
+STARKV_API starkv_status starkv_decode_attn_noalloc(const starkv_layer* layer, const void* pool, int64_t n_pages,
+                                                    const int32_t* page_table, int max_pages, int batch,
+                                                    const int32_t* seq_lens, const int32_t* q_pos, const void* q,
+                                                    void* out, starkv_stream_t stream);
+
 STARKV_API const char* starkv_status_string(starkv_status s);
 
 /* Message of the last host-side error on this thread ("" if none). */
