@@ -17,6 +17,19 @@ void set_error(const std::string& msg) { g_last_error = msg; }
 
 static size_t ru(size_t x, size_t m) { return (x + m - 1) / m * m; }
 
+int num_sms() {
+  static int cached[64] = {};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 0 || dev >= 64) return 148;
+  if (cached[dev] == 0) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
+    cached[dev] = n;
+  }
+  return cached[dev];
+}
+
 // Channels of the high-precision segment: ceil(top_fraction * r) (reading notes
 // "STAR-KV 阅读笔记" section 6.1; the model card's top_fraction).
 static int n_high(int r, float top_fraction) {
@@ -121,6 +134,8 @@ static starkv_status plan_layer(starkv_layer* L) {
   const float sc = c.softmax_scale > 0 ? c.softmax_scale : (float)(1.0 / sqrt((double)d));
   v.scale_log2 = sc * kLog2e;
   v.page_bytes = (long long)L->page_bytes;
+  L->Kp = (int)ru((size_t)c.n_heads * v.wv, 64);
+  L->Dp = (int)ru((size_t)c.hidden, 128);
   L->key_off.assign(Hkv + 1, 0);
   for (int h = 0; h < Hkv; ++h) L->key_off[h + 1] = L->key_off[h] + widths[h];
   const size_t mel = c.dtype == STARKV_F32 ? 4 : 2;
@@ -222,7 +237,8 @@ starkv_status starkv_load_factors(const starkv_layer_config* cfg, const void* A_
       cudaMalloc(&L->d_key_off, sizeof(int) * L->key_off.size()) != cudaSuccess ||
       cudaMalloc(&L->status, sizeof(uint32_t)) != cudaSuccess ||
       cudaMalloc(&L->A_T, es * (size_t)v.Ltot * D) != cudaSuccess ||
-      cudaMalloc(&L->M_T, (cfg->dtype == STARKV_F32 ? 4 : 2) * (size_t)D * H * v.wv) != cudaSuccess)
+      cudaMalloc(&L->M_T, cfg->dtype == STARKV_F32 ? 4 * (size_t)D * H * v.wv : 2 * (size_t)L->Dp * L->Kp) !=
+          cudaSuccess)
     return fail(STARKV_ERR_OOM, "cudaMalloc");
   if (!cfg->plain && cudaMalloc(&L->Bk, sizeof(float) * (size_t)v.Rk * d) != cudaSuccess)
     return fail(STARKV_ERR_OOM, "cudaMalloc");
@@ -232,7 +248,8 @@ starkv_status starkv_load_factors(const starkv_layer_config* cfg, const void* A_
   if (cudaMemcpyAsync(L->d_lat, L->lat.data(), sizeof(LatentDesc) * L->lat.size(), cudaMemcpyHostToDevice, s) ||
       cudaMemcpyAsync(L->d_grp, L->grp.data(), sizeof(GroupDesc) * L->grp.size(), cudaMemcpyHostToDevice, s) ||
       cudaMemcpyAsync(L->d_key_off, L->key_off.data(), sizeof(int) * L->key_off.size(), cudaMemcpyHostToDevice, s) ||
-      cudaMemsetAsync(L->status, 0, sizeof(uint32_t), s))
+      cudaMemsetAsync(L->status, 0, sizeof(uint32_t), s) ||
+      (cfg->dtype != STARKV_F32 && cudaMemsetAsync(L->M_T, 0, 2 * (size_t)L->Dp * L->Kp, s)))
     return fail(STARKV_ERR_CUDA, "upload tables");
   // Projection rows A_T[ch][k] for every latent channel (keys, then values).
   if (cfg->plain) {

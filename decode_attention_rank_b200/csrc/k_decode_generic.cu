@@ -254,6 +254,34 @@ __global__ void k_combine(LayerView v, RowInfo ri, int n_splits, const float* __
   }
 }
 
+// Same merge, written as fp16 into the swizzled B-operand tiles of the output kernel:
+// row r, column k = h*wv + j lives in tile (r / NB, k / 64), row r % NB, column k % 64.
+__global__ void k_combine_tiled(LayerView v, int n_splits, const float* __restrict__ pY, const float* __restrict__ pm,
+                                const float* __restrict__ pl, int NB, int KT, uint8_t* __restrict__ ytiles) {
+  const int row = blockIdx.x, h = blockIdx.y;
+  float m = -FLT_MAX;
+  for (int s = 0; s < n_splits; ++s) m = fmaxf(m, pm[((size_t)row * n_splits + s) * v.H + h]);
+  float den = 0.f;
+  for (int s = 0; s < n_splits; ++s) {
+    const size_t i = ((size_t)row * n_splits + s) * v.H + h;
+    if (pl[i] > 0.f) den += exp2f(pm[i] - m) * pl[i];
+  }
+  const int nt = row / NB, r = row % NB;
+  for (int j = threadIdx.x; j < v.wv; j += blockDim.x) {
+    float acc = 0.f;
+    for (int s = 0; s < n_splits; ++s) {
+      const size_t i = ((size_t)row * n_splits + s) * v.H + h;
+      if (pl[i] > 0.f) acc += exp2f(pm[i] - m) * pY[i * v.wv + j];
+    }
+    const uint32_t k = (uint32_t)(h * v.wv + j);
+    const uint32_t c = k & 63u;
+    uint8_t* tile = ytiles + ((size_t)nt * KT + (k >> 6)) * (size_t)NB * 128;
+    const uint32_t off = (uint32_t)(r >> 3) * 1024u + (uint32_t)(r & 7) * 128u + (((c >> 3) ^ (uint32_t)(r & 7)) << 4) +
+                         (c & 7u) * 2u;
+    *reinterpret_cast<__half*>(tile + off) = __float2half_rn(den > 0.f ? acc / den : 0.f);
+  }
+}
+
 // out[row][n] = sum_k y[row][k] * M_T[n][k]; one warp per output column, eight rows per pass.
 template <typename TY, typename TO>
 __global__ void k_out(const TY* __restrict__ y, const TY* __restrict__ MT, int rows, int K, int D,
@@ -284,7 +312,8 @@ __global__ void k_out(const TY* __restrict__ y, const TY* __restrict__ MT, int r
 int value_block(const LayerView& v) { return v.plain ? (v.d <= kVBlock ? v.d : v.d / 2) : kVBlock; }
 
 struct WsPlan {
-  size_t qrot, S, pm, pl, pY, y, total;
+  size_t qrot, S, pm, pl, pY, y, part, total;
+  size_t y_bytes;
   int n_splits, chunk, S_ld;
 };
 
@@ -309,7 +338,18 @@ WsPlan plan_ws(const starkv_layer* L, int rows, int max_len, bool prefill) {
   p.pm = o;   o += ru256(sizeof(float) * (size_t)rows * ns * v.H);
   p.pl = o;   o += ru256(sizeof(float) * (size_t)rows * ns * v.H);
   p.pY = o;   o += ru256(sizeof(float) * (size_t)rows * ns * v.H * v.wv);
-  p.y = o;    o += ru256(ys * (size_t)rows * v.H * v.wv);
+  if (v.dtype == STARKV_F32) {
+    p.y_bytes = ys * (size_t)rows * v.H * v.wv;
+    p.y = o;    o += ru256(p.y_bytes);
+    p.part = o;
+  } else {
+    // fp16 tiles [rows / NB][Kp / 64][NB][64] (swizzled) for the tensor-core output kernel
+    const int NB = outproj_nb(rows);
+    const size_t ntiles = (rows + NB - 1) / NB;
+    p.y_bytes = ntiles * (L->Kp / 64) * (size_t)NB * 128;
+    p.y = o;    o += ru256(p.y_bytes);
+    p.part = o; o += ru256(outproj_part_bytes(L, rows));
+  }
   p.total = o;
   return p;
 }
@@ -356,12 +396,19 @@ cudaError_t launch_decode_generic(const starkv_layer* L, const uint8_t* pool, lo
     k_combine<float><<<dim3(rows, v.H), 128, 0, s>>>(v, ri, p.n_splits, pY, pm, pl, (float*)y);
     k_out<float, float><<<(v.D * 32 + 255) / 256, 256, 0, s>>>((const float*)y, (const float*)L->M_T, rows,
                                                                 v.H * v.wv, v.D, (float*)out);
-  } else {
-    k_combine<__half><<<dim3(rows, v.H), 128, 0, s>>>(v, ri, p.n_splits, pY, pm, pl, (__half*)y);
-    k_out<__half, __nv_bfloat16><<<(v.D * 32 + 255) / 256, 256, 0, s>>>(
-        (const __half*)y, (const __half*)L->M_T, rows, v.H * v.wv, v.D, (__nv_bfloat16*)out);
+    return cudaGetLastError();
   }
-  return cudaGetLastError();
+  const int NB = outproj_nb(rows);
+  const int KT = L->Kp / 64;
+  // padding rows and columns of the y tiles must be zero
+  if (rows % NB != 0 || L->Kp != v.H * v.wv) {
+    cudaError_t e = cudaMemsetAsync(y, 0, p.y_bytes, s);
+    if (e != cudaSuccess) return e;
+  }
+  k_combine_tiled<<<dim3(rows, v.H), 128, 0, s>>>(v, p.n_splits, pY, pm, pl, NB, KT, (uint8_t*)y);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  return launch_outproj_tc(L, y, rows, out, (float*)(w + p.part), s);
 }
 
 }  // namespace starkv

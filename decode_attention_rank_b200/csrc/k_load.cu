@@ -9,6 +9,12 @@
 
 namespace starkv {
 
+// Element index of (row, col < 64) of a 16-bit tile with 128-byte swizzled rows.
+__device__ __forceinline__ uint32_t tc_sw128_elem(uint32_t row, uint32_t col) {
+  const uint32_t chunk = col >> 3;
+  return ((row >> 3) * 1024u + (row & 7u) * 128u + ((chunk ^ (row & 7u)) << 4)) / 2u + (col & 7u);
+}
+
 template <typename T>
 __device__ __forceinline__ float ld_f(const T* p, size_t i);
 template <>
@@ -101,9 +107,11 @@ cudaError_t launch_rotate_rows(const starkv_layer* L, const void* B, int dtype, 
 // M_T[n][h*wv + j] = sum_p Bsrc[j][kv(h)*d + p] * W_o[h*d + p][n], float32
 // accumulation; Bsrc = rotated B_v (joint layers) or the identity (plain
 // layers, wv = d).  64 x 64 output tiles, 256 threads, 4 x 4 per thread.
+// tiled = 0: row-major [D][H*wv] float32.  tiled = 1: fp16 tiles of 128 x 64
+// (n, k) elements, 128-byte swizzled, tile (n/128, k/64) at ((n/128)*KT + k/64) * 16 KB.
 template <typename T, typename TO>
 __global__ void k_fold_M(const float* __restrict__ Bsrc, int bsrc_ld, const T* __restrict__ Wo, int D, int d,
-                         int wv, int group_q, int H, TO* __restrict__ MT) {
+                         int wv, int group_q, int H, int tiled, int KT, TO* __restrict__ MT) {
   __shared__ float As[16][64];
   __shared__ float Ws[16][65];
   const int h = blockIdx.z, kv = h / group_q;
@@ -132,7 +140,16 @@ __global__ void k_fold_M(const float* __restrict__ Bsrc, int bsrc_ld, const T* _
   for (int a = 0; a < 4; ++a)
     for (int b = 0; b < 4; ++b) {
       const int j = j0 + ty * 4 + a, n = n0 + tx * 4 + b;
-      if (j < wv && n < D) MT[(size_t)n * H * wv + (size_t)h * wv + j] = (TO)acc[a][b];
+      if (j < wv && n < D) {
+        const size_t k = (size_t)h * wv + j;
+        if (!tiled) {
+          MT[(size_t)n * H * wv + k] = (TO)acc[a][b];
+        } else {
+          const size_t tile = ((size_t)(n >> 7) * KT + (k >> 6)) * (128 * 64);
+          const uint32_t off = tc_sw128_elem((uint32_t)(n & 127), (uint32_t)(k & 63));
+          MT[tile + off] = (TO)acc[a][b];
+        }
+      }
     }
 }
 
@@ -141,11 +158,11 @@ cudaError_t launch_fold_M(const starkv_layer* L, const float* Bv_rot, const void
   dim3 grid((v.D + 63) / 64, (v.wv + 63) / 64, v.H);
   const int bld = v.Hkv * v.d;
   if (v.dtype == STARKV_F32)
-    k_fold_M<float, float><<<grid, 256, 0, s>>>(Bv_rot, bld, (const float*)W_o, v.D, v.d, v.wv, v.group_q, v.H,
-                                                (float*)L->M_T);
+    k_fold_M<float, float><<<grid, 256, 0, s>>>(Bv_rot, bld, (const float*)W_o, v.D, v.d, v.wv, v.group_q, v.H, 0,
+                                                0, (float*)L->M_T);
   else
     k_fold_M<__nv_bfloat16, __half><<<grid, 256, 0, s>>>(Bv_rot, bld, (const __nv_bfloat16*)W_o, v.D, v.d, v.wv,
-                                                         v.group_q, v.H, (__half*)L->M_T);
+                                                         v.group_q, v.H, 1, L->Kp / 64, (__half*)L->M_T);
   return cudaGetLastError();
 }
 

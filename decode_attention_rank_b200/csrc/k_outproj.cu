@@ -1,0 +1,249 @@
+// Output through the fused value/output factors on tcgen05 tensor cores
+// ("STAR-KV 阅读笔记" section 5.3 and Algorithm 2 steps 7-8):
+//     out[b][n] = sum_k y[b][k] * M[k][n],   k = (query head h, value channel j)
+// computed swapped, out^T = M^T y^T, so the large operand M^T [D][H*wv] is the
+// 128-row A tile (K-major) and the small batch y [rows][H*wv] is the B tile.
+//
+// The work is HBM-bound on M (268 MB per layer for a LongChat-7B layer with
+// r_v = 1024).  Both operands are stored pre-tiled and pre-swizzled, so each
+// k-step is two plain bulk copies (16 KB of M and rows*128 B of y) into a ring
+// of shared-memory stages.  A persistent grid of one CTA per SM splits the
+// (D/128) x (K/64) k-steps evenly (stream-K); a CTA whose range crosses an
+// output tile boundary flushes its accumulator there.  Partial sums go to the
+// workspace and a small kernel adds them in a fixed order.
+#include "tc_common.cuh"
+
+namespace starkv {
+
+int outproj_nb(int rows) { return (std::min(std::max(rows, 1), 256) + 15) / 16 * 16; }
+
+OutGeom outproj_geom(const starkv_layer* L) {
+  OutGeom g;
+  g.KT = L->Kp / 64;
+  g.DT = L->Dp / 128;
+  const long long U = (long long)g.KT * g.DT;
+  g.G = (int)std::min<long long>(num_sms(), U);
+  const long long per = (U + g.G - 1) / g.G;
+  g.slots = (int)((per + g.KT - 1) / g.KT) + 1;
+  return g;
+}
+
+namespace {
+
+constexpr int kOutThreads = 192;  // warp 0 producer, warp 1 MMA, warps 2-5 epilogue
+
+struct OutArgs {
+  const uint8_t* M;   // [DT][KT] tiles of 128 x 64 fp16, 16 KB each
+  const uint8_t* y;   // [NTILES][KT] tiles of NB x 64 fp16
+  float* part;        // [grid.x][slots][NB][128] partial sums
+  int NB;             // rows of one B tile (multiple of 16, <= 256)
+  int KT, DT;         // k-tiles, output tiles
+  int slots;          // partial slots per CTA
+  int stages;
+  uint32_t tmem_cols;
+  uint32_t* status;
+};
+
+__device__ __forceinline__ long long unit_begin(int c, int G, long long U) { return (long long)c * U / G; }
+
+__global__ void __launch_bounds__(kOutThreads, 1) k_outproj_tc(OutArgs a) {
+  extern __shared__ uint8_t smem_raw[];
+  __shared__ __align__(8) uint64_t full[8], empty[8], seg_done[2], acc_free[2], fin;
+  __shared__ uint32_t tmem_base;
+  __shared__ volatile int abort_flag;
+  uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int G = gridDim.x, c = blockIdx.x, nt = blockIdx.y;
+  const long long U = (long long)a.DT * a.KT;
+  const long long u0 = unit_begin(c, G, U), u1 = unit_begin(c + 1, G, U);
+  const uint32_t a_bytes = 128 * 128, b_bytes = (uint32_t)a.NB * 128;
+  uint8_t* A_s = smem;
+  uint8_t* B_s = smem + (size_t)a.stages * a_bytes;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < a.stages; ++s) {
+      tc::mbar_init(&full[s], 1);
+      tc::mbar_init(&empty[s], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      tc::mbar_init(&seg_done[i], 1);
+      tc::mbar_init(&acc_free[i], 4);
+    }
+    tc::mbar_init(&fin, 1);
+    abort_flag = 0;
+    tc::fence_mbar_init();
+  }
+  if (warp == 1) tc::tmem_alloc(&tmem_base, a.tmem_cols);
+  tc::tc_fence_before();
+  __syncthreads();
+  tc::tc_fence_after();
+  const uint32_t tmem = tmem_base;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      int i = 0;
+      for (long long u = u0; u < u1; ++u, ++i) {
+        const int s = i % a.stages;
+        const uint32_t ph = (uint32_t)(i / a.stages) & 1u;
+        if (!tc::mbar_wait(&empty[s], ph ^ 1u, a.status)) {
+          abort_flag = 1;
+          break;
+        }
+        const int dt = (int)(u / a.KT), kt = (int)(u % a.KT);
+        tc::mbar_expect_tx(&full[s], a_bytes + b_bytes);
+        tc::bulk_g2s(A_s + (size_t)s * a_bytes, a.M + ((size_t)dt * a.KT + kt) * a_bytes, a_bytes, &full[s]);
+        tc::bulk_g2s(B_s + (size_t)s * b_bytes, a.y + ((size_t)nt * a.KT + kt) * b_bytes, b_bytes, &full[s]);
+      }
+      // copies still in flight land before this CTA may exit
+      const int issued = i;
+      for (int j = issued - a.stages; j < issued; ++j)
+        if (j >= 0) tc::mbar_wait(&full[j % a.stages], (uint32_t)(j / a.stages) & 1u, a.status);
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      const uint32_t idesc = tc::idesc_f16(128, a.NB, false, false, false);
+      int i = 0, seg = 0;
+      bool first = true;
+      for (long long u = u0; u < u1 && !abort_flag; ++u, ++i) {
+        const int s = i % a.stages;
+        const int acc = seg & 1;
+        if (first && !tc::mbar_wait(&acc_free[acc], (((uint32_t)seg >> 1) & 1u) ^ 1u, a.status)) {
+          abort_flag = 1;
+          break;
+        }
+        if (!tc::mbar_wait(&full[s], (uint32_t)(i / a.stages) & 1u, a.status)) {
+          abort_flag = 1;
+          break;
+        }
+        tc::tc_fence_after();
+        const uint32_t d = tmem + (uint32_t)(acc * a.NB);
+        const uint32_t abase = tc::smem_u32(A_s + (size_t)s * a_bytes);
+        const uint32_t bbase = tc::smem_u32(B_s + (size_t)s * b_bytes);
+#pragma unroll
+        for (int k = 0; k < 4; ++k)
+          tc::mma_f16_ss(d, tc::sdesc_sw128(abase + 32 * k, 0, 1024), tc::sdesc_sw128(bbase + 32 * k, 0, 1024),
+                         idesc, (first && k == 0) ? 0u : 1u);
+        tc::mma_commit(&empty[s]);
+        first = false;
+        if (u + 1 == u1 || (u + 1) % a.KT == 0) {
+          tc::mma_commit(&seg_done[acc]);
+          ++seg;
+          first = true;
+        }
+      }
+      tc::mma_commit(&fin);
+      tc::mbar_wait(&fin, 0, a.status);
+    }
+  } else {
+    // epilogue: warps 2..5 cover TMEM lane quarters (warp % 4)
+    const int q = warp & 3;
+    const int n_local = q * 32 + lane;
+    int seg = 0;
+    for (long long u = u0; u < u1; ++seg) {
+      const long long seg_end = min(u1, (u / a.KT + 1) * a.KT);
+      const int dt = (int)(u / a.KT);
+      const int acc = seg & 1;
+      const bool ok = tc::mbar_wait(&seg_done[acc], ((uint32_t)seg >> 1) & 1u, a.status);
+      tc::tc_fence_after();
+      const int slot = dt - (int)(u0 / a.KT);
+      float* dst = a.part + (((size_t)c * a.slots + slot) * a.NB) * 128 + n_local;
+      for (int b0 = 0; b0 < a.NB; b0 += 16) {
+        float v[16];
+        if (ok) {
+          tc::tmem_ld16_sync(tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * a.NB + b0), v);
+        } else {
+#pragma unroll
+          for (int i = 0; i < 16; ++i) v[i] = 0.f;
+        }
+#pragma unroll
+        for (int i = 0; i < 16; ++i) dst[(size_t)(b0 + i) * 128] = v[i];
+      }
+      tc::tc_fence_before();
+      __syncwarp();
+      if (lane == 0) tc::mbar_arrive(&acc_free[acc]);
+      u = seg_end;
+      if (!ok) break;
+    }
+  }
+  tc::tc_fence_before();
+  __syncthreads();
+  tc::tc_fence_after();
+  if (warp == 1) tc::tmem_dealloc(tmem, a.tmem_cols);
+}
+
+// out[row][n] = sum over the CTAs whose k-range touched output tile n / 128.
+template <typename TO>
+__global__ void k_outproj_reduce(const float* __restrict__ part, int G, int KT, int DT, int slots, int NB, int rows,
+                                 int D, TO* __restrict__ out) {
+  const int dt = blockIdx.x, row = blockIdx.y;
+  const int nt = row / NB, b = row % NB;
+  const long long U = (long long)DT * KT;
+  const long long lo = (long long)dt * KT, hi = lo + KT;
+  // CTAs c with [begin(c), begin(c+1)) intersecting [lo, hi)
+  int c_lo = (int)((lo * G) / U);
+  while (c_lo > 0 && unit_begin(c_lo, G, U) > lo) --c_lo;
+  while (unit_begin(c_lo + 1, G, U) <= lo) ++c_lo;
+  for (int n = threadIdx.x; n < 128; n += blockDim.x) {
+    const int d = dt * 128 + n;
+    if (d >= D) continue;
+    float acc = 0.f;
+    for (int cc = c_lo; cc < G && unit_begin(cc, G, U) < hi; ++cc) {
+      const long long b0 = unit_begin(cc, G, U), b1 = unit_begin(cc + 1, G, U);
+      if (b1 <= lo || b0 == b1) continue;
+      const int slot = dt - (int)(b0 / KT);
+      acc += part[((((size_t)nt * G + cc) * slots + slot) * NB + b) * 128 + n];
+    }
+    out[(size_t)row * D + d] = (TO)acc;
+  }
+}
+
+}  // namespace
+
+// Workspace of the partial sums for `rows` output rows.
+size_t outproj_part_bytes(const starkv_layer* L, int rows) {
+  const int NB = outproj_nb(rows);
+  const int ntiles = (rows + NB - 1) / NB;
+  const OutGeom g = outproj_geom(L);
+  return sizeof(float) * (size_t)ntiles * g.G * g.slots * NB * 128;
+}
+
+cudaError_t launch_outproj_tc(const starkv_layer* L, const void* y_tiles, int rows, void* out, float* part,
+                              cudaStream_t s) {
+  const OutGeom g = outproj_geom(L);
+  const int NB = outproj_nb(rows);
+  const int ntiles = (rows + NB - 1) / NB;
+  OutArgs a;
+  a.M = (const uint8_t*)L->M_T;
+  a.y = (const uint8_t*)y_tiles;
+  a.NB = NB;
+  a.KT = g.KT;
+  a.DT = g.DT;
+  a.slots = g.slots;
+  const size_t stage_bytes = 128 * 128 + (size_t)NB * 128;
+  a.stages = (int)std::min<size_t>(8, (200 * 1024) / stage_bytes);
+  uint32_t cols = 32;
+  while (cols < (uint32_t)(2 * NB)) cols <<= 1;
+  a.tmem_cols = cols;
+  a.status = L->status;
+  const size_t smem = (size_t)a.stages * stage_bytes + 1024;
+  static bool attr = false;
+  if (!attr) {
+    cudaFuncSetAttribute(k_outproj_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, 220 * 1024);
+    attr = true;
+  }
+  for (int t = 0; t < ntiles; ++t) {
+    OutArgs at = a;
+    at.y = a.y + (size_t)t * g.KT * NB * 128;
+    at.part = part + (size_t)t * g.G * g.slots * NB * 128;
+    k_outproj_tc<<<dim3(g.G, 1), kOutThreads, smem, s>>>(at);
+  }
+  if (L->view.dtype == STARKV_F32)
+    k_outproj_reduce<float><<<dim3(g.DT, rows), 128, 0, s>>>(part, g.G, g.KT, g.DT, g.slots, NB, rows, L->view.D,
+                                                             (float*)out);
+  else
+    k_outproj_reduce<__nv_bfloat16><<<dim3(g.DT, rows), 128, 0, s>>>(part, g.G, g.KT, g.DT, g.slots, NB, rows,
+                                                                     L->view.D, (__nv_bfloat16*)out);
+  return cudaGetLastError();
+}
+
+}  // namespace starkv

@@ -6,6 +6,7 @@
 #include <cuda_fp16.h>
 #include <stdint.h>
 
+#include <algorithm>
 #include <string>
 #include <vector>
 
@@ -80,7 +81,11 @@ struct starkv_layer {
   int* d_key_off = nullptr;
   void* A_T = nullptr;          // [Ltot][D] dtype: projection rows (unrotated)
   float* Bk = nullptr;          // [Rk][d] fp32: rotated key up-projections B' = R^T B
-  void* M_T = nullptr;          // [D][H * wv]: fp16 (bf16 layers) or fp32 (f32 layers)
+  // Fused output factors.  f32 layers: [D][H * wv] float32, row-major.  bf16
+  // layers: fp16 tiles [Dp/128][Kp/64] of 128 x 64 elements, 128-byte swizzled
+  // (the A operand of the tensor-core output kernel), zero padded.
+  void* M_T = nullptr;
+  int Kp = 0, Dp = 0;           // H * wv and D rounded up to 64 and 128
   uint32_t* status = nullptr;
 };
 
@@ -111,5 +116,17 @@ cudaError_t launch_decode_generic(const starkv_layer* L, const uint8_t* pool, lo
                                   const void* q, void* out, void* ws, size_t ws_bytes, bool prefill,
                                   cudaStream_t s);
 size_t decode_generic_ws_bytes(const starkv_layer* L, int rows, int max_len, bool prefill);
+
+int num_sms();
+
+// Tensor-core output kernel (bf16 layers).
+struct OutGeom {
+  int KT, DT, G, slots;
+};
+int outproj_nb(int rows);
+OutGeom outproj_geom(const starkv_layer* L);
+size_t outproj_part_bytes(const starkv_layer* L, int rows);
+cudaError_t launch_outproj_tc(const starkv_layer* L, const void* y_tiles, int rows, void* out, float* part,
+                              cudaStream_t s);
 
 }  // namespace starkv

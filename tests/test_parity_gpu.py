@@ -169,6 +169,32 @@ def test_prefill_causal_small():
         check_close(got[i], want[i], f"prefill query {i}")
 
 
+def test_batch_40_padded_output_tile():
+    # 40 rows -> one 48-row B tile of the tensor-core output kernel (8 zero rows)
+    run_decode(case(2), [64] * 3 + [17] * 37, check_pool=False, use_hidden=False)
+
+
+def test_prefill_two_output_tiles():
+    """300 query rows -> two B tiles (256 + 44) of the output kernel; sampled rows checked."""
+    c = case(1)
+    s = c.spec
+    L = c.load()
+    T0, n = 20, 300
+    cache = GpuCache(L, [T0 + n])
+    Z = c.latents_direct(0, T0 + n) if not s.plain else None
+    cache.append_latents(0, Z)
+    Q = queries(c, 1, n_pos=n)[0]
+    qt = torch.from_numpy(Q).cuda().to(torch.bfloat16)
+    out = torch.empty(n, s.hidden, device="cuda", dtype=torch.bfloat16)
+    ws = torch.empty(L.workspace_bytes(1, T0 + n, n), dtype=torch.uint8, device="cuda")
+    L.prefill(cache.pool, cache.n_pages, cache.page_table, [T0], [n], qt, out, ws)
+    got = out.double().cpu().numpy()
+    Zs = c.stored(Z)
+    for i in (0, 1, 255, 256, 299):
+        want = O.decode(s, c.f, Zs, Q[i], T0 + i, T0 + i + 1, c.B_rot)
+        check_close(got[i], want, f"prefill row {i}")
+
+
 def test_device_status_bad_page():
     """An out-of-range page id is caught by the kernels (status word), not dereferenced."""
     c = case(0)
