@@ -204,6 +204,8 @@ void starkv_free_layer(starkv_layer* L) {
   cudaFree(L->Bk);
   cudaFree(L->M_T);
   cudaFree(L->status);
+  cudaFree(L->d_items);
+  cudaFree(L->rope_E);
   cudaSetDevice(cur);
   delete L;
 }
@@ -291,6 +293,18 @@ starkv_status starkv_load_factors(const starkv_layer_config* cfg, const void* A_
     cudaFree(Bv_rot);
   }
   if (e != cudaSuccess) return fail(STARKV_ERR_CUDA, "fold M");
+  // tensor-core score kernel: MMA items, RoPE table
+  L->tc_scores = plan_scores_tc(L);
+  if (L->tc_scores) {
+    if (cudaMalloc(&L->d_items, sizeof(ScoreItem) * L->items.size()) != cudaSuccess ||
+        cudaMalloc(&L->rope_E, (size_t)L->rope_tiles * 32768) != cudaSuccess)
+      return fail(STARKV_ERR_OOM, "cudaMalloc");
+    if (cudaMemcpyAsync(L->d_items, L->items.data(), sizeof(ScoreItem) * L->items.size(), cudaMemcpyHostToDevice,
+                        s) != cudaSuccess ||
+        build_rope_table(L, s) != cudaSuccess)
+      return fail(STARKV_ERR_CUDA, "rope table");
+    cudaStreamSynchronize(s);   // the item table lives in a host vector that must outlive the copy
+  }
   *out = L;
   return STARKV_OK;
 }
@@ -356,6 +370,7 @@ size_t starkv_workspace_bytes(const starkv_layer* L, int batch, int max_ctx, int
   if (max_q < 1) max_q = 1;
   max_ctx = std::max(max_ctx, 1);
   size_t need = decode_generic_ws_bytes(L, batch, max_ctx, false);
+  if (L->tc_scores) need += scores_tc_ws_bytes(L, batch, max_ctx);
   if (max_q > 1) {
     const long long rows = std::min<long long>((long long)batch * max_q, 1 << 30);
     need = std::max(need, ru(sizeof(int32_t) * 3 * (size_t)rows, 256) +
@@ -374,14 +389,17 @@ starkv_status starkv_decode_attn(const starkv_layer* L, const void* pool, int64_
   CHECK_ARG(pool && page_table && seq_lens && q && out, "NULL buffer");
   CHECK_ARG(n_pages > 0 && max_pages > 0, "empty pool or page table");
   const int max_len = max_pages * kPage;
-  const size_t need = decode_generic_ws_bytes(L, batch, max_len, false);
+  const bool tc_ok = L->tc_scores && max_len <= L->rope_tiles * 128;
+  const bool use_tc_scores = tc_ok && (L->decode_path == 2 || L->decode_path == 0);
+  const size_t need = decode_generic_ws_bytes(L, batch, max_len, false) +
+                      (L->tc_scores ? scores_tc_ws_bytes(L, batch, max_len) : 0);
   if (workspace == nullptr || ws_bytes < need) {
     set_error("decode workspace too small: need " + std::to_string(need) + " bytes");
     return STARKV_ERR_WORKSPACE;
   }
   RowInfo ri{nullptr, seq_lens, q_pos};
   CUDA_TRY(launch_decode_generic(L, (const uint8_t*)pool, n_pages, page_table, max_pages, batch, ri, max_len, q, out,
-                                 workspace, ws_bytes, false, (cudaStream_t)stream));
+                                 workspace, ws_bytes, false, (cudaStream_t)stream, use_tc_scores));
   return STARKV_OK;
 }
 
@@ -426,6 +444,18 @@ starkv_status starkv_prefill_attn(const starkv_layer* L, const void* pool, int64
                                  (char*)workspace + tab_bytes, ws_bytes - tab_bytes, true, s));
   // pageable host source: make sure the copy has consumed `tab` before it is freed
   CUDA_TRY(cudaStreamSynchronize(s));
+  return STARKV_OK;
+}
+
+starkv_status starkv_set_decode_path(starkv_layer* L, int path) {
+  set_error("");
+  CHECK_ARG(L != nullptr, "layer is NULL");
+  CHECK_ARG(path >= 0 && path <= 2, "path must be 0, 1 or 2");
+  if (path == 2 && !L->tc_scores) {
+    set_error("this layer's shape does not fit the tensor-core score kernel");
+    return STARKV_ERR_UNSUPPORTED;
+  }
+  L->decode_path = path;
   return STARKV_OK;
 }
 

@@ -363,7 +363,7 @@ size_t decode_generic_ws_bytes(const starkv_layer* L, int rows, int max_len, boo
 cudaError_t launch_decode_generic(const starkv_layer* L, const uint8_t* pool, long long n_pages,
                                   const int32_t* page_table, int max_pages, int rows, RowInfo ri, int max_len,
                                   const void* q, void* out, void* ws, size_t ws_bytes, bool prefill,
-                                  cudaStream_t s) {
+                                  cudaStream_t s, bool tc_scores) {
   const LayerView& v = L->view;
   const WsPlan p = plan_ws(L, rows, max_len, prefill);
   if (ws_bytes < p.total) return cudaErrorInvalidValue;
@@ -381,13 +381,22 @@ cudaError_t launch_decode_generic(const starkv_layer* L, const uint8_t* pool, lo
   int rmax = 0;
   for (int g = 0; g < v.Hkv; ++g) rmax = std::max(rmax, L->lat[g].width);
   const size_t smem = sizeof(float) * kTile * (size_t)(rmax + v.d);
-  static bool attr_set = false;
-  if (!attr_set) {
-    cudaFuncSetAttribute(k_scores, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
-    attr_set = true;
+  static size_t attr_set = 0;
+  if (smem > attr_set) {
+    cudaError_t e = cudaFuncSetAttribute(k_scores, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    attr_set = smem;
   }
-  k_scores<<<dim3((max_len + kTile - 1) / kTile, v.Hkv, rows), 256, smem, s>>>(
-      v, pool, n_pages, page_table, max_pages, ri, L->Bk, L->d_key_off, qrot, S, p.S_ld);
+  if (tc_scores) {
+    // scores (log2 units) from the tensor-core kernel, written into S
+    ScoreOut so;
+    cudaError_t e = launch_scores_tc(L, pool, n_pages, page_table, max_pages, rows, ri.row_len, ri.row_pos, q,
+                                     w + p.total, &so, S, p.S_ld, s);
+    if (e != cudaSuccess) return e;
+  } else {
+    k_scores<<<dim3((max_len + kTile - 1) / kTile, v.Hkv, rows), 256, smem, s>>>(
+        v, pool, n_pages, page_table, max_pages, ri, L->Bk, L->d_key_off, qrot, S, p.S_ld);
+  }
   const int vb = value_block(v);
   const int cblocks = (v.rv + vb - 1) / vb;
   k_value<<<dim3(cblocks, p.n_splits, rows), kVBlock, 0, s>>>(v, pool, n_pages, page_table, max_pages, ri, S, p.S_ld,

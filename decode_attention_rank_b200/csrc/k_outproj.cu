@@ -226,10 +226,11 @@ cudaError_t launch_outproj_tc(const starkv_layer* L, const void* y_tiles, int ro
   a.tmem_cols = cols;
   a.status = L->status;
   const size_t smem = (size_t)a.stages * stage_bytes + 1024;
-  static bool attr = false;
-  if (!attr) {
-    cudaFuncSetAttribute(k_outproj_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, 220 * 1024);
-    attr = true;
+  static size_t attr = 0;
+  if (smem > attr) {
+    cudaError_t e = cudaFuncSetAttribute(k_outproj_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    attr = smem;
   }
   for (int t = 0; t < ntiles; ++t) {
     OutArgs at = a;

@@ -62,6 +62,26 @@ struct LayerView {
   uint32_t* status;
 };
 
+// One MMA item of the tensor-core score kernel: consecutive query heads whose
+// W'' rows (sum of ranks <= 128) form the B operand of one 128 x npad MMA.
+struct ScoreItem {
+  int h0, nh, npad;   // first query head, heads, MMA N (multiple of 16)
+  int w_off;          // byte offset of the item's W'' block in one sequence's W'' buffer
+  int key_off;        // byte range of the item's key latent blocks inside a page
+  int key_bytes;
+  int hcol[8];        // G column of each head's first latent channel
+  int hr[8];          // rank of each head
+};
+
+// Outputs of the tensor-core score kernel.
+struct ScoreOut {
+  __nv_bfloat16* P;   // [B][H][P_ld] exp2(s - m_st) per 256-token super-tile
+  float* m_st;        // [B][H][n_st]
+  float* l_st;        // [B][H][n_st] sum of the bf16 P values
+  long long P_ld;
+  int n_st;
+};
+
 }  // namespace starkv
 
 struct starkv_layer {
@@ -87,6 +107,15 @@ struct starkv_layer {
   void* M_T = nullptr;
   int Kp = 0, Dp = 0;           // H * wv and D rounded up to 64 and 128
   uint32_t* status = nullptr;
+  // tensor-core score kernel
+  bool tc_scores = false;
+  std::vector<starkv::ScoreItem> items;
+  starkv::ScoreItem* d_items = nullptr;
+  long long w_stride = 0;
+  int w_stage = 0, k_stage = 0, WS = 0, KS = 0;
+  int rope_tiles = 0;
+  void* rope_E = nullptr;       // RoPE table tiles, 32 KB per 128 positions
+  int decode_path = 0;          // 0 auto, 1 CUDA cores, 2 tensor-core scores + CUDA-core values
 };
 
 namespace starkv {
@@ -114,10 +143,17 @@ struct RowInfo {
 cudaError_t launch_decode_generic(const starkv_layer* L, const uint8_t* pool, long long n_pages,
                                   const int32_t* page_table, int max_pages, int rows, RowInfo ri, int max_len,
                                   const void* q, void* out, void* ws, size_t ws_bytes, bool prefill,
-                                  cudaStream_t s);
+                                  cudaStream_t s, bool tc_scores = false);
 size_t decode_generic_ws_bytes(const starkv_layer* L, int rows, int max_len, bool prefill);
 
 int num_sms();
+
+bool plan_scores_tc(starkv_layer* L);
+cudaError_t build_rope_table(starkv_layer* L, cudaStream_t s);
+size_t scores_tc_ws_bytes(const starkv_layer* L, int batch, int max_len);
+cudaError_t launch_scores_tc(const starkv_layer* L, const uint8_t* pool, long long n_pages, const int32_t* pt,
+                             int max_pages, int batch, const int32_t* seq_lens, const int32_t* q_pos, const void* q,
+                             void* ws, ScoreOut* out, float* S_dbg, long long S_ld, cudaStream_t s);
 
 // Tensor-core output kernel (bf16 layers).
 struct OutGeom {

@@ -64,6 +64,19 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint32
   return false;
 }
 
+// Bounded wait that also gives up as soon as another role of the CTA has
+// aborted (*abort != 0), so that every role drains quickly and in step.
+__device__ __forceinline__ bool mbar_wait_ab(uint64_t* bar, uint32_t parity, uint32_t* status,
+                                             volatile int* abort) {
+  for (uint32_t i = 0; i < kSpinLimit; ++i) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if ((i & 63u) == 63u && *abort) return false;
+  }
+  if (status) atomicOr(status, kTimeout);
+  *abort = 1;
+  return false;
+}
+
 // ---- bulk copies (global -> shared, completion on an mbarrier) -------------
 __device__ __forceinline__ void bulk_g2s(void* smem_dst, const void* gmem_src, uint32_t bytes, uint64_t* bar) {
   asm volatile(

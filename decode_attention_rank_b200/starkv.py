@@ -31,7 +31,7 @@ DEV_BAD_PAGE, DEV_BAD_POSITION, DEV_SCALE_OVF, DEV_TIMEOUT = 0x1, 0x2, 0x4, 0x8
 EXPORTED = ["starkv_load_factors", "starkv_free_layer", "starkv_layer_get_info", "starkv_page_bytes",
             "starkv_cache_init", "starkv_append", "starkv_append_workspace_bytes", "starkv_decode_attn",
             "starkv_prefill_attn", "starkv_workspace_bytes", "starkv_sync_status", "starkv_status_string",
-            "starkv_last_error", "starkv_version", "starkv_decode_attn_noalloc"]
+            "starkv_last_error", "starkv_version", "starkv_decode_attn_noalloc", "starkv_set_decode_path"]
 NOALLOC_SCRATCH_BYTES = 32 << 20
 
 
@@ -42,7 +42,7 @@ class _Config(ctypes.Structure):
                 ("top_fraction", ctypes.c_float), ("top_bits", ctypes.c_int), ("bottom_bits", ctypes.c_int),
                 ("group_size", ctypes.c_int), ("hadamard_block", ctypes.c_int), ("rope", ctypes.c_int),
                 ("rope_theta", ctypes.c_double), ("softmax_scale", ctypes.c_float), ("page_size", ctypes.c_int),
-                ("plain", ctypes.c_int)]
+                ("plain", ctypes.c_int), ("max_positions", ctypes.c_int)]
 
 
 class _Info(ctypes.Structure):
@@ -76,6 +76,7 @@ _lib.starkv_status_string.argtypes = [ctypes.c_int]
 _lib.starkv_status_string.restype = ctypes.c_char_p
 _lib.starkv_last_error.argtypes = []
 _lib.starkv_last_error.restype = ctypes.c_char_p
+_lib.starkv_set_decode_path.argtypes = [_vp, ctypes.c_int]
 _lib.starkv_version.argtypes = []
 _lib.starkv_version.restype = ctypes.c_char_p
 
@@ -130,6 +131,7 @@ class LayerConfig:
     softmax_scale: float = 0.0
     page_size: int = 16
     plain: bool = False
+    max_positions: int = 0
 
     @classmethod
     def from_spec(cls, spec) -> "LayerConfig":
@@ -145,7 +147,7 @@ class LayerConfig:
                     ctypes.cast(ranks, ctypes.POINTER(ctypes.c_int)) if self.key_ranks else None, self.value_rank,
                     STARKV_F32 if self.dtype == "f32" else STARKV_BF16, int(self.quantized), self.top_fraction,
                     self.top_bits, self.bottom_bits, self.group_size, self.hadamard_block, int(self.rope),
-                    self.rope_theta, self.softmax_scale, self.page_size, int(self.plain))
+                    self.rope_theta, self.softmax_scale, self.page_size, int(self.plain), self.max_positions)
         return c, ranks
 
 
@@ -216,6 +218,10 @@ class Layer:
                                         ctypes.cast(qs, _vp), ctypes.cast(ql, _vp), _ptr(q), _ptr(out),
                                         _ptr(workspace), workspace.numel() * workspace.element_size(),
                                         _stream(stream)), "starkv_prefill_attn")
+
+    def set_decode_path(self, path: int) -> None:
+        """0 automatic, 1 CUDA-core kernels, 2 tensor-core scores + CUDA-core values (diagnostics)."""
+        _check(_lib.starkv_set_decode_path(self._h, path), "starkv_set_decode_path")
 
     def sync_status(self, stream=None) -> int:
         bits = ctypes.c_uint32(0)

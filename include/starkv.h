@@ -92,6 +92,9 @@ typedef enum { STARKV_F32 = 0, STARKV_BF16 = 1 } starkv_dtype;
  *   plain: 1 = uncompressed layer (protected layers 0, 1 and 31 in the notes'
  *     Algorithm 1): K (after RoPE) and V are stored in dtype, width d per
  *     KV head each; no factors.
+ *   max_positions: length of the layer's RoPE table for the tensor-core score
+ *     kernel (0 selects 32768); 256 bytes of device memory per position.
+ *     Decodes whose page table reaches beyond it use the CUDA-core path.
  */
 typedef struct {
   int hidden, n_heads, n_kv_heads, head_dim;
@@ -108,6 +111,7 @@ typedef struct {
   float softmax_scale;
   int page_size;
   int plain;
+  int max_positions;
 } starkv_layer_config;
 
 typedef struct starkv_layer starkv_layer;   /* opaque */
@@ -256,6 +260,16 @@ STARKV_API const char* starkv_last_error(void);
 
 /* Library build string (version, target architecture). */
 STARKV_API const char* starkv_version(void);
+
+/*
+ * Diagnostics: choose the decode implementation of a layer.
+ *   0 = automatic (tensor-core kernels where the layer's shape allows them),
+ *   1 = CUDA-core kernels for every step,
+ *   2 = tensor-core score kernel feeding the CUDA-core value kernels.
+ * Results agree within the attention tolerance; the choice exists so that each
+ * implementation can be checked and timed on its own.
+ */
+STARKV_API starkv_status starkv_set_decode_path(starkv_layer* layer, int path);
 
 #ifdef __cplusplus
 }

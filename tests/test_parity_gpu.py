@@ -24,9 +24,11 @@ def case(cfg: int, quantized: bool = False, layer: int = 2) -> Case:
     return Case(spec, gen.LAYER_SEED[cfg], layer if cfg == 4 else 0)
 
 
-def run_decode(c: Case, lens, peaky=1.0, use_hidden=True, check_pool=True, q_pos=None, page_seed=0):
+def run_decode(c: Case, lens, peaky=1.0, use_hidden=True, check_pool=True, q_pos=None, page_seed=0, path=0):
     """Fill a cache (latent mode), decode one query per sequence, compare with the oracle."""
     L = c.load()
+    if path:
+        L.set_decode_path(path)
     s = c.spec
     cache = GpuCache(L, lens, seed=page_seed)
     lat_all = []
@@ -193,6 +195,17 @@ def test_prefill_two_output_tiles():
     for i in (0, 1, 255, 256, 299):
         want = O.decode(s, c.f, Zs, Q[i], T0 + i, T0 + i + 1, c.B_rot)
         check_close(got[i], want, f"prefill row {i}")
+
+
+@pytest.mark.parametrize("cfg,quant,lens", [
+    (2, False, [600, 257, 256, 1]),
+    (3, True, [300, 97]),
+])
+def test_tc_scores_feeding_cuda_core_values(cfg, quant, lens):
+    """Tensor-core score kernel (path 2) against the oracle, with multiple and
+    partial 256-token super-tiles."""
+    run_decode(case(cfg, quantized=quant), lens, use_hidden=False, check_pool=False, path=2)
+    run_decode(case(cfg, quantized=quant), lens[:2], peaky=25.0, use_hidden=False, check_pool=False, path=2)
 
 
 def test_device_status_bad_page():
