@@ -295,6 +295,7 @@ starkv_status starkv_load_factors(const starkv_layer_config* cfg, const void* A_
   if (e != cudaSuccess) return fail(STARKV_ERR_CUDA, "fold M");
   // tensor-core score kernel: MMA items, RoPE table
   L->tc_scores = plan_scores_tc(L);
+  L->tc_values = L->tc_scores && plan_values_tc(L);
   if (L->tc_scores) {
     if (cudaMalloc(&L->d_items, sizeof(ScoreItem) * L->items.size()) != cudaSuccess ||
         cudaMalloc(&L->rope_E, (size_t)L->rope_tiles * 32768) != cudaSuccess)
@@ -371,6 +372,7 @@ size_t starkv_workspace_bytes(const starkv_layer* L, int batch, int max_ctx, int
   max_ctx = std::max(max_ctx, 1);
   size_t need = decode_generic_ws_bytes(L, batch, max_ctx, false);
   if (L->tc_scores) need += scores_tc_ws_bytes(L, batch, max_ctx);
+  if (L->tc_values) need = std::max(need, decode_tc_ws_bytes(L, batch, max_ctx));
   if (max_q > 1) {
     const long long rows = std::min<long long>((long long)batch * max_q, 1 << 30);
     need = std::max(need, ru(sizeof(int32_t) * 3 * (size_t)rows, 256) +
@@ -390,12 +392,19 @@ starkv_status starkv_decode_attn(const starkv_layer* L, const void* pool, int64_
   CHECK_ARG(n_pages > 0 && max_pages > 0, "empty pool or page table");
   const int max_len = max_pages * kPage;
   const bool tc_ok = L->tc_scores && max_len <= L->rope_tiles * 128;
+  const bool use_tc_all = tc_ok && L->tc_values && L->decode_path == 0;
   const bool use_tc_scores = tc_ok && (L->decode_path == 2 || L->decode_path == 0);
-  const size_t need = decode_generic_ws_bytes(L, batch, max_len, false) +
-                      (L->tc_scores ? scores_tc_ws_bytes(L, batch, max_len) : 0);
+  size_t need = decode_generic_ws_bytes(L, batch, max_len, false) +
+                (L->tc_scores ? scores_tc_ws_bytes(L, batch, max_len) : 0);
+  if (use_tc_all) need = decode_tc_ws_bytes(L, batch, max_len);
   if (workspace == nullptr || ws_bytes < need) {
     set_error("decode workspace too small: need " + std::to_string(need) + " bytes");
     return STARKV_ERR_WORKSPACE;
+  }
+  if (use_tc_all) {
+    CUDA_TRY(launch_decode_tc(L, (const uint8_t*)pool, n_pages, page_table, max_pages, batch, seq_lens, q_pos, q, out,
+                              workspace, ws_bytes, (cudaStream_t)stream));
+    return STARKV_OK;
   }
   RowInfo ri{nullptr, seq_lens, q_pos};
   CUDA_TRY(launch_decode_generic(L, (const uint8_t*)pool, n_pages, page_table, max_pages, batch, ri, max_len, q, out,

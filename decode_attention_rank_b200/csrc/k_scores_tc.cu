@@ -50,7 +50,7 @@ struct ScoreArgs {
   int gq;                  // query heads per KV head
   int n_st;                // super-tiles per sequence
   long long U;             // batch * n_st
-  __nv_bfloat16* P;        // [B][H][P_ld]
+  __half* P;               // [B][H][P_ld]
   long long P_ld;
   float* m_st;             // [B][H][n_st]
   float* l_st;
@@ -351,9 +351,9 @@ __global__ void __launch_bounds__(kScoreThreads, 1) k_scores_tc(ScoreArgs a) {
           mloc[hh] = m;
           float p = 0.f;
           if (valid && hh < item.nh) {
-            const __nv_bfloat16 pb = __float2bfloat16_rn(exp2f(s[hh] - m));
+            const __half pb = __float2half_rn(exp2f(s[hh] - m));
             a.P[(hb + hh) * a.P_ld + t] = pb;
-            p = __bfloat162float(pb);
+            p = __half2float(pb);
           }
           for (int o = 16; o > 0; o >>= 1) p += __shfl_xor_sync(0xffffffffu, p, o);
           lsum[hh] = p;
@@ -523,7 +523,7 @@ cudaError_t launch_scores_tc(const starkv_layer* L, const uint8_t* pool, long lo
   w += r((size_t)batch * L->w_stride);
   out->P_ld = S_dbg ? S_ld : (long long)n_st * kSuper;
   out->n_st = n_st;
-  out->P = (__nv_bfloat16*)w;
+  out->P = (__half*)w;
   w += r(2 * (size_t)batch * v.H * n_st * kSuper);
   out->m_st = (float*)w;
   w += r(sizeof(float) * (size_t)batch * v.H * n_st);

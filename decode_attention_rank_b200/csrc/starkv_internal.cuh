@@ -75,7 +75,7 @@ struct ScoreItem {
 
 // Outputs of the tensor-core score kernel.
 struct ScoreOut {
-  __nv_bfloat16* P;   // [B][H][P_ld] exp2(s - m_st) per 256-token super-tile
+  __half* P;          // [B][H][P_ld] exp2(s - m_st) per 256-token super-tile, fp16
   float* m_st;        // [B][H][n_st]
   float* l_st;        // [B][H][n_st] sum of the bf16 P values
   long long P_ld;
@@ -116,6 +116,9 @@ struct starkv_layer {
   int rope_tiles = 0;
   void* rope_E = nullptr;       // RoPE table tiles, 32 KB per 128 positions
   int decode_path = 0;          // 0 auto, 1 CUDA cores, 2 tensor-core scores + CUDA-core values
+  // tensor-core value kernel
+  bool tc_values = false;
+  int vblk_off = 0, vblk_bytes = 0;
 };
 
 namespace starkv {
@@ -149,6 +152,15 @@ size_t decode_generic_ws_bytes(const starkv_layer* L, int rows, int max_len, boo
 int num_sms();
 
 bool plan_scores_tc(starkv_layer* L);
+bool plan_values_tc(starkv_layer* L);
+size_t values_tc_ws_bytes(const starkv_layer* L, int batch, int max_len);
+cudaError_t launch_values_tc(const starkv_layer* L, const uint8_t* pool, long long n_pages, const int32_t* pt,
+                             int max_pages, int batch, const int32_t* seq_lens, const ScoreOut& so, void* ws,
+                             void* ytiles, cudaStream_t s);
+cudaError_t launch_decode_tc(const starkv_layer* L, const uint8_t* pool, long long n_pages, const int32_t* pt,
+                             int max_pages, int batch, const int32_t* seq_lens, const int32_t* q_pos, const void* q,
+                             void* out, void* ws, size_t ws_bytes, cudaStream_t s);
+size_t decode_tc_ws_bytes(const starkv_layer* L, int batch, int max_len);
 cudaError_t build_rope_table(starkv_layer* L, cudaStream_t s);
 size_t scores_tc_ws_bytes(const starkv_layer* L, int batch, int max_len);
 cudaError_t launch_scores_tc(const starkv_layer* L, const uint8_t* pool, long long n_pages, const int32_t* pt,

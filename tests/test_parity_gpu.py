@@ -208,6 +208,20 @@ def test_tc_scores_feeding_cuda_core_values(cfg, quant, lens):
     run_decode(case(cfg, quantized=quant), lens[:2], peaky=25.0, use_hidden=False, check_pool=False, path=2)
 
 
+def test_tc_long_context_runs():
+    """All-tensor-core decode with more super-tiles than SMs: CTAs whose unit
+    ranges span several super-tiles and cross sequence boundaries."""
+    run_decode(case(2), [20000, 9000, 37], use_hidden=False, check_pool=False)
+    run_decode(case(2), [12000, 12000], peaky=25.0, use_hidden=False, check_pool=False)
+
+
+def test_decode_paths_agree():
+    """CUDA-core path (1), tensor-core scores (2) and all tensor-core (0) agree."""
+    outs = [run_decode(case(2), [700, 300], use_hidden=False, check_pool=False, path=p) for p in (1, 2, 0)]
+    for o in outs[1:]:
+        assert np.linalg.norm(o - outs[0]) <= 3e-3 * np.linalg.norm(outs[0])
+
+
 def test_device_status_bad_page():
     """An out-of-range page id is caught by the kernels (status word), not dereferenced."""
     c = case(0)
