@@ -249,10 +249,12 @@ def run_ours(args, rank, ws, local):
     t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     torch.cuda.synchronize()
     barrier(ws)
+    torch.cuda.nvtx.range_push("timed")
     t_start.record(stream)
     for k in range(K):
         step(W + k, page_table, evs[k])
     t_end.record(stream)
+    torch.cuda.nvtx.range_pop()
     torch.cuda.synchronize()
     barrier(ws)
     ms_total = t_start.elapsed_time(t_end)

@@ -25,7 +25,7 @@ int num_sms() {
   if (cached[dev] == 0) {
     int n = 0;
     if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
-    cached[dev] = n;
+    cached[dev] = std::min(n, 256);   // persistent grids: one CTA per SM, at most 256
   }
   return cached[dev];
 }
@@ -200,7 +200,9 @@ void starkv_free_layer(starkv_layer* L) {
   cudaFree(L->d_lat);
   cudaFree(L->d_grp);
   cudaFree(L->d_key_off);
+  cudaFree(L->d_grp_lat);
   cudaFree(L->A_T);
+  cudaFree(L->A_tiles);
   cudaFree(L->Bk);
   cudaFree(L->M_T);
   cudaFree(L->status);
@@ -247,6 +249,12 @@ starkv_status starkv_load_factors(const starkv_layer_config* cfg, const void* A_
   v.lat = L->d_lat;
   v.grp = L->d_grp;
   v.status = L->status;
+  std::vector<int> grp_lat(L->grp.size());
+  for (size_t li = 0; li < L->lat.size(); ++li)
+    for (int g = 0; g < L->lat[li].n_groups; ++g) grp_lat[L->lat[li].group0 + g] = (int)li;
+  if (cudaMalloc(&L->d_grp_lat, sizeof(int) * grp_lat.size()) != cudaSuccess) return fail(STARKV_ERR_OOM, "cudaMalloc");
+  if (cudaMemcpy(L->d_grp_lat, grp_lat.data(), sizeof(int) * grp_lat.size(), cudaMemcpyHostToDevice) != cudaSuccess)
+    return fail(STARKV_ERR_CUDA, "upload group table");
   if (cudaMemcpyAsync(L->d_lat, L->lat.data(), sizeof(LatentDesc) * L->lat.size(), cudaMemcpyHostToDevice, s) ||
       cudaMemcpyAsync(L->d_grp, L->grp.data(), sizeof(GroupDesc) * L->grp.size(), cudaMemcpyHostToDevice, s) ||
       cudaMemcpyAsync(L->d_key_off, L->key_off.data(), sizeof(int) * L->key_off.size(), cudaMemcpyHostToDevice, s) ||
@@ -276,6 +284,13 @@ starkv_status starkv_load_factors(const starkv_layer_config* cfg, const void* A_
         return fail(STARKV_ERR_CUDA, "rotate B_k");
       boff += (size_t)L->key_ranks[h] * d;
     }
+  }
+  // the projection rows again as fp16 128 x 64 tiles for the tensor-core projection
+  if (cfg->dtype == STARKV_BF16) {
+    const size_t tb = (size_t)((v.Ltot + 127) / 128) * ((D + 63) / 64) * 16384;
+    if (cudaMalloc(&L->A_tiles, tb) != cudaSuccess) return fail(STARKV_ERR_OOM, "cudaMalloc");
+    if (launch_pack_rows_tiles(L->A_T, v.Ltot, D, L->A_tiles, s, 128) != cudaSuccess)
+      return fail(STARKV_ERR_CUDA, "tile A");
   }
   // M_h = B'_v,kv(h) W_o,h, stored transposed as M_T [D][H * wv].
   float* Bv_rot = nullptr;
@@ -334,7 +349,10 @@ starkv_status starkv_cache_init(const starkv_layer* L, void* pool, int64_t n_pag
 
 size_t starkv_append_workspace_bytes(const starkv_layer* L, int n_tokens) {
   if (!L || n_tokens <= 0) return 0;
-  return ru(sizeof(float) * (size_t)n_tokens * L->view.Ltot, 256);
+  size_t b = ru(sizeof(float) * (size_t)n_tokens * L->view.Ltot, 256);
+  if (L->A_tiles)
+    b += ru(rows_tiles_bytes(n_tokens, L->view.D), 256) + ru(gemm_part_bytes(L->view.Ltot, L->view.D, n_tokens), 256);
+  return b;
 }
 
 starkv_status starkv_append(const starkv_layer* L, void* pool, int64_t n_pages, const int32_t* page_table,
@@ -356,7 +374,19 @@ starkv_status starkv_append(const starkv_layer* L, void* pool, int64_t n_pages, 
       set_error("append workspace too small");
       return STARKV_ERR_WORKSPACE;
     }
-    CUDA_TRY(launch_project(L, input, n_tokens, (float*)workspace, s));
+    if (L->A_tiles) {
+      // tensor cores: z^T = A_T x^T with the stream-K GEMM of the output projection
+      uint8_t* w = (uint8_t*)workspace;
+      float* zw = (float*)w;
+      w += ru(sizeof(float) * (size_t)n_tokens * L->view.Ltot, 256);
+      void* xt = w;
+      w += ru(rows_tiles_bytes(n_tokens, L->view.D), 256);
+      CUDA_TRY(launch_pack_rows_tiles(input, n_tokens, L->view.D, xt, s));
+      CUDA_TRY(launch_gemm_tc((const uint8_t*)L->A_tiles, L->view.Ltot, L->view.D, L->view.Ltot, xt, n_tokens, zw,
+                              true, (float*)w, L->status, s));
+    } else {
+      CUDA_TRY(launch_project(L, input, n_tokens, (float*)workspace, s));
+    }
     z = (const float*)workspace;
   }
   const int rotate = (!input_is_latent && L->view.hadamard) ? 1 : 0;

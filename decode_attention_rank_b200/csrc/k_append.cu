@@ -142,12 +142,71 @@ __global__ void k_pack(LayerView v, uint8_t* __restrict__ pool, long long n_page
   }
 }
 
+// Quantized latents: one warp per (token, group) so that no warp walks a
+// latent's groups one after another.
+__global__ void k_pack_groups(LayerView v, const int* __restrict__ grp_lat, int n_grp, uint8_t* __restrict__ pool,
+                              long long n_pages, const int32_t* __restrict__ pt, int n_seqs, int max_pages, int n,
+                              const int32_t* __restrict__ seq_idx, const int32_t* __restrict__ pos,
+                              const float* __restrict__ z, int rotate) {
+  const long long warp = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  const int i = (int)(warp / n_grp), fg = (int)(warp % n_grp);
+  if (i >= n) return;
+  const int b = seq_idx[i], t = pos[i];
+  const int li = grp_lat[fg];
+  const LatentDesc ld = v.lat[li];
+  const GroupDesc gd = v.grp[fg];
+  const int g = fg - ld.group0;
+  const bool first = (g == 0);
+  if (b < 0 || b >= n_seqs || t < 0 || t >= max_pages * kPage) {
+    if (lane == 0 && first) atomicOr(v.status, kBadPos);
+    return;
+  }
+  const int page = pt[(size_t)b * max_pages + t / kPage];
+  if (page < 0 || page >= n_pages) {
+    if (lane == 0 && first) atomicOr(v.status, kBadPage);
+    return;
+  }
+  const int slot = t % kPage;
+  uint8_t* blk = pool + (size_t)page * v.page_bytes + ld.block_off;
+  float x = lane < gd.n ? z[(size_t)i * v.Ltot + ld.ch_off + gd.start + lane] : 0.f;
+  if (rotate) x = group_fwht(x, lane, gd.n);
+  float amax = lane < gd.n ? fabsf(x) : 0.f;
+  for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+  const int qmax = (1 << (gd.bits - 1)) - 1;
+  const float s32 = __fdiv_rn(amax, (float)qmax);
+  if (!(s32 <= 65504.f)) {
+    if (lane == 0) atomicOr(v.status, kScaleOvf);
+    return;
+  }
+  const __half s16 = __float2half_ru(s32);
+  const float sf = __half2float(s16);
+  int q = 0;
+  if (sf != 0.f) q = min(max(__float2int_rn(__fdiv_rn(x, sf)), -qmax), qmax);
+  const uint32_t u = (uint32_t)(q + (1 << (gd.bits - 1)));
+  if (lane == 0) reinterpret_cast<__half*>(blk)[g * kPage + slot] = s16;
+  if (lane < gd.n) {
+    const uint32_t bit = (uint32_t)(slot * gd.n + lane) * gd.bits;
+    uint32_t* w = reinterpret_cast<uint32_t*>(blk + gd.code_off) + (bit >> 5);
+    const uint32_t sh = bit & 31;
+    atomicOr(w, u << sh);
+    if (sh + gd.bits > 32) atomicOr(w + 1, u >> (32 - sh));
+  }
+}
+
 cudaError_t launch_pack(const starkv_layer* L, uint8_t* pool, long long n_pages, const int32_t* page_table,
                         int n_seqs, int max_pages, int n, const int32_t* seq_idx, const int32_t* positions, const float* z,
                         int rotate, int rope_keys, cudaStream_t s) {
   const LayerView& v = L->view;
-  const long long warps = (long long)n * v.L;
   const int threads = 256;
+  if (v.quantized && L->d_grp_lat) {
+    const int ng = (int)L->grp.size();
+    const long long warps = (long long)n * ng;
+    k_pack_groups<<<(unsigned)((warps * 32 + threads - 1) / threads), threads, 0, s>>>(
+        v, L->d_grp_lat, ng, pool, n_pages, page_table, n_seqs, max_pages, n, seq_idx, positions, z, rotate);
+    return cudaGetLastError();
+  }
+  const long long warps = (long long)n * v.L;
   const unsigned blocks = (unsigned)((warps * 32 + threads - 1) / threads);
   k_pack<<<blocks, threads, 0, s>>>(v, pool, n_pages, page_table, n_seqs, max_pages, n, seq_idx, positions, z, rotate,
                                     rope_keys);

@@ -17,17 +17,6 @@ namespace starkv {
 
 int outproj_nb(int rows) { return (std::min(std::max(rows, 1), 256) + 15) / 16 * 16; }
 
-OutGeom outproj_geom(const starkv_layer* L) {
-  OutGeom g;
-  g.KT = L->Kp / 64;
-  g.DT = L->Dp / 128;
-  const long long U = (long long)g.KT * g.DT;
-  g.G = (int)std::min<long long>(num_sms(), U);
-  const long long per = (U + g.G - 1) / g.G;
-  g.slots = (int)((per + g.KT - 1) / g.KT) + 1;
-  return g;
-}
-
 namespace {
 
 constexpr int kOutThreads = 192;  // warp 0 producer, warp 1 MMA, warps 2-5 epilogue
@@ -175,24 +164,35 @@ __global__ void __launch_bounds__(kOutThreads, 1) k_outproj_tc(OutArgs a) {
 template <typename TO>
 __global__ void k_outproj_reduce(const float* __restrict__ part, int G, int KT, int DT, int slots, int NB, int rows,
                                  int D, TO* __restrict__ out) {
+  __shared__ long long seg_off[256];
+  __shared__ int n_seg;
   const int dt = blockIdx.x, row = blockIdx.y;
   const int nt = row / NB, b = row % NB;
-  const long long U = (long long)DT * KT;
-  const long long lo = (long long)dt * KT, hi = lo + KT;
-  // CTAs c with [begin(c), begin(c+1)) intersecting [lo, hi)
-  int c_lo = (int)((lo * G) / U);
-  while (c_lo > 0 && unit_begin(c_lo, G, U) > lo) --c_lo;
-  while (unit_begin(c_lo + 1, G, U) <= lo) ++c_lo;
+  if (threadIdx.x == 0) {
+    const long long U = (long long)DT * KT;
+    const long long lo = (long long)dt * KT, hi = lo + KT;
+    int c = (int)((lo * G) / U);
+    while (c > 0 && unit_begin(c, G, U) > lo) --c;
+    while (unit_begin(c + 1, G, U) <= lo) ++c;
+    int n = 0;
+    long long b0 = unit_begin(c, G, U);
+    for (; c < G && b0 < hi && n < 256; ++c) {
+      const long long b1 = unit_begin(c + 1, G, U);
+      if (b1 > lo && b1 > b0) {
+        const int slot = dt - (int)(b0 / KT);
+        seg_off[n++] = ((((long long)nt * G + c) * slots + slot) * NB + b) * 128;
+      }
+      b0 = b1;
+    }
+    n_seg = n;
+  }
+  __syncthreads();
+  const int ns = n_seg;
   for (int n = threadIdx.x; n < 128; n += blockDim.x) {
     const int d = dt * 128 + n;
     if (d >= D) continue;
     float acc = 0.f;
-    for (int cc = c_lo; cc < G && unit_begin(cc, G, U) < hi; ++cc) {
-      const long long b0 = unit_begin(cc, G, U), b1 = unit_begin(cc + 1, G, U);
-      if (b1 <= lo || b0 == b1) continue;
-      const int slot = dt - (int)(b0 / KT);
-      acc += part[((((size_t)nt * G + cc) * slots + slot) * NB + b) * 128 + n];
-    }
+    for (int k = 0; k < ns; ++k) acc += part[seg_off[k] + n];
     out[(size_t)row * D + d] = (TO)acc;
   }
 }
@@ -200,20 +200,34 @@ __global__ void k_outproj_reduce(const float* __restrict__ part, int G, int KT, 
 }  // namespace
 
 // Workspace of the partial sums for `rows` output rows.
-size_t outproj_part_bytes(const starkv_layer* L, int rows) {
+// Geometry of a GEMM over an (n_out x K) matrix of 128 x 64 tiles.
+OutGeom gemm_geom(int n_out, int K) {
+  OutGeom g;
+  g.KT = (K + 63) / 64;
+  g.DT = (n_out + 127) / 128;
+  const long long U = (long long)g.KT * g.DT;
+  g.G = (int)std::min<long long>(num_sms(), U);
+  const long long per = (U + g.G - 1) / g.G;
+  g.slots = (int)((per + g.KT - 1) / g.KT) + 1;
+  return g;
+}
+
+size_t gemm_part_bytes(int n_out, int K, int rows) {
   const int NB = outproj_nb(rows);
   const int ntiles = (rows + NB - 1) / NB;
-  const OutGeom g = outproj_geom(L);
+  const OutGeom g = gemm_geom(n_out, K);
   return sizeof(float) * (size_t)ntiles * g.G * g.slots * NB * 128;
 }
 
-cudaError_t launch_outproj_tc(const starkv_layer* L, const void* y_tiles, int rows, void* out, float* part,
-                              cudaStream_t s) {
-  const OutGeom g = outproj_geom(L);
+size_t outproj_part_bytes(const starkv_layer* L, int rows) { return gemm_part_bytes(L->Dp, L->Kp, rows); }
+
+cudaError_t launch_gemm_tc(const uint8_t* Mt, int n_out, int K, int n_valid, const void* y_tiles, int rows,
+                           void* out, bool out_f32, float* part, uint32_t* status, cudaStream_t s) {
+  const OutGeom g = gemm_geom(n_out, K);
   const int NB = outproj_nb(rows);
   const int ntiles = (rows + NB - 1) / NB;
   OutArgs a;
-  a.M = (const uint8_t*)L->M_T;
+  a.M = Mt;
   a.y = (const uint8_t*)y_tiles;
   a.NB = NB;
   a.KT = g.KT;
@@ -224,7 +238,7 @@ cudaError_t launch_outproj_tc(const starkv_layer* L, const void* y_tiles, int ro
   uint32_t cols = 32;
   while (cols < (uint32_t)(2 * NB)) cols <<= 1;
   a.tmem_cols = cols;
-  a.status = L->status;
+  a.status = status;
   const size_t smem = (size_t)a.stages * stage_bytes + 1024;
   static size_t attr = 0;
   if (smem > attr) {
@@ -238,13 +252,58 @@ cudaError_t launch_outproj_tc(const starkv_layer* L, const void* y_tiles, int ro
     at.part = part + (size_t)t * g.G * g.slots * NB * 128;
     k_outproj_tc<<<dim3(g.G, 1), kOutThreads, smem, s>>>(at);
   }
-  if (L->view.dtype == STARKV_F32)
-    k_outproj_reduce<float><<<dim3(g.DT, rows), 128, 0, s>>>(part, g.G, g.KT, g.DT, g.slots, NB, rows, L->view.D,
+  if (out_f32)
+    k_outproj_reduce<float><<<dim3(g.DT, rows), 128, 0, s>>>(part, g.G, g.KT, g.DT, g.slots, NB, rows, n_valid,
                                                              (float*)out);
   else
     k_outproj_reduce<__nv_bfloat16><<<dim3(g.DT, rows), 128, 0, s>>>(part, g.G, g.KT, g.DT, g.slots, NB, rows,
-                                                                     L->view.D, (__nv_bfloat16*)out);
+                                                                     n_valid, (__nv_bfloat16*)out);
   return cudaGetLastError();
+}
+
+cudaError_t launch_outproj_tc(const starkv_layer* L, const void* y_tiles, int rows, void* out, float* part,
+                              cudaStream_t s) {
+  return launch_gemm_tc((const uint8_t*)L->M_T, L->Dp, L->Kp, L->view.D, y_tiles, rows, out,
+                        L->view.dtype == STARKV_F32, part, L->status, s);
+}
+
+// fp16 B-operand tiles [rows / NB][K / 64][NB][64] (swizzled, zero padded) from a row-major bf16 matrix.
+__global__ void k_pack_rows_tiles(const __nv_bfloat16* __restrict__ x, int rows, int K, int NB, int KT,
+                                  uint8_t* __restrict__ tiles) {
+  const long long idx = (long long)blockIdx.x * blockDim.x + threadIdx.x;   // one 8-column chunk
+  const int nchunk = KT * 8;
+  const int ntiles = (rows + NB - 1) / NB;
+  if (idx >= (long long)ntiles * NB * nchunk) return;
+  const int row = (int)(idx / nchunk), ch = (int)(idx % nchunk);
+  const int kt = ch >> 3, c = ch & 7;
+  uint32_t o[4] = {0u, 0u, 0u, 0u};
+  if (row < rows) {
+#pragma unroll
+    for (int i = 0; i < 8; i += 2) {
+      const int k = kt * 64 + c * 8 + i;
+      const float f0 = k < K ? __bfloat162float(x[(size_t)row * K + k]) : 0.f;
+      const float f1 = k + 1 < K ? __bfloat162float(x[(size_t)row * K + k + 1]) : 0.f;
+      const __half2 h = __floats2half2_rn(f0, f1);
+      o[i / 2] = *reinterpret_cast<const uint32_t*>(&h);
+    }
+  }
+  uint8_t* tile = tiles + ((size_t)(row / NB) * KT + kt) * (size_t)NB * 128;
+  *reinterpret_cast<uint4*>(tile + tc::sw128((uint32_t)(row % NB), (uint32_t)c)) = make_uint4(o[0], o[1], o[2], o[3]);
+}
+
+cudaError_t launch_pack_rows_tiles(const void* x, int rows, int K, void* tiles, cudaStream_t s, int nb) {
+  const int NB = nb > 0 ? nb : outproj_nb(rows);
+  const int KT = (K + 63) / 64;
+  const int ntiles = (rows + NB - 1) / NB;
+  const long long n = (long long)ntiles * NB * KT * 8;
+  k_pack_rows_tiles<<<(unsigned)((n + 255) / 256), 256, 0, s>>>((const __nv_bfloat16*)x, rows, K, NB, KT,
+                                                               (uint8_t*)tiles);
+  return cudaGetLastError();
+}
+
+size_t rows_tiles_bytes(int rows, int K) {
+  const int NB = outproj_nb(rows);
+  return (size_t)((rows + NB - 1) / NB) * ((K + 63) / 64) * NB * 128;
 }
 
 }  // namespace starkv

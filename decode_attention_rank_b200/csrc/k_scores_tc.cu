@@ -18,9 +18,10 @@
 // super-tiles (two M = 128 tiles sharing one W'' load) of one sequence.
 //   warp 0      bulk copies: RoPE table tiles, W'' item blocks, key latent pages
 //   warp 1      tcgen05.mma issue (one thread), TMEM allocation
-//   warps 2-9   epilogue: TMEM -> registers, dequantize + dot, softmax
-//               statistics of the super-tile, P = exp2(s - m) as bf16
-// Outputs per (sequence, head, super-tile): P (bf16), m and l = sum P.
+//   warps 2-17  epilogue (16 warps: TMEM lane quarter x tile x head parity):
+//               TMEM -> registers, dequantize + dot, softmax statistics of
+//               the super-tile, P = exp2(s - m) as fp16
+// Outputs per (sequence, head): P (fp16), and per 32-token group m and l = sum P.
 #include <float.h>
 #include <math.h>
 
@@ -30,7 +31,8 @@ namespace starkv {
 
 namespace {
 
-constexpr int kScoreThreads = 320;
+constexpr int kEpiWarps = 16;
+constexpr int kScoreThreads = 64 + 32 * kEpiWarps;   // producer, MMA, 16 epilogue warps
 constexpr int kSuper = 256;          // tokens per super-tile
 constexpr int kETileBytes = 32768;   // one 128-position RoPE tile (128 x 128 fp16)
 
@@ -52,8 +54,9 @@ struct ScoreArgs {
   long long U;             // batch * n_st
   __half* P;               // [B][H][P_ld]
   long long P_ld;
-  float* m_st;             // [B][H][n_st]
+  float* m_st;             // [B][H][n_g] per 32-token group
   float* l_st;
+  int n_g;
   float* S_dbg;            // optional raw scores [B][H][P_ld]
   int H;
   int w_stage, k_stage, WS, KS;
@@ -62,27 +65,27 @@ struct ScoreArgs {
 
 __device__ __forceinline__ long long unit_lo(int c, int G, long long U) { return (long long)c * U / G; }
 
-__device__ __forceinline__ void tmem_ld8(uint32_t taddr, float* v) {
-  uint32_t r[8];
-  asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];\n\t"
-      "tcgen05.wait::ld.sync.aligned;"
-      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7])
-      : "r"(taddr)
-      : "memory");
-#pragma unroll
-  for (int i = 0; i < 8; ++i) v[i] = __uint_as_float(r[i]);
+// TMEM loads without a wait; tmem_wait() below must follow before any use.
+__device__ __forceinline__ void tmem_ld8_nw(uint32_t taddr, float* v) {
+  asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+               : "=f"(v[0]), "=f"(v[1]), "=f"(v[2]), "=f"(v[3]), "=f"(v[4]), "=f"(v[5]), "=f"(v[6]), "=f"(v[7])
+               : "r"(taddr));
 }
-__device__ __forceinline__ void tmem_ld2(uint32_t taddr, float* v) {
-  uint32_t r[2];
-  asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x2.b32 {%0,%1}, [%2];\n\t"
-      "tcgen05.wait::ld.sync.aligned;"
-      : "=r"(r[0]), "=r"(r[1])
-      : "r"(taddr)
-      : "memory");
-  v[0] = __uint_as_float(r[0]);
-  v[1] = __uint_as_float(r[1]);
+__device__ __forceinline__ void tmem_ld2_nw(uint32_t taddr, float* v) {
+  asm volatile("tcgen05.ld.sync.aligned.32x32b.x2.b32 {%0,%1}, [%2];" : "=f"(v[0]), "=f"(v[1]) : "r"(taddr));
+}
+// Wait for this thread's TMEM loads; the registers are operands so that no use
+// of them can be scheduled before the wait.
+__device__ __forceinline__ void tmem_wait(float* g, float* t) {
+  asm volatile("tcgen05.wait::ld.sync.aligned;"
+               : "+f"(g[0]), "+f"(g[1]), "+f"(g[2]), "+f"(g[3]), "+f"(g[4]), "+f"(g[5]), "+f"(g[6]), "+f"(g[7]),
+                 "+f"(g[8]), "+f"(g[9]), "+f"(g[10]), "+f"(g[11]), "+f"(g[12]), "+f"(g[13]), "+f"(g[14]),
+                 "+f"(g[15]), "+f"(g[16]), "+f"(g[17]), "+f"(g[18]), "+f"(g[19]), "+f"(g[20]), "+f"(g[21]),
+                 "+f"(g[22]), "+f"(g[23]), "+f"(g[24]), "+f"(g[25]), "+f"(g[26]), "+f"(g[27]), "+f"(g[28]),
+                 "+f"(g[29]), "+f"(g[30]), "+f"(g[31]), "+f"(t[0]), "+f"(t[1]), "+f"(t[2]), "+f"(t[3]),
+                 "+f"(t[4]), "+f"(t[5])
+               :
+               : "memory");
 }
 
 // 32 bits of a group's code stream starting at stream bit `bit` (shared memory).
@@ -91,64 +94,57 @@ __device__ __forceinline__ uint32_t code_run(const uint8_t* codes, uint32_t bit)
   return __funnelshift_r(w[0], w[1], bit & 31u);
 }
 
-// sum_i (u_i - off) * g_i for the first `cnt` codes of `run` (code i at bits [i*B, i*B + B)).
+// Code i of a run, as the float 1 + u / 2^B (u placed in the top mantissa bits).
+template <int B, int I>
+__device__ __forceinline__ float code_f(uint32_t run) {
+  constexpr int sh = 23 - B - I * B;
+  const uint32_t x = sh >= 0 ? (run << (sh >= 0 ? sh : 0)) : (run >> (sh < 0 ? -sh : 0));
+  return __uint_as_float((x & (((1u << B) - 1u) << (23 - B))) | 0x3F800000u);
+}
+
+// acc += sum_i (1 + u_i/2^B) g_i and gs += sum_i g_i over the first `cnt` codes (CNT compile-time bound).
 template <int B, int CNT>
-__device__ __forceinline__ float dot_codes(uint32_t run, const float* g, int cnt, float off_magic) {
-  float acc = 0.f;
+__device__ __forceinline__ void dot_run(uint32_t run, const float* g, int cnt, float& acc, float& gs) {
 #pragma unroll
   for (int i = 0; i < CNT; ++i) {
-    const uint32_t u = (run >> (i * B)) & ((1u << B) - 1u);
-    const float f = __uint_as_float(0x4B000000u | u) - off_magic;   // exactly u - 2^(B-1)
-    if (i < cnt) acc = fmaf(f, g[i], acc);
+    float f;
+    switch (i) {
+      case 0: f = code_f<B, 0>(run); break;
+      case 1: f = code_f<B, 1>(run); break;
+      case 2: f = code_f<B, 2>(run); break;
+      case 3: f = code_f<B, 3>(run); break;
+      case 4: f = code_f<B, 4>(run); break;
+      case 5: f = code_f<B, 5>(run); break;
+      case 6: f = code_f<B, 6>(run); break;
+      default: f = code_f<B, 7>(run); break;
+    }
+    if (i < cnt) {
+      acc = fmaf(f, g[i], acc);
+      gs += g[i];
+    }
   }
-  return acc;
 }
 
-__device__ __forceinline__ float dot_codes_any(uint32_t run, const float* g, int cnt, int bits, float off_magic) {
-  float acc = 0.f;
+// sum over one quantization group of (u - 2^(B-1)) * scale * G for one token:
+// nf full 8-code chunks from G[0..32), then `tail` codes from T.
+template <int B>
+__device__ __forceinline__ float group_dot(const uint8_t* codes, uint32_t bit0, int nf, int tail, const float* G,
+                                           const float* T) {
+  float acc = 0.f, gs = 0.f;
 #pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    const uint32_t u = (run >> (i * bits)) & ((1u << bits) - 1u);
-    const float f = __uint_as_float(0x4B000000u | u) - off_magic;
-    if (i < cnt) acc = fmaf(f, g[i], acc);
-  }
-  return acc;
+  for (int c = 0; c < 4; ++c)
+    if (c < nf) dot_run<B, 8>(code_run(codes, bit0 + (uint32_t)(c * 8 * B)), G + 8 * c, 8, acc, gs);
+  if (tail) dot_run<B, 6>(code_run(codes, bit0 + (uint32_t)(nf * 8 * B)), T, tail, acc, gs);
+  // sum (u - off) g = 2^B sum f g - (2^B + off) sum g
+  return (float)(1 << B) * acc - (float)((1 << B) + (1 << (B - 1))) * gs;
 }
 
-// Score of one (token, head): latent block `blk` (shared memory) of the token's page.
-__device__ __forceinline__ float score_one(const uint8_t* blk, int slot, const LatentDesc& ld,
-                                           const GroupDesc* __restrict__ grp, uint32_t tcol) {
-  float s = 0.f;
-  for (int gi = 0; gi < ld.n_groups; ++gi) {
-    const GroupDesc gd = grp[ld.group0 + gi];
-    const float scale = __half2float(reinterpret_cast<const __half*>(blk)[gi * kPage + slot]);
-    const uint8_t* codes = blk + gd.code_off;
-    const float off_magic = 8388608.f + (float)(1 << (gd.bits - 1));
-    const uint32_t bit0 = (uint32_t)(slot * gd.n) * gd.bits;
-    float acc = 0.f;
-    int c0 = 0;
-    for (; c0 + 8 <= gd.n; c0 += 8) {
-      float g[8];
-      tmem_ld8(tcol + gd.start + c0, g);
-      const uint32_t run = code_run(codes, bit0 + c0 * gd.bits);
-      if (gd.bits == 4)
-        acc += dot_codes<4, 8>(run, g, 8, off_magic);
-      else if (gd.bits == 3)
-        acc += dot_codes<3, 8>(run, g, 8, off_magic);
-      else
-        acc += dot_codes_any(run, g, 8, gd.bits, off_magic);
-    }
-    for (; c0 < gd.n; c0 += 2) {
-      float g[2];
-      tmem_ld2(tcol + gd.start + c0, g);
-      const int cnt = min(2, gd.n - c0);
-      const uint32_t run = code_run(codes, bit0 + c0 * gd.bits);
-      acc += dot_codes_any(run, g, cnt, gd.bits, off_magic);
-    }
-    s = fmaf(scale, acc, s);
-  }
-  return s;
-}
+// Per query head: its key latent's groups (start, n, bits, code offset), the
+// latent block's offset inside the item's key range, and its first G column.
+struct HeadPlan {
+  int ng, blk_rel, hcol, pad;
+  int4 grp[4];
+};
 
 __global__ void __launch_bounds__(kScoreThreads, 1) k_scores_tc(ScoreArgs a) {
   extern __shared__ uint8_t smem_raw[];
@@ -156,7 +152,9 @@ __global__ void __launch_bounds__(kScoreThreads, 1) k_scores_tc(ScoreArgs a) {
   __shared__ __align__(8) uint64_t acc_full[2], acc_free[2], fin;
   __shared__ uint32_t tmem_base;
   __shared__ volatile int abort_flag;
-  __shared__ float red_max[8][8], red_sum[8][8];
+  __shared__ ScoreItem items_s[64];
+  __shared__ HeadPlan hp_s[64];
+  __shared__ float sc_s[4][512];
   uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   uint8_t* E_s = smem;                                   // 2 x 32 KB
   uint8_t* W_s = E_s + 2 * kETileBytes;                  // WS x w_stage
@@ -170,17 +168,39 @@ __global__ void __launch_bounds__(kScoreThreads, 1) k_scores_tc(ScoreArgs a) {
       tc::mbar_init(&w_full[s], 1);
       tc::mbar_init(&w_empty[s], 1);
       tc::mbar_init(&k_full[s], 1);
-      tc::mbar_init(&k_empty[s], 8);
+      tc::mbar_init(&k_empty[s], kEpiWarps);
     }
     for (int s = 0; s < 2; ++s) {
       tc::mbar_init(&e_full[s], 1);
       tc::mbar_init(&e_empty[s], 1);
       tc::mbar_init(&acc_full[s], 1);
-      tc::mbar_init(&acc_free[s], 8);
+      tc::mbar_init(&acc_free[s], kEpiWarps);
     }
     tc::mbar_init(&fin, 1);
     abort_flag = 0;
     tc::fence_mbar_init();
+  }
+  // item table and per-head plans in shared memory
+  for (int it = threadIdx.x; it < a.n_items; it += blockDim.x) items_s[it] = a.items[it];
+  for (int h = threadIdx.x; h < a.H; h += blockDim.x) {
+    HeadPlan hp{};
+    const LatentDesc ld = a.lat[h / a.gq];
+    int item_key_off = 0, hcol = 0;
+    for (int it = 0; it < a.n_items; ++it) {
+      const ScoreItem& x = a.items[it];
+      if (h >= x.h0 && h < x.h0 + x.nh) {
+        item_key_off = x.key_off;
+        hcol = x.hcol[h - x.h0];
+      }
+    }
+    hp.ng = min(ld.n_groups, 4);
+    hp.blk_rel = ld.block_off - item_key_off;
+    hp.hcol = hcol;
+    for (int g = 0; g < hp.ng; ++g) {
+      const GroupDesc gd = a.grp[ld.group0 + g];
+      hp.grp[g] = make_int4(gd.start, gd.n, gd.bits, gd.code_off);
+    }
+    hp_s[h] = hp;
   }
   if (warp == 1) tc::tmem_alloc(&tmem_base, 512);
   tc::tc_fence_before();
@@ -285,9 +305,11 @@ __global__ void __launch_bounds__(kScoreThreads, 1) k_scores_tc(ScoreArgs a) {
     }
   } else {
     // ------------------------------------------------------------ epilogue
-    const int e = warp - 2;              // 0..7
-    const int q = warp & 3;              // TMEM lane quarter
-    const int k = e >> 2;                // tile of the super-tile
+    // 16 warps: TMEM lane quarter q = warp % 4, tile k, head parity hp
+    const int e = warp - 2;              // 0..15
+    const int q = warp & 3;
+    const int k = (e >> 2) & 1;
+    const int hpar = e >> 3;
     const int tau = k * 128 + q * 32 + lane;
     const int pg = tau >> 4, slot = tau & 15;
     int i = 0;
@@ -301,22 +323,46 @@ __global__ void __launch_bounds__(kScoreThreads, 1) k_scores_tc(ScoreArgs a) {
       const int t = t0 + tau;
       const bool valid = t < len;
       for (int it = 0; it < a.n_items; ++it, ++i) {
-        const ScoreItem item = a.items[it];
+        const ScoreItem& item = items_s[it];
+        const int nh = item.nh;
         const int ks = i % a.KS;
         const bool ok1 = tc::mbar_wait_ab(&k_full[ks], ((uint32_t)(i / a.KS)) & 1u, a.status, &abort_flag);
-        const bool ok2 = ok1 && tc::mbar_wait_ab(&acc_full[i & 1], ((uint32_t)(i >> 1)) & 1u, a.status, &abort_flag);
+        const bool ok = ok1 && tc::mbar_wait_ab(&acc_full[i & 1], ((uint32_t)(i >> 1)) & 1u, a.status, &abort_flag);
         tc::tc_fence_after();
-        float s[8];
         const uint8_t* page = K_s + (size_t)ks * a.k_stage + (size_t)pg * item.key_bytes;
         const uint32_t tcol = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)((i & 1) * 256 + k * 128);
+        for (int hh = hpar; hh < nh; hh += 2) {
+          const HeadPlan& hp = hp_s[item.h0 + hh];
+          const uint8_t* blk = page + hp.blk_rel;
+          float s = 0.f;
+          if (ok) {
+            for (int gi = 0; gi < hp.ng; ++gi) {
+              const int4 gd = hp.grp[gi];     // start, n, bits, code_off
+              const int nf = gd.y >> 3, tail = gd.y & 7;
+              float G[32], T[6];
+              const uint32_t c0 = tcol + (uint32_t)(hp.hcol + gd.x);
 #pragma unroll
-        for (int hh = 0; hh < 8; ++hh) {
-          s[hh] = 0.f;
-          if (hh < item.nh && ok1 && ok2) {
-            const int g = (item.h0 + hh) / a.gq;
-            const LatentDesc ld = a.lat[g];
-            s[hh] = score_one(page + (ld.block_off - item.key_off), slot, ld, a.grp, tcol + item.hcol[hh]);
+              for (int c = 0; c < 4; ++c)
+                if (c < nf) tmem_ld8_nw(c0 + 8 * c, G + 8 * c);
+              const uint32_t ct = c0 + (uint32_t)(8 * nf);
+              if (tail > 0) tmem_ld2_nw(ct, T);
+              if (tail > 2) tmem_ld2_nw(ct + 2, T + 2);
+              if (tail > 4) tmem_ld2_nw(ct + 4, T + 4);
+              tmem_wait(G, T);
+              const float scale = __half2float(reinterpret_cast<const __half*>(blk)[gi * kPage + slot]);
+              const uint8_t* codes = blk + gd.w;
+              const uint32_t bit0 = (uint32_t)(slot * gd.y * gd.z);
+              float d;
+              if (gd.z == 3)
+                d = group_dot<3>(codes, bit0, nf, tail, G, T);
+              else if (gd.z == 4)
+                d = group_dot<4>(codes, bit0, nf, tail, G, T);
+              else
+                d = 0.f;     // layers with other code widths do not take this kernel
+              s = fmaf(scale, d, s);
+            }
           }
+          sc_s[hh >> 1][e * 32 + lane] = s;
         }
         tc::tc_fence_before();
         __syncwarp();
@@ -324,54 +370,30 @@ __global__ void __launch_bounds__(kScoreThreads, 1) k_scores_tc(ScoreArgs a) {
           tc::mbar_arrive(&acc_free[i & 1]);
           tc::mbar_arrive(&k_empty[ks]);
         }
-        // softmax statistics of this super-tile, per head
         const size_t hb = (size_t)b * a.H + item.h0;
         if (a.S_dbg) {
-          for (int hh = 0; hh < item.nh; ++hh)
-            if (valid) a.S_dbg[(hb + hh) * a.P_ld + t] = s[hh];
+          for (int hh = hpar; hh < nh; hh += 2)
+            if (valid) a.S_dbg[(hb + hh) * a.P_ld + t] = sc_s[hh >> 1][e * 32 + lane];
           continue;
         }
-        float mloc[8];
-#pragma unroll
-        for (int hh = 0; hh < 8; ++hh) {
-          float m = valid ? s[hh] : -FLT_MAX;
+        // softmax statistics per 32-token group (this warp's tokens), per head:
+        // m = max s, P = exp2(s - m) rounded to fp16, l = sum of the fp16 P
+        const int grp = (t0 >> 5) + k * 4 + q;
+        for (int hh = hpar; hh < nh; hh += 2) {
+          const float sv = sc_s[hh >> 1][e * 32 + lane];
+          float m = valid ? sv : -FLT_MAX;
           for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-          mloc[hh] = m;
-        }
-        if (lane == 0)
-#pragma unroll
-          for (int hh = 0; hh < 8; ++hh) red_max[e][hh] = mloc[hh];
-        asm volatile("bar.sync 1, 256;" ::: "memory");
-        float lsum[8];
-#pragma unroll
-        for (int hh = 0; hh < 8; ++hh) {
-          float m = red_max[0][hh];
-#pragma unroll
-          for (int w = 1; w < 8; ++w) m = fmaxf(m, red_max[w][hh]);
-          mloc[hh] = m;
           float p = 0.f;
-          if (valid && hh < item.nh) {
-            const __half pb = __float2half_rn(exp2f(s[hh] - m));
+          if (valid) {
+            const __half pb = __float2half_rn(exp2f(sv - m));
             a.P[(hb + hh) * a.P_ld + t] = pb;
             p = __half2float(pb);
           }
           for (int o = 16; o > 0; o >>= 1) p += __shfl_xor_sync(0xffffffffu, p, o);
-          lsum[hh] = p;
-        }
-        if (lane == 0)
-#pragma unroll
-          for (int hh = 0; hh < 8; ++hh) red_sum[e][hh] = lsum[hh];
-        asm volatile("bar.sync 2, 256;" ::: "memory");
-        if (e == 0 && lane < item.nh) {
-          float l = 0.f;
-#pragma unroll
-          for (int w = 0; w < 8; ++w) l += red_sum[w][lane];
-          float m = mloc[0];
-#pragma unroll
-          for (int hh = 1; hh < 8; ++hh)
-            if (hh == lane) m = mloc[hh];
-          a.m_st[(hb + lane) * a.n_st + st] = m;
-          a.l_st[(hb + lane) * a.n_st + st] = l;
+          if (lane == 0) {
+            a.m_st[(hb + hh) * a.n_g + grp] = m;
+            a.l_st[(hb + hh) * a.n_g + grp] = p;
+          }
         }
       }
     }
@@ -384,10 +406,13 @@ __global__ void __launch_bounds__(kScoreThreads, 1) k_scores_tc(ScoreArgs a) {
 
 // W'' item blocks for every sequence: rows of W'' (grouped by item, zero
 // padded to the item's N), 128 columns, K-major with 128-byte swizzle, fp16.
-__global__ void k_qprep_tc(LayerView v, const __nv_bfloat16* __restrict__ q, const int32_t* __restrict__ seq_lens,
-                           const int32_t* __restrict__ q_pos, const float* __restrict__ Bk,
-                           const int* __restrict__ key_off, const ScoreItem* __restrict__ items, long long w_stride,
-                           uint8_t* __restrict__ W) {
+// One block per (sequence, item); a thread writes 8 columns of one row.
+__global__ void __launch_bounds__(512) k_qprep_tc(LayerView v, const __nv_bfloat16* __restrict__ q,
+                                                  const int32_t* __restrict__ seq_lens,
+                                                  const int32_t* __restrict__ q_pos, const float* __restrict__ Bk,
+                                                  const int* __restrict__ key_off,
+                                                  const ScoreItem* __restrict__ items, long long w_stride,
+                                                  uint8_t* __restrict__ W) {
   __shared__ float qs[8][128];
   const int b = blockIdx.x, it = blockIdx.y;
   const ScoreItem item = items[it];
@@ -396,33 +421,47 @@ __global__ void k_qprep_tc(LayerView v, const __nv_bfloat16* __restrict__ q, con
     const int hh = idx / 64, p = idx % 64;
     const int h = item.h0 + hh;
     const __nv_bfloat16* qh = q + ((size_t)b * v.H + h) * 128;
-    float a0 = __bfloat162float(qh[p]), b0 = __bfloat162float(qh[p + 64]);
-    const double freq = exp2(-(2.0 * p / 128.0) * (double)v.rope_log2_theta);
-    double sn, cs;
-    sincos((double)pos * freq, &sn, &cs);
-    qs[hh][p] = (float)(a0 * cs - b0 * sn) * v.scale_log2;
-    qs[hh][p + 64] = (float)(b0 * cs + a0 * sn) * v.scale_log2;
+    const float a0 = __bfloat162float(qh[p]), b0 = __bfloat162float(qh[p + 64]);
+    // angle pos * theta_p reduced modulo 2 pi in double, then a float sincos
+    const double ang = (double)pos * exp2(-(2.0 * p / 128.0) * (double)v.rope_log2_theta);
+    const double two_pi = 6.283185307179586476925286766559;
+    const float red = (float)(ang - two_pi * rint(ang / two_pi));
+    float sn, cs;
+    sincosf(red, &sn, &cs);
+    qs[hh][p] = (a0 * cs - b0 * sn) * v.scale_log2;
+    qs[hh][p + 64] = (b0 * cs + a0 * sn) * v.scale_log2;
   }
   __syncthreads();
   uint8_t* blk = W + (size_t)b * w_stride + item.w_off;
   const uint32_t atom = (uint32_t)item.npad * 128u;
-  for (int idx = threadIdx.x; idx < item.npad * 64; idx += blockDim.x) {
-    const int row = idx / 64, p = idx % 64;
-    float re = 0.f, im = 0.f;
+  for (int idx = threadIdx.x; idx < item.npad * 8; idx += blockDim.x) {
+    const int row = idx >> 3, c = idx & 7;       // 8-column chunk c of the 64 (cos | sin) pairs
     int hh = -1;
     for (int x = 0; x < item.nh; ++x)
       if (row >= item.hcol[x] && row < item.hcol[x] + item.hr[x]) hh = x;
+    uint32_t re[4] = {0u, 0u, 0u, 0u}, im[4] = {0u, 0u, 0u, 0u};
     if (hh >= 0) {
       const int h = item.h0 + hh, g = h / v.group_q, j = row - item.hcol[hh];
-      const float* B = Bk + ((size_t)key_off[g] + j) * 128;
-      const float x = B[p], y = B[p + 64];
-      const float aq = qs[hh][p], bq = qs[hh][p + 64];
-      re = aq * x + bq * y;
-      im = bq * x - aq * y;
+      const float* B = Bk + ((size_t)key_off[g] + j) * 128 + c * 8;
+      const float4 x0 = *reinterpret_cast<const float4*>(B), x1 = *reinterpret_cast<const float4*>(B + 4);
+      const float4 y0 = *reinterpret_cast<const float4*>(B + 64), y1 = *reinterpret_cast<const float4*>(B + 68);
+      const float xs[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
+      const float ys[8] = {y0.x, y0.y, y0.z, y0.w, y1.x, y1.y, y1.z, y1.w};
+#pragma unroll
+      for (int i = 0; i < 8; i += 2) {
+        const int p = c * 8 + i;
+        const float r0 = qs[hh][p] * xs[i] + qs[hh][p + 64] * ys[i];
+        const float r1 = qs[hh][p + 1] * xs[i + 1] + qs[hh][p + 65] * ys[i + 1];
+        const float i0 = qs[hh][p + 64] * xs[i] - qs[hh][p] * ys[i];
+        const float i1 = qs[hh][p + 65] * xs[i + 1] - qs[hh][p + 1] * ys[i + 1];
+        const __half2 rh = __floats2half2_rn(r0, r1), ih = __floats2half2_rn(i0, i1);
+        re[i / 2] = *reinterpret_cast<const uint32_t*>(&rh);
+        im[i / 2] = *reinterpret_cast<const uint32_t*>(&ih);
+      }
     }
-    const uint32_t o0 = tc::sw128((uint32_t)row, (uint32_t)(p >> 3)) + (uint32_t)(p & 7) * 2u;
-    *reinterpret_cast<__half*>(blk + o0) = __float2half_rn(re);
-    *reinterpret_cast<__half*>(blk + atom + o0) = __float2half_rn(im);
+    const uint32_t o = tc::sw128((uint32_t)row, (uint32_t)c);
+    *reinterpret_cast<uint4*>(blk + o) = make_uint4(re[0], re[1], re[2], re[3]);
+    *reinterpret_cast<uint4*>(blk + atom + o) = make_uint4(im[0], im[1], im[2], im[3]);
   }
 }
 
@@ -486,7 +525,8 @@ bool plan_scores_tc(starkv_layer* L) {
   L->k_stage = (kSuper / kPage) * max_key + 16;
   L->k_stage = (L->k_stage + 1023) / 1024 * 1024;
   L->w_stage = (max_w + 1023) / 1024 * 1024;
-  const size_t budget = 222 * 1024 - 2 * kETileBytes;
+  // dynamic shared memory next to ~21 KB of static tables and barriers
+  const size_t budget = 204 * 1024 - 2 * kETileBytes;
   L->WS = 3;
   L->KS = 2;
   while (L->WS > 2 && (size_t)L->WS * L->w_stage + (size_t)L->KS * L->k_stage > budget) --L->WS;
@@ -508,7 +548,7 @@ size_t scores_tc_ws_bytes(const starkv_layer* L, int batch, int max_len) {
   const size_t P_ld = (size_t)n_st * kSuper;
   auto r = [](size_t x) { return (x + 255) / 256 * 256; };
   return r((size_t)batch * L->w_stride) + r(2 * (size_t)batch * L->view.H * P_ld) +
-         2 * r(sizeof(float) * (size_t)batch * L->view.H * n_st);
+         2 * r(sizeof(float) * (size_t)batch * L->view.H * (P_ld / 32));
 }
 
 cudaError_t launch_scores_tc(const starkv_layer* L, const uint8_t* pool, long long n_pages, const int32_t* pt,
@@ -525,10 +565,11 @@ cudaError_t launch_scores_tc(const starkv_layer* L, const uint8_t* pool, long lo
   out->n_st = n_st;
   out->P = (__half*)w;
   w += r(2 * (size_t)batch * v.H * n_st * kSuper);
+  out->n_g = n_st * (kSuper / 32);
   out->m_st = (float*)w;
-  w += r(sizeof(float) * (size_t)batch * v.H * n_st);
+  w += r(sizeof(float) * (size_t)batch * v.H * out->n_g);
   out->l_st = (float*)w;
-  k_qprep_tc<<<dim3(batch, (unsigned)L->items.size()), 128, 0, s>>>(
+  k_qprep_tc<<<dim3(batch, (unsigned)L->items.size()), 512, 0, s>>>(
       v, (const __nv_bfloat16*)q, seq_lens, q_pos, L->Bk, L->d_key_off, L->d_items, L->w_stride, W);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
@@ -553,6 +594,7 @@ cudaError_t launch_scores_tc(const starkv_layer* L, const uint8_t* pool, long lo
   a.P_ld = out->P_ld;
   a.m_st = out->m_st;
   a.l_st = out->l_st;
+  a.n_g = out->n_g;
   a.S_dbg = S_dbg;
   a.H = v.H;
   a.w_stage = L->w_stage;

@@ -10,14 +10,15 @@
 // in), the stacked probabilities are B (N = heads, K-major), and Y^T for every
 // 128-channel block stays in TMEM for a whole run of super-tiles.
 //
-// P comes from the score kernel as exp2(s - m_st) per 256-token super-tile;
-// a CTA rescales it by exp2(m_st - M) with M the maximum over the CTA's run,
+// P comes from the score kernel as exp2(s - m_g) per 32-token group; a CTA
+// rescales it by exp2(m_g - M) with M the maximum over the CTA's run,
 // so no accumulator ever needs rescaling.  The CTA writes one partial
 // (M, l, Y) per run of one sequence; a combine kernel merges the runs.
 //   warp 0      bulk copies of the value latent blocks of each tile's pages
 //   warp 1      tcgen05.mma issue, TMEM allocation
-//   warps 2-9   P staging (scaled, fp16), dequantization of the 4/3-bit codes
-//               into the A tiles, and the TMEM epilogue of each run
+//   warps 2-17  P staging (scaled, fp16), dequantization of the 4/3-bit codes
+//               into the A tiles (one thread per token and 32-channel group),
+//               and the TMEM epilogue of each run
 #include <float.h>
 
 #include "tc_common.cuh"
@@ -26,7 +27,8 @@ namespace starkv {
 
 namespace {
 
-constexpr int kValThreads = 320;
+constexpr int kValWarps = 16;
+constexpr int kValThreads = 64 + 32 * kValWarps;   // producer, MMA, 16 staging/dequant/epilogue warps
 constexpr int kVSuper = 256;   // tokens per super-tile (matches the score kernel)
 
 struct ValArgs {
@@ -40,8 +42,9 @@ struct ValArgs {
   int rv, H;
   const __half* P;              // [B][H][P_ld]
   long long P_ld;
-  const float* m_st;            // [B][H][n_st]
+  const float* m_st;            // [B][H][n_g]: maximum of each 32-token group
   int n_st;
+  int n_g;
   long long U;                  // batch * n_st
   int slots;                    // partial slots per CTA
   float* Y;                     // [G][slots][H][rv]
@@ -53,31 +56,35 @@ struct ValArgs {
 
 __device__ __forceinline__ long long vunit_lo(int c, int G, long long U) { return (long long)c * U / G; }
 
-// fp16 pair (c0, c1) of (u - off) * s for two codes already placed at bits
-// [0, b) and [16, 16 + b) of `w`: exact integers via the 1024 + u bit
-// pattern, one exact subtraction, one correctly rounded multiply.
-__device__ __forceinline__ uint32_t deq_pair(uint32_t w, __half2 sub, __half2 s2) {
-  const uint32_t x = w | 0x64006400u;
+// Dequantization of 8 codes of one group into four fp16 pairs, in the chunk
+// order (c0,c2) (c1,c3) (c4,c6) (c5,c7): each 16-bit lane holds 1024 + u (an
+// exact fp16 integer), one exact subtraction of 1024 + 2^(B-1) and one
+// correctly rounded multiply by the fp16 scale give (u - 2^(B-1)) * scale.
+// The A tile therefore stores, inside every 8-channel chunk, channels
+// 0 2 1 3 4 6 5 7; the combine kernel puts them back in order.
+__device__ __forceinline__ uint32_t deq2(uint32_t lanes, __half2 sub, __half2 s2) {
+  const uint32_t x = lanes | 0x64006400u;
   __half2 h = *reinterpret_cast<const __half2*>(&x);
   h = __hmul2(__hsub2(h, sub), s2);
   return *reinterpret_cast<uint32_t*>(&h);
 }
-
-// 8 channels (codes c0..c7 of `bits` bits starting at bit 0 of `run`) -> 4 words of fp16 pairs.
-__device__ __forceinline__ void deq8(uint32_t run, int bits, __half2 sub, __half2 s2, uint32_t* o) {
-  if (bits == 4) {
-#pragma unroll
-    for (int k = 0; k < 4; ++k) {
-      const uint32_t b = (run >> (8 * k)) & 0xFFu;
-      o[k] = deq_pair((b & 0xFu) | ((b >> 4) << 16), sub, s2);
-    }
-  } else {
-#pragma unroll
-    for (int k = 0; k < 4; ++k) {
-      const uint32_t b = (run >> (6 * k)) & 0x3Fu;
-      o[k] = deq_pair((b & 0x7u) | ((b >> 3) << 16), sub, s2);
-    }
-  }
+__device__ __forceinline__ uint4 deq8_b4(uint32_t run, __half2 sub, __half2 s2) {
+  const uint32_t x01 = __byte_perm(run, 0u, 0x4140u);   // bytes c1c0 | c3c2 into the two 16-bit lanes
+  const uint32_t x23 = __byte_perm(run, 0u, 0x4342u);
+  uint4 o;
+  o.x = deq2(x01 & 0x000F000Fu, sub, s2);           // (c0, c2)
+  o.y = deq2((x01 >> 4) & 0x000F000Fu, sub, s2);    // (c1, c3)
+  o.z = deq2(x23 & 0x000F000Fu, sub, s2);           // (c4, c6)
+  o.w = deq2((x23 >> 4) & 0x000F000Fu, sub, s2);    // (c5, c7)
+  return o;
+}
+__device__ __forceinline__ uint4 deq8_b3(uint32_t run, __half2 sub, __half2 s2) {
+  uint4 o;
+  o.x = deq2((run & 0x7u) | ((run << 10) & 0x70000u), sub, s2);           // c0 bits 0-2, c2 bits 6-8
+  o.y = deq2(((run >> 3) & 0x7u) | ((run << 7) & 0x70000u), sub, s2);     // c1 bits 3-5, c3 bits 9-11
+  o.z = deq2(((run >> 12) & 0x7u) | ((run >> 2) & 0x70000u), sub, s2);    // c4 bits 12-14, c6 bits 18-20
+  o.w = deq2(((run >> 15) & 0x7u) | ((run >> 5) & 0x70000u), sub, s2);    // c5 bits 15-17, c7 bits 21-23
+  return o;
 }
 
 __global__ void __launch_bounds__(kValThreads, 1) k_values_tc(ValArgs a) {
@@ -86,7 +93,8 @@ __global__ void __launch_bounds__(kValThreads, 1) k_values_tc(ValArgs a) {
   __shared__ __align__(8) uint64_t seg_done, acc_free, fin;
   __shared__ uint32_t tmem_base;
   __shared__ volatile int abort_flag;
-  __shared__ float M_s[64], f_s[2][64], l_s[64];
+  __shared__ float M_s[64], l_s[64];
+  __shared__ int2 vg_s[128];     // per 32-channel value group: code width, code block offset
   uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   const int raw_stage = (8 * a.vblk_bytes + 1023) / 1024 * 1024;
   uint8_t* R_s = smem;                              // 2 x raw tile (8 value blocks)
@@ -101,18 +109,19 @@ __global__ void __launch_bounds__(kValThreads, 1) k_values_tc(ValArgs a) {
   if (threadIdx.x == 0) {
     for (int s = 0; s < 2; ++s) {
       tc::mbar_init(&raw_full[s], 1);
-      tc::mbar_init(&raw_empty[s], 8);
-      tc::mbar_init(&a_full[s], 8);
+      tc::mbar_init(&raw_empty[s], kValWarps);
+      tc::mbar_init(&a_full[s], kValWarps);
       tc::mbar_init(&a_empty[s], 1);
-      tc::mbar_init(&p_full[s], 8);
+      tc::mbar_init(&p_full[s], kValWarps);
       tc::mbar_init(&p_empty[s], 1);
     }
     tc::mbar_init(&seg_done, 1);
-    tc::mbar_init(&acc_free, 8);
+    tc::mbar_init(&acc_free, kValWarps);
     tc::mbar_init(&fin, 1);
     abort_flag = 0;
     tc::fence_mbar_init();
   }
+  for (int g = threadIdx.x; g < a.rv / 32; g += blockDim.x) vg_s[g] = make_int2(a.vgrp[g].bits, a.vgrp[g].code_off);
   if (warp == 1) tc::tmem_alloc(&tmem_base, a.tmem_cols);
   tc::tc_fence_before();
   __syncthreads();
@@ -203,18 +212,18 @@ __global__ void __launch_bounds__(kValThreads, 1) k_values_tc(ValArgs a) {
     }
   } else {
     // ------------------------------------------------ P staging, dequantization, epilogue
-    const int e = warp - 2;          // 0..7
-    const int tid = threadIdx.x - 64;  // 0..255
-    int nt = 0, na = 0, seg = 0, slot = -1, nu = 0;
+    const int e = warp - 2;            // 0..15
+    const int tid = threadIdx.x - 64;  // 0..511
+    int nt = 0, na = 0, seg = 0, slot = -1;
     int cur_b = -1;
     const long long ub = u0 / a.n_st;
-    auto finish_run = [&](int b) {
-      // epilogue of the run of sequence b: Y^T from TMEM, M and l
+    auto finish_run = [&]() {
+      // epilogue of a run: Y^T from TMEM (lanes = value channels), M and l
       const bool ok = tc::mbar_wait_ab(&seg_done, ((uint32_t)seg) & 1u, a.status, &abort_flag);
       tc::tc_fence_after();
-      const int q = warp & 3, half = e >> 2;
+      const int q = warp & 3;
       const size_t base = ((size_t)c * a.slots + slot) * a.H;
-      for (int cb = half; cb < nblk; cb += 2) {
+      for (int cb = e >> 2; cb < nblk; cb += 4) {
         for (int h0 = 0; h0 < a.H; h0 += 16) {
           float v[16];
           if (ok) {
@@ -223,7 +232,7 @@ __global__ void __launch_bounds__(kValThreads, 1) k_values_tc(ValArgs a) {
 #pragma unroll
             for (int i = 0; i < 16; ++i) v[i] = 0.f;
           }
-          const int ch = cb * 128 + q * 32 + lane;
+          const int ch = cb * 128 + q * 32 + lane;     // A-tile position (channel order permuted per 8)
 #pragma unroll
           for (int i = 0; i < 16; ++i) a.Y[(base + h0 + i) * a.rv + ch] = v[i];
         }
@@ -235,7 +244,6 @@ __global__ void __launch_bounds__(kValThreads, 1) k_values_tc(ValArgs a) {
         a.mseg[base + tid] = M_s[tid];
         a.lseg[base + tid] = l_s[tid];
       }
-      (void)b;
       ++seg;
     };
     // every slot of this CTA starts empty (a run with no valid token leaves l = 0)
@@ -244,32 +252,35 @@ __global__ void __launch_bounds__(kValThreads, 1) k_values_tc(ValArgs a) {
         a.mseg[((size_t)c * a.slots + sl) * a.H + tid] = -FLT_MAX;
         a.lseg[((size_t)c * a.slots + sl) * a.H + tid] = 0.f;
       }
+    // fixed per-thread roles inside a 128-token tile
+    const int tok = tid & 127;            // token of the tile
+    const int cq = tid >> 7;              // 32-channel group inside a 128-channel block
+    const uint32_t a_off = (uint32_t)(tok >> 3) * 2048u + (uint32_t)(cq >> 1) * 1024u + (uint32_t)(tok & 7) * 128u;
+    const uint32_t x7 = (uint32_t)(tok & 7);
+    const int ph = tid >> 4, pch = tid & 15;   // P staging: head, 8-token chunk
     for (long long u = u0; u < u1; ++u) {
       const int b = (int)(u / a.n_st), st = (int)(u % a.n_st);
       const int len = min(a.seq_lens[b], a.max_pages * kPage);
       if (st * kVSuper >= len) continue;
       if (b != cur_b) {
-        if (cur_b >= 0) finish_run(cur_b);
+        if (cur_b >= 0) finish_run();
         cur_b = b;
         slot = (int)(b - ub);
         // run maximum over the CTA's units of this sequence
-        asm volatile("bar.sync 1, 256;" ::: "memory");
+        asm volatile("bar.sync 1, 512;" ::: "memory");
         if (tid < a.H) {
           float m = -FLT_MAX;
           for (long long uu = u; uu < u1 && uu / a.n_st == b; ++uu) {
             const int s2 = (int)(uu % a.n_st);
-            if (s2 * kVSuper < len) m = fmaxf(m, a.m_st[((size_t)b * a.H + tid) * a.n_st + s2]);
+            if (s2 * kVSuper < len)
+              for (int g = 0; g < kVSuper / 32; ++g)
+                m = fmaxf(m, a.m_st[((size_t)b * a.H + tid) * a.n_g + s2 * (kVSuper / 32) + g]);
           }
           M_s[tid] = m;
           l_s[tid] = 0.f;
         }
-        asm volatile("bar.sync 1, 256;" ::: "memory");
+        asm volatile("bar.sync 1, 512;" ::: "memory");
       }
-      // per-unit scale exp2(m_st - M), double-buffered: no warp is ever a unit ahead of another
-      float* fu = f_s[nu & 1];
-      ++nu;
-      if (tid < a.H) fu[tid] = exp2f(a.m_st[((size_t)b * a.H + tid) * a.n_st + st] - M_s[tid]);
-      asm volatile("bar.sync 1, 256;" ::: "memory");
       for (int tile = 0; tile < 2; ++tile) {
         const int t0 = st * kVSuper + tile * 128;
         if (t0 >= len) break;
@@ -277,23 +288,23 @@ __global__ void __launch_bounds__(kValThreads, 1) k_values_tc(ValArgs a) {
         const int ps = nt & 1;
         tc::mbar_wait_ab(&p_empty[ps], (((uint32_t)(nt >> 1)) & 1u) ^ 1u, a.status, &abort_flag);
         uint8_t* pt_s = P_s + (size_t)ps * p_stage;
-        for (int idx = tid; idx < a.H * 16; idx += 256) {
-          const int h = idx >> 4, ch = idx & 15;        // 16 chunks of 8 tokens
-          const int t = t0 + ch * 8;
-          const float f = fu[h];
+        if (ph < a.H) {
+          const int tp = t0 + pch * 8;
+          const float mg = a.m_st[((size_t)b * a.H + ph) * a.n_g + (tp >> 5)];
+          const float f = exp2f(mg - M_s[ph]);
           uint4 raw = make_uint4(0, 0, 0, 0);
-          if (t < len) raw = *reinterpret_cast<const uint4*>(a.P + ((size_t)b * a.H + h) * a.P_ld + t);
+          if (tp < len) raw = *reinterpret_cast<const uint4*>(a.P + ((size_t)b * a.H + ph) * a.P_ld + tp);
           __half* hv = reinterpret_cast<__half*>(&raw);
           float lsum = 0.f;
 #pragma unroll
           for (int i = 0; i < 8; ++i) {
-            float p = (t + i < len) ? __half2float(hv[i]) * f : 0.f;
+            const float p = (tp + i < len) ? __half2float(hv[i]) * f : 0.f;
             hv[i] = __float2half_rn(p);
             lsum += __half2float(hv[i]);
           }
-          atomicAdd(&l_s[h], lsum);
-          const int atom = ch >> 3;
-          *reinterpret_cast<uint4*>(pt_s + atom * (a.H * 128) + tc::sw128((uint32_t)h, (uint32_t)(ch & 7))) = raw;
+          atomicAdd(&l_s[ph], lsum);
+          *reinterpret_cast<uint4*>(pt_s + (pch >> 3) * (a.H * 128) + tc::sw128((uint32_t)ph, (uint32_t)(pch & 7))) =
+              raw;
         }
         tc::fence_proxy_async();
         __syncwarp();
@@ -301,52 +312,48 @@ __global__ void __launch_bounds__(kValThreads, 1) k_values_tc(ValArgs a) {
         // ---- value latent codes -> A tiles, one 128-channel block at a time
         const int r = nt & 1;
         tc::mbar_wait_ab(&raw_full[r], ((uint32_t)(nt >> 1)) & 1u, a.status, &abort_flag);
-        const uint8_t* raw_s = R_s + (size_t)r * raw_stage;
-        const int tok = tid & 127, cg = tid >> 7;       // token of the tile, 64-channel half of the block
+        const uint8_t* blk = R_s + (size_t)r * raw_stage + (size_t)(tok >> 4) * a.vblk_bytes;
+        const int slot16 = tok & 15;
         const bool tvalid = t0 + tok < len;
-        const uint8_t* blk = raw_s + (size_t)(tok >> 4) * a.vblk_bytes;
-        const int slot = tok & 15;
         for (int cb = 0; cb < nblk; ++cb, ++na) {
           const int as = na & 1;
-          tc::mbar_wait_ab(&a_empty[as], (((uint32_t)(na >> 1)) & 1u) ^ 1u, a.status, &abort_flag);
-          uint8_t* at = A_s + (size_t)as * 32768;
-#pragma unroll
-          for (int gg = 0; gg < 2; ++gg) {
-            const int gi = cb * 4 + cg * 2 + gg;        // 32-channel group of the value latent
-            const GroupDesc gd = a.vgrp[gi];
-            uint32_t w[4] = {0u, 0u, 0u, 0u};
-            float sc = 0.f;
-            if (tvalid) {
-              sc = __half2float(reinterpret_cast<const __half*>(blk)[gi * kPage + slot]);
-              const uint32_t* cw = reinterpret_cast<const uint32_t*>(blk + gd.code_off) + slot * gd.bits;
-              if (gd.bits == 4) {
-                const uint4 v4 = *reinterpret_cast<const uint4*>(cw);
-                w[0] = v4.x; w[1] = v4.y; w[2] = v4.z; w[3] = v4.w;
-              } else {
-                w[0] = cw[0]; w[1] = cw[1]; w[2] = cw[2];
-              }
-            }
-            const __half2 s2 = __floats2half2_rn(sc, sc);
-            const float offm = 1024.f + (float)(1 << (gd.bits - 1));
-            const __half2 sub = __floats2half2_rn(offm, offm);
-#pragma unroll
-            for (int q8 = 0; q8 < 4; ++q8) {       // 8-channel chunk of the group
-              uint32_t run;
-              if (gd.bits == 4) {
-                run = w[q8];
-              } else {
-                const int bit = q8 * 24;
-                run = __funnelshift_r(w[bit >> 5], w[(bit >> 5) + 1 < 4 ? (bit >> 5) + 1 : 3], bit & 31);
-              }
-              uint32_t o[4];
-              deq8(run, gd.bits, sub, s2, o);
-              if (!tvalid) o[0] = o[1] = o[2] = o[3] = 0u;
-              const int chl = cg * 64 + gg * 32 + q8 * 8;     // channel within the block
-              const uint32_t off = (uint32_t)(tok >> 3) * 2048u + (uint32_t)(chl >> 6) * 1024u +
-                                   (uint32_t)(tok & 7) * 128u + ((((uint32_t)(chl & 63) >> 3) ^ (uint32_t)(tok & 7)) << 4);
-              *reinterpret_cast<uint4*>(at + off) = make_uint4(o[0], o[1], o[2], o[3]);
+          const int gi = cb * 4 + cq;
+          const int2 vg = vg_s[gi];
+          uint32_t w0 = 0, w1 = 0, w2 = 0, w3 = 0;
+          float sc = 0.f;
+          if (tvalid) {
+            sc = __half2float(reinterpret_cast<const __half*>(blk)[gi * kPage + slot16]);
+            const uint32_t* cw = reinterpret_cast<const uint32_t*>(blk + vg.y) + slot16 * vg.x;
+            if (vg.x == 4) {
+              const uint4 v4 = *reinterpret_cast<const uint4*>(cw);
+              w0 = v4.x; w1 = v4.y; w2 = v4.z; w3 = v4.w;
+            } else {
+              w0 = cw[0]; w1 = cw[1]; w2 = cw[2];
             }
           }
+          const __half2 s2 = __floats2half2_rn(sc, sc);
+          const float offm = 1024.f + (float)(1 << (vg.x - 1));
+          const __half2 sub = __floats2half2_rn(offm, offm);
+          uint4 o0, o1, o2, o3;
+          if (vg.x == 4) {
+            o0 = deq8_b4(w0, sub, s2);
+            o1 = deq8_b4(w1, sub, s2);
+            o2 = deq8_b4(w2, sub, s2);
+            o3 = deq8_b4(w3, sub, s2);
+          } else {
+            o0 = deq8_b3(w0, sub, s2);
+            o1 = deq8_b3(__funnelshift_r(w0, w1, 24), sub, s2);
+            o2 = deq8_b3(__funnelshift_r(w1, w2, 16), sub, s2);
+            o3 = deq8_b3(w2 >> 8, sub, s2);
+          }
+          if (!tvalid) o0 = o1 = o2 = o3 = make_uint4(0, 0, 0, 0);
+          tc::mbar_wait_ab(&a_empty[as], (((uint32_t)(na >> 1)) & 1u) ^ 1u, a.status, &abort_flag);
+          uint8_t* at = A_s + (size_t)as * 32768 + a_off;
+          const uint32_t c4 = (uint32_t)(cq & 1) * 4u;     // 8-channel chunk index of this group in its atom
+          *reinterpret_cast<uint4*>(at + (((c4 + 0u) ^ x7) << 4)) = o0;
+          *reinterpret_cast<uint4*>(at + (((c4 + 1u) ^ x7) << 4)) = o1;
+          *reinterpret_cast<uint4*>(at + (((c4 + 2u) ^ x7) << 4)) = o2;
+          *reinterpret_cast<uint4*>(at + (((c4 + 3u) ^ x7) << 4)) = o3;
           tc::fence_proxy_async();
           __syncwarp();
           if (lane == 0) tc::mbar_arrive(&a_full[as]);
@@ -356,7 +363,7 @@ __global__ void __launch_bounds__(kValThreads, 1) k_values_tc(ValArgs a) {
         ++nt;
       }
     }
-    if (cur_b >= 0) finish_run(cur_b);
+    if (cur_b >= 0) finish_run();
   }
   tc::tc_fence_before();
   __syncthreads();
@@ -369,38 +376,53 @@ __global__ void __launch_bounds__(kValThreads, 1) k_values_tc(ValArgs a) {
 __global__ void k_values_combine(const float* __restrict__ Y, const float* __restrict__ mseg,
                                  const float* __restrict__ lseg, int G, long long U, int n_st, int slots, int H,
                                  int rv, int NB, int KT, uint8_t* __restrict__ ytiles) {
+  // the runs of sequence b: partial slots of the CTAs whose unit ranges meet [b n_st, (b+1) n_st)
+  __shared__ int seg_i[256];
+  __shared__ float seg_w[256];
+  __shared__ int n_seg;
+  __shared__ float inv_den;
   const int b = blockIdx.x, h = blockIdx.y;
-  const long long lo = (long long)b * n_st, hi = lo + n_st;
-  int c_lo = (int)((lo * G) / U);
-  while (c_lo > 0 && vunit_lo(c_lo, G, U) > lo) --c_lo;
-  while (vunit_lo(c_lo + 1, G, U) <= lo) ++c_lo;
-  float m = -FLT_MAX;
-  for (int cc = c_lo; cc < G && vunit_lo(cc, G, U) < hi; ++cc) {
-    const long long b0 = vunit_lo(cc, G, U), b1 = vunit_lo(cc + 1, G, U);
-    if (b1 <= lo || b0 == b1) continue;
-    const size_t i = ((size_t)cc * slots + (b - (int)(b0 / n_st))) * H + h;
-    if (lseg[i] > 0.f) m = fmaxf(m, mseg[i]);
+  if (threadIdx.x == 0) {
+    const long long lo = (long long)b * n_st, hi = lo + n_st;
+    int c = (int)((lo * G) / U);
+    while (c > 0 && vunit_lo(c, G, U) > lo) --c;
+    while (vunit_lo(c + 1, G, U) <= lo) ++c;
+    int n = 0;
+    float m = -FLT_MAX;
+    long long b0 = vunit_lo(c, G, U);
+    for (; c < G && b0 < hi && n < 256; ++c) {
+      const long long b1 = vunit_lo(c + 1, G, U);
+      if (b1 > lo && b1 > b0) {
+        const int i = (c * slots + (b - (int)(b0 / n_st))) * H + h;
+        if (lseg[i] > 0.f) {
+          seg_i[n++] = i;
+          m = fmaxf(m, mseg[i]);
+        }
+      }
+      b0 = b1;
+    }
+    float den = 0.f;
+    for (int k = 0; k < n; ++k) {
+      seg_w[k] = exp2f(mseg[seg_i[k]] - m);
+      den += seg_w[k] * lseg[seg_i[k]];
+    }
+    n_seg = n;
+    inv_den = den > 0.f ? 1.f / den : 0.f;
   }
-  float den = 0.f;
-  for (int cc = c_lo; cc < G && vunit_lo(cc, G, U) < hi; ++cc) {
-    const long long b0 = vunit_lo(cc, G, U), b1 = vunit_lo(cc + 1, G, U);
-    if (b1 <= lo || b0 == b1) continue;
-    const size_t i = ((size_t)cc * slots + (b - (int)(b0 / n_st))) * H + h;
-    if (lseg[i] > 0.f) den += exp2f(mseg[i] - m) * lseg[i];
-  }
+  __syncthreads();
+  const int ns = n_seg;
+  const float idn = inv_den;
   const int nt = b / NB, r = b % NB;
   for (int j = threadIdx.x; j < rv; j += blockDim.x) {
+    // position of channel j in the value kernel's A tiles: 1 <-> 2 and 5 <-> 6 inside each chunk of 8
+    const int jw = j & 7;
+    const int jp = (j & ~7) | (jw == 1 ? 2 : jw == 2 ? 1 : jw == 5 ? 6 : jw == 6 ? 5 : jw);
     float acc = 0.f;
-    for (int cc = c_lo; cc < G && vunit_lo(cc, G, U) < hi; ++cc) {
-      const long long b0 = vunit_lo(cc, G, U), b1 = vunit_lo(cc + 1, G, U);
-      if (b1 <= lo || b0 == b1) continue;
-      const size_t i = ((size_t)cc * slots + (b - (int)(b0 / n_st))) * H + h;
-      if (lseg[i] > 0.f) acc += exp2f(mseg[i] - m) * Y[i * rv + j];
-    }
-    const uint32_t k = (uint32_t)(h * rv + j), cidx = k & 63u;
-    uint8_t* tile = ytiles + ((size_t)nt * KT + (k >> 6)) * (size_t)NB * 128;
+    for (int k = 0; k < ns; ++k) acc += seg_w[k] * Y[(size_t)seg_i[k] * rv + jp];
+    const uint32_t kk = (uint32_t)(h * rv + j), cidx = kk & 63u;
+    uint8_t* tile = ytiles + ((size_t)nt * KT + (kk >> 6)) * (size_t)NB * 128;
     const uint32_t off = tc::sw128((uint32_t)r, cidx >> 3) + (cidx & 7u) * 2u;
-    *reinterpret_cast<__half*>(tile + off) = __float2half_rn(den > 0.f ? acc / den : 0.f);
+    *reinterpret_cast<__half*>(tile + off) = __float2half_rn(acc * idn);
   }
 }
 
@@ -468,6 +490,7 @@ cudaError_t launch_values_tc(const starkv_layer* L, const uint8_t* pool, long lo
   a.P_ld = so.P_ld;
   a.m_st = so.m_st;
   a.n_st = so.n_st;
+  a.n_g = so.n_g;
   a.U = U;
   a.slots = slots;
   a.Y = (float*)w;

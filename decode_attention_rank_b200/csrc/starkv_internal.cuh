@@ -75,11 +75,12 @@ struct ScoreItem {
 
 // Outputs of the tensor-core score kernel.
 struct ScoreOut {
-  __half* P;          // [B][H][P_ld] exp2(s - m_st) per 256-token super-tile, fp16
-  float* m_st;        // [B][H][n_st]
-  float* l_st;        // [B][H][n_st] sum of the bf16 P values
+  __half* P;          // [B][H][P_ld] exp2(s - m) with m the maximum of the token's 32-token group, fp16
+  float* m_st;        // [B][H][n_g] per 32-token group
+  float* l_st;        // [B][H][n_g] sum of the fp16 P values of the group
   long long P_ld;
-  int n_st;
+  int n_st;           // 256-token super-tiles per sequence
+  int n_g;            // 32-token groups per sequence
 };
 
 }  // namespace starkv
@@ -99,7 +100,9 @@ struct starkv_layer {
   starkv::LatentDesc* d_lat = nullptr;
   starkv::GroupDesc* d_grp = nullptr;
   int* d_key_off = nullptr;
+  int* d_grp_lat = nullptr;     // latent index of every group
   void* A_T = nullptr;          // [Ltot][D] dtype: projection rows (unrotated)
+  void* A_tiles = nullptr;      // bf16 layers: A_T as fp16 128x64 swizzled tiles (tensor-core projection)
   float* Bk = nullptr;          // [Rk][d] fp32: rotated key up-projections B' = R^T B
   // Fused output factors.  f32 layers: [D][H * wv] float32, row-major.  bf16
   // layers: fp16 tiles [Dp/128][Kp/64] of 128 x 64 elements, 128-byte swizzled
@@ -172,8 +175,15 @@ struct OutGeom {
   int KT, DT, G, slots;
 };
 int outproj_nb(int rows);
-OutGeom outproj_geom(const starkv_layer* L);
+OutGeom gemm_geom(int n_out, int K);
+size_t gemm_part_bytes(int n_out, int K, int rows);
 size_t outproj_part_bytes(const starkv_layer* L, int rows);
+// out[row][n] = sum_k y[row][k] Mt[n][k] with Mt as fp16 128x64 swizzled tiles, y as fp16 B tiles.
+cudaError_t launch_gemm_tc(const uint8_t* Mt, int n_out, int K, int n_valid, const void* y_tiles, int rows,
+                           void* out, bool out_f32, float* part, uint32_t* status, cudaStream_t s);
+// Rows of a bf16 matrix as fp16 swizzled tiles of nb rows x 64 columns (nb = 0: the B-tile height for `rows`).
+cudaError_t launch_pack_rows_tiles(const void* x, int rows, int K, void* tiles, cudaStream_t s, int nb = 0);
+size_t rows_tiles_bytes(int rows, int K);
 cudaError_t launch_outproj_tc(const starkv_layer* L, const void* y_tiles, int rows, void* out, float* part,
                               cudaStream_t s);
 

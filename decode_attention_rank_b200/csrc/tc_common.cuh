@@ -17,9 +17,17 @@
 namespace starkv {
 namespace tc {
 
-// Iterations of a bounded wait before it gives up (about a second at the
-// fastest poll rate); a timed-out wait sets STARKV_DEV_TIMEOUT.
-constexpr uint32_t kSpinLimit = 1u << 26;
+// A bounded wait polls mbarrier.try_wait with a suspend-time hint, so a
+// waiting warp sleeps on the barrier instead of spinning; it gives up once two
+// seconds of the global timer have passed and sets STARKV_DEV_TIMEOUT.
+constexpr uint32_t kSuspendNs = 20000;
+constexpr unsigned long long kWaitLimitNs = 2000000000ull;
+
+__device__ __forceinline__ unsigned long long global_ns() {
+  unsigned long long t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -48,18 +56,22 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   uint32_t ok;
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
       "selp.u32 %0, 1, 0, p;\n\t}"
       : "=r"(ok)
-      : "r"(smem_u32(bar)), "r"(parity)
+      : "r"(smem_u32(bar)), "r"(parity), "r"(kSuspendNs)
       : "memory");
   return ok != 0;
 }
 // Bounded wait on the phase with the given parity.  Returns false (and sets
-// the timeout bit) if the phase did not complete within kSpinLimit polls.
+// the timeout bit) if the phase did not complete within kWaitLimitNs.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint32_t* status) {
-  for (uint32_t i = 0; i < kSpinLimit; ++i)
+  if (mbar_try_wait(bar, parity)) return true;
+  const unsigned long long t0 = global_ns();
+  for (uint32_t i = 1;; ++i) {
     if (mbar_try_wait(bar, parity)) return true;
+    if ((i & 15u) == 0u && global_ns() - t0 > kWaitLimitNs) break;
+  }
   if (status) atomicOr(status, kTimeout);
   return false;
 }
@@ -68,9 +80,12 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint32
 // aborted (*abort != 0), so that every role drains quickly and in step.
 __device__ __forceinline__ bool mbar_wait_ab(uint64_t* bar, uint32_t parity, uint32_t* status,
                                              volatile int* abort) {
-  for (uint32_t i = 0; i < kSpinLimit; ++i) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const unsigned long long t0 = global_ns();
+  for (uint32_t i = 1;; ++i) {
     if (mbar_try_wait(bar, parity)) return true;
-    if ((i & 63u) == 63u && *abort) return false;
+    if (*abort) return false;
+    if ((i & 15u) == 0u && global_ns() - t0 > kWaitLimitNs) break;
   }
   if (status) atomicOr(status, kTimeout);
   *abort = 1;
