@@ -382,7 +382,14 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--ref-ctx", type=int, default=0)
+    ap.add_argument("--ctx", type=int, default=0, help="context length (default: the headline 32768); a smaller "
+                    "value gives the small case used for profiler captures")
+    ap.add_argument("--batch", type=int, default=0, help="sequences per step (default 16)")
     args = ap.parse_args()
+    if args.ctx:
+        WORKLOAD["ctx"] = args.ctx
+    if args.batch:
+        WORKLOAD["batch"] = args.batch
     if args.impl == "reference":
         rank = int(os.environ.get("RANK", "0"))
         ws = int(os.environ.get("WORLD_SIZE", "1"))

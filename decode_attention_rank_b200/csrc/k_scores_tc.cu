@@ -25,6 +25,8 @@
 #include <float.h>
 #include <math.h>
 
+#include <utility>
+
 #include "tc_common.cuh"
 
 namespace starkv {
@@ -32,7 +34,7 @@ namespace starkv {
 namespace {
 
 constexpr int kEpiWarps = 16;
-constexpr int kScoreThreads = 64 + 32 * kEpiWarps;   // producer, MMA, 16 epilogue warps
+constexpr int kScoreThreads = 96 + 32 * kEpiWarps;   // key copies, MMA, W''/E copies, 16 epilogue warps
 constexpr int kSuper = 256;          // tokens per super-tile
 constexpr int kETileBytes = 32768;   // one 128-position RoPE tile (128 x 128 fp16)
 
@@ -47,6 +49,8 @@ struct ScoreArgs {
   long long w_stride;
   const ScoreItem* items;
   int n_items;
+  const ScoreEntry* ents;
+  int n_ents;
   const LatentDesc* lat;
   const GroupDesc* grp;
   int gq;                  // query heads per KV head
@@ -65,86 +69,142 @@ struct ScoreArgs {
 
 __device__ __forceinline__ long long unit_lo(int c, int G, long long U) { return (long long)c * U / G; }
 
-// TMEM loads without a wait; tmem_wait() below must follow before any use.
+// TMEM loads without a wait; tc::tmem_ld_wait() and reg_fence() must follow
+// before any use of the registers.
 __device__ __forceinline__ void tmem_ld8_nw(uint32_t taddr, float* v) {
   asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
                : "=f"(v[0]), "=f"(v[1]), "=f"(v[2]), "=f"(v[3]), "=f"(v[4]), "=f"(v[5]), "=f"(v[6]), "=f"(v[7])
                : "r"(taddr));
 }
+__device__ __forceinline__ void tmem_ld4_nw(uint32_t taddr, float* v) {
+  asm volatile("tcgen05.ld.sync.aligned.32x32b.x4.b32 {%0,%1,%2,%3}, [%4];"
+               : "=f"(v[0]), "=f"(v[1]), "=f"(v[2]), "=f"(v[3])
+               : "r"(taddr));
+}
 __device__ __forceinline__ void tmem_ld2_nw(uint32_t taddr, float* v) {
   asm volatile("tcgen05.ld.sync.aligned.32x32b.x2.b32 {%0,%1}, [%2];" : "=f"(v[0]), "=f"(v[1]) : "r"(taddr));
 }
-// Wait for this thread's TMEM loads; the registers are operands so that no use
-// of them can be scheduled before the wait.
-__device__ __forceinline__ void tmem_wait(float* g, float* t) {
-  asm volatile("tcgen05.wait::ld.sync.aligned;"
-               : "+f"(g[0]), "+f"(g[1]), "+f"(g[2]), "+f"(g[3]), "+f"(g[4]), "+f"(g[5]), "+f"(g[6]), "+f"(g[7]),
-                 "+f"(g[8]), "+f"(g[9]), "+f"(g[10]), "+f"(g[11]), "+f"(g[12]), "+f"(g[13]), "+f"(g[14]),
-                 "+f"(g[15]), "+f"(g[16]), "+f"(g[17]), "+f"(g[18]), "+f"(g[19]), "+f"(g[20]), "+f"(g[21]),
-                 "+f"(g[22]), "+f"(g[23]), "+f"(g[24]), "+f"(g[25]), "+f"(g[26]), "+f"(g[27]), "+f"(g[28]),
-                 "+f"(g[29]), "+f"(g[30]), "+f"(g[31]), "+f"(t[0]), "+f"(t[1]), "+f"(t[2]), "+f"(t[3]),
-                 "+f"(t[4]), "+f"(t[5])
-               :
-               : "memory");
-}
+// Emits nothing; makes the registers look rewritten here, so that no use of a
+// TMEM load's destination is scheduled above the preceding wait.
+__device__ __forceinline__ void reg_fence2(float* v) { asm volatile("" : "+f"(v[0]), "+f"(v[1])); }
 
-// 32 bits of a group's code stream starting at stream bit `bit` (shared memory).
-__device__ __forceinline__ uint32_t code_run(const uint8_t* codes, uint32_t bit) {
-  const uint32_t* w = reinterpret_cast<const uint32_t*>(codes) + (bit >> 5);
-  return __funnelshift_r(w[0], w[1], bit & 31u);
-}
-
-// Code i of a run, as the float 1 + u / 2^B (u placed in the top mantissa bits).
+// Code i of a group's per-token code stream (i * B bits in, LSB first), as the
+// float 1 + u / 2^B: the code is moved to mantissa bits [23 - B, 23) and the
+// exponent of 1.0 is or-ed in.  run[] holds the stream re-aligned to bit 0.
 template <int B, int I>
-__device__ __forceinline__ float code_f(uint32_t run) {
-  constexpr int sh = 23 - B - I * B;
-  const uint32_t x = sh >= 0 ? (run << (sh >= 0 ? sh : 0)) : (run >> (sh < 0 ? -sh : 0));
+__device__ __forceinline__ float code_float(const uint32_t* run) {
+  constexpr int p = I * B, k = p >> 5, o = p & 31;
+  constexpr int sh = o - (23 - B);
+  uint32_t x;
+  if constexpr (o + B > 32)
+    x = __funnelshift_r(run[k], run[k + 1], sh);   // the code straddles two words
+  else if constexpr (sh >= 0)
+    x = run[k] >> sh;
+  else
+    x = run[k] << (-sh);
   return __uint_as_float((x & (((1u << B) - 1u) << (23 - B))) | 0x3F800000u);
 }
 
-// acc += sum_i (1 + u_i/2^B) g_i and gs += sum_i g_i over the first `cnt` codes (CNT compile-time bound).
-template <int B, int CNT>
-__device__ __forceinline__ void dot_run(uint32_t run, const float* g, int cnt, float& acc, float& gs) {
+template <int B, int N, int... I>
+__device__ __forceinline__ void group_accumulate(const uint32_t* run, const float* G, float2& acc, float2& gs,
+                                                 std::integer_sequence<int, I...>) {
+  // pairs (2i, 2i + 1): packed fp32x2 multiply-add of the codes with G, and the
+  // running sum of G for the offset term
+  ((acc = __ffma2_rn(make_float2(code_float<B, 2 * I>(run), code_float<B, 2 * I + 1>(run)),
+                     make_float2(G[2 * I], G[2 * I + 1]), acc),
+    gs = __fadd2_rn(gs, make_float2(G[2 * I], G[2 * I + 1]))),
+   ...);
+}
+
+// One quantization group's part of the scores of two tokens (rows of the two
+// 128-token tiles, TMEM columns tcol.. and tcol + 128..):
+//     scale * sum_j (u_j - 2^(B-1)) G_j   over the group's N channels.
+// Row 0's codes start at bit slot * N * B of the code block at `codes`, row 1's
+// at the same bit of the block `row1` bytes further.  Uses f_j = 1 + u_j / 2^B:
+//     sum (u - off) G = 2^B sum f G - (2^B + off) sum G.
+template <int N, int B>
+__device__ __forceinline__ float2 group_score2(uint32_t tcol, const uint8_t* codes, uint32_t row1, int slot,
+                                               float scale0, float scale1) {
+  static_assert(N % 2 == 0 && N >= 2 && N <= 32, "group width");
+  float G0[N], G1[N];
 #pragma unroll
-  for (int i = 0; i < CNT; ++i) {
-    float f;
-    switch (i) {
-      case 0: f = code_f<B, 0>(run); break;
-      case 1: f = code_f<B, 1>(run); break;
-      case 2: f = code_f<B, 2>(run); break;
-      case 3: f = code_f<B, 3>(run); break;
-      case 4: f = code_f<B, 4>(run); break;
-      case 5: f = code_f<B, 5>(run); break;
-      case 6: f = code_f<B, 6>(run); break;
-      default: f = code_f<B, 7>(run); break;
-    }
-    if (i < cnt) {
-      acc = fmaf(f, g[i], acc);
-      gs += g[i];
-    }
+  for (int c = 0; c + 8 <= N; c += 8) {
+    tmem_ld8_nw(tcol + c, G0 + c);
+    tmem_ld8_nw(tcol + 128 + c, G1 + c);
+  }
+  if constexpr (N % 8 >= 4) {
+    tmem_ld4_nw(tcol + (N / 8) * 8, G0 + (N / 8) * 8);
+    tmem_ld4_nw(tcol + 128 + (N / 8) * 8, G1 + (N / 8) * 8);
+  }
+  if constexpr (N % 4 >= 2) {
+    tmem_ld2_nw(tcol + (N / 4) * 4, G0 + (N / 4) * 4);
+    tmem_ld2_nw(tcol + 128 + (N / 4) * 4, G1 + (N / 4) * 4);
+  }
+  constexpr int NR = (N * B + 31) / 32;
+  const uint32_t bit0 = (uint32_t)slot * (uint32_t)(N * B);
+  const uint32_t* w0 = reinterpret_cast<const uint32_t*>(codes) + (bit0 >> 5);
+  const uint32_t* w1 = reinterpret_cast<const uint32_t*>(codes + row1) + (bit0 >> 5);
+  const uint32_t sh = bit0 & 31u;
+  uint32_t raw0[NR + 1], raw1[NR + 1], run0[NR], run1[NR];
+#pragma unroll
+  for (int k = 0; k <= NR; ++k) {
+    raw0[k] = w0[k];
+    raw1[k] = w1[k];
+  }
+#pragma unroll
+  for (int k = 0; k < NR; ++k) {
+    run0[k] = __funnelshift_r(raw0[k], raw0[k + 1], sh);
+    run1[k] = __funnelshift_r(raw1[k], raw1[k + 1], sh);
+  }
+  tc::tmem_ld_wait();
+#pragma unroll
+  for (int c = 0; c < N; c += 2) {
+    reg_fence2(G0 + c);
+    reg_fence2(G1 + c);
+  }
+  float2 acc0 = make_float2(0.f, 0.f), gs0 = acc0, acc1 = acc0, gs1 = acc0;
+  group_accumulate<B, N>(run0, G0, acc0, gs0, std::make_integer_sequence<int, N / 2>{});
+  group_accumulate<B, N>(run1, G1, acc1, gs1, std::make_integer_sequence<int, N / 2>{});
+  constexpr float kf = (float)(1 << B), kg = (float)((1 << B) + (1 << (B - 1)));
+  return make_float2(scale0 * ((acc0.x + acc0.y) * kf - (gs0.x + gs0.y) * kg),
+                     scale1 * ((acc1.x + acc1.y) * kf - (gs1.x + gs1.y) * kg));
+}
+
+// Group kinds: (N / 2 - 1) + 16 * (B - 3) for even N in [2, 32], B in {3, 4}.
+__host__ __device__ __forceinline__ int group_kind(int n, int bits) { return (n / 2 - 1) + 16 * (bits - 3); }
+
+__device__ __forceinline__ float2 group_score2_any(int kind, uint32_t tcol, const uint8_t* codes, uint32_t row1,
+                                                   int slot, float scale0, float scale1) {
+  switch (kind) {
+#define STARKV_GS(n)                                                                     \
+  case (n) / 2 - 1: return group_score2<(n), 3>(tcol, codes, row1, slot, scale0, scale1); \
+  case 16 + (n) / 2 - 1: return group_score2<(n), 4>(tcol, codes, row1, slot, scale0, scale1);
+    STARKV_GS(2) STARKV_GS(4) STARKV_GS(6) STARKV_GS(8) STARKV_GS(10) STARKV_GS(12) STARKV_GS(14) STARKV_GS(16)
+    STARKV_GS(18) STARKV_GS(20) STARKV_GS(22) STARKV_GS(24) STARKV_GS(26) STARKV_GS(28) STARKV_GS(30) STARKV_GS(32)
+#undef STARKV_GS
+    default: return make_float2(0.f, 0.f);
   }
 }
 
-// sum over one quantization group of (u - 2^(B-1)) * scale * G for one token:
-// nf full 8-code chunks from G[0..32), then `tail` codes from T.
-template <int B>
-__device__ __forceinline__ float group_dot(const uint8_t* codes, uint32_t bit0, int nf, int tail, const float* G,
-                                           const float* T) {
-  float acc = 0.f, gs = 0.f;
-#pragma unroll
-  for (int c = 0; c < 4; ++c)
-    if (c < nf) dot_run<B, 8>(code_run(codes, bit0 + (uint32_t)(c * 8 * B)), G + 8 * c, 8, acc, gs);
-  if (tail) dot_run<B, 6>(code_run(codes, bit0 + (uint32_t)(nf * 8 * B)), T, tail, acc, gs);
-  // sum (u - off) g = 2^B sum f g - (2^B + off) sum g
-  return (float)(1 << B) * acc - (float)((1 << B) + (1 << (B - 1))) * gs;
+// Warp-wide maximum and integer sum in one instruction each.
+__device__ __forceinline__ float warp_max(float x) {
+  float r;
+  asm volatile("redux.sync.max.f32 %0, %1, 0xffffffff;" : "=f"(r) : "f"(x));
+  return r;
+}
+__device__ __forceinline__ int warp_sum(int x) {
+  int r;
+  asm volatile("redux.sync.add.s32 %0, %1, 0xffffffff;" : "=r"(r) : "r"(x));
+  return r;
 }
 
-// Per query head: its key latent's groups (start, n, bits, code offset), the
-// latent block's offset inside the item's key range, and its first G column.
-struct HeadPlan {
-  int ng, blk_rel, hcol, pad;
-  int4 grp[4];
-};
+// Barrier among the 16 epilogue warps only (id 1; id 0 is __syncthreads).
+__device__ __forceinline__ void epilogue_sync() { asm volatile("bar.sync 1, %0;" ::"n"(32 * kEpiWarps) : "memory"); }
+
+constexpr int kMaxGroups = 4;
+constexpr int kMaxEnts = 512;      // entries of all items, resident in shared memory
+constexpr int kMaxItemHeads = 8;
+
 
 __global__ void __launch_bounds__(kScoreThreads, 1) k_scores_tc(ScoreArgs a) {
   extern __shared__ uint8_t smem_raw[];
@@ -153,8 +213,8 @@ __global__ void __launch_bounds__(kScoreThreads, 1) k_scores_tc(ScoreArgs a) {
   __shared__ uint32_t tmem_base;
   __shared__ volatile int abort_flag;
   __shared__ ScoreItem items_s[64];
-  __shared__ HeadPlan hp_s[64];
-  __shared__ float sc_s[4][512];
+  __shared__ ScoreEntry ent_s[kMaxEnts];
+  __shared__ float sc_s[2][kMaxItemHeads][kSuper];   // per-item scores, summed over the entry parts
   uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   uint8_t* E_s = smem;                                   // 2 x 32 KB
   uint8_t* W_s = E_s + 2 * kETileBytes;                  // WS x w_stage
@@ -180,28 +240,10 @@ __global__ void __launch_bounds__(kScoreThreads, 1) k_scores_tc(ScoreArgs a) {
     abort_flag = 0;
     tc::fence_mbar_init();
   }
-  // item table and per-head plans in shared memory
+  // item and entry tables in shared memory; score accumulators zeroed
   for (int it = threadIdx.x; it < a.n_items; it += blockDim.x) items_s[it] = a.items[it];
-  for (int h = threadIdx.x; h < a.H; h += blockDim.x) {
-    HeadPlan hp{};
-    const LatentDesc ld = a.lat[h / a.gq];
-    int item_key_off = 0, hcol = 0;
-    for (int it = 0; it < a.n_items; ++it) {
-      const ScoreItem& x = a.items[it];
-      if (h >= x.h0 && h < x.h0 + x.nh) {
-        item_key_off = x.key_off;
-        hcol = x.hcol[h - x.h0];
-      }
-    }
-    hp.ng = min(ld.n_groups, 4);
-    hp.blk_rel = ld.block_off - item_key_off;
-    hp.hcol = hcol;
-    for (int g = 0; g < hp.ng; ++g) {
-      const GroupDesc gd = a.grp[ld.group0 + g];
-      hp.grp[g] = make_int4(gd.start, gd.n, gd.bits, gd.code_off);
-    }
-    hp_s[h] = hp;
-  }
+  for (int x = threadIdx.x; x < a.n_ents; x += blockDim.x) ent_s[x] = a.ents[x];
+  for (int x = threadIdx.x; x < 2 * kMaxItemHeads * kSuper; x += blockDim.x) (&sc_s[0][0][0])[x] = 0.f;
   if (warp == 1) tc::tmem_alloc(&tmem_base, 512);
   tc::tc_fence_before();
   __syncthreads();
@@ -209,56 +251,85 @@ __global__ void __launch_bounds__(kScoreThreads, 1) k_scores_tc(ScoreArgs a) {
   const uint32_t tmem = tmem_base;
 
   if (warp == 0) {
-    // ------------------------------------------------------------ producer
+    // ------------------------------------------------------------ key copies
+    // Warp-wide: lane 0 owns the barriers; every lane fetches one page id and
+    // issues that page's copy, so no copy waits behind a page-table load.
+    int i = 0, nk = 0;                    // nk: issued stage fills (for the drain below)
+    for (long long u = u0; u < u1; ++u) {
+      if (__shfl_sync(0xffffffffu, abort_flag, 0)) break;
+      const int b = (int)(u / a.n_st), st = (int)(u % a.n_st);
+      const int t0 = st * kSuper;
+      const int len = min(a.seq_lens[b], a.max_pages * kPage);
+      if (t0 >= len) continue;
+      const int npg = min(kSuper / kPage, (len - t0 + kPage - 1) / kPage);
+      int page = 0;
+      if (lane < npg) {
+        page = a.pt[(size_t)b * a.max_pages + st * (kSuper / kPage) + lane];
+        if (page < 0 || page >= a.n_pages) {
+          atomicOr(a.status, kBadPage);
+          page = 0;
+        }
+      }
+      const uint8_t* page_base = a.pool + (size_t)page * a.page_bytes;
+      for (int it = 0; it < a.n_items; ++it, ++i) {
+        const ScoreItem& item = items_s[it];
+        const int ks = i % a.KS;
+        bool ok = true;
+        if (lane == 0) {
+          ok = tc::mbar_wait_ab(&k_empty[ks], (((uint32_t)(i / a.KS)) & 1u) ^ 1u, a.status, &abort_flag);
+          if (ok) tc::mbar_expect_tx(&k_full[ks], (uint32_t)(npg * item.key_bytes));
+        }
+        ok = __shfl_sync(0xffffffffu, ok, 0);
+        if (!ok) break;
+        if (lane < npg)
+          tc::bulk_g2s(K_s + (size_t)ks * a.k_stage + (size_t)lane * item.key_bytes, page_base + item.key_off,
+                       (uint32_t)item.key_bytes, &k_full[ks]);
+        ++nk;
+      }
+    }
+    // let copies in flight land before the CTA can exit
     if (lane == 0) {
-      int i = 0, uc = 0;
-      int nk = 0, nw = 0, ne[2] = {0, 0};   // issued stage fills (for the drain below)
+      for (int j = max(0, nk - a.KS); j < nk; ++j)
+        tc::mbar_wait(&k_full[j % a.KS], ((uint32_t)(j / a.KS)) & 1u, a.status);
+    }
+    __syncwarp();
+  } else if (warp == 2) {
+    // ------------------------------------------------------------ W'' and RoPE tiles
+    // one thread; runs ahead of the key copies, bounded only by its own stages
+    if (lane == 0) {
+      int i = 0, uc = 0, nw = 0, ne[2] = {0, 0};
       for (long long u = u0; u < u1 && !abort_flag; ++u) {
         const int b = (int)(u / a.n_st), st = (int)(u % a.n_st);
         const int t0 = st * kSuper;
         const int len = min(a.seq_lens[b], a.max_pages * kPage);
         if (t0 >= len) continue;
-        const int npg = min(kSuper / kPage, (len - t0 + kPage - 1) / kPage);
-        for (int it = 0; it < a.n_items && !abort_flag; ++it, ++i) {
-          const ScoreItem item = a.items[it];
-          const int ks = i % a.KS, ws = i % a.WS;
-          if (!tc::mbar_wait_ab(&k_empty[ks], (((uint32_t)(i / a.KS)) & 1u) ^ 1u, a.status, &abort_flag)) break;
-          tc::mbar_expect_tx(&k_full[ks], (uint32_t)(npg * item.key_bytes));
-          for (int pg = 0; pg < npg; ++pg) {
-            int page = a.pt[(size_t)b * a.max_pages + st * (kSuper / kPage) + pg];
-            if (page < 0 || page >= a.n_pages) {
-              atomicOr(a.status, kBadPage);
-              page = 0;
-            }
-            tc::bulk_g2s(K_s + (size_t)ks * a.k_stage + (size_t)pg * item.key_bytes,
-                         a.pool + (size_t)page * a.page_bytes + item.key_off, (uint32_t)item.key_bytes, &k_full[ks]);
-          }
-          ++nk;
-          if (!tc::mbar_wait_ab(&w_empty[ws], (((uint32_t)(i / a.WS)) & 1u) ^ 1u, a.status, &abort_flag)) break;
+        bool ok = true;
+        for (int k = 0; k < 2 && ok; ++k) {
+          ok = tc::mbar_wait_ab(&e_empty[k], ((uint32_t)uc & 1u) ^ 1u, a.status, &abort_flag);
+          if (!ok) break;
+          tc::mbar_expect_tx(&e_full[k], kETileBytes);
+          tc::bulk_g2s(E_s + k * kETileBytes, a.E + (size_t)(t0 / 128 + k) * kETileBytes, kETileBytes, &e_full[k]);
+          ++ne[k];
+        }
+        for (int it = 0; it < a.n_items && ok; ++it, ++i) {
+          const ScoreItem& item = items_s[it];
+          const int ws = i % a.WS;
+          ok = tc::mbar_wait_ab(&w_empty[ws], (((uint32_t)(i / a.WS)) & 1u) ^ 1u, a.status, &abort_flag);
+          if (!ok) break;
           tc::mbar_expect_tx(&w_full[ws], (uint32_t)(item.npad * 256));
           tc::bulk_g2s(W_s + (size_t)ws * a.w_stage, a.W + (size_t)b * a.w_stride + item.w_off,
                        (uint32_t)(item.npad * 256), &w_full[ws]);
           ++nw;
-          if (it == 0) {
-            for (int k = 0; k < 2; ++k) {
-              if (!tc::mbar_wait_ab(&e_empty[k], ((uint32_t)uc & 1u) ^ 1u, a.status, &abort_flag)) break;
-              tc::mbar_expect_tx(&e_full[k], kETileBytes);
-              tc::bulk_g2s(E_s + k * kETileBytes, a.E + (size_t)(t0 / 128 + k) * kETileBytes, kETileBytes,
-                           &e_full[k]);
-              ++ne[k];
-            }
-          }
         }
+        if (!ok) break;
         ++uc;
       }
-      // let copies in flight land before the CTA can exit
-      for (int j = max(0, nk - a.KS); j < nk; ++j)
-        tc::mbar_wait(&k_full[j % a.KS], ((uint32_t)(j / a.KS)) & 1u, a.status);
       for (int j = max(0, nw - a.WS); j < nw; ++j)
         tc::mbar_wait(&w_full[j % a.WS], ((uint32_t)(j / a.WS)) & 1u, a.status);
       for (int k = 0; k < 2; ++k)
         if (ne[k] > 0) tc::mbar_wait(&e_full[k], (uint32_t)(ne[k] - 1) & 1u, a.status);
     }
+    __syncwarp();
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issue
     if (lane == 0) {
@@ -268,7 +339,7 @@ __global__ void __launch_bounds__(kScoreThreads, 1) k_scores_tc(ScoreArgs a) {
         const int len = min(a.seq_lens[b], a.max_pages * kPage);
         if (st * kSuper >= len) continue;
         for (int it = 0; it < a.n_items && !abort_flag; ++it, ++i) {
-          const int npad = a.items[it].npad;
+          const int npad = items_s[it].npad;
           const int ws = i % a.WS;
           if (!tc::mbar_wait_ab(&w_full[ws], ((uint32_t)(i / a.WS)) & 1u, a.status, &abort_flag)) { abort_flag = 1; break; }
           if (it == 0) {
@@ -305,64 +376,58 @@ __global__ void __launch_bounds__(kScoreThreads, 1) k_scores_tc(ScoreArgs a) {
     }
   } else {
     // ------------------------------------------------------------ epilogue
-    // 16 warps: TMEM lane quarter q = warp % 4, tile k, head parity hp
-    const int e = warp - 2;              // 0..15
+    // 16 warps.  Warp e reads TMEM lane quarter q = warp % 4: tokens q * 32 +
+    // lane of both 128-token tiles, and scores part e / 4 of each item's
+    // (head, group) entries; the parts meet in sc_s.  After a barrier of the
+    // epilogue warps the softmax statistics are taken per (head, 32 tokens).
+    const int e = warp - 3;              // 0..15
     const int q = warp & 3;
-    const int k = (e >> 2) & 1;
-    const int hpar = e >> 3;
-    const int tau = k * 128 + q * 32 + lane;
-    const int pg = tau >> 4, slot = tau & 15;
+    const int part = e >> 2;
+    const int tau0 = q * 32 + lane;      // tile-0 token; tile 1 holds tau0 + 128
+    const int pg0 = tau0 >> 4, slot = tau0 & 15;
     int i = 0;
-    // every epilogue warp runs the same loop (named barriers below); after an
+    // every epilogue warp runs the same loop (named barrier below); after an
     // abort the waits fail fast and the work is skipped
     for (long long u = u0; u < u1; ++u) {
       const int b = (int)(u / a.n_st), st = (int)(u % a.n_st);
       const int t0 = st * kSuper;
       const int len = min(a.seq_lens[b], a.max_pages * kPage);
       if (t0 >= len) continue;
-      const int t = t0 + tau;
-      const bool valid = t < len;
       for (int it = 0; it < a.n_items; ++it, ++i) {
         const ScoreItem& item = items_s[it];
-        const int nh = item.nh;
         const int ks = i % a.KS;
         const bool ok1 = tc::mbar_wait_ab(&k_full[ks], ((uint32_t)(i / a.KS)) & 1u, a.status, &abort_flag);
         const bool ok = ok1 && tc::mbar_wait_ab(&acc_full[i & 1], ((uint32_t)(i >> 1)) & 1u, a.status, &abort_flag);
         tc::tc_fence_after();
-        const uint8_t* page = K_s + (size_t)ks * a.k_stage + (size_t)pg * item.key_bytes;
-        const uint32_t tcol = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)((i & 1) * 256 + k * 128);
-        for (int hh = hpar; hh < nh; hh += 2) {
-          const HeadPlan& hp = hp_s[item.h0 + hh];
-          const uint8_t* blk = page + hp.blk_rel;
-          float s = 0.f;
-          if (ok) {
-            for (int gi = 0; gi < hp.ng; ++gi) {
-              const int4 gd = hp.grp[gi];     // start, n, bits, code_off
-              const int nf = gd.y >> 3, tail = gd.y & 7;
-              float G[32], T[6];
-              const uint32_t c0 = tcol + (uint32_t)(hp.hcol + gd.x);
-#pragma unroll
-              for (int c = 0; c < 4; ++c)
-                if (c < nf) tmem_ld8_nw(c0 + 8 * c, G + 8 * c);
-              const uint32_t ct = c0 + (uint32_t)(8 * nf);
-              if (tail > 0) tmem_ld2_nw(ct, T);
-              if (tail > 2) tmem_ld2_nw(ct + 2, T + 2);
-              if (tail > 4) tmem_ld2_nw(ct + 4, T + 4);
-              tmem_wait(G, T);
-              const float scale = __half2float(reinterpret_cast<const __half*>(blk)[gi * kPage + slot]);
-              const uint8_t* codes = blk + gd.w;
-              const uint32_t bit0 = (uint32_t)(slot * gd.y * gd.z);
-              float d;
-              if (gd.z == 3)
-                d = group_dot<3>(codes, bit0, nf, tail, G, T);
-              else if (gd.z == 4)
-                d = group_dot<4>(codes, bit0, nf, tail, G, T);
-              else
-                d = 0.f;     // layers with other code widths do not take this kernel
-              s = fmaf(scale, d, s);
+        float* sc = &sc_s[i & 1][0][0];
+        if (ok) {
+          const uint8_t* page0 = K_s + (size_t)ks * a.k_stage + (size_t)pg0 * item.key_bytes;
+          const uint32_t row1 = 8u * (uint32_t)item.key_bytes;   // tile 1's page is 8 pages on
+          const uint32_t tcol = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)((i & 1) * 256);
+          int hcur = -1;
+          float s0 = 0.f, s1 = 0.f;
+          const int x1 = item.ent0 + item.part[part + 1];
+          for (int x = item.ent0 + item.part[part]; x < x1; ++x) {
+            const ScoreEntry en = ent_s[x];
+            const int hh = en.y >> 8;
+            if (hh != hcur) {
+              if (hcur >= 0) {
+                atomicAdd(&sc[hcur * kSuper + tau0], s0);
+                atomicAdd(&sc[hcur * kSuper + tau0 + 128], s1);
+              }
+              hcur = hh;
+              s0 = s1 = 0.f;
             }
+            const __half* scl = reinterpret_cast<const __half*>(page0 + en.w);
+            const float2 r = group_score2_any(en.y & 255, tcol + (uint32_t)en.x, page0 + en.z, row1, slot,
+                                              __half2float(scl[slot]), __half2float(scl[slot + row1 / 2]));
+            s0 += r.x;
+            s1 += r.y;
           }
-          sc_s[hh >> 1][e * 32 + lane] = s;
+          if (hcur >= 0) {
+            atomicAdd(&sc[hcur * kSuper + tau0], s0);
+            atomicAdd(&sc[hcur * kSuper + tau0 + 128], s1);
+          }
         }
         tc::tc_fence_before();
         __syncwarp();
@@ -370,29 +435,34 @@ __global__ void __launch_bounds__(kScoreThreads, 1) k_scores_tc(ScoreArgs a) {
           tc::mbar_arrive(&acc_free[i & 1]);
           tc::mbar_arrive(&k_empty[ks]);
         }
-        const size_t hb = (size_t)b * a.H + item.h0;
-        if (a.S_dbg) {
-          for (int hh = hpar; hh < nh; hh += 2)
-            if (valid) a.S_dbg[(hb + hh) * a.P_ld + t] = sc_s[hh >> 1][e * 32 + lane];
-          continue;
-        }
-        // softmax statistics per 32-token group (this warp's tokens), per head:
-        // m = max s, P = exp2(s - m) rounded to fp16, l = sum of the fp16 P
-        const int grp = (t0 >> 5) + k * 4 + q;
-        for (int hh = hpar; hh < nh; hh += 2) {
-          const float sv = sc_s[hh >> 1][e * 32 + lane];
-          float m = valid ? sv : -FLT_MAX;
-          for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-          float p = 0.f;
+        epilogue_sync();
+        // softmax statistics per (head, 32-token group): m = max s, P =
+        // exp2(s - m) rounded to fp16, l = sum of the fp16 P (exact: each P is
+        // a multiple of 2^-24, summed as integers)
+        for (int task = e; task < item.nh * 8; task += kEpiWarps) {
+          const int hh = task >> 3, kq = task & 7;
+          const int tau = kq * 32 + lane;
+          float* cell = &sc[hh * kSuper + tau];
+          const float sv = *cell;
+          *cell = 0.f;
+          const int t = t0 + tau;
+          const bool valid = t < len;
+          const size_t row = (size_t)b * a.H + item.h0 + hh;
+          if (a.S_dbg) {
+            if (valid) a.S_dbg[row * a.P_ld + t] = sv;
+            continue;
+          }
+          const float m = warp_max(valid ? sv : -FLT_MAX);
+          int pi = 0;
           if (valid) {
             const __half pb = __float2half_rn(exp2f(sv - m));
-            a.P[(hb + hh) * a.P_ld + t] = pb;
-            p = __half2float(pb);
+            a.P[row * a.P_ld + t] = pb;
+            pi = __float2int_rn(__half2float(pb) * 16777216.f);
           }
-          for (int o = 16; o > 0; o >>= 1) p += __shfl_xor_sync(0xffffffffu, p, o);
+          const int ps = warp_sum(pi);
           if (lane == 0) {
-            a.m_st[(hb + hh) * a.n_g + grp] = m;
-            a.l_st[(hb + hh) * a.n_g + grp] = p;
+            a.m_st[row * a.n_g + (t0 >> 5) + kq] = m;
+            a.l_st[row * a.n_g + (t0 >> 5) + kq] = (float)ps * (1.f / 16777216.f);
           }
         }
       }
@@ -491,18 +561,24 @@ bool plan_scores_tc(starkv_layer* L) {
   const starkv_layer_config& c = L->cfg;
   if (c.dtype != STARKV_BF16 || c.plain || !c.rope || c.head_dim != 128 || !v.quantized) return false;
   if (c.n_heads > 64) return false;
-  // the epilogue reads TMEM in pairs of columns: every key group must have an even width
-  for (int g = 0; g < v.Hkv; ++g)
-    for (int k = 0; k < L->lat[g].n_groups; ++k)
-      if (L->grp[L->lat[g].group0 + k].n % 2) return false;
+  // the epilogue has compiled dot products for even group widths up to 32 at
+  // 3 or 4 bits, and at most kMaxGroups groups per key latent
+  for (int g = 0; g < v.Hkv; ++g) {
+    if (L->lat[g].n_groups > kMaxGroups) return false;
+    for (int k = 0; k < L->lat[g].n_groups; ++k) {
+      const GroupDesc& gd = L->grp[L->lat[g].group0 + k];
+      if (gd.n % 2 || gd.n > 32 || (gd.bits != 3 && gd.bits != 4)) return false;
+    }
+  }
   L->items.clear();
+  L->score_ents.clear();
   int w_off = 0, max_key = 0, max_w = 0;
   int h = 0;
   while (h < v.H) {
     ScoreItem it{};
     it.h0 = h;
     int cols = 0;
-    while (h < v.H && it.nh < 8) {
+    while (h < v.H && it.nh < kMaxItemHeads) {
       const int r = L->lat[h / v.group_q].width;
       if (cols + r > 128) break;
       it.hr[it.nh] = r;
@@ -519,17 +595,46 @@ bool plan_scores_tc(starkv_layer* L) {
     it.key_bytes = L->lat[g1 + 1].block_off - it.key_off;
     max_key = std::max(max_key, it.key_bytes);
     max_w = std::max(max_w, it.npad * 256);
+    // (head, group) entries and their split into four parts of about equal
+    // work (a group costs about 3.3 instructions per channel plus a fixed part)
+    it.ent0 = (int)L->score_ents.size();
+    std::vector<double> cost;
+    for (int hh = 0; hh < it.nh; ++hh) {
+      const LatentDesc& ld = L->lat[(it.h0 + hh) / v.group_q];
+      const int blk_rel = ld.block_off - it.key_off;
+      for (int k = 0; k < ld.n_groups; ++k) {
+        const GroupDesc& gd = L->grp[ld.group0 + k];
+        L->score_ents.push_back(make_int4(it.hcol[hh] + gd.start, group_kind(gd.n, gd.bits) | (hh << 8),
+                                          blk_rel + gd.code_off, blk_rel + k * kPage * 2));
+        cost.push_back(3.3 * gd.n + 16.0);
+      }
+    }
+    const int ne = (int)cost.size();
+    double total = 0.0;
+    for (double c : cost) total += c;
+    it.part[0] = 0;
+    double run = 0.0;
+    int p = 1;
+    for (int x = 0; x < ne && p < 4; ++x) {
+      run += cost[x];
+      // close part p - 1 after entry x once it holds its share
+      while (p < 4 && run >= total * p / 4.0 - 0.5 * cost[x]) it.part[p++] = x + 1;
+    }
+    while (p < 4) it.part[p++] = ne;
+    it.part[4] = ne;
     L->items.push_back(it);
   }
+  if (L->score_ents.size() > (size_t)kMaxEnts) return false;
   L->w_stride = w_off;
   L->k_stage = (kSuper / kPage) * max_key + 16;
   L->k_stage = (L->k_stage + 1023) / 1024 * 1024;
   L->w_stage = (max_w + 1023) / 1024 * 1024;
   // dynamic shared memory next to ~21 KB of static tables and barriers
-  const size_t budget = 204 * 1024 - 2 * kETileBytes;
+  const size_t budget = 194 * 1024 - 2 * kETileBytes;
   L->WS = 3;
-  L->KS = 2;
+  L->KS = 3;
   while (L->WS > 2 && (size_t)L->WS * L->w_stage + (size_t)L->KS * L->k_stage > budget) --L->WS;
+  while (L->KS > 2 && (size_t)L->WS * L->w_stage + (size_t)L->KS * L->k_stage > budget) --L->KS;
   if ((size_t)L->WS * L->w_stage + (size_t)L->KS * L->k_stage > budget) return false;
   const int mp = c.max_positions > 0 ? c.max_positions : 32768;
   L->rope_tiles = (mp + kSuper - 1) / kSuper * (kSuper / 128);
@@ -585,6 +690,8 @@ cudaError_t launch_scores_tc(const starkv_layer* L, const uint8_t* pool, long lo
   a.w_stride = L->w_stride;
   a.items = L->d_items;
   a.n_items = (int)L->items.size();
+  a.ents = L->d_score_ents;
+  a.n_ents = (int)L->score_ents.size();
   a.lat = L->d_lat;
   a.grp = L->d_grp;
   a.gq = v.group_q;

@@ -130,32 +130,46 @@ __global__ void __launch_bounds__(kValThreads, 1) k_values_tc(ValArgs a) {
 
   // The work list: units u0..u1-1 -> tiles (two per unit) with tokens < len.
   if (warp == 0) {
-    if (lane == 0) {
-      int nt = 0;
-      for (long long u = u0; u < u1 && !abort_flag; ++u) {
-        const int b = (int)(u / a.n_st), st = (int)(u % a.n_st);
-        const int len = min(a.seq_lens[b], a.max_pages * kPage);
-        for (int tile = 0; tile < 2 && !abort_flag; ++tile) {
-          const int t0 = st * kVSuper + tile * 128;
-          if (t0 >= len) break;
-          const int r = nt & 1;
-          if (!tc::mbar_wait_ab(&raw_empty[r], (((uint32_t)(nt >> 1)) & 1u) ^ 1u, a.status, &abort_flag)) break;
-          const int npg = min(8, (len - t0 + kPage - 1) / kPage);
-          tc::mbar_expect_tx(&raw_full[r], (uint32_t)(npg * a.vblk_bytes));
-          for (int pg = 0; pg < npg; ++pg) {
-            int page = a.pt[(size_t)b * a.max_pages + t0 / kPage + pg];
-            if (page < 0 || page >= a.n_pages) {
-              atomicOr(a.status, kBadPage);
-              page = 0;
-            }
-            tc::bulk_g2s(R_s + (size_t)r * raw_stage + (size_t)pg * a.vblk_bytes,
-                         a.pool + (size_t)page * a.page_bytes + a.vblk_off, (uint32_t)a.vblk_bytes, &raw_full[r]);
+    // warp-wide producer: every lane fetches one page id and issues that page's copy
+    int nt = 0;
+    for (long long u = u0; u < u1; ++u) {
+      if (__shfl_sync(0xffffffffu, abort_flag, 0)) break;
+      const int b = (int)(u / a.n_st), st = (int)(u % a.n_st);
+      const int len = min(a.seq_lens[b], a.max_pages * kPage);
+      bool stop = false;
+      for (int tile = 0; tile < 2; ++tile) {
+        const int t0 = st * kVSuper + tile * 128;
+        if (t0 >= len) break;
+        const int r = nt & 1;
+        const int npg = min(8, (len - t0 + kPage - 1) / kPage);
+        int page = 0;
+        if (lane < npg) {
+          page = a.pt[(size_t)b * a.max_pages + t0 / kPage + lane];
+          if (page < 0 || page >= a.n_pages) {
+            atomicOr(a.status, kBadPage);
+            page = 0;
           }
-          ++nt;
         }
+        bool ok = true;
+        if (lane == 0) {
+          ok = tc::mbar_wait_ab(&raw_empty[r], (((uint32_t)(nt >> 1)) & 1u) ^ 1u, a.status, &abort_flag);
+          if (ok) tc::mbar_expect_tx(&raw_full[r], (uint32_t)(npg * a.vblk_bytes));
+        }
+        ok = __shfl_sync(0xffffffffu, ok, 0);
+        if (!ok) {
+          stop = true;
+          break;
+        }
+        if (lane < npg)
+          tc::bulk_g2s(R_s + (size_t)r * raw_stage + (size_t)lane * a.vblk_bytes,
+                       a.pool + (size_t)page * a.page_bytes + a.vblk_off, (uint32_t)a.vblk_bytes, &raw_full[r]);
+        ++nt;
       }
-      for (int j = max(0, nt - 2); j < nt; ++j) tc::mbar_wait(&raw_full[j & 1], ((uint32_t)(j >> 1)) & 1u, a.status);
+      if (stop) break;
     }
+    if (lane == 0)
+      for (int j = max(0, nt - 2); j < nt; ++j) tc::mbar_wait(&raw_full[j & 1], ((uint32_t)(j >> 1)) & 1u, a.status);
+    __syncwarp();
   } else if (warp == 1) {
     if (lane == 0) {
       const uint32_t idesc = tc::idesc_f16(128, a.H, false, true, false);
