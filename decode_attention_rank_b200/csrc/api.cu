@@ -207,7 +207,7 @@ void starkv_free_layer(starkv_layer* L) {
   cudaFree(L->M_T);
   cudaFree(L->status);
   cudaFree(L->d_items);
-  cudaFree(L->d_score_ents);
+  cudaFree(L->d_score_heads);
   cudaFree(L->rope_E);
   cudaSetDevice(cur);
   delete L;
@@ -314,12 +314,12 @@ starkv_status starkv_load_factors(const starkv_layer_config* cfg, const void* A_
   L->tc_values = L->tc_scores && plan_values_tc(L);
   if (L->tc_scores) {
     if (cudaMalloc(&L->d_items, sizeof(ScoreItem) * L->items.size()) != cudaSuccess ||
-        cudaMalloc(&L->d_score_ents, sizeof(ScoreEntry) * L->score_ents.size()) != cudaSuccess ||
+        cudaMalloc(&L->d_score_heads, sizeof(ScoreHead) * L->score_heads.size()) != cudaSuccess ||
         cudaMalloc(&L->rope_E, (size_t)L->rope_tiles * 32768) != cudaSuccess)
       return fail(STARKV_ERR_OOM, "cudaMalloc");
     if (cudaMemcpyAsync(L->d_items, L->items.data(), sizeof(ScoreItem) * L->items.size(), cudaMemcpyHostToDevice,
                         s) != cudaSuccess ||
-        cudaMemcpyAsync(L->d_score_ents, L->score_ents.data(), sizeof(ScoreEntry) * L->score_ents.size(),
+        cudaMemcpyAsync(L->d_score_heads, L->score_heads.data(), sizeof(ScoreHead) * L->score_heads.size(),
                         cudaMemcpyHostToDevice, s) != cudaSuccess ||
         build_rope_table(L, s) != cudaSuccess)
       return fail(STARKV_ERR_CUDA, "rope table");

@@ -18,9 +18,13 @@
 // super-tiles (two M = 128 tiles sharing one W'' load) of one sequence.
 //   warp 0      bulk copies: RoPE table tiles, W'' item blocks, key latent pages
 //   warp 1      tcgen05.mma issue (one thread), TMEM allocation
-//   warps 2-17  epilogue (16 warps: TMEM lane quarter x tile x head parity):
-//               TMEM -> registers, dequantize + dot, softmax statistics of
-//               the super-tile, P = exp2(s - m) as fp16
+//   warp 2      bulk copies of the RoPE table tiles and W'' item blocks
+//   warps 3-18  epilogue, two sets of 8 warps taking alternate MMA items; in
+//               a set, warp (tile, lane quarter) owns 32 tokens of one
+//               128-token tile.  A thread scores its token for every head of
+//               the item (TMEM -> registers, dot with the 4/3-bit codes), and
+//               the warp takes the softmax statistics of its 32-token group
+//               in registers: m = max s, P = exp2(s - m) as fp16, l = sum P
 // Outputs per (sequence, head): P (fp16), and per 32-token group m and l = sum P.
 #include <float.h>
 #include <math.h>
@@ -49,8 +53,7 @@ struct ScoreArgs {
   long long w_stride;
   const ScoreItem* items;
   int n_items;
-  const ScoreEntry* ents;
-  int n_ents;
+  const ScoreHead* heads;  // [H]
   const LatentDesc* lat;
   const GroupDesc* grp;
   int gq;                  // query heads per KV head
@@ -69,25 +72,6 @@ struct ScoreArgs {
 
 __device__ __forceinline__ long long unit_lo(int c, int G, long long U) { return (long long)c * U / G; }
 
-// TMEM loads without a wait; tc::tmem_ld_wait() and reg_fence() must follow
-// before any use of the registers.
-__device__ __forceinline__ void tmem_ld8_nw(uint32_t taddr, float* v) {
-  asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
-               : "=f"(v[0]), "=f"(v[1]), "=f"(v[2]), "=f"(v[3]), "=f"(v[4]), "=f"(v[5]), "=f"(v[6]), "=f"(v[7])
-               : "r"(taddr));
-}
-__device__ __forceinline__ void tmem_ld4_nw(uint32_t taddr, float* v) {
-  asm volatile("tcgen05.ld.sync.aligned.32x32b.x4.b32 {%0,%1,%2,%3}, [%4];"
-               : "=f"(v[0]), "=f"(v[1]), "=f"(v[2]), "=f"(v[3])
-               : "r"(taddr));
-}
-__device__ __forceinline__ void tmem_ld2_nw(uint32_t taddr, float* v) {
-  asm volatile("tcgen05.ld.sync.aligned.32x32b.x2.b32 {%0,%1}, [%2];" : "=f"(v[0]), "=f"(v[1]) : "r"(taddr));
-}
-// Emits nothing; makes the registers look rewritten here, so that no use of a
-// TMEM load's destination is scheduled above the preceding wait.
-__device__ __forceinline__ void reg_fence2(float* v) { asm volatile("" : "+f"(v[0]), "+f"(v[1])); }
-
 // Code i of a group's per-token code stream (i * B bits in, LSB first), as the
 // float 1 + u / 2^B: the code is moved to mantissa bits [23 - B, 23) and the
 // exponent of 1.0 is or-ed in.  run[] holds the stream re-aligned to bit 0.
@@ -105,84 +89,134 @@ __device__ __forceinline__ float code_float(const uint32_t* run) {
   return __uint_as_float((x & (((1u << B) - 1u) << (23 - B))) | 0x3F800000u);
 }
 
-template <int B, int N, int... I>
-__device__ __forceinline__ void group_accumulate(const uint32_t* run, const float* G, float2& acc, float2& gs,
-                                                 std::integer_sequence<int, I...>) {
-  // pairs (2i, 2i + 1): packed fp32x2 multiply-add of the codes with G, and the
-  // running sum of G for the offset term
+// sum_i f_i G[C + i] and sum_i G[C + i] over one group of N channels, in
+// packed fp32x2 pairs (a scalar step for an odd tail).
+template <int B, int C, int... I>
+__device__ __forceinline__ void group_pairs(const uint32_t* run, const float* G, float2& acc, float2& gs,
+                                            std::integer_sequence<int, I...>) {
   ((acc = __ffma2_rn(make_float2(code_float<B, 2 * I>(run), code_float<B, 2 * I + 1>(run)),
-                     make_float2(G[2 * I], G[2 * I + 1]), acc),
-    gs = __fadd2_rn(gs, make_float2(G[2 * I], G[2 * I + 1]))),
+                     make_float2(G[C + 2 * I], G[C + 2 * I + 1]), acc),
+    gs = __fadd2_rn(gs, make_float2(G[C + 2 * I], G[C + 2 * I + 1]))),
    ...);
 }
 
-// One quantization group's part of the scores of two tokens (rows of the two
-// 128-token tiles, TMEM columns tcol.. and tcol + 128..):
-//     scale * sum_j (u_j - 2^(B-1)) G_j   over the group's N channels.
-// Row 0's codes start at bit slot * N * B of the code block at `codes`, row 1's
-// at the same bit of the block `row1` bytes further.  Uses f_j = 1 + u_j / 2^B:
-//     sum (u - off) G = 2^B sum f G - (2^B + off) sum G.
-template <int N, int B>
-__device__ __forceinline__ float2 group_score2(uint32_t tcol, const uint8_t* codes, uint32_t row1, int slot,
-                                               float scale0, float scale1) {
-  static_assert(N % 2 == 0 && N >= 2 && N <= 32, "group width");
-  float G0[N], G1[N];
-#pragma unroll
-  for (int c = 0; c + 8 <= N; c += 8) {
-    tmem_ld8_nw(tcol + c, G0 + c);
-    tmem_ld8_nw(tcol + 128 + c, G1 + c);
-  }
-  if constexpr (N % 8 >= 4) {
-    tmem_ld4_nw(tcol + (N / 8) * 8, G0 + (N / 8) * 8);
-    tmem_ld4_nw(tcol + 128 + (N / 8) * 8, G1 + (N / 8) * 8);
-  }
-  if constexpr (N % 4 >= 2) {
-    tmem_ld2_nw(tcol + (N / 4) * 4, G0 + (N / 4) * 4);
-    tmem_ld2_nw(tcol + 128 + (N / 4) * 4, G1 + (N / 4) * 4);
-  }
+// One quantization group's part of a token's score: scale * sum_i (u_i - 2^(B-1)) G[C + i].
+// With f = 1 + u / 2^B:  sum (u - off) G = 2^B sum f G - (2^B + off) sum G.
+// `w` points at the group's code stream for this token (bit offset `sh` into w[0]).
+template <int N, int B, int C>
+__device__ __forceinline__ float group_dot(const uint32_t* w, uint32_t sh, float scale, const float* G) {
   constexpr int NR = (N * B + 31) / 32;
-  const uint32_t bit0 = (uint32_t)slot * (uint32_t)(N * B);
-  const uint32_t* w0 = reinterpret_cast<const uint32_t*>(codes) + (bit0 >> 5);
-  const uint32_t* w1 = reinterpret_cast<const uint32_t*>(codes + row1) + (bit0 >> 5);
-  const uint32_t sh = bit0 & 31u;
-  uint32_t raw0[NR + 1], raw1[NR + 1], run0[NR], run1[NR];
+  uint32_t run[NR];
 #pragma unroll
-  for (int k = 0; k <= NR; ++k) {
-    raw0[k] = w0[k];
-    raw1[k] = w1[k];
+  for (int k = 0; k < NR; ++k) run[k] = __funnelshift_r(w[k], w[k + 1], sh);
+  float2 acc = make_float2(0.f, 0.f), gs = acc;
+  group_pairs<B, C>(run, G, acc, gs, std::make_integer_sequence<int, N / 2>{});
+  float a = acc.x + acc.y, g = gs.x + gs.y;
+  if constexpr (N % 2) {
+    const float gl = G[C + N - 1];
+    a = fmaf(code_float<B, N - 1>(run), gl, a);
+    g += gl;
   }
-#pragma unroll
-  for (int k = 0; k < NR; ++k) {
-    run0[k] = __funnelshift_r(raw0[k], raw0[k + 1], sh);
-    run1[k] = __funnelshift_r(raw1[k], raw1[k + 1], sh);
-  }
-  tc::tmem_ld_wait();
-#pragma unroll
-  for (int c = 0; c < N; c += 2) {
-    reg_fence2(G0 + c);
-    reg_fence2(G1 + c);
-  }
-  float2 acc0 = make_float2(0.f, 0.f), gs0 = acc0, acc1 = acc0, gs1 = acc0;
-  group_accumulate<B, N>(run0, G0, acc0, gs0, std::make_integer_sequence<int, N / 2>{});
-  group_accumulate<B, N>(run1, G1, acc1, gs1, std::make_integer_sequence<int, N / 2>{});
   constexpr float kf = (float)(1 << B), kg = (float)((1 << B) + (1 << (B - 1)));
-  return make_float2(scale0 * ((acc0.x + acc0.y) * kf - (gs0.x + gs0.y) * kg),
-                     scale1 * ((acc1.x + acc1.y) * kf - (gs1.x + gs1.y) * kg));
+  return scale * (a * kf - g * kg);
 }
 
-// Group kinds: (N / 2 - 1) + 16 * (B - 3) for even N in [2, 32], B in {3, 4}.
-__host__ __device__ __forceinline__ int group_kind(int n, int bits) { return (n / 2 - 1) + 16 * (bits - 3); }
+// TMEM -> registers: columns [C, R) of this warp's lane quarter, no wait.
+template <int C, int R>
+__device__ __forceinline__ void tmem_cols(uint32_t taddr, float* G) {
+  if constexpr (C + 16 <= R) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+        : "=f"(G[C]), "=f"(G[C + 1]), "=f"(G[C + 2]), "=f"(G[C + 3]), "=f"(G[C + 4]), "=f"(G[C + 5]),
+          "=f"(G[C + 6]), "=f"(G[C + 7]), "=f"(G[C + 8]), "=f"(G[C + 9]), "=f"(G[C + 10]), "=f"(G[C + 11]),
+          "=f"(G[C + 12]), "=f"(G[C + 13]), "=f"(G[C + 14]), "=f"(G[C + 15])
+        : "r"(taddr + C));
+    tmem_cols<C + 16, R>(taddr, G);
+  } else if constexpr (C + 8 <= R) {
+    asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+                 : "=f"(G[C]), "=f"(G[C + 1]), "=f"(G[C + 2]), "=f"(G[C + 3]), "=f"(G[C + 4]), "=f"(G[C + 5]),
+                   "=f"(G[C + 6]), "=f"(G[C + 7])
+                 : "r"(taddr + C));
+    tmem_cols<C + 8, R>(taddr, G);
+  } else if constexpr (C + 4 <= R) {
+    asm volatile("tcgen05.ld.sync.aligned.32x32b.x4.b32 {%0,%1,%2,%3}, [%4];"
+                 : "=f"(G[C]), "=f"(G[C + 1]), "=f"(G[C + 2]), "=f"(G[C + 3])
+                 : "r"(taddr + C));
+    tmem_cols<C + 4, R>(taddr, G);
+  } else if constexpr (C + 2 <= R) {
+    asm volatile("tcgen05.ld.sync.aligned.32x32b.x2.b32 {%0,%1}, [%2];" : "=f"(G[C]), "=f"(G[C + 1]) : "r"(taddr + C));
+    tmem_cols<C + 2, R>(taddr, G);
+  } else if constexpr (C < R) {
+    asm volatile("tcgen05.ld.sync.aligned.32x32b.x1.b32 {%0}, [%1];" : "=f"(G[C]) : "r"(taddr + C));
+  }
+}
 
-__device__ __forceinline__ float2 group_score2_any(int kind, uint32_t tcol, const uint8_t* codes, uint32_t row1,
-                                                   int slot, float scale0, float scale1) {
-  switch (kind) {
-#define STARKV_GS(n)                                                                     \
-  case (n) / 2 - 1: return group_score2<(n), 3>(tcol, codes, row1, slot, scale0, scale1); \
-  case 16 + (n) / 2 - 1: return group_score2<(n), 4>(tcol, codes, row1, slot, scale0, scale1);
-    STARKV_GS(2) STARKV_GS(4) STARKV_GS(6) STARKV_GS(8) STARKV_GS(10) STARKV_GS(12) STARKV_GS(14) STARKV_GS(16)
-    STARKV_GS(18) STARKV_GS(20) STARKV_GS(22) STARKV_GS(24) STARKV_GS(26) STARKV_GS(28) STARKV_GS(30) STARKV_GS(32)
-#undef STARKV_GS
-    default: return make_float2(0.f, 0.f);
+// Makes the registers look rewritten here (emits nothing), so that no use of a
+// TMEM load's destination is scheduled above the preceding wait.
+template <int R>
+__device__ __forceinline__ void reg_fence(float* G) {
+#pragma unroll
+  for (int c = 0; c < R; ++c) asm volatile("" : "+f"(G[c]));
+}
+
+// Groups of a segment of S channels: 32 from the segment's start, the last shorter.
+__host__ __device__ constexpr int seg_groups(int S) { return (S + 31) / 32; }
+__host__ __device__ constexpr int seg_width(int S, int g) { return (g + 1) * 32 <= S ? 32 : S - g * 32; }
+
+template <int S, int B, int C0, int G0, int g = 0>
+__device__ __forceinline__ float segment_dot(const uint8_t* blk, const ScoreHead& hd, int slot, const float* G) {
+  if constexpr (g >= seg_groups(S)) {
+    return 0.f;
+  } else {
+    constexpr int N = seg_width(S, g);
+    const uint32_t bit0 = (uint32_t)slot * (uint32_t)(N * B);
+    const uint32_t* w = reinterpret_cast<const uint32_t*>(blk + hd.code_off[G0 + g]) + (bit0 >> 5);
+    const float scale = __half2float(reinterpret_cast<const __half*>(blk)[(G0 + g) * kPage + slot]);
+    return group_dot<N, B, C0 + g * 32>(w, bit0 & 31u, scale, G) +
+           segment_dot<S, B, C0, G0, g + 1>(blk, hd, slot, G);
+  }
+}
+
+// The score of one token for one head whose key latent has NHI 4-bit channels
+// then NLO 3-bit channels: all R = NHI + NLO G columns come out of TMEM with
+// one wait, the code groups are read from the page in shared memory.
+template <int NHI, int NLO>
+__device__ __forceinline__ float head_score(uint32_t taddr, const uint8_t* blk, const ScoreHead& hd, int slot) {
+  constexpr int R = NHI + NLO;
+  float G[R];
+  tmem_cols<0, R>(taddr, G);
+  tc::tmem_ld_wait();
+  reg_fence<R>(G);
+  return segment_dot<NHI, 4, 0, 0>(blk, hd, slot, G) +
+         segment_dot<NLO, 3, NHI, seg_groups(NHI)>(blk, hd, slot, G);
+}
+
+// Compiled head shapes (hi channels, lo channels): 25 % and 20 % of ranks
+// 16..64 at 4 bits, the rest at 3 bits, and uniform 4-bit latents.
+#define STARKV_HEAD_SHAPES(X)                                                                          \
+  X(0, 4, 12) X(1, 6, 18) X(2, 8, 24) X(3, 10, 30) X(4, 12, 36) X(5, 14, 42) X(6, 16, 48)             \
+  X(7, 5, 19) X(8, 7, 25) X(9, 8, 32) X(10, 10, 38) X(11, 12, 44) X(12, 13, 51)                       \
+  X(13, 16, 0) X(14, 24, 0) X(15, 32, 0) X(16, 40, 0) X(17, 48, 0) X(18, 56, 0) X(19, 64, 0) X(20, 8, 0)
+constexpr int kHeadShapes = 21;
+
+__host__ __device__ constexpr int shape_hi(int k) {
+#define STARKV_HI(i, h, l) k == i ? h:
+  return STARKV_HEAD_SHAPES(STARKV_HI) - 1;
+#undef STARKV_HI
+}
+__host__ __device__ constexpr int shape_lo(int k) {
+#define STARKV_LO(i, h, l) k == i ? l:
+  return STARKV_HEAD_SHAPES(STARKV_LO) - 1;
+#undef STARKV_LO
+}
+
+__device__ __forceinline__ float head_score_any(uint32_t taddr, const uint8_t* blk, const ScoreHead& hd, int slot) {
+  switch (hd.kind) {
+#define STARKV_CASE(i, h, l) \
+  case i: return head_score<h, l>(taddr, blk, hd, slot);
+    STARKV_HEAD_SHAPES(STARKV_CASE)
+#undef STARKV_CASE
+    default: return 0.f;
   }
 }
 
@@ -198,12 +232,8 @@ __device__ __forceinline__ int warp_sum(int x) {
   return r;
 }
 
-// Barrier among the 16 epilogue warps only (id 1; id 0 is __syncthreads).
-__device__ __forceinline__ void epilogue_sync() { asm volatile("bar.sync 1, %0;" ::"n"(32 * kEpiWarps) : "memory"); }
-
-constexpr int kMaxGroups = 4;
-constexpr int kMaxEnts = 512;      // entries of all items, resident in shared memory
 constexpr int kMaxItemHeads = 8;
+constexpr int kMaxHeads = 64;
 
 
 __global__ void __launch_bounds__(kScoreThreads, 1) k_scores_tc(ScoreArgs a) {
@@ -213,8 +243,7 @@ __global__ void __launch_bounds__(kScoreThreads, 1) k_scores_tc(ScoreArgs a) {
   __shared__ uint32_t tmem_base;
   __shared__ volatile int abort_flag;
   __shared__ ScoreItem items_s[64];
-  __shared__ ScoreEntry ent_s[kMaxEnts];
-  __shared__ float sc_s[2][kMaxItemHeads][kSuper];   // per-item scores, summed over the entry parts
+  __shared__ ScoreHead heads_s[kMaxHeads];
   uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   uint8_t* E_s = smem;                                   // 2 x 32 KB
   uint8_t* W_s = E_s + 2 * kETileBytes;                  // WS x w_stage
@@ -228,22 +257,21 @@ __global__ void __launch_bounds__(kScoreThreads, 1) k_scores_tc(ScoreArgs a) {
       tc::mbar_init(&w_full[s], 1);
       tc::mbar_init(&w_empty[s], 1);
       tc::mbar_init(&k_full[s], 1);
-      tc::mbar_init(&k_empty[s], kEpiWarps);
+      tc::mbar_init(&k_empty[s], kEpiWarps / 2);
     }
     for (int s = 0; s < 2; ++s) {
       tc::mbar_init(&e_full[s], 1);
       tc::mbar_init(&e_empty[s], 1);
       tc::mbar_init(&acc_full[s], 1);
-      tc::mbar_init(&acc_free[s], kEpiWarps);
+      tc::mbar_init(&acc_free[s], kEpiWarps / 2);
     }
     tc::mbar_init(&fin, 1);
     abort_flag = 0;
     tc::fence_mbar_init();
   }
-  // item and entry tables in shared memory; score accumulators zeroed
+  // item and head tables in shared memory
   for (int it = threadIdx.x; it < a.n_items; it += blockDim.x) items_s[it] = a.items[it];
-  for (int x = threadIdx.x; x < a.n_ents; x += blockDim.x) ent_s[x] = a.ents[x];
-  for (int x = threadIdx.x; x < 2 * kMaxItemHeads * kSuper; x += blockDim.x) (&sc_s[0][0][0])[x] = 0.f;
+  for (int h = threadIdx.x; h < a.H; h += blockDim.x) heads_s[h] = a.heads[h];
   if (warp == 1) tc::tmem_alloc(&tmem_base, 512);
   tc::tc_fence_before();
   __syncthreads();
@@ -376,94 +404,63 @@ __global__ void __launch_bounds__(kScoreThreads, 1) k_scores_tc(ScoreArgs a) {
     }
   } else {
     // ------------------------------------------------------------ epilogue
-    // 16 warps.  Warp e reads TMEM lane quarter q = warp % 4: tokens q * 32 +
-    // lane of both 128-token tiles, and scores part e / 4 of each item's
-    // (head, group) entries; the parts meet in sc_s.  After a barrier of the
-    // epilogue warps the softmax statistics are taken per (head, 32 tokens).
+    // Set `set` takes the items i with i % 2 == set (accumulator stage set);
+    // warp (tile, q) scores tokens tile * 128 + q * 32 + lane of the
+    // super-tile, which are exactly one 32-token softmax group.
     const int e = warp - 3;              // 0..15
-    const int q = warp & 3;
-    const int part = e >> 2;
-    const int tau0 = q * 32 + lane;      // tile-0 token; tile 1 holds tau0 + 128
-    const int pg0 = tau0 >> 4, slot = tau0 & 15;
+    const int set = e >> 3, tile = (e >> 2) & 1;
+    const int q = warp & 3;              // TMEM lane quarter of this warp
+    const int tau = tile * 128 + q * 32 + lane;
+    const int pg = tau >> 4, slot = tau & 15;
+    const int grp32 = tile * 4 + q;      // 32-token group inside the super-tile
     int i = 0;
-    // every epilogue warp runs the same loop (named barrier below); after an
-    // abort the waits fail fast and the work is skipped
     for (long long u = u0; u < u1; ++u) {
       const int b = (int)(u / a.n_st), st = (int)(u % a.n_st);
       const int t0 = st * kSuper;
       const int len = min(a.seq_lens[b], a.max_pages * kPage);
       if (t0 >= len) continue;
+      const int t = t0 + tau;
+      const bool valid = t < len;
       for (int it = 0; it < a.n_items; ++it, ++i) {
+        if ((i & 1) != set) continue;
         const ScoreItem& item = items_s[it];
         const int ks = i % a.KS;
-        const bool ok1 = tc::mbar_wait_ab(&k_full[ks], ((uint32_t)(i / a.KS)) & 1u, a.status, &abort_flag);
-        const bool ok = ok1 && tc::mbar_wait_ab(&acc_full[i & 1], ((uint32_t)(i >> 1)) & 1u, a.status, &abort_flag);
+        const bool ok = tc::mbar_wait_ab(&k_full[ks], ((uint32_t)(i / a.KS)) & 1u, a.status, &abort_flag) &&
+                        tc::mbar_wait_ab(&acc_full[set], ((uint32_t)(i >> 1)) & 1u, a.status, &abort_flag);
         tc::tc_fence_after();
-        float* sc = &sc_s[i & 1][0][0];
         if (ok) {
-          const uint8_t* page0 = K_s + (size_t)ks * a.k_stage + (size_t)pg0 * item.key_bytes;
-          const uint32_t row1 = 8u * (uint32_t)item.key_bytes;   // tile 1's page is 8 pages on
-          const uint32_t tcol = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)((i & 1) * 256);
-          int hcur = -1;
-          float s0 = 0.f, s1 = 0.f;
-          const int x1 = item.ent0 + item.part[part + 1];
-          for (int x = item.ent0 + item.part[part]; x < x1; ++x) {
-            const ScoreEntry en = ent_s[x];
-            const int hh = en.y >> 8;
-            if (hh != hcur) {
-              if (hcur >= 0) {
-                atomicAdd(&sc[hcur * kSuper + tau0], s0);
-                atomicAdd(&sc[hcur * kSuper + tau0 + 128], s1);
-              }
-              hcur = hh;
-              s0 = s1 = 0.f;
+          const uint8_t* page = K_s + (size_t)ks * a.k_stage + (size_t)pg * item.key_bytes;
+          const uint32_t trow = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(set * 256 + tile * 128);
+          for (int hh = 0; hh < item.nh; ++hh) {
+            const ScoreHead& hd = heads_s[item.h0 + hh];
+            const float sv = head_score_any(trow + (uint32_t)hd.gcol, page + hd.blk_rel, hd, slot);
+            const size_t row = (size_t)b * a.H + item.h0 + hh;
+            if (a.S_dbg) {
+              if (valid) a.S_dbg[row * a.P_ld + t] = sv;
+              continue;
             }
-            const __half* scl = reinterpret_cast<const __half*>(page0 + en.w);
-            const float2 r = group_score2_any(en.y & 255, tcol + (uint32_t)en.x, page0 + en.z, row1, slot,
-                                              __half2float(scl[slot]), __half2float(scl[slot + row1 / 2]));
-            s0 += r.x;
-            s1 += r.y;
-          }
-          if (hcur >= 0) {
-            atomicAdd(&sc[hcur * kSuper + tau0], s0);
-            atomicAdd(&sc[hcur * kSuper + tau0 + 128], s1);
+            // softmax statistics of the 32-token group: m = max s, P = exp2(s - m)
+            // rounded to fp16, l = sum of the fp16 P (exact: each P is a multiple
+            // of 2^-24, summed as integers)
+            const float m = warp_max(valid ? sv : -FLT_MAX);
+            int pi = 0;
+            if (valid) {
+              const __half pb = __float2half_rn(exp2f(sv - m));
+              a.P[row * a.P_ld + t] = pb;
+              pi = __float2int_rn(__half2float(pb) * 16777216.f);
+            }
+            const int ps = warp_sum(pi);
+            if (lane == 0) {
+              a.m_st[row * a.n_g + (t0 >> 5) + grp32] = m;
+              a.l_st[row * a.n_g + (t0 >> 5) + grp32] = (float)ps * (1.f / 16777216.f);
+            }
           }
         }
         tc::tc_fence_before();
         __syncwarp();
         if (lane == 0) {
-          tc::mbar_arrive(&acc_free[i & 1]);
+          tc::mbar_arrive(&acc_free[set]);
           tc::mbar_arrive(&k_empty[ks]);
-        }
-        epilogue_sync();
-        // softmax statistics per (head, 32-token group): m = max s, P =
-        // exp2(s - m) rounded to fp16, l = sum of the fp16 P (exact: each P is
-        // a multiple of 2^-24, summed as integers)
-        for (int task = e; task < item.nh * 8; task += kEpiWarps) {
-          const int hh = task >> 3, kq = task & 7;
-          const int tau = kq * 32 + lane;
-          float* cell = &sc[hh * kSuper + tau];
-          const float sv = *cell;
-          *cell = 0.f;
-          const int t = t0 + tau;
-          const bool valid = t < len;
-          const size_t row = (size_t)b * a.H + item.h0 + hh;
-          if (a.S_dbg) {
-            if (valid) a.S_dbg[row * a.P_ld + t] = sv;
-            continue;
-          }
-          const float m = warp_max(valid ? sv : -FLT_MAX);
-          int pi = 0;
-          if (valid) {
-            const __half pb = __float2half_rn(exp2f(sv - m));
-            a.P[row * a.P_ld + t] = pb;
-            pi = __float2int_rn(__half2float(pb) * 16777216.f);
-          }
-          const int ps = warp_sum(pi);
-          if (lane == 0) {
-            a.m_st[row * a.n_g + (t0 >> 5) + kq] = m;
-            a.l_st[row * a.n_g + (t0 >> 5) + kq] = (float)ps * (1.f / 16777216.f);
-          }
         }
       }
     }
@@ -560,18 +557,31 @@ bool plan_scores_tc(starkv_layer* L) {
   const LayerView& v = L->view;
   const starkv_layer_config& c = L->cfg;
   if (c.dtype != STARKV_BF16 || c.plain || !c.rope || c.head_dim != 128 || !v.quantized) return false;
-  if (c.n_heads > 64) return false;
-  // the epilogue has compiled dot products for even group widths up to 32 at
-  // 3 or 4 bits, and at most kMaxGroups groups per key latent
+  if (c.n_heads > kMaxHeads) return false;
+  // Every key latent must have one of the compiled head shapes: NHI 4-bit
+  // channels then NLO 3-bit channels, each segment cut into groups of 32 from
+  // its start.
+  std::vector<int> kv_kind(v.Hkv, -1);
   for (int g = 0; g < v.Hkv; ++g) {
-    if (L->lat[g].n_groups > kMaxGroups) return false;
-    for (int k = 0; k < L->lat[g].n_groups; ++k) {
-      const GroupDesc& gd = L->grp[L->lat[g].group0 + k];
-      if (gd.n % 2 || gd.n > 32 || (gd.bits != 3 && gd.bits != 4)) return false;
+    const LatentDesc& ld = L->lat[g];
+    if (ld.n_groups > 4) return false;
+    for (int k = 0; k < kHeadShapes && kv_kind[g] < 0; ++k) {
+      const int nhi = shape_hi(k), nlo = shape_lo(k);
+      if (nhi + nlo != ld.width) continue;
+      std::vector<std::pair<int, int>> want;   // (width, bits) of each group
+      for (int x = 0; x < nhi; x += 32) want.push_back({std::min(32, nhi - x), 4});
+      for (int x = 0; x < nlo; x += 32) want.push_back({std::min(32, nlo - x), 3});
+      bool match = (int)want.size() == ld.n_groups;
+      for (int j = 0; match && j < ld.n_groups; ++j) {
+        const GroupDesc& gd = L->grp[ld.group0 + j];
+        match = gd.n == want[j].first && gd.bits == want[j].second;
+      }
+      if (match) kv_kind[g] = k;
     }
+    if (kv_kind[g] < 0) return false;
   }
   L->items.clear();
-  L->score_ents.clear();
+  L->score_heads.assign(v.H, ScoreHead{});
   int w_off = 0, max_key = 0, max_w = 0;
   int h = 0;
   while (h < v.H) {
@@ -595,36 +605,18 @@ bool plan_scores_tc(starkv_layer* L) {
     it.key_bytes = L->lat[g1 + 1].block_off - it.key_off;
     max_key = std::max(max_key, it.key_bytes);
     max_w = std::max(max_w, it.npad * 256);
-    // (head, group) entries and their split into four parts of about equal
-    // work (a group costs about 3.3 instructions per channel plus a fixed part)
-    it.ent0 = (int)L->score_ents.size();
-    std::vector<double> cost;
     for (int hh = 0; hh < it.nh; ++hh) {
-      const LatentDesc& ld = L->lat[(it.h0 + hh) / v.group_q];
-      const int blk_rel = ld.block_off - it.key_off;
-      for (int k = 0; k < ld.n_groups; ++k) {
-        const GroupDesc& gd = L->grp[ld.group0 + k];
-        L->score_ents.push_back(make_int4(it.hcol[hh] + gd.start, group_kind(gd.n, gd.bits) | (hh << 8),
-                                          blk_rel + gd.code_off, blk_rel + k * kPage * 2));
-        cost.push_back(3.3 * gd.n + 16.0);
-      }
+      const int g = (it.h0 + hh) / v.group_q;
+      const LatentDesc& ld = L->lat[g];
+      ScoreHead& hd = L->score_heads[it.h0 + hh];
+      hd.gcol = it.hcol[hh];
+      hd.kind = kv_kind[g];
+      hd.blk_rel = ld.block_off - it.key_off;
+      hd.n_groups = ld.n_groups;
+      for (int k = 0; k < ld.n_groups; ++k) hd.code_off[k] = L->grp[ld.group0 + k].code_off;
     }
-    const int ne = (int)cost.size();
-    double total = 0.0;
-    for (double c : cost) total += c;
-    it.part[0] = 0;
-    double run = 0.0;
-    int p = 1;
-    for (int x = 0; x < ne && p < 4; ++x) {
-      run += cost[x];
-      // close part p - 1 after entry x once it holds its share
-      while (p < 4 && run >= total * p / 4.0 - 0.5 * cost[x]) it.part[p++] = x + 1;
-    }
-    while (p < 4) it.part[p++] = ne;
-    it.part[4] = ne;
     L->items.push_back(it);
   }
-  if (L->score_ents.size() > (size_t)kMaxEnts) return false;
   L->w_stride = w_off;
   L->k_stage = (kSuper / kPage) * max_key + 16;
   L->k_stage = (L->k_stage + 1023) / 1024 * 1024;
@@ -690,8 +682,7 @@ cudaError_t launch_scores_tc(const starkv_layer* L, const uint8_t* pool, long lo
   a.w_stride = L->w_stride;
   a.items = L->d_items;
   a.n_items = (int)L->items.size();
-  a.ents = L->d_score_ents;
-  a.n_ents = (int)L->score_ents.size();
+  a.heads = L->d_score_heads;
   a.lat = L->d_lat;
   a.grp = L->d_grp;
   a.gq = v.group_q;

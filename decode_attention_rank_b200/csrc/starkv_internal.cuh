@@ -71,18 +71,17 @@ struct ScoreItem {
   int key_bytes;
   int hcol[8];        // G column of each head's first latent channel
   int hr[8];          // rank of each head
-  // The item's (head, quantization group) pairs, in order, are entries
-  // ent0 .. ent0 + part[4] - 1 of the entry table; the score epilogue splits
-  // them into four parts of about equal work, part p = [part[p], part[p + 1]).
-  int ent0;
-  int part[5];
 };
 
-// One (head, quantization group) pair of a score item: x = G column of the
-// group's first channel (item-relative), y = group kind | head-in-item << 8,
-// z = byte offset of the group's code block and w = byte offset of its scale
-// column, both relative to the item's key range inside one page.
-using ScoreEntry = int4;
+// The score epilogue's view of one query head: where its G columns and its
+// key latent's code groups are, and which compiled channel shape reads them.
+struct ScoreHead {
+  int gcol;          // G column of the head's first latent channel (item-relative)
+  int kind;          // index of the compiled (hi channels, lo channels) shape
+  int blk_rel;       // byte offset of the key latent block, relative to the item's key range in a page
+  int n_groups;
+  int code_off[4];   // byte offset of each group's code block inside the latent block
+};
 
 // Outputs of the tensor-core score kernel.
 struct ScoreOut {
@@ -125,8 +124,8 @@ struct starkv_layer {
   bool tc_scores = false;
   std::vector<starkv::ScoreItem> items;
   starkv::ScoreItem* d_items = nullptr;
-  std::vector<starkv::ScoreEntry> score_ents;
-  starkv::ScoreEntry* d_score_ents = nullptr;
+  std::vector<starkv::ScoreHead> score_heads;   // one per query head
+  starkv::ScoreHead* d_score_heads = nullptr;
   long long w_stride = 0;
   int w_stage = 0, k_stage = 0, WS = 0, KS = 0;
   int rope_tiles = 0;
