@@ -58,7 +58,8 @@ struct ScoreArgs {
   const GroupDesc* grp;
   int gq;                  // query heads per KV head
   int n_st;                // super-tiles per sequence
-  long long U;             // batch * n_st
+  int batch;
+  long long U;             // batch * n_st; unit u = (super-tile u / batch, sequence u % batch)
   __half* P;               // [B][H][P_ld]
   long long P_ld;
   float* m_st;             // [B][H][n_g] per 32-token group
@@ -163,32 +164,37 @@ __device__ __forceinline__ void reg_fence(float* G) {
 __host__ __device__ constexpr int seg_groups(int S) { return (S + 31) / 32; }
 __host__ __device__ constexpr int seg_width(int S, int g) { return (g + 1) * 32 <= S ? 32 : S - g * 32; }
 
+// Groups g, g + 1, ... of a segment of S channels at B bits whose first
+// channel is G column C0 of the head and whose first group is group G0 of the
+// latent.  Each group's G columns come out of TMEM on their own (at most 32
+// registers live), the code words are read while the TMEM load is in flight.
 template <int S, int B, int C0, int G0, int g = 0>
-__device__ __forceinline__ float segment_dot(const uint8_t* blk, const ScoreHead& hd, int slot, const float* G) {
+__device__ __forceinline__ float segment_dot(uint32_t taddr, const uint8_t* blk, const ScoreHead& hd, int slot) {
   if constexpr (g >= seg_groups(S)) {
     return 0.f;
   } else {
     constexpr int N = seg_width(S, g);
+    constexpr int NR = (N * B + 31) / 32;
+    float G[N];
+    tmem_cols<0, N>(taddr + (uint32_t)(C0 + g * 32), G);
     const uint32_t bit0 = (uint32_t)slot * (uint32_t)(N * B);
     const uint32_t* w = reinterpret_cast<const uint32_t*>(blk + hd.code_off[G0 + g]) + (bit0 >> 5);
+    uint32_t wr[NR + 1];
+#pragma unroll
+    for (int k = 0; k <= NR; ++k) wr[k] = w[k];
     const float scale = __half2float(reinterpret_cast<const __half*>(blk)[(G0 + g) * kPage + slot]);
-    return group_dot<N, B, C0 + g * 32>(w, bit0 & 31u, scale, G) +
-           segment_dot<S, B, C0, G0, g + 1>(blk, hd, slot, G);
+    tc::tmem_ld_wait();
+    reg_fence<N>(G);
+    return group_dot<N, B, 0>(wr, bit0 & 31u, scale, G) + segment_dot<S, B, C0, G0, g + 1>(taddr, blk, hd, slot);
   }
 }
 
 // The score of one token for one head whose key latent has NHI 4-bit channels
-// then NLO 3-bit channels: all R = NHI + NLO G columns come out of TMEM with
-// one wait, the code groups are read from the page in shared memory.
+// then NLO 3-bit channels (G columns 0 .. NHI + NLO - 1 from `taddr`).
 template <int NHI, int NLO>
 __device__ __forceinline__ float head_score(uint32_t taddr, const uint8_t* blk, const ScoreHead& hd, int slot) {
-  constexpr int R = NHI + NLO;
-  float G[R];
-  tmem_cols<0, R>(taddr, G);
-  tc::tmem_ld_wait();
-  reg_fence<R>(G);
-  return segment_dot<NHI, 4, 0, 0>(blk, hd, slot, G) +
-         segment_dot<NLO, 3, NHI, seg_groups(NHI)>(blk, hd, slot, G);
+  return segment_dot<NHI, 4, 0, 0>(taddr, blk, hd, slot) +
+         segment_dot<NLO, 3, NHI, seg_groups(NHI)>(taddr, blk, hd, slot);
 }
 
 // Compiled head shapes (hi channels, lo channels): 25 % and 20 % of ranks
@@ -238,8 +244,8 @@ constexpr int kMaxHeads = 64;
 
 __global__ void __launch_bounds__(kScoreThreads, 1) k_scores_tc(ScoreArgs a) {
   extern __shared__ uint8_t smem_raw[];
-  __shared__ __align__(8) uint64_t w_full[4], w_empty[4], k_full[4], k_empty[4], e_full[2], e_empty[2];
-  __shared__ __align__(8) uint64_t acc_full[2], acc_free[2], fin;
+  __shared__ __align__(8) uint64_t w_full[4], w_empty[4], k_full[4], k_empty[4], e_full, e_empty;
+  __shared__ __align__(8) uint64_t acc_full[4], acc_free[4], fin;
   __shared__ uint32_t tmem_base;
   __shared__ volatile int abort_flag;
   __shared__ ScoreItem items_s[64];
@@ -259,11 +265,11 @@ __global__ void __launch_bounds__(kScoreThreads, 1) k_scores_tc(ScoreArgs a) {
       tc::mbar_init(&k_full[s], 1);
       tc::mbar_init(&k_empty[s], kEpiWarps / 2);
     }
-    for (int s = 0; s < 2; ++s) {
-      tc::mbar_init(&e_full[s], 1);
-      tc::mbar_init(&e_empty[s], 1);
+    tc::mbar_init(&e_full, 1);
+    tc::mbar_init(&e_empty, 1);
+    for (int s = 0; s < 4; ++s) {
       tc::mbar_init(&acc_full[s], 1);
-      tc::mbar_init(&acc_free[s], kEpiWarps / 2);
+      tc::mbar_init(&acc_free[s], 4);
     }
     tc::mbar_init(&fin, 1);
     abort_flag = 0;
@@ -285,7 +291,7 @@ __global__ void __launch_bounds__(kScoreThreads, 1) k_scores_tc(ScoreArgs a) {
     int i = 0, nk = 0;                    // nk: issued stage fills (for the drain below)
     for (long long u = u0; u < u1; ++u) {
       if (__shfl_sync(0xffffffffu, abort_flag, 0)) break;
-      const int b = (int)(u / a.n_st), st = (int)(u % a.n_st);
+      const int st = (int)(u / a.batch), b = (int)(u % a.batch);
       const int t0 = st * kSuper;
       const int len = min(a.seq_lens[b], a.max_pages * kPage);
       if (t0 >= len) continue;
@@ -325,19 +331,22 @@ __global__ void __launch_bounds__(kScoreThreads, 1) k_scores_tc(ScoreArgs a) {
     // ------------------------------------------------------------ W'' and RoPE tiles
     // one thread; runs ahead of the key copies, bounded only by its own stages
     if (lane == 0) {
-      int i = 0, uc = 0, nw = 0, ne[2] = {0, 0};
+      // RoPE tiles are reloaded only when the super-tile position changes
+      int i = 0, nw = 0, ne = 0, cur_st = -1;
       for (long long u = u0; u < u1 && !abort_flag; ++u) {
-        const int b = (int)(u / a.n_st), st = (int)(u % a.n_st);
+        const int st = (int)(u / a.batch), b = (int)(u % a.batch);
         const int t0 = st * kSuper;
         const int len = min(a.seq_lens[b], a.max_pages * kPage);
         if (t0 >= len) continue;
         bool ok = true;
-        for (int k = 0; k < 2 && ok; ++k) {
-          ok = tc::mbar_wait_ab(&e_empty[k], ((uint32_t)uc & 1u) ^ 1u, a.status, &abort_flag);
+        if (st != cur_st) {
+          ok = tc::mbar_wait_ab(&e_empty, ((uint32_t)ne & 1u) ^ 1u, a.status, &abort_flag);
           if (!ok) break;
-          tc::mbar_expect_tx(&e_full[k], kETileBytes);
-          tc::bulk_g2s(E_s + k * kETileBytes, a.E + (size_t)(t0 / 128 + k) * kETileBytes, kETileBytes, &e_full[k]);
-          ++ne[k];
+          tc::mbar_expect_tx(&e_full, 2 * kETileBytes);
+          for (int k = 0; k < 2; ++k)
+            tc::bulk_g2s(E_s + k * kETileBytes, a.E + (size_t)(t0 / 128 + k) * kETileBytes, kETileBytes, &e_full);
+          ++ne;
+          cur_st = st;
         }
         for (int it = 0; it < a.n_items && ok; ++it, ++i) {
           const ScoreItem& item = items_s[it];
@@ -350,87 +359,97 @@ __global__ void __launch_bounds__(kScoreThreads, 1) k_scores_tc(ScoreArgs a) {
           ++nw;
         }
         if (!ok) break;
-        ++uc;
       }
       for (int j = max(0, nw - a.WS); j < nw; ++j)
         tc::mbar_wait(&w_full[j % a.WS], ((uint32_t)(j / a.WS)) & 1u, a.status);
-      for (int k = 0; k < 2; ++k)
-        if (ne[k] > 0) tc::mbar_wait(&e_full[k], (uint32_t)(ne[k] - 1) & 1u, a.status);
+      if (ne > 0) tc::mbar_wait(&e_full, (uint32_t)(ne - 1) & 1u, a.status);
     }
     __syncwarp();
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issue
     if (lane == 0) {
-      int i = 0, uc = 0;
+      int i = 0, nc = 0, cur_st = -1;
+      const uint64_t e0 = tc::sdesc_sw128(tc::smem_u32(E_s), 0, 1024), w0 = tc::sdesc_sw128(tc::smem_u32(W_s), 0, 1024);
+      const uint32_t e_lo0 = tc::desc_lo(e0), w_lo0 = tc::desc_lo(w0), sw_hi = tc::desc_hi(e0);
       for (long long u = u0; u < u1 && !abort_flag; ++u) {
-        const int b = (int)(u / a.n_st), st = (int)(u % a.n_st);
+        const int st = (int)(u / a.batch), b = (int)(u % a.batch);
         const int len = min(a.seq_lens[b], a.max_pages * kPage);
         if (st * kSuper >= len) continue;
+        if (st != cur_st) {
+          // release the previous RoPE tiles once every MMA issued so far has
+          // completed, then wait for this position's tiles
+          if (nc > 0) tc::mma_commit(&e_empty);
+          if (!tc::mbar_wait_ab(&e_full, (uint32_t)nc & 1u, a.status, &abort_flag)) { abort_flag = 1; break; }
+          ++nc;
+          cur_st = st;
+        }
         for (int it = 0; it < a.n_items && !abort_flag; ++it, ++i) {
           const int npad = items_s[it].npad;
           const int ws = i % a.WS;
           if (!tc::mbar_wait_ab(&w_full[ws], ((uint32_t)(i / a.WS)) & 1u, a.status, &abort_flag)) { abort_flag = 1; break; }
-          if (it == 0) {
-            if (!tc::mbar_wait_ab(&e_full[0], (uint32_t)uc & 1u, a.status, &abort_flag) ||
-                !tc::mbar_wait_ab(&e_full[1], (uint32_t)uc & 1u, a.status, &abort_flag)) { abort_flag = 1; break; }
-          }
-          if (!tc::mbar_wait_ab(&acc_free[i & 1], (((uint32_t)(i >> 1)) & 1u) ^ 1u, a.status, &abort_flag)) { abort_flag = 1; break; }
-          tc::tc_fence_after();
           const uint32_t idesc = tc::idesc_f16(128, npad, false, false, false);
-          const uint32_t wbase = tc::smem_u32(W_s + (size_t)ws * a.w_stage);
-          const uint32_t watom = (uint32_t)npad * 128u;
-#pragma unroll
-          for (int k = 0; k < 2; ++k) {
-            const uint32_t ebase = tc::smem_u32(E_s + k * kETileBytes);
-            const uint32_t d = tmem + (uint32_t)((i & 1) * 256 + k * 128);
-#pragma unroll
-            for (int kk = 0; kk < 8; ++kk) {
-              const uint32_t ea = ebase + (uint32_t)(kk >> 2) * 16384u + (uint32_t)(kk & 3) * 32u;
-              const uint32_t wa = wbase + (uint32_t)(kk >> 2) * watom + (uint32_t)(kk & 3) * 32u;
-              tc::mma_f16_ss(d, tc::sdesc_sw128(ea, 0, 1024), tc::sdesc_sw128(wa, 0, 1024), idesc, kk ? 1u : 0u);
+          // descriptors as (low, high) halves, stepped in 16-byte units on the low half
+          const uint32_t w_lo = w_lo0 + (uint32_t)ws * ((uint32_t)a.w_stage >> 4);
+          const uint32_t watom = (uint32_t)npad * 8u;   // one 64-column K atom of W'': npad rows x 128 B
+          bool ok = true;
+          for (int k = 0; k < 2 && ok; ++k) {
+            // job j = 2 i + k: tile k of item i, accumulator stage j % 4
+            const int j = 2 * i + k;
+            if (!tc::mbar_wait_ab(&acc_free[j & 3], (((uint32_t)(j >> 2)) & 1u) ^ 1u, a.status, &abort_flag)) {
+              ok = false;
+              break;
             }
+            tc::tc_fence_after();
+            const uint32_t e_lo = e_lo0 + (uint32_t)k * (kETileBytes >> 4);
+            const uint32_t d = tmem + (uint32_t)((j & 3) * 128);
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk)
+              tc::mma_f16_ss2(d, e_lo + (uint32_t)(kk >> 2) * 1024u + (uint32_t)(kk & 3) * 2u, sw_hi,
+                              w_lo + (uint32_t)(kk >> 2) * watom + (uint32_t)(kk & 3) * 2u, sw_hi, idesc, kk ? 1u : 0u);
+            tc::mma_commit(&acc_full[j & 3]);
+          }
+          if (!ok) {
+            abort_flag = 1;
+            break;
           }
           tc::mma_commit(&w_empty[ws]);
-          tc::mma_commit(&acc_full[i & 1]);
-          if (it == a.n_items - 1) {
-            tc::mma_commit(&e_empty[0]);
-            tc::mma_commit(&e_empty[1]);
-          }
         }
-        ++uc;
       }
       tc::mma_commit(&fin);
       tc::mbar_wait(&fin, 0, a.status);
     }
   } else {
     // ------------------------------------------------------------ epilogue
-    // Set `set` takes the items i with i % 2 == set (accumulator stage set);
-    // warp (tile, q) scores tokens tile * 128 + q * 32 + lane of the
-    // super-tile, which are exactly one 32-token softmax group.
+    // Job j = 2 i + tile (tile `tile` of item i) sits in accumulator stage
+    // j % 4; set `set` (4 warps, one per TMEM lane quarter) takes the jobs
+    // with j % 4 == set.  Warp q scores tokens tile * 128 + q * 32 + lane of
+    // the super-tile, which are exactly one 32-token softmax group.
     const int e = warp - 3;              // 0..15
-    const int set = e >> 3, tile = (e >> 2) & 1;
+    const int set = e >> 2;
+    const int tile = set & 1, ipar = set >> 1;
     const int q = warp & 3;              // TMEM lane quarter of this warp
     const int tau = tile * 128 + q * 32 + lane;
     const int pg = tau >> 4, slot = tau & 15;
     const int grp32 = tile * 4 + q;      // 32-token group inside the super-tile
     int i = 0;
     for (long long u = u0; u < u1; ++u) {
-      const int b = (int)(u / a.n_st), st = (int)(u % a.n_st);
+      const int st = (int)(u / a.batch), b = (int)(u % a.batch);
       const int t0 = st * kSuper;
       const int len = min(a.seq_lens[b], a.max_pages * kPage);
       if (t0 >= len) continue;
       const int t = t0 + tau;
       const bool valid = t < len;
       for (int it = 0; it < a.n_items; ++it, ++i) {
-        if ((i & 1) != set) continue;
+        if ((i & 1) != ipar) continue;
         const ScoreItem& item = items_s[it];
         const int ks = i % a.KS;
+        const int j = 2 * i + tile;
         const bool ok = tc::mbar_wait_ab(&k_full[ks], ((uint32_t)(i / a.KS)) & 1u, a.status, &abort_flag) &&
-                        tc::mbar_wait_ab(&acc_full[set], ((uint32_t)(i >> 1)) & 1u, a.status, &abort_flag);
+                        tc::mbar_wait_ab(&acc_full[set], ((uint32_t)(j >> 2)) & 1u, a.status, &abort_flag);
         tc::tc_fence_after();
         if (ok) {
           const uint8_t* page = K_s + (size_t)ks * a.k_stage + (size_t)pg * item.key_bytes;
-          const uint32_t trow = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(set * 256 + tile * 128);
+          const uint32_t trow = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(set * 128);
           for (int hh = 0; hh < item.nh; ++hh) {
             const ScoreHead& hd = heads_s[item.h0 + hh];
             const float sv = head_score_any(trow + (uint32_t)hd.gcol, page + hd.blk_rel, hd, slot);
@@ -618,16 +637,24 @@ bool plan_scores_tc(starkv_layer* L) {
     L->items.push_back(it);
   }
   L->w_stride = w_off;
-  L->k_stage = (kSuper / kPage) * max_key + 16;
-  L->k_stage = (L->k_stage + 1023) / 1024 * 1024;
+  L->k_stage = (kSuper / kPage) * max_key + 16;   // + 16: code reads run one word past a block
+  L->k_stage = (L->k_stage + 127) / 128 * 128;
   L->w_stage = (max_w + 1023) / 1024 * 1024;
-  // dynamic shared memory next to ~21 KB of static tables and barriers
-  const size_t budget = 194 * 1024 - 2 * kETileBytes;
-  L->WS = 3;
-  L->KS = 3;
-  while (L->WS > 2 && (size_t)L->WS * L->w_stage + (size_t)L->KS * L->k_stage > budget) --L->WS;
-  while (L->KS > 2 && (size_t)L->WS * L->w_stage + (size_t)L->KS * L->k_stage > budget) --L->KS;
-  if ((size_t)L->WS * L->w_stage + (size_t)L->KS * L->k_stage > budget) return false;
+  // dynamic shared memory: what the opt-in limit leaves beside the static
+  // tables and barriers, less the alignment slack and the two RoPE tiles
+  cudaFuncAttributes fa;
+  if (cudaFuncGetAttributes(&fa, k_scores_tc) != cudaSuccess) return false;
+  const long long budget = 232448LL - (long long)fa.sharedSizeBytes - 1024 - 2LL * kETileBytes;
+  const int stages[5][2] = {{3, 4}, {3, 3}, {2, 4}, {2, 3}, {2, 2}};
+  L->WS = 0;
+  for (const auto& ws_ks : stages) {
+    if ((long long)ws_ks[0] * L->w_stage + (long long)ws_ks[1] * L->k_stage <= budget) {
+      L->WS = ws_ks[0];
+      L->KS = ws_ks[1];
+      break;
+    }
+  }
+  if (L->WS == 0) return false;
   const int mp = c.max_positions > 0 ? c.max_positions : 32768;
   L->rope_tiles = (mp + kSuper - 1) / kSuper * (kSuper / 128);
   return true;
@@ -687,6 +714,7 @@ cudaError_t launch_scores_tc(const starkv_layer* L, const uint8_t* pool, long lo
   a.grp = L->d_grp;
   a.gq = v.group_q;
   a.n_st = n_st;
+  a.batch = batch;
   a.U = (long long)batch * n_st;
   a.P = out->P;
   a.P_ld = out->P_ld;

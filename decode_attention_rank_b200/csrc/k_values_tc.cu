@@ -10,15 +10,18 @@
 // in), the stacked probabilities are B (N = heads, K-major), and Y^T for every
 // 128-channel block stays in TMEM for a whole run of super-tiles.
 //
-// P comes from the score kernel as exp2(s - m_g) per 32-token group; a CTA
-// rescales it by exp2(m_g - M) with M the maximum over the CTA's run,
-// so no accumulator ever needs rescaling.  The CTA writes one partial
-// (M, l, Y) per run of one sequence; a combine kernel merges the runs.
-//   warp 0      bulk copies of the value latent blocks of each tile's pages
-//   warp 1      tcgen05.mma issue, TMEM allocation
-//   warps 2-17  P staging (scaled, fp16), dequantization of the 4/3-bit codes
-//               into the A tiles (one thread per token and 32-channel group),
-//               and the TMEM epilogue of each run
+// P comes from the score kernel as exp2(s - m_g) per 32-token group; it is
+// rescaled by exp2(m_g - M) with M the maximum over the CTA's run of the
+// sequence, so no accumulator ever needs rescaling.  The CTA writes one
+// partial (M, l, Y) per run of one sequence; a combine kernel merges the runs.
+//   warp 0      tcgen05.mma issue, TMEM allocation
+//   warps 1-4   P staging: rescaled fp16 P tiles (the B operand), M and l;
+//               warp s takes the 32-token group s of every tile
+//   warp 5      bulk copies of the pages' value blocks, 32 tokens at a time
+//   warps 6-21  workers: worker w dequantizes items w, w + 16, ... (an item =
+//               32 tokens x 128 value channels, a lane per token) from the
+//               copied pages into A stage w, and reads Y^T out of TMEM at the
+//               end of each run
 #include <float.h>
 
 #include "tc_common.cuh"
@@ -27,9 +30,21 @@ namespace starkv {
 
 namespace {
 
-constexpr int kValWarps = 16;
-constexpr int kValThreads = 64 + 32 * kValWarps;   // producer, MMA, 16 staging/dequant/epilogue warps
-constexpr int kVSuper = 256;   // tokens per super-tile (matches the score kernel)
+constexpr int kValWorkers = 16;                          // dequantizing warps
+constexpr int kStagers = 4;                              // P staging warps, one per 32-token group of a tile
+constexpr int kValThreads = 32 * (2 + kStagers + kValWorkers);   // MMA, P staging, page copies, workers
+// A stages: item n sits in stage n % kAStages, and worker w takes the items
+// n = w (mod kValWorkers), so each stage has one writer and a worker is never
+// more than one barrier phase ahead of the stage it writes.
+constexpr int kAStages = kValWorkers;
+// Raw 32-token chunks (two pages' value blocks) in flight.  A worker's
+// consecutive items lie at most max(4, 16 / nblk) chunks apart; at least that
+// many raw stages keep a worker within one barrier phase of the raw stage it
+// reads.
+constexpr int kMaxRawStages = 16;
+constexpr int kVSuper = 256;     // tokens per super-tile (matches the score kernel)
+constexpr int kAStage = 8192;    // one A stage: 32 tokens x 128 value channels, fp16
+constexpr int kMaxRuns = 64;     // runs (sequences) per CTA
 
 struct ValArgs {
   const uint8_t* pool;
@@ -38,14 +53,17 @@ struct ValArgs {
   int max_pages;
   const int32_t* seq_lens;
   int vblk_off, vblk_bytes;     // value latent block inside a page
+  int raw_stage;                // bytes of one raw chunk stage (two value blocks, 16-byte aligned)
+  int n_raw;                    // raw chunk stages (2 .. kMaxRawStages)
   const GroupDesc* vgrp;        // value latent groups (all of 32 channels)
   int rv, H;
+  int lg_nblk;                  // log2 of the 128-channel blocks of the value latent
   const __half* P;              // [B][H][P_ld]
   long long P_ld;
   const float* m_st;            // [B][H][n_g]: maximum of each 32-token group
   int n_st;
   int n_g;
-  long long U;                  // batch * n_st
+  long long U;                  // batch * n_st; unit u = (sequence u / n_st, super-tile u % n_st)
   int slots;                    // partial slots per CTA
   float* Y;                     // [G][slots][H][rv]
   float* mseg;                  // [G][slots][H]
@@ -55,6 +73,19 @@ struct ValArgs {
 };
 
 __device__ __forceinline__ long long vunit_lo(int c, int G, long long U) { return (long long)c * U / G; }
+
+// The CTA's 128-token tiles, in order: units u0 .. u1 - 1, up to two tiles
+// each, those that start below the sequence length.  A run is a maximal
+// stretch of tiles of one sequence.  Built once per CTA in shared memory:
+// per tile (sequence, first token, length, run) and its eight page ids.
+constexpr int kMaxTiles = 256;
+
+// One lane's data of a worker item (value channels [128 cb, 128 cb + 128) of
+// one token): the four groups' code words and fp16 scales.
+struct VData {
+  uint32_t w[4][4];
+  uint32_t sc[4];
+};
 
 // Dequantization of 8 codes of one group into four fp16 pairs, in the chunk
 // order (c0,c2) (c1,c3) (c4,c6) (c5,c7): each 16-bit lane holds 1024 + u (an
@@ -89,300 +120,399 @@ __device__ __forceinline__ uint4 deq8_b3(uint32_t run, __half2 sub, __half2 s2) 
 
 __global__ void __launch_bounds__(kValThreads, 1) k_values_tc(ValArgs a) {
   extern __shared__ uint8_t smem_raw[];
-  __shared__ __align__(8) uint64_t raw_full[2], raw_empty[2], a_full[2], a_empty[2], p_full[2], p_empty[2];
+  __shared__ __align__(8) uint64_t a_full[kAStages], a_empty[kAStages], r_full[kMaxRawStages], r_empty[kMaxRawStages];
+  __shared__ __align__(8) uint64_t p_full[2], p_empty[2];
   __shared__ __align__(8) uint64_t seg_done, acc_free, fin;
   __shared__ uint32_t tmem_base;
   __shared__ volatile int abort_flag;
-  __shared__ float M_s[64], l_s[64];
-  __shared__ int2 vg_s[128];     // per 32-channel value group: code width, code block offset
+  __shared__ int4 vg_s[128];              // per value group: code width, code block offset, fp16x2 of 1024 + 2^(bits-1)
+  __shared__ int4 tile_s[kMaxTiles];      // per tile: sequence, first token, length, run
+  __shared__ int pid_s[kMaxTiles][8];     // per tile: page of each 16-token slot block
+  __shared__ int run_b[kMaxRuns];
+  __shared__ int n_tiles_s, n_runs_s;
+  __shared__ float l_stage[64];           // run sums of the staged P, per head
   uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
-  const int raw_stage = (8 * a.vblk_bytes + 1023) / 1024 * 1024;
-  uint8_t* R_s = smem;                              // 2 x raw tile (8 value blocks)
-  uint8_t* A_s = R_s + 2 * raw_stage;               // 2 x 32 KB A tiles
-  uint8_t* P_s = A_s + 2 * 32768;                   // 2 x (H x 128 fp16, K-major swizzled)
+  uint8_t* A_s = smem;                                   // kAStages x 8 KB A stages
+  uint8_t* P_s = A_s + kAStages * kAStage;               // 2 x (H x 128 fp16, K-major swizzled)
+  uint8_t* R_s = P_s + 2 * a.H * 256;                    // n_raw raw chunks
   const int p_stage = a.H * 256;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int G = gridDim.x, c = blockIdx.x;
-  const long long u0 = vunit_lo(c, G, a.U), u1 = vunit_lo(c + 1, G, a.U);
-  const int nblk = a.rv / 128;
+  const int G = gridDim.x, cta = blockIdx.x;
+  const long long u0 = vunit_lo(cta, G, a.U), u1 = vunit_lo(cta + 1, G, a.U);
+  const int lnb = a.lg_nblk;                             // 128-channel blocks: 1 << lnb
+  const int nblk = 1 << lnb;
+  const int lg_ipt = lnb + 2;                            // worker items per tile: 4 * nblk
+  const int b_first = (int)(u0 / a.n_st);
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < 2; ++s) {
-      tc::mbar_init(&raw_full[s], 1);
-      tc::mbar_init(&raw_empty[s], kValWarps);
-      tc::mbar_init(&a_full[s], kValWarps);
+    for (int s = 0; s < kAStages; ++s) {
+      tc::mbar_init(&a_full[s], 1);
       tc::mbar_init(&a_empty[s], 1);
-      tc::mbar_init(&p_full[s], kValWarps);
+    }
+    for (int s = 0; s < a.n_raw; ++s) {
+      tc::mbar_init(&r_full[s], 1);
+      tc::mbar_init(&r_empty[s], 1 << a.lg_nblk);   // the chunk's items, one per 128-channel block
+    }
+    for (int s = 0; s < 2; ++s) {
+      tc::mbar_init(&p_full[s], kStagers);
       tc::mbar_init(&p_empty[s], 1);
     }
     tc::mbar_init(&seg_done, 1);
-    tc::mbar_init(&acc_free, kValWarps);
+    tc::mbar_init(&acc_free, kValWorkers);
     tc::mbar_init(&fin, 1);
     abort_flag = 0;
+    for (int h = 0; h < 64; ++h) l_stage[h] = 0.f;
     tc::fence_mbar_init();
   }
-  for (int g = threadIdx.x; g < a.rv / 32; g += blockDim.x) vg_s[g] = make_int2(a.vgrp[g].bits, a.vgrp[g].code_off);
-  if (warp == 1) tc::tmem_alloc(&tmem_base, a.tmem_cols);
+  for (int g = threadIdx.x; g < a.rv / 32; g += blockDim.x) {
+    const int bits = a.vgrp[g].bits;
+    const float offm = 1024.f + (float)(1 << (bits - 1));
+    const __half2 sub = __floats2half2_rn(offm, offm);
+    vg_s[g] = make_int4(bits, a.vgrp[g].code_off, *reinterpret_cast<const int*>(&sub), 0);
+  }
+  if (warp == 0) {
+    // tile table: 32 units at a time, tiles placed by a warp prefix count
+    int nt = 0, nr = 0, last_b = -1;
+    for (long long ub = u0; ub < u1; ub += 32) {
+      const long long u = ub + lane;
+      int b = 0, st = 0, len = 0, ntl = 0;
+      if (u < u1) {
+        b = (int)(u / a.n_st);
+        st = (int)(u - (long long)b * a.n_st);
+        len = min(a.seq_lens[b], a.max_pages * kPage);
+        ntl = (st * kVSuper < len) + (st * kVSuper + 128 < len);
+      }
+      int pre = ntl;   // inclusive prefix sum of tile counts
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, pre, o);
+        if (lane >= o) pre += y;
+      }
+      // run index: a new run starts at each unit with tiles whose sequence differs from the previous such unit's
+      const unsigned has = __ballot_sync(0xffffffffu, ntl > 0);
+      const int prev_lane = 31 - __clz(has & ((1u << lane) - 1u));   // -1 when none
+      const int prev_b = __shfl_sync(0xffffffffu, b, prev_lane < 0 ? 0 : prev_lane);
+      const bool starts = ntl > 0 && (prev_lane < 0 ? b != last_b : b != prev_b);
+      const unsigned st_mask = __ballot_sync(0xffffffffu, starts);
+      const int run = nr + __popc(st_mask & ((2u << lane) - 1u)) - 1;
+      if (starts && run < kMaxRuns) run_b[run] = b;
+      for (int k = 0; k < ntl; ++k) {
+        const int T = nt + pre - ntl + k;
+        if (T < kMaxTiles) tile_s[T] = make_int4(b, st * kVSuper + k * 128, len, run);
+      }
+      nt += __shfl_sync(0xffffffffu, pre, 31);
+      nr += __popc(st_mask);
+      if (has) last_b = __shfl_sync(0xffffffffu, b, 31 - __clz(has));
+    }
+    if (lane == 0) {
+      n_tiles_s = min(nt, kMaxTiles);
+      n_runs_s = min(nr, kMaxRuns);
+    }
+  }
+  if (warp == 0) tc::tmem_alloc(&tmem_base, a.tmem_cols);
   tc::tc_fence_before();
   __syncthreads();
   tc::tc_fence_after();
   const uint32_t tmem = tmem_base;
-
-  // The work list: units u0..u1-1 -> tiles (two per unit) with tokens < len.
-  if (warp == 0) {
-    // warp-wide producer: every lane fetches one page id and issues that page's copy
-    int nt = 0;
-    for (long long u = u0; u < u1; ++u) {
-      if (__shfl_sync(0xffffffffu, abort_flag, 0)) break;
-      const int b = (int)(u / a.n_st), st = (int)(u % a.n_st);
-      const int len = min(a.seq_lens[b], a.max_pages * kPage);
-      bool stop = false;
-      for (int tile = 0; tile < 2; ++tile) {
-        const int t0 = st * kVSuper + tile * 128;
-        if (t0 >= len) break;
-        const int r = nt & 1;
-        const int npg = min(8, (len - t0 + kPage - 1) / kPage);
-        int page = 0;
-        if (lane < npg) {
-          page = a.pt[(size_t)b * a.max_pages + t0 / kPage + lane];
-          if (page < 0 || page >= a.n_pages) {
-            atomicOr(a.status, kBadPage);
-            page = 0;
-          }
-        }
-        bool ok = true;
-        if (lane == 0) {
-          ok = tc::mbar_wait_ab(&raw_empty[r], (((uint32_t)(nt >> 1)) & 1u) ^ 1u, a.status, &abort_flag);
-          if (ok) tc::mbar_expect_tx(&raw_full[r], (uint32_t)(npg * a.vblk_bytes));
-        }
-        ok = __shfl_sync(0xffffffffu, ok, 0);
-        if (!ok) {
-          stop = true;
-          break;
-        }
-        if (lane < npg)
-          tc::bulk_g2s(R_s + (size_t)r * raw_stage + (size_t)lane * a.vblk_bytes,
-                       a.pool + (size_t)page * a.page_bytes + a.vblk_off, (uint32_t)a.vblk_bytes, &raw_full[r]);
-        ++nt;
+  const int n_tiles = n_tiles_s, n_runs = n_runs_s;
+  // page ids of every tile (out-of-range entries set the status bit and read page 0)
+  for (int e = threadIdx.x; e < n_tiles * 8; e += blockDim.x) {
+    const int4 tl = tile_s[e >> 3];
+    const int t = tl.y + (e & 7) * kPage;
+    int page = -1;
+    if (t < tl.z) {
+      page = a.pt[(size_t)tl.x * a.max_pages + t / kPage];
+      if (page < 0 || page >= a.n_pages) {
+        atomicOr(a.status, kBadPage);
+        page = 0;
       }
-      if (stop) break;
     }
-    if (lane == 0)
-      for (int j = max(0, nt - 2); j < nt; ++j) tc::mbar_wait(&raw_full[j & 1], ((uint32_t)(j >> 1)) & 1u, a.status);
-    __syncwarp();
-  } else if (warp == 1) {
+    pid_s[e >> 3][e & 7] = page;
+  }
+  __syncthreads();
+
+  if (warp == 0) {
+    // ------------------------------------------------ MMA issue
+    // Item n of the CTA (tile n / ipt, item n % ipt = 4 cb + k) sits in A
+    // stage n % kAStages; its two K = 16 steps add block cb's Y^T.  The four
+    // items of a block are consecutive, so eight MMAs in a row accumulate into
+    // one TMEM block (an MMA that switches accumulators costs about twice as
+    // much as one that continues a chain).
     if (lane == 0) {
       const uint32_t idesc = tc::idesc_f16(128, a.H, false, true, false);
-      int nt = 0, na = 0, seg = 0;
-      int cur_b = -1;
-      bool first = true;
-      for (long long u = u0; u < u1 && !abort_flag; ++u) {
-        const int b = (int)(u / a.n_st), st = (int)(u % a.n_st);
-        const int len = min(a.seq_lens[b], a.max_pages * kPage);
-        if (st * kVSuper >= len) continue;
-        if (b != cur_b) {
-          if (cur_b >= 0) {
+      // descriptors as (low, high) halves; steps are 16-byte units on the low half
+      const uint64_t a0 = tc::sdesc_sw128(tc::smem_u32(A_s), 1024, 2048);   // A: MN-major, 64-channel atoms 1 KB apart
+      const uint64_t b0 = tc::sdesc_sw128(tc::smem_u32(P_s), 0, 1024);      // B: K-major, 64-token atoms of H rows
+      const uint32_t a_lo0 = tc::desc_lo(a0), a_hi = tc::desc_hi(a0);
+      const uint32_t b_lo0 = tc::desc_lo(b0), b_hi = tc::desc_hi(b0);
+      const uint32_t b_atom = (uint32_t)(a.H * 128) >> 4, p_step = (uint32_t)p_stage >> 4;
+      int n = 0, cur_run = -1;
+      bool first = false;
+      for (int T = 0; T < n_tiles && !abort_flag; ++T) {
+        const int run = tile_s[T].w;
+        if (run != cur_run) {
+          if (cur_run >= 0) {
             tc::mma_commit(&seg_done);
-            ++seg;
-          }
-          cur_b = b;
-          first = true;
-          if (!tc::mbar_wait_ab(&acc_free, (((uint32_t)seg) & 1u) ^ 1u, a.status, &abort_flag)) break;
-          tc::tc_fence_after();
-        }
-        for (int tile = 0; tile < 2 && !abort_flag; ++tile) {
-          const int t0 = st * kVSuper + tile * 128;
-          if (t0 >= len) break;
-          const int ps = nt & 1;
-          if (!tc::mbar_wait_ab(&p_full[ps], ((uint32_t)(nt >> 1)) & 1u, a.status, &abort_flag)) break;
-          tc::tc_fence_after();
-          const uint32_t pbase = tc::smem_u32(P_s + (size_t)ps * p_stage);
-          for (int cb = 0; cb < nblk; ++cb, ++na) {
-            const int as = na & 1;
-            if (!tc::mbar_wait_ab(&a_full[as], ((uint32_t)(na >> 1)) & 1u, a.status, &abort_flag)) break;
+            if (!tc::mbar_wait_ab(&acc_free, (uint32_t)cur_run & 1u, a.status, &abort_flag)) break;
             tc::tc_fence_after();
-            const uint32_t abase = tc::smem_u32(A_s + (size_t)as * 32768);
-            const uint32_t d = tmem + (uint32_t)(cb * a.H);
-#pragma unroll
-            for (int kk = 0; kk < 8; ++kk) {
-              // A: MN-major, 64-channel atoms 1024 B apart, 8-token groups 2048 B apart
-              const uint64_t ad = tc::sdesc_sw128(abase + (uint32_t)kk * 4096u, 1024, 2048);
-              // B: K-major, 64-token atoms of H rows
-              const uint64_t bd = tc::sdesc_sw128(pbase + (uint32_t)(kk >> 2) * (uint32_t)(a.H * 128) +
-                                                      (uint32_t)(kk & 3) * 32u,
-                                                  0, 1024);
-              tc::mma_f16_ss(d, ad, bd, idesc, (first && kk == 0) ? 0u : 1u);
-            }
-            tc::mma_commit(&a_empty[as]);
           }
-          tc::mma_commit(&p_empty[ps]);
-          first = false;
-          ++nt;
+          cur_run = run;
+          first = true;
         }
+        const int ps = T & 1;
+        if (!tc::mbar_wait_ab(&p_full[ps], ((uint32_t)(T >> 1)) & 1u, a.status, &abort_flag)) break;
+        tc::tc_fence_after();
+        const uint32_t b_lo = b_lo0 + (uint32_t)ps * p_step;
+        bool ok = true;
+        for (int cb = 0; cb < nblk && ok; ++cb) {
+          const uint32_t d = tmem + (uint32_t)(cb * a.H);
+#pragma unroll
+          for (int k = 0; k < 4; ++k, ++n) {
+            const int s = n % kAStages;
+            if (!tc::mbar_wait_ab(&a_full[s], ((uint32_t)(n / kAStages)) & 1u, a.status, &abort_flag)) {
+              ok = false;
+              break;
+            }
+            tc::tc_fence_after();
+            const uint32_t a_lo = a_lo0 + (uint32_t)s * (kAStage >> 4);
+            // tokens 32 k .. 32 k + 31: 16-token steps 2 k and 2 k + 1 of the P tile
+            tc::mma_f16_ss2(d, a_lo, a_hi, b_lo + (uint32_t)(k >> 1) * b_atom + (uint32_t)(k & 1) * 4u, b_hi, idesc,
+                            (first && k == 0) ? 0u : 1u);
+            tc::mma_f16_ss2(d, a_lo + (4096u >> 4), a_hi, b_lo + (uint32_t)(k >> 1) * b_atom + (uint32_t)(k & 1) * 4u + 2u,
+                            b_hi, idesc, 1u);
+            tc::mma_commit(&a_empty[s]);
+          }
+        }
+        if (!ok) break;
+        tc::mma_commit(&p_empty[ps]);
+        first = false;
       }
-      if (cur_b >= 0) tc::mma_commit(&seg_done);
+      if (cur_run >= 0) tc::mma_commit(&seg_done);
       tc::mma_commit(&fin);
       tc::mbar_wait(&fin, 0, a.status);
     }
-  } else {
-    // ------------------------------------------------ P staging, dequantization, epilogue
-    const int e = warp - 2;            // 0..15
-    const int tid = threadIdx.x - 64;  // 0..511
-    int nt = 0, na = 0, seg = 0, slot = -1;
-    int cur_b = -1;
-    const long long ub = u0 / a.n_st;
-    auto finish_run = [&]() {
-      // epilogue of a run: Y^T from TMEM (lanes = value channels), M and l
-      const bool ok = tc::mbar_wait_ab(&seg_done, ((uint32_t)seg) & 1u, a.status, &abort_flag);
-      tc::tc_fence_after();
-      const int q = warp & 3;
-      const size_t base = ((size_t)c * a.slots + slot) * a.H;
-      for (int cb = e >> 2; cb < nblk; cb += 4) {
-        for (int h0 = 0; h0 < a.H; h0 += 16) {
-          float v[16];
-          if (ok) {
-            tc::tmem_ld16_sync(tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(cb * a.H + h0), v);
-          } else {
-#pragma unroll
-            for (int i = 0; i < 16; ++i) v[i] = 0.f;
-          }
-          const int ch = cb * 128 + q * 32 + lane;     // A-tile position (channel order permuted per 8)
-#pragma unroll
-          for (int i = 0; i < 16; ++i) a.Y[(base + h0 + i) * a.rv + ch] = v[i];
+  } else if (warp <= kStagers) {
+    // ------------------------------------------------ P staging
+    // Stager warp s stages the 32-token group s of every tile, lane h for
+    // head h (and h + 32): P * exp2(m_g - M) rounded to fp16, with M the
+    // maximum over the run; l = sum of the staged values.
+    const int sw = warp - 1;
+    if (sw == 0)
+      for (int sl = 0; sl < a.slots; ++sl)
+        for (int h = lane; h < a.H; h += 32) {
+          a.mseg[((size_t)cta * a.slots + sl) * a.H + h] = -FLT_MAX;
+          a.lseg[((size_t)cta * a.slots + sl) * a.H + h] = 0.f;
         }
+    float Mh[2] = {-FLT_MAX, -FLT_MAX}, lh[2] = {0.f, 0.f};
+    int cur_run = -1, cur_b = -1;
+    auto flush = [&]() {
+      // the four stager warps add their partial sums, then warp 0 writes the run's (M, l)
+#pragma unroll
+      for (int hh = 0; hh < 2; ++hh)
+        if (lane + 32 * hh < a.H) atomicAdd(&l_stage[lane + 32 * hh], lh[hh]);
+      asm volatile("bar.sync 1, %0;" ::"n"(32 * kStagers) : "memory");
+      if (sw == 0) {
+        const size_t base = ((size_t)cta * a.slots + (cur_b - b_first)) * a.H;
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh) {
+          const int h = lane + 32 * hh;
+          if (h < a.H) {
+            a.mseg[base + h] = Mh[hh];
+            a.lseg[base + h] = l_stage[h];
+            l_stage[h] = 0.f;
+          }
+        }
+      }
+      asm volatile("bar.sync 1, %0;" ::"n"(32 * kStagers) : "memory");
+    };
+    for (int T = 0; T < n_tiles; ++T) {
+      const int4 tl = tile_s[T];   // sequence, first token, length, run
+      if (tl.w != cur_run) {
+        if (cur_run >= 0) flush();
+        cur_run = tl.w;
+        cur_b = tl.x;
+        // the run maximum over its tiles' 32-token groups
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh) {
+          const int h = lane + 32 * hh;
+          float m = -FLT_MAX;
+          if (h < a.H) {
+            const float* mr = a.m_st + ((size_t)tl.x * a.H + h) * a.n_g;
+            for (int T2 = T; T2 < n_tiles && tile_s[T2].w == tl.w; ++T2) {
+              const float4 g4 = *reinterpret_cast<const float4*>(mr + (tile_s[T2].y >> 5));
+              m = fmaxf(m, fmaxf(fmaxf(g4.x, g4.y), fmaxf(g4.z, g4.w)));
+            }
+          }
+          Mh[hh] = m;
+          lh[hh] = 0.f;
+        }
+      }
+      const int t0 = tl.y + 32 * sw;   // this warp's 32 tokens
+      // loads first, then the wait for the stage
+      uint4 raw[2][4];
+      float mg[2];
+#pragma unroll
+      for (int hh = 0; hh < 2; ++hh) {
+        const int h = lane + 32 * hh;
+        mg[hh] = 0.f;
+#pragma unroll
+        for (int c8 = 0; c8 < 4; ++c8) raw[hh][c8] = make_uint4(0, 0, 0, 0);
+        if (h < a.H && t0 < tl.z) {
+          const size_t row = (size_t)tl.x * a.H + h;
+          mg[hh] = a.m_st[row * a.n_g + (t0 >> 5)];
+#pragma unroll
+          for (int c8 = 0; c8 < 4; ++c8)
+            if (t0 + c8 * 8 < tl.z) raw[hh][c8] = *reinterpret_cast<const uint4*>(a.P + row * a.P_ld + t0 + c8 * 8);
+        }
+      }
+      const int ps = T & 1;
+      if (!tc::mbar_wait_ab(&p_empty[ps], (((uint32_t)(T >> 1)) & 1u) ^ 1u, a.status, &abort_flag)) break;
+      uint8_t* pt_s = P_s + (size_t)ps * p_stage;
+#pragma unroll
+      for (int hh = 0; hh < 2; ++hh) {
+        const int h = lane + 32 * hh;
+        if (h >= a.H) continue;
+        const float f = t0 < tl.z ? exp2f(mg[hh] - Mh[hh]) : 0.f;
+        float lsum = 0.f;
+#pragma unroll
+        for (int c8 = 0; c8 < 4; ++c8) {   // 8-token chunks
+          const int ch = sw * 4 + c8;
+          const int tp = t0 + c8 * 8;
+          __half* hv = reinterpret_cast<__half*>(&raw[hh][c8]);
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            const float p = (tp + i < tl.z) ? __half2float(hv[i]) * f : 0.f;
+            hv[i] = __float2half_rn(p);
+            lsum += __half2float(hv[i]);
+          }
+          *reinterpret_cast<uint4*>(pt_s + (ch >> 3) * (a.H * 128) + tc::sw128((uint32_t)h, (uint32_t)(ch & 7))) =
+              raw[hh][c8];
+        }
+        lh[hh] += lsum;
+      }
+      tc::fence_proxy_async();
+      __syncwarp();
+      if (lane == 0) tc::mbar_arrive(&p_full[ps]);
+    }
+    if (cur_run >= 0) flush();
+  } else if (warp == kStagers + 1) {
+
+    // ------------------------------------------------ page copies
+    // Chunk c = 4 T + k (tokens 32 k .. 32 k + 31 of tile T): the value blocks
+    // of its two pages into raw stage c % n_raw.
+    if (lane == 0) {
+      const int n_chunks = n_tiles * 4;
+      for (int c = 0; c < n_chunks; ++c) {
+        const int rs = c % a.n_raw;
+        if (!tc::mbar_wait_ab(&r_empty[rs], (((uint32_t)(c / a.n_raw)) & 1u) ^ 1u, a.status, &abort_flag)) break;
+        const int p0 = pid_s[c >> 2][2 * (c & 3)], p1 = pid_s[c >> 2][2 * (c & 3) + 1];
+        tc::mbar_expect_tx(&r_full[rs], (uint32_t)(((p0 >= 0) + (p1 >= 0)) * a.vblk_bytes));
+        uint8_t* dst = R_s + (size_t)rs * a.raw_stage;
+        if (p0 >= 0)
+          tc::bulk_g2s(dst, a.pool + (size_t)p0 * a.page_bytes + a.vblk_off, (uint32_t)a.vblk_bytes, &r_full[rs]);
+        if (p1 >= 0)
+          tc::bulk_g2s(dst + a.vblk_bytes, a.pool + (size_t)p1 * a.page_bytes + a.vblk_off, (uint32_t)a.vblk_bytes,
+                       &r_full[rs]);
+      }
+      // let copies in flight land before the CTA can exit
+      for (int c = max(0, n_chunks - a.n_raw); c < n_chunks; ++c)
+        tc::mbar_wait(&r_full[c % a.n_raw], ((uint32_t)(c / a.n_raw)) & 1u, a.status);
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------ workers: codes -> A stages, run epilogues
+    // Worker w takes the CTA's items w, w + 16, w + 32, ...; item n is item
+    // x = n % ipt = 4 cb + k of tile T = n / ipt: value channels
+    // [128 cb, 128 cb + 128) of tokens 32 k .. 32 k + 31, read from raw chunk
+    // 4 T + k and dequantized (a lane per token) into A stage n % kAStages.
+    const int w = warp - 2 - kStagers;
+    const int q = warp & 3, part = w >> 2;   // epilogue: TMEM lane quarter, column part
+    const int n_items = n_tiles << lg_ipt;
+    int epi_run = 0;
+    auto epilogue = [&](int r) {
+      // Y^T of run r from TMEM (lanes = value channels), 16 columns at a time
+      const bool ok = tc::mbar_wait_ab(&seg_done, (uint32_t)r & 1u, a.status, &abort_flag);
+      tc::tc_fence_after();
+      const size_t base = ((size_t)cta * a.slots + (run_b[r] - b_first)) * a.H;
+      for (int col = part * 16; col < nblk * a.H; col += 64) {
+        float v[16];
+        if (ok) {
+          tc::tmem_ld16_sync(tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)col, v);
+        } else {
+#pragma unroll
+          for (int i = 0; i < 16; ++i) v[i] = 0.f;
+        }
+        const int cb = col / a.H, h0 = col % a.H;
+        const int ch = cb * 128 + q * 32 + lane;     // A-tile position (channel order permuted per 8)
+#pragma unroll
+        for (int i = 0; i < 16; ++i) a.Y[(base + h0 + i) * a.rv + ch] = v[i];
       }
       tc::tc_fence_before();
       __syncwarp();
       if (lane == 0) tc::mbar_arrive(&acc_free);
-      if (tid < a.H) {
-        a.mseg[base + tid] = M_s[tid];
-        a.lseg[base + tid] = l_s[tid];
-      }
-      ++seg;
     };
-    // every slot of this CTA starts empty (a run with no valid token leaves l = 0)
-    if (tid < a.H)
-      for (int sl = 0; sl < a.slots; ++sl) {
-        a.mseg[((size_t)c * a.slots + sl) * a.H + tid] = -FLT_MAX;
-        a.lseg[((size_t)c * a.slots + sl) * a.H + tid] = 0.f;
-      }
-    // fixed per-thread roles inside a 128-token tile
-    const int tok = tid & 127;            // token of the tile
-    const int cq = tid >> 7;              // 32-channel group inside a 128-channel block
-    const uint32_t a_off = (uint32_t)(tok >> 3) * 2048u + (uint32_t)(cq >> 1) * 1024u + (uint32_t)(tok & 7) * 128u;
-    const uint32_t x7 = (uint32_t)(tok & 7);
-    const int ph = tid >> 4, pch = tid & 15;   // P staging: head, 8-token chunk
-    for (long long u = u0; u < u1; ++u) {
-      const int b = (int)(u / a.n_st), st = (int)(u % a.n_st);
-      const int len = min(a.seq_lens[b], a.max_pages * kPage);
-      if (st * kVSuper >= len) continue;
-      if (b != cur_b) {
-        if (cur_b >= 0) finish_run();
-        cur_b = b;
-        slot = (int)(b - ub);
-        // run maximum over the CTA's units of this sequence
-        asm volatile("bar.sync 1, 512;" ::: "memory");
-        if (tid < a.H) {
-          float m = -FLT_MAX;
-          for (long long uu = u; uu < u1 && uu / a.n_st == b; ++uu) {
-            const int s2 = (int)(uu % a.n_st);
-            if (s2 * kVSuper < len)
-              for (int g = 0; g < kVSuper / 32; ++g)
-                m = fmaxf(m, a.m_st[((size_t)b * a.H + tid) * a.n_g + s2 * (kVSuper / 32) + g]);
-          }
-          M_s[tid] = m;
-          l_s[tid] = 0.f;
-        }
-        asm volatile("bar.sync 1, 512;" ::: "memory");
-      }
-      for (int tile = 0; tile < 2; ++tile) {
-        const int t0 = st * kVSuper + tile * 128;
-        if (t0 >= len) break;
-        // ---- P^T tile: rows = heads, 128 tokens, K-major swizzled, scaled, fp16
-        const int ps = nt & 1;
-        tc::mbar_wait_ab(&p_empty[ps], (((uint32_t)(nt >> 1)) & 1u) ^ 1u, a.status, &abort_flag);
-        uint8_t* pt_s = P_s + (size_t)ps * p_stage;
-        if (ph < a.H) {
-          const int tp = t0 + pch * 8;
-          const float mg = a.m_st[((size_t)b * a.H + ph) * a.n_g + (tp >> 5)];
-          const float f = exp2f(mg - M_s[ph]);
-          uint4 raw = make_uint4(0, 0, 0, 0);
-          if (tp < len) raw = *reinterpret_cast<const uint4*>(a.P + ((size_t)b * a.H + ph) * a.P_ld + tp);
-          __half* hv = reinterpret_cast<__half*>(&raw);
-          float lsum = 0.f;
+    const uint32_t x7 = (uint32_t)(lane & 7);
+    const int slot = lane & 15;
+    for (int n = w; n < n_items; n += kValWorkers) {
+      const int T = n >> lg_ipt;
+      const int run = tile_s[T].w;
+      while (epi_run < run && epi_run < n_runs) epilogue(epi_run++);
+      const int x = n & ((1 << lg_ipt) - 1);
+      const int c = T * 4 + (x & 3);          // raw chunk
+      const int cb = x >> 2;
+      const int rs = c % a.n_raw, as = n % kAStages;
+      const bool valid = pid_s[T][2 * (c & 3) + (lane >> 4)] >= 0;
+      // A stage first: once item n - 16 is consumed, every chunk up to its
+      // chunk has landed; with at least max(4, 16 / nblk) raw stages the raw
+      // stage is then at most one phase from chunk c
+      const bool ok = tc::mbar_wait_ab(&a_empty[as], (((uint32_t)(n / kAStages)) & 1u) ^ 1u, a.status, &abort_flag) &&
+                      tc::mbar_wait_ab(&r_full[rs], ((uint32_t)(c / a.n_raw)) & 1u, a.status, &abort_flag);
+      if (ok) {
+        const uint8_t* blk = R_s + (size_t)rs * a.raw_stage + (size_t)(lane >> 4) * a.vblk_bytes;
+        uint8_t* st = A_s + (size_t)as * kAStage + (lane >> 3) * 2048 + (lane & 7) * 128;
 #pragma unroll
-          for (int i = 0; i < 8; ++i) {
-            const float p = (tp + i < len) ? __half2float(hv[i]) * f : 0.f;
-            hv[i] = __float2half_rn(p);
-            lsum += __half2float(hv[i]);
-          }
-          atomicAdd(&l_s[ph], lsum);
-          *reinterpret_cast<uint4*>(pt_s + (pch >> 3) * (a.H * 128) + tc::sw128((uint32_t)ph, (uint32_t)(pch & 7))) =
-              raw;
-        }
-        tc::fence_proxy_async();
-        __syncwarp();
-        if (lane == 0) tc::mbar_arrive(&p_full[ps]);
-        // ---- value latent codes -> A tiles, one 128-channel block at a time
-        const int r = nt & 1;
-        tc::mbar_wait_ab(&raw_full[r], ((uint32_t)(nt >> 1)) & 1u, a.status, &abort_flag);
-        const uint8_t* blk = R_s + (size_t)r * raw_stage + (size_t)(tok >> 4) * a.vblk_bytes;
-        const int slot16 = tok & 15;
-        const bool tvalid = t0 + tok < len;
-        for (int cb = 0; cb < nblk; ++cb, ++na) {
-          const int as = na & 1;
-          const int gi = cb * 4 + cq;
-          const int2 vg = vg_s[gi];
-          uint32_t w0 = 0, w1 = 0, w2 = 0, w3 = 0;
-          float sc = 0.f;
-          if (tvalid) {
-            sc = __half2float(reinterpret_cast<const __half*>(blk)[gi * kPage + slot16]);
-            const uint32_t* cw = reinterpret_cast<const uint32_t*>(blk + vg.y) + slot16 * vg.x;
-            if (vg.x == 4) {
-              const uint4 v4 = *reinterpret_cast<const uint4*>(cw);
-              w0 = v4.x; w1 = v4.y; w2 = v4.z; w3 = v4.w;
-            } else {
-              w0 = cw[0]; w1 = cw[1]; w2 = cw[2];
-            }
-          }
-          const __half2 s2 = __floats2half2_rn(sc, sc);
-          const float offm = 1024.f + (float)(1 << (vg.x - 1));
-          const __half2 sub = __floats2half2_rn(offm, offm);
+        for (int gg = 0; gg < 4; ++gg) {
+          const int g = cb * 4 + gg;
+          const int4 vg = vg_s[g];
+          const __half hs = valid ? reinterpret_cast<const __half*>(blk)[g * kPage + slot] : __ushort_as_half(0);
+          const __half2 s2 = __halves2half2(hs, hs);
+          const __half2 sub = *reinterpret_cast<const __half2*>(&vg.z);
+          const uint32_t* cw = reinterpret_cast<const uint32_t*>(blk + vg.y) + slot * vg.x;
           uint4 o0, o1, o2, o3;
           if (vg.x == 4) {
-            o0 = deq8_b4(w0, sub, s2);
-            o1 = deq8_b4(w1, sub, s2);
-            o2 = deq8_b4(w2, sub, s2);
-            o3 = deq8_b4(w3, sub, s2);
+            const uint4 v4 = *reinterpret_cast<const uint4*>(cw);
+            o0 = deq8_b4(v4.x, sub, s2);
+            o1 = deq8_b4(v4.y, sub, s2);
+            o2 = deq8_b4(v4.z, sub, s2);
+            o3 = deq8_b4(v4.w, sub, s2);
           } else {
+            const uint32_t w0 = cw[0], w1 = cw[1], w2 = cw[2];
             o0 = deq8_b3(w0, sub, s2);
             o1 = deq8_b3(__funnelshift_r(w0, w1, 24), sub, s2);
             o2 = deq8_b3(__funnelshift_r(w1, w2, 16), sub, s2);
             o3 = deq8_b3(w2 >> 8, sub, s2);
           }
-          if (!tvalid) o0 = o1 = o2 = o3 = make_uint4(0, 0, 0, 0);
-          tc::mbar_wait_ab(&a_empty[as], (((uint32_t)(na >> 1)) & 1u) ^ 1u, a.status, &abort_flag);
-          uint8_t* at = A_s + (size_t)as * 32768 + a_off;
-          const uint32_t c4 = (uint32_t)(cq & 1) * 4u;     // 8-channel chunk index of this group in its atom
+          uint8_t* at = st + (gg >> 1) * 1024;
+          const uint32_t c4 = (uint32_t)(gg & 1) * 4u;   // 8-channel chunk of this group in its atom
           *reinterpret_cast<uint4*>(at + (((c4 + 0u) ^ x7) << 4)) = o0;
           *reinterpret_cast<uint4*>(at + (((c4 + 1u) ^ x7) << 4)) = o1;
           *reinterpret_cast<uint4*>(at + (((c4 + 2u) ^ x7) << 4)) = o2;
           *reinterpret_cast<uint4*>(at + (((c4 + 3u) ^ x7) << 4)) = o3;
-          tc::fence_proxy_async();
-          __syncwarp();
-          if (lane == 0) tc::mbar_arrive(&a_full[as]);
         }
-        __syncwarp();
-        if (lane == 0) tc::mbar_arrive(&raw_empty[r]);
-        ++nt;
+      }
+      tc::fence_proxy_async();
+      __syncwarp();
+      if (lane == 0) {
+        tc::mbar_arrive(&a_full[as]);
+        tc::mbar_arrive(&r_empty[rs]);
       }
     }
-    if (cur_b >= 0) finish_run();
+    while (epi_run < n_runs) epilogue(epi_run++);
   }
   tc::tc_fence_before();
   __syncthreads();
   tc::tc_fence_after();
-  if (warp == 1) tc::tmem_dealloc(tmem, a.tmem_cols);
+  if (warp == 0) tc::tmem_dealloc(tmem, a.tmem_cols);
 }
 
 // Merge the runs of each sequence: y = sum exp2(M_r - M) Y_r / sum exp2(M_r - M) l_r,
@@ -442,11 +572,34 @@ __global__ void k_values_combine(const float* __restrict__ Y, const float* __res
 
 }  // namespace
 
+// Dynamic shared memory of the value kernel: the A stages and two P stages.
+static size_t values_raw_stage(int vblk_bytes) { return (size_t)(2 * vblk_bytes + 127) / 128 * 128; }
+static size_t values_smem(int H, int vblk_bytes, int n_raw) {
+  return (size_t)kAStages * kAStage + 2 * (size_t)H * 256 + n_raw * values_raw_stage(vblk_bytes) + 1024;
+}
+
+// Grid of the value kernel: one CTA per SM, more when a CTA would hold more
+// than kMaxRuns sequences or kMaxTiles tiles.  *slots = the most runs one CTA
+// can hold.
+static int values_grid(long long U, int n_st, int* slots) {
+  long long G = std::min<long long>(num_sms(), U);
+  for (;;) {
+    const long long per = (U + G - 1) / G;
+    const int sl = (int)((per + n_st - 1) / n_st) + 1;
+    if ((sl <= kMaxRuns && per <= kMaxTiles / 2) || G >= U) {
+      *slots = sl;
+      return (int)G;
+    }
+    G = std::min(U, G * 2);
+  }
+}
+
 bool plan_values_tc(starkv_layer* L) {
   const LayerView& v = L->view;
   const starkv_layer_config& c = L->cfg;
   if (!L->tc_scores) return false;
-  if (v.rv % 128 != 0 || v.H % 16 != 0 || v.H > 64) return false;
+  // power-of-two count of 128-channel value blocks, heads a multiple of 16
+  if (v.rv % 128 != 0 || ((v.rv / 128) & (v.rv / 128 - 1)) != 0 || v.H % 16 != 0 || v.H > 64) return false;
   if ((long long)(v.rv / 128) * v.H > 512) return false;
   const LatentDesc& ld = L->lat[v.L - 1];
   if (ld.n_groups * 32 != v.rv) return false;
@@ -460,17 +613,22 @@ bool plan_values_tc(starkv_layer* L) {
   size_t bytes = ld.scale_bytes;
   for (int g = 0; g < ld.n_groups; ++g) bytes += (size_t)kPage * 32 * L->grp[ld.group0 + g].bits / 8;
   L->vblk_bytes = (int)bytes;
-  const size_t raw_stage = (8 * bytes + 1023) / 1024 * 1024;
-  const size_t smem = 2 * raw_stage + 2 * 32768 + 2 * (size_t)v.H * 256 + 1024;
-  return smem <= 226 * 1024;
+  // as many raw stages as fit next to the static tables and barriers, and at
+  // least 16 / nblk of them
+  cudaFuncAttributes fa;
+  if (cudaFuncGetAttributes(&fa, k_values_tc) != cudaSuccess) return false;
+  const int min_raw = std::max(4, kValWorkers / (v.rv / 128));
+  L->val_raw = 0;
+  for (int n_raw = kMaxRawStages; n_raw >= min_raw && !L->val_raw; --n_raw)
+    if (values_smem(v.H, L->vblk_bytes, n_raw) + fa.sharedSizeBytes <= 232448) L->val_raw = n_raw;
+  return L->val_raw > 0;
 }
 
 size_t values_tc_ws_bytes(const starkv_layer* L, int batch, int max_len) {
   const int n_st = (max_len + kVSuper - 1) / kVSuper;
   const long long U = (long long)batch * n_st;
-  const int G = (int)std::min<long long>(num_sms(), U);
-  const long long per = (U + G - 1) / G;
-  const int slots = (int)((per + n_st - 1) / n_st) + 1;
+  int slots = 0;
+  const int G = values_grid(U, n_st, &slots);
   auto r = [](size_t x) { return (x + 255) / 256 * 256; };
   const LayerView& v = L->view;
   return r(sizeof(float) * (size_t)G * slots * v.H * v.rv) + 2 * r(sizeof(float) * (size_t)G * slots * v.H);
@@ -483,9 +641,8 @@ cudaError_t launch_values_tc(const starkv_layer* L, const uint8_t* pool, long lo
   const int max_len = max_pages * kPage;
   const int n_st = (max_len + kVSuper - 1) / kVSuper;
   const long long U = (long long)batch * n_st;
-  const int G = (int)std::min<long long>(num_sms(), U);
-  const long long per = (U + G - 1) / G;
-  const int slots = (int)((per + n_st - 1) / n_st) + 1;
+  int slots = 0;
+  const int G = values_grid(U, n_st, &slots);
   auto r = [](size_t x) { return (x + 255) / 256 * 256; };
   uint8_t* w = (uint8_t*)ws;
   ValArgs a;
@@ -497,9 +654,13 @@ cudaError_t launch_values_tc(const starkv_layer* L, const uint8_t* pool, long lo
   a.seq_lens = seq_lens;
   a.vblk_off = L->vblk_off;
   a.vblk_bytes = L->vblk_bytes;
+  a.raw_stage = (int)values_raw_stage(L->vblk_bytes);
+  a.n_raw = L->val_raw;
   a.vgrp = L->d_grp + L->lat[v.L - 1].group0;
   a.rv = v.rv;
   a.H = v.H;
+  a.lg_nblk = 0;
+  while ((128 << a.lg_nblk) < v.rv) ++a.lg_nblk;
   a.P = (const __half*)so.P;
   a.P_ld = so.P_ld;
   a.m_st = so.m_st;
@@ -516,8 +677,7 @@ cudaError_t launch_values_tc(const starkv_layer* L, const uint8_t* pool, long lo
   while (cols < (uint32_t)((v.rv / 128) * v.H)) cols <<= 1;
   a.tmem_cols = cols;
   a.status = L->status;
-  const size_t raw_stage = (8 * (size_t)L->vblk_bytes + 1023) / 1024 * 1024;
-  const size_t smem = 2 * raw_stage + 2 * 32768 + 2 * (size_t)v.H * 256 + 1024;
+  const size_t smem = values_smem(v.H, L->vblk_bytes, L->val_raw);
   static size_t attr = 0;
   if (smem > attr) {
     cudaError_t e = cudaFuncSetAttribute(k_values_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);

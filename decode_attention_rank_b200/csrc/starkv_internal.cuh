@@ -134,6 +134,7 @@ struct starkv_layer {
   // tensor-core value kernel
   bool tc_values = false;
   int vblk_off = 0, vblk_bytes = 0;
+  int val_raw = 0;              // raw chunk stages of the value kernel
 };
 
 namespace starkv {
