@@ -120,7 +120,10 @@ __device__ __forceinline__ uint4 deq8_b3(uint32_t run, __half2 sub, __half2 s2) 
 
 __global__ void __launch_bounds__(kValThreads, 1) k_values_tc(ValArgs a) {
   extern __shared__ uint8_t smem_raw[];
-  __shared__ __align__(8) uint64_t a_full[kAStages], a_empty[kAStages], r_full[kMaxRawStages], r_empty[kMaxRawStages];
+  // chain c = items 4 c .. 4 c + 3 (one 128-channel block of a tile, four
+  // workers, A stages (4 c .. 4 c + 3) % kAStages): ch_full[c % 4] when the
+  // four are written, ch_done[c % 4] when their MMAs have completed
+  __shared__ __align__(8) uint64_t ch_full[4], ch_done[4], r_full[kMaxRawStages], r_empty[kMaxRawStages];
   __shared__ __align__(8) uint64_t p_full[2], p_empty[2];
   __shared__ __align__(8) uint64_t seg_done, acc_free, fin;
   __shared__ uint32_t tmem_base;
@@ -145,9 +148,9 @@ __global__ void __launch_bounds__(kValThreads, 1) k_values_tc(ValArgs a) {
   const int b_first = (int)(u0 / a.n_st);
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < kAStages; ++s) {
-      tc::mbar_init(&a_full[s], 1);
-      tc::mbar_init(&a_empty[s], 1);
+    for (int s = 0; s < 4; ++s) {
+      tc::mbar_init(&ch_full[s], 4);
+      tc::mbar_init(&ch_done[s], 1);
     }
     for (int s = 0; s < a.n_raw; ++s) {
       tc::mbar_init(&r_full[s], 1);
@@ -235,9 +238,9 @@ __global__ void __launch_bounds__(kValThreads, 1) k_values_tc(ValArgs a) {
     // ------------------------------------------------ MMA issue
     // Item n of the CTA (tile n / ipt, item n % ipt = 4 cb + k) sits in A
     // stage n % kAStages; its two K = 16 steps add block cb's Y^T.  The four
-    // items of a block are consecutive, so eight MMAs in a row accumulate into
-    // one TMEM block (an MMA that switches accumulators costs about twice as
-    // much as one that continues a chain).
+    // items of a block are waited for together and their eight MMAs issued
+    // back to back: an N = 32 MMA takes only about 45 cycles on the tensor
+    // pipe, so the issuing thread must spend very few instructions per MMA.
     if (lane == 0) {
       const uint32_t idesc = tc::idesc_f16(128, a.H, false, true, false);
       // descriptors as (low, high) halves; steps are 16-byte units on the low half
@@ -264,24 +267,23 @@ __global__ void __launch_bounds__(kValThreads, 1) k_values_tc(ValArgs a) {
         tc::tc_fence_after();
         const uint32_t b_lo = b_lo0 + (uint32_t)ps * p_step;
         bool ok = true;
-        for (int cb = 0; cb < nblk && ok; ++cb) {
+        for (int cb = 0; cb < nblk && ok; ++cb, n += 4) {
+          // the chain's four items, then its eight MMAs back to back and one commit
+          const int c = n >> 2;
+          ok = tc::mbar_wait_ab(&ch_full[c & 3], ((uint32_t)(c >> 2)) & 1u, a.status, &abort_flag);
+          if (!ok) break;
+          tc::tc_fence_after();
           const uint32_t d = tmem + (uint32_t)(cb * a.H);
+          const uint32_t a_lo = a_lo0 + (uint32_t)(n % kAStages) * (kAStage >> 4);
 #pragma unroll
-          for (int k = 0; k < 4; ++k, ++n) {
-            const int s = n % kAStages;
-            if (!tc::mbar_wait_ab(&a_full[s], ((uint32_t)(n / kAStages)) & 1u, a.status, &abort_flag)) {
-              ok = false;
-              break;
-            }
-            tc::tc_fence_after();
-            const uint32_t a_lo = a_lo0 + (uint32_t)s * (kAStage >> 4);
-            // tokens 32 k .. 32 k + 31: 16-token steps 2 k and 2 k + 1 of the P tile
-            tc::mma_f16_ss2(d, a_lo, a_hi, b_lo + (uint32_t)(k >> 1) * b_atom + (uint32_t)(k & 1) * 4u, b_hi, idesc,
-                            (first && k == 0) ? 0u : 1u);
-            tc::mma_f16_ss2(d, a_lo + (4096u >> 4), a_hi, b_lo + (uint32_t)(k >> 1) * b_atom + (uint32_t)(k & 1) * 4u + 2u,
-                            b_hi, idesc, 1u);
-            tc::mma_commit(&a_empty[s]);
+          for (int k = 0; k < 4; ++k) {
+            // tokens 32 k .. 32 k + 31: 16-token steps 2 k and 2 k + 1 of the P tile; stages wrap at kAStages
+            const uint32_t ak = a_lo + (uint32_t)(((n + k) % kAStages) - (n % kAStages)) * (kAStage >> 4);
+            const uint32_t bk = b_lo + (uint32_t)(k >> 1) * b_atom + (uint32_t)(k & 1) * 4u;
+            tc::mma_f16_ss2(d, ak, a_hi, bk, b_hi, idesc, (first && k == 0) ? 0u : 1u);
+            tc::mma_f16_ss2(d, ak + (4096u >> 4), a_hi, bk + 2u, b_hi, idesc, 1u);
           }
+          tc::mma_commit(&ch_done[c & 3]);
         }
         if (!ok) break;
         tc::mma_commit(&p_empty[ps]);
@@ -465,7 +467,8 @@ __global__ void __launch_bounds__(kValThreads, 1) k_values_tc(ValArgs a) {
       // A stage first: once item n - 16 is consumed, every chunk up to its
       // chunk has landed; with at least max(4, 16 / nblk) raw stages the raw
       // stage is then at most one phase from chunk c
-      const bool ok = tc::mbar_wait_ab(&a_empty[as], (((uint32_t)(n / kAStages)) & 1u) ^ 1u, a.status, &abort_flag) &&
+      const int ch = n >> 2;                   // chain of this item; the worker's previous item was in chain ch - 4
+      const bool ok = tc::mbar_wait_ab(&ch_done[ch & 3], (((uint32_t)(ch >> 2)) & 1u) ^ 1u, a.status, &abort_flag) &&
                       tc::mbar_wait_ab(&r_full[rs], ((uint32_t)(c / a.n_raw)) & 1u, a.status, &abort_flag);
       if (ok) {
         const uint8_t* blk = R_s + (size_t)rs * a.raw_stage + (size_t)(lane >> 4) * a.vblk_bytes;
@@ -503,7 +506,7 @@ __global__ void __launch_bounds__(kValThreads, 1) k_values_tc(ValArgs a) {
       tc::fence_proxy_async();
       __syncwarp();
       if (lane == 0) {
-        tc::mbar_arrive(&a_full[as]);
+        tc::mbar_arrive(&ch_full[ch & 3]);
         tc::mbar_arrive(&r_empty[rs]);
       }
     }

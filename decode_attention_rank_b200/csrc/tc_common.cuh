@@ -77,33 +77,34 @@ __device__ __forceinline__ bool mbar_test_wait(uint64_t* bar, uint32_t parity) {
       : "memory");
   return ok != 0;
 }
-// Bounded wait on the phase with the given parity.  Returns false (and sets
-// the timeout bit) if the phase did not complete within kWaitLimitNs.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint32_t* status) {
-  if (mbar_test_wait(bar, parity) || mbar_try_wait(bar, parity)) return true;
+// Slow paths of the waits below, out of line: a phase that has not completed
+// is polled with a suspending try_wait until the limit.
+static __device__ __noinline__ bool mbar_wait_slow(uint64_t* bar, uint32_t parity, uint32_t* status, volatile int* abort) {
+  if (mbar_try_wait(bar, parity)) return true;
   const unsigned long long t0 = global_ns();
   for (uint32_t i = 1;; ++i) {
     if (mbar_try_wait(bar, parity)) return true;
+    if (abort && *abort) return false;
     if ((i & 15u) == 0u && global_ns() - t0 > kWaitLimitNs) break;
   }
   if (status) atomicOr(status, kTimeout);
+  if (abort) *abort = 1;
   return false;
+}
+
+// Bounded wait on the phase with the given parity.  Returns false (and sets
+// the timeout bit) if the phase did not complete within kWaitLimitNs.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint32_t* status) {
+  if (mbar_test_wait(bar, parity)) return true;
+  return mbar_wait_slow(bar, parity, status, nullptr);
 }
 
 // Bounded wait that also gives up as soon as another role of the CTA has
 // aborted (*abort != 0), so that every role drains quickly and in step.
 __device__ __forceinline__ bool mbar_wait_ab(uint64_t* bar, uint32_t parity, uint32_t* status,
                                              volatile int* abort) {
-  if (mbar_test_wait(bar, parity) || mbar_try_wait(bar, parity)) return true;
-  const unsigned long long t0 = global_ns();
-  for (uint32_t i = 1;; ++i) {
-    if (mbar_try_wait(bar, parity)) return true;
-    if (*abort) return false;
-    if ((i & 15u) == 0u && global_ns() - t0 > kWaitLimitNs) break;
-  }
-  if (status) atomicOr(status, kTimeout);
-  *abort = 1;
-  return false;
+  if (mbar_test_wait(bar, parity)) return true;
+  return mbar_wait_slow(bar, parity, status, abort);
 }
 
 // ---- bulk copies (global -> shared, completion on an mbarrier) -------------
