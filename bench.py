@@ -181,6 +181,32 @@ def fill_cache(spec, f, L, B, T0, rank, ctx, tail_pages):
     return pool, n_pages, page_table, page_table_e2e
 
 
+def latent_bytes(spec, r):
+    """Algorithmic bytes of one token's latent of rank r (codes + fp16 scales, no page padding)."""
+    if not spec.quantized:
+        return r * (4 if spec.dtype == "f32" else 2)
+    n_hi = math.ceil(spec.top_fraction * r)
+    n_lo = r - n_hi
+    bits = spec.top_bits * n_hi + spec.bottom_bits * n_lo
+    return bits / 8 + 2 * (math.ceil(n_hi / spec.group_size) + math.ceil(n_lo / spec.group_size))
+
+
+PHASES = ["query prep + key scoring (k_qprep_tc, k_scores_tc)", "joint value contraction (k_values_tc)",
+          "run merge (k_values_combine)", "output through M (k_outproj_tc, k_outproj_reduce)"]
+
+
+def phase_bytes(spec, B, ctx):
+    """Algorithmic HBM bytes of each decode phase: key cache + B'_k; value cache;
+    nothing (the merge reads kernel intermediates only); M + y/out."""
+    key = sum(latent_bytes(spec, r) for r in spec.key_ranks)
+    val = latent_bytes(spec, spec.value_rank)
+    d = spec.head_dim
+    return [B * ctx * key + 2 * d * sum(spec.key_ranks) + B * spec.n_heads * d * 2,
+            B * ctx * val,
+            0.0,
+            2 * spec.n_heads * spec.value_rank * spec.hidden + B * spec.hidden * 2]
+
+
 def decode_bytes(spec, L, B, ctx):
     """Algorithmic HBM bytes of one decode step: cache + B'_k + M + q/out."""
     return B * ctx * L.bytes_per_token + L.factor_bytes + B * (spec.n_heads * spec.head_dim + spec.hidden) * 2
@@ -249,6 +275,7 @@ def run_ours(args, rank, ws, local):
     t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     torch.cuda.synchronize()
     barrier(ws)
+    L.profile_decode(K)   # CUDA events between the decode's kernels, on its stream
     torch.cuda.nvtx.range_push("timed")
     t_start.record(stream)
     for k in range(K):
@@ -259,6 +286,9 @@ def run_ours(args, rank, ws, local):
     barrier(ws)
     ms_total = t_start.elapsed_time(t_end)
     dec_ms = sum(a.elapsed_time(b) for a, b in evs) / K
+    ph = L.decode_phase_ms(K)
+    L.profile_decode(0)
+    ph_ms = [max_over_ranks(sum(c[p] for c in ph) / K, ws) for p in range(len(PHASES))]
     clk = clocks.stop()
     assert L.sync_status() == 0, "device status word set during the benchmark"
     ms_step = max_over_ranks(ms_total / K, ws)
@@ -300,6 +330,12 @@ def run_ours(args, rank, ws, local):
     peak, peak_kind = measured_peaks()
     dbytes = decode_bytes(spec, L, B, T0 + W + K // 2)
     achieved = dbytes / (dec_ms * 1e-3) / 1e9
+    pbytes = phase_bytes(spec, B, T0 + W + K // 2)
+    kernels = [{"phase": PHASES[p], "us": ph_ms[p] * 1e3, "algorithmic_bytes": pbytes[p],
+                "GB/s": (pbytes[p] / (ph_ms[p] * 1e-3) / 1e9) if ph_ms[p] > 0 else None,
+                "frac": (pbytes[p] / (ph_ms[p] * 1e-3) / 1e9 / peak) if ph_ms[p] > 0 else None}
+               for p in range(len(PHASES))]
+    dom = max(range(len(PHASES)), key=lambda p: ph_ms[p])
     tokens_per_s = B * ws / (ms_step * 1e-3)
     res = {
         "metric": METRIC,
@@ -322,12 +358,15 @@ def run_ours(args, rank, ws, local):
                                                                             L.factor_bytes / 1e6)},
         "us_per_layer_step": ms_step * 1e3,
         "decode_us": dec_ms * 1e3,
-        "roofline": {"bound": "hbm", "kernel": "starkv_decode_attn (all decode kernels of one call)",
-                     "achieved": achieved, "peak": peak, "peak_kind": peak_kind, "unit": "GB/s",
-                     "frac": achieved / peak, "traffic": None, "algorithmic_bytes": dbytes},
+        "roofline": {"bound": "hbm", "kernel": PHASES[dom], "achieved": kernels[dom]["GB/s"], "peak": peak,
+                     "peak_kind": peak_kind, "unit": "GB/s", "frac": kernels[dom]["frac"], "traffic": None,
+                     "algorithmic_bytes": pbytes[dom], "us_per_launch": ph_ms[dom] * 1e3,
+                     "whole_decode": {"achieved": achieved, "frac": achieved / peak, "algorithmic_bytes": dbytes,
+                                      "us": dec_ms * 1e3}},
+        "kernels": kernels,
         "e2e": {"value": B * ws / (e2e_ms * 1e-3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h},
-        "gpu_launches": K * 7,
+        "gpu_launches": K * 10,   # append: 3 kernels; decode: 7 (see the launch list under profiles/)
         "clocks": clk,
     }
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:

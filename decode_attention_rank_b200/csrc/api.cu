@@ -209,6 +209,7 @@ void starkv_free_layer(starkv_layer* L) {
   cudaFree(L->d_items);
   cudaFree(L->d_score_heads);
   cudaFree(L->rope_E);
+  for (cudaEvent_t e : L->prof_ev) cudaEventDestroy(e);
   cudaSetDevice(cur);
   delete L;
 }
@@ -499,6 +500,50 @@ starkv_status starkv_set_decode_path(starkv_layer* L, int path) {
     return STARKV_ERR_UNSUPPORTED;
   }
   L->decode_path = path;
+  return STARKV_OK;
+}
+
+starkv_status starkv_profile_decode(starkv_layer* L, int n_calls) {
+  set_error("");
+  CHECK_ARG(L != nullptr, "layer is NULL");
+  CHECK_ARG(n_calls >= 0 && n_calls <= 4096, "n_calls must be in [0, 4096]");
+  int cur = 0;
+  cudaGetDevice(&cur);
+  cudaSetDevice(L->device);
+  for (cudaEvent_t e : L->prof_ev) cudaEventDestroy(e);
+  L->prof_ev.clear();
+  L->prof_used.assign(n_calls, 0);
+  L->prof_n = 0;
+  L->prof_calls = 0;
+  for (int i = 0; i < n_calls * (STARKV_N_PHASES + 1); ++i) {
+    cudaEvent_t e;
+    if (cudaEventCreate(&e) != cudaSuccess) {
+      cudaSetDevice(cur);
+      set_error("cudaEventCreate failed");
+      return STARKV_ERR_CUDA;
+    }
+    L->prof_ev.push_back(e);
+  }
+  L->prof_n = n_calls;
+  cudaSetDevice(cur);
+  return STARKV_OK;
+}
+
+starkv_status starkv_decode_phase_ms(const starkv_layer* L, float* ms, int n_calls) {
+  set_error("");
+  CHECK_ARG(L != nullptr && ms != nullptr, "layer or ms is NULL");
+  CHECK_ARG(n_calls >= 0 && n_calls <= L->prof_n, "n_calls exceeds the timed calls kept");
+  for (int c = 0; c < n_calls; ++c) {
+    const cudaEvent_t* ev = &L->prof_ev[(size_t)c * (STARKV_N_PHASES + 1)];
+    for (int p = 0; p < STARKV_N_PHASES; ++p) {
+      float t = 0.f;
+      if (L->prof_used[c]) {
+        CUDA_TRY(cudaEventSynchronize(ev[p + 1]));
+        CUDA_TRY(cudaEventElapsedTime(&t, ev[p], ev[p + 1]));
+      }
+      ms[(size_t)c * STARKV_N_PHASES + p] = t;
+    }
+  }
   return STARKV_OK;
 }
 

@@ -639,7 +639,7 @@ size_t values_tc_ws_bytes(const starkv_layer* L, int batch, int max_len) {
 
 cudaError_t launch_values_tc(const starkv_layer* L, const uint8_t* pool, long long n_pages, const int32_t* pt,
                              int max_pages, int batch, const int32_t* seq_lens, const ScoreOut& so, void* ws,
-                             void* ytiles, cudaStream_t s) {
+                             void* ytiles, cudaStream_t s, cudaEvent_t ev_mid) {
   const LayerView& v = L->view;
   const int max_len = max_pages * kPage;
   const int n_st = (max_len + kVSuper - 1) / kVSuper;
@@ -690,6 +690,7 @@ cudaError_t launch_values_tc(const starkv_layer* L, const uint8_t* pool, long lo
   k_values_tc<<<G, kValThreads, smem, s>>>(a);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
+  if (ev_mid && (e = cudaEventRecord(ev_mid, s)) != cudaSuccess) return e;
   const int NB = outproj_nb(batch);
   k_values_combine<<<dim3(batch, v.H), 256, 0, s>>>(a.Y, a.mseg, a.lseg, G, U, n_st, slots, v.H, v.rv, NB,
                                                    L->Kp / 64, (uint8_t*)ytiles);
@@ -728,17 +729,31 @@ cudaError_t launch_decode_tc(const starkv_layer* L, const uint8_t* pool, long lo
   uint8_t* ytiles = w;
   w += r(y_bytes);
   float* part = (float*)w;
+  // optional timing events between the kernels (see starkv_profile_decode)
+  cudaEvent_t* ev = nullptr;
+  if (L->prof_n > 0) {
+    starkv_layer* Lm = const_cast<starkv_layer*>(L);
+    const int slot = (int)(Lm->prof_calls++ % Lm->prof_n);
+    ev = &Lm->prof_ev[(size_t)slot * (STARKV_N_PHASES + 1)];
+    Lm->prof_used[slot] = 1;
+  }
+  cudaError_t e;
+  if (ev && (e = cudaEventRecord(ev[0], s)) != cudaSuccess) return e;
   ScoreOut so;
-  cudaError_t e = launch_scores_tc(L, pool, n_pages, pt, max_pages, batch, seq_lens, q_pos, q, w_scores, &so, nullptr,
-                                   0, s);
+  e = launch_scores_tc(L, pool, n_pages, pt, max_pages, batch, seq_lens, q_pos, q, w_scores, &so, nullptr, 0, s);
   if (e != cudaSuccess) return e;
+  if (ev && (e = cudaEventRecord(ev[1], s)) != cudaSuccess) return e;
   if (batch % NB != 0 || L->Kp != L->view.H * L->view.wv) {
     e = cudaMemsetAsync(ytiles, 0, y_bytes, s);
     if (e != cudaSuccess) return e;
   }
-  e = launch_values_tc(L, pool, n_pages, pt, max_pages, batch, seq_lens, so, w_values, ytiles, s);
+  e = launch_values_tc(L, pool, n_pages, pt, max_pages, batch, seq_lens, so, w_values, ytiles, s, ev ? ev[2] : nullptr);
   if (e != cudaSuccess) return e;
-  return launch_outproj_tc(L, ytiles, batch, out, part, s);
+  if (ev && (e = cudaEventRecord(ev[3], s)) != cudaSuccess) return e;
+  e = launch_outproj_tc(L, ytiles, batch, out, part, s);
+  if (e != cudaSuccess) return e;
+  if (ev && (e = cudaEventRecord(ev[4], s)) != cudaSuccess) return e;
+  return cudaSuccess;
 }
 
 }  // namespace starkv

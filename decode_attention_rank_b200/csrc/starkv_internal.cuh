@@ -135,6 +135,12 @@ struct starkv_layer {
   bool tc_values = false;
   int vblk_off = 0, vblk_bytes = 0;
   int val_raw = 0;              // raw chunk stages of the value kernel
+  // optional per-kernel timing of the tensor-core decode: prof_n sets of
+  // STARKV_N_PHASES + 1 events, the decode call number prof_calls picks the set
+  std::vector<cudaEvent_t> prof_ev;
+  int prof_n = 0;
+  long long prof_calls = 0;
+  std::vector<char> prof_used;
 };
 
 namespace starkv {
@@ -172,7 +178,7 @@ bool plan_values_tc(starkv_layer* L);
 size_t values_tc_ws_bytes(const starkv_layer* L, int batch, int max_len);
 cudaError_t launch_values_tc(const starkv_layer* L, const uint8_t* pool, long long n_pages, const int32_t* pt,
                              int max_pages, int batch, const int32_t* seq_lens, const ScoreOut& so, void* ws,
-                             void* ytiles, cudaStream_t s);
+                             void* ytiles, cudaStream_t s, cudaEvent_t ev_mid);
 cudaError_t launch_decode_tc(const starkv_layer* L, const uint8_t* pool, long long n_pages, const int32_t* pt,
                              int max_pages, int batch, const int32_t* seq_lens, const int32_t* q_pos, const void* q,
                              void* out, void* ws, size_t ws_bytes, cudaStream_t s);

@@ -77,6 +77,9 @@ _lib.starkv_status_string.restype = ctypes.c_char_p
 _lib.starkv_last_error.argtypes = []
 _lib.starkv_last_error.restype = ctypes.c_char_p
 _lib.starkv_set_decode_path.argtypes = [_vp, ctypes.c_int]
+_lib.starkv_profile_decode.argtypes = [_vp, ctypes.c_int]
+_lib.starkv_decode_phase_ms.argtypes = [_vp, ctypes.POINTER(ctypes.c_float), ctypes.c_int]
+N_PHASES = 4   # query preparation + scores, joint values, run merge, output projection
 _lib.starkv_version.argtypes = []
 _lib.starkv_version.restype = ctypes.c_char_p
 
@@ -222,6 +225,16 @@ class Layer:
     def set_decode_path(self, path: int) -> None:
         """0 automatic, 1 CUDA-core kernels, 2 tensor-core scores + CUDA-core values (diagnostics)."""
         _check(_lib.starkv_set_decode_path(self._h, path), "starkv_set_decode_path")
+
+    def profile_decode(self, n_calls: int) -> None:
+        """Keep CUDA-event timings of the next n_calls tensor-core decodes (0 = off)."""
+        _check(_lib.starkv_profile_decode(self._h, n_calls), "starkv_profile_decode")
+
+    def decode_phase_ms(self, n_calls: int) -> list:
+        """Per-call lists of the phase times (ms) recorded since profile_decode."""
+        buf = (ctypes.c_float * (n_calls * N_PHASES))()
+        _check(_lib.starkv_decode_phase_ms(self._h, buf, n_calls), "starkv_decode_phase_ms")
+        return [list(buf[c * N_PHASES:(c + 1) * N_PHASES]) for c in range(n_calls)]
 
     def sync_status(self, stream=None) -> int:
         bits = ctypes.c_uint32(0)

@@ -271,6 +271,24 @@ STARKV_API const char* starkv_version(void);
  */
 STARKV_API starkv_status starkv_set_decode_path(starkv_layer* layer, int path);
 
+/*
+ * Measurement: per-kernel device time of the tensor-core decode, taken with
+ * CUDA events recorded on the decode's own stream between its kernels (no
+ * synchronisation is added to the calls).
+ *   starkv_profile_decode(layer, n_calls) keeps n_calls sets of events (the
+ *     next n_calls decodes fill them in order; 0 switches timing off and frees
+ *     them).  Must not be called while a decode of the layer is in flight.
+ *   starkv_decode_phase_ms(layer, ms, n_calls) waits for the recorded events
+ *     and writes ms[c * STARKV_N_PHASES + p]: call c, phase p in the order
+ *     query preparation + scores, joint values, run merge, output projection.
+ *     Calls that took another decode path report zeros.
+ * Returns STARKV_ERR_ARG for a NULL layer or an n_calls outside [0, 4096],
+ * STARKV_ERR_CUDA if events cannot be created or read.
+ */
+#define STARKV_N_PHASES 4
+STARKV_API starkv_status starkv_profile_decode(starkv_layer* layer, int n_calls);
+STARKV_API starkv_status starkv_decode_phase_ms(const starkv_layer* layer, float* ms, int n_calls);
+
 #ifdef __cplusplus
 }
 #endif
