@@ -29,7 +29,7 @@ Sources (page titles and sections of the STAR-KV material):
     top_bits 4, bottom_bits 3; protected layers.
   * The arXiv abstract (as reprinted on the gptget.net summary page).
 
-Readings where the pages are silent (listed again in the design doc):
+Readings where the pages are silent:
   * quantizer: symmetric, zero point 0, qmax = 2^(b-1) - 1, one fp16 scale per
     (token, 32-channel group), scale = fp16 rounded toward +inf of amax/qmax
     (IEEE fp32 division), codes = round-half-even(z / scale) clamped to
