@@ -45,6 +45,15 @@ constexpr int kMaxRawStages = 16;
 constexpr int kVSuper = 256;     // tokens per super-tile (matches the score kernel)
 constexpr int kAStage = 8192;    // one A stage: 32 tokens x 128 value channels, fp16
 constexpr int kMaxRuns = 64;     // runs (sequences) per CTA
+constexpr int kRunMaxCache = 16; // runs whose per-head maxima are computed up front
+
+// Atomic maximum of floats (no NaN) through their integer orderings.
+__device__ __forceinline__ void atomic_max_float(float* addr, float v) {
+  if (v >= 0.f)
+    atomicMax(reinterpret_cast<int*>(addr), __float_as_int(v));
+  else
+    atomicMin(reinterpret_cast<unsigned int*>(addr), __float_as_uint(v));
+}
 
 struct ValArgs {
   const uint8_t* pool;
@@ -134,6 +143,7 @@ __global__ void __launch_bounds__(kValThreads, 1) k_values_tc(ValArgs a) {
   __shared__ int run_b[kMaxRuns];
   __shared__ int n_tiles_s, n_runs_s;
   __shared__ float l_stage[64];           // run sums of the staged P, per head
+  __shared__ float runM_s[kRunMaxCache][64];   // per run and head: the maximum of the 32-token group maxima
   uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   uint8_t* A_s = smem;                                   // kAStages x 8 KB A stages
   uint8_t* P_s = A_s + kAStages * kAStage;               // 2 x (H x 128 fp16, K-major swizzled)
@@ -231,6 +241,17 @@ __global__ void __launch_bounds__(kValThreads, 1) k_values_tc(ValArgs a) {
       }
     }
     pid_s[e >> 3][e & 7] = page;
+  }
+  for (int x = threadIdx.x; x < kRunMaxCache * 64; x += blockDim.x) (&runM_s[0][0])[x] = -FLT_MAX;
+  __syncthreads();
+  // run maxima, all threads at once (a tile contributes its four groups)
+  for (int e = threadIdx.x; e < n_tiles * a.H; e += blockDim.x) {
+    const int T = e / a.H, h = e - T * a.H;
+    const int4 tl = tile_s[T];
+    if (tl.w < kRunMaxCache) {
+      const float4 g4 = *reinterpret_cast<const float4*>(a.m_st + ((size_t)tl.x * a.H + h) * a.n_g + (tl.y >> 5));
+      atomic_max_float(&runM_s[tl.w][h], fmaxf(fmaxf(g4.x, g4.y), fmaxf(g4.z, g4.w)));
+    }
   }
   __syncthreads();
 
@@ -338,7 +359,9 @@ __global__ void __launch_bounds__(kValThreads, 1) k_values_tc(ValArgs a) {
         for (int hh = 0; hh < 2; ++hh) {
           const int h = lane + 32 * hh;
           float m = -FLT_MAX;
-          if (h < a.H) {
+          if (h < a.H && tl.w < kRunMaxCache) {
+            m = runM_s[tl.w][h];
+          } else if (h < a.H) {
             const float* mr = a.m_st + ((size_t)tl.x * a.H + h) * a.n_g;
             for (int T2 = T; T2 < n_tiles && tile_s[T2].w == tl.w; ++T2) {
               const float4 g4 = *reinterpret_cast<const float4*>(mr + (tile_s[T2].y >> 5));
@@ -523,37 +546,57 @@ __global__ void __launch_bounds__(kValThreads, 1) k_values_tc(ValArgs a) {
 __global__ void k_values_combine(const float* __restrict__ Y, const float* __restrict__ mseg,
                                  const float* __restrict__ lseg, int G, long long U, int n_st, int slots, int H,
                                  int rv, int NB, int KT, uint8_t* __restrict__ ytiles) {
-  // the runs of sequence b: partial slots of the CTAs whose unit ranges meet [b n_st, (b+1) n_st)
+  // the runs of sequence b: partial slots of the CTAs whose unit ranges meet
+  // [b n_st, (b+1) n_st); their (M, l) are read in parallel, one per thread
   __shared__ int seg_i[256];
   __shared__ float seg_w[256];
-  __shared__ int n_seg;
+  __shared__ int n_seg, c_first;
+  __shared__ float red_s[8];
   __shared__ float inv_den;
   const int b = blockIdx.x, h = blockIdx.y;
+  const long long lo = (long long)b * n_st, hi = lo + n_st;
   if (threadIdx.x == 0) {
-    const long long lo = (long long)b * n_st, hi = lo + n_st;
     int c = (int)((lo * G) / U);
     while (c > 0 && vunit_lo(c, G, U) > lo) --c;
     while (vunit_lo(c + 1, G, U) <= lo) ++c;
-    int n = 0;
-    float m = -FLT_MAX;
-    long long b0 = vunit_lo(c, G, U);
-    for (; c < G && b0 < hi && n < 256; ++c) {
-      const long long b1 = vunit_lo(c + 1, G, U);
-      if (b1 > lo && b1 > b0) {
-        const int i = (c * slots + (b - (int)(b0 / n_st))) * H + h;
-        if (lseg[i] > 0.f) {
-          seg_i[n++] = i;
-          m = fmaxf(m, mseg[i]);
-        }
-      }
-      b0 = b1;
+    int c1 = c;
+    while (c1 < G && vunit_lo(c1, G, U) < hi) ++c1;
+    c_first = c;
+    n_seg = min(c1 - c, 256);
+  }
+  __syncthreads();
+  const int nc = n_seg;
+  float mk = -FLT_MAX, lk = 0.f;
+  int ik = -1;
+  if ((int)threadIdx.x < nc) {
+    const int c = c_first + threadIdx.x;
+    const long long b0 = vunit_lo(c, G, U), b1 = vunit_lo(c + 1, G, U);
+    if (b1 > b0) {
+      ik = (c * slots + (b - (int)(b0 / n_st))) * H + h;
+      lk = lseg[ik];
+      mk = lk > 0.f ? mseg[ik] : -FLT_MAX;
     }
+  }
+  // block maximum of M over the runs with l > 0
+  float m = mk;
+  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+  if ((threadIdx.x & 31) == 0) red_s[threadIdx.x >> 5] = m;
+  __syncthreads();
+  m = -FLT_MAX;
+  for (int w = 0; w < (int)(blockDim.x >> 5); ++w) m = fmaxf(m, red_s[w]);
+  const float wk = (lk > 0.f) ? exp2f(mk - m) : 0.f;
+  if ((int)threadIdx.x < nc) {
+    seg_i[threadIdx.x] = ik < 0 ? 0 : ik;
+    seg_w[threadIdx.x] = wk;
+  }
+  float dn = wk * lk;
+  for (int o = 16; o > 0; o >>= 1) dn += __shfl_xor_sync(0xffffffffu, dn, o);
+  __syncthreads();
+  if ((threadIdx.x & 31) == 0) red_s[threadIdx.x >> 5] = dn;
+  __syncthreads();
+  if (threadIdx.x == 0) {
     float den = 0.f;
-    for (int k = 0; k < n; ++k) {
-      seg_w[k] = exp2f(mseg[seg_i[k]] - m);
-      den += seg_w[k] * lseg[seg_i[k]];
-    }
-    n_seg = n;
+    for (int w = 0; w < (int)(blockDim.x >> 5); ++w) den += red_s[w];
     inv_den = den > 0.f ? 1.f / den : 0.f;
   }
   __syncthreads();
@@ -564,8 +607,25 @@ __global__ void k_values_combine(const float* __restrict__ Y, const float* __res
     // position of channel j in the value kernel's A tiles: 1 <-> 2 and 5 <-> 6 inside each chunk of 8
     const int jw = j & 7;
     const int jp = (j & ~7) | (jw == 1 ? 2 : jw == 2 ? 1 : jw == 5 ? 6 : jw == 6 ? 5 : jw);
-    float acc = 0.f;
-    for (int k = 0; k < ns; ++k) acc += seg_w[k] * Y[(size_t)seg_i[k] * rv + jp];
+    // runs with no valid token (l = 0) wrote no Y: their loads are skipped
+    float acc0 = 0.f, acc1 = 0.f, acc2 = 0.f, acc3 = 0.f;
+    int k = 0;
+    for (; k + 4 <= ns; k += 4) {
+      const float w0 = seg_w[k], w1 = seg_w[k + 1], w2 = seg_w[k + 2], w3 = seg_w[k + 3];
+      const float y0 = w0 != 0.f ? Y[(size_t)seg_i[k] * rv + jp] : 0.f;
+      const float y1 = w1 != 0.f ? Y[(size_t)seg_i[k + 1] * rv + jp] : 0.f;
+      const float y2 = w2 != 0.f ? Y[(size_t)seg_i[k + 2] * rv + jp] : 0.f;
+      const float y3 = w3 != 0.f ? Y[(size_t)seg_i[k + 3] * rv + jp] : 0.f;
+      acc0 += w0 * y0;
+      acc1 += w1 * y1;
+      acc2 += w2 * y2;
+      acc3 += w3 * y3;
+    }
+    for (; k < ns; ++k) {
+      const float wgt = seg_w[k];
+      if (wgt != 0.f) acc0 += wgt * Y[(size_t)seg_i[k] * rv + jp];
+    }
+    const float acc = (acc0 + acc1) + (acc2 + acc3);
     const uint32_t kk = (uint32_t)(h * rv + j), cidx = kk & 63u;
     uint8_t* tile = ytiles + ((size_t)nt * KT + (kk >> 6)) * (size_t)NB * 128;
     const uint32_t off = tc::sw128((uint32_t)r, cidx >> 3) + (cidx & 7u) * 2u;
