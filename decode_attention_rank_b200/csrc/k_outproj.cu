@@ -70,18 +70,26 @@ __global__ void __launch_bounds__(kOutThreads, 1) k_outproj_tc(OutArgs a) {
 
   if (warp == 0) {
     if (lane == 0) {
-      int i = 0;
+      // unit u = (output tile u / KT, k-tile u % KT); M tiles are stored in unit order
+      int i = 0, s = 0;
+      uint32_t ph = 0;
+      int kt = (int)(u0 % a.KT);
+      const uint8_t* msrc = a.M + (size_t)u0 * a_bytes;
+      const uint8_t* ybase = a.y + (size_t)nt * a.KT * b_bytes;
       for (long long u = u0; u < u1; ++u, ++i) {
-        const int s = i % a.stages;
-        const uint32_t ph = (uint32_t)(i / a.stages) & 1u;
         if (!tc::mbar_wait(&empty[s], ph ^ 1u, a.status)) {
           abort_flag = 1;
           break;
         }
-        const int dt = (int)(u / a.KT), kt = (int)(u % a.KT);
         tc::mbar_expect_tx(&full[s], a_bytes + b_bytes);
-        tc::bulk_g2s(A_s + (size_t)s * a_bytes, a.M + ((size_t)dt * a.KT + kt) * a_bytes, a_bytes, &full[s]);
-        tc::bulk_g2s(B_s + (size_t)s * b_bytes, a.y + ((size_t)nt * a.KT + kt) * b_bytes, b_bytes, &full[s]);
+        tc::bulk_g2s(A_s + (size_t)s * a_bytes, msrc, a_bytes, &full[s]);
+        tc::bulk_g2s(B_s + (size_t)s * b_bytes, ybase + (size_t)kt * b_bytes, b_bytes, &full[s]);
+        msrc += a_bytes;
+        if (++kt == a.KT) kt = 0;
+        if (++s == a.stages) {
+          s = 0;
+          ph ^= 1u;
+        }
       }
       // copies still in flight land before this CTA may exit
       const int issued = i;
@@ -91,33 +99,40 @@ __global__ void __launch_bounds__(kOutThreads, 1) k_outproj_tc(OutArgs a) {
   } else if (warp == 1) {
     if (lane == 0) {
       const uint32_t idesc = tc::idesc_f16(128, a.NB, false, false, false);
-      int i = 0, seg = 0;
+      // descriptors as (low, high) halves, stepped in 16-byte units on the low half
+      const uint64_t a0 = tc::sdesc_sw128(tc::smem_u32(A_s), 0, 1024), b0 = tc::sdesc_sw128(tc::smem_u32(B_s), 0, 1024);
+      const uint32_t a_lo0 = tc::desc_lo(a0), b_lo0 = tc::desc_lo(b0), d_hi = tc::desc_hi(a0);
+      int i = 0, seg = 0, s = 0;
+      uint32_t ph = 0;
+      int kt = (int)(u0 % a.KT);
       bool first = true;
       for (long long u = u0; u < u1 && !abort_flag; ++u, ++i) {
-        const int s = i % a.stages;
         const int acc = seg & 1;
         if (first && !tc::mbar_wait(&acc_free[acc], (((uint32_t)seg >> 1) & 1u) ^ 1u, a.status)) {
           abort_flag = 1;
           break;
         }
-        if (!tc::mbar_wait(&full[s], (uint32_t)(i / a.stages) & 1u, a.status)) {
+        if (!tc::mbar_wait(&full[s], ph, a.status)) {
           abort_flag = 1;
           break;
         }
         tc::tc_fence_after();
         const uint32_t d = tmem + (uint32_t)(acc * a.NB);
-        const uint32_t abase = tc::smem_u32(A_s + (size_t)s * a_bytes);
-        const uint32_t bbase = tc::smem_u32(B_s + (size_t)s * b_bytes);
+        const uint32_t alo = a_lo0 + (uint32_t)s * (a_bytes >> 4), blo = b_lo0 + (uint32_t)s * (b_bytes >> 4);
 #pragma unroll
         for (int k = 0; k < 4; ++k)
-          tc::mma_f16_ss(d, tc::sdesc_sw128(abase + 32 * k, 0, 1024), tc::sdesc_sw128(bbase + 32 * k, 0, 1024),
-                         idesc, (first && k == 0) ? 0u : 1u);
+          tc::mma_f16_ss2(d, alo + 2u * k, d_hi, blo + 2u * k, d_hi, idesc, (first && k == 0) ? 0u : 1u);
         tc::mma_commit(&empty[s]);
         first = false;
-        if (u + 1 == u1 || (u + 1) % a.KT == 0) {
+        if (++kt == a.KT) kt = 0;
+        if (u + 1 == u1 || kt == 0) {
           tc::mma_commit(&seg_done[acc]);
           ++seg;
           first = true;
+        }
+        if (++s == a.stages) {
+          s = 0;
+          ph ^= 1u;
         }
       }
       tc::mma_commit(&fin);
