@@ -207,6 +207,29 @@ def phase_bytes(spec, B, ctx):
             2 * spec.n_heads * spec.value_rank * spec.hidden + B * spec.hidden * 2]
 
 
+def measured_traffic(phase, tokens):
+    """DRAM bytes of one launch of the phase's main kernel, from the ncu capture
+    recorded in profiles/dram_traffic.json and scaled by cached tokens; None when
+    there is no capture or the kernel's sources changed since it was taken."""
+    import hashlib
+    try:
+        rec = json.load(open(os.path.join(ROOT, "profiles", "dram_traffic.json")))
+    except (OSError, ValueError):
+        return None
+    csrc = os.path.join(ROOT, "decode_attention_rank_b200", "csrc")
+    for name, k in rec.get("kernels", {}).items():
+        if k.get("phase") != phase:
+            continue
+        h = hashlib.sha1()
+        for f in [name + ".cu", "tc_common.cuh", "starkv_internal.cuh"]:
+            with open(os.path.join(csrc, f), "rb") as fh:
+                h.update(fh.read())
+        if h.hexdigest() != k.get("source_sha1"):
+            return None
+        return (k["dram_read_bytes"] + k["dram_write_bytes"]) * tokens / k["tokens"]
+    return None
+
+
 def decode_bytes(spec, L, B, ctx):
     """Algorithmic HBM bytes of one decode step: cache + B'_k + M + q/out."""
     return B * ctx * L.bytes_per_token + L.factor_bytes + B * (spec.n_heads * spec.head_dim + spec.hidden) * 2
@@ -359,7 +382,8 @@ def run_ours(args, rank, ws, local):
         "us_per_layer_step": ms_step * 1e3,
         "decode_us": dec_ms * 1e3,
         "roofline": {"bound": "hbm", "kernel": PHASES[dom], "achieved": kernels[dom]["GB/s"], "peak": peak,
-                     "peak_kind": peak_kind, "unit": "GB/s", "frac": kernels[dom]["frac"], "traffic": None,
+                     "peak_kind": peak_kind, "unit": "GB/s", "frac": kernels[dom]["frac"],
+                     "traffic": measured_traffic(dom, B * (T0 + W + K // 2)),
                      "algorithmic_bytes": pbytes[dom], "us_per_launch": ph_ms[dom] * 1e3,
                      "whole_decode": {"achieved": achieved, "frac": achieved / peak, "algorithmic_bytes": dbytes,
                                       "us": dec_ms * 1e3}},
