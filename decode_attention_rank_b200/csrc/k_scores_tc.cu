@@ -24,8 +24,8 @@
 //               128-token tile.  A thread scores its token for every head of
 //               the item (TMEM -> registers, dot with the 4/3-bit codes), and
 //               the warp takes the softmax statistics of its 32-token group
-//               in registers: m = max s, P = exp2(s - m) as fp16, l = sum P
-// Outputs per (sequence, head): P (fp16), and per 32-token group m and l = sum P.
+//               in registers: m = max s and P = exp2(s - m) as fp16
+// Outputs per (sequence, head): P (fp16), and the maximum m of every 32-token group.
 #include <float.h>
 #include <math.h>
 
@@ -63,7 +63,6 @@ struct ScoreArgs {
   __half* P;               // [B][H][P_ld]
   long long P_ld;
   float* m_st;             // [B][H][n_g] per 32-token group
-  float* l_st;
   int n_g;
   float* S_dbg;            // optional raw scores [B][H][P_ld]
   int H;
@@ -226,15 +225,18 @@ __device__ __forceinline__ float head_score_any(uint32_t taddr, const uint8_t* b
   }
 }
 
-// Warp-wide maximum and integer sum in one instruction each.
+// 2^x for x <= 0 (hardware approximation, relative error about 2^-22; the
+// result is rounded to fp16 next).
+__device__ __forceinline__ float ex2_approx(float x) {
+  float r;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(x));
+  return r;
+}
+
+// Warp-wide maximum in one instruction.
 __device__ __forceinline__ float warp_max(float x) {
   float r;
   asm volatile("redux.sync.max.f32 %0, %1, 0xffffffff;" : "=f"(r) : "f"(x));
-  return r;
-}
-__device__ __forceinline__ int warp_sum(int x) {
-  int r;
-  asm volatile("redux.sync.add.s32 %0, %1, 0xffffffff;" : "=r"(r) : "r"(x));
   return r;
 }
 
@@ -450,29 +452,21 @@ __global__ void __launch_bounds__(kScoreThreads, 1) k_scores_tc(ScoreArgs a) {
         if (ok) {
           const uint8_t* page = K_s + (size_t)ks * a.k_stage + (size_t)pg * item.key_bytes;
           const uint32_t trow = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(set * 128);
-          for (int hh = 0; hh < item.nh; ++hh) {
+          const size_t row0 = (size_t)b * a.H + item.h0;
+          __half* prow = a.P + row0 * a.P_ld + t;                          // this token's P of the item's first head
+          float* mrow = a.m_st + row0 * a.n_g + (t0 >> 5) + grp32;
+          for (int hh = 0; hh < item.nh; ++hh, prow += a.P_ld, mrow += a.n_g) {
             const ScoreHead& hd = heads_s[item.h0 + hh];
             const float sv = head_score_any(trow + (uint32_t)hd.gcol, page + hd.blk_rel, hd, slot);
-            const size_t row = (size_t)b * a.H + item.h0 + hh;
             if (a.S_dbg) {
-              if (valid) a.S_dbg[row * a.P_ld + t] = sv;
+              if (valid) a.S_dbg[(row0 + hh) * a.P_ld + t] = sv;
               continue;
             }
-            // softmax statistics of the 32-token group: m = max s, P = exp2(s - m)
-            // rounded to fp16, l = sum of the fp16 P (exact: each P is a multiple
-            // of 2^-24, summed as integers)
+            // softmax statistics of the 32-token group: m = max s and P =
+            // exp2(s - m) rounded to fp16 (the value kernel sums the P it uses)
             const float m = warp_max(valid ? sv : -FLT_MAX);
-            int pi = 0;
-            if (valid) {
-              const __half pb = __float2half_rn(exp2f(sv - m));
-              a.P[row * a.P_ld + t] = pb;
-              pi = __float2int_rn(__half2float(pb) * 16777216.f);
-            }
-            const int ps = warp_sum(pi);
-            if (lane == 0) {
-              a.m_st[row * a.n_g + (t0 >> 5) + grp32] = m;
-              a.l_st[row * a.n_g + (t0 >> 5) + grp32] = (float)ps * (1.f / 16777216.f);
-            }
+            if (valid) *prow = __float2half_rn(ex2_approx(sv - m));
+            if (lane == 0) *mrow = m;
           }
         }
         tc::tc_fence_before();
@@ -672,7 +666,7 @@ size_t scores_tc_ws_bytes(const starkv_layer* L, int batch, int max_len) {
   const size_t P_ld = (size_t)n_st * kSuper;
   auto r = [](size_t x) { return (x + 255) / 256 * 256; };
   return r((size_t)batch * L->w_stride) + r(2 * (size_t)batch * L->view.H * P_ld) +
-         2 * r(sizeof(float) * (size_t)batch * L->view.H * (P_ld / 32));
+         r(sizeof(float) * (size_t)batch * L->view.H * (P_ld / 32));
 }
 
 cudaError_t launch_scores_tc(const starkv_layer* L, const uint8_t* pool, long long n_pages, const int32_t* pt,
@@ -691,8 +685,6 @@ cudaError_t launch_scores_tc(const starkv_layer* L, const uint8_t* pool, long lo
   w += r(2 * (size_t)batch * v.H * n_st * kSuper);
   out->n_g = n_st * (kSuper / 32);
   out->m_st = (float*)w;
-  w += r(sizeof(float) * (size_t)batch * v.H * out->n_g);
-  out->l_st = (float*)w;
   k_qprep_tc<<<dim3(batch, (unsigned)L->items.size()), 512, 0, s>>>(
       v, (const __nv_bfloat16*)q, seq_lens, q_pos, L->Bk, L->d_key_off, L->d_items, L->w_stride, W);
   cudaError_t e = cudaGetLastError();
@@ -719,7 +711,6 @@ cudaError_t launch_scores_tc(const starkv_layer* L, const uint8_t* pool, long lo
   a.P = out->P;
   a.P_ld = out->P_ld;
   a.m_st = out->m_st;
-  a.l_st = out->l_st;
   a.n_g = out->n_g;
   a.S_dbg = S_dbg;
   a.H = v.H;

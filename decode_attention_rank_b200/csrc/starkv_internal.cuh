@@ -87,7 +87,6 @@ struct ScoreHead {
 struct ScoreOut {
   __half* P;          // [B][H][P_ld] exp2(s - m) with m the maximum of the token's 32-token group, fp16
   float* m_st;        // [B][H][n_g] per 32-token group
-  float* l_st;        // [B][H][n_g] sum of the fp16 P values of the group
   long long P_ld;
   int n_st;           // 256-token super-tiles per sequence
   int n_g;            // 32-token groups per sequence
