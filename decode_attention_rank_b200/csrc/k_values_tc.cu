@@ -17,10 +17,10 @@
 //   warp 0      tcgen05.mma issue, TMEM allocation
 //   warps 1-4   P staging: rescaled fp16 P tiles (the B operand), M and l;
 //               warp s takes the 32-token group s of every tile
-//   warp 5      bulk copies of the pages' value blocks, 32 tokens at a time
+//   warp 5      bulk copies of the pages' value blocks, a page at a time
 //   warps 6-21  workers: worker w dequantizes items w, w + 16, ... (an item =
-//               32 tokens x 128 value channels, a lane per token) from the
-//               copied pages into A stage w, and reads Y^T out of TMEM at the
+//               one page's 16 tokens x 128 value channels) from the
+//               copied pages into its two A stages, and reads Y^T out of TMEM at the
 //               end of each run
 #include <float.h>
 
@@ -33,17 +33,17 @@ namespace {
 constexpr int kValWorkers = 16;                          // dequantizing warps
 constexpr int kStagers = 4;                              // P staging warps, one per 32-token group of a tile
 constexpr int kValThreads = 32 * (2 + kStagers + kValWorkers);   // MMA, P staging, page copies, workers
-// A stages: item n sits in stage n % kAStages, and worker w takes the items
-// n = w (mod kValWorkers), so each stage has one writer and a worker is never
-// more than one barrier phase ahead of the stage it writes.
-constexpr int kAStages = kValWorkers;
-// Raw 32-token chunks (two pages' value blocks) in flight.  A worker's
-// consecutive items lie at most max(4, 16 / nblk) chunks apart; at least that
-// many raw stages keep a worker within one barrier phase of the raw stage it
-// reads.
-constexpr int kMaxRawStages = 16;
+// A stages: item n sits in stage n % kAStages and worker w takes the items
+// n = w (mod kValWorkers), so each stage has one writer, every worker owns two
+// stages, and a worker is never more than one barrier phase ahead of a stage.
+constexpr int kAStages = 2 * kValWorkers;
+// Raw stages: page p of the CTA's tiles (the value block of 16 tokens) lands
+// in stage p % n_raw.  A worker's consecutive items lie 32 / nblk pages apart;
+// at least that many raw stages keep a worker within one barrier phase of the
+// raw stage it reads.
+constexpr int kMaxRawStages = 32;
 constexpr int kVSuper = 256;     // tokens per super-tile (matches the score kernel)
-constexpr int kAStage = 8192;    // one A stage: 32 tokens x 128 value channels, fp16
+constexpr int kAStage = 4096;    // one A stage: 16 tokens (one page) x 128 value channels, fp16
 constexpr int kMaxRuns = 64;     // runs (sequences) per CTA
 constexpr int kRunMaxCache = 16; // runs whose per-head maxima are computed up front
 
@@ -62,8 +62,8 @@ struct ValArgs {
   int max_pages;
   const int32_t* seq_lens;
   int vblk_off, vblk_bytes;     // value latent block inside a page
-  int raw_stage;                // bytes of one raw chunk stage (two value blocks, 16-byte aligned)
-  int n_raw;                    // raw chunk stages (2 .. kMaxRawStages)
+  int raw_stage;                // bytes of one raw stage (a page's value block, 128-byte aligned)
+  int n_raw;                    // raw stages
   const GroupDesc* vgrp;        // value latent groups (all of 32 channels)
   int rv, H;
   int lg_nblk;                  // log2 of the 128-channel blocks of the value latent
@@ -129,9 +129,9 @@ __device__ __forceinline__ uint4 deq8_b3(uint32_t run, __half2 sub, __half2 s2) 
 
 __global__ void __launch_bounds__(kValThreads, 1) k_values_tc(ValArgs a) {
   extern __shared__ uint8_t smem_raw[];
-  // chain c = items 4 c .. 4 c + 3 (one 128-channel block of a tile, four
-  // workers, A stages (4 c .. 4 c + 3) % kAStages): ch_full[c % 4] when the
-  // four are written, ch_done[c % 4] when their MMAs have completed
+  // chain c = items 8 c .. 8 c + 7 (eight workers, A stages (8 c .. 8 c + 7)
+  // % kAStages): ch_full[c % 4] when the eight are written, ch_done[c % 4]
+  // when their MMAs have completed
   __shared__ __align__(8) uint64_t ch_full[4], ch_done[4], r_full[kMaxRawStages], r_empty[kMaxRawStages];
   __shared__ __align__(8) uint64_t p_full[2], p_empty[2];
   __shared__ __align__(8) uint64_t seg_done, acc_free, fin;
@@ -147,24 +147,24 @@ __global__ void __launch_bounds__(kValThreads, 1) k_values_tc(ValArgs a) {
   uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   uint8_t* A_s = smem;                                   // kAStages x 8 KB A stages
   uint8_t* P_s = A_s + kAStages * kAStage;               // 2 x (H x 128 fp16, K-major swizzled)
-  uint8_t* R_s = P_s + 2 * a.H * 256;                    // n_raw raw chunks
+  uint8_t* R_s = P_s + 2 * a.H * 256;                    // n_raw raw stages
   const int p_stage = a.H * 256;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int G = gridDim.x, cta = blockIdx.x;
   const long long u0 = vunit_lo(cta, G, a.U), u1 = vunit_lo(cta + 1, G, a.U);
   const int lnb = a.lg_nblk;                             // 128-channel blocks: 1 << lnb
   const int nblk = 1 << lnb;
-  const int lg_ipt = lnb + 2;                            // worker items per tile: 4 * nblk
+  const int lg_ipt = lnb + 3;                            // worker items per tile: 8 * nblk
   const int b_first = (int)(u0 / a.n_st);
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < 4; ++s) {
-      tc::mbar_init(&ch_full[s], 4);
+      tc::mbar_init(&ch_full[s], 8);
       tc::mbar_init(&ch_done[s], 1);
     }
     for (int s = 0; s < a.n_raw; ++s) {
       tc::mbar_init(&r_full[s], 1);
-      tc::mbar_init(&r_empty[s], 1 << a.lg_nblk);   // the chunk's items, one per 128-channel block
+      tc::mbar_init(&r_empty[s], 1 << a.lg_nblk);   // the page's items, one per 128-channel block
     }
     for (int s = 0; s < 2; ++s) {
       tc::mbar_init(&p_full[s], kStagers);
@@ -257,11 +257,12 @@ __global__ void __launch_bounds__(kValThreads, 1) k_values_tc(ValArgs a) {
 
   if (warp == 0) {
     // ------------------------------------------------ MMA issue
-    // Item n of the CTA (tile n / ipt, item n % ipt = 4 cb + k) sits in A
-    // stage n % kAStages; its two K = 16 steps add block cb's Y^T.  The four
-    // items of a block are waited for together and their eight MMAs issued
-    // back to back: an N = 32 MMA takes only about 45 cycles on the tensor
-    // pipe, so the issuing thread must spend very few instructions per MMA.
+    // Item n of the CTA (tile n / ipt, item n % ipt = nblk k + cb: page k of
+    // the tile, 128-channel block cb) sits in A stage n % kAStages; its one
+    // K = 16 MMA adds block cb's Y^T.  A chain's eight items are waited for
+    // together and their MMAs issued back to back: an N = 32 MMA takes only
+    // about 45 cycles on the tensor pipe, so the issuing thread must spend
+    // very few instructions per MMA.
     if (lane == 0) {
       const uint32_t idesc = tc::idesc_f16(128, a.H, false, true, false);
       // descriptors as (low, high) halves; steps are 16-byte units on the low half
@@ -288,21 +289,20 @@ __global__ void __launch_bounds__(kValThreads, 1) k_values_tc(ValArgs a) {
         tc::tc_fence_after();
         const uint32_t b_lo = b_lo0 + (uint32_t)ps * p_step;
         bool ok = true;
-        for (int cb = 0; cb < nblk && ok; ++cb, n += 4) {
-          // the chain's four items, then its eight MMAs back to back and one commit
-          const int c = n >> 2;
+        for (int x0 = 0; x0 < (1 << lg_ipt) && ok; x0 += 8, n += 8) {
+          const int c = n >> 3;
           ok = tc::mbar_wait_ab(&ch_full[c & 3], ((uint32_t)(c >> 2)) & 1u, a.status, &abort_flag);
           if (!ok) break;
           tc::tc_fence_after();
-          const uint32_t d = tmem + (uint32_t)(cb * a.H);
+          // the chain's stages are (n .. n + 7) % kAStages: n is a multiple of 8, no wrap
           const uint32_t a_lo = a_lo0 + (uint32_t)(n % kAStages) * (kAStage >> 4);
 #pragma unroll
-          for (int k = 0; k < 4; ++k) {
-            // tokens 32 k .. 32 k + 31: 16-token steps 2 k and 2 k + 1 of the P tile; stages wrap at kAStages
-            const uint32_t ak = a_lo + (uint32_t)(((n + k) % kAStages) - (n % kAStages)) * (kAStage >> 4);
-            const uint32_t bk = b_lo + (uint32_t)(k >> 1) * b_atom + (uint32_t)(k & 1) * 4u;
-            tc::mma_f16_ss2(d, ak, a_hi, bk, b_hi, idesc, (first && k == 0) ? 0u : 1u);
-            tc::mma_f16_ss2(d, ak + (4096u >> 4), a_hi, bk + 2u, b_hi, idesc, 1u);
+          for (int i = 0; i < 8; ++i) {
+            const int x = x0 + i, k = x >> lnb, cb = x & (nblk - 1);
+            // tokens 16 k .. 16 k + 15: K = 16 step k of the P tile
+            tc::mma_f16_ss2(tmem + (uint32_t)(cb * a.H), a_lo + (uint32_t)i * (kAStage >> 4), a_hi,
+                            b_lo + (uint32_t)(k >> 2) * b_atom + (uint32_t)(k & 3) * 2u, b_hi, idesc,
+                            (first && k == 0) ? 0u : 1u);
           }
           tc::mma_commit(&ch_done[c & 3]);
         }
@@ -423,33 +423,31 @@ __global__ void __launch_bounds__(kValThreads, 1) k_values_tc(ValArgs a) {
   } else if (warp == kStagers + 1) {
 
     // ------------------------------------------------ page copies
-    // Chunk c = 4 T + k (tokens 32 k .. 32 k + 31 of tile T): the value blocks
-    // of its two pages into raw stage c % n_raw.
+    // Page p = 8 T + k (tokens 16 k .. 16 k + 15 of tile T): its value block
+    // into raw stage p % n_raw.
     if (lane == 0) {
-      const int n_chunks = n_tiles * 4;
-      for (int c = 0; c < n_chunks; ++c) {
-        const int rs = c % a.n_raw;
-        if (!tc::mbar_wait_ab(&r_empty[rs], (((uint32_t)(c / a.n_raw)) & 1u) ^ 1u, a.status, &abort_flag)) break;
-        const int p0 = pid_s[c >> 2][2 * (c & 3)], p1 = pid_s[c >> 2][2 * (c & 3) + 1];
-        tc::mbar_expect_tx(&r_full[rs], (uint32_t)(((p0 >= 0) + (p1 >= 0)) * a.vblk_bytes));
-        uint8_t* dst = R_s + (size_t)rs * a.raw_stage;
-        if (p0 >= 0)
-          tc::bulk_g2s(dst, a.pool + (size_t)p0 * a.page_bytes + a.vblk_off, (uint32_t)a.vblk_bytes, &r_full[rs]);
-        if (p1 >= 0)
-          tc::bulk_g2s(dst + a.vblk_bytes, a.pool + (size_t)p1 * a.page_bytes + a.vblk_off, (uint32_t)a.vblk_bytes,
-                       &r_full[rs]);
+      const int n_pg = n_tiles * 8;
+      for (int pg = 0; pg < n_pg; ++pg) {
+        const int rs = pg % a.n_raw;
+        if (!tc::mbar_wait_ab(&r_empty[rs], (((uint32_t)(pg / a.n_raw)) & 1u) ^ 1u, a.status, &abort_flag)) break;
+        const int page = pid_s[pg >> 3][pg & 7];
+        tc::mbar_expect_tx(&r_full[rs], page >= 0 ? (uint32_t)a.vblk_bytes : 0u);
+        if (page >= 0)
+          tc::bulk_g2s(R_s + (size_t)rs * a.raw_stage, a.pool + (size_t)page * a.page_bytes + a.vblk_off,
+                       (uint32_t)a.vblk_bytes, &r_full[rs]);
       }
       // let copies in flight land before the CTA can exit
-      for (int c = max(0, n_chunks - a.n_raw); c < n_chunks; ++c)
-        tc::mbar_wait(&r_full[c % a.n_raw], ((uint32_t)(c / a.n_raw)) & 1u, a.status);
+      for (int pg = max(0, n_pg - a.n_raw); pg < n_pg; ++pg)
+        tc::mbar_wait(&r_full[pg % a.n_raw], ((uint32_t)(pg / a.n_raw)) & 1u, a.status);
     }
     __syncwarp();
   } else {
     // ------------------------------------------------ workers: codes -> A stages, run epilogues
     // Worker w takes the CTA's items w, w + 16, w + 32, ...; item n is item
-    // x = n % ipt = 4 cb + k of tile T = n / ipt: value channels
-    // [128 cb, 128 cb + 128) of tokens 32 k .. 32 k + 31, read from raw chunk
-    // 4 T + k and dequantized (a lane per token) into A stage n % kAStages.
+    // x = n % ipt = nblk k + cb of tile T = n / ipt: value channels
+    // [128 cb, 128 cb + 128) of page k (tokens 16 k .. 16 k + 15), read from
+    // raw stage (8 T + k) % n_raw and dequantized into A stage n % kAStages;
+    // lane l takes token l % 16 and the 64 channels of half l / 16.
     const int w = warp - 2 - kStagers;
     const int q = warp & 3, part = w >> 2;   // epilogue: TMEM lane quarter, column part
     const int n_items = n_tiles << lg_ipt;
@@ -476,29 +474,30 @@ __global__ void __launch_bounds__(kValThreads, 1) k_values_tc(ValArgs a) {
       __syncwarp();
       if (lane == 0) tc::mbar_arrive(&acc_free);
     };
-    const uint32_t x7 = (uint32_t)(lane & 7);
-    const int slot = lane & 15;
+    const int slot = lane & 15, half = lane >> 4;
+    const uint32_t x7 = (uint32_t)(slot & 7);
+    const size_t st_off = (size_t)(slot >> 3) * 2048 + (size_t)half * 1024 + (size_t)(slot & 7) * 128;
     for (int n = w; n < n_items; n += kValWorkers) {
       const int T = n >> lg_ipt;
       const int run = tile_s[T].w;
       while (epi_run < run && epi_run < n_runs) epilogue(epi_run++);
       const int x = n & ((1 << lg_ipt) - 1);
-      const int c = T * 4 + (x & 3);          // raw chunk
-      const int cb = x >> 2;
-      const int rs = c % a.n_raw, as = n % kAStages;
-      const bool valid = pid_s[T][2 * (c & 3) + (lane >> 4)] >= 0;
-      // A stage first: once item n - 16 is consumed, every chunk up to its
-      // chunk has landed; with at least max(4, 16 / nblk) raw stages the raw
-      // stage is then at most one phase from chunk c
-      const int ch = n >> 2;                   // chain of this item; the worker's previous item was in chain ch - 4
+      const int k = x >> lnb, cb = x & (nblk - 1);
+      const int pg = T * 8 + k;                // page of the CTA's tiles
+      const int rs = pg % a.n_raw, as = n % kAStages;
+      const bool valid = pid_s[T][k] >= 0;
+      // A stage first: the stage's previous item was in chain ch - 4; once that
+      // chain is consumed every page up to it has landed, and with at least
+      // 32 / nblk raw stages the raw stage is then at most one phase from pg
+      const int ch = n >> 3;                   // chain of this item
       const bool ok = tc::mbar_wait_ab(&ch_done[ch & 3], (((uint32_t)(ch >> 2)) & 1u) ^ 1u, a.status, &abort_flag) &&
-                      tc::mbar_wait_ab(&r_full[rs], ((uint32_t)(c / a.n_raw)) & 1u, a.status, &abort_flag);
+                      tc::mbar_wait_ab(&r_full[rs], ((uint32_t)(pg / a.n_raw)) & 1u, a.status, &abort_flag);
       if (ok) {
-        const uint8_t* blk = R_s + (size_t)rs * a.raw_stage + (size_t)(lane >> 4) * a.vblk_bytes;
-        uint8_t* st = A_s + (size_t)as * kAStage + (lane >> 3) * 2048 + (lane & 7) * 128;
+        const uint8_t* blk = R_s + (size_t)rs * a.raw_stage;
+        uint8_t* st = A_s + (size_t)as * kAStage + st_off;
 #pragma unroll
-        for (int gg = 0; gg < 4; ++gg) {
-          const int g = cb * 4 + gg;
+        for (int gg = 0; gg < 2; ++gg) {
+          const int g = cb * 4 + half * 2 + gg;
           const int4 vg = vg_s[g];
           const __half hs = valid ? reinterpret_cast<const __half*>(blk)[g * kPage + slot] : __ushort_as_half(0);
           const __half2 s2 = __halves2half2(hs, hs);
@@ -518,12 +517,11 @@ __global__ void __launch_bounds__(kValThreads, 1) k_values_tc(ValArgs a) {
             o2 = deq8_b3(__funnelshift_r(w1, w2, 16), sub, s2);
             o3 = deq8_b3(w2 >> 8, sub, s2);
           }
-          uint8_t* at = st + (gg >> 1) * 1024;
-          const uint32_t c4 = (uint32_t)(gg & 1) * 4u;   // 8-channel chunk of this group in its atom
-          *reinterpret_cast<uint4*>(at + (((c4 + 0u) ^ x7) << 4)) = o0;
-          *reinterpret_cast<uint4*>(at + (((c4 + 1u) ^ x7) << 4)) = o1;
-          *reinterpret_cast<uint4*>(at + (((c4 + 2u) ^ x7) << 4)) = o2;
-          *reinterpret_cast<uint4*>(at + (((c4 + 3u) ^ x7) << 4)) = o3;
+          const uint32_t c4 = (uint32_t)gg * 4u;   // 8-channel chunk of this group in the half's atom
+          *reinterpret_cast<uint4*>(st + (((c4 + 0u) ^ x7) << 4)) = o0;
+          *reinterpret_cast<uint4*>(st + (((c4 + 1u) ^ x7) << 4)) = o1;
+          *reinterpret_cast<uint4*>(st + (((c4 + 2u) ^ x7) << 4)) = o2;
+          *reinterpret_cast<uint4*>(st + (((c4 + 3u) ^ x7) << 4)) = o3;
         }
       }
       tc::fence_proxy_async();
@@ -636,7 +634,7 @@ __global__ void k_values_combine(const float* __restrict__ Y, const float* __res
 }  // namespace
 
 // Dynamic shared memory of the value kernel: the A stages and two P stages.
-static size_t values_raw_stage(int vblk_bytes) { return (size_t)(2 * vblk_bytes + 127) / 128 * 128; }
+static size_t values_raw_stage(int vblk_bytes) { return (size_t)(vblk_bytes + 127) / 128 * 128; }
 static size_t values_smem(int H, int vblk_bytes, int n_raw) {
   return (size_t)kAStages * kAStage + 2 * (size_t)H * 256 + n_raw * values_raw_stage(vblk_bytes) + 1024;
 }
@@ -680,7 +678,7 @@ bool plan_values_tc(starkv_layer* L) {
   // least 16 / nblk of them
   cudaFuncAttributes fa;
   if (cudaFuncGetAttributes(&fa, k_values_tc) != cudaSuccess) return false;
-  const int min_raw = std::max(4, kValWorkers / (v.rv / 128));
+  const int min_raw = std::max(4, 32 / (v.rv / 128));
   L->val_raw = 0;
   for (int n_raw = kMaxRawStages; n_raw >= min_raw && !L->val_raw; --n_raw)
     if (values_smem(v.H, L->vblk_bytes, n_raw) + fa.sharedSizeBytes <= 232448) L->val_raw = n_raw;
