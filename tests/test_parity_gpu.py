@@ -243,3 +243,33 @@ def test_device_status_bad_page():
     L.append(cache.pool, cache.n_pages, cache.page_table, torch.zeros(1, dtype=torch.int32, device="cuda"),
              torch.tensor([cache.page_table.shape[1] * 16], dtype=torch.int32, device="cuda"), z, True)
     assert L.sync_status() & 0x2
+
+
+def test_phase_timing_leaves_results_unchanged():
+    """starkv_profile_decode records per-kernel times without changing the output."""
+    c = case(2)
+    L = c.load()
+    lens = [600, 257, 33]
+    cache = GpuCache(L, lens, seed=3)
+    for b, T in enumerate(lens):
+        cache.append_latents(b, c.latents_direct(b, T))
+    B = len(lens)
+    q = torch.from_numpy(queries(c, B)[:, 0]).cuda().to(torch.bfloat16)
+    ws = torch.empty(L.workspace_bytes(B, cache.page_table.shape[1] * 16), dtype=torch.uint8, device="cuda")
+    seq_lens = torch.tensor(lens, dtype=torch.int32, device="cuda")
+    outs = []
+    for prof in (0, 3):
+        L.profile_decode(prof)
+        out = torch.empty(B, c.spec.hidden, device="cuda", dtype=torch.bfloat16)
+        for _ in range(3):
+            L.decode(cache.pool, cache.n_pages, cache.page_table, seq_lens, q, out, ws)
+        torch.cuda.synchronize()
+        outs.append(out.float().cpu().numpy())
+        if prof:
+            ms = L.decode_phase_ms(3)
+            assert len(ms) == 3 and all(len(m) == 4 for m in ms)
+            assert all(t > 0.0 for m in ms for t in m), ms
+            assert all(sum(m) < 1000.0 for m in ms), ms
+    L.profile_decode(0)
+    assert L.sync_status() == 0
+    np.testing.assert_array_equal(outs[0], outs[1])
