@@ -108,7 +108,7 @@ __device__ __forceinline__ float group_dot(const uint32_t* w, uint32_t sh, float
   constexpr int NR = (N * B + 31) / 32;
   uint32_t run[NR];
 #pragma unroll
-  for (int k = 0; k < NR; ++k) run[k] = __funnelshift_r(w[k], w[k + 1], sh);
+  for (int k = 0; k < NR; ++k) run[k] = (N * B) % 32 == 0 ? w[k] : __funnelshift_r(w[k], w[k + 1], sh);
   float2 acc = make_float2(0.f, 0.f), gs = acc;
   group_pairs<B, C>(run, G, acc, gs, std::make_integer_sequence<int, N / 2>{});
   float a = acc.x + acc.y, g = gs.x + gs.y;
@@ -178,9 +178,12 @@ __device__ __forceinline__ float segment_dot(uint32_t taddr, const uint8_t* blk,
     tmem_cols<0, N>(taddr + (uint32_t)(C0 + g * 32), G);
     const uint32_t bit0 = (uint32_t)slot * (uint32_t)(N * B);
     const uint32_t* w = reinterpret_cast<const uint32_t*>(blk + hd.code_off[G0 + g]) + (bit0 >> 5);
+    // a group whose per-token code run is a whole number of words starts on a
+    // word boundary for every token: no re-alignment, no extra word
+    constexpr int NW = (N * B) % 32 == 0 ? NR : NR + 1;
     uint32_t wr[NR + 1];
 #pragma unroll
-    for (int k = 0; k <= NR; ++k) wr[k] = w[k];
+    for (int k = 0; k < NW; ++k) wr[k] = w[k];
     const float scale = __half2float(reinterpret_cast<const __half*>(blk)[(G0 + g) * kPage + slot]);
     tc::tmem_ld_wait();
     reg_fence<N>(G);
@@ -241,12 +244,14 @@ __device__ __forceinline__ float warp_max(float x) {
 }
 
 constexpr int kMaxItemHeads = 8;
+constexpr int kMaxStages = 8;        // W'' and key-page stages
 constexpr int kMaxHeads = 64;
 
 
 __global__ void __launch_bounds__(kScoreThreads, 1) k_scores_tc(ScoreArgs a) {
   extern __shared__ uint8_t smem_raw[];
-  __shared__ __align__(8) uint64_t w_full[4], w_empty[4], k_full[4], k_empty[4], e_full, e_empty;
+  __shared__ __align__(8) uint64_t w_full[kMaxStages], w_empty[kMaxStages], k_full[kMaxStages], k_empty[kMaxStages], e_full,
+      e_empty;
   __shared__ __align__(8) uint64_t acc_full[4], acc_free[4], fin;
   __shared__ uint32_t tmem_base;
   __shared__ volatile int abort_flag;
@@ -261,7 +266,7 @@ __global__ void __launch_bounds__(kScoreThreads, 1) k_scores_tc(ScoreArgs a) {
   const long long u0 = unit_lo(c, G, a.U), u1 = unit_lo(c + 1, G, a.U);
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < 4; ++s) {
+    for (int s = 0; s < kMaxStages; ++s) {
       tc::mbar_init(&w_full[s], 1);
       tc::mbar_init(&w_empty[s], 1);
       tc::mbar_init(&k_full[s], 1);
@@ -290,21 +295,33 @@ __global__ void __launch_bounds__(kScoreThreads, 1) k_scores_tc(ScoreArgs a) {
     // ------------------------------------------------------------ key copies
     // Warp-wide: lane 0 owns the barriers; every lane fetches one page id and
     // issues that page's copy, so no copy waits behind a page-table load.
+    // The sequence length and page ids of the next unit are loaded one unit
+    // ahead, so a unit's first copies do not wait behind them.
     int i = 0, nk = 0;                    // nk: issued stage fills (for the drain below)
+    int len_n = 0, page_n = 0;
+    auto load_unit = [&](long long uu) {
+      const int st = (int)(uu / a.batch), b = (int)(uu % a.batch);
+      const int pidx = st * (kSuper / kPage) + lane;
+      len_n = a.seq_lens[b];
+      page_n = (lane < kSuper / kPage && pidx < a.max_pages) ? a.pt[(size_t)b * a.max_pages + pidx] : 0;
+    };
+    if (u0 < u1) load_unit(u0);
     for (long long u = u0; u < u1; ++u) {
+      const int len = min(len_n, a.max_pages * kPage);
+      int page = page_n;
+      if (u + 1 < u1) load_unit(u + 1);
       if (__shfl_sync(0xffffffffu, abort_flag, 0)) break;
       const int st = (int)(u / a.batch), b = (int)(u % a.batch);
       const int t0 = st * kSuper;
-      const int len = min(a.seq_lens[b], a.max_pages * kPage);
       if (t0 >= len) continue;
       const int npg = min(kSuper / kPage, (len - t0 + kPage - 1) / kPage);
-      int page = 0;
       if (lane < npg) {
-        page = a.pt[(size_t)b * a.max_pages + st * (kSuper / kPage) + lane];
         if (page < 0 || page >= a.n_pages) {
           atomicOr(a.status, kBadPage);
           page = 0;
         }
+      } else {
+        page = 0;
       }
       const uint8_t* page_base = a.pool + (size_t)page * a.page_bytes;
       for (int it = 0; it < a.n_items; ++it, ++i) {
@@ -639,16 +656,11 @@ bool plan_scores_tc(starkv_layer* L) {
   cudaFuncAttributes fa;
   if (cudaFuncGetAttributes(&fa, k_scores_tc) != cudaSuccess) return false;
   const long long budget = 232448LL - (long long)fa.sharedSizeBytes - 1024 - 2LL * kETileBytes;
-  const int stages[5][2] = {{3, 4}, {3, 3}, {2, 4}, {2, 3}, {2, 2}};
-  L->WS = 0;
-  for (const auto& ws_ks : stages) {
-    if ((long long)ws_ks[0] * L->w_stage + (long long)ws_ks[1] * L->k_stage <= budget) {
-      L->WS = ws_ks[0];
-      L->KS = ws_ks[1];
-      break;
-    }
-  }
-  if (L->WS == 0) return false;
+  // Two W'' stages (read from L2, short latency) and as many key stages as fit:
+  // the key copies read HBM and need the most bytes in flight.
+  L->WS = 2;
+  L->KS = (int)std::min<long long>(kMaxStages, (budget - 2LL * L->w_stage) / L->k_stage);
+  if (L->KS < 2) return false;
   const int mp = c.max_positions > 0 ? c.max_positions : 32768;
   L->rope_tiles = (mp + kSuper - 1) / kSuper * (kSuper / 128);
   return true;
