@@ -179,35 +179,36 @@ __global__ void __launch_bounds__(kOutThreads, 1) k_outproj_tc(OutArgs a) {
 template <typename TO>
 __global__ void k_outproj_reduce(const float* __restrict__ part, int G, int KT, int DT, int slots, int NB, int rows,
                                  int D, TO* __restrict__ out) {
-  __shared__ long long seg_off[256];
-  __shared__ int n_seg;
+  __shared__ long long seg_off[512];
   const int dt = blockIdx.x, row = blockIdx.y;
   const int nt = row / NB, b = row % NB;
-  if (threadIdx.x == 0) {
-    const long long U = (long long)DT * KT;
-    const long long lo = (long long)dt * KT, hi = lo + KT;
-    int c = (int)((lo * G) / U);
-    while (c > 0 && unit_begin(c, G, U) > lo) --c;
-    while (unit_begin(c + 1, G, U) <= lo) ++c;
-    int n = 0;
-    long long b0 = unit_begin(c, G, U);
-    for (; c < G && b0 < hi && n < 256; ++c) {
-      const long long b1 = unit_begin(c + 1, G, U);
-      if (b1 > lo && b1 > b0) {
-        const int slot = dt - (int)(b0 / KT);
-        seg_off[n++] = ((((long long)nt * G + c) * slots + slot) * NB + b) * 128;
-      }
-      b0 = b1;
+  // The CTAs whose unit ranges [begin(c), begin(c + 1)) meet this output
+  // tile's k-range [lo, hi): candidates c_lo, c_lo + 1, ... tested one per
+  // thread (offset -1 for a CTA that holds none of it), kept in order of c.
+  const long long U = (long long)DT * KT;
+  const long long lo = (long long)dt * KT, hi = lo + KT;
+  const int c_lo = max(0, (int)((lo * G) / U) - 1);
+  const int c_hi = min(G, (int)((hi * G + U - 1) / U) + 1);
+  const int nc = min(c_hi - c_lo, 512);
+  for (int t = threadIdx.x; t < nc; t += blockDim.x) {
+    const int c = c_lo + t;
+    const long long b0 = unit_begin(c, G, U), b1 = unit_begin(c + 1, G, U);
+    long long off = -1;
+    if (b1 > b0 && b1 > lo && b0 < hi) {
+      const int slot = dt - (int)(b0 / KT);
+      off = ((((long long)nt * G + c) * slots + slot) * NB + b) * 128;
     }
-    n_seg = n;
+    seg_off[t] = off;
   }
   __syncthreads();
-  const int ns = n_seg;
   for (int n = threadIdx.x; n < 128; n += blockDim.x) {
     const int d = dt * 128 + n;
     if (d >= D) continue;
     float acc = 0.f;
-    for (int k = 0; k < ns; ++k) acc += part[seg_off[k] + n];
+    for (int k = 0; k < nc; ++k) {
+      const long long o = seg_off[k];
+      if (o >= 0) acc += part[o + n];
+    }
     out[(size_t)row * D + d] = (TO)acc;
   }
 }

@@ -544,90 +544,102 @@ __global__ void __launch_bounds__(kValThreads, 1) k_values_tc(ValArgs a) {
 __global__ void k_values_combine(const float* __restrict__ Y, const float* __restrict__ mseg,
                                  const float* __restrict__ lseg, int G, long long U, int n_st, int slots, int H,
                                  int rv, int NB, int KT, uint8_t* __restrict__ ytiles) {
-  // the runs of sequence b: partial slots of the CTAs whose unit ranges meet
-  // [b n_st, (b+1) n_st); their (M, l) are read in parallel, one per thread
-  __shared__ int seg_i[256];
-  __shared__ float seg_w[256];
-  __shared__ int n_seg, c_first;
-  __shared__ float red_s[8];
-  __shared__ float inv_den;
+  // The runs of sequence b are the partial slots of the CTAs whose unit
+  // ranges meet [b n_st, (b + 1) n_st).  Candidates c_lo, c_lo + 1, ... are
+  // tested one per thread, with their (M, l) read in parallel; a candidate
+  // that holds none of the sequence, or whose run saw no valid token, gets
+  // weight 0 and its Y is never read.
+  constexpr int kCand = 512;
+  __shared__ int seg_i[kCand];
+  __shared__ float seg_m[kCand], seg_w[kCand];
+  __shared__ float red_s[32];
+  __shared__ float bmax, inv_den;
   const int b = blockIdx.x, h = blockIdx.y;
+  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5, nw = (int)(blockDim.x >> 5);
   const long long lo = (long long)b * n_st, hi = lo + n_st;
-  if (threadIdx.x == 0) {
-    int c = (int)((lo * G) / U);
-    while (c > 0 && vunit_lo(c, G, U) > lo) --c;
-    while (vunit_lo(c + 1, G, U) <= lo) ++c;
-    int c1 = c;
-    while (c1 < G && vunit_lo(c1, G, U) < hi) ++c1;
-    c_first = c;
-    n_seg = min(c1 - c, 256);
-  }
-  __syncthreads();
-  const int nc = n_seg;
-  float mk = -FLT_MAX, lk = 0.f;
-  int ik = -1;
-  if ((int)threadIdx.x < nc) {
-    const int c = c_first + threadIdx.x;
+  const int c_lo = max(0, (int)((lo * G) / U) - 1);
+  const int c_hi = min(G, (int)((hi * G + U - 1) / U) + 1);
+  const int nc = min(c_hi - c_lo, kCand);
+  float m = -FLT_MAX;
+  for (int t = threadIdx.x; t < nc; t += blockDim.x) {
+    const int c = c_lo + t;
     const long long b0 = vunit_lo(c, G, U), b1 = vunit_lo(c + 1, G, U);
-    if (b1 > b0) {
+    int ik = 0;
+    float mk = -FLT_MAX, lk = 0.f;
+    if (b1 > b0 && b1 > lo && b0 < hi) {
       ik = (c * slots + (b - (int)(b0 / n_st))) * H + h;
       lk = lseg[ik];
       mk = lk > 0.f ? mseg[ik] : -FLT_MAX;
     }
+    seg_i[t] = ik;
+    seg_m[t] = mk;
+    seg_w[t] = lk;
+    m = fmaxf(m, mk);
   }
   // block maximum of M over the runs with l > 0
-  float m = mk;
   for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-  if ((threadIdx.x & 31) == 0) red_s[threadIdx.x >> 5] = m;
+  if (lane == 0) red_s[wid] = m;
   __syncthreads();
-  m = -FLT_MAX;
-  for (int w = 0; w < (int)(blockDim.x >> 5); ++w) m = fmaxf(m, red_s[w]);
-  const float wk = (lk > 0.f) ? exp2f(mk - m) : 0.f;
-  if ((int)threadIdx.x < nc) {
-    seg_i[threadIdx.x] = ik < 0 ? 0 : ik;
-    seg_w[threadIdx.x] = wk;
+  if (threadIdx.x == 0) {
+    float x = -FLT_MAX;
+    for (int w = 0; w < nw; ++w) x = fmaxf(x, red_s[w]);
+    bmax = x;
   }
-  float dn = wk * lk;
-  for (int o = 16; o > 0; o >>= 1) dn += __shfl_xor_sync(0xffffffffu, dn, o);
   __syncthreads();
-  if ((threadIdx.x & 31) == 0) red_s[threadIdx.x >> 5] = dn;
+  const float M = bmax;
+  // weights exp2(M_r - M) and the denominator sum w_r l_r
+  float dn = 0.f;
+  for (int t = threadIdx.x; t < nc; t += blockDim.x) {
+    const float l = seg_w[t];
+    const float w = l > 0.f ? exp2f(seg_m[t] - M) : 0.f;
+    seg_w[t] = w;
+    dn += w * l;
+  }
+  for (int o = 16; o > 0; o >>= 1) dn += __shfl_xor_sync(0xffffffffu, dn, o);
+  if (lane == 0) red_s[wid] = dn;
   __syncthreads();
   if (threadIdx.x == 0) {
     float den = 0.f;
-    for (int w = 0; w < (int)(blockDim.x >> 5); ++w) den += red_s[w];
+    for (int w = 0; w < nw; ++w) den += red_s[w];
     inv_den = den > 0.f ? 1.f / den : 0.f;
   }
   __syncthreads();
-  const int ns = n_seg;
   const float idn = inv_den;
   const int nt = b / NB, r = b % NB;
-  for (int j = threadIdx.x; j < rv; j += blockDim.x) {
-    // position of channel j in the value kernel's A tiles: 1 <-> 2 and 5 <-> 6 inside each chunk of 8
-    const int jw = j & 7;
-    const int jp = (j & ~7) | (jw == 1 ? 2 : jw == 2 ? 1 : jw == 5 ? 6 : jw == 6 ? 5 : jw);
-    // runs with no valid token (l = 0) wrote no Y: their loads are skipped
-    float acc0 = 0.f, acc1 = 0.f, acc2 = 0.f, acc3 = 0.f;
+  // four channels per thread, one 16-byte load per run.  Inside every chunk
+  // of 8 the value kernel's A tiles hold channels 0 2 1 3 4 6 5 7, so the
+  // loaded positions (0, 1, 2, 3) are channels (0, 2, 1, 3) of the four.
+  for (int j = 4 * (int)threadIdx.x; j < rv; j += 4 * (int)blockDim.x) {
+    float4 a0 = make_float4(0.f, 0.f, 0.f, 0.f), a1 = a0;
     int k = 0;
-    for (; k + 4 <= ns; k += 4) {
-      const float w0 = seg_w[k], w1 = seg_w[k + 1], w2 = seg_w[k + 2], w3 = seg_w[k + 3];
-      const float y0 = w0 != 0.f ? Y[(size_t)seg_i[k] * rv + jp] : 0.f;
-      const float y1 = w1 != 0.f ? Y[(size_t)seg_i[k + 1] * rv + jp] : 0.f;
-      const float y2 = w2 != 0.f ? Y[(size_t)seg_i[k + 2] * rv + jp] : 0.f;
-      const float y3 = w3 != 0.f ? Y[(size_t)seg_i[k + 3] * rv + jp] : 0.f;
-      acc0 += w0 * y0;
-      acc1 += w1 * y1;
-      acc2 += w2 * y2;
-      acc3 += w3 * y3;
+    for (; k + 2 <= nc; k += 2) {
+      const float w0 = seg_w[k], w1 = seg_w[k + 1];
+      const float4 y0 = w0 != 0.f ? *reinterpret_cast<const float4*>(Y + (size_t)seg_i[k] * rv + j) : a1;
+      const float4 y1 = w1 != 0.f ? *reinterpret_cast<const float4*>(Y + (size_t)seg_i[k + 1] * rv + j) : a1;
+      a0.x += w0 * y0.x;
+      a0.y += w0 * y0.y;
+      a0.z += w0 * y0.z;
+      a0.w += w0 * y0.w;
+      a1.x += w1 * y1.x;
+      a1.y += w1 * y1.y;
+      a1.z += w1 * y1.z;
+      a1.w += w1 * y1.w;
     }
-    for (; k < ns; ++k) {
-      const float wgt = seg_w[k];
-      if (wgt != 0.f) acc0 += wgt * Y[(size_t)seg_i[k] * rv + jp];
+    if (k < nc && seg_w[k] != 0.f) {
+      const float w0 = seg_w[k];
+      const float4 y0 = *reinterpret_cast<const float4*>(Y + (size_t)seg_i[k] * rv + j);
+      a0.x += w0 * y0.x;
+      a0.y += w0 * y0.y;
+      a0.z += w0 * y0.z;
+      a0.w += w0 * y0.w;
     }
-    const float acc = (acc0 + acc1) + (acc2 + acc3);
+    const __half2 lo2 = __floats2half2_rn((a0.x + a1.x) * idn, (a0.z + a1.z) * idn);   // channels j, j + 1
+    const __half2 hi2 = __floats2half2_rn((a0.y + a1.y) * idn, (a0.w + a1.w) * idn);   // channels j + 2, j + 3
     const uint32_t kk = (uint32_t)(h * rv + j), cidx = kk & 63u;
     uint8_t* tile = ytiles + ((size_t)nt * KT + (kk >> 6)) * (size_t)NB * 128;
     const uint32_t off = tc::sw128((uint32_t)r, cidx >> 3) + (cidx & 7u) * 2u;
-    *reinterpret_cast<__half*>(tile + off) = __float2half_rn(acc * idn);
+    *reinterpret_cast<uint2*>(tile + off) =
+        make_uint2(*reinterpret_cast<const uint32_t*>(&lo2), *reinterpret_cast<const uint32_t*>(&hi2));
   }
 }
 
