@@ -221,12 +221,14 @@ def measured_traffic(phase, tokens):
         if k.get("phase") != phase:
             continue
         h = hashlib.sha1()
-        for f in [name + ".cu", "tc_common.cuh", "starkv_internal.cuh"]:
+        for f in [k.get("source", name + ".cu"), "tc_common.cuh", "starkv_internal.cuh"]:
             with open(os.path.join(csrc, f), "rb") as fh:
                 h.update(fh.read())
         if h.hexdigest() != k.get("source_sha1"):
             return None
-        return (k["dram_read_bytes"] + k["dram_write_bytes"]) * tokens / k["tokens"]
+        per_launch = k["dram_read_bytes"] + k["dram_write_bytes"]
+        # the output GEMM reads the same factors whatever the context length
+        return per_launch if not k.get("scales_with_tokens", True) else per_launch * tokens / k["tokens"]
     return None
 
 
