@@ -16,7 +16,7 @@
 // Heads are grouped into MMA items of N <= 128 rows of W'' (an N of 32 per head
 // would leave the tensor pipe two-thirds idle); a CTA walks 256-token
 // super-tiles (two M = 128 tiles sharing one W'' load) of one sequence.
-//   warp 0      bulk copies: RoPE table tiles, W'' item blocks, key latent pages
+//   warp 0      bulk copies of the key latent pages
 //   warp 1      tcgen05.mma issue (one thread), TMEM allocation
 //   warp 2      bulk copies of the RoPE table tiles and W'' item blocks
 //   warps 3-18  epilogue, two sets of 8 warps taking alternate MMA items; in
@@ -72,37 +72,55 @@ struct ScoreArgs {
 
 __device__ __forceinline__ long long unit_lo(int c, int G, long long U) { return (long long)c * U / G; }
 
-// Code i of a group's per-token code stream (i * B bits in, LSB first), as the
-// float 1 + u / 2^B: the code is moved to mantissa bits [23 - B, 23) and the
-// exponent of 1.0 is or-ed in.  run[] holds the stream re-aligned to bit 0.
-template <int B, int I>
+// Codes are turned into floats by the exponent trick: B code bits placed in
+// the mantissa of 1.0 at bit position p give the float 1 + u 2^(p - 23).  One
+// shift brings a tuple of TB = 2 (4-bit) or 3 (3-bit) consecutive codes to
+// mantissa bits [23 - TB B, 23), and one mask per code then gives
+//     f = 1 + u 2^((c - TB) B)      for the code at place c of its tuple.
+// The W'' row of that channel is pre-scaled by 2^(-c B) (exact), so with
+// G' = 2^(-c B) G every code contributes f G' = G' + u G 2^(-TB B) on one scale:
+//     sum (u - 2^(B-1)) G = 2^(TB B) sum f G' - sum g_c G',  g_c = 2^(TB B) + 2^(B-1) 2^(c B).
+template <int B>
+__host__ __device__ constexpr int tuple_len() { return B == 4 ? 2 : 3; }
+
+// Code I of a group of N codes whose per-token stream starts at bit 0 of run[].
+template <int N, int B, int I>
 __device__ __forceinline__ float code_float(const uint32_t* run) {
-  constexpr int p = I * B, k = p >> 5, o = p & 31;
-  constexpr int sh = o - (23 - B);
-  uint32_t x;
-  if constexpr (o + B > 32)
-    x = __funnelshift_r(run[k], run[k + 1], sh);   // the code straddles two words
-  else if constexpr (sh >= 0)
-    x = run[k] >> sh;
+  constexpr int TB = tuple_len<B>(), S0 = 23 - TB * B;
+  constexpr int k = I / TB, c = I % TB;
+  constexpr int pos = k * TB * B, wi = pos >> 5, o = pos & 31;
+  constexpr int span = (N - k * TB < TB ? N - k * TB : TB) * B;   // bits of this (possibly partial) tuple
+  uint32_t y;
+  if constexpr (o <= S0)
+    y = run[wi] << (S0 - o);
+  else if constexpr (o + span <= 32)
+    y = run[wi] >> (o - S0);
   else
-    x = run[k] << (-sh);
-  return __uint_as_float((x & (((1u << B) - 1u) << (23 - B))) | 0x3F800000u);
+    y = __funnelshift_r(run[wi], run[wi + 1], o - S0);   // the tuple straddles two words
+  constexpr uint32_t m = ((1u << B) - 1u) << (S0 + c * B);
+  return __uint_as_float((y & m) | 0x3F800000u);
+}
+template <int B, int I>
+__host__ __device__ constexpr float code_g() {
+  constexpr int TB = tuple_len<B>(), c = I % TB;
+  return (float)(1 << (TB * B)) + (float)(1 << (B - 1)) * (float)(1 << (c * B));
 }
 
-// sum_i f_i G[C + i] and sum_i G[C + i] over one group of N channels, in
+// sum_i f_i G'[C + i] and sum_i g_i G'[C + i] over one group of N channels, in
 // packed fp32x2 pairs (a scalar step for an odd tail).
-template <int B, int C, int... I>
+template <int N, int B, int C, int... I>
 __device__ __forceinline__ void group_pairs(const uint32_t* run, const float* G, float2& acc, float2& gs,
                                             std::integer_sequence<int, I...>) {
-  ((acc = __ffma2_rn(make_float2(code_float<B, 2 * I>(run), code_float<B, 2 * I + 1>(run)),
+  ((acc = __ffma2_rn(make_float2(code_float<N, B, 2 * I>(run), code_float<N, B, 2 * I + 1>(run)),
                      make_float2(G[C + 2 * I], G[C + 2 * I + 1]), acc),
-    gs = __fadd2_rn(gs, make_float2(G[C + 2 * I], G[C + 2 * I + 1]))),
+    gs = __ffma2_rn(make_float2(code_g<B, 2 * I>(), code_g<B, 2 * I + 1>()),
+                    make_float2(G[C + 2 * I], G[C + 2 * I + 1]), gs)),
    ...);
 }
 
-// One quantization group's part of a token's score: scale * sum_i (u_i - 2^(B-1)) G[C + i].
-// With f = 1 + u / 2^B:  sum (u - off) G = 2^B sum f G - (2^B + off) sum G.
-// `w` points at the group's code stream for this token (bit offset `sh` into w[0]).
+// One quantization group's part of a token's score: scale * sum_i (u_i - 2^(B-1)) G[C + i]
+// from the pre-scaled G' (see above).  `w` points at the group's code stream
+// for this token (bit offset `sh` into w[0]).
 template <int N, int B, int C>
 __device__ __forceinline__ float group_dot(const uint32_t* w, uint32_t sh, float scale, const float* G) {
   constexpr int NR = (N * B + 31) / 32;
@@ -110,15 +128,15 @@ __device__ __forceinline__ float group_dot(const uint32_t* w, uint32_t sh, float
 #pragma unroll
   for (int k = 0; k < NR; ++k) run[k] = (N * B) % 32 == 0 ? w[k] : __funnelshift_r(w[k], w[k + 1], sh);
   float2 acc = make_float2(0.f, 0.f), gs = acc;
-  group_pairs<B, C>(run, G, acc, gs, std::make_integer_sequence<int, N / 2>{});
+  group_pairs<N, B, C>(run, G, acc, gs, std::make_integer_sequence<int, N / 2>{});
   float a = acc.x + acc.y, g = gs.x + gs.y;
   if constexpr (N % 2) {
     const float gl = G[C + N - 1];
-    a = fmaf(code_float<B, N - 1>(run), gl, a);
-    g += gl;
+    a = fmaf(code_float<N, B, N - 1>(run), gl, a);
+    g = fmaf(code_g<B, N - 1>(), gl, g);
   }
-  constexpr float kf = (float)(1 << B), kg = (float)((1 << B) + (1 << (B - 1)));
-  return scale * (a * kf - g * kg);
+  constexpr float kf = (float)(1 << (tuple_len<B>() * B));
+  return scale * (a * kf - g);
 }
 
 // TMEM -> registers: columns [C, R) of this warp's lane quarter, no wait.
@@ -298,6 +316,8 @@ __global__ void __launch_bounds__(kScoreThreads, 1) k_scores_tc(ScoreArgs a) {
     // The sequence length and page ids of the next unit are loaded one unit
     // ahead, so a unit's first copies do not wait behind them.
     int i = 0, nk = 0;                    // nk: issued stage fills (for the drain below)
+    int ks_n = 0;                         // stage of item i and its phase parity, stepped per item
+    uint32_t kph_n = 0;
     int len_n = 0, page_n = 0;
     auto load_unit = [&](long long uu) {
       const int st = (int)(uu / a.batch), b = (int)(uu % a.batch);
@@ -311,8 +331,7 @@ __global__ void __launch_bounds__(kScoreThreads, 1) k_scores_tc(ScoreArgs a) {
       int page = page_n;
       if (u + 1 < u1) load_unit(u + 1);
       if (__shfl_sync(0xffffffffu, abort_flag, 0)) break;
-      const int st = (int)(u / a.batch), b = (int)(u % a.batch);
-      const int t0 = st * kSuper;
+      const int t0 = (int)(u / a.batch) * kSuper;
       if (t0 >= len) continue;
       const int npg = min(kSuper / kPage, (len - t0 + kPage - 1) / kPage);
       if (lane < npg) {
@@ -326,10 +345,15 @@ __global__ void __launch_bounds__(kScoreThreads, 1) k_scores_tc(ScoreArgs a) {
       const uint8_t* page_base = a.pool + (size_t)page * a.page_bytes;
       for (int it = 0; it < a.n_items; ++it, ++i) {
         const ScoreItem& item = items_s[it];
-        const int ks = i % a.KS;
+        const int ks = ks_n;
+        const uint32_t kph = kph_n;
+        if (++ks_n == a.KS) {
+          ks_n = 0;
+          kph_n ^= 1u;
+        }
         bool ok = true;
         if (lane == 0) {
-          ok = tc::mbar_wait_ab(&k_empty[ks], (((uint32_t)(i / a.KS)) & 1u) ^ 1u, a.status, &abort_flag);
+          ok = tc::mbar_wait_ab(&k_empty[ks], kph ^ 1u, a.status, &abort_flag);
           if (ok) tc::mbar_expect_tx(&k_full[ks], (uint32_t)(npg * item.key_bytes));
         }
         ok = __shfl_sync(0xffffffffu, ok, 0);
@@ -351,9 +375,15 @@ __global__ void __launch_bounds__(kScoreThreads, 1) k_scores_tc(ScoreArgs a) {
     // one thread; runs ahead of the key copies, bounded only by its own stages
     if (lane == 0) {
       // RoPE tiles are reloaded only when the super-tile position changes
-      int i = 0, nw = 0, ne = 0, cur_st = -1;
+      int i = 0, nw = 0, ne = 0, cur_st = -1, ws_n = 0;
+      uint32_t wph_n = 0;
+      int st_n = (int)(u0 / a.batch), b_n = (int)(u0 % a.batch);
       for (long long u = u0; u < u1 && !abort_flag; ++u) {
-        const int st = (int)(u / a.batch), b = (int)(u % a.batch);
+        const int st = st_n, b = b_n;
+        if (++b_n == a.batch) {
+          b_n = 0;
+          ++st_n;
+        }
         const int t0 = st * kSuper;
         const int len = min(a.seq_lens[b], a.max_pages * kPage);
         if (t0 >= len) continue;
@@ -369,8 +399,13 @@ __global__ void __launch_bounds__(kScoreThreads, 1) k_scores_tc(ScoreArgs a) {
         }
         for (int it = 0; it < a.n_items && ok; ++it, ++i) {
           const ScoreItem& item = items_s[it];
-          const int ws = i % a.WS;
-          ok = tc::mbar_wait_ab(&w_empty[ws], (((uint32_t)(i / a.WS)) & 1u) ^ 1u, a.status, &abort_flag);
+          const int ws = ws_n;
+          const uint32_t wph = wph_n;
+          if (++ws_n == a.WS) {
+            ws_n = 0;
+            wph_n ^= 1u;
+          }
+          ok = tc::mbar_wait_ab(&w_empty[ws], wph ^ 1u, a.status, &abort_flag);
           if (!ok) break;
           tc::mbar_expect_tx(&w_full[ws], (uint32_t)(item.npad * 256));
           tc::bulk_g2s(W_s + (size_t)ws * a.w_stage, a.W + (size_t)b * a.w_stride + item.w_off,
@@ -387,11 +422,17 @@ __global__ void __launch_bounds__(kScoreThreads, 1) k_scores_tc(ScoreArgs a) {
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issue
     if (lane == 0) {
-      int i = 0, nc = 0, cur_st = -1;
+      int i = 0, nc = 0, cur_st = -1, ws_n = 0;
+      uint32_t wph_n = 0;
+      int st_n = (int)(u0 / a.batch), b_n = (int)(u0 % a.batch);
       const uint64_t e0 = tc::sdesc_sw128(tc::smem_u32(E_s), 0, 1024), w0 = tc::sdesc_sw128(tc::smem_u32(W_s), 0, 1024);
       const uint32_t e_lo0 = tc::desc_lo(e0), w_lo0 = tc::desc_lo(w0), sw_hi = tc::desc_hi(e0);
       for (long long u = u0; u < u1 && !abort_flag; ++u) {
-        const int st = (int)(u / a.batch), b = (int)(u % a.batch);
+        const int st = st_n, b = b_n;
+        if (++b_n == a.batch) {
+          b_n = 0;
+          ++st_n;
+        }
         const int len = min(a.seq_lens[b], a.max_pages * kPage);
         if (st * kSuper >= len) continue;
         if (st != cur_st) {
@@ -404,8 +445,13 @@ __global__ void __launch_bounds__(kScoreThreads, 1) k_scores_tc(ScoreArgs a) {
         }
         for (int it = 0; it < a.n_items && !abort_flag; ++it, ++i) {
           const int npad = items_s[it].npad;
-          const int ws = i % a.WS;
-          if (!tc::mbar_wait_ab(&w_full[ws], ((uint32_t)(i / a.WS)) & 1u, a.status, &abort_flag)) { abort_flag = 1; break; }
+          const int ws = ws_n;
+          const uint32_t wph = wph_n;
+          if (++ws_n == a.WS) {
+            ws_n = 0;
+            wph_n ^= 1u;
+          }
+          if (!tc::mbar_wait_ab(&w_full[ws], wph, a.status, &abort_flag)) { abort_flag = 1; break; }
           const uint32_t idesc = tc::idesc_f16(128, npad, false, false, false);
           // descriptors as (low, high) halves, stepped in 16-byte units on the low half
           const uint32_t w_lo = w_lo0 + (uint32_t)ws * ((uint32_t)a.w_stage >> 4);
@@ -450,20 +496,31 @@ __global__ void __launch_bounds__(kScoreThreads, 1) k_scores_tc(ScoreArgs a) {
     const int tau = tile * 128 + q * 32 + lane;
     const int pg = tau >> 4, slot = tau & 15;
     const int grp32 = tile * 4 + q;      // 32-token group inside the super-tile
-    int i = 0;
+    int i = 0, ks_n = 0;
+    uint32_t kph_n = 0;
+    int st_n = (int)(u0 / a.batch), b_n = (int)(u0 % a.batch);
     for (long long u = u0; u < u1; ++u) {
-      const int st = (int)(u / a.batch), b = (int)(u % a.batch);
+      const int st = st_n, b = b_n;
+      if (++b_n == a.batch) {
+        b_n = 0;
+        ++st_n;
+      }
       const int t0 = st * kSuper;
       const int len = min(a.seq_lens[b], a.max_pages * kPage);
       if (t0 >= len) continue;
       const int t = t0 + tau;
       const bool valid = t < len;
       for (int it = 0; it < a.n_items; ++it, ++i) {
+        const int ks = ks_n;
+        const uint32_t kph = kph_n;
+        if (++ks_n == a.KS) {
+          ks_n = 0;
+          kph_n ^= 1u;
+        }
         if ((i & 1) != ipar) continue;
         const ScoreItem& item = items_s[it];
-        const int ks = i % a.KS;
         const int j = 2 * i + tile;
-        const bool ok = tc::mbar_wait_ab(&k_full[ks], ((uint32_t)(i / a.KS)) & 1u, a.status, &abort_flag) &&
+        const bool ok = tc::mbar_wait_ab(&k_full[ks], kph, a.status, &abort_flag) &&
                         tc::mbar_wait_ab(&acc_full[set], ((uint32_t)(j >> 2)) & 1u, a.status, &abort_flag);
         tc::tc_fence_after();
         if (ok) {
@@ -502,13 +559,15 @@ __global__ void __launch_bounds__(kScoreThreads, 1) k_scores_tc(ScoreArgs a) {
 }
 
 // W'' item blocks for every sequence: rows of W'' (grouped by item, zero
-// padded to the item's N), 128 columns, K-major with 128-byte swizzle, fp16.
+// padded to the item's N), 128 columns, K-major with 128-byte swizzle, fp16;
+// each row pre-scaled by 2^(-c B) for its channel's place c in a code tuple.
 // One block per (sequence, item); a thread writes 8 columns of one row.
 __global__ void __launch_bounds__(512) k_qprep_tc(LayerView v, const __nv_bfloat16* __restrict__ q,
                                                   const int32_t* __restrict__ seq_lens,
                                                   const int32_t* __restrict__ q_pos, const float* __restrict__ Bk,
                                                   const int* __restrict__ key_off,
-                                                  const ScoreItem* __restrict__ items, long long w_stride,
+                                                  const ScoreItem* __restrict__ items,
+                                                  const ScoreHead* __restrict__ heads, long long w_stride,
                                                   uint8_t* __restrict__ W) {
   __shared__ float qs[8][128];
   const int b = blockIdx.x, it = blockIdx.y;
@@ -539,6 +598,10 @@ __global__ void __launch_bounds__(512) k_qprep_tc(LayerView v, const __nv_bfloat
     uint32_t re[4] = {0u, 0u, 0u, 0u}, im[4] = {0u, 0u, 0u, 0u};
     if (hh >= 0) {
       const int h = item.h0 + hh, g = h / v.group_q, j = row - item.hcol[hh];
+      // pre-scale 2^(-c B) of the channel's place c in its code tuple (see code_float)
+      const int nhi = shape_hi(heads[h].kind);
+      const float pre = j < nhi ? ((j % 32) % 2 ? 1.f / 16.f : 1.f)
+                                : (((j - nhi) % 32) % 3 == 0 ? 1.f : ((j - nhi) % 32) % 3 == 1 ? 1.f / 8.f : 1.f / 64.f);
       const float* B = Bk + ((size_t)key_off[g] + j) * 128 + c * 8;
       const float4 x0 = *reinterpret_cast<const float4*>(B), x1 = *reinterpret_cast<const float4*>(B + 4);
       const float4 y0 = *reinterpret_cast<const float4*>(B + 64), y1 = *reinterpret_cast<const float4*>(B + 68);
@@ -547,10 +610,10 @@ __global__ void __launch_bounds__(512) k_qprep_tc(LayerView v, const __nv_bfloat
 #pragma unroll
       for (int i = 0; i < 8; i += 2) {
         const int p = c * 8 + i;
-        const float r0 = qs[hh][p] * xs[i] + qs[hh][p + 64] * ys[i];
-        const float r1 = qs[hh][p + 1] * xs[i + 1] + qs[hh][p + 65] * ys[i + 1];
-        const float i0 = qs[hh][p + 64] * xs[i] - qs[hh][p] * ys[i];
-        const float i1 = qs[hh][p + 65] * xs[i + 1] - qs[hh][p + 1] * ys[i + 1];
+        const float r0 = (qs[hh][p] * xs[i] + qs[hh][p + 64] * ys[i]) * pre;
+        const float r1 = (qs[hh][p + 1] * xs[i + 1] + qs[hh][p + 65] * ys[i + 1]) * pre;
+        const float i0 = (qs[hh][p + 64] * xs[i] - qs[hh][p] * ys[i]) * pre;
+        const float i1 = (qs[hh][p + 65] * xs[i + 1] - qs[hh][p + 1] * ys[i + 1]) * pre;
         const __half2 rh = __floats2half2_rn(r0, r1), ih = __floats2half2_rn(i0, i1);
         re[i / 2] = *reinterpret_cast<const uint32_t*>(&rh);
         im[i / 2] = *reinterpret_cast<const uint32_t*>(&ih);
@@ -698,7 +761,7 @@ cudaError_t launch_scores_tc(const starkv_layer* L, const uint8_t* pool, long lo
   out->n_g = n_st * (kSuper / 32);
   out->m_st = (float*)w;
   k_qprep_tc<<<dim3(batch, (unsigned)L->items.size()), 512, 0, s>>>(
-      v, (const __nv_bfloat16*)q, seq_lens, q_pos, L->Bk, L->d_key_off, L->d_items, L->w_stride, W);
+      v, (const __nv_bfloat16*)q, seq_lens, q_pos, L->Bk, L->d_key_off, L->d_items, L->d_score_heads, L->w_stride, W);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   ScoreArgs a;
