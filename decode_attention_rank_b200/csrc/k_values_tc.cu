@@ -140,6 +140,7 @@ __global__ void __launch_bounds__(kValThreads, 1) k_values_tc(ValArgs a) {
   __shared__ int4 vg_s[128];              // per value group: code width, code block offset, fp16x2 of 1024 + 2^(bits-1)
   __shared__ int4 tile_s[kMaxTiles];      // per tile: sequence, first token, length, run
   __shared__ int pid_s[kMaxTiles][8];     // per tile: page of each 16-token slot block
+  __shared__ uint8_t rsp_s[kMaxTiles * 8];   // per page of the CTA: raw stage | phase parity << 7
   __shared__ int run_b[kMaxRuns];
   __shared__ int n_tiles_s, n_runs_s;
   __shared__ float l_stage[64];           // run sums of the staged P, per head
@@ -241,6 +242,7 @@ __global__ void __launch_bounds__(kValThreads, 1) k_values_tc(ValArgs a) {
       }
     }
     pid_s[e >> 3][e & 7] = page;
+    rsp_s[e] = (uint8_t)((e % a.n_raw) | (((e / a.n_raw) & 1) << 7));
   }
   for (int x = threadIdx.x; x < kRunMaxCache * 64; x += blockDim.x) (&runM_s[0][0])[x] = -FLT_MAX;
   __syncthreads();
@@ -428,8 +430,9 @@ __global__ void __launch_bounds__(kValThreads, 1) k_values_tc(ValArgs a) {
     if (lane == 0) {
       const int n_pg = n_tiles * 8;
       for (int pg = 0; pg < n_pg; ++pg) {
-        const int rs = pg % a.n_raw;
-        if (!tc::mbar_wait_ab(&r_empty[rs], (((uint32_t)(pg / a.n_raw)) & 1u) ^ 1u, a.status, &abort_flag)) break;
+        const uint32_t rsp = rsp_s[pg];
+        const int rs = (int)(rsp & 127u);
+        if (!tc::mbar_wait_ab(&r_empty[rs], (rsp >> 7) ^ 1u, a.status, &abort_flag)) break;
         const int page = pid_s[pg >> 3][pg & 7];
         tc::mbar_expect_tx(&r_full[rs], page >= 0 ? (uint32_t)a.vblk_bytes : 0u);
         if (page >= 0)
@@ -484,14 +487,15 @@ __global__ void __launch_bounds__(kValThreads, 1) k_values_tc(ValArgs a) {
       const int x = n & ((1 << lg_ipt) - 1);
       const int k = x >> lnb, cb = x & (nblk - 1);
       const int pg = T * 8 + k;                // page of the CTA's tiles
-      const int rs = pg % a.n_raw, as = n % kAStages;
+      const uint32_t rsp = rsp_s[pg];
+      const int rs = (int)(rsp & 127u), as = n % kAStages;
       const bool valid = pid_s[T][k] >= 0;
       // A stage first: the stage's previous item was in chain ch - 4; once that
       // chain is consumed every page up to it has landed, and with at least
       // 32 / nblk raw stages the raw stage is then at most one phase from pg
       const int ch = n >> 3;                   // chain of this item
       const bool ok = tc::mbar_wait_ab(&ch_done[ch & 3], (((uint32_t)(ch >> 2)) & 1u) ^ 1u, a.status, &abort_flag) &&
-                      tc::mbar_wait_ab(&r_full[rs], ((uint32_t)(pg / a.n_raw)) & 1u, a.status, &abort_flag);
+                      tc::mbar_wait_ab(&r_full[rs], rsp >> 7, a.status, &abort_flag);
       if (ok) {
         const uint8_t* blk = R_s + (size_t)rs * a.raw_stage;
         uint8_t* st = A_s + (size_t)as * kAStage + st_off;
