@@ -185,8 +185,23 @@ __host__ __device__ constexpr int seg_width(int S, int g) { return (g + 1) * 32 
 // channel is G column C0 of the head and whose first group is group G0 of the
 // latent.  Each group's G columns come out of TMEM on their own (at most 32
 // registers live), the code words are read while the TMEM load is in flight.
-template <int S, int B, int C0, int G0, int g = 0>
-__device__ __forceinline__ float segment_dot(uint32_t taddr, const uint8_t* blk, const ScoreHead& hd, int slot) {
+// Byte offset of group g's code block inside the key latent block of a head
+// with NHI 4-bit and NLO 3-bit channels: the fp16 scales of every group first
+// (one per slot), then each group's codes for the page's slots, padded to 16
+// bytes.  plan_scores_tc checks the layer's layout against it.
+__host__ __device__ constexpr int code_block_off(int nhi, int nlo, int g) {
+  const int ng = seg_groups(nhi) + seg_groups(nlo);
+  int off = (ng * kPage * 2 + 15) / 16 * 16;
+  for (int x = 0; x < g; ++x) {
+    const bool hi = x < seg_groups(nhi);
+    const int n = hi ? seg_width(nhi, x) : seg_width(nlo, x - seg_groups(nhi));
+    off += (kPage * n * (hi ? 4 : 3) / 8 + 15) / 16 * 16;
+  }
+  return off;
+}
+
+template <int NHI, int NLO, int S, int B, int C0, int G0, int g = 0>
+__device__ __forceinline__ float segment_dot(uint32_t taddr, const uint8_t* blk, int slot) {
   if constexpr (g >= seg_groups(S)) {
     return 0.f;
   } else {
@@ -195,7 +210,8 @@ __device__ __forceinline__ float segment_dot(uint32_t taddr, const uint8_t* blk,
     float G[N];
     tmem_cols<0, N>(taddr + (uint32_t)(C0 + g * 32), G);
     const uint32_t bit0 = (uint32_t)slot * (uint32_t)(N * B);
-    const uint32_t* w = reinterpret_cast<const uint32_t*>(blk + hd.code_off[G0 + g]) + (bit0 >> 5);
+    constexpr int CO = code_block_off(NHI, NLO, G0 + g);
+    const uint32_t* w = reinterpret_cast<const uint32_t*>(blk + CO) + (bit0 >> 5);
     // a group whose per-token code run is a whole number of words starts on a
     // word boundary for every token: no re-alignment, no extra word
     constexpr int NW = (N * B) % 32 == 0 ? NR : NR + 1;
@@ -205,16 +221,17 @@ __device__ __forceinline__ float segment_dot(uint32_t taddr, const uint8_t* blk,
     const float scale = __half2float(reinterpret_cast<const __half*>(blk)[(G0 + g) * kPage + slot]);
     tc::tmem_ld_wait();
     reg_fence<N>(G);
-    return group_dot<N, B, 0>(wr, bit0 & 31u, scale, G) + segment_dot<S, B, C0, G0, g + 1>(taddr, blk, hd, slot);
+    return group_dot<N, B, 0>(wr, bit0 & 31u, scale, G) +
+           segment_dot<NHI, NLO, S, B, C0, G0, g + 1>(taddr, blk, slot);
   }
 }
 
 // The score of one token for one head whose key latent has NHI 4-bit channels
 // then NLO 3-bit channels (G columns 0 .. NHI + NLO - 1 from `taddr`).
 template <int NHI, int NLO>
-__device__ __forceinline__ float head_score(uint32_t taddr, const uint8_t* blk, const ScoreHead& hd, int slot) {
-  return segment_dot<NHI, 4, 0, 0>(taddr, blk, hd, slot) +
-         segment_dot<NLO, 3, NHI, seg_groups(NHI)>(taddr, blk, hd, slot);
+__device__ __forceinline__ float head_score(uint32_t taddr, const uint8_t* blk, int slot) {
+  return segment_dot<NHI, NLO, NHI, 4, 0, 0>(taddr, blk, slot) +
+         segment_dot<NHI, NLO, NLO, 3, NHI, seg_groups(NHI)>(taddr, blk, slot);
 }
 
 // Compiled head shapes (hi channels, lo channels): 25 % and 20 % of ranks
@@ -236,10 +253,10 @@ __host__ __device__ constexpr int shape_lo(int k) {
 #undef STARKV_LO
 }
 
-__device__ __forceinline__ float head_score_any(uint32_t taddr, const uint8_t* blk, const ScoreHead& hd, int slot) {
-  switch (hd.kind) {
+__device__ __forceinline__ float head_score_any(uint32_t taddr, const uint8_t* blk, int kind, int slot) {
+  switch (kind) {
 #define STARKV_CASE(i, h, l) \
-  case i: return head_score<h, l>(taddr, blk, hd, slot);
+  case i: return head_score<h, l>(taddr, blk, slot);
     STARKV_HEAD_SHAPES(STARKV_CASE)
 #undef STARKV_CASE
     default: return 0.f;
@@ -531,7 +548,7 @@ __global__ void __launch_bounds__(kScoreThreads, 1) k_scores_tc(ScoreArgs a) {
           float* mrow = a.m_st + row0 * a.n_g + (t0 >> 5) + grp32;
           for (int hh = 0; hh < item.nh; ++hh, prow += a.P_ld, mrow += a.n_g) {
             const ScoreHead& hd = heads_s[item.h0 + hh];
-            const float sv = head_score_any(trow + (uint32_t)hd.gcol, page + hd.blk_rel, hd, slot);
+            const float sv = head_score_any(trow + (uint32_t)hd.gcol, page + hd.blk_rel, hd.kind, slot);
             if (a.S_dbg) {
               if (valid) a.S_dbg[(row0 + hh) * a.P_ld + t] = sv;
               continue;
@@ -667,7 +684,7 @@ bool plan_scores_tc(starkv_layer* L) {
       bool match = (int)want.size() == ld.n_groups;
       for (int j = 0; match && j < ld.n_groups; ++j) {
         const GroupDesc& gd = L->grp[ld.group0 + j];
-        match = gd.n == want[j].first && gd.bits == want[j].second;
+        match = gd.n == want[j].first && gd.bits == want[j].second && gd.code_off == code_block_off(nhi, nlo, j);
       }
       if (match) kv_kind[g] = k;
     }
@@ -705,8 +722,6 @@ bool plan_scores_tc(starkv_layer* L) {
       hd.gcol = it.hcol[hh];
       hd.kind = kv_kind[g];
       hd.blk_rel = ld.block_off - it.key_off;
-      hd.n_groups = ld.n_groups;
-      for (int k = 0; k < ld.n_groups; ++k) hd.code_off[k] = L->grp[ld.group0 + k].code_off;
     }
     L->items.push_back(it);
   }

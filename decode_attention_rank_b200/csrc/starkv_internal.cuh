@@ -74,13 +74,13 @@ struct ScoreItem {
 };
 
 // The score epilogue's view of one query head: where its G columns and its
-// key latent's code groups are, and which compiled channel shape reads them.
+// key latent block are, and which compiled channel shape reads them (the
+// shape fixes the block's layout).
 struct ScoreHead {
   int gcol;          // G column of the head's first latent channel (item-relative)
   int kind;          // index of the compiled (hi channels, lo channels) shape
   int blk_rel;       // byte offset of the key latent block, relative to the item's key range in a page
-  int n_groups;
-  int code_off[4];   // byte offset of each group's code block inside the latent block
+  int pad_;
 };
 
 // Outputs of the tensor-core score kernel.
