@@ -31,9 +31,12 @@ int num_sms() {
 }
 
 // Channels of the high-precision segment: ceil(top_fraction * r) (reading notes
-// "STAR-KV 阅读笔记" section 6.1; the model card's top_fraction).
+// "STAR-KV 阅读笔记" section 6.1; the model card's top_fraction).  The fraction
+// arrives as a float: a product within its rounding error (r * 2^-23) of an
+// integer is that integer, so that e.g. 0.2 (stored as 0.2000000030) gives 8
+// channels of 40, not 9.
 static int n_high(int r, float top_fraction) {
-  return (int)ceil((double)top_fraction * (double)r - 1e-9);
+  return (int)ceil((double)top_fraction * (double)r - (double)r * 0x1p-23 - 1e-9);
 }
 
 }  // namespace starkv

@@ -208,6 +208,20 @@ def test_tc_scores_feeding_cuda_core_values(cfg, quant, lens):
     run_decode(case(cfg, quantized=quant), lens[:2], peaky=25.0, use_hidden=False, check_pool=False, path=2)
 
 
+@pytest.mark.parametrize("top", [0.2, 1.0])
+def test_tc_other_bit_splits(top):
+    """The compiled head shapes of the 20 % split (odd group widths in both
+    segments) and of all-4-bit latents (full 32-channel 4-bit groups), with
+    every rank 16..64, through the tensor-core score path; packed pages
+    checked bit for bit."""
+    import dataclasses
+    spec = dataclasses.replace(gen.config_spec(2, quantized=True), top_fraction=top,
+                               key_ranks=[16, 24, 32, 40, 48, 56, 64, 16] * 4)
+    c = Case(spec, gen.LAYER_SEED[2], 0)
+    run_decode(c, [600, 257, 33], use_hidden=False, check_pool=True)
+    run_decode(c, [300, 40], peaky=25.0, use_hidden=False, check_pool=False)
+
+
 def test_tc_long_context_runs():
     """All-tensor-core decode with more super-tiles than SMs: CTAs whose unit
     ranges span several super-tiles and cross sequence boundaries."""
