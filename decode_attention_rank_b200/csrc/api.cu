@@ -404,6 +404,34 @@ starkv_status starkv_append(const starkv_layer* L, void* pool, int64_t n_pages, 
   return STARKV_OK;
 }
 
+namespace starkv {
+namespace {
+
+// Prefill rows go through the tensor-core decode kernels in batches of at most
+// this many query rows (the output GEMM's widest B tile).
+constexpr int kPrefillRows = 256;
+
+// Page-table rows of query rows: out[r][p] = page_table[seq[r]][p].
+__global__ void k_expand_rows(const int32_t* __restrict__ page_table, int max_pages, const int32_t* __restrict__ seq,
+                              int rows, int32_t* __restrict__ out) {
+  const long long n = (long long)rows * max_pages;
+  for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (long long)gridDim.x * blockDim.x) {
+    const int r = (int)(i / max_pages), p = (int)(i % max_pages);
+    out[i] = page_table[(size_t)seq[r] * max_pages + p];
+  }
+}
+
+// Workspace of a tensor-core prefill: the row table, one batch of expanded
+// page-table rows and one batch's decode workspace.
+size_t prefill_tc_ws_bytes(const starkv_layer* L, long long rows, int max_pages) {
+  const int nb = (int)std::min<long long>(rows, kPrefillRows);
+  return ru(sizeof(int32_t) * 3 * (size_t)rows, 256) + ru(sizeof(int32_t) * (size_t)nb * max_pages, 256) +
+         decode_tc_ws_bytes(L, nb, max_pages * kPage);
+}
+
+}  // namespace
+}  // namespace starkv
+
 size_t starkv_workspace_bytes(const starkv_layer* L, int batch, int max_ctx, int max_q) {
   if (!L || batch <= 0) return 0;
   if (max_q < 1) max_q = 1;
@@ -415,6 +443,8 @@ size_t starkv_workspace_bytes(const starkv_layer* L, int batch, int max_ctx, int
     const long long rows = std::min<long long>((long long)batch * max_q, 1 << 30);
     need = std::max(need, ru(sizeof(int32_t) * 3 * (size_t)rows, 256) +
                               decode_generic_ws_bytes(L, (int)rows, max_ctx, true));
+    if (L->tc_scores && L->tc_values)
+      need = std::max(need, prefill_tc_ws_bytes(L, rows, (max_ctx + kPage - 1) / kPage));
   }
   return need;
 }
@@ -478,13 +508,43 @@ starkv_status starkv_prefill_attn(const starkv_layer* L, const void* pool, int64
       tab[2 * rows + r] = q_start_host[b] + i;   // RoPE position
     }
   const size_t tab_bytes = ru(sizeof(int32_t) * tab.size(), 256);
+  cudaStream_t s = (cudaStream_t)stream;
+  int32_t* dtab = (int32_t*)workspace;
+  // Tensor-core path: every query row is a decode of its sequence at its
+  // visible length and RoPE position, run through the tensor-core decode
+  // kernels in batches of kPrefillRows rows that share the workspace.
+  const bool tc = L->tc_scores && L->tc_values && L->decode_path == 0 && max_pages * kPage <= L->rope_tiles * 128;
+  if (tc) {
+    const size_t need = prefill_tc_ws_bytes(L, rows, max_pages);
+    if (workspace == nullptr || ws_bytes < need) {
+      set_error("prefill workspace too small: need " + std::to_string(need) + " bytes");
+      return STARKV_ERR_WORKSPACE;
+    }
+    const int nb = std::min(rows, kPrefillRows);
+    int32_t* pt_rows = (int32_t*)((char*)workspace + tab_bytes);
+    char* ws_tc = (char*)workspace + tab_bytes + ru(sizeof(int32_t) * (size_t)nb * max_pages, 256);
+    const size_t ws_tc_bytes = ws_bytes - (size_t)(ws_tc - (char*)workspace);
+    const size_t qrow = (size_t)L->view.H * L->cfg.head_dim * sizeof(uint16_t);
+    const size_t orow = (size_t)L->view.D * sizeof(uint16_t);
+    CUDA_TRY(cudaMemcpyAsync(dtab, tab.data(), sizeof(int32_t) * tab.size(), cudaMemcpyHostToDevice, s));
+    for (int r0 = 0; r0 < rows; r0 += nb) {
+      const int n = std::min(nb, rows - r0);
+      k_expand_rows<<<std::max(1, std::min(1024, (int)(((long long)n * max_pages + 255) / 256))), 256, 0, s>>>(
+          page_table, max_pages, dtab + r0, n, pt_rows);
+      CUDA_TRY(cudaGetLastError());
+      CUDA_TRY(launch_decode_tc(L, (const uint8_t*)pool, n_pages, pt_rows, max_pages, n, dtab + rows + r0,
+                                dtab + 2 * rows + r0, (const char*)q + (size_t)r0 * qrow, (char*)out + (size_t)r0 * orow,
+                                ws_tc, ws_tc_bytes, s, false));
+    }
+    // pageable host source: make sure the copy has consumed `tab` before it is freed
+    CUDA_TRY(cudaStreamSynchronize(s));
+    return STARKV_OK;
+  }
   const size_t need = tab_bytes + decode_generic_ws_bytes(L, rows, max_len, true);
   if (workspace == nullptr || ws_bytes < need) {
     set_error("prefill workspace too small: need " + std::to_string(need) + " bytes");
     return STARKV_ERR_WORKSPACE;
   }
-  cudaStream_t s = (cudaStream_t)stream;
-  int32_t* dtab = (int32_t*)workspace;
   CUDA_TRY(cudaMemcpyAsync(dtab, tab.data(), sizeof(int32_t) * tab.size(), cudaMemcpyHostToDevice, s));
   RowInfo ri{dtab, dtab + rows, dtab + 2 * rows};
   CUDA_TRY(launch_decode_generic(L, (const uint8_t*)pool, n_pages, page_table, max_pages, rows, ri, max_len, q, out,

@@ -788,7 +788,7 @@ size_t decode_tc_ws_bytes(const starkv_layer* L, int batch, int max_len) {
 
 cudaError_t launch_decode_tc(const starkv_layer* L, const uint8_t* pool, long long n_pages, const int32_t* pt,
                              int max_pages, int batch, const int32_t* seq_lens, const int32_t* q_pos, const void* q,
-                             void* out, void* ws, size_t ws_bytes, cudaStream_t s) {
+                             void* out, void* ws, size_t ws_bytes, cudaStream_t s, bool profile) {
   auto r = [](size_t x) { return (x + 255) / 256 * 256; };
   const int max_len = max_pages * kPage;
   if (ws_bytes < decode_tc_ws_bytes(L, batch, max_len)) return cudaErrorInvalidValue;
@@ -805,7 +805,7 @@ cudaError_t launch_decode_tc(const starkv_layer* L, const uint8_t* pool, long lo
   float* part = (float*)w;
   // optional timing events between the kernels (see starkv_profile_decode)
   cudaEvent_t* ev = nullptr;
-  if (L->prof_n > 0) {
+  if (profile && L->prof_n > 0) {
     starkv_layer* Lm = const_cast<starkv_layer*>(L);
     const int slot = (int)(Lm->prof_calls++ % Lm->prof_n);
     ev = &Lm->prof_ev[(size_t)slot * (STARKV_N_PHASES + 1)];

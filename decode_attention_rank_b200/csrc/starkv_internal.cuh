@@ -178,9 +178,10 @@ size_t values_tc_ws_bytes(const starkv_layer* L, int batch, int max_len);
 cudaError_t launch_values_tc(const starkv_layer* L, const uint8_t* pool, long long n_pages, const int32_t* pt,
                              int max_pages, int batch, const int32_t* seq_lens, const ScoreOut& so, void* ws,
                              void* ytiles, cudaStream_t s, cudaEvent_t ev_mid);
+// `profile`: record the phase events of starkv_profile_decode (decode calls only).
 cudaError_t launch_decode_tc(const starkv_layer* L, const uint8_t* pool, long long n_pages, const int32_t* pt,
                              int max_pages, int batch, const int32_t* seq_lens, const int32_t* q_pos, const void* q,
-                             void* out, void* ws, size_t ws_bytes, cudaStream_t s);
+                             void* out, void* ws, size_t ws_bytes, cudaStream_t s, bool profile = true);
 size_t decode_tc_ws_bytes(const starkv_layer* L, int batch, int max_len);
 cudaError_t build_rope_table(starkv_layer* L, cudaStream_t s);
 size_t scores_tc_ws_bytes(const starkv_layer* L, int batch, int max_len);

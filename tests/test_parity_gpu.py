@@ -197,6 +197,43 @@ def test_prefill_two_output_tiles():
         check_close(got[i], want, f"prefill row {i}")
 
 
+def test_prefill_tc_row_batches():
+    """A quantized RoPE layer's prefill runs its query rows through the
+    tensor-core decode kernels, 256 rows at a time: two sequences with
+    different history lengths, 320 rows (256 + 64), sampled rows and a
+    peaky-attention rerun against the oracle; the CUDA-core path agrees."""
+    c = case(2)
+    s = c.spec
+    starts, ns = [100, 30], [200, 120]
+    for peaky in (1.0, 25.0):
+        outs = []
+        for path in (0, 1):
+            L = c.load()
+            if path:
+                L.set_decode_path(path)
+            cache = GpuCache(L, [a + n for a, n in zip(starts, ns)])
+            Zs = []
+            for b, (a, n) in enumerate(zip(starts, ns)):
+                Z = c.latents_direct(b, a + n)
+                cache.append_latents(b, Z)
+                Zs.append(c.stored(Z))
+            Qall = queries(c, 2, peaky=peaky, n_pos=max(ns))
+            Q = np.concatenate([Qall[b][:n] for b, n in enumerate(ns)])
+            qt = torch.from_numpy(Q).cuda().to(torch.bfloat16)
+            out = torch.empty(sum(ns), s.hidden, device="cuda", dtype=torch.bfloat16)
+            ws = torch.empty(L.workspace_bytes(2, max(a + n for a, n in zip(starts, ns)), max(ns)), dtype=torch.uint8,
+                             device="cuda")
+            L.prefill(cache.pool, cache.n_pages, cache.page_table, starts, ns, qt, out, ws)
+            outs.append(out.double().cpu().numpy())
+        got = outs[0]
+        for r in (0, 1, 199, 200, 255, 256, 319):
+            b = 0 if r < ns[0] else 1
+            i = r if b == 0 else r - ns[0]
+            want = O.decode(s, c.f, Zs[b], Q[r], starts[b] + i, starts[b] + i + 1, c.B_rot)
+            check_close(got[r], want, f"prefill row {r} (peaky {peaky})")
+        assert np.linalg.norm(outs[1] - got) <= 3e-3 * np.linalg.norm(got)
+
+
 @pytest.mark.parametrize("cfg,quant,lens", [
     (2, False, [600, 257, 256, 1]),
     (3, True, [300, 97]),
