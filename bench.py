@@ -439,6 +439,44 @@ def run_reference(args, rank, ws):
             "e2e": {"value": v, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
 
 
+def run_prefill(args):
+    """Time one causal prefill chunk: `args.prefill` queries after ctx - prefill
+    tokens of history, batch 1, on the workload's layer (separate JSON line;
+    not the headline metric)."""
+    import torch
+    n = args.prefill
+    T = WORKLOAD["ctx"] if args.ctx else 4096
+    assert T % 16 == 0 and 0 < n <= T, "prefill chunk must fit the context"
+    torch.cuda.set_device(0)
+    spec, f, L = build_layer()
+    pool, n_pages, page_table, _ = fill_cache(spec, f, L, 1, T, 0, T, 0)
+    g = torch.Generator(device="cuda")
+    g.manual_seed(91)
+    q = (torch.randn(n, spec.n_heads, spec.head_dim, generator=g, device="cuda") /
+         math.sqrt(spec.head_dim)).to(torch.bfloat16)
+    out = torch.empty(n, spec.hidden, dtype=torch.bfloat16, device="cuda")
+    ws = torch.empty(L.workspace_bytes(1, T, n), dtype=torch.uint8, device="cuda")
+    for _ in range(args.warmup):
+        L.prefill(pool, n_pages, page_table, [T - n], [n], q, out, ws)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(args.steps):
+        L.prefill(pool, n_pages, page_table, [T - n], [n], q, out, ws)
+    e1.record()
+    torch.cuda.synchronize()
+    status = L.sync_status()
+    ms = e0.elapsed_time(e1) / args.steps
+    return {"metric": "causal prefill query tokens/s (latent attention over the paged cache)", "value": n / (ms * 1e-3),
+            "unit": "query tokens/s", "n_gpus": 1, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "u3/u4 latent codes + fp16 "
+            "scales, bf16 factors/q/out, fp32 accumulate", "data": "synthetic", "mode": "prefill",
+            "config": {"workload": f"prefill chunk of {n} queries after {T - n} tokens of history, batch 1 "
+                                   "(LongChat-7B-shaped layer, 4/3-bit latents)", "batch": 1, "ctx": T,
+                       "queries": n},
+            "device_status": status}
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -450,11 +488,16 @@ def main():
     ap.add_argument("--ctx", type=int, default=0, help="context length (default: the headline 32768); a smaller "
                     "value gives the small case used for profiler captures")
     ap.add_argument("--batch", type=int, default=0, help="sequences per step (default 16)")
+    ap.add_argument("--prefill", type=int, default=0, help="time a causal prefill chunk of this many queries "
+                    "(history = ctx - queries, ctx default 4096) instead of the decode step")
     args = ap.parse_args()
     if args.ctx:
         WORKLOAD["ctx"] = args.ctx
     if args.batch:
         WORKLOAD["batch"] = args.batch
+    if args.prefill:
+        print(json.dumps(run_prefill(args)), flush=True)
+        return
     if args.impl == "reference":
         rank = int(os.environ.get("RANK", "0"))
         ws = int(os.environ.get("WORLD_SIZE", "1"))
