@@ -513,13 +513,11 @@ starkv_status starkv_prefill_attn(const starkv_layer* L, const void* pool, int64
   // Tensor-core path: every query row is a decode of its sequence at its
   // visible length and RoPE position, run through the tensor-core decode
   // kernels in batches of kPrefillRows rows that share the workspace.
-  const bool tc = L->tc_scores && L->tc_values && L->decode_path == 0 && max_pages * kPage <= L->rope_tiles * 128;
+  // A workspace sized for a shorter context than the page table's capacity
+  // (enough for the CUDA-core kernels) takes the CUDA-core path.
+  const bool tc = L->tc_scores && L->tc_values && L->decode_path == 0 && max_pages * kPage <= L->rope_tiles * 128 &&
+                  workspace != nullptr && ws_bytes >= prefill_tc_ws_bytes(L, rows, max_pages);
   if (tc) {
-    const size_t need = prefill_tc_ws_bytes(L, rows, max_pages);
-    if (workspace == nullptr || ws_bytes < need) {
-      set_error("prefill workspace too small: need " + std::to_string(need) + " bytes");
-      return STARKV_ERR_WORKSPACE;
-    }
     const int nb = std::min(rows, kPrefillRows);
     int32_t* pt_rows = (int32_t*)((char*)workspace + tab_bytes);
     char* ws_tc = (char*)workspace + tab_bytes + ru(sizeof(int32_t) * (size_t)nb * max_pages, 256);

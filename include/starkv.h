@@ -206,7 +206,11 @@ STARKV_API starkv_status starkv_decode_attn(const starkv_layer* layer, const voi
  *   q_start_host, q_len_host: HOST int32 arrays [batch] (they set the launch shape).
  *   q: [sum q_len][H][d] in dtype, sequences one after another; out: [sum q_len][D].
  *   workspace: at least starkv_workspace_bytes(layer, batch, max_ctx, max q_len)
- *     bytes, where max_ctx >= every q_start[b] + q_len[b].
+ *     bytes, where max_ctx >= every q_start[b] + q_len[b].  Layers that the
+ *     tensor-core kernels take (bf16, RoPE, quantized, compiled head shapes)
+ *     run every query row through them, 256 rows at a time, when max_ctx is the
+ *     page table's capacity (max_pages * 16); a workspace sized for a shorter
+ *     max_ctx runs the CUDA-core kernels instead.
  */
 STARKV_API starkv_status starkv_prefill_attn(const starkv_layer* layer, const void* pool, int64_t n_pages,
                                   const int32_t* page_table, int max_pages, int batch, const int32_t* q_start_host,
