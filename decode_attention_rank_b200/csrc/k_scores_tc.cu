@@ -14,8 +14,10 @@
 // epilogue straight out of TMEM.
 //
 // Heads are grouped into MMA items of N <= 128 rows of W'' (an N of 32 per head
-// would leave the tensor pipe two-thirds idle); a CTA walks 256-token
-// super-tiles (two M = 128 tiles sharing one W'' load) of one sequence.
+// would leave the tensor pipe two-thirds idle).  A unit is one 256-token
+// super-tile (two M = 128 tiles sharing one W'' load) of one sequence; a CTA
+// walks a contiguous range of units ordered position-major, so its RoPE tiles
+// stay resident across the sequences of one position.
 //   warp 0      bulk copies of the key latent pages
 //   warp 1      tcgen05.mma issue (one thread), TMEM allocation
 //   warp 2      bulk copies of the RoPE table tiles and W'' item blocks
@@ -181,10 +183,6 @@ __device__ __forceinline__ void reg_fence(float* G) {
 __host__ __device__ constexpr int seg_groups(int S) { return (S + 31) / 32; }
 __host__ __device__ constexpr int seg_width(int S, int g) { return (g + 1) * 32 <= S ? 32 : S - g * 32; }
 
-// Groups g, g + 1, ... of a segment of S channels at B bits whose first
-// channel is G column C0 of the head and whose first group is group G0 of the
-// latent.  Each group's G columns come out of TMEM on their own (at most 32
-// registers live), the code words are read while the TMEM load is in flight.
 // Byte offset of group g's code block inside the key latent block of a head
 // with NHI 4-bit and NLO 3-bit channels: the fp16 scales of every group first
 // (one per slot), then each group's codes for the page's slots, padded to 16
@@ -200,6 +198,11 @@ __host__ __device__ constexpr int code_block_off(int nhi, int nlo, int g) {
   return off;
 }
 
+// Groups g, g + 1, ... of a segment of S channels at B bits (of a head with
+// NHI 4-bit and NLO 3-bit channels) whose first channel is G column C0 of the
+// head and whose first group is group G0 of the latent.  Each group's G
+// columns come out of TMEM on their own (at most 32 registers live), the code
+// words are read while the TMEM load is in flight.
 template <int NHI, int NLO, int S, int B, int C0, int G0, int g = 0>
 __device__ __forceinline__ float segment_dot(uint32_t taddr, const uint8_t* blk, int slot) {
   if constexpr (g >= seg_groups(S)) {
