@@ -118,13 +118,20 @@ def barrier(ws):
 
 
 def max_over_ranks(x: float, ws: int) -> float:
+    """The maximum of x over the ranks (device times are taken as the slowest rank's)."""
     if ws == 1:
         return x
     import torch
     import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def job_tokens_per_s(batch_per_rank: int, ws: int, ms_step_max: float) -> float:
+    """Whole-job decode throughput: every rank's sequences over the slowest rank's step time."""
+    return batch_per_rank * ws / (ms_step_max * 1e-3)
 
 
 # ---------------------------------------------------------------------------
@@ -361,7 +368,7 @@ def run_ours(args, rank, ws, local):
                 "frac": (pbytes[p] / (ph_ms[p] * 1e-3) / 1e9 / peak) if ph_ms[p] > 0 else None}
                for p in range(len(PHASES))]
     dom = max(range(len(PHASES)), key=lambda p: ph_ms[p])
-    tokens_per_s = B * ws / (ms_step * 1e-3)
+    tokens_per_s = job_tokens_per_s(B, ws, ms_step)
     res = {
         "metric": METRIC,
         "value": tokens_per_s,
