@@ -96,6 +96,17 @@ def test_groups_and_segments():
     assert [(x.start, x.n, x.bits) for x in g] == [(0, 14, 4), (14, 32, 3), (46, 10, 3)]
 
 
+def test_hi_width_is_the_exact_ceiling():
+    """n_hi = ceil(top_fraction * r) computed exactly (rationals) for the 25 % of the
+    model card, the 20 % of the reading notes section 6.1 and all-4-bit latents:
+    a product that is an integer (0.2 * 40 = 8) must not round up."""
+    from fractions import Fraction
+    for frac in ("0.25", "0.2", "1"):
+        for r in list(range(1, 129)) + [256, 1000, 1024, 4096]:
+            want = -((-Fraction(frac) * r) // 1)
+            assert O.n_high(r, float(frac)) == want, (frac, r)
+
+
 # ---------------------------------------------------------------------------
 # Page format: hand-derived golden bytes
 # ---------------------------------------------------------------------------
