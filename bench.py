@@ -42,6 +42,16 @@ def measured_peaks():
     return 6650.0, "fallback"
 
 
+def measured_tensor_peak():
+    """Dense fp16/bf16 tensor peak in TFLOP/s (the kernels time in a long step: the sustained figure)."""
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d.get("bf16_tflops_sustained", d.get("bf16_tflops", 1400.0)), "measured (sustained bf16)"
+    return 1400.0, "fallback"
+
+
 class ClockSampler:
     """nvidia-smi clocks and throttle reasons sampled during the timed region."""
 
@@ -214,6 +224,17 @@ def phase_bytes(spec, B, ctx):
             2 * spec.n_heads * spec.value_rank * spec.hidden + B * spec.hidden * 2]
 
 
+def phase_flops(spec, B, ctx):
+    """Algorithmic tensor flops of each decode phase: 2 r_h d per (token, head) to
+    reconstruct, rope and score the keys (the G contraction); 2 r_v per (token,
+    query head) for P Z_v; none for the merge; 2 H r_v D per sequence for M."""
+    d = spec.head_dim
+    return [B * ctx * 2.0 * d * sum(spec.key_ranks) * (spec.n_heads // spec.n_kv_heads),
+            B * ctx * 2.0 * spec.value_rank * spec.n_heads,
+            0.0,
+            B * 2.0 * spec.n_heads * spec.value_rank * spec.hidden]
+
+
 def measured_traffic(phase, tokens):
     """DRAM bytes of one launch of the phase's main kernel, from the ncu capture
     recorded in profiles/dram_traffic.json and scaled by cached tokens; None when
@@ -363,9 +384,15 @@ def run_ours(args, rank, ws, local):
     dbytes = decode_bytes(spec, L, B, T0 + W + K // 2)
     achieved = dbytes / (dec_ms * 1e-3) / 1e9
     pbytes = phase_bytes(spec, B, T0 + W + K // 2)
+    pflops = phase_flops(spec, B, T0 + W + K // 2)
+    tpeak, tpeak_kind = measured_tensor_peak()
     kernels = [{"phase": PHASES[p], "us": ph_ms[p] * 1e3, "algorithmic_bytes": pbytes[p],
                 "GB/s": (pbytes[p] / (ph_ms[p] * 1e-3) / 1e9) if ph_ms[p] > 0 else None,
-                "frac": (pbytes[p] / (ph_ms[p] * 1e-3) / 1e9 / peak) if ph_ms[p] > 0 else None}
+                "frac": (pbytes[p] / (ph_ms[p] * 1e-3) / 1e9 / peak) if ph_ms[p] > 0 else None,
+                # tensor-pipe co-bound: algorithmic flops over the measured dense fp16 peak
+                "algorithmic_flops": pflops[p],
+                "TFLOP/s": (pflops[p] / (ph_ms[p] * 1e-3) / 1e12) if ph_ms[p] > 0 else None,
+                "tensor_frac": (pflops[p] / (ph_ms[p] * 1e-3) / 1e12 / tpeak) if ph_ms[p] > 0 else None}
                for p in range(len(PHASES))]
     dom = max(range(len(PHASES)), key=lambda p: ph_ms[p])
     tokens_per_s = job_tokens_per_s(B, ws, ms_step)
@@ -395,7 +422,10 @@ def run_ours(args, rank, ws, local):
                      "traffic": measured_traffic(dom, B * (T0 + W + K // 2)),
                      "algorithmic_bytes": pbytes[dom], "us_per_launch": ph_ms[dom] * 1e3,
                      "whole_decode": {"achieved": achieved, "frac": achieved / peak, "algorithmic_bytes": dbytes,
-                                      "us": dec_ms * 1e3}},
+                                      "us": dec_ms * 1e3},
+                     "tensor_cobound": {"achieved": kernels[dom]["TFLOP/s"], "peak": tpeak, "peak_kind": tpeak_kind,
+                                        "unit": "TFLOP/s", "frac": kernels[dom]["tensor_frac"],
+                                        "algorithmic_flops": pflops[dom]}},
         "kernels": kernels,
         "e2e": {"value": B * ws / (e2e_ms * 1e-3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h},
