@@ -590,8 +590,19 @@ __global__ void __launch_bounds__(512) k_qprep_tc(LayerView v, const __nv_bfloat
                                                   const ScoreHead* __restrict__ heads, long long w_stride,
                                                   uint8_t* __restrict__ W) {
   __shared__ float qs[8][128];
+  __shared__ ScoreItem item;
+  __shared__ int row_head[128];   // head of each W'' row of the item (-1: padding)
+  __shared__ int nhi_s[kMaxItemHeads];
   const int b = blockIdx.x, it = blockIdx.y;
-  const ScoreItem item = items[it];
+  if (threadIdx.x == 0) item = items[it];
+  __syncthreads();
+  for (int row = threadIdx.x; row < item.npad; row += blockDim.x) {
+    int hh = -1;
+    for (int x = 0; x < item.nh; ++x)
+      if (row >= item.hcol[x] && row < item.hcol[x] + item.hr[x]) hh = x;
+    row_head[row] = hh;
+  }
+  if (threadIdx.x < item.nh) nhi_s[threadIdx.x] = shape_hi(heads[item.h0 + threadIdx.x].kind);
   const int pos = q_pos ? q_pos[b] : seq_lens[b] - 1;
   for (int idx = threadIdx.x; idx < item.nh * 64; idx += blockDim.x) {
     const int hh = idx / 64, p = idx % 64;
@@ -612,14 +623,12 @@ __global__ void __launch_bounds__(512) k_qprep_tc(LayerView v, const __nv_bfloat
   const uint32_t atom = (uint32_t)item.npad * 128u;
   for (int idx = threadIdx.x; idx < item.npad * 8; idx += blockDim.x) {
     const int row = idx >> 3, c = idx & 7;       // 8-column chunk c of the 64 (cos | sin) pairs
-    int hh = -1;
-    for (int x = 0; x < item.nh; ++x)
-      if (row >= item.hcol[x] && row < item.hcol[x] + item.hr[x]) hh = x;
+    const int hh = row_head[row];
     uint32_t re[4] = {0u, 0u, 0u, 0u}, im[4] = {0u, 0u, 0u, 0u};
     if (hh >= 0) {
       const int h = item.h0 + hh, g = h / v.group_q, j = row - item.hcol[hh];
       // pre-scale 2^(-c B) of the channel's place c in its code tuple (see code_float)
-      const int nhi = shape_hi(heads[h].kind);
+      const int nhi = nhi_s[hh];
       const float pre = j < nhi ? ((j % 32) % 2 ? 1.f / 16.f : 1.f)
                                 : (((j - nhi) % 32) % 3 == 0 ? 1.f : ((j - nhi) % 32) % 3 == 1 ? 1.f / 8.f : 1.f / 64.f);
       const float* B = Bk + ((size_t)key_off[g] + j) * 128 + c * 8;
