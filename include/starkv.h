@@ -50,7 +50,7 @@ typedef struct CUstream_st* starkv_stream_t;   /* same type as cudaStream_t */
 typedef enum {
   STARKV_OK = 0,
   STARKV_ERR_ARG = 1,          /* invalid argument (null pointer, bad size, bad shape) */
-  STARKV_ERR_UNSUPPORTED = 2,  /* valid, but not a combination this build implements */
+  STARKV_ERR_UNSUPPORTED = 2,  /* valid, but not a combination the library implements */
   STARKV_ERR_OOM = 3,          /* device allocation failed (load only) */
   STARKV_ERR_CUDA = 4,         /* a CUDA runtime call failed */
   STARKV_ERR_DEVICE = 5,       /* the device status word was set (see starkv_sync_status) */

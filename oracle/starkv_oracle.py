@@ -200,7 +200,7 @@ def dequantize_group(u: np.ndarray, s16: np.float16, bits: int) -> np.ndarray:
 
 # ---------------------------------------------------------------------------
 # Page format (16-token pages, as in vLLM-style paged KV blocks on the model
-# card; the byte layout itself is this build's reading).
+# card; the pages fix no byte layout, so this one is a reading).
 #
 #   page = latent block 0 | latent block 1 | ... | latent block L-1 | pad to 128 B
 #   latents in order: key latent of KV head 0 .. H_kv-1, then the joint value latent
