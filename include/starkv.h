@@ -204,6 +204,8 @@ STARKV_API starkv_status starkv_decode_attn(const starkv_layer* layer, const voi
  * appended).  Sequence b has q_len[b] queries at positions q_start[b] ..
  * q_start[b] + q_len[b] - 1; query i attends to slots [0, q_start[b] + i].
  *   q_start_host, q_len_host: HOST int32 arrays [batch] (they set the launch shape).
+ *     The per-row table built from them is copied from pageable host memory,
+ *     so this call synchronises `stream` before it returns.
  *   q: [sum q_len][H][d] in dtype, sequences one after another; out: [sum q_len][D].
  *   workspace: at least starkv_workspace_bytes(layer, batch, max_ctx, max q_len)
  *     bytes, where max_ctx >= every q_start[b] + q_len[b].  Layers that the
