@@ -259,6 +259,18 @@ def test_tc_other_bit_splits(top):
     run_decode(c, [300, 40], peaky=25.0, use_hidden=False, check_pool=False)
 
 
+def test_tc_empty_sequences_and_tile_edges():
+    """All-tensor-core decode with empty sequences (zero output rows) between
+    sequences that end exactly on and just past 128- and 256-token tile edges."""
+    run_decode(case(2), [300, 0, 128, 129, 0, 256, 17], use_hidden=False, check_pool=False)
+
+
+def test_tc_full_rope_table_length():
+    """A sequence as long as the RoPE table the layer was loaded with (32768
+    positions): the last score tile and the last RoPE tile coincide."""
+    run_decode(case(2), [32768, 5], use_hidden=False, check_pool=False)
+
+
 def test_tc_long_context_runs():
     """All-tensor-core decode with more super-tiles than SMs: CTAs whose unit
     ranges span several super-tiles and cross sequence boundaries."""
