@@ -63,3 +63,10 @@ def test_host_validation_before_cuda():
     assert raw.starkv_decode_attn(None, None, 0, None, 0, 1, None, None, None, None, None, 0, None) == 1
     assert raw.starkv_append(None, None, 0, None, 0, 0, 1, None, None, None, 0, None, 0, None) == 1
     assert raw.starkv_workspace_bytes(None, 1, 1, 1) == 0
+    assert raw.starkv_prefill_attn(None, None, 0, None, 0, 1, None, None, None, None, None, 0, None) == 1
+    # a top fraction outside [0, 1] is rejected before anything is allocated
+    cfg = lib.LayerConfig(hidden=64, n_heads=2, n_kv_heads=2, head_dim=8, key_ranks=[4, 4], value_rank=8,
+                          quantized=True, top_fraction=1.5)
+    with pytest.raises(lib.StarKVError) as e:
+        lib.load_factors(cfg, None, None, None, None, None, stream=0)
+    assert e.value.status == 1
