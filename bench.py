@@ -514,6 +514,70 @@ def run_prefill(args):
             "device_status": status}
 
 
+def run_plain(args):
+    """Time the decode of one uncompressed (plain) layer of the 32-layer stack
+    (K stored after RoPE and V in bf16 pages; the CUDA-core decode kernels and
+    the tensor-core output GEMM): batch and ctx from --batch/--ctx (default 16
+    and 4096).  Separate JSON line; not the headline metric."""
+    import numpy as np
+    import torch
+    from decode_attention_rank_b200 import starkv as lib
+    from synth import gen
+    B = args.batch or 16
+    T = args.ctx or 4096
+    assert T % 16 == 0
+    torch.cuda.set_device(0)
+    spec = gen.config_spec(4, layer=0)
+    f = gen.make_factors(spec, gen.LAYER_SEED[4], 0)
+
+    def t(x):
+        return torch.from_numpy(np.ascontiguousarray(x)).cuda().to(torch.bfloat16)
+    L = lib.load_factors(lib.LayerConfig.from_spec(spec), t(f.W_k), None, t(f.W_v), None, t(f.W_o))
+    pages = T // 16 + 1
+    n_pages = B * pages
+    g = torch.Generator(device="cuda")
+    g.manual_seed(2024)
+    page_table = torch.randperm(n_pages, generator=g, device="cuda").to(torch.int32).reshape(B, pages).contiguous()
+    pool = torch.empty(n_pages * L.page_bytes, dtype=torch.uint8, device="cuda")
+    L.cache_init(pool, n_pages)
+    for b in range(B):
+        for c0 in range(0, T, 4096):
+            n = min(4096, T - c0)
+            z = torch.randn(n, L.latent_total, generator=g, device="cuda")
+            L.append(pool, n_pages, page_table, torch.full((n,), b, dtype=torch.int32, device="cuda"),
+                     torch.arange(c0, c0 + n, dtype=torch.int32, device="cuda"), z, True)
+    q = (torch.randn(B, spec.n_heads, spec.head_dim, generator=g, device="cuda") /
+         math.sqrt(spec.head_dim)).to(torch.bfloat16)
+    out = torch.empty(B, spec.hidden, dtype=torch.bfloat16, device="cuda")
+    ws = torch.empty(L.workspace_bytes(B, pages * 16), dtype=torch.uint8, device="cuda")
+    lens = torch.full((B,), T, dtype=torch.int32, device="cuda")
+    for _ in range(args.warmup):
+        L.decode(pool, n_pages, page_table, lens, q, out, ws)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(args.steps):
+        L.decode(pool, n_pages, page_table, lens, q, out, ws)
+    e1.record()
+    torch.cuda.synchronize()
+    status = L.sync_status()
+    ms = e0.elapsed_time(e1) / args.steps
+    peak, peak_kind = measured_peaks()
+    # algorithmic bytes: K and V of every cached token (bf16) + W_o + q/out
+    dbytes = B * T * 2 * 2 * spec.n_kv_heads * spec.head_dim + 2 * spec.n_heads * spec.head_dim * spec.hidden + \
+        B * (spec.n_heads * spec.head_dim + spec.hidden) * 2
+    gbs = dbytes / (ms * 1e-3) / 1e9
+    return {"metric": "plain-layer decode tokens/s (uncompressed bf16 K/V)", "value": B / (ms * 1e-3),
+            "unit": "tokens/s", "n_gpus": 1, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16 K/V, fp32 accumulate",
+            "data": "synthetic", "mode": "plain",
+            "config": {"workload": f"plain layer (workload-4 layers 0, 1, 31) decode, batch {B}, ctx {T}",
+                       "batch": B, "ctx": T},
+            "roofline": {"bound": "hbm", "achieved": gbs, "peak": peak, "peak_kind": peak_kind, "unit": "GB/s",
+                         "frac": gbs / peak, "algorithmic_bytes": dbytes},
+            "device_status": status}
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -527,7 +591,12 @@ def main():
     ap.add_argument("--batch", type=int, default=0, help="sequences per step (default 16)")
     ap.add_argument("--prefill", type=int, default=0, help="time a causal prefill chunk of this many queries "
                     "(history = ctx - queries, ctx default 4096) instead of the decode step")
+    ap.add_argument("--plain", action="store_true", help="time the decode of an uncompressed layer of the "
+                    "32-layer stack instead (batch/ctx from --batch/--ctx, default 16 and 4096)")
     args = ap.parse_args()
+    if args.plain:
+        print(json.dumps(run_plain(args)), flush=True)
+        return
     if args.ctx:
         WORKLOAD["ctx"] = args.ctx
     if args.batch:
