@@ -429,7 +429,7 @@ def run_ours(args, rank, ws, local):
         "kernels": kernels,
         "e2e": {"value": B * ws / (e2e_ms * 1e-3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h},
-        "gpu_launches": K * 10,   # append: 3 kernels; decode: 7 (see the launch list under profiles/)
+        "gpu_launches": K * 10,   # append: 4 kernels; decode: 6 (see the launch list under profiles/)
         "clocks": clk,
     }
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:
