@@ -202,7 +202,7 @@ def latent_bytes(spec, r):
     """Algorithmic bytes of one token's latent of rank r (codes + fp16 scales, no page padding)."""
     if not spec.quantized:
         return r * (4 if spec.dtype == "f32" else 2)
-    n_hi = math.ceil(spec.top_fraction * r)
+    n_hi = math.ceil(spec.top_fraction * r - 1e-9)   # 0.2 * 40 is 8.000000000000002 in floating point
     n_lo = r - n_hi
     bits = spec.top_bits * n_hi + spec.bottom_bits * n_lo
     return bits / 8 + 2 * (math.ceil(n_hi / spec.group_size) + math.ceil(n_lo / spec.group_size))
