@@ -219,6 +219,12 @@ STARKV_API starkv_status starkv_prefill_attn(const starkv_layer* layer, const vo
                                   const int32_t* q_len_host, const void* q, void* out, void* workspace,
                                   size_t ws_bytes, starkv_stream_t stream);
 
+/*
+ * Workspace bytes for a decode of `batch` sequences (max_q = 1) or a prefill
+ * of `batch` sequences with up to max_q queries each, over a page table whose
+ * capacity is max_ctx tokens (max_pages * 16).  0 for a NULL layer.  The size
+ * covers whichever kernel path the layer can take (tensor-core or CUDA-core).
+ */
 STARKV_API size_t starkv_workspace_bytes(const starkv_layer* layer, int batch, int max_ctx, int max_q);
 
 /*
