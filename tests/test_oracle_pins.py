@@ -222,6 +222,34 @@ def test_hadamard_golden_and_orthogonal():
     assert np.allclose(np.abs(R), 1 / math.sqrt(32)) and np.all(R[0] > 0)
 
 
+def test_rotation_block_assembly():
+    # "STAR-KV 阅读笔记" section 6.1: the high-magnitude block and the ordinary block are rotated
+    # separately; the quantization groups (32 channels from each segment start) are the rotation
+    # blocks.  A latent's rotation is therefore the direct sum of the group rotations in channel
+    # order, assembled here by a library routine (scipy's block_diag), and each group rotation is
+    # the direct sum of normalised Sylvester matrices (scipy's hadamard) over the binary
+    # decomposition of its length, largest first.
+    import scipy.linalg as sl
+
+    def sylv(n):
+        return sl.hadamard(n) / math.sqrt(n)
+
+    spec = gen.LayerSpec(hidden=1, n_heads=1, n_kv_heads=1, head_dim=128, key_ranks=[20], value_rank=20,
+                         quantized=True, hadamard_block=32)
+    assert O.n_high(20, 0.25) == 5
+    np.testing.assert_allclose(O.group_rotation(5), sl.block_diag(sylv(4), sylv(1)), atol=1e-15)
+    np.testing.assert_allclose(O.group_rotation(15), sl.block_diag(sylv(8), sylv(4), sylv(2), sylv(1)),
+                               atol=1e-15)
+    want = sl.block_diag(sl.block_diag(sylv(4), sylv(1)), sl.block_diag(sylv(8), sylv(4), sylv(2), sylv(1)))
+    np.testing.assert_allclose(O.rotation(20, spec), want, atol=1e-15)
+    # r = 56: hi segment 14 channels (one group of 14 = 8 + 4 + 2), lo segment 42 = a group of 32 and one of 10
+    want = sl.block_diag(sylv(8), sylv(4), sylv(2), sylv(32), sylv(8), sylv(2))
+    np.testing.assert_allclose(O.rotation(56, spec), want, atol=1e-15)
+    # no rotation without a Hadamard block, or without quantization
+    np.testing.assert_array_equal(O.rotation(20, gen.LayerSpec(**{**spec.__dict__, "hadamard_block": 0})), np.eye(20))
+    np.testing.assert_array_equal(O.rotation(20, gen.LayerSpec(**{**spec.__dict__, "quantized": False})), np.eye(20))
+
+
 def test_absorbed_rotation_leaves_kv_unchanged():
     spec = small_spec(quantized=True, hadamard_block=32, key_ranks=[20], n_kv_heads=1, n_heads=1, value_rank=40,
                       head_dim=64, hidden=96)
@@ -377,6 +405,92 @@ def test_brute_force_tiny():
     np.testing.assert_allclose(out, [y[0], 3.0 * y[1]], rtol=1e-14)
 
 
+def _gqa_tiny():
+    # H = 4 query heads over H_kv = 2 KV heads, d = 2, T = 2, no RoPE, identity up-projections
+    # (r = d per KV head, r_v = H_kv d), so the stored latents are the keys and values themselves.
+    spec = gen.LayerSpec(hidden=2, n_heads=4, n_kv_heads=2, head_dim=2, key_ranks=[2, 2], value_rank=4, dtype="f32")
+    Wo = np.zeros((8, 2))
+    for h in range(4):
+        Wo[2 * h:2 * h + 2] = (h + 1) * np.eye(2)        # W_o,h = (h + 1) I: every head weighs differently
+    f = gen.LayerFactors(A_k=[None, None], B_k=[np.eye(2), np.eye(2)], A_v=None, B_v=np.eye(4), W_o=Wo)
+    keys = [np.array([[1.0, 0.0], [0.0, 1.0]]),             # KV head 0
+            np.array([[0.0, 4.0], [-2.0, 0.0]])]            # KV head 1: very different keys
+    vals = np.array([[1.0, 0.0, 5.0, 0.0],                  # token 0: V_0 = (1, 0),  V_1 = (5, 0)
+                     [0.0, 1.0, 0.0, -7.0]])                # token 1: V_0 = (0, 1),  V_1 = (0, -7)
+    q = np.array([[2.0, 0.0], [0.0, 1.0], [1.0, 1.0], [-1.0, 3.0]])
+    return spec, f, keys + [vals], q
+
+
+def test_gqa_head_map_brute_force():
+    # SURVEY reading Q9 of the LLaMA-3-8B-shaped workload ("4 query heads per KV head sharing each
+    # latent tile"): contiguous groups, kv(h) = h // (H / H_kv), here [0, 0, 1, 1].  Expected output
+    # by hand: s_t = q_h . k_t / sqrt(2); p_0 = 1 / (1 + exp(s_1 - s_0)); y_h = p_0 v_0 + p_1 v_1.
+    spec, f, Zh, q = _gqa_tiny()
+    out = O.decode(spec, f, Zh, q, 1, 2)
+    kv = [0, 0, 1, 1]
+    keys, vals = Zh[:2], Zh[2]
+    want = np.zeros(2)
+    for h in range(4):
+        g = kv[h]
+        s0 = float(q[h] @ keys[g][0]) / math.sqrt(2.0)
+        s1 = float(q[h] @ keys[g][1]) / math.sqrt(2.0)
+        p0 = 1.0 / (1.0 + math.exp(s1 - s0))
+        y = p0 * vals[0, 2 * g:2 * g + 2] + (1.0 - p0) * vals[1, 2 * g:2 * g + 2]
+        want += (h + 1) * y
+    np.testing.assert_allclose(out, want, rtol=1e-13)
+    assert [O.kv_of(h, spec) for h in range(4)] == kv
+
+
+def _plain_and_latent_specs():
+    # GQA, RoPE on, so that the plain-layer path also exercises the head map and both RoPE sides.
+    kw = dict(hidden=24, n_heads=4, n_kv_heads=2, head_dim=8, dtype="f32", rope=True, rope_theta=10000.0)
+    plain = gen.LayerSpec(key_ranks=[8, 8], value_rank=16, plain=True, **kw)
+    latent = gen.LayerSpec(key_ranks=[8, 8], value_rank=16, **kw)
+    return plain, latent
+
+
+def test_plain_layer_equals_full_rank_latent_layer():
+    # Full-rank identity (spec: at full rank with orthogonal factors the method equals plain
+    # attention): A_k,g = W_k,g, B_k,g = I, A_v = W_v, B_v = I.  The latent-layer oracle (itself
+    # pinned to textbook attention and to brute force above) must then agree with the plain-layer
+    # oracle over the stored post-RoPE keys and plain values of the same hidden states.
+    plain, latent = _plain_and_latent_specs()
+    f = gen.make_factors(plain, 21)
+    T, d = 11, plain.head_dim
+    X = gen.hidden_states(21, 0, 0, T, plain.hidden)
+    Zp = O.plain_latents(plain, f, X, np.arange(T))
+    Khat, Vhat = Zp[:, :2 * d].astype(np.float64), Zp[:, 2 * d:].astype(np.float64)
+    fl = gen.LayerFactors(A_k=[f.W_k[:, :d], f.W_k[:, d:]], B_k=[np.eye(d), np.eye(d)], A_v=f.W_v,
+                          B_v=np.eye(2 * d), W_o=f.W_o)
+    Zl = [O.project(X, fl.A_k[0], np.eye(d)), O.project(X, fl.A_k[1], np.eye(d)), O.project(X, f.W_v, np.eye(2 * d))]
+    Zl = [z.astype(np.float64) for z in Zl]
+    q = gen.queries(21, 0, 1, plain.n_heads, d)[0, 0] * 4.0
+    for q_pos, n in ((T - 1, T), (T + 5, T), (3, 7)):
+        a = O.decode_plain(plain, f, Khat, Vhat, q, n, q_pos)
+        b = O.decode(latent, fl, Zl, q, q_pos, n)
+        np.testing.assert_allclose(a, b, rtol=2e-6, atol=2e-7)   # float32 rounding of the stored values only
+
+
+def test_plain_layer_single_token_closed_form():
+    # T = 1: every head's softmax is [1], so out = sum_h v_0[kv(h)] W_o,h whatever the query.
+    plain, _ = _plain_and_latent_specs()
+    f = gen.make_factors(plain, 22)
+    d = plain.head_dim
+    X = gen.hidden_states(22, 0, 0, 1, plain.hidden)
+    Zp = O.plain_latents(plain, f, X, np.arange(1)).astype(np.float64)
+    q = gen.queries(22, 0, 1, plain.n_heads, d)[0, 0]
+    out = O.decode_plain(plain, f, Zp[:, :2 * d], Zp[:, 2 * d:], q, 1, 0)
+    v0 = (X @ f.W_v)[0]
+    want = sum(v0[(h // 2) * d:(h // 2 + 1) * d] @ f.W_o[h * d:(h + 1) * d] for h in range(4))
+    np.testing.assert_allclose(out, want, rtol=1e-6, atol=1e-7)
+    # the stored key at position 0 is not rotated (angle 0), and RoPE keeps norms at any position
+    np.testing.assert_allclose(Zp[0, :2 * d], (X @ f.W_k)[0], rtol=1e-6, atol=1e-7)
+    Zp5 = O.plain_latents(plain, f, np.repeat(X, 6, axis=0), np.arange(6)).astype(np.float64)
+    for g in range(2):
+        np.testing.assert_allclose(np.linalg.norm(Zp5[:, g * d:(g + 1) * d], axis=1),
+                                   np.linalg.norm((X @ f.W_k)[0, g * d:(g + 1) * d]), rtol=1e-6)
+
+
 def test_prefill_is_causal():
     spec = small_spec(rope=True)
     f, X, Z, Zh, q = _unq_inputs(spec, 7, seed=6)
@@ -461,3 +575,24 @@ def test_planted_mistakes_are_caught(monkeypatch):
         e = np.exp(s)
         return e / np.sum(e, axis=-1, keepdims=True) * 0.999
     _fails(test_brute_force_tiny, monkeypatch, "softmax", softmax_no_max)
+
+    def kv_modulo(h, spec):             # interleaved instead of contiguous head groups
+        return h % spec.n_kv_heads
+    _fails(test_gqa_head_map_brute_force, monkeypatch, "kv_of", kv_modulo)
+
+    good_decode_plain = O.decode_plain
+
+    def plain_query_not_roped(spec, f, Khat, Vhat, q, seq_len, q_pos):
+        return good_decode_plain(gen.LayerSpec(**{**spec.__dict__, "rope": False}), f, Khat, Vhat, q, seq_len, q_pos)
+    _fails(test_plain_layer_equals_full_rank_latent_layer, monkeypatch, "decode_plain", plain_query_not_roped)
+
+    good_plain_latents = O.plain_latents
+
+    def plain_keys_shifted(spec, f, X, positions):   # keys roped one position late
+        return good_plain_latents(spec, f, X, np.asarray(positions) + 1)
+    _fails(test_plain_layer_equals_full_rank_latent_layer, monkeypatch, "plain_latents", plain_keys_shifted)
+    _fails(test_plain_layer_single_token_closed_form, monkeypatch, "plain_latents", plain_keys_shifted)
+
+    def rotation_whole_latent(r, spec):  # one rotation across the hi and lo segments
+        return O.group_rotation(r) if spec.quantized and spec.hadamard_block else np.eye(r)
+    _fails(test_rotation_block_assembly, monkeypatch, "rotation", rotation_whole_latent)
