@@ -1,10 +1,13 @@
 // Host side of the C ABI: argument checks, layer planning (page layout, group
 // tables), factor folding at load time, and kernel dispatch.
+#include <limits.h>
 #include <math.h>
 #include <stdio.h>
 #include <string.h>
 
 #include <algorithm>
+#include <map>
+#include <mutex>
 #include <string>
 
 #include "starkv_internal.cuh"
@@ -28,6 +31,20 @@ int num_sms() {
     cached[dev] = std::min(n, 256);   // persistent grids: one CTA per SM, at most 256
   }
   return cached[dev];
+}
+
+cudaError_t set_smem_limit(const void* kernel, size_t bytes) {
+  static std::mutex mu;
+  static std::map<std::pair<const void*, int>, size_t> done;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  std::lock_guard<std::mutex> lock(mu);
+  size_t& have = done[{kernel, dev}];
+  if (have >= bytes) return cudaSuccess;
+  e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+  if (e == cudaSuccess) have = bytes;
+  return e;
 }
 
 // Channels of the high-precision segment: ceil(top_fraction * r) (reading notes
@@ -87,6 +104,7 @@ static starkv_status plan_layer(starkv_layer* L) {
     ld.block_off = (int)off;
     ld.ch_off = ch;
     ld.group0 = (int)L->grp.size();
+    ld.cmajor = (quant && li + 1 == widths.size()) ? 1 : 0;
     if (!quant) {
       L->grp.push_back(GroupDesc{0, ld.width, 0, 0});
       ld.n_groups = 1;
@@ -374,6 +392,7 @@ starkv_status starkv_append(const starkv_layer* L, void* pool, int64_t n_pages, 
   CHECK_ARG(pool && page_table && seq_idx && positions && input, "NULL buffer");
   CHECK_ARG(((uintptr_t)pool & 15) == 0, "pool must be 16-byte aligned");
   CHECK_ARG(n_pages > 0 && max_pages > 0 && n_seqs > 0, "empty pool or page table");
+  CHECK_ARG(max_pages <= INT_MAX / kPage, "max_pages * 16 overflows int");
   cudaStream_t s = (cudaStream_t)stream;
   const float* z = (const float*)input;
   if (!input_is_latent) {
@@ -458,6 +477,7 @@ starkv_status starkv_decode_attn(const starkv_layer* L, const void* pool, int64_
   if (batch == 0) return STARKV_OK;
   CHECK_ARG(pool && page_table && seq_lens && q && out, "NULL buffer");
   CHECK_ARG(n_pages > 0 && max_pages > 0, "empty pool or page table");
+  CHECK_ARG(max_pages <= INT_MAX / kPage, "max_pages * 16 overflows int");
   const int max_len = max_pages * kPage;
   const bool tc_ok = L->tc_scores && max_len <= L->rope_tiles * 128;
   const bool use_tc_all = tc_ok && L->tc_values && L->decode_path == 0;
@@ -489,6 +509,7 @@ starkv_status starkv_prefill_attn(const starkv_layer* L, const void* pool, int64
   if (batch == 0) return STARKV_OK;
   CHECK_ARG(pool && page_table && q_start_host && q_len_host && q && out, "NULL buffer");
   CHECK_ARG(n_pages > 0 && max_pages > 0, "empty pool or page table");
+  CHECK_ARG(max_pages <= INT_MAX / kPage, "max_pages * 16 overflows int");
   std::vector<int32_t> tab;
   int rows = 0, max_len = 0;
   for (int b = 0; b < batch; ++b) {

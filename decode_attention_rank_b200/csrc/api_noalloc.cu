@@ -1,6 +1,8 @@
 // Decode attention for callers that cannot allocate device memory: the same
 // kernels as starkv_decode_attn, with their scratch in a fixed device array of
 // this library instead of a caller workspace.
+#include <limits.h>
+
 #include <mutex>
 #include <string>
 
@@ -57,6 +59,10 @@ extern "C" starkv_status starkv_decode_attn_noalloc(const starkv_layer* L, const
   if (batch == 0) return STARKV_OK;
   if (!(pool && page_table && seq_lens && q && out) || n_pages <= 0 || max_pages <= 0) {
     set_error("NULL buffer or empty pool / page table");
+    return STARKV_ERR_ARG;
+  }
+  if (max_pages > INT_MAX / kPage) {
+    set_error("max_pages * 16 overflows int");
     return STARKV_ERR_ARG;
   }
   const size_t need = starkv_workspace_bytes(L, batch, max_pages * kPage, 1);

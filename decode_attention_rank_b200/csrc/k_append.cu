@@ -133,7 +133,7 @@ __global__ void k_pack(LayerView v, uint8_t* __restrict__ pool, long long n_page
     const uint32_t u = (uint32_t)(q + (1 << (gd.bits - 1)));
     if (lane == 0) reinterpret_cast<__half*>(blk)[g * kPage + slot] = s16;
     if (lane < gd.n) {
-      const uint32_t bit = (uint32_t)(slot * gd.n + lane) * gd.bits;
+      const uint32_t bit = code_bit(slot, lane, gd.n, gd.bits, ld.cmajor);
       uint32_t* w = reinterpret_cast<uint32_t*>(blk + gd.code_off) + (bit >> 5);
       const uint32_t sh = bit & 31;
       atomicOr(w, u << sh);
@@ -186,7 +186,7 @@ __global__ void k_pack_groups(LayerView v, const int* __restrict__ grp_lat, int 
   const uint32_t u = (uint32_t)(q + (1 << (gd.bits - 1)));
   if (lane == 0) reinterpret_cast<__half*>(blk)[g * kPage + slot] = s16;
   if (lane < gd.n) {
-    const uint32_t bit = (uint32_t)(slot * gd.n + lane) * gd.bits;
+    const uint32_t bit = code_bit(slot, lane, gd.n, gd.bits, ld.cmajor);
     uint32_t* w = reinterpret_cast<uint32_t*>(blk + gd.code_off) + (bit >> 5);
     const uint32_t sh = bit & 31;
     atomicOr(w, u << sh);

@@ -50,7 +50,7 @@ __device__ __forceinline__ float latent_value(const LayerView& v, const uint8_t*
     if (j >= v.grp[ld.group0 + k].start) g = k;
   const GroupDesc gd = v.grp[ld.group0 + g];
   const float s = __half2float(reinterpret_cast<const __half*>(blk)[g * kPage + slot]);
-  const uint32_t bit = (uint32_t)(slot * gd.n + (j - gd.start)) * gd.bits;
+  const uint32_t bit = code_bit(slot, j - gd.start, gd.n, gd.bits, ld.cmajor);
   const uint32_t* w = reinterpret_cast<const uint32_t*>(blk + gd.code_off) + (bit >> 5);
   const uint32_t sh = bit & 31;
   uint32_t u = w[0] >> sh;
@@ -381,17 +381,13 @@ cudaError_t launch_decode_generic(const starkv_layer* L, const uint8_t* pool, lo
   int rmax = 0;
   for (int g = 0; g < v.Hkv; ++g) rmax = std::max(rmax, L->lat[g].width);
   const size_t smem = sizeof(float) * kTile * (size_t)(rmax + v.d);
-  static size_t attr_set = 0;
-  if (smem > attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(k_scores, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
-    attr_set = smem;
-  }
+  cudaError_t e = set_smem_limit((const void*)k_scores, smem);
+  if (e != cudaSuccess) return e;
   if (tc_scores) {
     // scores (log2 units) from the tensor-core kernel, written into S
     ScoreOut so;
-    cudaError_t e = launch_scores_tc(L, pool, n_pages, page_table, max_pages, rows, ri.row_len, ri.row_pos, q,
-                                     w + p.total, &so, S, p.S_ld, s);
+    e = launch_scores_tc(L, pool, n_pages, page_table, max_pages, rows, ri.row_len, ri.row_pos, q, w + p.total, &so,
+                         S, p.S_ld, s);
     if (e != cudaSuccess) return e;
   } else {
     k_scores<<<dim3((max_len + kTile - 1) / kTile, v.Hkv, rows), 256, smem, s>>>(
@@ -411,11 +407,11 @@ cudaError_t launch_decode_generic(const starkv_layer* L, const uint8_t* pool, lo
   const int KT = L->Kp / 64;
   // padding rows and columns of the y tiles must be zero
   if (rows % NB != 0 || L->Kp != v.H * v.wv) {
-    cudaError_t e = cudaMemsetAsync(y, 0, p.y_bytes, s);
+    e = cudaMemsetAsync(y, 0, p.y_bytes, s);
     if (e != cudaSuccess) return e;
   }
   k_combine_tiled<<<dim3(rows, v.H), 128, 0, s>>>(v, p.n_splits, pY, pm, pl, NB, KT, (uint8_t*)y);
-  cudaError_t e = cudaGetLastError();
+  e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   return launch_outproj_tc(L, y, rows, out, (float*)(w + p.part), s);
 }

@@ -256,12 +256,8 @@ cudaError_t launch_gemm_tc(const uint8_t* Mt, int n_out, int K, int n_valid, con
   a.tmem_cols = cols;
   a.status = status;
   const size_t smem = (size_t)a.stages * stage_bytes + 1024;
-  static size_t attr = 0;
-  if (smem > attr) {
-    cudaError_t e = cudaFuncSetAttribute(k_outproj_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
-    attr = smem;
-  }
+  cudaError_t e = set_smem_limit((const void*)k_outproj_tc, smem);
+  if (e != cudaSuccess) return e;
   for (int t = 0; t < ntiles; ++t) {
     OutArgs at = a;
     at.y = a.y + (size_t)t * g.KT * NB * 128;

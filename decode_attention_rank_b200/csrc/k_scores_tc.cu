@@ -822,12 +822,8 @@ cudaError_t launch_scores_tc(const starkv_layer* L, const uint8_t* pool, long lo
   a.KS = L->KS;
   a.status = L->status;
   const size_t smem = 2 * kETileBytes + (size_t)a.WS * a.w_stage + (size_t)a.KS * a.k_stage + 1024;
-  static size_t attr = 0;
-  if (smem > attr) {
-    e = cudaFuncSetAttribute(k_scores_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
-    attr = smem;
-  }
+  e = set_smem_limit((const void*)k_scores_tc, smem);
+  if (e != cudaSuccess) return e;
   const int G = (int)std::min<long long>(num_sms(), a.U);
   k_scores_tc<<<G, kScoreThreads, smem, s>>>(a);
   return cudaGetLastError();

@@ -4,11 +4,15 @@
 //
 //     Y_h = sum_t p_h(t) zhat_v(t)       for all query heads h at once
 //
-// computed transposed, Y^T = Zv^T P^T: the dequantized value latent of a
-// 128-token tile is the A operand (M = 128 value channels per block, stored
-// MN-major as [token][channel] fp16, which is the order the codes are decoded
-// in), the stacked probabilities are B (N = heads, K-major), and Y^T for every
-// 128-channel block stays in TMEM for a whole run of super-tiles.
+// computed transposed, Y^T = Zv^T P^T: the dequantized value latent of one
+// 16-token page is the A operand (M = 128 value channels per block, K = the
+// page's 16 tokens), the stacked probabilities are B (N = heads, K-major in
+// shared memory), and Y^T for every 128-channel block stays in TMEM for a
+// whole run of pages.  The A tiles never touch shared memory: the value
+// latent's codes are stored channel-major, so a thread that owns one channel
+// (one TMEM lane) finds that channel's 16 codes in one field, turns them into
+// fp16 token pairs in registers and stores them straight into TMEM, where the
+// MMA reads A.
 //
 // P comes from the score kernel as exp2(s - m_g) per 32-token group; it is
 // rescaled by exp2(m_g - M) with M the maximum over the CTA's run of the
@@ -16,12 +20,12 @@
 // partial (M, l, Y) per run of one sequence; a combine kernel merges the runs.
 //   warp 0      tcgen05.mma issue, TMEM allocation
 //   warps 1-4   P staging: rescaled fp16 P tiles (the B operand), M and l;
-//               warp s takes the 32-token group s of every tile
+//               warp s takes the 32-token group s of every 128-token tile
 //   warp 5      bulk copies of the pages' value blocks, a page at a time
-//   warps 6-21  workers: worker w dequantizes items w, w + 16, ... (an item =
-//               one page's 16 tokens x 128 value channels) from the
-//               copied pages into its two A stages, and reads Y^T out of TMEM at the
-//               end of each run
+//   warps 6-21  workers: every page is split over the 16 workers by (TMEM
+//               lane quarter, 128-channel block); each dequantizes its
+//               channel groups of the page into the page's A slot in TMEM,
+//               and reads Y^T out of TMEM at the end of each run
 #include <float.h>
 
 #include "tc_common.cuh"
@@ -30,22 +34,15 @@ namespace starkv {
 
 namespace {
 
-constexpr int kValWorkers = 16;                          // dequantizing warps
+constexpr int kValWorkers = 16;                          // dequantizing warps (four per TMEM lane quarter)
 constexpr int kStagers = 4;                              // P staging warps, one per 32-token group of a tile
 constexpr int kValThreads = 32 * (2 + kStagers + kValWorkers);   // MMA, P staging, page copies, workers
-// A stages: item n sits in stage n % kAStages and worker w takes the items
-// n = w (mod kValWorkers), so each stage has one writer, every worker owns two
-// stages, and a worker is never more than one barrier phase ahead of a stage.
-constexpr int kAStages = 2 * kValWorkers;
-// Raw stages: page p of the CTA's tiles (the value block of 16 tokens) lands
-// in stage p % n_raw.  A worker's consecutive items lie 32 / nblk pages apart;
-// at least that many raw stages keep a worker within one barrier phase of the
-// raw stage it reads.
 constexpr int kMaxRawStages = 32;
+constexpr int kMaxASlots = 8;    // pages whose A tiles are in TMEM at once
 constexpr int kVSuper = 256;     // tokens per super-tile (matches the score kernel)
-constexpr int kAStage = 4096;    // one A stage: 16 tokens (one page) x 128 value channels, fp16
 constexpr int kMaxRuns = 64;     // runs (sequences) per CTA
 constexpr int kRunMaxCache = 16; // runs whose per-head maxima are computed up front
+constexpr int kMaxTiles = 256;   // 128-token tiles per CTA
 
 // Atomic maximum of floats (no NaN) through their integer orderings.
 __device__ __forceinline__ void atomic_max_float(float* addr, float v) {
@@ -64,6 +61,7 @@ struct ValArgs {
   int vblk_off, vblk_bytes;     // value latent block inside a page
   int raw_stage;                // bytes of one raw stage (a page's value block, 128-byte aligned)
   int n_raw;                    // raw stages
+  int na;                       // A slots in TMEM
   const GroupDesc* vgrp;        // value latent groups (all of 32 channels)
   int rv, H;
   int lg_nblk;                  // log2 of the 128-channel blocks of the value latent
@@ -77,62 +75,51 @@ struct ValArgs {
   float* Y;                     // [G][slots][H][rv]
   float* mseg;                  // [G][slots][H]
   float* lseg;
-  uint32_t tmem_cols;
   uint32_t* status;
 };
 
 __device__ __forceinline__ long long vunit_lo(int c, int G, long long U) { return (long long)c * U / G; }
 
-// The CTA's 128-token tiles, in order: units u0 .. u1 - 1, up to two tiles
-// each, those that start below the sequence length.  A run is a maximal
-// stretch of tiles of one sequence.  Built once per CTA in shared memory:
-// per tile (sequence, first token, length, run) and its eight page ids.
-constexpr int kMaxTiles = 256;
-
-// One lane's data of a worker item (value channels [128 cb, 128 cb + 128) of
-// one token): the four groups' code words and fp16 scales.
-struct VData {
-  uint32_t w[4][4];
-  uint32_t sc[4];
-};
-
-// Dequantization of 8 codes of one group into four fp16 pairs, in the chunk
-// order (c0,c2) (c1,c3) (c4,c6) (c5,c7): each 16-bit lane holds 1024 + u (an
-// exact fp16 integer), one exact subtraction of 1024 + 2^(B-1) and one
-// correctly rounded multiply by the fp16 scale give (u - 2^(B-1)) * scale.
-// The A tile therefore stores, inside every 8-channel chunk, channels
-// 0 2 1 3 4 6 5 7; the combine kernel puts them back in order.
-__device__ __forceinline__ uint32_t deq2(uint32_t lanes, __half2 sub, __half2 s2) {
-  const uint32_t x = lanes | 0x64006400u;
-  __half2 h = *reinterpret_cast<const __half2*>(&x);
-  h = __hmul2(__hsub2(h, sub), s2);
+// Two fp16 lanes holding 1024 + u (an exact fp16 integer: the code in the
+// low mantissa bits of 0x6400) -> (u - 2^(B-1)) * scale: one exact
+// subtraction of 1024 + 2^(B-1), one correctly rounded multiply by the
+// token's fp16 scale.
+__device__ __forceinline__ uint32_t deq_pair(uint32_t x, __half2 sub, uint32_t scales) {
+  __half2 h = __hmul2(__hsub2(*reinterpret_cast<const __half2*>(&x), sub),
+                      *reinterpret_cast<const __half2*>(&scales));
   return *reinterpret_cast<uint32_t*>(&h);
 }
-__device__ __forceinline__ uint4 deq8_b4(uint32_t run, __half2 sub, __half2 s2) {
-  const uint32_t x01 = __byte_perm(run, 0u, 0x4140u);   // bytes c1c0 | c3c2 into the two 16-bit lanes
-  const uint32_t x23 = __byte_perm(run, 0u, 0x4342u);
-  uint4 o;
-  o.x = deq2(x01 & 0x000F000Fu, sub, s2);           // (c0, c2)
-  o.y = deq2((x01 >> 4) & 0x000F000Fu, sub, s2);    // (c1, c3)
-  o.z = deq2(x23 & 0x000F000Fu, sub, s2);           // (c4, c6)
-  o.w = deq2((x23 >> 4) & 0x000F000Fu, sub, s2);    // (c5, c7)
-  return o;
+
+// One channel's 16 codes (its field of a channel-major code block) -> eight
+// fp16 pairs, pair c = tokens (2c, 2c + 1) of the page, the layout of one
+// 128 x 16 A tile row in TMEM.  The field holds the even slots first, then
+// the odd slots, so each pair comes out of one shift and mask.
+//   4-bit: word 0 = slots 0 2 4 .. 14, word 1 = slots 1 3 .. 15 (a nibble each);
+//          byte j of both words, side by side, gives pairs 2j and 2j + 1.
+//   3-bit: 48 bits, slots 0 2 .. 14 at bits 0-23, slots 1 3 .. 15 at 24-47;
+//          pair c sits at bits 3c and 24 + 3c.
+__device__ __forceinline__ void deq_channel4(uint32_t w0, uint32_t w1, __half2 sub, const uint32_t* sc,
+                                             uint32_t* out) {
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const uint32_t r = __byte_perm(w0, w1, (uint32_t)j | ((uint32_t)(4 + j) << 8));
+    out[2 * j] = deq_pair((r & 0x000F000Fu) | 0x64006400u, sub, sc[2 * j]);
+    out[2 * j + 1] = deq_pair(((r >> 4) & 0x000F000Fu) | 0x64006400u, sub, sc[2 * j + 1]);
+  }
 }
-__device__ __forceinline__ uint4 deq8_b3(uint32_t run, __half2 sub, __half2 s2) {
-  uint4 o;
-  o.x = deq2((run & 0x7u) | ((run << 10) & 0x70000u), sub, s2);           // c0 bits 0-2, c2 bits 6-8
-  o.y = deq2(((run >> 3) & 0x7u) | ((run << 7) & 0x70000u), sub, s2);     // c1 bits 3-5, c3 bits 9-11
-  o.z = deq2(((run >> 12) & 0x7u) | ((run >> 2) & 0x70000u), sub, s2);    // c4 bits 12-14, c6 bits 18-20
-  o.w = deq2(((run >> 15) & 0x7u) | ((run >> 5) & 0x70000u), sub, s2);    // c5 bits 15-17, c7 bits 21-23
-  return o;
+__device__ __forceinline__ void deq_channel3(uint64_t x, __half2 sub, const uint32_t* sc, uint32_t* out) {
+#pragma unroll
+  for (int c = 0; c < 8; ++c) {
+    // codes at bits 0-2 and 24-26 -> bytes 0 and 2, 0x64 into bytes 1 and 3
+    const uint32_t t = (uint32_t)(x >> (3 * c)) & 0x07000007u;
+    out[c] = deq_pair(__byte_perm(t, 0x64646464u, 0x4340u), sub, sc[c]);
+  }
 }
 
 __global__ void __launch_bounds__(kValThreads, 1) k_values_tc(ValArgs a) {
   extern __shared__ uint8_t smem_raw[];
-  // chain c = items 8 c .. 8 c + 7 (eight workers, A stages (8 c .. 8 c + 7)
-  // % kAStages): ch_full[c % 4] when the eight are written, ch_done[c % 4]
-  // when their MMAs have completed
-  __shared__ __align__(8) uint64_t ch_full[4], ch_done[4], r_full[kMaxRawStages], r_empty[kMaxRawStages];
+  __shared__ __align__(8) uint64_t a_full[kMaxASlots], a_free[kMaxASlots], r_full[kMaxRawStages],
+      r_empty[kMaxRawStages];
   __shared__ __align__(8) uint64_t p_full[2], p_empty[2];
   __shared__ __align__(8) uint64_t seg_done, acc_free, fin;
   __shared__ uint32_t tmem_base;
@@ -143,11 +130,10 @@ __global__ void __launch_bounds__(kValThreads, 1) k_values_tc(ValArgs a) {
   __shared__ uint8_t rsp_s[kMaxTiles * 8];   // per page of the CTA: raw stage | phase parity << 7
   __shared__ int run_b[kMaxRuns];
   __shared__ int n_tiles_s, n_runs_s;
-  __shared__ float l_stage[64];           // run sums of the staged P, per head
+  __shared__ float l_part[kStagers][64];  // per stager warp and head: its part of the run sum of the staged P
   __shared__ float runM_s[kRunMaxCache][64];   // per run and head: the maximum of the 32-token group maxima
   uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
-  uint8_t* A_s = smem;                                   // kAStages x 8 KB A stages
-  uint8_t* P_s = A_s + kAStages * kAStage;               // 2 x (H x 128 fp16, K-major swizzled)
+  uint8_t* P_s = smem;                                   // 2 x (H x 128 fp16, K-major swizzled)
   uint8_t* R_s = P_s + 2 * a.H * 256;                    // n_raw raw stages
   const int p_stage = a.H * 256;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -155,17 +141,18 @@ __global__ void __launch_bounds__(kValThreads, 1) k_values_tc(ValArgs a) {
   const long long u0 = vunit_lo(cta, G, a.U), u1 = vunit_lo(cta + 1, G, a.U);
   const int lnb = a.lg_nblk;                             // 128-channel blocks: 1 << lnb
   const int nblk = 1 << lnb;
-  const int lg_ipt = lnb + 3;                            // worker items per tile: 8 * nblk
+  const uint32_t ycols = (uint32_t)(nblk * a.H);         // TMEM columns of Y^T; the A slots follow
+  const int n_act = 4 * min(4, nblk);                    // workers with at least one channel block
   const int b_first = (int)(u0 / a.n_st);
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < 4; ++s) {
-      tc::mbar_init(&ch_full[s], 8);
-      tc::mbar_init(&ch_done[s], 1);
+    for (int s = 0; s < a.na; ++s) {
+      tc::mbar_init(&a_full[s], n_act);
+      tc::mbar_init(&a_free[s], 1);
     }
     for (int s = 0; s < a.n_raw; ++s) {
       tc::mbar_init(&r_full[s], 1);
-      tc::mbar_init(&r_empty[s], 1 << a.lg_nblk);   // the page's items, one per 128-channel block
+      tc::mbar_init(&r_empty[s], n_act);
     }
     for (int s = 0; s < 2; ++s) {
       tc::mbar_init(&p_full[s], kStagers);
@@ -175,7 +162,6 @@ __global__ void __launch_bounds__(kValThreads, 1) k_values_tc(ValArgs a) {
     tc::mbar_init(&acc_free, kValWorkers);
     tc::mbar_init(&fin, 1);
     abort_flag = 0;
-    for (int h = 0; h < 64; ++h) l_stage[h] = 0.f;
     tc::fence_mbar_init();
   }
   for (int g = threadIdx.x; g < a.rv / 32; g += blockDim.x) {
@@ -223,7 +209,7 @@ __global__ void __launch_bounds__(kValThreads, 1) k_values_tc(ValArgs a) {
       n_runs_s = min(nr, kMaxRuns);
     }
   }
-  if (warp == 0) tc::tmem_alloc(&tmem_base, a.tmem_cols);
+  if (warp == 0) tc::tmem_alloc(&tmem_base, 512);
   tc::tc_fence_before();
   __syncthreads();
   tc::tc_fence_after();
@@ -259,21 +245,16 @@ __global__ void __launch_bounds__(kValThreads, 1) k_values_tc(ValArgs a) {
 
   if (warp == 0) {
     // ------------------------------------------------ MMA issue
-    // Item n of the CTA (tile n / ipt, item n % ipt = nblk k + cb: page k of
-    // the tile, 128-channel block cb) sits in A stage n % kAStages; its one
-    // K = 16 MMA adds block cb's Y^T.  A chain's eight items are waited for
-    // together and their MMAs issued back to back: an N = 32 MMA takes only
-    // about 45 cycles on the tensor pipe, so the issuing thread must spend
-    // very few instructions per MMA.
+    // Page p of the CTA (page k = p % 8 of tile p / 8) sits in A slot p % na:
+    // block cb's 128 x 16 A tile at TMEM column ycols + (slot * nblk + cb) * 8;
+    // its K = 16 MMA adds block cb's Y^T (columns cb * H ..).
     if (lane == 0) {
-      const uint32_t idesc = tc::idesc_f16(128, a.H, false, true, false);
-      // descriptors as (low, high) halves; steps are 16-byte units on the low half
-      const uint64_t a0 = tc::sdesc_sw128(tc::smem_u32(A_s), 1024, 2048);   // A: MN-major, 64-channel atoms 1 KB apart
+      const uint32_t idesc = tc::idesc_f16(128, a.H, false, false, false);
       const uint64_t b0 = tc::sdesc_sw128(tc::smem_u32(P_s), 0, 1024);      // B: K-major, 64-token atoms of H rows
-      const uint32_t a_lo0 = tc::desc_lo(a0), a_hi = tc::desc_hi(a0);
       const uint32_t b_lo0 = tc::desc_lo(b0), b_hi = tc::desc_hi(b0);
       const uint32_t b_atom = (uint32_t)(a.H * 128) >> 4, p_step = (uint32_t)p_stage >> 4;
-      int n = 0, cur_run = -1;
+      int cur_run = -1, as = 0;
+      uint32_t aph = 0;
       bool first = false;
       for (int T = 0; T < n_tiles && !abort_flag; ++T) {
         const int run = tile_s[T].w;
@@ -291,22 +272,22 @@ __global__ void __launch_bounds__(kValThreads, 1) k_values_tc(ValArgs a) {
         tc::tc_fence_after();
         const uint32_t b_lo = b_lo0 + (uint32_t)ps * p_step;
         bool ok = true;
-        for (int x0 = 0; x0 < (1 << lg_ipt) && ok; x0 += 8, n += 8) {
-          const int c = n >> 3;
-          ok = tc::mbar_wait_ab(&ch_full[c & 3], ((uint32_t)(c >> 2)) & 1u, a.status, &abort_flag);
-          if (!ok) break;
-          tc::tc_fence_after();
-          // the chain's stages are (n .. n + 7) % kAStages: n is a multiple of 8, no wrap
-          const uint32_t a_lo = a_lo0 + (uint32_t)(n % kAStages) * (kAStage >> 4);
-#pragma unroll
-          for (int i = 0; i < 8; ++i) {
-            const int x = x0 + i, k = x >> lnb, cb = x & (nblk - 1);
-            // tokens 16 k .. 16 k + 15: K = 16 step k of the P tile
-            tc::mma_f16_ss2(tmem + (uint32_t)(cb * a.H), a_lo + (uint32_t)i * (kAStage >> 4), a_hi,
-                            b_lo + (uint32_t)(k >> 2) * b_atom + (uint32_t)(k & 3) * 2u, b_hi, idesc,
-                            (first && k == 0) ? 0u : 1u);
+        for (int k = 0; k < 8; ++k) {
+          if (!tc::mbar_wait_ab(&a_full[as], aph, a.status, &abort_flag)) {
+            ok = false;
+            break;
           }
-          tc::mma_commit(&ch_done[c & 3]);
+          tc::tc_fence_after();
+          const uint32_t acol = tmem + ycols + (uint32_t)(as * nblk) * 8u;
+          const uint32_t bk = b_lo + (uint32_t)(k >> 2) * b_atom + (uint32_t)(k & 3) * 2u;
+          for (int cb = 0; cb < nblk; ++cb)
+            tc::mma_f16_ts(tmem + (uint32_t)(cb * a.H), acol + (uint32_t)cb * 8u, bk, b_hi, idesc,
+                           (first && k == 0) ? 0u : 1u);
+          tc::mma_commit(&a_free[as]);
+          if (++as == a.na) {
+            as = 0;
+            aph ^= 1u;
+          }
         }
         if (!ok) break;
         tc::mma_commit(&p_empty[ps]);
@@ -320,7 +301,8 @@ __global__ void __launch_bounds__(kValThreads, 1) k_values_tc(ValArgs a) {
     // ------------------------------------------------ P staging
     // Stager warp s stages the 32-token group s of every tile, lane h for
     // head h (and h + 32): P * exp2(m_g - M) rounded to fp16, with M the
-    // maximum over the run; l = sum of the staged values.
+    // maximum over the run; l = sum of the staged values, added in a fixed
+    // order over the four stagers.
     const int sw = warp - 1;
     if (sw == 0)
       for (int sl = 0; sl < a.slots; ++sl)
@@ -331,10 +313,9 @@ __global__ void __launch_bounds__(kValThreads, 1) k_values_tc(ValArgs a) {
     float Mh[2] = {-FLT_MAX, -FLT_MAX}, lh[2] = {0.f, 0.f};
     int cur_run = -1, cur_b = -1;
     auto flush = [&]() {
-      // the four stager warps add their partial sums, then warp 0 writes the run's (M, l)
 #pragma unroll
       for (int hh = 0; hh < 2; ++hh)
-        if (lane + 32 * hh < a.H) atomicAdd(&l_stage[lane + 32 * hh], lh[hh]);
+        if (lane + 32 * hh < a.H) l_part[sw][lane + 32 * hh] = lh[hh];
       asm volatile("bar.sync 1, %0;" ::"n"(32 * kStagers) : "memory");
       if (sw == 0) {
         const size_t base = ((size_t)cta * a.slots + (cur_b - b_first)) * a.H;
@@ -343,8 +324,7 @@ __global__ void __launch_bounds__(kValThreads, 1) k_values_tc(ValArgs a) {
           const int h = lane + 32 * hh;
           if (h < a.H) {
             a.mseg[base + h] = Mh[hh];
-            a.lseg[base + h] = l_stage[h];
-            l_stage[h] = 0.f;
+            a.lseg[base + h] = ((l_part[0][h] + l_part[1][h]) + l_part[2][h]) + l_part[3][h];
           }
         }
       }
@@ -423,7 +403,6 @@ __global__ void __launch_bounds__(kValThreads, 1) k_values_tc(ValArgs a) {
     }
     if (cur_run >= 0) flush();
   } else if (warp == kStagers + 1) {
-
     // ------------------------------------------------ page copies
     // Page p = 8 T + k (tokens 16 k .. 16 k + 15 of tile T): its value block
     // into raw stage p % n_raw.
@@ -445,31 +424,31 @@ __global__ void __launch_bounds__(kValThreads, 1) k_values_tc(ValArgs a) {
     }
     __syncwarp();
   } else {
-    // ------------------------------------------------ workers: codes -> A stages, run epilogues
-    // Worker w takes the CTA's items w, w + 16, w + 32, ...; item n is item
-    // x = n % ipt = nblk k + cb of tile T = n / ipt: value channels
-    // [128 cb, 128 cb + 128) of page k (tokens 16 k .. 16 k + 15), read from
-    // raw stage (8 T + k) % n_raw and dequantized into A stage n % kAStages;
-    // lane l takes token l % 16 and the 64 channels of half l / 16.
-    const int w = warp - 2 - kStagers;
-    const int q = warp & 3, part = w >> 2;   // epilogue: TMEM lane quarter, column part
-    const int n_items = n_tiles << lg_ipt;
+    // ------------------------------------------------ workers: codes -> A tiles in TMEM, run epilogues
+    // A warp may address only its TMEM lane quarter q = warp % 4, i.e. the
+    // channels 32 q .. 32 q + 31 of every 128-channel block: channel group
+    // 4 cb + q of block cb.  The four workers of a quarter (j = 0..3) take
+    // the blocks cb = j, j + 4, ...; lane = channel inside the group.
+    const int wid = warp - 2 - kStagers;
+    const int q = warp & 3, j = wid >> 2;
+    const uint32_t lane_base = (uint32_t)(q * 32) << 16;
+    const int n_pg = n_tiles * 8;
     int epi_run = 0;
     auto epilogue = [&](int r) {
       // Y^T of run r from TMEM (lanes = value channels), 16 columns at a time
       const bool ok = tc::mbar_wait_ab(&seg_done, (uint32_t)r & 1u, a.status, &abort_flag);
       tc::tc_fence_after();
       const size_t base = ((size_t)cta * a.slots + (run_b[r] - b_first)) * a.H;
-      for (int col = part * 16; col < nblk * a.H; col += 64) {
+      for (int col = j * 16; col < (int)ycols; col += 64) {
         float v[16];
         if (ok) {
-          tc::tmem_ld16_sync(tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)col, v);
+          tc::tmem_ld16_sync(tmem + lane_base + (uint32_t)col, v);
         } else {
 #pragma unroll
           for (int i = 0; i < 16; ++i) v[i] = 0.f;
         }
         const int cb = col / a.H, h0 = col % a.H;
-        const int ch = cb * 128 + q * 32 + lane;     // A-tile position (channel order permuted per 8)
+        const int ch = cb * 128 + q * 32 + lane;
 #pragma unroll
         for (int i = 0; i < 16; ++i) a.Y[(base + h0 + i) * a.rv + ch] = v[i];
       }
@@ -477,61 +456,57 @@ __global__ void __launch_bounds__(kValThreads, 1) k_values_tc(ValArgs a) {
       __syncwarp();
       if (lane == 0) tc::mbar_arrive(&acc_free);
     };
-    const int slot = lane & 15, half = lane >> 4;
-    const uint32_t x7 = (uint32_t)(slot & 7);
-    const size_t st_off = (size_t)(slot >> 3) * 2048 + (size_t)half * 1024 + (size_t)(slot & 7) * 128;
-    for (int n = w; n < n_items; n += kValWorkers) {
-      const int T = n >> lg_ipt;
+    int as = 0;
+    uint32_t aph = 0;
+    for (int p = 0; p < n_pg; ++p) {
+      const int T = p >> 3, k = p & 7;
       const int run = tile_s[T].w;
       while (epi_run < run && epi_run < n_runs) epilogue(epi_run++);
-      const int x = n & ((1 << lg_ipt) - 1);
-      const int k = x >> lnb, cb = x & (nblk - 1);
-      const int pg = T * 8 + k;                // page of the CTA's tiles
-      const uint32_t rsp = rsp_s[pg];
-      const int rs = (int)(rsp & 127u), as = n % kAStages;
+      const int cur_as = as;
+      const uint32_t cur_aph = aph;
+      if (++as == a.na) {
+        as = 0;
+        aph ^= 1u;
+      }
+      if (j >= nblk) continue;   // no channel block for this worker (fewer than four blocks)
+      const uint32_t rsp = rsp_s[p];
+      const int rs = (int)(rsp & 127u);
       const bool valid = pid_s[T][k] >= 0;
-      // A stage first: the stage's previous item was in chain ch - 4; once that
-      // chain is consumed every page up to it has landed, and with at least
-      // 32 / nblk raw stages the raw stage is then at most one phase from pg
-      const int ch = n >> 3;                   // chain of this item
-      const bool ok = tc::mbar_wait_ab(&ch_done[ch & 3], (((uint32_t)(ch >> 2)) & 1u) ^ 1u, a.status, &abort_flag) &&
+      const bool ok = tc::mbar_wait_ab(&a_free[cur_as], cur_aph ^ 1u, a.status, &abort_flag) &&
                       tc::mbar_wait_ab(&r_full[rs], rsp >> 7, a.status, &abort_flag);
       if (ok) {
         const uint8_t* blk = R_s + (size_t)rs * a.raw_stage;
-        uint8_t* st = A_s + (size_t)as * kAStage + st_off;
-#pragma unroll
-        for (int gg = 0; gg < 2; ++gg) {
-          const int g = cb * 4 + half * 2 + gg;
+        for (int cb = j; cb < nblk; cb += 4) {
+          const int g = cb * 4 + q;
           const int4 vg = vg_s[g];
-          const __half hs = valid ? reinterpret_cast<const __half*>(blk)[g * kPage + slot] : __ushort_as_half(0);
-          const __half2 s2 = __halves2half2(hs, hs);
           const __half2 sub = *reinterpret_cast<const __half2*>(&vg.z);
-          const uint32_t* cw = reinterpret_cast<const uint32_t*>(blk + vg.y) + slot * vg.x;
-          uint4 o0, o1, o2, o3;
-          if (vg.x == 4) {
-            const uint4 v4 = *reinterpret_cast<const uint4*>(cw);
-            o0 = deq8_b4(v4.x, sub, s2);
-            o1 = deq8_b4(v4.y, sub, s2);
-            o2 = deq8_b4(v4.z, sub, s2);
-            o3 = deq8_b4(v4.w, sub, s2);
+          uint32_t sc[8], out[8];
+          if (valid) {
+            const uint4 s0 = *reinterpret_cast<const uint4*>(blk + g * 32);
+            const uint4 s1 = *reinterpret_cast<const uint4*>(blk + g * 32 + 16);
+            sc[0] = s0.x; sc[1] = s0.y; sc[2] = s0.z; sc[3] = s0.w;
+            sc[4] = s1.x; sc[5] = s1.y; sc[6] = s1.z; sc[7] = s1.w;
           } else {
-            const uint32_t w0 = cw[0], w1 = cw[1], w2 = cw[2];
-            o0 = deq8_b3(w0, sub, s2);
-            o1 = deq8_b3(__funnelshift_r(w0, w1, 24), sub, s2);
-            o2 = deq8_b3(__funnelshift_r(w1, w2, 16), sub, s2);
-            o3 = deq8_b3(w2 >> 8, sub, s2);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) sc[i] = 0u;
           }
-          const uint32_t c4 = (uint32_t)gg * 4u;   // 8-channel chunk of this group in the half's atom
-          *reinterpret_cast<uint4*>(st + (((c4 + 0u) ^ x7) << 4)) = o0;
-          *reinterpret_cast<uint4*>(st + (((c4 + 1u) ^ x7) << 4)) = o1;
-          *reinterpret_cast<uint4*>(st + (((c4 + 2u) ^ x7) << 4)) = o2;
-          *reinterpret_cast<uint4*>(st + (((c4 + 3u) ^ x7) << 4)) = o3;
+          if (vg.x == 4) {
+            const uint2 cw = *reinterpret_cast<const uint2*>(blk + vg.y + lane * 8);
+            deq_channel4(cw.x, cw.y, sub, sc, out);
+          } else {
+            const int bit = 48 * lane;
+            const uint32_t* cw = reinterpret_cast<const uint32_t*>(blk + vg.y) + (bit >> 5);
+            const uint64_t x = ((uint64_t)cw[1] << 32 | cw[0]) >> (bit & 31);
+            deq_channel3(x, sub, sc, out);
+          }
+          tc::tmem_st8(tmem + lane_base + ycols + (uint32_t)(cur_as * nblk + cb) * 8u, out);
         }
       }
-      tc::fence_proxy_async();
+      tc::tmem_st_wait();
+      tc::tc_fence_before();
       __syncwarp();
       if (lane == 0) {
-        tc::mbar_arrive(&ch_full[ch & 3]);
+        tc::mbar_arrive(&a_full[cur_as]);
         tc::mbar_arrive(&r_empty[rs]);
       }
     }
@@ -540,7 +515,7 @@ __global__ void __launch_bounds__(kValThreads, 1) k_values_tc(ValArgs a) {
   tc::tc_fence_before();
   __syncthreads();
   tc::tc_fence_after();
-  if (warp == 0) tc::tmem_dealloc(tmem, a.tmem_cols);
+  if (warp == 0) tc::tmem_dealloc(tmem, 512);
 }
 
 // Merge the runs of each sequence: y = sum exp2(M_r - M) Y_r / sum exp2(M_r - M) l_r,
@@ -610,9 +585,7 @@ __global__ void k_values_combine(const float* __restrict__ Y, const float* __res
   __syncthreads();
   const float idn = inv_den;
   const int nt = b / NB, r = b % NB;
-  // four channels per thread, one 16-byte load per run.  Inside every chunk
-  // of 8 the value kernel's A tiles hold channels 0 2 1 3 4 6 5 7, so the
-  // loaded positions (0, 1, 2, 3) are channels (0, 2, 1, 3) of the four.
+  // four channels per thread, one 16-byte load per run
   for (int j = 4 * (int)threadIdx.x; j < rv; j += 4 * (int)blockDim.x) {
     float4 a0 = make_float4(0.f, 0.f, 0.f, 0.f), a1 = a0;
     int k = 0;
@@ -637,8 +610,8 @@ __global__ void k_values_combine(const float* __restrict__ Y, const float* __res
       a0.z += w0 * y0.z;
       a0.w += w0 * y0.w;
     }
-    const __half2 lo2 = __floats2half2_rn((a0.x + a1.x) * idn, (a0.z + a1.z) * idn);   // channels j, j + 1
-    const __half2 hi2 = __floats2half2_rn((a0.y + a1.y) * idn, (a0.w + a1.w) * idn);   // channels j + 2, j + 3
+    const __half2 lo2 = __floats2half2_rn((a0.x + a1.x) * idn, (a0.y + a1.y) * idn);   // channels j, j + 1
+    const __half2 hi2 = __floats2half2_rn((a0.z + a1.z) * idn, (a0.w + a1.w) * idn);   // channels j + 2, j + 3
     const uint32_t kk = (uint32_t)(h * rv + j), cidx = kk & 63u;
     uint8_t* tile = ytiles + ((size_t)nt * KT + (kk >> 6)) * (size_t)NB * 128;
     const uint32_t off = tc::sw128((uint32_t)r, cidx >> 3) + (cidx & 7u) * 2u;
@@ -649,10 +622,10 @@ __global__ void k_values_combine(const float* __restrict__ Y, const float* __res
 
 }  // namespace
 
-// Dynamic shared memory of the value kernel: the A stages and two P stages.
+// Dynamic shared memory of the value kernel: two P stages and the raw page stages.
 static size_t values_raw_stage(int vblk_bytes) { return (size_t)(vblk_bytes + 127) / 128 * 128; }
 static size_t values_smem(int H, int vblk_bytes, int n_raw) {
-  return (size_t)kAStages * kAStage + 2 * (size_t)H * 256 + n_raw * values_raw_stage(vblk_bytes) + 1024;
+  return 2 * (size_t)H * 256 + n_raw * values_raw_stage(vblk_bytes) + 1024;
 }
 
 // Grid of the value kernel: one CTA per SM, more when a CTA would hold more
@@ -675,11 +648,15 @@ bool plan_values_tc(starkv_layer* L) {
   const LayerView& v = L->view;
   const starkv_layer_config& c = L->cfg;
   if (!L->tc_scores) return false;
-  // power-of-two count of 128-channel value blocks, heads a multiple of 16
+  // power-of-two count of 128-channel value blocks, heads a multiple of 16;
+  // TMEM holds Y^T (nblk * H columns) and at least two pages of A tiles
+  // (nblk * 8 columns each) in its 512 columns
   if (v.rv % 128 != 0 || ((v.rv / 128) & (v.rv / 128 - 1)) != 0 || v.H % 16 != 0 || v.H > 64) return false;
-  if ((long long)(v.rv / 128) * v.H > 512) return false;
+  const int nblk = v.rv / 128;
+  if (nblk * v.H + 2 * nblk * 8 > 512) return false;
+  L->val_na = std::min(kMaxASlots, (512 - nblk * v.H) / (nblk * 8));
   const LatentDesc& ld = L->lat[v.L - 1];
-  if (ld.n_groups * 32 != v.rv) return false;
+  if (ld.n_groups * 32 != v.rv || !ld.cmajor) return false;
   for (int g = 0; g < ld.n_groups; ++g) {
     const GroupDesc& gd = L->grp[ld.group0 + g];
     if (gd.n != 32 || (gd.bits != 3 && gd.bits != 4) || gd.start != g * 32) return false;
@@ -690,11 +667,10 @@ bool plan_values_tc(starkv_layer* L) {
   size_t bytes = ld.scale_bytes;
   for (int g = 0; g < ld.n_groups; ++g) bytes += (size_t)kPage * 32 * L->grp[ld.group0 + g].bits / 8;
   L->vblk_bytes = (int)bytes;
-  // as many raw stages as fit next to the static tables and barriers, and at
-  // least 16 / nblk of them
+  // as many raw stages as fit next to the static tables and barriers
   cudaFuncAttributes fa;
   if (cudaFuncGetAttributes(&fa, k_values_tc) != cudaSuccess) return false;
-  const int min_raw = std::max(4, 32 / (v.rv / 128));
+  const int min_raw = 4;
   L->val_raw = 0;
   for (int n_raw = kMaxRawStages; n_raw >= min_raw && !L->val_raw; --n_raw)
     if (values_smem(v.H, L->vblk_bytes, n_raw) + fa.sharedSizeBytes <= 232448) L->val_raw = n_raw;
@@ -733,6 +709,7 @@ cudaError_t launch_values_tc(const starkv_layer* L, const uint8_t* pool, long lo
   a.vblk_bytes = L->vblk_bytes;
   a.raw_stage = (int)values_raw_stage(L->vblk_bytes);
   a.n_raw = L->val_raw;
+  a.na = L->val_na;
   a.vgrp = L->d_grp + L->lat[v.L - 1].group0;
   a.rv = v.rv;
   a.H = v.H;
@@ -750,19 +727,12 @@ cudaError_t launch_values_tc(const starkv_layer* L, const uint8_t* pool, long lo
   a.mseg = (float*)w;
   w += r(sizeof(float) * (size_t)G * slots * v.H);
   a.lseg = (float*)w;
-  uint32_t cols = 32;
-  while (cols < (uint32_t)((v.rv / 128) * v.H)) cols <<= 1;
-  a.tmem_cols = cols;
   a.status = L->status;
   const size_t smem = values_smem(v.H, L->vblk_bytes, L->val_raw);
-  static size_t attr = 0;
-  if (smem > attr) {
-    cudaError_t e = cudaFuncSetAttribute(k_values_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
-    attr = smem;
-  }
+  cudaError_t e = set_smem_limit((const void*)k_values_tc, smem);
+  if (e != cudaSuccess) return e;
   k_values_tc<<<G, kValThreads, smem, s>>>(a);
-  cudaError_t e = cudaGetLastError();
+  e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   if (ev_mid && (e = cudaEventRecord(ev_mid, s)) != cudaSuccess) return e;
   const int NB = outproj_nb(batch);

@@ -30,9 +30,21 @@ struct LatentDesc {
   int group0;       // index of the first group in the group table
   int ch_off;       // offset of this latent in the concatenated latent vector
   int scale_bytes;  // bytes of the scale block (0 when unquantized)
+  int cmajor;       // 1: code blocks channel-major (the quantized value latent), see code_bit
 };
 
 constexpr int kPage = 16;
+
+// First bit of the code of (slot, channel i) inside a group's code block of n
+// channels at `bits` bits.  Key latents are slot-major: a token's codes of
+// the group are one run.  The value latent is channel-major: the 16 codes of
+// a channel are one field of 16 * bits bits, even slots first, odd slots
+// after them (place (s % 2) * 8 + s / 2), so that one shift and mask of the
+// field puts the codes of slots 2k and 2k + 1 side by side.
+__host__ __device__ __forceinline__ uint32_t code_bit(int slot, int i, int n, int bits, int cmajor) {
+  return cmajor ? (uint32_t)(i * kPage + (slot & 1) * (kPage / 2) + (slot >> 1)) * (uint32_t)bits
+                : (uint32_t)(slot * n + i) * (uint32_t)bits;
+}
 
 // Device status bits (mirror of STARKV_DEV_* in the public header).
 constexpr uint32_t kBadPage = STARKV_DEV_BAD_PAGE;
@@ -133,7 +145,8 @@ struct starkv_layer {
   // tensor-core value kernel
   bool tc_values = false;
   int vblk_off = 0, vblk_bytes = 0;
-  int val_raw = 0;              // raw chunk stages of the value kernel
+  int val_raw = 0;              // raw page stages of the value kernel
+  int val_na = 0;               // pages of A tiles the value kernel keeps in TMEM
   // optional per-kernel timing of the tensor-core decode: prof_n sets of
   // STARKV_N_PHASES + 1 events, the decode call number prof_calls picks the set
   std::vector<cudaEvent_t> prof_ev;
@@ -171,6 +184,11 @@ cudaError_t launch_decode_generic(const starkv_layer* L, const uint8_t* pool, lo
 size_t decode_generic_ws_bytes(const starkv_layer* L, int rows, int max_len, bool prefill);
 
 int num_sms();
+
+// Raise a kernel's dynamic shared-memory limit to `bytes` on the current
+// device.  The attribute is per (function, device); the last value set is
+// remembered per pair so that repeated launches skip the call.
+cudaError_t set_smem_limit(const void* kernel, size_t bytes);
 
 bool plan_scores_tc(starkv_layer* L);
 bool plan_values_tc(starkv_layer* L);

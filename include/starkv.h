@@ -23,9 +23,10 @@
  *     starkv_load_factors, which allocates the layer's own folded factors.
  *   - Errors found on the host return at once, before any launch, with a
  *     message available from starkv_last_error().  Errors found by a kernel
- *     (a page id outside the pool, a position that is not the sequence's next
- *     slot, an fp16 scale overflow) set the layer's device status word; no
- *     kernel traps.  starkv_sync_status() reads and clears it.
+ *     (a page id outside the pool, a position outside the page table, a
+ *     sequence length above the page table's capacity, an fp16 scale
+ *     overflow, a bounded wait that expired) set the layer's device status
+ *     word; no kernel traps.  starkv_sync_status() reads and clears it.
  *   - Not thread-safe per layer: calls on one layer from several host threads
  *     must be serialised by the caller.
  */
@@ -175,7 +176,12 @@ STARKV_API starkv_status starkv_cache_init(const starkv_layer* layer, void* pool
  *   workspace: at least starkv_append_workspace_bytes(layer, n_tokens) bytes
  *     (may be NULL when that is 0).
  * Tokens of one call must go to distinct (sequence, position) slots whose
- * bytes are still zero.  Packed bytes are bit-exact for given float32 latents.
+ * bytes are still zero.  This is the caller's obligation: the kernel checks
+ * only that a position lies inside the page table (else
+ * STARKV_DEV_BAD_POSITION) and that its page id lies inside the pool (else
+ * STARKV_DEV_BAD_PAGE).  Codes are ORed into the slot, so writing a slot that
+ * already holds a token corrupts it.  Packed bytes are bit-exact for given
+ * float32 latents.  max_pages * 16 must fit in an int (else STARKV_ERR_ARG).
  */
 STARKV_API starkv_status starkv_append(const starkv_layer* layer, void* pool, int64_t n_pages, const int32_t* page_table,
                             int n_seqs, int max_pages, int n_tokens, const int32_t* seq_idx, const int32_t* positions,
@@ -188,7 +194,8 @@ STARKV_API size_t starkv_append_workspace_bytes(const starkv_layer* layer, int n
  * Decode attention for one new query per sequence (Algorithm 2 steps 4-8).
  *   seq_lens: int32 [batch]; sequence b attends to slots [0, seq_lens[b]).
  *     A length of 0 gives a zero output row; a length above max_pages * 16
- *     sets STARKV_DEV_BAD_POSITION and is clamped.
+ *     sets STARKV_DEV_BAD_POSITION and is clamped.  max_pages * 16 must fit
+ *     in an int (else STARKV_ERR_ARG).
  *   q_pos: int32 [batch] RoPE position of each query, or NULL for seq_lens[b]-1.
  *   q: [batch][H][d] in dtype (before RoPE).   out: [batch][D] in dtype.
  *   workspace: at least starkv_workspace_bytes(layer, batch, max_pages * 16, 1)
@@ -249,11 +256,16 @@ STARKV_API starkv_status starkv_sync_status(const starkv_layer* layer, starkv_st
  * library, kept until the process exits.  The call returns
  * STARKV_ERR_WORKSPACE, before any launch and with a message naming both
  * sizes, when starkv_workspace_bytes(layer, batch, max_pages * 16, 1) exceeds
- * that size.  It allocates nothing: no cudaMalloc, no cudaFree, no
+ * that size.  That figure is the largest workspace over every decode path the
+ * layer can take, so a decode that the selected path could fit in the array
+ * may still be refused.  It allocates nothing: no cudaMalloc, no cudaFree, no
  * allocating library routine.
  *
  * The first call on each device looks up the array's device address (with
- * that device current); make that first call before any stream capture.
+ * that device current); make that first call before any stream capture.  The
+ * address is kept for the life of the process: after cudaDeviceReset (or any
+ * other teardown of the device's primary context) the cached address is
+ * stale, so do not call this entry point again in that process.
  * Every call on a device shares the one array and leaves its contents behind;
  * each call writes every scratch element before reading it, so nothing needs
  * to start at zero.  Calls whose work overlaps on the GPU (several streams,

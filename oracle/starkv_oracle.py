@@ -206,10 +206,14 @@ def dequantize_group(u: np.ndarray, s16: np.float16, bits: int) -> np.ndarray:
 #   latents in order: key latent of KV head 0 .. H_kv-1, then the joint value latent
 #   unquantized block: element (slot, j) at byte (slot * r + j) * elem_size; pad to 16 B
 #   quantized block:   scales [group][slot] fp16, pad to 16 B; then for each group g
-#                      a code block of P * n_g * b_g bits, pad to 16 B.  The code of
-#                      (slot, channel i of g) occupies stream bits
-#                      [(slot * n_g + i) * b_g, ... + b_g), least significant bit first;
-#                      stream bit k is bit (k mod 8) of byte k div 8.
+#                      a code block of P * n_g * b_g bits, pad to 16 B, a bitstream
+#                      written least significant bit first (stream bit k is bit
+#                      (k mod 8) of byte k div 8).  The code of (slot, channel i of g)
+#                      occupies stream bits [k, k + b_g) with
+#                        key latents (slot-major):     k = (slot * n_g + i) * b_g
+#                        value latent (channel-major): k = (i * P + sigma(slot)) * b_g,
+#                      sigma(s) = (P/2) (s mod 2) + s div 2: each channel's P codes form
+#                      one field, even slots first, then odd slots.
 # ---------------------------------------------------------------------------
 
 def _ru(x: int, m: int) -> int:
@@ -256,11 +260,24 @@ def read_bits(buf: np.ndarray, bit_offset: int, nbits: int) -> int:
     return v
 
 
-def pack_block(Z: np.ndarray, r: int, spec) -> np.ndarray:
+def slot_place(slot: int, P: int) -> int:
+    """Place of a slot inside a channel field of the value latent: even slots first."""
+    return (P // 2) * (slot % 2) + slot // 2
+
+
+def code_bit(slot: int, i: int, n: int, bits: int, P: int, channel_major: bool) -> int:
+    """First stream bit of the code of (slot, channel i) in a group of n channels."""
+    if channel_major:
+        return (i * P + slot_place(slot, P)) * bits
+    return (slot * n + i) * bits
+
+
+def pack_block(Z: np.ndarray, r: int, spec, channel_major: bool = False) -> np.ndarray:
     """Bytes of one latent block holding the float32 latents Z [P, r] (rows = slots).
 
     Rows of Z that are NaN-free are written; a slot that holds no token should
     be passed as None rows (see `pack_page`), which leaves its bytes zero.
+    channel_major selects the value latent's code order (see the page format above).
     """
     P = spec.page_size
     out = np.zeros(block_bytes(r, spec), dtype=np.uint8)
@@ -291,7 +308,7 @@ def pack_block(Z: np.ndarray, r: int, spec) -> np.ndarray:
             so = (gi * P + slot) * 2
             out[so:so + 2] = sb
             for i in range(g.n):
-                write_bits(cb, (slot * g.n + i) * g.bits, int(u[i]), g.bits)
+                write_bits(cb, code_bit(slot, i, g.n, g.bits, P, channel_major), int(u[i]), g.bits)
         code_off += _ru(P * g.n * g.bits // 8, 16)
     return out
 
@@ -310,7 +327,7 @@ def pack_page(latents_per_slot, spec) -> np.ndarray:
         for slot in range(P):
             if latents_per_slot[slot] is not None:
                 Z[slot] = latents_per_slot[slot][li]
-        blk = pack_block(Z, r, spec)
+        blk = pack_block(Z, r, spec, channel_major=(li == len(spec.latent_widths) - 1))
         page[offs[li]:offs[li] + blk.size] = blk
     return page
 

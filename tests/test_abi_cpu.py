@@ -70,3 +70,21 @@ def test_host_validation_before_cuda():
     with pytest.raises(lib.StarKVError) as e:
         lib.load_factors(cfg, None, None, None, None, None, stream=0)
     assert e.value.status == 1
+
+
+def test_page_table_capacity_overflow_rejected_on_the_host():
+    # max_pages * 16 must fit in an int: a larger page table is refused before the layer is read
+    # or any size is computed from it (dummy non-NULL pointers, never dereferenced).
+    from decode_attention_rank_b200 import starkv as lib
+    raw = lib.raw_lib()
+    dummy = ctypes.create_string_buffer(4096)
+    p = ctypes.cast(dummy, ctypes.c_void_p).value
+    big = (2 ** 31 - 1) // 16 + 1
+    assert raw.starkv_decode_attn(p, p, 1, p, big, 1, p, None, p, p, p, 1 << 20, None) == 1
+    assert "overflows" in raw.starkv_last_error().decode()
+    assert raw.starkv_decode_attn_noalloc(p, p, 1, p, big, 1, p, None, p, p, None) == 1
+    assert "overflows" in raw.starkv_last_error().decode()
+    assert raw.starkv_prefill_attn(p, p, 1, p, big, 1, p, p, p, p, p, 1 << 20, None) == 1
+    assert "overflows" in raw.starkv_last_error().decode()
+    assert raw.starkv_append(p, p, 1, p, 1, big, 1, p, p, p, 1, p, 0, None) == 1
+    assert "overflows" in raw.starkv_last_error().decode()

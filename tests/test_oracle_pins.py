@@ -140,6 +140,44 @@ def test_pack_block_golden_bytes():
     np.testing.assert_array_equal(blk, want)
 
 
+def test_pack_value_block_golden_bytes():
+    # The joint value latent's code blocks are channel-major with the even slots of a
+    # channel's field first (page format reading: the pages fix no byte layout).
+    meta, hexes = _read_golden("pack_value_r4_three_slots.txt")
+    r = int(meta["r"][0])
+    spec = gen.LayerSpec(hidden=1, n_heads=1, n_kv_heads=1, head_dim=8, key_ranks=[r], value_rank=r,
+                         quantized=True, top_fraction=float(meta["top_fraction"][0]))
+    Z = np.full((16, r), np.nan, dtype=np.float32)
+    for s in range(3):
+        Z[s] = [float(x) for x in meta[f"slot{s}"]]
+    blk = O.pack_block(Z, r, spec, channel_major=True)
+    want = np.zeros(int(meta["bytes"][0]), dtype=np.uint8)
+    for off, bs in hexes:
+        want[off:off + len(bs)] = bs
+    np.testing.assert_array_equal(blk, want)
+
+
+def test_pack_value_block_roundtrip():
+    # Every code of a channel-major block is found at (i P + sigma(slot)) b with sigma a
+    # permutation of the P places: the fields do not overlap and cover the stream.
+    spec = gen.config_spec(2)
+    places = sorted(O.slot_place(s, 16) for s in range(16))
+    assert places == list(range(16))
+    assert [O.slot_place(s, 16) for s in (0, 1, 2, 3, 14, 15)] == [0, 8, 1, 9, 7, 15]
+    r = 64
+    Z = (gen.normals(gen.stream_key(4, 90), 16 * r).reshape(16, r)).astype(np.float32)
+    blk = O.pack_block(Z, r, spec, channel_major=True)
+    gs = O.groups(r, spec)
+    code_off = ((len(gs) * 16 * 2) + 15) // 16 * 16
+    for g in gs:
+        for slot in range(16):
+            s16, u = O.quantize_group(Z[slot, g.start:g.start + g.n], g.bits)
+            for i in range(g.n):
+                k = (i * 16 + (8 * (slot % 2) + slot // 2)) * g.bits
+                assert O.read_bits(blk[code_off:], k, g.bits) == u[i]
+        code_off += (16 * g.n * g.bits // 8 + 15) // 16 * 16
+
+
 def test_pack_roundtrip_and_layout():
     spec = gen.config_spec(2)
     offs, pb = O.page_layout(spec)
@@ -194,7 +232,8 @@ def test_pool_page_table_permutation():
         Zs = [lat[0][li][t] if t < T else None for t in range(32, 48)]
         rows = [None if z is None else [z] for z in Zs]
         sub = gen.LayerSpec(**{**spec.__dict__, "key_ranks": [r], "n_kv_heads": 1})
-        ref = O.pack_block(np.stack([z if z is not None else np.full(r, np.nan, np.float32) for z in Zs]), r, spec)
+        ref = O.pack_block(np.stack([z if z is not None else np.full(r, np.nan, np.float32) for z in Zs]), r, spec,
+                           channel_major=(li == len(spec.latent_widths) - 1))
         np.testing.assert_array_equal(last[offs[li]:offs[li] + ref.size], ref)
 
 
@@ -596,3 +635,7 @@ def test_planted_mistakes_are_caught(monkeypatch):
     def rotation_whole_latent(r, spec):  # one rotation across the hi and lo segments
         return O.group_rotation(r) if spec.quantized and spec.hadamard_block else np.eye(r)
     _fails(test_rotation_block_assembly, monkeypatch, "rotation", rotation_whole_latent)
+
+    def place_natural(slot, P):          # channel-major fields without the even/odd interleave
+        return slot
+    _fails(test_pack_value_block_golden_bytes, monkeypatch, "slot_place", place_natural)

@@ -5,9 +5,12 @@ plugin inside a serving engine whose allocator already holds the GPU's memory),
 so the library offers a decode entry point whose scratch is a fixed device
 array inside the library.  This checks, through the C ABI, that two calls in a
 row give the same output as the regular entry point with a caller workspace,
-within the attention tolerance the other parity tests use, and that a size
-beyond the array is refused before any launch.  This file is collected last on
-purpose.
+and that a size beyond the array is refused before any launch.  Both entry
+points run the same kernels on the same inputs and every step of the decode
+is deterministic (no floating-point atomics; partial sums are added in a
+fixed order), so the outputs must agree bit for bit: a stale or unwritten
+scratch element would show up as a difference.  This file is collected last
+on purpose.
 """
 import numpy as np
 import pytest
@@ -15,7 +18,7 @@ import torch
 
 from synth import gen
 
-from harness import Case, GpuCache, check_close, queries
+from harness import Case, GpuCache, queries
 
 pytestmark = pytest.mark.gpu
 
@@ -41,10 +44,9 @@ def test_noalloc_decode_matches_workspace_decode():
         L.decode_noalloc(cache.pool, cache.n_pages, cache.page_table, seq_lens, q, got)
         torch.cuda.synchronize()
         assert L.sync_status() == 0
-        g, r = got.double().cpu().numpy(), ref.double().cpu().numpy()
+        g = got.double().cpu().numpy()
         assert np.isfinite(g).all()
-        for b in range(B):
-            check_close(g[b], r[b], f"call {call} seq {b}")
+        assert torch.equal(got, ref), f"call {call}: {int((got != ref).sum())} elements differ"
 
 
 def test_noalloc_refuses_sizes_beyond_the_array():
