@@ -629,6 +629,14 @@ starkv_status starkv_decode_phase_ms(const starkv_layer* L, float* ms, int n_cal
   return STARKV_OK;
 }
 
+starkv_status starkv_check_wait_timeout(const starkv_layer* L, uint32_t limit_us, starkv_stream_t stream) {
+  set_error("");
+  CHECK_ARG(L != nullptr, "layer is NULL");
+  CHECK_ARG(limit_us >= 1 && limit_us <= 2000000, "limit_us must be in [1, 2000000]");
+  CUDA_TRY(launch_wait_timeout_check(L->status, 1000ull * limit_us, (cudaStream_t)stream));
+  return STARKV_OK;
+}
+
 starkv_status starkv_sync_status(const starkv_layer* L, starkv_stream_t stream, uint32_t* bits) {
   set_error("");
   CHECK_ARG(L != nullptr, "layer is NULL");

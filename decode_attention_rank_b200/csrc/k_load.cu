@@ -5,7 +5,7 @@
 //    up projection);
 //  - value-side output fusion M_h = B'_v,kv(h) W_o,h (section 5.3), stored as
 //    M_T [D][H * wv], the operand layout of the output kernel.
-#include "starkv_internal.cuh"
+#include "tc_common.cuh"
 
 namespace starkv {
 
@@ -163,6 +163,44 @@ cudaError_t launch_fold_M(const starkv_layer* L, const float* Bv_rot, const void
   else
     k_fold_M<__nv_bfloat16, __half><<<grid, 256, 0, s>>>(Bv_rot, bld, (const __nv_bfloat16*)W_o, v.D, v.d, v.wv,
                                                          v.group_q, v.H, 1, L->Kp / 64, (__half*)L->M_T);
+  return cudaGetLastError();
+}
+
+}  // namespace starkv
+
+namespace starkv {
+namespace {
+
+// One CTA of two roles that share the decode kernels' bounded wait: thread 0
+// of warp 1 waits on an mbarrier that nothing will complete (no copy is issued
+// and nobody arrives), so the wait gives up after limit_ns, sets the timeout
+// bit of the status word and raises the CTA's abort flag; warp 0 waits on a
+// second such barrier with the abort flag and drains as soon as it sees it,
+// the way the other roles of a decode kernel follow an aborting role.  No
+// copy, MMA or TMEM allocation is ever in flight.
+__global__ void k_wait_timeout_check(uint32_t* status, unsigned long long limit_ns) {
+  __shared__ __align__(8) uint64_t never, never2;
+  __shared__ volatile int abort_flag;
+  if (threadIdx.x == 0) {
+    tc::mbar_init(&never, 1);
+    tc::mbar_init(&never2, 1);
+    abort_flag = 0;
+    tc::fence_mbar_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 32) {
+    if (!tc::mbar_test_wait(&never, 0)) tc::mbar_wait_slow(&never, 0, status, &abort_flag, limit_ns);
+  } else if (threadIdx.x == 0) {
+    // bounded by its own limit too (four times the other's), in case the flag is never raised
+    if (!tc::mbar_test_wait(&never2, 0)) tc::mbar_wait_slow(&never2, 0, nullptr, &abort_flag, 4 * limit_ns);
+  }
+  __syncthreads();
+}
+
+}  // namespace
+
+cudaError_t launch_wait_timeout_check(uint32_t* status, unsigned long long limit_ns, cudaStream_t s) {
+  k_wait_timeout_check<<<1, 64, 0, s>>>(status, limit_ns);
   return cudaGetLastError();
 }
 

@@ -14,18 +14,24 @@
 // fp16 token pairs in registers and stores them straight into TMEM, where the
 // MMA reads A.
 //
+// An M = 128, N = 32 MMA does little work per instruction, and one thread
+// cannot issue tcgen05.mma much faster than one every ~50 cycles, so the MMAs
+// are issued by four threads on the four schedulers: the 16 dequantizing
+// warps form four teams (one warp per TMEM lane quarter each), team j owns
+// the channel blocks j, j + 4, ... with their own ring of A slots in TMEM, and
+// one warp of the team issues the team's MMAs once the four have stored a
+// page.  Teams meet only at the shared page copies and P tiles.
+//
 // P comes from the score kernel as exp2(s - m_g) per 32-token group; it is
 // rescaled by exp2(m_g - M) with M the maximum over the CTA's run of the
 // sequence, so no accumulator ever needs rescaling.  The CTA writes one
 // partial (M, l, Y) per run of one sequence; a combine kernel merges the runs.
-//   warp 0      tcgen05.mma issue, TMEM allocation
+//   warp 0      bulk copies of the pages' value blocks, TMEM allocation
 //   warps 1-4   P staging: rescaled fp16 P tiles (the B operand), M and l;
 //               warp s takes the 32-token group s of every 128-token tile
-//   warp 5      bulk copies of the pages' value blocks, a page at a time
-//   warps 6-21  workers: every page is split over the 16 workers by (TMEM
-//               lane quarter, 128-channel block); each dequantizes its
-//               channel groups of the page into the page's A slot in TMEM,
-//               and reads Y^T out of TMEM at the end of each run
+//   warps 5-20  four teams of four workers: dequantize the team's channel
+//               groups of each page into its A slot, issue its MMAs (one
+//               warp per team), read its blocks of Y^T at the end of a run
 #include <float.h>
 
 #include "tc_common.cuh"
@@ -34,11 +40,13 @@ namespace starkv {
 
 namespace {
 
-constexpr int kValWorkers = 16;                          // dequantizing warps (four per TMEM lane quarter)
+constexpr int kTeams = 4;                                // MMA-issuing teams, four warps each
+constexpr int kValWorkers = 4 * kTeams;                  // dequantizing warps
 constexpr int kStagers = 4;                              // P staging warps, one per 32-token group of a tile
-constexpr int kValThreads = 32 * (2 + kStagers + kValWorkers);   // MMA, P staging, page copies, workers
+constexpr int kWorker0 = 1 + kStagers;                   // first worker warp
+constexpr int kValThreads = 32 * (kWorker0 + kValWorkers);   // page copies, P staging, workers
 constexpr int kMaxRawStages = 32;
-constexpr int kMaxASlots = 8;    // pages whose A tiles are in TMEM at once
+constexpr int kMaxASlots = 8;    // pages whose A tiles a team keeps in TMEM at once
 constexpr int kVSuper = 256;     // tokens per super-tile (matches the score kernel)
 constexpr int kMaxRuns = 64;     // runs (sequences) per CTA
 constexpr int kRunMaxCache = 16; // runs whose per-head maxima are computed up front
@@ -61,7 +69,7 @@ struct ValArgs {
   int vblk_off, vblk_bytes;     // value latent block inside a page
   int raw_stage;                // bytes of one raw stage (a page's value block, 128-byte aligned)
   int n_raw;                    // raw stages
-  int na;                       // A slots in TMEM
+  int na;                       // A slots of each team in TMEM
   const GroupDesc* vgrp;        // value latent groups (all of 32 channels)
   int rv, H;
   int lg_nblk;                  // log2 of the 128-channel blocks of the value latent
@@ -116,12 +124,14 @@ __device__ __forceinline__ void deq_channel3(uint64_t x, __half2 sub, const uint
   }
 }
 
+// NBT: 128-channel blocks per team (the value latent has 128 * nblk channels,
+// team j owns blocks j + 4 i, i < NBT).
+template <int NBT>
 __global__ void __launch_bounds__(kValThreads, 1) k_values_tc(ValArgs a) {
   extern __shared__ uint8_t smem_raw[];
-  __shared__ __align__(8) uint64_t a_full[kMaxASlots], a_free[kMaxASlots], r_full[kMaxRawStages],
+  __shared__ __align__(8) uint64_t t_free[kTeams][kMaxASlots], t_seg[kTeams], r_full[kMaxRawStages],
       r_empty[kMaxRawStages];
   __shared__ __align__(8) uint64_t p_full[2], p_empty[2];
-  __shared__ __align__(8) uint64_t seg_done, acc_free, fin;
   __shared__ uint32_t tmem_base;
   __shared__ volatile int abort_flag;
   __shared__ int4 vg_s[128];              // per value group: code width, code block offset, fp16x2 of 1024 + 2^(bits-1)
@@ -139,28 +149,24 @@ __global__ void __launch_bounds__(kValThreads, 1) k_values_tc(ValArgs a) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int G = gridDim.x, cta = blockIdx.x;
   const long long u0 = vunit_lo(cta, G, a.U), u1 = vunit_lo(cta + 1, G, a.U);
-  const int lnb = a.lg_nblk;                             // 128-channel blocks: 1 << lnb
-  const int nblk = 1 << lnb;
-  const uint32_t ycols = (uint32_t)(nblk * a.H);         // TMEM columns of Y^T; the A slots follow
-  const int n_act = 4 * min(4, nblk);                    // workers with at least one channel block
+  const int nblk = 1 << a.lg_nblk;                       // 128-channel blocks
+  const int n_teams = min(kTeams, nblk);                 // teams with blocks
+  const uint32_t ycols = (uint32_t)(nblk * a.H);         // TMEM columns of Y^T; the teams' A rings follow
   const int b_first = (int)(u0 / a.n_st);
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < a.na; ++s) {
-      tc::mbar_init(&a_full[s], n_act);
-      tc::mbar_init(&a_free[s], 1);
+    for (int t = 0; t < kTeams; ++t) {
+      for (int s = 0; s < a.na; ++s) tc::mbar_init(&t_free[t][s], 1);
+      tc::mbar_init(&t_seg[t], 1);
     }
     for (int s = 0; s < a.n_raw; ++s) {
       tc::mbar_init(&r_full[s], 1);
-      tc::mbar_init(&r_empty[s], n_act);
+      tc::mbar_init(&r_empty[s], 4 * n_teams);
     }
     for (int s = 0; s < 2; ++s) {
       tc::mbar_init(&p_full[s], kStagers);
-      tc::mbar_init(&p_empty[s], 1);
+      tc::mbar_init(&p_empty[s], n_teams);
     }
-    tc::mbar_init(&seg_done, 1);
-    tc::mbar_init(&acc_free, kValWorkers);
-    tc::mbar_init(&fin, 1);
     abort_flag = 0;
     tc::fence_mbar_init();
   }
@@ -208,13 +214,13 @@ __global__ void __launch_bounds__(kValThreads, 1) k_values_tc(ValArgs a) {
       n_tiles_s = min(nt, kMaxTiles);
       n_runs_s = min(nr, kMaxRuns);
     }
+    tc::tmem_alloc(&tmem_base, 512);
   }
-  if (warp == 0) tc::tmem_alloc(&tmem_base, 512);
   tc::tc_fence_before();
   __syncthreads();
   tc::tc_fence_after();
   const uint32_t tmem = tmem_base;
-  const int n_tiles = n_tiles_s, n_runs = n_runs_s;
+  const int n_tiles = n_tiles_s;
   // page ids of every tile (out-of-range entries set the status bit and read page 0)
   for (int e = threadIdx.x; e < n_tiles * 8; e += blockDim.x) {
     const int4 tl = tile_s[e >> 3];
@@ -244,59 +250,28 @@ __global__ void __launch_bounds__(kValThreads, 1) k_values_tc(ValArgs a) {
   __syncthreads();
 
   if (warp == 0) {
-    // ------------------------------------------------ MMA issue
-    // Page p of the CTA (page k = p % 8 of tile p / 8) sits in A slot p % na:
-    // block cb's 128 x 16 A tile at TMEM column ycols + (slot * nblk + cb) * 8;
-    // its K = 16 MMA adds block cb's Y^T (columns cb * H ..).
+    // ------------------------------------------------ page copies
+    // Page p = 8 T + k (tokens 16 k .. 16 k + 15 of tile T): its value block
+    // into raw stage p % n_raw.
     if (lane == 0) {
-      const uint32_t idesc = tc::idesc_f16(128, a.H, false, false, false);
-      const uint64_t b0 = tc::sdesc_sw128(tc::smem_u32(P_s), 0, 1024);      // B: K-major, 64-token atoms of H rows
-      const uint32_t b_lo0 = tc::desc_lo(b0), b_hi = tc::desc_hi(b0);
-      const uint32_t b_atom = (uint32_t)(a.H * 128) >> 4, p_step = (uint32_t)p_stage >> 4;
-      int cur_run = -1, as = 0;
-      uint32_t aph = 0;
-      bool first = false;
-      for (int T = 0; T < n_tiles && !abort_flag; ++T) {
-        const int run = tile_s[T].w;
-        if (run != cur_run) {
-          if (cur_run >= 0) {
-            tc::mma_commit(&seg_done);
-            if (!tc::mbar_wait_ab(&acc_free, (uint32_t)cur_run & 1u, a.status, &abort_flag)) break;
-            tc::tc_fence_after();
-          }
-          cur_run = run;
-          first = true;
-        }
-        const int ps = T & 1;
-        if (!tc::mbar_wait_ab(&p_full[ps], ((uint32_t)(T >> 1)) & 1u, a.status, &abort_flag)) break;
-        tc::tc_fence_after();
-        const uint32_t b_lo = b_lo0 + (uint32_t)ps * p_step;
-        bool ok = true;
-        for (int k = 0; k < 8; ++k) {
-          if (!tc::mbar_wait_ab(&a_full[as], aph, a.status, &abort_flag)) {
-            ok = false;
-            break;
-          }
-          tc::tc_fence_after();
-          const uint32_t acol = tmem + ycols + (uint32_t)(as * nblk) * 8u;
-          const uint32_t bk = b_lo + (uint32_t)(k >> 2) * b_atom + (uint32_t)(k & 3) * 2u;
-          for (int cb = 0; cb < nblk; ++cb)
-            tc::mma_f16_ts(tmem + (uint32_t)(cb * a.H), acol + (uint32_t)cb * 8u, bk, b_hi, idesc,
-                           (first && k == 0) ? 0u : 1u);
-          tc::mma_commit(&a_free[as]);
-          if (++as == a.na) {
-            as = 0;
-            aph ^= 1u;
-          }
-        }
-        if (!ok) break;
-        tc::mma_commit(&p_empty[ps]);
-        first = false;
+      const int n_pg = n_tiles * 8;
+      int issued = 0;
+      for (int pg = 0; pg < n_pg; ++pg) {
+        const uint32_t rsp = rsp_s[pg];
+        const int rs = (int)(rsp & 127u);
+        if (!tc::mbar_wait_ab(&r_empty[rs], (rsp >> 7) ^ 1u, a.status, &abort_flag)) break;
+        const int page = pid_s[pg >> 3][pg & 7];
+        tc::mbar_expect_tx(&r_full[rs], page >= 0 ? (uint32_t)a.vblk_bytes : 0u);
+        if (page >= 0)
+          tc::bulk_g2s(R_s + (size_t)rs * a.raw_stage, a.pool + (size_t)page * a.page_bytes + a.vblk_off,
+                       (uint32_t)a.vblk_bytes, &r_full[rs]);
+        issued = pg + 1;
       }
-      if (cur_run >= 0) tc::mma_commit(&seg_done);
-      tc::mma_commit(&fin);
-      tc::mbar_wait(&fin, 0, a.status);
+      // let copies in flight land before the CTA can exit
+      for (int pg = max(0, issued - a.n_raw); pg < issued; ++pg)
+        tc::mbar_wait(&r_full[pg % a.n_raw], ((uint32_t)(pg / a.n_raw)) & 1u, a.status);
     }
+    __syncwarp();
   } else if (warp <= kStagers) {
     // ------------------------------------------------ P staging
     // Stager warp s stages the 32-token group s of every tile, lane h for
@@ -402,115 +377,140 @@ __global__ void __launch_bounds__(kValThreads, 1) k_values_tc(ValArgs a) {
       if (lane == 0) tc::mbar_arrive(&p_full[ps]);
     }
     if (cur_run >= 0) flush();
-  } else if (warp == kStagers + 1) {
-    // ------------------------------------------------ page copies
-    // Page p = 8 T + k (tokens 16 k .. 16 k + 15 of tile T): its value block
-    // into raw stage p % n_raw.
-    if (lane == 0) {
-      const int n_pg = n_tiles * 8;
-      for (int pg = 0; pg < n_pg; ++pg) {
-        const uint32_t rsp = rsp_s[pg];
-        const int rs = (int)(rsp & 127u);
-        if (!tc::mbar_wait_ab(&r_empty[rs], (rsp >> 7) ^ 1u, a.status, &abort_flag)) break;
-        const int page = pid_s[pg >> 3][pg & 7];
-        tc::mbar_expect_tx(&r_full[rs], page >= 0 ? (uint32_t)a.vblk_bytes : 0u);
-        if (page >= 0)
-          tc::bulk_g2s(R_s + (size_t)rs * a.raw_stage, a.pool + (size_t)page * a.page_bytes + a.vblk_off,
-                       (uint32_t)a.vblk_bytes, &r_full[rs]);
-      }
-      // let copies in flight land before the CTA can exit
-      for (int pg = max(0, n_pg - a.n_raw); pg < n_pg; ++pg)
-        tc::mbar_wait(&r_full[pg % a.n_raw], ((uint32_t)(pg / a.n_raw)) & 1u, a.status);
-    }
-    __syncwarp();
   } else {
-    // ------------------------------------------------ workers: codes -> A tiles in TMEM, run epilogues
+    // ------------------------------------------------ worker teams
     // A warp may address only its TMEM lane quarter q = warp % 4, i.e. the
     // channels 32 q .. 32 q + 31 of every 128-channel block: channel group
-    // 4 cb + q of block cb.  The four workers of a quarter (j = 0..3) take
-    // the blocks cb = j, j + 4, ...; lane = channel inside the group.
-    const int wid = warp - 2 - kStagers;
+    // 4 cb + q of block cb, lane = channel inside the group.  Team j = the
+    // four consecutive workers (one per quarter) owning blocks j + 4 i; its
+    // MMAs are issued by lane 0 of its warp with q == j, so that the four
+    // teams issue from the four schedulers.
+    const int wid = warp - kWorker0;
     const int q = warp & 3, j = wid >> 2;
-    const uint32_t lane_base = (uint32_t)(q * 32) << 16;
-    const int n_pg = n_tiles * 8;
-    int epi_run = 0;
-    auto epilogue = [&](int r) {
-      // Y^T of run r from TMEM (lanes = value channels), 16 columns at a time
-      const bool ok = tc::mbar_wait_ab(&seg_done, (uint32_t)r & 1u, a.status, &abort_flag);
-      tc::tc_fence_after();
-      const size_t base = ((size_t)cta * a.slots + (run_b[r] - b_first)) * a.H;
-      for (int col = j * 16; col < (int)ycols; col += 64) {
-        float v[16];
+    if (j >= n_teams) {
+      // a team without channel blocks (fewer than four blocks): nothing to do
+    } else {
+      const bool issuer = (q == j);
+      const uint32_t lane_base = (uint32_t)(q * 32) << 16;
+      const uint32_t abase = ycols + (uint32_t)(j * a.na * NBT * 8);   // this team's A ring
+      const int nbt = min(NBT, (nblk - j + 3) / 4);                    // blocks of this team
+      const int n_pg = n_tiles * 8;
+      const uint32_t bar_id = 2u + (uint32_t)j;
+      const uint32_t idesc = tc::idesc_f16(128, a.H, false, false, false);
+      const uint64_t b0 = tc::sdesc_sw128(tc::smem_u32(P_s), 0, 1024);   // B: K-major, 64-token atoms of H rows
+      const uint32_t b_lo0 = tc::desc_lo(b0), b_hi = tc::desc_hi(b0);
+      const uint32_t b_atom = (uint32_t)(a.H * 128) >> 4, p_step = (uint32_t)p_stage >> 4;
+      int cur_run = -1, n_epi = 0, as = 0;
+      uint32_t aph = 0;
+      bool first = false;
+      auto team_sync = [&]() { asm volatile("bar.sync %0, 128;" ::"r"(bar_id) : "memory"); };
+      auto epilogue = [&](int r) {
+        // Y^T of this team's blocks for run r (lanes = value channels), 16 columns at a time
+        if (issuer && lane == 0) tc::mma_commit(&t_seg[j]);
+        const bool ok = tc::mbar_wait_ab(&t_seg[j], (uint32_t)n_epi & 1u, a.status, &abort_flag);
+        ++n_epi;
+        tc::tc_fence_after();
+        const size_t base = ((size_t)cta * a.slots + (run_b[r] - b_first)) * a.H;
+#pragma unroll
+        for (int i = 0; i < NBT; ++i) {
+          if (i >= nbt) break;
+          const int cb = j + 4 * i;
+          const int ch = cb * 128 + q * 32 + lane;
+          for (int h0 = 0; h0 < a.H; h0 += 16) {
+            float v[16];
+            if (ok) {
+              tc::tmem_ld16_sync(tmem + lane_base + (uint32_t)(cb * a.H + h0), v);
+            } else {
+#pragma unroll
+              for (int x = 0; x < 16; ++x) v[x] = 0.f;
+            }
+#pragma unroll
+            for (int x = 0; x < 16; ++x) a.Y[(base + h0 + x) * a.rv + ch] = v[x];
+          }
+        }
+        tc::tc_fence_before();
+        team_sync();   // every quarter has read before the issuer overwrites D
+      };
+      for (int p = 0; p < n_pg; ++p) {
+        const int T = p >> 3, k = p & 7;
+        const int run = tile_s[T].w;
+        if (run != cur_run) {
+          if (cur_run >= 0) epilogue(cur_run);
+          cur_run = run;
+          first = true;
+        }
+        const int cur_as = as;
+        const uint32_t cur_aph = aph;
+        if (++as == a.na) {
+          as = 0;
+          aph ^= 1u;
+        }
+        const uint32_t rsp = rsp_s[p];
+        const int rs = (int)(rsp & 127u);
+        const bool valid = pid_s[T][k] >= 0;
+        const uint32_t slot_col = abase + (uint32_t)(cur_as * NBT * 8);
+        const bool ok = tc::mbar_wait_ab(&t_free[j][cur_as], cur_aph ^ 1u, a.status, &abort_flag) &&
+                        tc::mbar_wait_ab(&r_full[rs], rsp >> 7, a.status, &abort_flag);
         if (ok) {
-          tc::tmem_ld16_sync(tmem + lane_base + (uint32_t)col, v);
-        } else {
+          const uint8_t* blk = R_s + (size_t)rs * a.raw_stage;
 #pragma unroll
-          for (int i = 0; i < 16; ++i) v[i] = 0.f;
-        }
-        const int cb = col / a.H, h0 = col % a.H;
-        const int ch = cb * 128 + q * 32 + lane;
+          for (int i = 0; i < NBT; ++i) {
+            if (i >= nbt) break;
+            const int g = (j + 4 * i) * 4 + q;
+            const int4 vg = vg_s[g];
+            const __half2 sub = *reinterpret_cast<const __half2*>(&vg.z);
+            uint32_t sc[8], out[8];
+            if (valid) {
+              const uint4 s0 = *reinterpret_cast<const uint4*>(blk + g * 32);
+              const uint4 s1 = *reinterpret_cast<const uint4*>(blk + g * 32 + 16);
+              sc[0] = s0.x; sc[1] = s0.y; sc[2] = s0.z; sc[3] = s0.w;
+              sc[4] = s1.x; sc[5] = s1.y; sc[6] = s1.z; sc[7] = s1.w;
+            } else {
 #pragma unroll
-        for (int i = 0; i < 16; ++i) a.Y[(base + h0 + i) * a.rv + ch] = v[i];
-      }
-      tc::tc_fence_before();
-      __syncwarp();
-      if (lane == 0) tc::mbar_arrive(&acc_free);
-    };
-    int as = 0;
-    uint32_t aph = 0;
-    for (int p = 0; p < n_pg; ++p) {
-      const int T = p >> 3, k = p & 7;
-      const int run = tile_s[T].w;
-      while (epi_run < run && epi_run < n_runs) epilogue(epi_run++);
-      const int cur_as = as;
-      const uint32_t cur_aph = aph;
-      if (++as == a.na) {
-        as = 0;
-        aph ^= 1u;
-      }
-      if (j >= nblk) continue;   // no channel block for this worker (fewer than four blocks)
-      const uint32_t rsp = rsp_s[p];
-      const int rs = (int)(rsp & 127u);
-      const bool valid = pid_s[T][k] >= 0;
-      const bool ok = tc::mbar_wait_ab(&a_free[cur_as], cur_aph ^ 1u, a.status, &abort_flag) &&
-                      tc::mbar_wait_ab(&r_full[rs], rsp >> 7, a.status, &abort_flag);
-      if (ok) {
-        const uint8_t* blk = R_s + (size_t)rs * a.raw_stage;
-        for (int cb = j; cb < nblk; cb += 4) {
-          const int g = cb * 4 + q;
-          const int4 vg = vg_s[g];
-          const __half2 sub = *reinterpret_cast<const __half2*>(&vg.z);
-          uint32_t sc[8], out[8];
-          if (valid) {
-            const uint4 s0 = *reinterpret_cast<const uint4*>(blk + g * 32);
-            const uint4 s1 = *reinterpret_cast<const uint4*>(blk + g * 32 + 16);
-            sc[0] = s0.x; sc[1] = s0.y; sc[2] = s0.z; sc[3] = s0.w;
-            sc[4] = s1.x; sc[5] = s1.y; sc[6] = s1.z; sc[7] = s1.w;
-          } else {
-#pragma unroll
-            for (int i = 0; i < 8; ++i) sc[i] = 0u;
+              for (int x = 0; x < 8; ++x) sc[x] = 0u;
+            }
+            if (vg.x == 4) {
+              const uint2 cw = *reinterpret_cast<const uint2*>(blk + vg.y + lane * 8);
+              deq_channel4(cw.x, cw.y, sub, sc, out);
+            } else {
+              const int bit = 48 * lane;
+              const uint32_t* cw = reinterpret_cast<const uint32_t*>(blk + vg.y) + (bit >> 5);
+              const uint64_t x = ((uint64_t)cw[1] << 32 | cw[0]) >> (bit & 31);
+              deq_channel3(x, sub, sc, out);
+            }
+            tc::tmem_st8(tmem + lane_base + slot_col + (uint32_t)i * 8u, out);
           }
-          if (vg.x == 4) {
-            const uint2 cw = *reinterpret_cast<const uint2*>(blk + vg.y + lane * 8);
-            deq_channel4(cw.x, cw.y, sub, sc, out);
-          } else {
-            const int bit = 48 * lane;
-            const uint32_t* cw = reinterpret_cast<const uint32_t*>(blk + vg.y) + (bit >> 5);
-            const uint64_t x = ((uint64_t)cw[1] << 32 | cw[0]) >> (bit & 31);
-            deq_channel3(x, sub, sc, out);
-          }
-          tc::tmem_st8(tmem + lane_base + ycols + (uint32_t)(cur_as * nblk + cb) * 8u, out);
         }
+        tc::tmem_st_wait();
+        tc::tc_fence_before();
+        __syncwarp();
+        if (lane == 0) tc::mbar_arrive(&r_empty[rs]);
+        team_sync();   // the four quarters of the page's A tiles are in TMEM
+        if (issuer && lane == 0) {
+          tc::tc_fence_after();
+          const int ps = T & 1;
+          bool okp = true;
+          if (k == 0) {
+            okp = tc::mbar_wait_ab(&p_full[ps], ((uint32_t)(T >> 1)) & 1u, a.status, &abort_flag);
+            tc::tc_fence_after();
+          }
+          if (okp) {
+            const uint32_t bk = b_lo0 + (uint32_t)ps * p_step + (uint32_t)(k >> 2) * b_atom + (uint32_t)(k & 3) * 2u;
+            const uint32_t acc = (first && k == 0) ? 0u : 1u;
+#pragma unroll
+            for (int i = 0; i < NBT; ++i) {
+              if (i >= nbt) break;
+              tc::mma_f16_ts(tmem + (uint32_t)((j + 4 * i) * a.H), tmem + slot_col + (uint32_t)i * 8u, bk, b_hi,
+                             idesc, acc);
+            }
+          }
+          tc::mma_commit(&t_free[j][cur_as]);
+          if (k == 7) tc::mma_commit(&p_empty[ps]);
+        }
+        if (k == 7) first = false;
       }
-      tc::tmem_st_wait();
-      tc::tc_fence_before();
-      __syncwarp();
-      if (lane == 0) {
-        tc::mbar_arrive(&a_full[cur_as]);
-        tc::mbar_arrive(&r_empty[rs]);
-      }
+      if (cur_run >= 0) epilogue(cur_run);
     }
-    while (epi_run < n_runs) epilogue(epi_run++);
   }
   tc::tc_fence_before();
   __syncthreads();
@@ -648,13 +648,15 @@ bool plan_values_tc(starkv_layer* L) {
   const LayerView& v = L->view;
   const starkv_layer_config& c = L->cfg;
   if (!L->tc_scores) return false;
-  // power-of-two count of 128-channel value blocks, heads a multiple of 16;
-  // TMEM holds Y^T (nblk * H columns) and at least two pages of A tiles
-  // (nblk * 8 columns each) in its 512 columns
+  // power-of-two count of 128-channel value blocks (at most two per team),
+  // heads a multiple of 16; TMEM holds Y^T (nblk * H columns) and each team's
+  // ring of at least two pages of A tiles (8 columns per block)
   if (v.rv % 128 != 0 || ((v.rv / 128) & (v.rv / 128 - 1)) != 0 || v.H % 16 != 0 || v.H > 64) return false;
   const int nblk = v.rv / 128;
-  if (nblk * v.H + 2 * nblk * 8 > 512) return false;
-  L->val_na = std::min(kMaxASlots, (512 - nblk * v.H) / (nblk * 8));
+  if (nblk > 2 * kTeams) return false;
+  const int nbt = nblk > kTeams ? 2 : 1, n_teams = std::min(kTeams, nblk);
+  L->val_na = std::min(kMaxASlots, (512 - nblk * v.H) / (n_teams * nbt * 8));
+  if (L->val_na < 2) return false;
   const LatentDesc& ld = L->lat[v.L - 1];
   if (ld.n_groups * 32 != v.rv || !ld.cmajor) return false;
   for (int g = 0; g < ld.n_groups; ++g) {
@@ -669,7 +671,7 @@ bool plan_values_tc(starkv_layer* L) {
   L->vblk_bytes = (int)bytes;
   // as many raw stages as fit next to the static tables and barriers
   cudaFuncAttributes fa;
-  if (cudaFuncGetAttributes(&fa, k_values_tc) != cudaSuccess) return false;
+  if (cudaFuncGetAttributes(&fa, k_values_tc<2>) != cudaSuccess) return false;
   const int min_raw = 4;
   L->val_raw = 0;
   for (int n_raw = kMaxRawStages; n_raw >= min_raw && !L->val_raw; --n_raw)
@@ -729,9 +731,14 @@ cudaError_t launch_values_tc(const starkv_layer* L, const uint8_t* pool, long lo
   a.lseg = (float*)w;
   a.status = L->status;
   const size_t smem = values_smem(v.H, L->vblk_bytes, L->val_raw);
-  cudaError_t e = set_smem_limit((const void*)k_values_tc, smem);
+  const bool two = v.rv / 128 > kTeams;   // two channel blocks per team
+  const void* kern = two ? (const void*)k_values_tc<2> : (const void*)k_values_tc<1>;
+  cudaError_t e = set_smem_limit(kern, smem);
   if (e != cudaSuccess) return e;
-  k_values_tc<<<G, kValThreads, smem, s>>>(a);
+  if (two)
+    k_values_tc<2><<<G, kValThreads, smem, s>>>(a);
+  else
+    k_values_tc<1><<<G, kValThreads, smem, s>>>(a);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   if (ev_mid && (e = cudaEventRecord(ev_mid, s)) != cudaSuccess) return e;

@@ -166,6 +166,8 @@ cudaError_t launch_rotate_rows(const starkv_layer* L, const void* B, int dtype, 
                                cudaStream_t s);
 cudaError_t launch_fold_M(const starkv_layer* L, const float* Bv_rot, const void* W_o, cudaStream_t s);
 
+cudaError_t launch_wait_timeout_check(uint32_t* status, unsigned long long limit_ns, cudaStream_t s);
+
 cudaError_t launch_project(const starkv_layer* L, const void* x, int n, float* z, cudaStream_t s);
 cudaError_t launch_pack(const starkv_layer* L, uint8_t* pool, long long n_pages, const int32_t* page_table,
                         int n_seqs, int max_pages, int n, const int32_t* seq_idx, const int32_t* positions, const float* z,

@@ -78,14 +78,16 @@ __device__ __forceinline__ bool mbar_test_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 // Slow paths of the waits below, out of line: a phase that has not completed
-// is polled with a suspending try_wait until the limit.
-static __device__ __noinline__ bool mbar_wait_slow(uint64_t* bar, uint32_t parity, uint32_t* status, volatile int* abort) {
+// is polled with a suspending try_wait until `limit_ns` of the global timer
+// have passed.
+static __device__ __noinline__ bool mbar_wait_slow(uint64_t* bar, uint32_t parity, uint32_t* status, volatile int* abort,
+                                                   unsigned long long limit_ns = kWaitLimitNs) {
   if (mbar_try_wait(bar, parity)) return true;
   const unsigned long long t0 = global_ns();
   for (uint32_t i = 1;; ++i) {
     if (mbar_try_wait(bar, parity)) return true;
     if (abort && *abort) return false;
-    if ((i & 15u) == 0u && global_ns() - t0 > kWaitLimitNs) break;
+    if ((i & 15u) == 0u && global_ns() - t0 > limit_ns) break;
   }
   if (status) atomicOr(status, kTimeout);
   if (abort) *abort = 1;

@@ -31,7 +31,8 @@ DEV_BAD_PAGE, DEV_BAD_POSITION, DEV_SCALE_OVF, DEV_TIMEOUT = 0x1, 0x2, 0x4, 0x8
 EXPORTED = ["starkv_load_factors", "starkv_free_layer", "starkv_layer_get_info", "starkv_page_bytes",
             "starkv_cache_init", "starkv_append", "starkv_append_workspace_bytes", "starkv_decode_attn",
             "starkv_prefill_attn", "starkv_workspace_bytes", "starkv_sync_status", "starkv_status_string",
-            "starkv_last_error", "starkv_version", "starkv_decode_attn_noalloc", "starkv_set_decode_path"]
+            "starkv_last_error", "starkv_version", "starkv_decode_attn_noalloc", "starkv_set_decode_path",
+            "starkv_check_wait_timeout"]
 NOALLOC_SCRATCH_BYTES = 32 << 20
 
 
@@ -77,6 +78,7 @@ _lib.starkv_status_string.restype = ctypes.c_char_p
 _lib.starkv_last_error.argtypes = []
 _lib.starkv_last_error.restype = ctypes.c_char_p
 _lib.starkv_set_decode_path.argtypes = [_vp, ctypes.c_int]
+_lib.starkv_check_wait_timeout.argtypes = [_vp, ctypes.c_uint32, _vp]
 _lib.starkv_profile_decode.argtypes = [_vp, ctypes.c_int]
 _lib.starkv_decode_phase_ms.argtypes = [_vp, ctypes.POINTER(ctypes.c_float), ctypes.c_int]
 N_PHASES = 4   # query preparation + scores, joint values, run merge, output projection
@@ -235,6 +237,16 @@ class Layer:
         buf = (ctypes.c_float * (n_calls * N_PHASES))()
         _check(_lib.starkv_decode_phase_ms(self._h, buf, n_calls), "starkv_decode_phase_ms")
         return [list(buf[c * N_PHASES:(c + 1) * N_PHASES]) for c in range(n_calls)]
+
+    def check_wait_timeout(self, limit_us: int, stream=None) -> None:
+        """Run the bounded-wait diagnostic kernel (see starkv_check_wait_timeout)."""
+        _check(_lib.starkv_check_wait_timeout(self._h, limit_us, _stream(stream)), "starkv_check_wait_timeout")
+
+    def sync_status_code(self, stream=None) -> tuple:
+        """(status code of starkv_sync_status, status bits)."""
+        bits = ctypes.c_uint32(0)
+        st = _lib.starkv_sync_status(self._h, _stream(stream), ctypes.byref(bits))
+        return st, bits.value
 
     def sync_status(self, stream=None) -> int:
         bits = ctypes.c_uint32(0)

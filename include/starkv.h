@@ -310,6 +310,21 @@ STARKV_API starkv_status starkv_set_decode_path(starkv_layer* layer, int path);
  * STARKV_ERR_CUDA if events cannot be created or read.
  */
 #define STARKV_N_PHASES 4
+/*
+ * Diagnostics: exercise the bounded device-side wait that every pipelined
+ * kernel of the decode uses, without a fault.  One CTA waits on a barrier that
+ * nothing completes (no copy is issued, nobody arrives); after limit_us
+ * microseconds the wait gives up, sets STARKV_DEV_TIMEOUT in the layer's
+ * status word and raises the CTA's abort flag, and a second waiting role sees
+ * the flag and drains, as the other roles of a decode kernel do when one
+ * aborts.  No copy, MMA or tensor-memory allocation is in flight, and the CUDA
+ * context stays usable: starkv_sync_status() then returns STARKV_ERR_TIMEOUT.
+ * (The decode kernels' own limit is 2 seconds; "STAR-KV 阅读笔记" has no
+ * counterpart, this is failure detection of the library.)
+ * Returns STARKV_ERR_ARG for a NULL layer or limit_us outside [1, 2000000].
+ */
+STARKV_API starkv_status starkv_check_wait_timeout(const starkv_layer* layer, uint32_t limit_us,
+                                                   starkv_stream_t stream);
 STARKV_API starkv_status starkv_profile_decode(starkv_layer* layer, int n_calls);
 STARKV_API starkv_status starkv_decode_phase_ms(const starkv_layer* layer, float* ms, int n_calls);
 

@@ -308,6 +308,35 @@ def test_device_status_bad_page():
     assert L.sync_status() & 0x2
 
 
+def test_bounded_wait_expires_into_the_status_word():
+    """A bounded device wait on a barrier that nothing completes gives up after its limit, sets
+    STARKV_DEV_TIMEOUT and lets the waiting roles drain; the host reads STARKV_ERR_TIMEOUT and the
+    context stays usable for a normal decode afterwards."""
+    import time
+    from decode_attention_rank_b200 import starkv as lib
+    c = case(0)
+    L = c.load()
+    cache = GpuCache(L, [40])
+    Z = c.latents_direct(0, 40)
+    cache.append_latents(0, Z)
+    torch.cuda.synchronize()
+    assert L.sync_status() == 0
+    t0 = time.perf_counter()
+    L.check_wait_timeout(50000)                 # 50 ms
+    st, bits = L.sync_status_code()
+    dt = time.perf_counter() - t0
+    assert st == 6 and bits == lib.DEV_TIMEOUT, (st, bits)
+    assert 0.04 < dt < 5.0, dt
+    assert L.sync_status_code() == (0, 0)       # read-and-clear
+    q = queries(c, 1)[:, 0]
+    out = torch.empty(1, c.spec.hidden, device="cuda")
+    ws = torch.empty(L.workspace_bytes(1, cache.page_table.shape[1] * 16), dtype=torch.uint8, device="cuda")
+    L.decode(cache.pool, cache.n_pages, cache.page_table, torch.tensor([40], dtype=torch.int32, device="cuda"),
+             torch.from_numpy(q).cuda().float(), out, ws)
+    assert L.sync_status() == 0
+    check_close(out.double().cpu().numpy()[0], c.oracle_decode(c.stored(Z), q[0], 39, 40), "decode after timeout")
+
+
 def test_phase_timing_leaves_results_unchanged():
     """starkv_profile_decode records per-kernel times without changing the output."""
     c = case(2)
