@@ -148,7 +148,7 @@ def job_tokens_per_s(batch_per_rank: int, ws: int, ms_step_max: float) -> float:
 # Our arm
 # ---------------------------------------------------------------------------
 
-def build_layer(seed_offset: int = 0):
+def build_layer(seed_offset: int = 0, unfused: bool = False, max_positions: int = 0):
     """Seeded layer of the workload, loaded into the library."""
     import numpy as np
     import torch
@@ -161,7 +161,10 @@ def build_layer(seed_offset: int = 0):
         return torch.from_numpy(np.ascontiguousarray(x)).cuda().to(torch.bfloat16)
     A_k = torch.cat([t(a).reshape(-1) for a in f.A_k])
     B_k = torch.cat([t(b).reshape(-1) for b in f.B_k])
-    L = lib.load_factors(lib.LayerConfig.from_spec(spec), A_k, B_k, t(f.A_v), t(f.B_v), t(f.W_o))
+    cfg = lib.LayerConfig.from_spec(spec)
+    cfg.unfused_output = unfused
+    cfg.max_positions = max_positions
+    L = lib.load_factors(cfg, A_k, B_k, t(f.A_v), t(f.B_v), t(f.W_o))
     torch.cuda.synchronize()
     return spec, f, L
 
@@ -212,27 +215,33 @@ PHASES = ["query prep + key scoring (k_qprep_tc, k_scores_tc)", "joint value con
           "run merge (k_values_combine)", "output through M (k_outproj_tc, k_outproj_reduce)"]
 
 
-def phase_bytes(spec, B, ctx):
+def phase_bytes(spec, B, ctx, unfused=False):
     """Algorithmic HBM bytes of each decode phase: key cache + B'_k; value cache;
-    nothing (the merge reads kernel intermediates only); M + y/out."""
+    nothing (the merge reads kernel intermediates only); the output factors
+    (M, or B'_v per query head and W_o when unfused) + y/out."""
     key = sum(latent_bytes(spec, r) for r in spec.key_ranks)
     val = latent_bytes(spec, spec.value_rank)
     d = spec.head_dim
+    out_f = (2 * spec.n_heads * d * (spec.value_rank + spec.hidden) if unfused
+             else 2 * spec.n_heads * spec.value_rank * spec.hidden)
     return [B * ctx * key + 2 * d * sum(spec.key_ranks) + B * spec.n_heads * d * 2,
             B * ctx * val,
             0.0,
-            2 * spec.n_heads * spec.value_rank * spec.hidden + B * spec.hidden * 2]
+            out_f + B * spec.hidden * 2]
 
 
-def phase_flops(spec, B, ctx):
+def phase_flops(spec, B, ctx, unfused=False):
     """Algorithmic tensor flops of each decode phase: 2 r_h d per (token, head) to
     reconstruct, rope and score the keys (the G contraction); 2 r_v per (token,
-    query head) for P Z_v; none for the merge; 2 H r_v D per sequence for M."""
+    query head) for P Z_v; none for the merge; 2 H r_v D per sequence for M
+    (unfused: 2 H d (r_v + D))."""
     d = spec.head_dim
+    out_f = (B * 2.0 * spec.n_heads * d * (spec.value_rank + spec.hidden) if unfused
+             else B * 2.0 * spec.n_heads * spec.value_rank * spec.hidden)
     return [B * ctx * 2.0 * d * sum(spec.key_ranks) * (spec.n_heads // spec.n_kv_heads),
             B * ctx * 2.0 * spec.value_rank * spec.n_heads,
             0.0,
-            B * 2.0 * spec.n_heads * spec.value_rank * spec.hidden]
+            out_f]
 
 
 def measured_traffic(phase, tokens):
@@ -291,7 +300,7 @@ def run_ours(args, rank, ws, local):
     import torch
     B, ctx = WORKLOAD["batch"], WORKLOAD["ctx"]
     K, W = args.steps, args.warmup
-    spec, f, L = build_layer()
+    spec, f, L = build_layer(unfused=args.unfused)
     tail_pages = (W + K + 15) // 16
     T0 = ctx - 16 * tail_pages      # each step appends one token at T0 + i and decodes T0 + i + 1 tokens
     pool, n_pages, page_table, page_table_e2e = fill_cache(spec, f, L, B, T0, rank, ctx, tail_pages)
@@ -383,8 +392,8 @@ def run_ours(args, rank, ws, local):
     peak, peak_kind = measured_peaks()
     dbytes = decode_bytes(spec, L, B, T0 + W + K // 2)
     achieved = dbytes / (dec_ms * 1e-3) / 1e9
-    pbytes = phase_bytes(spec, B, T0 + W + K // 2)
-    pflops = phase_flops(spec, B, T0 + W + K // 2)
+    pbytes = phase_bytes(spec, B, T0 + W + K // 2, args.unfused)
+    pflops = phase_flops(spec, B, T0 + W + K // 2, args.unfused)
     tpeak, tpeak_kind = measured_tensor_peak()
     kernels = [{"phase": PHASES[p], "us": ph_ms[p] * 1e3, "algorithmic_bytes": pbytes[p],
                 "GB/s": (pbytes[p] / (ph_ms[p] * 1e-3) / 1e9) if ph_ms[p] > 0 else None,
@@ -411,7 +420,8 @@ def run_ours(args, rank, ws, local):
         "data": "synthetic (seeded latents with the factor spectrum; random-init factors)",
         "config": {"workload": f"STAR-KV decode step: append 1 token/seq + decode, batch {B}, ctx ~{ctx} "
                                f"(LongChat-7B-shaped layer: H 32, d 128, D 4096, R_k 1024, r_v 1024, "
-                               f"block Hadamard 32, 4/3-bit latents, 16-token pages)",
+                               f"block Hadamard 32, 4/3-bit latents, 16-token pages"
+                               + (", unfused value output y_h B_v,h then W_o)" if args.unfused else ")"),
                    "batch": B, "ctx": ctx, "ctx_range": [T0 + W + 1, T0 + W + K], "parallelism": f"replicas x{ws}",
                    "l2": "inputs larger than L2 (cache %.0f MB + M %.0f MB)" % (B * ctx * L.bytes_per_token / 1e6,
                                                                             L.factor_bytes / 1e6)},
@@ -429,9 +439,12 @@ def run_ours(args, rank, ws, local):
         "kernels": kernels,
         "e2e": {"value": B * ws / (e2e_ms * 1e-3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h},
-        "gpu_launches": K * 10,   # append: 4 kernels; decode: 6 (see the launch list under profiles/)
+        # append: 4 kernels; decode: 6 (unfused output: 9); see the launch list under profiles/
+        "gpu_launches": K * (13 if args.unfused else 10),
         "clocks": clk,
     }
+    if args.unfused:
+        res["mode"] = "unfused value output"
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:
         dt, cores = cpu_baseline(ctx)
         res["cpu_baseline"] = {"value": 1.0 / dt, "unit": "tokens/s", "cores": cores, "kind": "oracle",
@@ -496,12 +509,16 @@ def run_prefill(args):
     for _ in range(args.warmup):
         L.prefill(pool, n_pages, page_table, [T - n], [n], q, out, ws)
     torch.cuda.synchronize()
+    clocks = ClockSampler(0)
+    clocks.start()
+    time.sleep(0.3)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record()
     for _ in range(args.steps):
         L.prefill(pool, n_pages, page_table, [T - n], [n], q, out, ws)
     e1.record()
     torch.cuda.synchronize()
+    clk = clocks.stop()
     status = L.sync_status()
     ms = e0.elapsed_time(e1) / args.steps
     return {"metric": "causal prefill query tokens/s (latent attention over the paged cache)", "value": n / (ms * 1e-3),
@@ -511,7 +528,7 @@ def run_prefill(args):
             "config": {"workload": f"prefill chunk of {n} queries after {T - n} tokens of history, batch 1 "
                                    "(LongChat-7B-shaped layer, 4/3-bit latents)", "batch": 1, "ctx": T,
                        "queries": n},
-            "device_status": status}
+            "clocks": clk, "device_status": status}
 
 
 def run_plain(args):
@@ -551,17 +568,12 @@ def run_plain(args):
     out = torch.empty(B, spec.hidden, dtype=torch.bfloat16, device="cuda")
     ws = torch.empty(L.workspace_bytes(B, pages * 16), dtype=torch.uint8, device="cuda")
     lens = torch.full((B,), T, dtype=torch.int32, device="cuda")
-    for _ in range(args.warmup):
-        L.decode(pool, n_pages, page_table, lens, q, out, ws)
-    torch.cuda.synchronize()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record()
-    for _ in range(args.steps):
-        L.decode(pool, n_pages, page_table, lens, q, out, ws)
-    e1.record()
-    torch.cuda.synchronize()
+    clocks = ClockSampler(0)
+    clocks.start()
+    time.sleep(0.3)
+    ms = _time_decodes(L, pool, n_pages, page_table, lens, q, out, ws, args.steps, args.warmup)
+    clk = clocks.stop()
     status = L.sync_status()
-    ms = e0.elapsed_time(e1) / args.steps
     peak, peak_kind = measured_peaks()
     # algorithmic bytes: K and V of every cached token (bf16) + W_o + q/out
     dbytes = B * T * 2 * 2 * spec.n_kv_heads * spec.head_dim + 2 * spec.n_heads * spec.head_dim * spec.hidden + \
@@ -575,7 +587,94 @@ def run_plain(args):
                        "batch": B, "ctx": T},
             "roofline": {"bound": "hbm", "achieved": gbs, "peak": peak, "peak_kind": peak_kind, "unit": "GB/s",
                          "frac": gbs / peak, "algorithmic_bytes": dbytes},
-            "device_status": status}
+            "clocks": clk, "device_status": status}
+
+
+def _time_decodes(L, pool, n_pages, page_table, lens, q, out, ws, steps, warmup):
+    import torch
+    for _ in range(warmup):
+        L.decode(pool, n_pages, page_table, lens, q, out, ws)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(steps):
+        L.decode(pool, n_pages, page_table, lens, q, out, ws)
+    e1.record()
+    torch.cuda.synchronize()
+    assert L.sync_status() == 0
+    return e0.elapsed_time(e1) / steps
+
+
+def run_compare_plain(args):
+    """The in-house counterpart of the reading notes' attention-module speed-up
+    (section 8.1-8.2: latent attention against uncompressed attention at batch
+    16, long contexts): decode of one uncompressed bf16 layer (plain K/V) and of
+    one 4/3-bit latent layer of the same LongChat-7B / LLaMA-2-7B shape (H 32,
+    d 128, D 4096) at batch 16 over a list of contexts, one JSON line."""
+    import numpy as np
+    import torch
+    from decode_attention_rank_b200 import starkv as lib
+    from synth import gen
+    torch.cuda.set_device(0)
+    B = args.batch or 16
+    ctxs = [int(x) for x in args.compare_plain.split(",")]
+    pspec = gen.config_spec(4, layer=0)
+    pf = gen.make_factors(pspec, gen.LAYER_SEED[4], 0)
+
+    def t(x):
+        return torch.from_numpy(np.ascontiguousarray(x)).cuda().to(torch.bfloat16)
+    pcfg = lib.LayerConfig.from_spec(pspec)
+    PL = lib.load_factors(pcfg, t(pf.W_k), None, t(pf.W_v), None, t(pf.W_o))
+    clocks = ClockSampler(0)
+    clocks.start()
+    rows = []
+    g = torch.Generator(device="cuda")
+    g.manual_seed(4242)
+    q = (torch.randn(B, 32, 128, generator=g, device="cuda") / math.sqrt(128)).to(torch.bfloat16)
+    out = torch.empty(B, 4096, dtype=torch.bfloat16, device="cuda")
+    for T in ctxs:
+        pages = T // 16
+        lens = torch.full((B,), T, dtype=torch.int32, device="cuda")
+        # plain layer: K (after RoPE) and V, bf16
+        n_pages = B * pages
+        pt = torch.randperm(n_pages, generator=g, device="cuda").to(torch.int32).reshape(B, pages).contiguous()
+        pool = torch.empty(n_pages * PL.page_bytes, dtype=torch.uint8, device="cuda")
+        PL.cache_init(pool, n_pages)
+        for b in range(B):
+            for c0 in range(0, T, 4096):
+                n = min(4096, T - c0)
+                z = torch.randn(n, PL.latent_total, generator=g, device="cuda")
+                PL.append(pool, n_pages, pt, torch.full((n,), b, dtype=torch.int32, device="cuda"),
+                          torch.arange(c0, c0 + n, dtype=torch.int32, device="cuda"), z, True)
+        ws = torch.empty(PL.workspace_bytes(B, pages * 16), dtype=torch.uint8, device="cuda")
+        ms_plain = _time_decodes(PL, pool, n_pages, pt, lens, q, out, ws, args.steps, args.warmup)
+        plain_bytes = B * T * PL.bytes_per_token + PL.factor_bytes
+        del pool, ws
+        torch.cuda.empty_cache()
+        # latent layer (4/3-bit, block Hadamard), RoPE table covering the context
+        spec, f, L = build_layer(max_positions=max(T, 32768))
+        lpool, ln_pages, lpt, _ = fill_cache(spec, f, L, B, T, 0, T, 0)
+        lws = torch.empty(L.workspace_bytes(B, lpt.shape[1] * 16), dtype=torch.uint8, device="cuda")
+        ms_lat = _time_decodes(L, lpool, ln_pages, lpt, lens, q, out, lws, args.steps, args.warmup)
+        lat_bytes = B * T * L.bytes_per_token + L.factor_bytes
+        del lpool, lws, L
+        torch.cuda.empty_cache()
+        rows.append({"ctx": T, "plain_us": ms_plain * 1e3, "latent_us": ms_lat * 1e3,
+                     "speedup": ms_plain / ms_lat,
+                     "plain_GBps": plain_bytes / (ms_plain * 1e-3) / 1e9,
+                     "latent_GBps": lat_bytes / (ms_lat * 1e-3) / 1e9,
+                     "plain_bytes": plain_bytes, "latent_bytes": lat_bytes})
+    clk = clocks.stop()
+    peak, peak_kind = measured_peaks()
+    return {"metric": "attention-module decode speed-up, latent 4/3-bit layer vs uncompressed bf16 layer",
+            "value": rows[-1]["speedup"], "unit": "x (plain time / latent time)", "n_gpus": 1,
+            "steps": args.steps, "warmup": args.warmup, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16 K/V vs u3/u4 latent codes + fp16 scales", "data": "synthetic",
+            "mode": "compare_plain",
+            "config": {"workload": f"decode of one LongChat-7B / LLaMA-2-7B-shaped attention layer (H 32, d 128, "
+                                   f"D 4096), batch {B}: uncompressed bf16 K/V against STAR-KV 4/3-bit latents "
+                                   f"(ragged key ranks mean 32, r_v 1024, fused M_h)", "batch": B, "ctxs": ctxs},
+            "points": rows, "hbm_peak": peak, "hbm_peak_kind": peak_kind, "clocks": clk}
 
 
 def main():
@@ -591,9 +690,16 @@ def main():
     ap.add_argument("--batch", type=int, default=0, help="sequences per step (default 16)")
     ap.add_argument("--prefill", type=int, default=0, help="time a causal prefill chunk of this many queries "
                     "(history = ctx - queries, ctx default 4096) instead of the decode step")
+    ap.add_argument("--unfused", action="store_true", help="the workload with the unfused value output "
+                    "(y_h B_v,h then W_o) instead of the fused M_h (separate line; the fused form is the headline)")
     ap.add_argument("--plain", action="store_true", help="time the decode of an uncompressed layer of the "
                     "32-layer stack instead (batch/ctx from --batch/--ctx, default 16 and 4096)")
+    ap.add_argument("--compare-plain", default="", help="comma-separated contexts: time an uncompressed layer "
+                    "against a 4/3-bit latent layer at each (batch from --batch, default 16); one JSON line")
     args = ap.parse_args()
+    if args.compare_plain:
+        print(json.dumps(run_compare_plain(args)), flush=True)
+        return
     if args.plain:
         print(json.dumps(run_plain(args)), flush=True)
         return

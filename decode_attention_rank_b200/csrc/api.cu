@@ -160,8 +160,10 @@ static starkv_status plan_layer(starkv_layer* L) {
   L->key_off.assign(Hkv + 1, 0);
   for (int h = 0; h < Hkv; ++h) L->key_off[h + 1] = L->key_off[h] + widths[h];
   const size_t mel = c.dtype == STARKV_F32 ? 4 : 2;
+  L->unfused = c.unfused_output ? 1 : 0;
   L->factor_bytes = (c.plain ? 0 : (size_t)v.Rk * d * (c.dtype == STARKV_F32 ? 4 : 2)) +
-                    (size_t)c.hidden * c.n_heads * v.wv * mel;
+                    (L->unfused ? 2 * (size_t)c.n_heads * d * ((size_t)v.rv + c.hidden)   // B'_v per head + W_o
+                                : (size_t)c.hidden * c.n_heads * v.wv * mel);             // M
   return STARKV_OK;
 }
 
@@ -190,6 +192,10 @@ static starkv_status check_config(const starkv_layer_config* c) {
     CHECK_ARG(c->hadamard_block == c->group_size, "hadamard_block must equal group_size");
   }
   if (c->rope) CHECK_ARG(c->rope_theta > 1.0, "rope_theta must be > 1");
+  if (c->unfused_output) {
+    CHECK_ARG(c->dtype == STARKV_BF16 && !c->plain && c->head_dim == 128 && c->value_rank % 64 == 0,
+              "unfused_output needs a bf16 compressed layer with head_dim 128 and value_rank a multiple of 64");
+  }
   return STARKV_OK;
 }
 
@@ -226,6 +232,8 @@ void starkv_free_layer(starkv_layer* L) {
   cudaFree(L->A_tiles);
   cudaFree(L->Bk);
   cudaFree(L->M_T);
+  cudaFree(L->Bv_tiles);
+  cudaFree(L->Wo_tiles);
   cudaFree(L->status);
   cudaFree(L->d_items);
   cudaFree(L->d_score_heads);
@@ -263,10 +271,17 @@ starkv_status starkv_load_factors(const starkv_layer_config* cfg, const void* A_
       cudaMalloc(&L->d_grp, sizeof(GroupDesc) * L->grp.size()) != cudaSuccess ||
       cudaMalloc(&L->d_key_off, sizeof(int) * L->key_off.size()) != cudaSuccess ||
       cudaMalloc(&L->status, sizeof(uint32_t)) != cudaSuccess ||
-      cudaMalloc(&L->A_T, es * (size_t)v.Ltot * D) != cudaSuccess ||
-      cudaMalloc(&L->M_T, cfg->dtype == STARKV_F32 ? 4 * (size_t)D * H * v.wv : 2 * (size_t)L->Dp * L->Kp) !=
-          cudaSuccess)
+      cudaMalloc(&L->A_T, es * (size_t)v.Ltot * D) != cudaSuccess)
     return fail(STARKV_ERR_OOM, "cudaMalloc");
+  const size_t wo_tiles_bytes = (size_t)(L->Dp / 128) * (H * d / 64) * 16384;
+  if (L->unfused) {
+    if (cudaMalloc(&L->Bv_tiles, (size_t)H * (v.rv / 64) * 16384) != cudaSuccess ||
+        cudaMalloc(&L->Wo_tiles, wo_tiles_bytes) != cudaSuccess)
+      return fail(STARKV_ERR_OOM, "cudaMalloc");
+  } else if (cudaMalloc(&L->M_T, cfg->dtype == STARKV_F32 ? 4 * (size_t)D * H * v.wv : 2 * (size_t)L->Dp * L->Kp) !=
+             cudaSuccess) {
+    return fail(STARKV_ERR_OOM, "cudaMalloc");
+  }
   if (!cfg->plain && cudaMalloc(&L->Bk, sizeof(float) * (size_t)v.Rk * d) != cudaSuccess)
     return fail(STARKV_ERR_OOM, "cudaMalloc");
   v.lat = L->d_lat;
@@ -282,7 +297,8 @@ starkv_status starkv_load_factors(const starkv_layer_config* cfg, const void* A_
       cudaMemcpyAsync(L->d_grp, L->grp.data(), sizeof(GroupDesc) * L->grp.size(), cudaMemcpyHostToDevice, s) ||
       cudaMemcpyAsync(L->d_key_off, L->key_off.data(), sizeof(int) * L->key_off.size(), cudaMemcpyHostToDevice, s) ||
       cudaMemsetAsync(L->status, 0, sizeof(uint32_t), s) ||
-      (cfg->dtype != STARKV_F32 && cudaMemsetAsync(L->M_T, 0, 2 * (size_t)L->Dp * L->Kp, s)))
+      (L->M_T && cfg->dtype != STARKV_F32 && cudaMemsetAsync(L->M_T, 0, 2 * (size_t)L->Dp * L->Kp, s)) ||
+      (L->Wo_tiles && cudaMemsetAsync(L->Wo_tiles, 0, wo_tiles_bytes, s)))
     return fail(STARKV_ERR_CUDA, "upload tables");
   // Projection rows A_T[ch][k] for every latent channel (keys, then values).
   if (cfg->plain) {
@@ -325,7 +341,7 @@ starkv_status starkv_load_factors(const starkv_layer_config* cfg, const void* A_
       return fail(STARKV_ERR_CUDA, "rotate B_v");
     }
   }
-  cudaError_t e = launch_fold_M(L, Bv_rot, W_o, s);
+  cudaError_t e = L->unfused ? launch_build_unfused(L, Bv_rot, W_o, s) : launch_fold_M(L, Bv_rot, W_o, s);
   if (Bv_rot) {
     cudaStreamSynchronize(s);
     cudaFree(Bv_rot);

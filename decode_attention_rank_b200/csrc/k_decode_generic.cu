@@ -327,6 +327,11 @@ WsPlan plan_ws(const starkv_layer* L, int rows, int max_len, bool prefill) {
   const int cblocks = (v.rv + value_block(v) - 1) / value_block(v);
   int ns = (int)((2 * 148 * 2 + (long long)rows * cblocks - 1) / ((long long)rows * cblocks));
   ns = std::max(1, std::min(ns, (max_len + 511) / 512));
+  if (plain_decode_supported(v)) {
+    // streaming plain-layer kernel: (row, KV head, split) CTAs, four or more per SM, >= 256 tokens each
+    const long long per = (long long)rows * v.Hkv;
+    ns = (int)std::max(1LL, std::min((4LL * num_sms() + per - 1) / per, (long long)(max_len + 255) / 256));
+  }
   if (prefill) ns = 1;
   p.n_splits = ns;
   p.chunk = (max_len + ns - 1) / ns;
@@ -383,7 +388,12 @@ cudaError_t launch_decode_generic(const starkv_layer* L, const uint8_t* pool, lo
   const size_t smem = sizeof(float) * kTile * (size_t)(rmax + v.d);
   cudaError_t e = set_smem_limit((const void*)k_scores, smem);
   if (e != cudaSuccess) return e;
-  if (tc_scores) {
+  if (plain_decode_supported(v) && !tc_scores) {
+    // uncompressed bf16 layer: one streaming pass over K and V, partials for the merge below
+    e = launch_plain_decode(L, pool, n_pages, page_table, max_pages, rows, ri, qrot, p.n_splits, p.chunk, pY, pm, pl,
+                            s);
+    if (e != cudaSuccess) return e;
+  } else if (tc_scores) {
     // scores (log2 units) from the tensor-core kernel, written into S
     ScoreOut so;
     e = launch_scores_tc(L, pool, n_pages, page_table, max_pages, rows, ri.row_len, ri.row_pos, q, w + p.total, &so,
@@ -393,10 +403,12 @@ cudaError_t launch_decode_generic(const starkv_layer* L, const uint8_t* pool, lo
     k_scores<<<dim3((max_len + kTile - 1) / kTile, v.Hkv, rows), 256, smem, s>>>(
         v, pool, n_pages, page_table, max_pages, ri, L->Bk, L->d_key_off, qrot, S, p.S_ld);
   }
-  const int vb = value_block(v);
-  const int cblocks = (v.rv + vb - 1) / vb;
-  k_value<<<dim3(cblocks, p.n_splits, rows), kVBlock, 0, s>>>(v, pool, n_pages, page_table, max_pages, ri, S, p.S_ld,
-                                                              p.n_splits, p.chunk, vb, pY, pm, pl);
+  if (!(plain_decode_supported(v) && !tc_scores)) {
+    const int vb = value_block(v);
+    const int cblocks = (v.rv + vb - 1) / vb;
+    k_value<<<dim3(cblocks, p.n_splits, rows), kVBlock, 0, s>>>(v, pool, n_pages, page_table, max_pages, ri, S,
+                                                                p.S_ld, p.n_splits, p.chunk, vb, pY, pm, pl);
+  }
   if (v.dtype == STARKV_F32) {
     k_combine<float><<<dim3(rows, v.H), 128, 0, s>>>(v, ri, p.n_splits, pY, pm, pl, (float*)y);
     k_out<float, float><<<(v.D * 32 + 255) / 256, 256, 0, s>>>((const float*)y, (const float*)L->M_T, rows,

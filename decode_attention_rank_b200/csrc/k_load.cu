@@ -166,6 +166,36 @@ cudaError_t launch_fold_M(const starkv_layer* L, const float* Bv_rot, const void
   return cudaGetLastError();
 }
 
+// B'_v per query head as the A operand of the grouped output GEMM: tile
+// (h, j / 64) holds rows p < d (output z[h d + p]) and columns j (value
+// channel), element B'_v[j][kv(h) d + p], fp16, 128-byte swizzled.
+__global__ void k_bv_tiles(const float* __restrict__ Bv_rot, int rv, int d, int Hkv, int group_q, int H,
+                           __half* __restrict__ tiles) {
+  const long long idx = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  if (idx >= (long long)H * rv * d) return;
+  const int p = (int)(idx % d);
+  const long long r = idx / d;
+  const int j = (int)(r % rv), h = (int)(r / rv);
+  const int kv = h / group_q;
+  const int KT = rv / 64;
+  const size_t tile = ((size_t)h * KT + (j >> 6)) * (128 * 64);
+  tiles[tile + tc_sw128_elem((uint32_t)p, (uint32_t)(j & 63))] = __float2half_rn(Bv_rot[(size_t)j * Hkv * d + kv * d + p]);
+}
+
+cudaError_t launch_build_unfused(starkv_layer* L, const float* Bv_rot, const void* W_o, cudaStream_t s) {
+  const LayerView& v = L->view;
+  const long long n = (long long)v.H * v.rv * v.d;
+  k_bv_tiles<<<(unsigned)((n + 255) / 256), 256, 0, s>>>(Bv_rot, v.rv, v.d, v.Hkv, v.group_q, v.H,
+                                                         (__half*)L->Bv_tiles);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  // W_o^T tiles: the fold with the identity in place of B'_v (k = h d + p)
+  dim3 grid((v.D + 63) / 64, (v.d + 63) / 64, v.H);
+  k_fold_M<__nv_bfloat16, __half><<<grid, 256, 0, s>>>(nullptr, 0, (const __nv_bfloat16*)W_o, v.D, v.d, v.d,
+                                                       v.group_q, v.H, 1, v.H * v.d / 64, (__half*)L->Wo_tiles);
+  return cudaGetLastError();
+}
+
 }  // namespace starkv
 
 namespace starkv {

@@ -23,7 +23,9 @@ constexpr int kOutThreads = 192;  // warp 0 producer, warp 1 MMA, warps 2-5 epil
 
 struct OutArgs {
   const uint8_t* M;   // [DT][KT] tiles of 128 x 64 fp16, 16 KB each
-  const uint8_t* y;   // [NTILES][KT] tiles of NB x 64 fp16
+  const uint8_t* y;   // [NTILES][KTy] tiles of NB x 64 fp16
+  int KTy;            // k-tiles of one row tile of y
+  int y_step;         // output tile dt reads y k-tiles dt * y_step .. dt * y_step + KT - 1 (0: all read 0 .. KT - 1)
   float* part;        // [grid.x][slots][NB][128] partial sums
   int NB;             // rows of one B tile (multiple of 16, <= 256)
   int KT, DT;         // k-tiles, output tiles
@@ -75,7 +77,8 @@ __global__ void __launch_bounds__(kOutThreads, 1) k_outproj_tc(OutArgs a) {
       uint32_t ph = 0;
       int kt = (int)(u0 % a.KT);
       const uint8_t* msrc = a.M + (size_t)u0 * a_bytes;
-      const uint8_t* ybase = a.y + (size_t)nt * a.KT * b_bytes;
+      const uint8_t* ybase = a.y + (size_t)nt * a.KTy * b_bytes;
+      int dt = (int)(u0 / a.KT);
       for (long long u = u0; u < u1; ++u, ++i) {
         if (!tc::mbar_wait(&empty[s], ph ^ 1u, a.status)) {
           abort_flag = 1;
@@ -83,9 +86,12 @@ __global__ void __launch_bounds__(kOutThreads, 1) k_outproj_tc(OutArgs a) {
         }
         tc::mbar_expect_tx(&full[s], a_bytes + b_bytes);
         tc::bulk_g2s(A_s + (size_t)s * a_bytes, msrc, a_bytes, &full[s]);
-        tc::bulk_g2s(B_s + (size_t)s * b_bytes, ybase + (size_t)kt * b_bytes, b_bytes, &full[s]);
+        tc::bulk_g2s(B_s + (size_t)s * b_bytes, ybase + (size_t)(dt * a.y_step + kt) * b_bytes, b_bytes, &full[s]);
         msrc += a_bytes;
-        if (++kt == a.KT) kt = 0;
+        if (++kt == a.KT) {
+          kt = 0;
+          ++dt;
+        }
         if (++s == a.stages) {
           s = 0;
           ph ^= 1u;
@@ -235,16 +241,35 @@ size_t gemm_part_bytes(int n_out, int K, int rows) {
   return sizeof(float) * (size_t)ntiles * g.G * g.slots * NB * 128;
 }
 
-size_t outproj_part_bytes(const starkv_layer* L, int rows) { return gemm_part_bytes(L->Dp, L->Kp, rows); }
+// Unfused output ("STAR-KV 阅读笔记" section 5.3 states the fusion M_h =
+// B_v,h W_o,h as an exact reorder, so either order is the same product):
+// z_h = y_h B'_v,kv(h) (a grouped GEMM, one 128-output tile per head over that
+// head's r_v columns of y), then out = z W_o.  The workspace holds z (fp32),
+// z as fp16 B tiles, and the partial sums of either GEMM.
+static size_t unfused_z_bytes(const starkv_layer* L, int rows) {
+  return ((sizeof(float) * (size_t)rows * L->view.H * L->view.d) + 255) / 256 * 256;
+}
+static size_t unfused_zt_bytes(const starkv_layer* L, int rows) {
+  return (rows_tiles_bytes(rows, L->view.H * L->view.d) + 255) / 256 * 256;
+}
+
+size_t outproj_part_bytes(const starkv_layer* L, int rows) {
+  if (!L->unfused) return gemm_part_bytes(L->Dp, L->Kp, rows);
+  const LayerView& v = L->view;
+  return unfused_z_bytes(L, rows) + unfused_zt_bytes(L, rows) +
+         std::max(gemm_part_bytes(v.H * v.d, v.wv, rows), gemm_part_bytes(L->Dp, v.H * v.d, rows));
+}
 
 cudaError_t launch_gemm_tc(const uint8_t* Mt, int n_out, int K, int n_valid, const void* y_tiles, int rows,
-                           void* out, bool out_f32, float* part, uint32_t* status, cudaStream_t s) {
+                           void* out, bool out_f32, float* part, uint32_t* status, cudaStream_t s, int y_group) {
   const OutGeom g = gemm_geom(n_out, K);
   const int NB = outproj_nb(rows);
   const int ntiles = (rows + NB - 1) / NB;
   OutArgs a;
   a.M = Mt;
   a.y = (const uint8_t*)y_tiles;
+  a.KTy = y_group ? g.KT * g.DT : g.KT;
+  a.y_step = y_group ? g.KT : 0;
   a.NB = NB;
   a.KT = g.KT;
   a.DT = g.DT;
@@ -260,7 +285,7 @@ cudaError_t launch_gemm_tc(const uint8_t* Mt, int n_out, int K, int n_valid, con
   if (e != cudaSuccess) return e;
   for (int t = 0; t < ntiles; ++t) {
     OutArgs at = a;
-    at.y = a.y + (size_t)t * g.KT * NB * 128;
+    at.y = a.y + (size_t)t * a.KTy * NB * 128;
     at.part = part + (size_t)t * g.G * g.slots * NB * 128;
     k_outproj_tc<<<dim3(g.G, 1), kOutThreads, smem, s>>>(at);
   }
@@ -275,12 +300,31 @@ cudaError_t launch_gemm_tc(const uint8_t* Mt, int n_out, int K, int n_valid, con
 
 cudaError_t launch_outproj_tc(const starkv_layer* L, const void* y_tiles, int rows, void* out, float* part,
                               cudaStream_t s) {
+  if (L->unfused) {
+    const LayerView& v = L->view;
+    uint8_t* w = (uint8_t*)part;
+    float* z = (float*)w;
+    w += unfused_z_bytes(L, rows);
+    void* zt = w;
+    w += unfused_zt_bytes(L, rows);
+    float* p2 = (float*)w;
+    cudaError_t e = launch_gemm_tc((const uint8_t*)L->Bv_tiles, v.H * v.d, v.wv, v.H * v.d, y_tiles, rows, z, true,
+                                   p2, L->status, s, 1);
+    if (e != cudaSuccess) return e;
+    e = launch_pack_rows_tiles_f32(z, rows, v.H * v.d, zt, s);
+    if (e != cudaSuccess) return e;
+    return launch_gemm_tc((const uint8_t*)L->Wo_tiles, L->Dp, v.H * v.d, v.D, zt, rows, out, false, p2, L->status, s);
+  }
   return launch_gemm_tc((const uint8_t*)L->M_T, L->Dp, L->Kp, L->view.D, y_tiles, rows, out,
                         L->view.dtype == STARKV_F32, part, L->status, s);
 }
 
-// fp16 B-operand tiles [rows / NB][K / 64][NB][64] (swizzled, zero padded) from a row-major bf16 matrix.
-__global__ void k_pack_rows_tiles(const __nv_bfloat16* __restrict__ x, int rows, int K, int NB, int KT,
+__device__ __forceinline__ float ld_any(const __nv_bfloat16* p, size_t i) { return __bfloat162float(p[i]); }
+__device__ __forceinline__ float ld_any(const float* p, size_t i) { return p[i]; }
+
+// fp16 B-operand tiles [rows / NB][K / 64][NB][64] (swizzled, zero padded) from a row-major bf16 or fp32 matrix.
+template <typename T>
+__global__ void k_pack_rows_tiles(const T* __restrict__ x, int rows, int K, int NB, int KT,
                                   uint8_t* __restrict__ tiles) {
   const long long idx = (long long)blockIdx.x * blockDim.x + threadIdx.x;   // one 8-column chunk
   const int nchunk = KT * 8;
@@ -293,8 +337,8 @@ __global__ void k_pack_rows_tiles(const __nv_bfloat16* __restrict__ x, int rows,
 #pragma unroll
     for (int i = 0; i < 8; i += 2) {
       const int k = kt * 64 + c * 8 + i;
-      const float f0 = k < K ? __bfloat162float(x[(size_t)row * K + k]) : 0.f;
-      const float f1 = k + 1 < K ? __bfloat162float(x[(size_t)row * K + k + 1]) : 0.f;
+      const float f0 = k < K ? ld_any(x, (size_t)row * K + k) : 0.f;
+      const float f1 = k + 1 < K ? ld_any(x, (size_t)row * K + k + 1) : 0.f;
       const __half2 h = __floats2half2_rn(f0, f1);
       o[i / 2] = *reinterpret_cast<const uint32_t*>(&h);
     }
@@ -308,8 +352,17 @@ cudaError_t launch_pack_rows_tiles(const void* x, int rows, int K, void* tiles, 
   const int KT = (K + 63) / 64;
   const int ntiles = (rows + NB - 1) / NB;
   const long long n = (long long)ntiles * NB * KT * 8;
-  k_pack_rows_tiles<<<(unsigned)((n + 255) / 256), 256, 0, s>>>((const __nv_bfloat16*)x, rows, K, NB, KT,
-                                                               (uint8_t*)tiles);
+  k_pack_rows_tiles<__nv_bfloat16><<<(unsigned)((n + 255) / 256), 256, 0, s>>>((const __nv_bfloat16*)x, rows, K, NB,
+                                                                              KT, (uint8_t*)tiles);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_pack_rows_tiles_f32(const float* x, int rows, int K, void* tiles, cudaStream_t s) {
+  const int NB = outproj_nb(rows);
+  const int KT = (K + 63) / 64;
+  const int ntiles = (rows + NB - 1) / NB;
+  const long long n = (long long)ntiles * NB * KT * 8;
+  k_pack_rows_tiles<float><<<(unsigned)((n + 255) / 256), 256, 0, s>>>(x, rows, K, NB, KT, (uint8_t*)tiles);
   return cudaGetLastError();
 }
 

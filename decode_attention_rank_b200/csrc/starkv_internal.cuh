@@ -130,6 +130,10 @@ struct starkv_layer {
   // (the A operand of the tensor-core output kernel), zero padded.
   void* M_T = nullptr;
   int Kp = 0, Dp = 0;           // H * wv and D rounded up to 64 and 128
+  // unfused output (config unfused_output = 1): no M; y_h B'_v,kv(h) then W_o on the tensor cores
+  int unfused = 0;
+  void* Bv_tiles = nullptr;     // fp16 tiles [H][r_v / 64] of 128 x 64: row p, column j = B'_v[j][kv(h) d + p]
+  void* Wo_tiles = nullptr;     // fp16 tiles [Dp / 128][H d / 64] of 128 x 64: row n, column k = W_o[k][n]
   uint32_t* status = nullptr;
   // tensor-core score kernel
   bool tc_scores = false;
@@ -185,6 +189,13 @@ cudaError_t launch_decode_generic(const starkv_layer* L, const uint8_t* pool, lo
                                   cudaStream_t s, bool tc_scores = false);
 size_t decode_generic_ws_bytes(const starkv_layer* L, int rows, int max_len, bool prefill);
 
+// Uncompressed bf16 layers with head_dim 128: a streaming CUDA-core decode
+// writing split partials (pY [rows][n_splits][H][128], pm, pl) for the merge.
+bool plain_decode_supported(const LayerView& v);
+cudaError_t launch_plain_decode(const starkv_layer* L, const uint8_t* pool, long long n_pages, const int32_t* pt,
+                                int max_pages, int rows, RowInfo ri, const float* qrot, int n_splits, int chunk,
+                                float* pY, float* pm, float* pl, cudaStream_t s);
+
 int num_sms();
 
 // Raise a kernel's dynamic shared-memory limit to `bytes` on the current
@@ -218,10 +229,16 @@ OutGeom gemm_geom(int n_out, int K);
 size_t gemm_part_bytes(int n_out, int K, int rows);
 size_t outproj_part_bytes(const starkv_layer* L, int rows);
 // out[row][n] = sum_k y[row][k] Mt[n][k] with Mt as fp16 128x64 swizzled tiles, y as fp16 B tiles.
+// y_group != 0: a block-diagonal (grouped) product, output tile dt (128 outputs) contracting only
+// y's k-range [dt * K, dt * K + K) (y has n_out / 128 * K columns).
 cudaError_t launch_gemm_tc(const uint8_t* Mt, int n_out, int K, int n_valid, const void* y_tiles, int rows,
-                           void* out, bool out_f32, float* part, uint32_t* status, cudaStream_t s);
+                           void* out, bool out_f32, float* part, uint32_t* status, cudaStream_t s, int y_group = 0);
 // Rows of a bf16 matrix as fp16 swizzled tiles of nb rows x 64 columns (nb = 0: the B-tile height for `rows`).
 cudaError_t launch_pack_rows_tiles(const void* x, int rows, int K, void* tiles, cudaStream_t s, int nb = 0);
+cudaError_t launch_pack_rows_tiles_f32(const float* x, int rows, int K, void* tiles, cudaStream_t s);
+// Unfused output factors: B'_v,kv(h) per query head as 128 x 64 fp16 tiles [H][r_v / 64], and W_o^T
+// as tiles [Dp / 128][H d / 64] (built from the same inputs as M).
+cudaError_t launch_build_unfused(starkv_layer* L, const float* Bv_rot, const void* W_o, cudaStream_t s);
 size_t rows_tiles_bytes(int rows, int K);
 cudaError_t launch_outproj_tc(const starkv_layer* L, const void* y_tiles, int rows, void* out, float* part,
                               cudaStream_t s);

@@ -43,7 +43,7 @@ class _Config(ctypes.Structure):
                 ("top_fraction", ctypes.c_float), ("top_bits", ctypes.c_int), ("bottom_bits", ctypes.c_int),
                 ("group_size", ctypes.c_int), ("hadamard_block", ctypes.c_int), ("rope", ctypes.c_int),
                 ("rope_theta", ctypes.c_double), ("softmax_scale", ctypes.c_float), ("page_size", ctypes.c_int),
-                ("plain", ctypes.c_int), ("max_positions", ctypes.c_int)]
+                ("plain", ctypes.c_int), ("max_positions", ctypes.c_int), ("unfused_output", ctypes.c_int)]
 
 
 class _Info(ctypes.Structure):
@@ -137,6 +137,7 @@ class LayerConfig:
     page_size: int = 16
     plain: bool = False
     max_positions: int = 0
+    unfused_output: bool = False
 
     @classmethod
     def from_spec(cls, spec) -> "LayerConfig":
@@ -152,7 +153,8 @@ class LayerConfig:
                     ctypes.cast(ranks, ctypes.POINTER(ctypes.c_int)) if self.key_ranks else None, self.value_rank,
                     STARKV_F32 if self.dtype == "f32" else STARKV_BF16, int(self.quantized), self.top_fraction,
                     self.top_bits, self.bottom_bits, self.group_size, self.hadamard_block, int(self.rope),
-                    self.rope_theta, self.softmax_scale, self.page_size, int(self.plain), self.max_positions)
+                    self.rope_theta, self.softmax_scale, self.page_size, int(self.plain), self.max_positions,
+                    int(self.unfused_output))
         return c, ranks
 
 

@@ -96,6 +96,12 @@ typedef enum { STARKV_F32 = 0, STARKV_BF16 = 1 } starkv_dtype;
  *   max_positions: length of the layer's RoPE table for the tensor-core score
  *     kernel (0 selects 32768); 256 bytes of device memory per position.
  *     Decodes whose page table reaches beyond it use the CUDA-core path.
+ *   unfused_output: 0 (default) = value-side output fusion, out = sum_h y_h M_h
+ *     with M_h = B_v,h W_o,h folded at load (section 5.3); 1 = the same
+ *     product in the other order, z_h = y_h B_v,kv(h) then out = z W_o,
+ *     which reads H d (r_v + D) factor values per step instead of
+ *     H r_v D (section 5.3 states the fusion as an exact reorder).  Needs a
+ *     bf16 compressed layer with head_dim 128 and value_rank a multiple of 64.
  */
 typedef struct {
   int hidden, n_heads, n_kv_heads, head_dim;
@@ -113,6 +119,7 @@ typedef struct {
   int page_size;
   int plain;
   int max_positions;
+  int unfused_output;
 } starkv_layer_config;
 
 typedef struct starkv_layer starkv_layer;   /* opaque */
@@ -124,7 +131,7 @@ typedef struct {
   int key_rank_total;       /* R_k = sum of key ranks (plain: H_kv*d) */
   size_t page_bytes;        /* bytes of one 16-token page, a multiple of 128 */
   double bytes_per_token;   /* algorithmic cache bytes per token (codes + scales, no padding) */
-  size_t factor_bytes;      /* bytes decode reads from the layer's factors per step (B_k' + M) */
+  size_t factor_bytes;      /* bytes decode reads from the layer's factors per step (B_k' + M, or B_k' + B_v + W_o unfused) */
 } starkv_layer_info;
 
 /*

@@ -95,10 +95,11 @@ class Case:
         return O.decode(s, self.f, Zs, q, q_pos, seq_len, self.B_rot)
 
     # ---- library ---------------------------------------------------------
-    def load(self, dev="cuda"):
+    def load(self, dev="cuda", unfused_output=False):
         from decode_attention_rank_b200 import starkv as lib
         s = self.spec
         cfg = lib.LayerConfig.from_spec(s)
+        cfg.unfused_output = unfused_output
         dt = tdtype(s)
 
         def t(x):

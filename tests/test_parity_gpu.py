@@ -24,9 +24,10 @@ def case(cfg: int, quantized: bool = False, layer: int = 2) -> Case:
     return Case(spec, gen.LAYER_SEED[cfg], layer if cfg == 4 else 0)
 
 
-def run_decode(c: Case, lens, peaky=1.0, use_hidden=True, check_pool=True, q_pos=None, page_seed=0, path=0):
+def run_decode(c: Case, lens, peaky=1.0, use_hidden=True, check_pool=True, q_pos=None, page_seed=0, path=0,
+               unfused=False):
     """Fill a cache (latent mode), decode one query per sequence, compare with the oracle."""
-    L = c.load()
+    L = c.load(unfused_output=unfused)
     if path:
         L.set_decode_path(path)
     s = c.spec
@@ -335,6 +336,20 @@ def test_bounded_wait_expires_into_the_status_word():
              torch.from_numpy(q).cuda().float(), out, ws)
     assert L.sync_status() == 0
     check_close(out.double().cpu().numpy()[0], c.oracle_decode(c.stored(Z), q[0], 39, 40), "decode after timeout")
+
+
+@pytest.mark.parametrize("cfg,quant", [(2, False), (3, True), (1, False)])
+def test_unfused_value_output(cfg, quant):
+    """Output in the unfused order (y_h B'_v,kv(h), then W_o; "STAR-KV 阅读笔记" section 5.3 states the
+    fusion as an exact reorder) against the oracle, which uses W_o and the explicit values; GQA
+    (workload 3) and the CUDA-core decode path (workload 1, unquantized) included; and the fused
+    layer's output agrees within the tolerance."""
+    c = case(cfg, quantized=quant)
+    lens = [333, 64, 5]
+    a = run_decode(c, lens, use_hidden=False, check_pool=False, unfused=True)
+    run_decode(c, lens[:2], peaky=25.0, use_hidden=False, check_pool=False, unfused=True)
+    b = run_decode(c, lens, use_hidden=False, check_pool=False)
+    assert np.linalg.norm(a - b) <= 3e-3 * np.linalg.norm(b)
 
 
 def test_phase_timing_leaves_results_unchanged():
