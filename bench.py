@@ -677,6 +677,128 @@ def run_compare_plain(args):
             "points": rows, "hbm_peak": peak, "hbm_peak_kind": peak_kind, "clocks": clk}
 
 
+def _stack_layer(layer: int, max_positions: int):
+    """Layer `layer` of the 32-layer LongChat-7B-shaped stack: layers 0, 1 and 31 uncompressed (bf16 K/V),
+    the others 4/3-bit latents with block Hadamard and their own seeded ragged key ranks.  For timing only
+    the factors are seeded random bf16 tensors of the right shapes (the cost does not depend on their
+    values; parity is tested with the SVD factors elsewhere)."""
+    import torch
+    from decode_attention_rank_b200 import starkv as lib
+    from synth import gen
+    spec = gen.config_spec(4, layer=layer)
+    g = torch.Generator(device="cuda")
+    g.manual_seed(7000 + layer)
+    D, d, H, Hkv = spec.hidden, spec.head_dim, spec.n_heads, spec.n_kv_heads
+
+    def r(*shape, scale=1.0):
+        return (torch.randn(*shape, generator=g, device="cuda") * scale).to(torch.bfloat16)
+    cfg = lib.LayerConfig.from_spec(spec)
+    cfg.max_positions = max_positions
+    if spec.plain:
+        return spec, lib.load_factors(cfg, r(D, Hkv * d, scale=D ** -0.5), None, r(D, Hkv * d, scale=D ** -0.5),
+                                      None, r(H * d, D, scale=D ** -0.5))
+    Rk = sum(spec.key_ranks)
+    return spec, lib.load_factors(cfg, r(D * Rk, scale=D ** -0.5), r(Rk * d, scale=d ** -0.5),
+                                  r(D, spec.value_rank, scale=D ** -0.5), r(spec.value_rank, Hkv * d, scale=0.03),
+                                  r(H * d, D, scale=D ** -0.5))
+
+
+def _fill_random(L, B, T, g):
+    """Page table and pool of B sequences of T tokens, appended in latent mode from seeded normals."""
+    import torch
+    pages = (T + 15) // 16
+    n_pages = B * pages
+    pt = torch.randperm(n_pages, generator=g, device="cuda").to(torch.int32).reshape(B, pages).contiguous()
+    pool = torch.empty(n_pages * L.page_bytes, dtype=torch.uint8, device="cuda")
+    L.cache_init(pool, n_pages)
+    chunk = max(16, min(T, (1 << 26) // max(1, L.latent_total * 4)) // 16 * 16)
+    for b in range(B):
+        for c0 in range(0, T, chunk):
+            n = min(chunk, T - c0)
+            z = torch.randn(n, L.latent_total, generator=g, device="cuda") * 0.3
+            L.append(pool, n_pages, pt, torch.full((n,), b, dtype=torch.int32, device="cuda"),
+                     torch.arange(c0, c0 + n, dtype=torch.int32, device="cuda"), z, True)
+    return pool, n_pages, pt
+
+
+def run_stack(args):
+    """The 32-layer stack of the long-context workload: a causal chunked prefill of 4096 tokens (chunks of
+    1024, each appended before its attention) and a decode-step sweep over batch x context, the step time
+    being the sum over the 32 layers.  The layers are timed one at a time (each with its own cache, built,
+    timed and freed), since the whole stack's caches at batch 64 and 32K tokens (~175 GB) would not fit
+    beside the workspaces.  One JSON line."""
+    import torch
+    torch.cuda.set_device(0)
+    points = [tuple(int(x) for x in p.split("x")) for p in args.stack.split(",")]
+    g = torch.Generator(device="cuda")
+    g.manual_seed(31337)
+    clocks = ClockSampler(0)
+    clocks.start()
+    # prefill: batch 1, 4096 tokens in four chunks of 1024
+    pre_ms = [0.0] * 32
+    n_chunk, T_pre = 1024, 4096
+    for layer in range(32):
+        spec, L = _stack_layer(layer, 32768)
+        pages = T_pre // 16
+        pt = torch.randperm(pages, generator=g, device="cuda").to(torch.int32).reshape(1, pages).contiguous()
+        pool = torch.empty(pages * L.page_bytes, dtype=torch.uint8, device="cuda")
+        L.cache_init(pool, pages)
+        x = (torch.randn(T_pre, spec.hidden, generator=g, device="cuda")).to(torch.bfloat16)
+        q = (torch.randn(T_pre, spec.n_heads, spec.head_dim, generator=g, device="cuda") /
+             math.sqrt(spec.head_dim)).to(torch.bfloat16)
+        out = torch.empty(n_chunk, spec.hidden, dtype=torch.bfloat16, device="cuda")
+        ws = torch.empty(L.workspace_bytes(1, T_pre, n_chunk), dtype=torch.uint8, device="cuda")
+        wsa = torch.empty(max(256, L.append_workspace_bytes(n_chunk)), dtype=torch.uint8, device="cuda")
+        seq = torch.zeros(n_chunk, dtype=torch.int32, device="cuda")
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for c in range(T_pre // n_chunk):
+            pos = torch.arange(c * n_chunk, (c + 1) * n_chunk, dtype=torch.int32, device="cuda")
+            L.append(pool, pages, pt, seq, pos, x[c * n_chunk:(c + 1) * n_chunk], False, workspace=wsa)
+            L.prefill(pool, pages, pt, [c * n_chunk], [n_chunk], q[c * n_chunk:(c + 1) * n_chunk], out, ws)
+        e1.record()
+        torch.cuda.synchronize()
+        assert L.sync_status() == 0
+        pre_ms[layer] = e0.elapsed_time(e1)
+        del pool, ws, wsa, L
+        torch.cuda.empty_cache()
+    # decode sweep
+    sweep = []
+    for B, T in points:
+        per_layer = [0.0] * 32
+        for layer in range(32):
+            spec, L = _stack_layer(layer, max(T, 32768))
+            pool, n_pages, pt = _fill_random(L, B, T, g)
+            q = (torch.randn(B, spec.n_heads, spec.head_dim, generator=g, device="cuda") /
+                 math.sqrt(spec.head_dim)).to(torch.bfloat16)
+            out = torch.empty(B, spec.hidden, dtype=torch.bfloat16, device="cuda")
+            ws = torch.empty(L.workspace_bytes(B, pt.shape[1] * 16), dtype=torch.uint8, device="cuda")
+            lens = torch.full((B,), T, dtype=torch.int32, device="cuda")
+            per_layer[layer] = _time_decodes(L, pool, n_pages, pt, lens, q, out, ws, args.steps, args.warmup)
+            del pool, ws, L
+            torch.cuda.empty_cache()
+        step_ms = sum(per_layer)
+        sweep.append({"batch": B, "ctx": T, "step_ms": step_ms, "tokens_per_s": B / (step_ms * 1e-3),
+                      "plain_layer_ms": [per_layer[i] for i in (0, 1, 31)],
+                      "compressed_layer_ms_mean": sum(per_layer[2:31]) / 29,
+                      "compressed_layer_ms_min_max": [min(per_layer[2:31]), max(per_layer[2:31])]})
+    clk = clocks.stop()
+    return {"metric": "32-layer stack: chunked prefill time and decode tokens/s over batch x context", "mode": "stack",
+            "value": sweep[-1]["tokens_per_s"] if sweep else None, "unit": "tokens/s", "n_gpus": 1,
+            "steps": args.steps, "warmup": args.warmup, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "u3/u4 latent codes + fp16 scales (layers 2-30), bf16 K/V (0, 1, 31)",
+            "data": "synthetic (seeded random factors and latents; layers timed one at a time)",
+            "config": {"workload": "LongChat-7B-shaped 32-layer stack (attention only): layers 0, 1, 31 uncompressed, "
+                                   "2-30 4/3-bit latents with block Hadamard and per-layer ragged key ranks; prefill "
+                                   "4096 tokens in chunks of 1024, batch 1; decode sweep", "points": points},
+            "prefill": {"tokens": T_pre, "chunk": n_chunk, "total_ms": sum(pre_ms),
+                        "plain_layer_ms": [pre_ms[i] for i in (0, 1, 31)],
+                        "compressed_layer_ms_mean": sum(pre_ms[2:31]) / 29,
+                        "tokens_per_s": T_pre / (sum(pre_ms) * 1e-3)},
+            "sweep": sweep, "clocks": clk}
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -696,7 +818,12 @@ def main():
                     "32-layer stack instead (batch/ctx from --batch/--ctx, default 16 and 4096)")
     ap.add_argument("--compare-plain", default="", help="comma-separated contexts: time an uncompressed layer "
                     "against a 4/3-bit latent layer at each (batch from --batch, default 16); one JSON line")
+    ap.add_argument("--stack", default="", help="comma-separated BxT decode points for the 32-layer stack "
+                    "(e.g. 1x4096,16x32768); also times its 4096-token chunked prefill; one JSON line")
     args = ap.parse_args()
+    if args.stack:
+        print(json.dumps(run_stack(args)), flush=True)
+        return
     if args.compare_plain:
         print(json.dumps(run_compare_plain(args)), flush=True)
         return

@@ -19,7 +19,10 @@
 // walks a contiguous range of units ordered position-major, so its RoPE tiles
 // stay resident across the sequences of one position.
 //   warp 0      bulk copies of the key latent pages
-//   warp 1      tcgen05.mma issue (one thread), TMEM allocation
+//   warps 1, 19 tcgen05.mma issue (one thread each): warp 1 the first
+//               128-token tile of every item, warp 19 the second, so the
+//               MMAs are issued from two schedulers (one thread issues
+//               tcgen05.mma at best every ~50 cycles); warp 1 allocates TMEM
 //   warp 2      bulk copies of the RoPE table tiles and W'' item blocks
 //   warps 3-18  epilogue, two sets of 8 warps taking alternate MMA items; in
 //               a set, warp (tile, lane quarter) owns 32 tokens of one
@@ -40,7 +43,8 @@ namespace starkv {
 namespace {
 
 constexpr int kEpiWarps = 16;
-constexpr int kScoreThreads = 96 + 32 * kEpiWarps;   // key copies, MMA, W''/E copies, 16 epilogue warps
+constexpr int kScoreThreads = 128 + 32 * kEpiWarps;   // key copies, 2 MMA, W''/E copies, 16 epilogue warps
+constexpr int kMma2Warp = 3 + kEpiWarps;              // the second MMA warp
 constexpr int kSuper = 256;          // tokens per super-tile
 constexpr int kETileBytes = 32768;   // one 128-position RoPE tile (128 x 128 fp16)
 
@@ -306,17 +310,17 @@ __global__ void __launch_bounds__(kScoreThreads, 1) k_scores_tc(ScoreArgs a) {
   if (threadIdx.x == 0) {
     for (int s = 0; s < kMaxStages; ++s) {
       tc::mbar_init(&w_full[s], 1);
-      tc::mbar_init(&w_empty[s], 1);
+      tc::mbar_init(&w_empty[s], 2);   // both tiles' MMAs of the item
       tc::mbar_init(&k_full[s], 1);
       tc::mbar_init(&k_empty[s], kEpiWarps / 2);
     }
     tc::mbar_init(&e_full, 1);
-    tc::mbar_init(&e_empty, 1);
+    tc::mbar_init(&e_empty, 2);
     for (int s = 0; s < 4; ++s) {
       tc::mbar_init(&acc_full[s], 1);
       tc::mbar_init(&acc_free[s], 4);
     }
-    tc::mbar_init(&fin, 1);
+    tc::mbar_init(&fin, 2);
     abort_flag = 0;
     tc::fence_mbar_init();
   }
@@ -439,14 +443,20 @@ __global__ void __launch_bounds__(kScoreThreads, 1) k_scores_tc(ScoreArgs a) {
       if (ne > 0) tc::mbar_wait(&e_full, (uint32_t)(ne - 1) & 1u, a.status);
     }
     __syncwarp();
-  } else if (warp == 1) {
+  } else if (warp == 1 || warp == kMma2Warp) {
     // ------------------------------------------------------------ MMA issue
+    // warp 1 issues tile 0 and warp kMma2Warp tile 1 of every item: job
+    // j = 2 i + tile in accumulator stage j % 4.  Both wait for the item's
+    // W'' stage and release it (w_empty counts two commits); both release the
+    // RoPE tiles when the position changes.
+    const int tile = warp == 1 ? 0 : 1;
     if (lane == 0) {
       int i = 0, nc = 0, cur_st = -1, ws_n = 0;
       uint32_t wph_n = 0;
       int st_n = (int)(u0 / a.batch), b_n = (int)(u0 % a.batch);
       const uint64_t e0 = tc::sdesc_sw128(tc::smem_u32(E_s), 0, 1024), w0 = tc::sdesc_sw128(tc::smem_u32(W_s), 0, 1024);
-      const uint32_t e_lo0 = tc::desc_lo(e0), w_lo0 = tc::desc_lo(w0), sw_hi = tc::desc_hi(e0);
+      const uint32_t e_lo = tc::desc_lo(e0) + (uint32_t)tile * (kETileBytes >> 4), w_lo0 = tc::desc_lo(w0);
+      const uint32_t sw_hi = tc::desc_hi(e0);
       for (long long u = u0; u < u1 && !abort_flag; ++u) {
         const int st = st_n, b = b_n;
         if (++b_n == a.batch) {
@@ -476,27 +486,18 @@ __global__ void __launch_bounds__(kScoreThreads, 1) k_scores_tc(ScoreArgs a) {
           // descriptors as (low, high) halves, stepped in 16-byte units on the low half
           const uint32_t w_lo = w_lo0 + (uint32_t)ws * ((uint32_t)a.w_stage >> 4);
           const uint32_t watom = (uint32_t)npad * 8u;   // one 64-column K atom of W'': npad rows x 128 B
-          bool ok = true;
-          for (int k = 0; k < 2 && ok; ++k) {
-            // job j = 2 i + k: tile k of item i, accumulator stage j % 4
-            const int j = 2 * i + k;
-            if (!tc::mbar_wait_ab(&acc_free[j & 3], (((uint32_t)(j >> 2)) & 1u) ^ 1u, a.status, &abort_flag)) {
-              ok = false;
-              break;
-            }
-            tc::tc_fence_after();
-            const uint32_t e_lo = e_lo0 + (uint32_t)k * (kETileBytes >> 4);
-            const uint32_t d = tmem + (uint32_t)((j & 3) * 128);
-#pragma unroll
-            for (int kk = 0; kk < 8; ++kk)
-              tc::mma_f16_ss2(d, e_lo + (uint32_t)(kk >> 2) * 1024u + (uint32_t)(kk & 3) * 2u, sw_hi,
-                              w_lo + (uint32_t)(kk >> 2) * watom + (uint32_t)(kk & 3) * 2u, sw_hi, idesc, kk ? 1u : 0u);
-            tc::mma_commit(&acc_full[j & 3]);
-          }
-          if (!ok) {
+          const int j = 2 * i + tile;
+          if (!tc::mbar_wait_ab(&acc_free[j & 3], (((uint32_t)(j >> 2)) & 1u) ^ 1u, a.status, &abort_flag)) {
             abort_flag = 1;
             break;
           }
+          tc::tc_fence_after();
+          const uint32_t d = tmem + (uint32_t)((j & 3) * 128);
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk)
+            tc::mma_f16_ss2(d, e_lo + (uint32_t)(kk >> 2) * 1024u + (uint32_t)(kk & 3) * 2u, sw_hi,
+                            w_lo + (uint32_t)(kk >> 2) * watom + (uint32_t)(kk & 3) * 2u, sw_hi, idesc, kk ? 1u : 0u);
+          tc::mma_commit(&acc_full[j & 3]);
           tc::mma_commit(&w_empty[ws]);
         }
       }

@@ -19,8 +19,9 @@
 // are issued by four threads on the four schedulers: the 16 dequantizing
 // warps form four teams (one warp per TMEM lane quarter each), team j owns
 // the channel blocks j, j + 4, ... with their own ring of A slots in TMEM, and
-// one warp of the team issues the team's MMAs once the four have stored a
-// page.  Teams meet only at the shared page copies and P tiles.
+// the team's own MMA warp issues its MMAs once the four have stored a page,
+// while they go on to the next page.  Teams meet only at the shared page
+// copies and P tiles.
 //
 // P comes from the score kernel as exp2(s - m_g) per 32-token group; it is
 // rescaled by exp2(m_g - M) with M the maximum over the CTA's run of the
@@ -29,9 +30,10 @@
 //   warp 0      bulk copies of the pages' value blocks, TMEM allocation
 //   warps 1-4   P staging: rescaled fp16 P tiles (the B operand), M and l;
 //               warp s takes the 32-token group s of every 128-token tile
-//   warps 5-20  four teams of four workers: dequantize the team's channel
-//               groups of each page into its A slot, issue its MMAs (one
-//               warp per team), read its blocks of Y^T at the end of a run
+//   warps 5-8   MMA issue, one warp (lane 0) per team, on four schedulers
+//   warps 9-24  four teams of four workers: dequantize the team's channel
+//               groups of each page into its A slot, read its blocks of Y^T
+//               at the end of a run
 #include <float.h>
 
 #include "tc_common.cuh"
@@ -43,8 +45,9 @@ namespace {
 constexpr int kTeams = 4;                                // MMA-issuing teams, four warps each
 constexpr int kValWorkers = 4 * kTeams;                  // dequantizing warps
 constexpr int kStagers = 4;                              // P staging warps, one per 32-token group of a tile
-constexpr int kWorker0 = 1 + kStagers;                   // first worker warp
-constexpr int kValThreads = 32 * (kWorker0 + kValWorkers);   // page copies, P staging, workers
+constexpr int kIssuer0 = 1 + kStagers;                   // first MMA warp (one per team)
+constexpr int kWorker0 = kIssuer0 + kTeams;              // first worker warp
+constexpr int kValThreads = 32 * (kWorker0 + kValWorkers);   // page copies, P staging, MMA, workers
 constexpr int kMaxRawStages = 32;
 constexpr int kMaxASlots = 8;    // pages whose A tiles a team keeps in TMEM at once
 constexpr int kVSuper = 256;     // tokens per super-tile (matches the score kernel)
@@ -129,8 +132,8 @@ __device__ __forceinline__ void deq_channel3(uint64_t x, __half2 sub, const uint
 template <int NBT>
 __global__ void __launch_bounds__(kValThreads, 1) k_values_tc(ValArgs a) {
   extern __shared__ uint8_t smem_raw[];
-  __shared__ __align__(8) uint64_t t_free[kTeams][kMaxASlots], t_seg[kTeams], r_full[kMaxRawStages],
-      r_empty[kMaxRawStages];
+  __shared__ __align__(8) uint64_t t_full[kTeams][kMaxASlots], t_free[kTeams][kMaxASlots], t_seg[kTeams],
+      t_acc[kTeams], r_full[kMaxRawStages], r_empty[kMaxRawStages];
   __shared__ __align__(8) uint64_t p_full[2], p_empty[2];
   __shared__ uint32_t tmem_base;
   __shared__ volatile int abort_flag;
@@ -156,8 +159,12 @@ __global__ void __launch_bounds__(kValThreads, 1) k_values_tc(ValArgs a) {
 
   if (threadIdx.x == 0) {
     for (int t = 0; t < kTeams; ++t) {
-      for (int s = 0; s < a.na; ++s) tc::mbar_init(&t_free[t][s], 1);
+      for (int s = 0; s < a.na; ++s) {
+        tc::mbar_init(&t_full[t][s], 4);
+        tc::mbar_init(&t_free[t][s], 1);
+      }
       tc::mbar_init(&t_seg[t], 1);
+      tc::mbar_init(&t_acc[t], 4);
     }
     for (int s = 0; s < a.n_raw; ++s) {
       tc::mbar_init(&r_full[s], 1);
@@ -377,36 +384,87 @@ __global__ void __launch_bounds__(kValThreads, 1) k_values_tc(ValArgs a) {
       if (lane == 0) tc::mbar_arrive(&p_full[ps]);
     }
     if (cur_run >= 0) flush();
+  } else if (warp < kWorker0) {
+    // ------------------------------------------------ MMA issue, one warp per team
+    // Team j's page p sits in its A slot p % na: block j + 4 i's 128 x 16 A tile
+    // at TMEM column abase + (slot NBT + i) 8; its K = 16 MMA adds that block's
+    // Y^T (columns (j + 4 i) H ..).  At the end of a run the warp commits
+    // t_seg and waits for the team to have read Y^T (t_acc) before the next
+    // run's first MMA overwrites it.
+    const int j = warp - kIssuer0;
+    if (j < n_teams && lane == 0) {
+      const int nbt = min(NBT, (nblk - j + 3) / 4);
+      const uint32_t abase = ycols + (uint32_t)(j * a.na * NBT * 8);
+      const uint32_t idesc = tc::idesc_f16(128, a.H, false, false, false);
+      const uint64_t b0 = tc::sdesc_sw128(tc::smem_u32(P_s), 0, 1024);   // B: K-major, 64-token atoms of H rows
+      const uint32_t b_lo0 = tc::desc_lo(b0), b_hi = tc::desc_hi(b0);
+      const uint32_t b_atom = (uint32_t)(a.H * 128) >> 4, p_step = (uint32_t)p_stage >> 4;
+      int cur_run = -1, n_runs_done = 0, as = 0;
+      uint32_t aph = 0;
+      bool first = false;
+      for (int T = 0; T < n_tiles && !abort_flag; ++T) {
+        const int run = tile_s[T].w;
+        if (run != cur_run) {
+          if (cur_run >= 0) {
+            tc::mma_commit(&t_seg[j]);
+            if (!tc::mbar_wait_ab(&t_acc[j], (uint32_t)n_runs_done & 1u, a.status, &abort_flag)) break;
+            ++n_runs_done;
+            tc::tc_fence_after();
+          }
+          cur_run = run;
+          first = true;
+        }
+        const int ps = T & 1;
+        if (!tc::mbar_wait_ab(&p_full[ps], ((uint32_t)(T >> 1)) & 1u, a.status, &abort_flag)) break;
+        tc::tc_fence_after();
+        const uint32_t b_lo = b_lo0 + (uint32_t)ps * p_step;
+        bool ok = true;
+        for (int k = 0; k < 8; ++k) {
+          if (!tc::mbar_wait_ab(&t_full[j][as], aph, a.status, &abort_flag)) {
+            ok = false;
+            break;
+          }
+          tc::tc_fence_after();
+          const uint32_t acol = tmem + abase + (uint32_t)(as * NBT * 8);
+          const uint32_t bk = b_lo + (uint32_t)(k >> 2) * b_atom + (uint32_t)(k & 3) * 2u;
+          const uint32_t acc = (first && k == 0) ? 0u : 1u;
+#pragma unroll
+          for (int i = 0; i < NBT; ++i) {
+            if (i >= nbt) break;
+            tc::mma_f16_ts(tmem + (uint32_t)((j + 4 * i) * a.H), acol + (uint32_t)i * 8u, bk, b_hi, idesc, acc);
+          }
+          tc::mma_commit(&t_free[j][as]);
+          if (++as == a.na) {
+            as = 0;
+            aph ^= 1u;
+          }
+        }
+        if (!ok) break;
+        tc::mma_commit(&p_empty[ps]);
+        first = false;
+      }
+      if (cur_run >= 0) tc::mma_commit(&t_seg[j]);
+      // every MMA of this thread has completed before the CTA may exit
+      tc::mma_commit(&t_free[j][as]);
+      tc::mbar_wait(&t_free[j][as], aph, a.status);
+    }
   } else {
     // ------------------------------------------------ worker teams
     // A warp may address only its TMEM lane quarter q = warp % 4, i.e. the
     // channels 32 q .. 32 q + 31 of every 128-channel block: channel group
     // 4 cb + q of block cb, lane = channel inside the group.  Team j = the
-    // four consecutive workers (one per quarter) owning blocks j + 4 i; its
-    // MMAs are issued by lane 0 of its warp with q == j, so that the four
-    // teams issue from the four schedulers.
+    // four consecutive workers (one per quarter) owning blocks j + 4 i.
     const int wid = warp - kWorker0;
     const int q = warp & 3, j = wid >> 2;
-    if (j >= n_teams) {
-      // a team without channel blocks (fewer than four blocks): nothing to do
-    } else {
-      const bool issuer = (q == j);
+    if (j < n_teams) {
       const uint32_t lane_base = (uint32_t)(q * 32) << 16;
       const uint32_t abase = ycols + (uint32_t)(j * a.na * NBT * 8);   // this team's A ring
       const int nbt = min(NBT, (nblk - j + 3) / 4);                    // blocks of this team
       const int n_pg = n_tiles * 8;
-      const uint32_t bar_id = 2u + (uint32_t)j;
-      const uint32_t idesc = tc::idesc_f16(128, a.H, false, false, false);
-      const uint64_t b0 = tc::sdesc_sw128(tc::smem_u32(P_s), 0, 1024);   // B: K-major, 64-token atoms of H rows
-      const uint32_t b_lo0 = tc::desc_lo(b0), b_hi = tc::desc_hi(b0);
-      const uint32_t b_atom = (uint32_t)(a.H * 128) >> 4, p_step = (uint32_t)p_stage >> 4;
       int cur_run = -1, n_epi = 0, as = 0;
       uint32_t aph = 0;
-      bool first = false;
-      auto team_sync = [&]() { asm volatile("bar.sync %0, 128;" ::"r"(bar_id) : "memory"); };
       auto epilogue = [&](int r) {
         // Y^T of this team's blocks for run r (lanes = value channels), 16 columns at a time
-        if (issuer && lane == 0) tc::mma_commit(&t_seg[j]);
         const bool ok = tc::mbar_wait_ab(&t_seg[j], (uint32_t)n_epi & 1u, a.status, &abort_flag);
         ++n_epi;
         tc::tc_fence_after();
@@ -429,7 +487,8 @@ __global__ void __launch_bounds__(kValThreads, 1) k_values_tc(ValArgs a) {
           }
         }
         tc::tc_fence_before();
-        team_sync();   // every quarter has read before the issuer overwrites D
+        __syncwarp();
+        if (lane == 0) tc::mbar_arrive(&t_acc[j]);   // the MMA warp may overwrite Y^T
       };
       for (int p = 0; p < n_pg; ++p) {
         const int T = p >> 3, k = p & 7;
@@ -437,7 +496,6 @@ __global__ void __launch_bounds__(kValThreads, 1) k_values_tc(ValArgs a) {
         if (run != cur_run) {
           if (cur_run >= 0) epilogue(cur_run);
           cur_run = run;
-          first = true;
         }
         const int cur_as = as;
         const uint32_t cur_aph = aph;
@@ -484,30 +542,10 @@ __global__ void __launch_bounds__(kValThreads, 1) k_values_tc(ValArgs a) {
         tc::tmem_st_wait();
         tc::tc_fence_before();
         __syncwarp();
-        if (lane == 0) tc::mbar_arrive(&r_empty[rs]);
-        team_sync();   // the four quarters of the page's A tiles are in TMEM
-        if (issuer && lane == 0) {
-          tc::tc_fence_after();
-          const int ps = T & 1;
-          bool okp = true;
-          if (k == 0) {
-            okp = tc::mbar_wait_ab(&p_full[ps], ((uint32_t)(T >> 1)) & 1u, a.status, &abort_flag);
-            tc::tc_fence_after();
-          }
-          if (okp) {
-            const uint32_t bk = b_lo0 + (uint32_t)ps * p_step + (uint32_t)(k >> 2) * b_atom + (uint32_t)(k & 3) * 2u;
-            const uint32_t acc = (first && k == 0) ? 0u : 1u;
-#pragma unroll
-            for (int i = 0; i < NBT; ++i) {
-              if (i >= nbt) break;
-              tc::mma_f16_ts(tmem + (uint32_t)((j + 4 * i) * a.H), tmem + slot_col + (uint32_t)i * 8u, bk, b_hi,
-                             idesc, acc);
-            }
-          }
-          tc::mma_commit(&t_free[j][cur_as]);
-          if (k == 7) tc::mma_commit(&p_empty[ps]);
+        if (lane == 0) {
+          tc::mbar_arrive(&t_full[j][cur_as]);
+          tc::mbar_arrive(&r_empty[rs]);
         }
-        if (k == 7) first = false;
       }
       if (cur_run >= 0) epilogue(cur_run);
     }
