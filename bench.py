@@ -30,7 +30,25 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 METRIC = "latent decode-attn tokens/s & HBM GB/s (% of ~8 TB/s) at ctx 4K-32K, 1 B200"
-WORKLOAD = dict(cfg=2, batch=16, ctx=32768)
+WORKLOAD = dict(cfg=2, batch=16, ctx=32768, quantized=None)
+
+
+def workload_spec():
+    from synth import gen
+    return gen.config_spec(WORKLOAD["cfg"], quantized=WORKLOAD["quantized"])
+
+
+def workload_label(spec, B, ctx):
+    """What the timed step is, in words (shapes of the layer)."""
+    if spec.quantized:
+        store = (f"block Hadamard {spec.hadamard_block}, " if spec.hadamard_block else "") + \
+            f"{spec.top_bits}/{spec.bottom_bits}-bit latents"
+    else:
+        store = "bf16 latents"
+    shape = f"H {spec.n_heads}" + (f"/{spec.n_kv_heads} KV" if spec.n_kv_heads != spec.n_heads else "") + \
+        f", d {spec.head_dim}, D {spec.hidden}, R_k {sum(spec.key_ranks)}, r_v {spec.value_rank}, RoPE {spec.rope_theta:g}"
+    name = {1: "LongChat-7B-shaped", 2: "LongChat-7B-shaped", 3: "LLaMA-3-8B-shaped GQA"}.get(WORKLOAD["cfg"], "")
+    return f"batch {B}, ctx ~{ctx} ({name} layer: {shape}, {store}, 16-token pages)"
 
 
 def measured_peaks():
@@ -154,7 +172,7 @@ def build_layer(seed_offset: int = 0, unfused: bool = False, max_positions: int 
     import torch
     from decode_attention_rank_b200 import starkv as lib
     from synth import gen
-    spec = gen.config_spec(WORKLOAD["cfg"])
+    spec = workload_spec()
     f = gen.make_factors(spec, gen.LAYER_SEED[WORKLOAD["cfg"]])
 
     def t(x):
@@ -274,26 +292,29 @@ def decode_bytes(spec, L, B, ctx):
     return B * ctx * L.bytes_per_token + L.factor_bytes + B * (spec.n_heads * spec.head_dim + spec.hidden) * 2
 
 
-def cpu_baseline(sample_T: int):
-    """Time the float64 oracle on one sequence of the workload (host cores)."""
-    import numpy as np
+def _oracle_case(T: int):
+    """Seeded inputs of one sequence of the workload, and the C++ float64 oracle's decode of it."""
     sys.path.insert(0, os.path.join(ROOT, "tests"))
     from harness import Case, queries
+    from oracle import cpp as C
     from synth import gen
-    c = Case(gen.config_spec(WORKLOAD["cfg"]), gen.LAYER_SEED[WORKLOAD["cfg"]])
-    Z = c.latents_direct(0, sample_T)
-    Zs = c.stored(Z)
+    c = Case(workload_spec(), gen.LAYER_SEED[WORKLOAD["cfg"]])
+    Zs = c.stored(c.latents_direct(0, T))
     q = queries(c, 1)[0, 0]
-    c.B_rot
+    B_rot = C.up_projections(c.spec, c.f)
+    threads = len(os.sched_getaffinity(0))
+
+    def run():
+        C.decode(c.spec, c.f, Zs, q, T - 1, T, B_rot, threads=threads)
+    return run, min(threads, c.spec.n_heads)
+
+
+def cpu_baseline(sample_T: int):
+    """Time the float64 C++ oracle on one sequence of the workload (host cores, one thread per head)."""
+    run, cores = _oracle_case(sample_T)
     t0 = time.perf_counter()
-    c.oracle_decode(Zs, q, sample_T - 1, sample_T)
-    dt = time.perf_counter() - t0
-    try:
-        from threadpoolctl import threadpool_info
-        cores = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
-    except Exception:
-        cores = os.cpu_count()
-    return dt, cores
+    run()
+    return time.perf_counter() - t0, cores
 
 
 def run_ours(args, rank, ws, local):
@@ -416,12 +437,11 @@ def run_ours(args, rank, ws, local):
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
-        "dtype": "u3/u4 latent codes + fp16 scales, bf16 factors/q/out, fp32 accumulate",
+        "dtype": ("u3/u4 latent codes + fp16 scales, bf16 factors/q/out, fp32 accumulate" if spec.quantized
+                  else "bf16 latents/factors/q/out, fp32 accumulate"),
         "data": "synthetic (seeded latents with the factor spectrum; random-init factors)",
-        "config": {"workload": f"STAR-KV decode step: append 1 token/seq + decode, batch {B}, ctx ~{ctx} "
-                               f"(LongChat-7B-shaped layer: H 32, d 128, D 4096, R_k 1024, r_v 1024, "
-                               f"block Hadamard 32, 4/3-bit latents, 16-token pages"
-                               + (", unfused value output y_h B_v,h then W_o)" if args.unfused else ")"),
+        "config": {"workload": "STAR-KV decode step: append 1 token/seq + decode, " + workload_label(spec, B, ctx)
+                               + (", unfused value output y_h B_v,h then W_o" if args.unfused else ""),
                    "batch": B, "ctx": ctx, "ctx_range": [T0 + W + 1, T0 + W + K], "parallelism": f"replicas x{ws}",
                    "l2": "inputs larger than L2 (cache %.0f MB + M %.0f MB)" % (B * ctx * L.bytes_per_token / 1e6,
                                                                             L.factor_bytes / 1e6)},
@@ -448,7 +468,7 @@ def run_ours(args, rank, ws, local):
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:
         dt, cores = cpu_baseline(ctx)
         res["cpu_baseline"] = {"value": 1.0 / dt, "unit": "tokens/s", "cores": cores, "kind": "oracle",
-                               "sample": f"1 sequence of the batch at ctx {ctx}: float64 explicit K/V "
+                               "sample": f"1 sequence of the batch at ctx {ctx}: float64 C++ oracle, explicit K/V "
                                          f"reconstruction + softmax attention + W_o ({dt:.1f} s)"}
     return res
 
@@ -459,25 +479,14 @@ def run_reference(args, rank, ws):
         return None
     B, ctx = WORKLOAD["batch"], WORKLOAD["ctx"]
     K, W = args.steps, args.warmup
-    sys.path.insert(0, os.path.join(ROOT, "tests"))
-    from harness import Case, queries
-    from synth import gen
     T = args.ref_ctx or ctx
-    c = Case(gen.config_spec(WORKLOAD["cfg"]), gen.LAYER_SEED[WORKLOAD["cfg"]])
-    c.B_rot
-    Zs = c.stored(c.latents_direct(0, T))
-    q = queries(c, 1)[0, 0]
+    run, cores = _oracle_case(T)
     for _ in range(W):
-        c.oracle_decode(Zs, q, T - 1, T)
+        run()
     t0 = time.perf_counter()
     for _ in range(K):
-        c.oracle_decode(Zs, q, T - 1, T)
+        run()
     dt = (time.perf_counter() - t0) / K
-    try:
-        from threadpoolctl import threadpool_info
-        cores = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
-    except Exception:
-        cores = os.cpu_count()
     v = 1.0 / dt
     return {"metric": METRIC, "value": v, "unit": "tokens/s", "n_gpus": ws, "steps": K, "warmup": W,
             "ms_per_step": dt * 1e3, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
@@ -812,6 +821,9 @@ def main():
     ap.add_argument("--batch", type=int, default=0, help="sequences per step (default 16)")
     ap.add_argument("--prefill", type=int, default=0, help="time a causal prefill chunk of this many queries "
                     "(history = ctx - queries, ctx default 4096) instead of the decode step")
+    ap.add_argument("--cfg", type=int, default=0, help="time the decode step of workload 1, 2 or 3 at its own "
+                    "batch and context (default: workload 2, the headline)")
+    ap.add_argument("--quantized", action="store_true", help="with --cfg 3: the 4/3-bit variant")
     ap.add_argument("--unfused", action="store_true", help="the workload with the unfused value output "
                     "(y_h B_v,h then W_o) instead of the fused M_h (separate line; the fused form is the headline)")
     ap.add_argument("--plain", action="store_true", help="time the decode of an uncompressed layer of the "
@@ -830,6 +842,13 @@ def main():
     if args.plain:
         print(json.dumps(run_plain(args)), flush=True)
         return
+    if args.cfg:
+        from synth import gen
+        assert args.cfg in (1, 2, 3), "--cfg takes 1, 2 or 3"
+        WORKLOAD["cfg"] = args.cfg
+        WORKLOAD["batch"] = gen.CONFIG_SHAPES[args.cfg]["batch"]
+        WORKLOAD["ctx"] = gen.CONFIG_SHAPES[args.cfg]["ctx"]
+        WORKLOAD["quantized"] = bool(args.quantized) if args.cfg == 3 else None
     if args.ctx:
         WORKLOAD["ctx"] = args.ctx
     if args.batch:

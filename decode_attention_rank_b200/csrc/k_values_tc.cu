@@ -49,7 +49,7 @@ constexpr int kIssuer0 = 1 + kStagers;                   // first MMA warp (one 
 constexpr int kWorker0 = kIssuer0 + kTeams;              // first worker warp
 constexpr int kValThreads = 32 * (kWorker0 + kValWorkers);   // page copies, P staging, MMA, workers
 constexpr int kMaxRawStages = 32;
-constexpr int kMaxASlots = 8;    // pages whose A tiles a team keeps in TMEM at once
+constexpr int kMaxASlots = 8;    // A slots (two pages each) a team keeps in TMEM at once
 constexpr int kVSuper = 256;     // tokens per super-tile (matches the score kernel)
 constexpr int kMaxRuns = 64;     // runs (sequences) per CTA
 constexpr int kRunMaxCache = 16; // runs whose per-head maxima are computed up front
@@ -386,15 +386,15 @@ __global__ void __launch_bounds__(kValThreads, 1) k_values_tc(ValArgs a) {
     if (cur_run >= 0) flush();
   } else if (warp < kWorker0) {
     // ------------------------------------------------ MMA issue, one warp per team
-    // Team j's page p sits in its A slot p % na: block j + 4 i's 128 x 16 A tile
-    // at TMEM column abase + (slot NBT + i) 8; its K = 16 MMA adds that block's
-    // Y^T (columns (j + 4 i) H ..).  At the end of a run the warp commits
-    // t_seg and waits for the team to have read Y^T (t_acc) before the next
-    // run's first MMA overwrites it.
+    // Team j's pages 2 m and 2 m + 1 sit in its A slot m % na: block j + 4 i's
+    // 128 x 16 A tile of page e at TMEM column abase + (slot NBT + i) 16 + 8 e;
+    // its K = 16 MMA adds that block's Y^T (columns (j + 4 i) H ..).  At the
+    // end of a run the warp commits t_seg and waits for the team to have read
+    // Y^T (t_acc) before the next run's first MMA overwrites it.
     const int j = warp - kIssuer0;
     if (j < n_teams && lane == 0) {
       const int nbt = min(NBT, (nblk - j + 3) / 4);
-      const uint32_t abase = ycols + (uint32_t)(j * a.na * NBT * 8);
+      const uint32_t abase = ycols + (uint32_t)(j * a.na * NBT * 16);
       const uint32_t idesc = tc::idesc_f16(128, a.H, false, false, false);
       const uint64_t b0 = tc::sdesc_sw128(tc::smem_u32(P_s), 0, 1024);   // B: K-major, 64-token atoms of H rows
       const uint32_t b_lo0 = tc::desc_lo(b0), b_hi = tc::desc_hi(b0);
@@ -419,19 +419,21 @@ __global__ void __launch_bounds__(kValThreads, 1) k_values_tc(ValArgs a) {
         tc::tc_fence_after();
         const uint32_t b_lo = b_lo0 + (uint32_t)ps * p_step;
         bool ok = true;
-        for (int k = 0; k < 8; ++k) {
+        for (int k = 0; k < 8; k += 2) {
           if (!tc::mbar_wait_ab(&t_full[j][as], aph, a.status, &abort_flag)) {
             ok = false;
             break;
           }
           tc::tc_fence_after();
-          const uint32_t acol = tmem + abase + (uint32_t)(as * NBT * 8);
-          const uint32_t bk = b_lo + (uint32_t)(k >> 2) * b_atom + (uint32_t)(k & 3) * 2u;
+          const uint32_t acol = tmem + abase + (uint32_t)(as * NBT * 16);
+          const uint32_t bk = b_lo + (uint32_t)(k >> 2) * b_atom + (uint32_t)(k & 3) * 2u;   // pages k, k + 1: K steps
           const uint32_t acc = (first && k == 0) ? 0u : 1u;
 #pragma unroll
           for (int i = 0; i < NBT; ++i) {
             if (i >= nbt) break;
-            tc::mma_f16_ts(tmem + (uint32_t)((j + 4 * i) * a.H), acol + (uint32_t)i * 8u, bk, b_hi, idesc, acc);
+            const uint32_t dcol = tmem + (uint32_t)((j + 4 * i) * a.H);
+            tc::mma_f16_ts(dcol, acol + (uint32_t)i * 16u, bk, b_hi, idesc, acc);
+            tc::mma_f16_ts(dcol, acol + (uint32_t)i * 16u + 8u, bk + 2u, b_hi, idesc, 1u);
           }
           tc::mma_commit(&t_free[j][as]);
           if (++as == a.na) {
@@ -458,7 +460,7 @@ __global__ void __launch_bounds__(kValThreads, 1) k_values_tc(ValArgs a) {
     const int q = warp & 3, j = wid >> 2;
     if (j < n_teams) {
       const uint32_t lane_base = (uint32_t)(q * 32) << 16;
-      const uint32_t abase = ycols + (uint32_t)(j * a.na * NBT * 8);   // this team's A ring
+      const uint32_t abase = ycols + (uint32_t)(j * a.na * NBT * 16);   // this team's A ring (slots of two pages)
       const int nbt = min(NBT, (nblk - j + 3) / 4);                    // blocks of this team
       const int n_pg = n_tiles * 8;
       int cur_run = -1, n_epi = 0, as = 0;
@@ -490,7 +492,8 @@ __global__ void __launch_bounds__(kValThreads, 1) k_values_tc(ValArgs a) {
         __syncwarp();
         if (lane == 0) tc::mbar_arrive(&t_acc[j]);   // the MMA warp may overwrite Y^T
       };
-      for (int p = 0; p < n_pg; ++p) {
+      for (int p = 0; p < n_pg; p += 2) {
+        // pages p and p + 1 (same tile, same run) go into one A slot
         const int T = p >> 3, k = p & 7;
         const int run = tile_s[T].w;
         if (run != cur_run) {
@@ -503,40 +506,45 @@ __global__ void __launch_bounds__(kValThreads, 1) k_values_tc(ValArgs a) {
           as = 0;
           aph ^= 1u;
         }
-        const uint32_t rsp = rsp_s[p];
-        const int rs = (int)(rsp & 127u);
-        const bool valid = pid_s[T][k] >= 0;
-        const uint32_t slot_col = abase + (uint32_t)(cur_as * NBT * 8);
+        const uint32_t rsp0 = rsp_s[p], rsp1 = rsp_s[p + 1];
+        const int rs0 = (int)(rsp0 & 127u), rs1 = (int)(rsp1 & 127u);
+        const bool valid0 = pid_s[T][k] >= 0, valid1 = pid_s[T][k + 1] >= 0;
+        const uint32_t slot_col = abase + (uint32_t)(cur_as * NBT * 16);
         const bool ok = tc::mbar_wait_ab(&t_free[j][cur_as], cur_aph ^ 1u, a.status, &abort_flag) &&
-                        tc::mbar_wait_ab(&r_full[rs], rsp >> 7, a.status, &abort_flag);
+                        tc::mbar_wait_ab(&r_full[rs0], rsp0 >> 7, a.status, &abort_flag) &&
+                        tc::mbar_wait_ab(&r_full[rs1], rsp1 >> 7, a.status, &abort_flag);
         if (ok) {
-          const uint8_t* blk = R_s + (size_t)rs * a.raw_stage;
 #pragma unroll
           for (int i = 0; i < NBT; ++i) {
             if (i >= nbt) break;
             const int g = (j + 4 * i) * 4 + q;
             const int4 vg = vg_s[g];
             const __half2 sub = *reinterpret_cast<const __half2*>(&vg.z);
-            uint32_t sc[8], out[8];
-            if (valid) {
-              const uint4 s0 = *reinterpret_cast<const uint4*>(blk + g * 32);
-              const uint4 s1 = *reinterpret_cast<const uint4*>(blk + g * 32 + 16);
-              sc[0] = s0.x; sc[1] = s0.y; sc[2] = s0.z; sc[3] = s0.w;
-              sc[4] = s1.x; sc[5] = s1.y; sc[6] = s1.z; sc[7] = s1.w;
-            } else {
 #pragma unroll
-              for (int x = 0; x < 8; ++x) sc[x] = 0u;
+            for (int e = 0; e < 2; ++e) {
+              const uint8_t* blk = R_s + (size_t)(e ? rs1 : rs0) * a.raw_stage;
+              const bool valid = e ? valid1 : valid0;
+              uint32_t sc[8], out[8];
+              if (valid) {
+                const uint4 s0 = *reinterpret_cast<const uint4*>(blk + g * 32);
+                const uint4 s1 = *reinterpret_cast<const uint4*>(blk + g * 32 + 16);
+                sc[0] = s0.x; sc[1] = s0.y; sc[2] = s0.z; sc[3] = s0.w;
+                sc[4] = s1.x; sc[5] = s1.y; sc[6] = s1.z; sc[7] = s1.w;
+              } else {
+#pragma unroll
+                for (int x = 0; x < 8; ++x) sc[x] = 0u;
+              }
+              if (vg.x == 4) {
+                const uint2 cw = *reinterpret_cast<const uint2*>(blk + vg.y + lane * 8);
+                deq_channel4(cw.x, cw.y, sub, sc, out);
+              } else {
+                const int bit = 48 * lane;
+                const uint32_t* cw = reinterpret_cast<const uint32_t*>(blk + vg.y) + (bit >> 5);
+                const uint64_t x = ((uint64_t)cw[1] << 32 | cw[0]) >> (bit & 31);
+                deq_channel3(x, sub, sc, out);
+              }
+              tc::tmem_st8(tmem + lane_base + slot_col + (uint32_t)(i * 16 + e * 8), out);
             }
-            if (vg.x == 4) {
-              const uint2 cw = *reinterpret_cast<const uint2*>(blk + vg.y + lane * 8);
-              deq_channel4(cw.x, cw.y, sub, sc, out);
-            } else {
-              const int bit = 48 * lane;
-              const uint32_t* cw = reinterpret_cast<const uint32_t*>(blk + vg.y) + (bit >> 5);
-              const uint64_t x = ((uint64_t)cw[1] << 32 | cw[0]) >> (bit & 31);
-              deq_channel3(x, sub, sc, out);
-            }
-            tc::tmem_st8(tmem + lane_base + slot_col + (uint32_t)i * 8u, out);
           }
         }
         tc::tmem_st_wait();
@@ -544,7 +552,8 @@ __global__ void __launch_bounds__(kValThreads, 1) k_values_tc(ValArgs a) {
         __syncwarp();
         if (lane == 0) {
           tc::mbar_arrive(&t_full[j][cur_as]);
-          tc::mbar_arrive(&r_empty[rs]);
+          tc::mbar_arrive(&r_empty[rs0]);
+          tc::mbar_arrive(&r_empty[rs1]);
         }
       }
       if (cur_run >= 0) epilogue(cur_run);
@@ -693,7 +702,7 @@ bool plan_values_tc(starkv_layer* L) {
   const int nblk = v.rv / 128;
   if (nblk > 2 * kTeams) return false;
   const int nbt = nblk > kTeams ? 2 : 1, n_teams = std::min(kTeams, nblk);
-  L->val_na = std::min(kMaxASlots, (512 - nblk * v.H) / (n_teams * nbt * 8));
+  L->val_na = std::min(kMaxASlots, (512 - nblk * v.H) / (n_teams * nbt * 16));   // slots of two pages
   if (L->val_na < 2) return false;
   const LatentDesc& ld = L->lat[v.L - 1];
   if (ld.n_groups * 32 != v.rv || !ld.cmajor) return false;
