@@ -104,7 +104,7 @@ static starkv_status plan_layer(starkv_layer* L) {
     ld.block_off = (int)off;
     ld.ch_off = ch;
     ld.group0 = (int)L->grp.size();
-    ld.cmajor = (quant && li + 1 == widths.size()) ? 1 : 0;
+    ld.cmajor = (!c.plain && li + 1 == widths.size()) ? 1 : 0;
     if (!quant) {
       L->grp.push_back(GroupDesc{0, ld.width, 0, 0});
       ld.n_groups = 1;
@@ -274,14 +274,15 @@ starkv_status starkv_load_factors(const starkv_layer_config* cfg, const void* A_
       cudaMalloc(&L->A_T, es * (size_t)v.Ltot * D) != cudaSuccess)
     return fail(STARKV_ERR_OOM, "cudaMalloc");
   const size_t wo_tiles_bytes = (size_t)(L->Dp / 128) * (H * d / 64) * 16384;
-  if (L->unfused) {
-    if (cudaMalloc(&L->Bv_tiles, (size_t)H * (v.rv / 64) * 16384) != cudaSuccess ||
-        cudaMalloc(&L->Wo_tiles, wo_tiles_bytes) != cudaSuccess)
-      return fail(STARKV_ERR_OOM, "cudaMalloc");
-  } else if (cudaMalloc(&L->M_T, cfg->dtype == STARKV_F32 ? 4 * (size_t)D * H * v.wv : 2 * (size_t)L->Dp * L->Kp) !=
-             cudaSuccess) {
+  // B'_v per head and W_o as tiles: the unfused output's factors, and the
+  // prefill's value reconstruction and output (bf16 compressed layers)
+  const bool bv_wo = L->unfused || (cfg->dtype == STARKV_BF16 && !cfg->plain && d == 128 && v.rv % 64 == 0);
+  if (bv_wo && (cudaMalloc(&L->Bv_tiles, (size_t)H * (v.rv / 64) * 16384) != cudaSuccess ||
+                cudaMalloc(&L->Wo_tiles, wo_tiles_bytes) != cudaSuccess))
     return fail(STARKV_ERR_OOM, "cudaMalloc");
-  }
+  if (!L->unfused &&
+      cudaMalloc(&L->M_T, cfg->dtype == STARKV_F32 ? 4 * (size_t)D * H * v.wv : 2 * (size_t)L->Dp * L->Kp) != cudaSuccess)
+    return fail(STARKV_ERR_OOM, "cudaMalloc");
   if (!cfg->plain && cudaMalloc(&L->Bk, sizeof(float) * (size_t)v.Rk * d) != cudaSuccess)
     return fail(STARKV_ERR_OOM, "cudaMalloc");
   v.lat = L->d_lat;
@@ -342,6 +343,7 @@ starkv_status starkv_load_factors(const starkv_layer_config* cfg, const void* A_
     }
   }
   cudaError_t e = L->unfused ? launch_build_unfused(L, Bv_rot, W_o, s) : launch_fold_M(L, Bv_rot, W_o, s);
+  if (e == cudaSuccess && !L->unfused && L->Bv_tiles) e = launch_build_unfused(L, Bv_rot, W_o, s);
   if (Bv_rot) {
     cudaStreamSynchronize(s);
     cudaFree(Bv_rot);
@@ -480,6 +482,7 @@ size_t starkv_workspace_bytes(const starkv_layer* L, int batch, int max_ctx, int
                               decode_generic_ws_bytes(L, (int)rows, max_ctx, true));
     if (L->tc_scores && L->tc_values)
       need = std::max(need, prefill_tc_ws_bytes(L, rows, (max_ctx + kPage - 1) / kPage));
+    if (prefill_flash_supported(L)) need = std::max(need, prefill_flash_ws_bytes(L, max_ctx, max_q));
   }
   return need;
 }
@@ -536,6 +539,28 @@ starkv_status starkv_prefill_attn(const starkv_layer* L, const void* pool, int64
     max_len = std::max(max_len, q_start_host[b] + q_len_host[b]);
   }
   if (rows == 0) return STARKV_OK;
+  cudaStream_t s = (cudaStream_t)stream;
+  // Tensor-core prefill: per sequence, keys and values rebuilt once for the
+  // chunk, then tiled causal attention and the output through W_o.
+  {
+    int max_q = 0;
+    for (int b = 0; b < batch; ++b) max_q = std::max(max_q, q_len_host[b]);
+    const bool flash = prefill_flash_supported(L) && L->decode_path == 0 &&
+                       (L->view.plain || max_len <= L->rope_tiles * 128) && workspace != nullptr &&
+                       ws_bytes >= prefill_flash_ws_bytes(L, max_len, max_q);
+    if (flash) {
+      const size_t qrow = (size_t)L->view.H * L->cfg.head_dim * sizeof(uint16_t);
+      const size_t orow = (size_t)L->view.D * (L->cfg.dtype == STARKV_F32 ? 4 : 2);
+      long long r0 = 0;
+      for (int b = 0; b < batch; ++b) {
+        CUDA_TRY(launch_prefill_flash(L, (const uint8_t*)pool, n_pages, page_table + (size_t)b * max_pages,
+                                      q_start_host[b], q_len_host[b], (const char*)q + r0 * qrow,
+                                      (char*)out + r0 * orow, workspace, max_len, max_q, s));
+        r0 += q_len_host[b];
+      }
+      return STARKV_OK;
+    }
+  }
   tab.resize(3 * (size_t)rows);
   int r = 0;
   for (int b = 0; b < batch; ++b)
@@ -545,7 +570,6 @@ starkv_status starkv_prefill_attn(const starkv_layer* L, const void* pool, int64
       tab[2 * rows + r] = q_start_host[b] + i;   // RoPE position
     }
   const size_t tab_bytes = ru(sizeof(int32_t) * tab.size(), 256);
-  cudaStream_t s = (cudaStream_t)stream;
   int32_t* dtab = (int32_t*)workspace;
   // Tensor-core path: every query row is a decode of its sequence at its
   // visible length and RoPE position, run through the tensor-core decode

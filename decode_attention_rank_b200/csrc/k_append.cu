@@ -106,7 +106,7 @@ __global__ void k_pack(LayerView v, uint8_t* __restrict__ pool, long long n_page
         const float a = zi[p], bb = zi[p + half];
         val = j < half ? (float)(a * cs - bb * sn) : (float)(bb * cs + a * sn);
       }
-      const size_t o = (size_t)(slot * ld.width + j);
+      const size_t o = elem_index(slot, j, ld.width, ld.cmajor);
       if (v.es == 4)
         reinterpret_cast<float*>(blk)[o] = val;
       else

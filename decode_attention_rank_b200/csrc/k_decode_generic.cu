@@ -37,27 +37,6 @@ __device__ __forceinline__ int row_len_of(const RowInfo& ri, int row, int cap, u
   return len;
 }
 
-// Stored value of channel j of latent `ld` for token slot `slot` of a page block.
-__device__ __forceinline__ float latent_value(const LayerView& v, const uint8_t* blk, const LatentDesc& ld,
-                                              int slot, int j) {
-  if (!v.quantized) {
-    const size_t o = (size_t)slot * ld.width + j;
-    return v.es == 4 ? reinterpret_cast<const float*>(blk)[o]
-                     : __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(blk)[o]);
-  }
-  int g = 0;
-  for (int k = 1; k < ld.n_groups; ++k)
-    if (j >= v.grp[ld.group0 + k].start) g = k;
-  const GroupDesc gd = v.grp[ld.group0 + g];
-  const float s = __half2float(reinterpret_cast<const __half*>(blk)[g * kPage + slot]);
-  const uint32_t bit = code_bit(slot, j - gd.start, gd.n, gd.bits, ld.cmajor);
-  const uint32_t* w = reinterpret_cast<const uint32_t*>(blk + gd.code_off) + (bit >> 5);
-  const uint32_t sh = bit & 31;
-  uint32_t u = w[0] >> sh;
-  if (sh + gd.bits > 32) u |= w[1] << (32 - sh);
-  u &= (1u << gd.bits) - 1u;
-  return (float)((int)u - (1 << (gd.bits - 1))) * s;
-}
 
 __device__ __forceinline__ double rope_freq(int p, int d, float log2_theta) {
   return exp2(-(2.0 * p / d) * (double)log2_theta);

@@ -357,8 +357,8 @@ cudaError_t launch_pack_rows_tiles(const void* x, int rows, int K, void* tiles, 
   return cudaGetLastError();
 }
 
-cudaError_t launch_pack_rows_tiles_f32(const float* x, int rows, int K, void* tiles, cudaStream_t s) {
-  const int NB = outproj_nb(rows);
+cudaError_t launch_pack_rows_tiles_f32(const float* x, int rows, int K, void* tiles, cudaStream_t s, int nb) {
+  const int NB = nb > 0 ? nb : outproj_nb(rows);
   const int KT = (K + 63) / 64;
   const int ntiles = (rows + NB - 1) / NB;
   const long long n = (long long)ntiles * NB * KT * 8;

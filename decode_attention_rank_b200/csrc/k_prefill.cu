@@ -1,0 +1,741 @@
+// Causal prefill attention on the tensor cores.
+//
+// A chunk of new queries of one sequence attends to every cached key up to
+// its own position (the causal prefill of a chunked prompt; the model card
+// "tenosra/longchat-7b-starkv-proxima" reports a prefill kernel of its own,
+// and the pages give no algorithm for it).  Prefill differs from decode in
+// that a key is seen by up to a whole chunk of queries, so here the keys and
+// values are reconstructed once per chunk, K_h = RoPE(Zhat_k,kv(h) B'_k) and
+// V_h = Zhat_v B'_v[:, kv(h)] ("STAR-KV 阅读笔记" section 5.3: keys are
+// rebuilt from the pre-RoPE latents and rotated at their positions; the value
+// fusion of section 5.3 is an exact reorder, so the output may equally be
+// taken through W_o after the values are rebuilt), and the attention itself
+// is the standard one over 128 x 128 tiles:
+//
+//   k_prefill_q        Q tiles: RoPE at the query positions, softmax scale * log2(e), fp16
+//   k_prefill_keys     K tiles: dequantize, K = Zhat B'_k (CUDA cores, r <= 64 MACs per output), RoPE, fp16
+//   k_prefill_zv       the dequantized value latent as fp16 B tiles
+//   k_gemm_full        V^T tiles = (B'_v)^T Zhat_v^T on tcgen05; also out = y W_o
+//   k_prefill_plain_kv plain layers: their stored K (already rotated) and V as tiles
+//   k_flash_prefill    S = Q K^T and O += P V on tcgen05, online softmax in registers
+//
+// Tiles are 128 rows x 128 fp16 columns stored as two K-major 128-byte
+// swizzled atoms of 64 columns (32 KB), the operand layout of the MMAs.
+#include <float.h>
+#include <math.h>
+
+#include "tc_common.cuh"
+
+namespace starkv {
+
+namespace {
+
+constexpr int kT = 128;            // queries per query tile, keys per key tile
+constexpr int kTileB = 32768;      // one 128 x 128 fp16 tile
+constexpr int kAtomB = 16384;      // one 128 x 64 atom
+constexpr int kMaxPrefillRank = 64;   // key ranks the key reconstruction holds in registers
+
+// Byte offset of element (row, col) inside a tile.
+__device__ __forceinline__ uint32_t tile_off(int row, int col) {
+  return (uint32_t)(col >> 6) * kAtomB + tc::sw128((uint32_t)row, (uint32_t)((col & 63) >> 3)) + (uint32_t)(col & 7) * 2u;
+}
+
+__device__ __forceinline__ uint32_t pack_half2(float a, float b) {
+  const __half2 h = __floats2half2_rn(a, b);
+  return *reinterpret_cast<const uint32_t*>(&h);
+}
+
+// ------------------------------------------------------------------ Q tiles
+// Query i of the chunk (position q_start + i): RoPE (rotate-half pairs, angle
+// reduced modulo 2 pi in double), times softmax scale * log2(e), as row i % 128
+// of tile [h][i / 128].  Rows past the chunk are zero.
+__global__ void __launch_bounds__(kT) k_prefill_q(LayerView v, const __nv_bfloat16* __restrict__ q, int q_len,
+                                                  int q_start, int n_qt, uint8_t* __restrict__ Qt) {
+  const int qt = blockIdx.x, h = blockIdx.y, r = threadIdx.x;
+  const int i = qt * kT + r;
+  uint8_t* tile = Qt + ((size_t)h * n_qt + qt) * kTileB;
+  const __nv_bfloat16* qr = q + ((size_t)i * v.H + h) * 128;
+  const int pos = q_start + i;
+  for (int c8 = 0; c8 < 8; ++c8) {   // pairs p = 8 c8 .. 8 c8 + 7 and p + 64
+    uint32_t lo[4], hi[4];
+#pragma unroll
+    for (int k = 0; k < 8; k += 2) {
+      float re[2] = {0.f, 0.f}, im[2] = {0.f, 0.f};
+      if (i < q_len) {
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          const int p = c8 * 8 + k + e;
+          const float a = __bfloat162float(qr[p]), b = __bfloat162float(qr[p + 64]);
+          float cs = 1.f, sn = 0.f;
+          if (v.rope) {
+            const double ang = (double)pos * exp2(-(2.0 * p / 128.0) * (double)v.rope_log2_theta);
+            const double two_pi = 6.283185307179586476925286766559;
+            sincosf((float)(ang - two_pi * rint(ang / two_pi)), &sn, &cs);
+          }
+          re[e] = (a * cs - b * sn) * v.scale_log2;
+          im[e] = (b * cs + a * sn) * v.scale_log2;
+        }
+      }
+      lo[k / 2] = pack_half2(re[0], re[1]);
+      hi[k / 2] = pack_half2(im[0], im[1]);
+    }
+    *reinterpret_cast<uint4*>(tile + tile_off(r, c8 * 8)) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+    *reinterpret_cast<uint4*>(tile + tile_off(r, 64 + c8 * 8)) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+  }
+}
+
+// ------------------------------------------------------------------ K tiles (latent layers)
+// Token t = kt * 128 + r of the sequence, KV head g: the dequantized key
+// latent (r_g <= 64 channels), K = zhat B'_k,g, rotated at position t with
+// the layer's RoPE table (the same fp16 cos / sin the decode scores use).
+__global__ void __launch_bounds__(kT) k_prefill_keys(LayerView v, const uint8_t* __restrict__ pool,
+                                                     long long n_pages, const int32_t* __restrict__ pt_row,
+                                                     int T, const float* __restrict__ Bk,
+                                                     const int* __restrict__ key_off, const uint8_t* __restrict__ E,
+                                                     int n_kt, uint8_t* __restrict__ Kt) {
+  __shared__ float Bs[kMaxPrefillRank][128];
+  const int kt = blockIdx.x, g = blockIdx.y, r = threadIdx.x;
+  const LatentDesc ld = v.lat[g];
+  const int R = ld.width;
+  for (int e = threadIdx.x; e < R * 128; e += blockDim.x) Bs[e >> 7][e & 127] = Bk[(size_t)key_off[g] * 128 + e];
+  const int t = kt * kT + r;
+  float z[kMaxPrefillRank];
+  if (t < T) {
+    int page = pt_row[t / kPage];
+    if (page < 0 || page >= n_pages) {
+      atomicOr(v.status, kBadPage);
+      page = 0;
+    }
+    const uint8_t* blk = pool + (size_t)page * v.page_bytes + ld.block_off;
+#pragma unroll
+    for (int j = 0; j < kMaxPrefillRank; ++j) z[j] = j < R ? latent_value(v, blk, ld, t % kPage, j) : 0.f;
+  } else {
+#pragma unroll
+    for (int j = 0; j < kMaxPrefillRank; ++j) z[j] = 0.f;
+  }
+  __syncthreads();
+  uint8_t* tile = Kt + ((size_t)g * n_kt + kt) * kTileB;
+  const uint8_t* Et = E + (size_t)(t / kT) * kTileB;
+  for (int c8 = 0; c8 < 8; ++c8) {
+    float re[8], im[8];
+#pragma unroll
+    for (int k = 0; k < 8; ++k) re[k] = im[k] = 0.f;
+#pragma unroll
+    for (int j = 0; j < kMaxPrefillRank; ++j) {
+      if (j >= R) break;
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        re[k] = fmaf(z[j], Bs[j][c8 * 8 + k], re[k]);
+        im[k] = fmaf(z[j], Bs[j][64 + c8 * 8 + k], im[k]);
+      }
+    }
+    uint32_t lo[4], hi[4];
+#pragma unroll
+    for (int k = 0; k < 8; k += 2) {
+      float a[2], b[2];
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        const int p = c8 * 8 + k + e;
+        float cs = 1.f, sn = 0.f;
+        if (v.rope && t < T) {
+          cs = __half2float(*reinterpret_cast<const __half*>(Et + tile_off(t % kT, p)));
+          sn = __half2float(*reinterpret_cast<const __half*>(Et + tile_off(t % kT, 64 + p)));
+        }
+        a[e] = re[k + e] * cs - im[k + e] * sn;
+        b[e] = im[k + e] * cs + re[k + e] * sn;
+      }
+      lo[k / 2] = pack_half2(a[0], a[1]);
+      hi[k / 2] = pack_half2(b[0], b[1]);
+    }
+    *reinterpret_cast<uint4*>(tile + tile_off(r, c8 * 8)) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+    *reinterpret_cast<uint4*>(tile + tile_off(r, 64 + c8 * 8)) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+  }
+}
+
+// ------------------------------------------------------------------ dequantized value latent
+// B tiles [kt][rv / 64] of 128 tokens x 64 channels (fp16, swizzled) for the
+// V^T product; tokens past T are zero.
+__global__ void k_prefill_zv(LayerView v, const uint8_t* __restrict__ pool, long long n_pages,
+                             const int32_t* __restrict__ pt_row, int T, int n_kt, uint8_t* __restrict__ Zt) {
+  const int KT = v.rv / 64;
+  const long long idx = (long long)blockIdx.x * blockDim.x + threadIdx.x;   // (tile kt, k-tile, row, chunk)
+  if (idx >= (long long)n_kt * KT * kT * 8) return;
+  const int c = (int)(idx & 7);
+  const int row = (int)((idx >> 3) % kT);
+  const long long tk = (idx >> 3) / kT;
+  const int kk = (int)(tk % KT), kt = (int)(tk / KT);
+  const int t = kt * kT + row;
+  const LatentDesc ld = v.lat[v.L - 1];
+  uint32_t o[4] = {0u, 0u, 0u, 0u};
+  if (t < T) {
+    int page = pt_row[t / kPage];
+    if (page < 0 || page >= n_pages) {
+      atomicOr(v.status, kBadPage);
+      page = 0;
+    }
+    const uint8_t* blk = pool + (size_t)page * v.page_bytes + ld.block_off;
+#pragma unroll
+    for (int k = 0; k < 8; k += 2) {
+      const int j = kk * 64 + c * 8 + k;
+      o[k / 2] = pack_half2(latent_value(v, blk, ld, t % kPage, j), latent_value(v, blk, ld, t % kPage, j + 1));
+    }
+  }
+  uint8_t* tile = Zt + ((size_t)kt * KT + kk) * kAtomB;
+  *reinterpret_cast<uint4*>(tile + tc::sw128((uint32_t)row, (uint32_t)c)) = make_uint4(o[0], o[1], o[2], o[3]);
+}
+
+// ------------------------------------------------------------------ plain layers: stored K, V as tiles
+// K block of KV head g: [slot][128] bf16 (already rotated); V block:
+// [slot][H_kv 128] bf16.  One CTA per (key tile, KV head); V is transposed
+// through shared memory.
+__global__ void __launch_bounds__(256) k_prefill_plain_kv(LayerView v, const uint8_t* __restrict__ pool,
+                                                         long long n_pages, const int32_t* __restrict__ pt_row,
+                                                         int T, int n_kt, uint8_t* __restrict__ Kt,
+                                                         uint8_t* __restrict__ Vt) {
+  __shared__ __half Vs[kT][kT + 8];
+  const int kt = blockIdx.x, g = blockIdx.y;
+  const LatentDesc kd = v.lat[g], vd = v.lat[v.L - 1];
+  uint8_t* ktile = Kt + ((size_t)g * n_kt + kt) * kTileB;
+  uint8_t* vtile = Vt + ((size_t)g * n_kt + kt) * kTileB;
+  for (int e = threadIdx.x; e < kT * 16; e += blockDim.x) {   // (token row, 8-channel chunk)
+    const int row = e >> 4, c = e & 15;
+    const int t = kt * kT + row;
+    uint4 kk = make_uint4(0, 0, 0, 0), vv = kk;
+    if (t < T) {
+      int page = pt_row[t / kPage];
+      if (page < 0 || page >= n_pages) {
+        atomicOr(v.status, kBadPage);
+        page = 0;
+      }
+      const uint8_t* base = pool + (size_t)page * v.page_bytes;
+      kk = *reinterpret_cast<const uint4*>(base + kd.block_off + ((size_t)(t % kPage) * 128 + c * 8) * 2);
+      vv = *reinterpret_cast<const uint4*>(base + vd.block_off + ((size_t)(t % kPage) * v.rv + g * 128 + c * 8) * 2);
+    }
+    const uint32_t kw[4] = {kk.x, kk.y, kk.z, kk.w}, vw[4] = {vv.x, vv.y, vv.z, vv.w};
+    uint32_t ko[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const float a = __uint_as_float(kw[k] << 16), b = __uint_as_float(kw[k] & 0xFFFF0000u);
+      ko[k] = pack_half2(a, b);
+      Vs[row][c * 8 + 2 * k] = __float2half_rn(__uint_as_float(vw[k] << 16));
+      Vs[row][c * 8 + 2 * k + 1] = __float2half_rn(__uint_as_float(vw[k] & 0xFFFF0000u));
+    }
+    *reinterpret_cast<uint4*>(ktile + tile_off(row, c * 8)) = make_uint4(ko[0], ko[1], ko[2], ko[3]);
+  }
+  __syncthreads();
+  for (int e = threadIdx.x; e < kT * 16; e += blockDim.x) {   // (channel row p, 8-token chunk)
+    const int p = e >> 4, c = e & 15;
+    uint32_t o[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const __half2 h = __halves2half2(Vs[c * 8 + 2 * k][p], Vs[c * 8 + 2 * k + 1][p]);
+      o[k] = *reinterpret_cast<const uint32_t*>(&h);
+    }
+    *reinterpret_cast<uint4*>(vtile + tile_off(p, c * 8)) = make_uint4(o[0], o[1], o[2], o[3]);
+  }
+}
+
+// ------------------------------------------------------------------ full-K GEMM on tcgen05
+// D[m][n] = sum_k A[m][k] B[n][k] for one 128 x 128 output tile, all of K in
+// one CTA.  A: 128 x 64 tiles at a_base + blockIdx.y * a_step, k-tiles 16 KB
+// apart; B: 128 x 64 tiles at b_base + blockIdx.x * b_step, likewise.
+//   EPI_VT:  the tile is V^T of KV head blockIdx.y, key tile blockIdx.x:
+//            written as a flash-attention V^T tile (fp16)
+//   EPI_OUT: out[n][m] for rows n < rows and columns m < n_valid (bf16 or fp32)
+constexpr int kGemmThreads = 256;
+constexpr int kGemmStages = 4;
+enum { EPI_VT = 0, EPI_OUT_BF16 = 1, EPI_OUT_F32 = 2 };
+
+struct GemmArgs {
+  const uint8_t* A;
+  long long a_step;
+  const uint8_t* B;
+  long long b_step;
+  int KT;
+  void* out;            // EPI_VT: tiles [blockIdx.y][n_tiles]; EPI_OUT: row-major [rows][ld]
+  int n_tiles;          // EPI_VT
+  int rows, n_valid, ld;   // EPI_OUT
+  uint32_t* status;
+};
+
+template <int EPI>
+__global__ void __launch_bounds__(kGemmThreads, 1) k_gemm_full(GemmArgs a) {
+  extern __shared__ uint8_t smem_raw[];
+  __shared__ __align__(8) uint64_t full[kGemmStages], empty[kGemmStages], done;
+  __shared__ uint32_t tmem_base;
+  __shared__ volatile int abort_flag;
+  uint8_t* smem = smem_raw + ((1024u - (tc::smem_u32(smem_raw) & 1023u)) & 1023u);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint8_t* Ab = a.A + (size_t)blockIdx.y * a.a_step;
+  const uint8_t* Bb = a.B + (size_t)blockIdx.x * a.b_step;
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kGemmStages; ++s) {
+      tc::mbar_init(&full[s], 1);
+      tc::mbar_init(&empty[s], 1);
+    }
+    tc::mbar_init(&done, 1);
+    abort_flag = 0;
+    tc::fence_mbar_init();
+  }
+  if (warp == 1) tc::tmem_alloc(&tmem_base, 128);
+  tc::tc_fence_before();
+  __syncthreads();
+  tc::tc_fence_after();
+  const uint32_t tmem = tmem_base;
+  if (warp == 0) {
+    if (lane == 0) {
+      int k = 0;
+      for (; k < a.KT; ++k) {
+        const int s = k % kGemmStages;
+        if (!tc::mbar_wait_ab_lazy(&empty[s], (((uint32_t)(k / kGemmStages)) & 1u) ^ 1u, a.status, &abort_flag)) break;
+        tc::mbar_expect_tx(&full[s], 2 * kAtomB);
+        tc::bulk_g2s(smem + (size_t)s * 2 * kAtomB, Ab + (size_t)k * kAtomB, kAtomB, &full[s]);
+        tc::bulk_g2s(smem + (size_t)s * 2 * kAtomB + kAtomB, Bb + (size_t)k * kAtomB, kAtomB, &full[s]);
+      }
+      for (int j = max(0, k - kGemmStages); j < k; ++j)
+        tc::mbar_wait(&full[j % kGemmStages], ((uint32_t)(j / kGemmStages)) & 1u, a.status);
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    if (lane == 0) {
+      const uint32_t idesc = tc::idesc_f16(128, 128, false, false, false);
+      const uint64_t d0 = tc::sdesc_sw128(tc::smem_u32(smem), 0, 1024);
+      const uint32_t lo0 = tc::desc_lo(d0), hi = tc::desc_hi(d0);
+      int k = 0;
+      for (; k < a.KT && !abort_flag; ++k) {
+        const int s = k % kGemmStages;
+        if (!tc::mbar_wait_ab(&full[s], ((uint32_t)(k / kGemmStages)) & 1u, a.status, &abort_flag)) {
+          abort_flag = 1;
+          break;
+        }
+        tc::tc_fence_after();
+        const uint32_t alo = lo0 + (uint32_t)(s * 2 * kAtomB >> 4), blo = alo + (uint32_t)(kAtomB >> 4);
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk)
+          tc::mma_f16_ss2(tmem, alo + 2u * kk, hi, blo + 2u * kk, hi, idesc, (k | kk) ? 1u : 0u);
+        tc::mma_commit(&empty[s]);
+      }
+      tc::mma_commit(&done);
+    }
+    __syncwarp();
+  } else if (warp >= 4) {
+    const int q = warp & 3;
+    const int m = q * 32 + lane;   // TMEM lane = output row m
+    const bool ok = tc::mbar_wait_ab(&done, 0, a.status, &abort_flag);
+    tc::tc_fence_after();
+    for (int c0 = 0; c0 < 128; c0 += 16) {
+      float x[16];
+      if (ok) {
+        tc::tmem_ld16_sync(tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)c0, x);
+      } else {
+#pragma unroll
+        for (int i = 0; i < 16; ++i) x[i] = 0.f;
+      }
+      if constexpr (EPI == EPI_VT) {
+        uint8_t* tile = (uint8_t*)a.out + ((size_t)blockIdx.y * a.n_tiles + blockIdx.x) * kTileB;
+#pragma unroll
+        for (int h8 = 0; h8 < 2; ++h8)
+          *reinterpret_cast<uint4*>(tile + tile_off(m, c0 + h8 * 8)) =
+              make_uint4(pack_half2(x[h8 * 8], x[h8 * 8 + 1]), pack_half2(x[h8 * 8 + 2], x[h8 * 8 + 3]),
+                         pack_half2(x[h8 * 8 + 4], x[h8 * 8 + 5]), pack_half2(x[h8 * 8 + 6], x[h8 * 8 + 7]));
+      } else {
+        const int col = blockIdx.y * 128 + m;
+        if (col < a.n_valid) {
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            const int row = blockIdx.x * 128 + c0 + i;
+            if (row < a.rows) {
+              if constexpr (EPI == EPI_OUT_F32)
+                reinterpret_cast<float*>(a.out)[(size_t)row * a.ld + col] = x[i];
+              else
+                reinterpret_cast<__nv_bfloat16*>(a.out)[(size_t)row * a.ld + col] = __float2bfloat16_rn(x[i]);
+            }
+          }
+        }
+      }
+    }
+  }
+  tc::tc_fence_before();
+  __syncthreads();
+  tc::tc_fence_after();
+  if (warp == 1) tc::tmem_dealloc(tmem, 128);
+}
+
+// ------------------------------------------------------------------ flash attention over the tiles
+// One CTA per (query tile, query head).  TMEM: S in two 128-column buffers,
+// O in columns 256 .. 383.
+//   warp 0     bulk copies: the Q tile, then K and V^T tiles into two stages
+//   warp 1     MMA issue: S(k + 1) = Q K(k + 1)^T is issued before O += P(k) V(k)
+//   warps 4-7  softmax, one query row per thread: S row from TMEM, causal
+//              mask, running maximum; O is rescaled only when the maximum
+//              grew by more than 2^8 since the last rescale (P then stays
+//              below 256, exact in fp16), P written as the fp16 A operand of
+//              the next MMA; at the end y = O / l
+constexpr int kFlashThreads = 256;
+constexpr float kRescaleSlack = 8.f;   // log2 units
+
+struct FlashArgs {
+  const uint8_t* Q;     // [H][n_qt] tiles
+  const uint8_t* K;     // [Hkv][n_kt] tiles: rows = keys, columns = channels
+  const uint8_t* Vt;    // [Hkv][n_kt] tiles: rows = channels, columns = keys
+  int n_qt, n_kt;
+  int q_len, q_start;   // queries at positions q_start .. q_start + q_len - 1
+  int group_q;
+  float* y;             // [q_len][y_ld]: head h at columns 128 h ..
+  int y_ld;
+  uint32_t* status;
+};
+
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float* v) {
+  uint32_t r[32];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
+        "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
+        "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr));
+#pragma unroll
+  for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+}
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const float* v) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
+      "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(taddr),
+      "f"(v[0]), "f"(v[1]), "f"(v[2]), "f"(v[3]), "f"(v[4]), "f"(v[5]), "f"(v[6]), "f"(v[7]), "f"(v[8]),
+      "f"(v[9]), "f"(v[10]), "f"(v[11]), "f"(v[12]), "f"(v[13]), "f"(v[14]), "f"(v[15]), "f"(v[16]), "f"(v[17]),
+      "f"(v[18]), "f"(v[19]), "f"(v[20]), "f"(v[21]), "f"(v[22]), "f"(v[23]), "f"(v[24]), "f"(v[25]), "f"(v[26]),
+      "f"(v[27]), "f"(v[28]), "f"(v[29]), "f"(v[30]), "f"(v[31])
+      : "memory");
+}
+
+__global__ void __launch_bounds__(kFlashThreads, 1) k_flash_prefill(FlashArgs a) {
+  extern __shared__ uint8_t smem_raw[];
+  __shared__ __align__(8) uint64_t q_full, kv_full[2], kv_empty[2], s_full[2], s_free[2], p_full, o_done, fin;
+  __shared__ uint32_t tmem_base;
+  __shared__ volatile int abort_flag;
+  uint8_t* smem = smem_raw + ((1024u - (tc::smem_u32(smem_raw) & 1023u)) & 1023u);
+  uint8_t* Q_s = smem;
+  uint8_t* K_s = Q_s + kTileB;        // two stages
+  uint8_t* V_s = K_s + 2 * kTileB;    // two stages
+  uint8_t* P_s = V_s + 2 * kTileB;
+  const int qt = blockIdx.x, h = blockIdx.y, g = h / a.group_q;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int q0 = qt * kT;
+  const int nq = min(kT, a.q_len - q0);
+  const int n_kt = (a.q_start + q0 + nq - 1) / kT + 1;   // key tiles holding a key visible to this tile
+  if (threadIdx.x == 0) {
+    tc::mbar_init(&q_full, 1);
+    for (int s = 0; s < 2; ++s) {
+      tc::mbar_init(&kv_full[s], 1);
+      tc::mbar_init(&kv_empty[s], 1);
+      tc::mbar_init(&s_full[s], 1);
+      tc::mbar_init(&s_free[s], 4);
+    }
+    tc::mbar_init(&p_full, 4);
+    tc::mbar_init(&o_done, 1);
+    tc::mbar_init(&fin, 1);
+    abort_flag = 0;
+    tc::fence_mbar_init();
+  }
+  if (warp == 1) tc::tmem_alloc(&tmem_base, 512);
+  tc::tc_fence_before();
+  __syncthreads();
+  tc::tc_fence_after();
+  const uint32_t tmem = tmem_base;
+  const uint32_t o_col = 256;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      tc::mbar_expect_tx(&q_full, kTileB);
+      tc::bulk_g2s(Q_s, a.Q + ((size_t)h * a.n_qt + qt) * kTileB, kTileB, &q_full);
+      int k = 0;
+      for (; k < n_kt; ++k) {
+        const int s = k & 1;
+        if (!tc::mbar_wait_ab_lazy(&kv_empty[s], (((uint32_t)(k >> 1)) & 1u) ^ 1u, a.status, &abort_flag)) break;
+        tc::mbar_expect_tx(&kv_full[s], 2 * kTileB);
+        tc::bulk_g2s(K_s + (size_t)s * kTileB, a.K + ((size_t)g * a.n_kt + k) * kTileB, kTileB, &kv_full[s]);
+        tc::bulk_g2s(V_s + (size_t)s * kTileB, a.Vt + ((size_t)g * a.n_kt + k) * kTileB, kTileB, &kv_full[s]);
+      }
+      tc::mbar_wait(&q_full, 0, a.status);
+      for (int j = max(0, k - 2); j < k; ++j) tc::mbar_wait(&kv_full[j & 1], ((uint32_t)(j >> 1)) & 1u, a.status);
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    if (lane == 0) {
+      const uint32_t idesc = tc::idesc_f16(128, 128, false, false, false);
+      const uint64_t d0 = tc::sdesc_sw128(tc::smem_u32(smem), 0, 1024);
+      const uint32_t base_lo = tc::desc_lo(d0), hi = tc::desc_hi(d0);
+      const uint32_t q_lo = base_lo, k_lo = base_lo + (kTileB >> 4), v_lo = base_lo + (3 * kTileB >> 4),
+                     p_lo = base_lo + (5 * kTileB >> 4);
+      bool ok = tc::mbar_wait_ab(&q_full, 0, a.status, &abort_flag);
+      // S(k) = Q K(k)^T into S buffer k & 1
+      auto issue_s = [&](int k) -> bool {
+        const int s = k & 1;
+        if (!tc::mbar_wait_ab(&kv_full[s], ((uint32_t)(k >> 1)) & 1u, a.status, &abort_flag)) return false;
+        if (!tc::mbar_wait_ab(&s_free[s], (((uint32_t)(k >> 1)) & 1u) ^ 1u, a.status, &abort_flag)) return false;
+        tc::tc_fence_after();
+        const uint32_t kb = k_lo + (uint32_t)(s * kTileB >> 4);
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)
+          tc::mma_f16_ss2(tmem + (uint32_t)(s * 128), q_lo + (uint32_t)(kk >> 2) * (kAtomB >> 4) + 2u * (kk & 3), hi,
+                          kb + (uint32_t)(kk >> 2) * (kAtomB >> 4) + 2u * (kk & 3), hi, idesc, kk ? 1u : 0u);
+        tc::mma_commit(&s_full[s]);
+        return true;
+      };
+      tc::tc_fence_after();
+      if (ok) ok = issue_s(0);
+      for (int k = 0; k < n_kt && ok; ++k) {
+        if (k + 1 < n_kt && !(ok = issue_s(k + 1))) break;
+        // O += P(k) V(k)
+        if (!(ok = tc::mbar_wait_ab(&p_full, (uint32_t)k & 1u, a.status, &abort_flag))) break;
+        tc::tc_fence_after();
+        const uint32_t vb = v_lo + (uint32_t)((k & 1) * kTileB >> 4);
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)
+          tc::mma_f16_ss2(tmem + o_col, p_lo + (uint32_t)(kk >> 2) * (kAtomB >> 4) + 2u * (kk & 3), hi,
+                          vb + (uint32_t)(kk >> 2) * (kAtomB >> 4) + 2u * (kk & 3), hi, idesc, (k | kk) ? 1u : 0u);
+        tc::mma_commit(&o_done);
+        tc::mma_commit(&kv_empty[k & 1]);
+      }
+      if (!ok) abort_flag = 1;
+      // every MMA has completed before the CTA may exit
+      tc::mma_commit(&fin);
+      tc::mbar_wait(&fin, 0, a.status);
+    }
+    __syncwarp();
+  } else if (warp >= 4) {
+    const int qq = warp & 3;
+    const int r = qq * 32 + lane;                 // query row of the tile = TMEM lane
+    const int pos = a.q_start + q0 + r;           // its position
+    const uint32_t lane_base = (uint32_t)(qq * 32) << 16;
+    float m_used = -FLT_MAX, l = 0.f;
+    bool ok = true;
+    for (int k = 0; k < n_kt; ++k) {
+      const int b = k & 1;
+      ok = ok && tc::mbar_wait_ab(&s_full[b], ((uint32_t)(k >> 1)) & 1u, a.status, &abort_flag);
+      tc::tc_fence_after();
+      float s[128];
+      if (ok) {
+#pragma unroll
+        for (int c = 0; c < 128; c += 32) tmem_ld32(tmem + lane_base + (uint32_t)(b * 128 + c), s + c);
+        tc::tmem_ld_wait();
+      } else {
+#pragma unroll
+        for (int c = 0; c < 128; ++c) s[c] = 0.f;
+      }
+      // the S buffer may be overwritten once every warp has it in registers
+      tc::tc_fence_before();
+      __syncwarp();
+      if (lane == 0) tc::mbar_arrive(&s_free[b]);
+      // causal mask: key k * 128 + c is visible to the query at `pos` if it is not later
+      const int lim = pos - k * kT;   // columns c <= lim are visible
+      float mx = -FLT_MAX;
+#pragma unroll
+      for (int c = 0; c < 128; ++c) {
+        if (c > lim) s[c] = -FLT_MAX;
+        mx = fmaxf(mx, s[c]);
+      }
+      // rescale O only when the maximum moved far enough
+      float f = 1.f;
+      if (mx > m_used + kRescaleSlack || k == 0) {
+        f = k == 0 ? 0.f : exp2f(m_used - mx);
+        m_used = mx;
+      }
+      uint32_t p2[64];
+      float ls = 0.f;
+#pragma unroll
+      for (int c = 0; c < 128; c += 2) {
+        const float e0 = s[c] == -FLT_MAX ? 0.f : exp2f(s[c] - m_used);
+        const float e1 = s[c + 1] == -FLT_MAX ? 0.f : exp2f(s[c + 1] - m_used);
+        const __half2 hp = __floats2half2_rn(e0, e1);
+        const float2 back = __half22float2(hp);
+        ls += back.x + back.y;
+        p2[c / 2] = *reinterpret_cast<const uint32_t*>(&hp);
+      }
+      l = l * f + ls;
+      // P(k - 1) V(k - 1) must be done before O is touched and P is overwritten
+      if (k > 0) {
+        ok = ok && tc::mbar_wait_ab(&o_done, ((uint32_t)(k - 1)) & 1u, a.status, &abort_flag);
+        tc::tc_fence_after();
+        if (ok && f != 1.f) {
+#pragma unroll 1
+          for (int c = 0; c < 128; c += 32) {
+            float o[32];
+            tmem_ld32(tmem + lane_base + o_col + (uint32_t)c, o);
+            tc::tmem_ld_wait();
+#pragma unroll
+            for (int i = 0; i < 32; ++i) o[i] *= f;
+            tmem_st32(tmem + lane_base + o_col + (uint32_t)c, o);
+          }
+          tc::tmem_st_wait();
+        }
+      }
+#pragma unroll
+      for (int c8 = 0; c8 < 16; ++c8)
+        *reinterpret_cast<uint4*>(P_s + tile_off(r, c8 * 8)) =
+            make_uint4(p2[c8 * 4], p2[c8 * 4 + 1], p2[c8 * 4 + 2], p2[c8 * 4 + 3]);
+      tc::fence_proxy_async();
+      tc::tc_fence_before();
+      __syncwarp();
+      if (lane == 0) tc::mbar_arrive(&p_full);
+    }
+    ok = ok && tc::mbar_wait_ab(&o_done, ((uint32_t)(n_kt - 1)) & 1u, a.status, &abort_flag);
+    tc::tc_fence_after();
+    const float inv = l > 0.f ? 1.f / l : 0.f;
+    const bool row_ok = r < nq;
+#pragma unroll 1
+    for (int c = 0; c < 128; c += 32) {
+      float o[32];
+      if (ok) {
+        tmem_ld32(tmem + lane_base + o_col + (uint32_t)c, o);
+        tc::tmem_ld_wait();
+      }
+      if (row_ok) {
+        float* yr = a.y + (size_t)(q0 + r) * a.y_ld + (size_t)h * 128 + c;
+#pragma unroll
+        for (int i = 0; i < 32; i += 4)
+          *reinterpret_cast<float4*>(yr + i) =
+              ok ? make_float4(o[i] * inv, o[i + 1] * inv, o[i + 2] * inv, o[i + 3] * inv) : make_float4(0, 0, 0, 0);
+      }
+    }
+  }
+  tc::tc_fence_before();
+  __syncthreads();
+  tc::tc_fence_after();
+  if (warp == 1) tc::tmem_dealloc(tmem, 512);
+}
+
+size_t al256(size_t x) { return (x + 255) / 256 * 256; }
+
+struct PrefillWs {
+  uint8_t *Qt, *Kt, *Vt, *Zt, *yt;
+  float* y;
+};
+
+PrefillWs prefill_ws_layout(const starkv_layer* L, void* ws, int max_T, int max_q) {
+  const LayerView& v = L->view;
+  const int n_qt = (max_q + kT - 1) / kT, n_kt = (max_T + kT - 1) / kT;
+  PrefillWs w;
+  uint8_t* p = (uint8_t*)ws;
+  w.Qt = p;
+  p += al256((size_t)v.H * n_qt * kTileB);
+  w.Kt = p;
+  p += al256((size_t)v.Hkv * n_kt * kTileB);
+  w.Vt = p;
+  p += al256((size_t)v.Hkv * n_kt * kTileB);
+  w.Zt = p;
+  p += al256(v.plain ? 0 : (size_t)n_kt * (v.rv / 64) * kAtomB);
+  w.y = (float*)p;
+  p += al256(sizeof(float) * (size_t)n_qt * kT * v.H * 128);
+  w.yt = p;
+  return w;
+}
+
+}  // namespace
+
+// W_o as A tiles [Dp / 128][H d / 64] of 128 x 64 (row n, column k = W_o[k][n]):
+// a plain layer's output factors are W_o itself.
+static const void* prefill_wo_tiles(const starkv_layer* L) { return L->view.plain ? L->M_T : L->Wo_tiles; }
+
+bool prefill_flash_supported(const starkv_layer* L) {
+  const LayerView& v = L->view;
+  if (v.dtype != STARKV_BF16 || v.d != 128 || !prefill_wo_tiles(L)) return false;
+  if (v.plain) return true;
+  if (!L->tc_scores || !L->Bv_tiles || v.rv % 64 != 0) return false;
+  for (int g = 0; g < v.Hkv; ++g)
+    if (L->lat[g].width > kMaxPrefillRank) return false;
+  return true;
+}
+
+size_t prefill_flash_ws_bytes(const starkv_layer* L, int max_T, int max_q) {
+  const LayerView& v = L->view;
+  const int n_qt = (max_q + kT - 1) / kT, n_kt = (max_T + kT - 1) / kT;
+  return al256((size_t)v.H * n_qt * kTileB) + 2 * al256((size_t)v.Hkv * n_kt * kTileB) +
+         al256(v.plain ? 0 : (size_t)n_kt * (v.rv / 64) * kAtomB) +
+         al256(sizeof(float) * (size_t)n_qt * kT * v.H * 128) + al256((size_t)n_qt * (v.H * 128 / 64) * kAtomB);
+}
+
+// One chunk of q_len queries of one sequence (page table row pt_row) at
+// positions q_start ..; q: [q_len][H][128] bf16; out: [q_len][D] in the layer dtype.
+cudaError_t launch_prefill_flash(const starkv_layer* L, const uint8_t* pool, long long n_pages, const int32_t* pt_row,
+                                 int q_start, int q_len, const void* q, void* out, void* ws, int max_T, int max_q,
+                                 cudaStream_t s) {
+  const LayerView& v = L->view;
+  const int T = q_start + q_len;
+  if (q_len <= 0) return cudaSuccess;
+  if (T > max_T || q_len > max_q || (!v.plain && T > L->rope_tiles * 128)) return cudaErrorInvalidValue;
+  // tiles this chunk fills, and the strides of the tile arrays (laid out for max_q / max_T)
+  const int n_qt = (q_len + kT - 1) / kT, n_kt = (T + kT - 1) / kT;
+  const int n_qt_l = (max_q + kT - 1) / kT, n_kt_l = (max_T + kT - 1) / kT;
+  PrefillWs w = prefill_ws_layout(L, ws, max_T, max_q);
+  cudaError_t e;
+  k_prefill_q<<<dim3(n_qt, v.H), kT, 0, s>>>(v, (const __nv_bfloat16*)q, q_len, q_start, n_qt_l, w.Qt);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  if (v.plain) {
+    k_prefill_plain_kv<<<dim3(n_kt, v.Hkv), 256, 0, s>>>(v, pool, n_pages, pt_row, T, n_kt_l, w.Kt, w.Vt);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  } else {
+    k_prefill_keys<<<dim3(n_kt, v.Hkv), kT, 0, s>>>(v, pool, n_pages, pt_row, T, L->Bk, L->d_key_off,
+                                                    (const uint8_t*)L->rope_E, n_kt_l, w.Kt);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    const long long nz = (long long)n_kt * (v.rv / 64) * kT * 8;
+    k_prefill_zv<<<(unsigned)((nz + 255) / 256), 256, 0, s>>>(v, pool, n_pages, pt_row, T, n_kt, w.Zt);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    // V^T of KV head g = (B'_v columns of g)^T Zhat_v^T: A = the 128 x r_v B'_v tiles of query head g * group_q
+    GemmArgs ga{};
+    ga.A = (const uint8_t*)L->Bv_tiles;
+    ga.a_step = (long long)v.group_q * (v.rv / 64) * kAtomB;
+    ga.B = w.Zt;
+    ga.b_step = (long long)(v.rv / 64) * kAtomB;
+    ga.KT = v.rv / 64;
+    ga.out = w.Vt;
+    ga.n_tiles = n_kt_l;
+    ga.status = v.status;
+    const size_t smem = (size_t)kGemmStages * 2 * kAtomB + 1024;
+    if ((e = set_smem_limit((const void*)k_gemm_full<EPI_VT>, smem)) != cudaSuccess) return e;
+    k_gemm_full<EPI_VT><<<dim3(n_kt, v.Hkv), kGemmThreads, smem, s>>>(ga);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  }
+  FlashArgs fa;
+  fa.Q = w.Qt;
+  fa.K = w.Kt;
+  fa.Vt = w.Vt;
+  fa.n_qt = n_qt_l;
+  fa.n_kt = n_kt_l;
+  fa.q_len = q_len;
+  fa.q_start = q_start;
+  fa.group_q = v.group_q;
+  fa.y = w.y;
+  fa.y_ld = v.H * 128;
+  fa.status = v.status;
+  const size_t fsmem = 6 * (size_t)kTileB + 1024;
+  if ((e = set_smem_limit((const void*)k_flash_prefill, fsmem)) != cudaSuccess) return e;
+  k_flash_prefill<<<dim3(n_qt, v.H), kFlashThreads, fsmem, s>>>(fa);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  // out = y W_o: y as fp16 B tiles of 128 rows, W_o as the A tiles
+  if ((e = launch_pack_rows_tiles_f32(w.y, q_len, v.H * 128, w.yt, s, 128)) != cudaSuccess) return e;
+  GemmArgs go{};
+  go.A = (const uint8_t*)prefill_wo_tiles(L);
+  go.a_step = (long long)(v.H * 128 / 64) * kAtomB;
+  go.B = w.yt;
+  go.b_step = (long long)(v.H * 128 / 64) * kAtomB;
+  go.KT = v.H * 128 / 64;
+  go.out = out;
+  go.rows = q_len;
+  go.n_valid = v.D;
+  go.ld = v.D;
+  go.status = v.status;
+  const size_t smem = (size_t)kGemmStages * 2 * kAtomB + 1024;
+  const void* gk = v.dtype == STARKV_F32 ? (const void*)k_gemm_full<EPI_OUT_F32> : (const void*)k_gemm_full<EPI_OUT_BF16>;
+  if ((e = set_smem_limit(gk, smem)) != cudaSuccess) return e;
+  const dim3 grid(n_qt, (v.D + 127) / 128);
+  if (v.dtype == STARKV_F32)
+    k_gemm_full<EPI_OUT_F32><<<grid, kGemmThreads, smem, s>>>(go);
+  else
+    k_gemm_full<EPI_OUT_BF16><<<grid, kGemmThreads, smem, s>>>(go);
+  return cudaGetLastError();
+}
+
+}  // namespace starkv

@@ -14,7 +14,8 @@
 // epilogue straight out of TMEM.
 //
 // Heads are grouped into MMA items of N <= 128 rows of W'' (an N of 32 per head
-// would leave the tensor pipe two-thirds idle).  A unit is one 256-token
+// would leave the tensor pipe two-thirds idle).  Each (item, tile) job has
+// its own 128-column TMEM accumulator stage, one per epilogue set.  A unit is one 256-token
 // super-tile (two M = 128 tiles sharing one W'' load) of one sequence; a CTA
 // walks a contiguous range of units ordered position-major, so its RoPE tiles
 // stay resident across the sequences of one position.
@@ -46,6 +47,8 @@ constexpr int kEpiWarps = 16;
 constexpr int kScoreThreads = 128 + 32 * kEpiWarps;   // key copies, 2 MMA, W''/E copies, 16 epilogue warps
 constexpr int kMma2Warp = 3 + kEpiWarps;              // the second MMA warp
 constexpr int kSuper = 256;          // tokens per super-tile
+constexpr int kItemCols = 128;       // TMEM columns of one accumulator stage: an item's MMA N is at most this
+constexpr int kAccStages = 512 / kItemCols;   // one stage per epilogue set (two when items are 64 columns)
 constexpr int kETileBytes = 32768;   // one 128-position RoPE tile (128 x 128 fp16)
 
 struct ScoreArgs {
@@ -84,14 +87,24 @@ __device__ __forceinline__ long long unit_lo(int c, int G, long long U) { return
 // mantissa bits [23 - TB B, 23), and one mask per code then gives
 //     f = 1 + u 2^((c - TB) B)      for the code at place c of its tuple.
 // The W'' row of that channel is pre-scaled by 2^(-c B) (exact), so with
-// G' = 2^(-c B) G every code contributes f G' = G' + u G 2^(-TB B) on one scale:
-//     sum (u - 2^(B-1)) G = 2^(TB B) sum f G' - sum g_c G',  g_c = 2^(TB B) + 2^(B-1) 2^(c B).
+// G' = 2^(-c B) G every code contributes f G' = G' + u G 2^(-TB B) on one scale.
+// With S_c the sum of G' over the channels at place c,
+//     sum (u - 2^(B-1)) G = 2^(TB B) (sum f G' - sum_c S_c) - 2^(B-1) sum_c 2^(c B) S_c.
 template <int B>
 __host__ __device__ constexpr int tuple_len() { return B == 4 ? 2 : 3; }
 
+// The bits of 1.0f in a register the compiler treats as opaque, so that each
+// code costs one three-input logic op (mask immediate, exponent register)
+// instead of a mask and a separate OR of a second immediate.
+__device__ __forceinline__ uint32_t one_bits() {
+  uint32_t e;
+  asm("mov.b32 %0, 0x3F800000;" : "=r"(e));
+  return e;
+}
+
 // Code I of a group of N codes whose per-token stream starts at bit 0 of run[].
 template <int N, int B, int I>
-__device__ __forceinline__ float code_float(const uint32_t* run) {
+__device__ __forceinline__ float code_float(const uint32_t* run, uint32_t one) {
   constexpr int TB = tuple_len<B>(), S0 = 23 - TB * B;
   constexpr int k = I / TB, c = I % TB;
   constexpr int pos = k * TB * B, wi = pos >> 5, o = pos & 31;
@@ -104,23 +117,23 @@ __device__ __forceinline__ float code_float(const uint32_t* run) {
   else
     y = __funnelshift_r(run[wi], run[wi + 1], o - S0);   // the tuple straddles two words
   constexpr uint32_t m = ((1u << B) - 1u) << (S0 + c * B);
-  return __uint_as_float((y & m) | 0x3F800000u);
-}
-template <int B, int I>
-__host__ __device__ constexpr float code_g() {
-  constexpr int TB = tuple_len<B>(), c = I % TB;
-  return (float)(1 << (TB * B)) + (float)(1 << (B - 1)) * (float)(1 << (c * B));
+  return __uint_as_float((y & m) | one);
 }
 
-// sum_i f_i G'[C + i] and sum_i g_i G'[C + i] over one group of N channels, in
-// packed fp32x2 pairs (a scalar step for an odd tail).
+// Accumulator of the place sums that channel pair I adds to: a 4-bit pair is
+// always places (0, 1) (two chains); a 3-bit pair cycles through (0, 1),
+// (2, 0), (1, 2).
+template <int B, int I>
+__host__ __device__ constexpr int place_acc() { return B == 4 ? (I & 1) : (I % 3); }
+
+// sum_i f_i G'[C + i] in packed fp32x2 FMAs (pair I to chain I % 2) and the
+// place sums in packed adds, over the N / 2 channel pairs of one group.
 template <int N, int B, int C, int... I>
-__device__ __forceinline__ void group_pairs(const uint32_t* run, const float* G, float2& acc, float2& gs,
-                                            std::integer_sequence<int, I...>) {
-  ((acc = __ffma2_rn(make_float2(code_float<N, B, 2 * I>(run), code_float<N, B, 2 * I + 1>(run)),
-                     make_float2(G[C + 2 * I], G[C + 2 * I + 1]), acc),
-    gs = __ffma2_rn(make_float2(code_g<B, 2 * I>(), code_g<B, 2 * I + 1>()),
-                    make_float2(G[C + 2 * I], G[C + 2 * I + 1]), gs)),
+__device__ __forceinline__ void group_pairs(const uint32_t* run, uint32_t one, const float* G, float2* acc,
+                                            float2* ps, std::integer_sequence<int, I...>) {
+  ((acc[I & 1] = __ffma2_rn(make_float2(code_float<N, B, 2 * I>(run, one), code_float<N, B, 2 * I + 1>(run, one)),
+                            make_float2(G[C + 2 * I], G[C + 2 * I + 1]), acc[I & 1]),
+    ps[place_acc<B, I>()] = __fadd2_rn(make_float2(G[C + 2 * I], G[C + 2 * I + 1]), ps[place_acc<B, I>()])),
    ...);
 }
 
@@ -133,16 +146,34 @@ __device__ __forceinline__ float group_dot(const uint32_t* w, uint32_t sh, float
   uint32_t run[NR];
 #pragma unroll
   for (int k = 0; k < NR; ++k) run[k] = (N * B) % 32 == 0 ? w[k] : __funnelshift_r(w[k], w[k + 1], sh);
-  float2 acc = make_float2(0.f, 0.f), gs = acc;
-  group_pairs<N, B, C>(run, G, acc, gs, std::make_integer_sequence<int, N / 2>{});
-  float a = acc.x + acc.y, g = gs.x + gs.y;
+  const uint32_t one = one_bits();
+  const float2 z = make_float2(0.f, 0.f);
+  float2 acc[2] = {z, z}, ps[3] = {z, z, z};
+  group_pairs<N, B, C>(run, one, G, acc, ps, std::make_integer_sequence<int, N / 2>{});
+  float a = (acc[0].x + acc[1].x) + (acc[0].y + acc[1].y);
+  // place sums S_0, S_1 (, S_2)
+  float S0, S1, S2 = 0.f;
+  if constexpr (B == 4) {
+    S0 = ps[0].x + ps[1].x;
+    S1 = ps[0].y + ps[1].y;
+  } else {
+    S0 = ps[0].x + ps[1].y;
+    S1 = ps[0].y + ps[2].x;
+    S2 = ps[1].x + ps[2].y;
+  }
   if constexpr (N % 2) {
+    constexpr int c = (N - 1) % tuple_len<B>();
     const float gl = G[C + N - 1];
-    a = fmaf(code_float<N, B, N - 1>(run), gl, a);
-    g = fmaf(code_g<B, N - 1>(), gl, g);
+    a = fmaf(code_float<N, B, N - 1>(run, one), gl, a);
+    if constexpr (c == 0) S0 += gl;
+    else if constexpr (c == 1) S1 += gl;
+    else S2 += gl;
   }
   constexpr float kf = (float)(1 << (tuple_len<B>() * B));
-  return scale * (a * kf - g);
+  constexpr float h = (float)(1 << (B - 1));
+  // 2^(B-1) sum_c 2^(c B) S_c
+  const float off = B == 4 ? h * fmaf(16.f, S1, S0) : h * fmaf(64.f, S2, fmaf(8.f, S1, S0));
+  return scale * fmaf(kf, a - ((S0 + S1) + S2), -off);
 }
 
 // TMEM -> registers: columns [C, R) of this warp's lane quarter, no wait.
@@ -260,13 +291,65 @@ __host__ __device__ constexpr int shape_lo(int k) {
 #undef STARKV_LO
 }
 
+// Unquantized bf16 key latents: kinds kHeadShapes + k hold R = 8 (k + 1)
+// channels, stored [slot][j] (2 R bytes per token, 16-byte aligned).  The W''
+// rows of these heads are not pre-scaled, so G holds the plain G columns and
+// the score is the dot of the bf16 latent with them: 16 channels per TMEM
+// load (a tail of 8), the bf16 pairs of a word split into two floats.
+constexpr int kBf16Kinds = 8;
+__host__ __device__ constexpr bool kind_is_bf16(int k) { return k >= kHeadShapes; }
+__host__ __device__ constexpr int bf16_kind_rank(int k) { return 8 * (k - kHeadShapes + 1); }
+
+template <int R, int C = 0>
+__device__ __forceinline__ float bf16_chunks(uint32_t taddr, const uint8_t* row) {
+  if constexpr (C >= R) {
+    return 0.f;
+  } else {
+    constexpr int N = R - C >= 16 ? 16 : 8;
+    float G[N];
+    tmem_cols<0, N>(taddr + (uint32_t)C, G);
+    uint32_t w[N / 2];
+    const uint4 a = *reinterpret_cast<const uint4*>(row + 2 * C);
+    w[0] = a.x; w[1] = a.y; w[2] = a.z; w[3] = a.w;
+    if constexpr (N == 16) {
+      const uint4 b = *reinterpret_cast<const uint4*>(row + 2 * C + 16);
+      w[4] = b.x; w[5] = b.y; w[6] = b.z; w[7] = b.w;
+    }
+    tc::tmem_ld_wait();
+    reg_fence<N>(G);
+    float2 acc[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+#pragma unroll
+    for (int k = 0; k < N / 2; ++k)
+      acc[k & 1] = __ffma2_rn(make_float2(__uint_as_float(w[k] << 16), __uint_as_float(w[k] & 0xFFFF0000u)),
+                              make_float2(G[2 * k], G[2 * k + 1]), acc[k & 1]);
+    return ((acc[0].x + acc[1].x) + (acc[0].y + acc[1].y)) + bf16_chunks<R, C + N>(taddr, row);
+  }
+}
+
+// One layer's heads are all quantized or all bf16, so each kernel instance
+// compiles only the kinds of its format (less code for the instruction cache).
+template <bool kBf16>
 __device__ __forceinline__ float head_score_any(uint32_t taddr, const uint8_t* blk, int kind, int slot) {
-  switch (kind) {
+  if constexpr (!kBf16) {
+    switch (kind) {
 #define STARKV_CASE(i, h, l) \
   case i: return head_score<h, l>(taddr, blk, slot);
-    STARKV_HEAD_SHAPES(STARKV_CASE)
+      STARKV_HEAD_SHAPES(STARKV_CASE)
 #undef STARKV_CASE
-    default: return 0.f;
+      default: return 0.f;
+    }
+  } else {
+    switch (kind) {
+      case kHeadShapes + 0: return bf16_chunks<8>(taddr, blk + slot * 16);
+      case kHeadShapes + 1: return bf16_chunks<16>(taddr, blk + slot * 32);
+      case kHeadShapes + 2: return bf16_chunks<24>(taddr, blk + slot * 48);
+      case kHeadShapes + 3: return bf16_chunks<32>(taddr, blk + slot * 64);
+      case kHeadShapes + 4: return bf16_chunks<40>(taddr, blk + slot * 80);
+      case kHeadShapes + 5: return bf16_chunks<48>(taddr, blk + slot * 96);
+      case kHeadShapes + 6: return bf16_chunks<56>(taddr, blk + slot * 112);
+      case kHeadShapes + 7: return bf16_chunks<64>(taddr, blk + slot * 128);
+      default: return 0.f;
+    }
   }
 }
 
@@ -290,16 +373,20 @@ constexpr int kMaxStages = 8;        // W'' and key-page stages
 constexpr int kMaxHeads = 64;
 
 
+// kDbg: write the raw scores to S_dbg instead of the softmax statistics.
+template <bool kDbg, bool kBf16>
 __global__ void __launch_bounds__(kScoreThreads, 1) k_scores_tc(ScoreArgs a) {
   extern __shared__ uint8_t smem_raw[];
   __shared__ __align__(8) uint64_t w_full[kMaxStages], w_empty[kMaxStages], k_full[kMaxStages], k_empty[kMaxStages], e_full,
       e_empty;
-  __shared__ __align__(8) uint64_t acc_full[4], acc_free[4], fin;
+  __shared__ __align__(8) uint64_t acc_full[kAccStages], acc_free[kAccStages], fin;
   __shared__ uint32_t tmem_base;
   __shared__ volatile int abort_flag;
   __shared__ ScoreItem items_s[64];
   __shared__ ScoreHead heads_s[kMaxHeads];
-  uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+  // 1024-byte aligned, derived from the shared array itself so that the
+  // compiler keeps the shared state space (plain LDS for the code words)
+  uint8_t* smem = smem_raw + ((1024u - (tc::smem_u32(smem_raw) & 1023u)) & 1023u);
   uint8_t* E_s = smem;                                   // 2 x 32 KB
   uint8_t* W_s = E_s + 2 * kETileBytes;                  // WS x w_stage
   uint8_t* K_s = W_s + (size_t)a.WS * a.w_stage;         // KS x k_stage
@@ -316,7 +403,7 @@ __global__ void __launch_bounds__(kScoreThreads, 1) k_scores_tc(ScoreArgs a) {
     }
     tc::mbar_init(&e_full, 1);
     tc::mbar_init(&e_empty, 2);
-    for (int s = 0; s < 4; ++s) {
+    for (int s = 0; s < kAccStages; ++s) {
       tc::mbar_init(&acc_full[s], 1);
       tc::mbar_init(&acc_free[s], 4);
     }
@@ -377,7 +464,7 @@ __global__ void __launch_bounds__(kScoreThreads, 1) k_scores_tc(ScoreArgs a) {
         }
         bool ok = true;
         if (lane == 0) {
-          ok = tc::mbar_wait_ab(&k_empty[ks], kph ^ 1u, a.status, &abort_flag);
+          ok = tc::mbar_wait_ab_lazy(&k_empty[ks], kph ^ 1u, a.status, &abort_flag);
           if (ok) tc::mbar_expect_tx(&k_full[ks], (uint32_t)(npg * item.key_bytes));
         }
         ok = __shfl_sync(0xffffffffu, ok, 0);
@@ -413,7 +500,7 @@ __global__ void __launch_bounds__(kScoreThreads, 1) k_scores_tc(ScoreArgs a) {
         if (t0 >= len) continue;
         bool ok = true;
         if (st != cur_st) {
-          ok = tc::mbar_wait_ab(&e_empty, ((uint32_t)ne & 1u) ^ 1u, a.status, &abort_flag);
+          ok = tc::mbar_wait_ab_lazy(&e_empty, ((uint32_t)ne & 1u) ^ 1u, a.status, &abort_flag);
           if (!ok) break;
           tc::mbar_expect_tx(&e_full, 2 * kETileBytes);
           for (int k = 0; k < 2; ++k)
@@ -429,7 +516,7 @@ __global__ void __launch_bounds__(kScoreThreads, 1) k_scores_tc(ScoreArgs a) {
             ws_n = 0;
             wph_n ^= 1u;
           }
-          ok = tc::mbar_wait_ab(&w_empty[ws], wph ^ 1u, a.status, &abort_flag);
+          ok = tc::mbar_wait_ab_lazy(&w_empty[ws], wph ^ 1u, a.status, &abort_flag);
           if (!ok) break;
           tc::mbar_expect_tx(&w_full[ws], (uint32_t)(item.npad * 256));
           tc::bulk_g2s(W_s + (size_t)ws * a.w_stage, a.W + (size_t)b * a.w_stride + item.w_off,
@@ -446,7 +533,7 @@ __global__ void __launch_bounds__(kScoreThreads, 1) k_scores_tc(ScoreArgs a) {
   } else if (warp == 1 || warp == kMma2Warp) {
     // ------------------------------------------------------------ MMA issue
     // warp 1 issues tile 0 and warp kMma2Warp tile 1 of every item: job
-    // j = 2 i + tile in accumulator stage j % 4.  Both wait for the item's
+    // j = 2 i + tile in accumulator stage j % kAccStages.  Both wait for the item's
     // W'' stage and release it (w_empty counts two commits); both release the
     // RoPE tiles when the position changes.
     const int tile = warp == 1 ? 0 : 1;
@@ -482,22 +569,23 @@ __global__ void __launch_bounds__(kScoreThreads, 1) k_scores_tc(ScoreArgs a) {
             wph_n ^= 1u;
           }
           if (!tc::mbar_wait_ab(&w_full[ws], wph, a.status, &abort_flag)) { abort_flag = 1; break; }
-          const uint32_t idesc = tc::idesc_f16(128, npad, false, false, false);
           // descriptors as (low, high) halves, stepped in 16-byte units on the low half
           const uint32_t w_lo = w_lo0 + (uint32_t)ws * ((uint32_t)a.w_stage >> 4);
           const uint32_t watom = (uint32_t)npad * 8u;   // one 64-column K atom of W'': npad rows x 128 B
           const int j = 2 * i + tile;
-          if (!tc::mbar_wait_ab(&acc_free[j & 3], (((uint32_t)(j >> 2)) & 1u) ^ 1u, a.status, &abort_flag)) {
+          const int stg = j % kAccStages;
+          if (!tc::mbar_wait_ab(&acc_free[stg], (((uint32_t)(j / kAccStages)) & 1u) ^ 1u, a.status, &abort_flag)) {
             abort_flag = 1;
             break;
           }
           tc::tc_fence_after();
-          const uint32_t d = tmem + (uint32_t)((j & 3) * 128);
+          const uint32_t idesc = tc::idesc_f16(128, npad, false, false, false);
+          const uint32_t d = tmem + (uint32_t)(stg * kItemCols);
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk)
             tc::mma_f16_ss2(d, e_lo + (uint32_t)(kk >> 2) * 1024u + (uint32_t)(kk & 3) * 2u, sw_hi,
                             w_lo + (uint32_t)(kk >> 2) * watom + (uint32_t)(kk & 3) * 2u, sw_hi, idesc, kk ? 1u : 0u);
-          tc::mma_commit(&acc_full[j & 3]);
+          tc::mma_commit(&acc_full[stg]);
           tc::mma_commit(&w_empty[ws]);
         }
       }
@@ -507,8 +595,8 @@ __global__ void __launch_bounds__(kScoreThreads, 1) k_scores_tc(ScoreArgs a) {
   } else {
     // ------------------------------------------------------------ epilogue
     // Job j = 2 i + tile (tile `tile` of item i) sits in accumulator stage
-    // j % 4; set `set` (4 warps, one per TMEM lane quarter) takes the jobs
-    // with j % 4 == set.  Warp q scores tokens tile * 128 + q * 32 + lane of
+    // j % kAccStages; set `set` (4 warps, one per TMEM lane quarter) takes
+    // the jobs with j % 4 == set.  Warp q scores tokens tile * 128 + q * 32 + lane of
     // the super-tile, which are exactly one 32-token softmax group.
     const int e = warp - 3;              // 0..15
     const int set = e >> 2;
@@ -541,33 +629,35 @@ __global__ void __launch_bounds__(kScoreThreads, 1) k_scores_tc(ScoreArgs a) {
         if ((i & 1) != ipar) continue;
         const ScoreItem& item = items_s[it];
         const int j = 2 * i + tile;
+        const int stg = j % kAccStages;
+        const int nh = item.nh;
         const bool ok = tc::mbar_wait_ab(&k_full[ks], kph, a.status, &abort_flag) &&
-                        tc::mbar_wait_ab(&acc_full[set], ((uint32_t)(j >> 2)) & 1u, a.status, &abort_flag);
+                        tc::mbar_wait_ab(&acc_full[stg], ((uint32_t)(j / kAccStages)) & 1u, a.status, &abort_flag);
         tc::tc_fence_after();
-        if (ok) {
-          const uint8_t* page = K_s + (size_t)ks * a.k_stage + (size_t)pg * item.key_bytes;
-          const uint32_t trow = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(set * 128);
-          const size_t row0 = (size_t)b * a.H + item.h0;
-          __half* prow = a.P + row0 * a.P_ld + t;                          // this token's P of the item's first head
-          float* mrow = a.m_st + row0 * a.n_g + (t0 >> 5) + grp32;
-          for (int hh = 0; hh < item.nh; ++hh, prow += a.P_ld, mrow += a.n_g) {
+        const uint8_t* page = K_s + (size_t)ks * a.k_stage + (size_t)pg * item.key_bytes;
+        const uint32_t trow = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(stg * kItemCols);
+        const size_t row0 = (size_t)b * a.H + item.h0;
+        __half* prow = a.P + row0 * a.P_ld + t;                          // this token's P of the item's first head
+        float* mrow = a.m_st + row0 * a.n_g + (t0 >> 5) + grp32;
+        for (int hh = 0; hh < nh; ++hh, prow += a.P_ld, mrow += a.n_g) {
+          if (ok) {
             const ScoreHead& hd = heads_s[item.h0 + hh];
-            const float sv = head_score_any(trow + (uint32_t)hd.gcol, page + hd.blk_rel, hd.kind, slot);
-            if (a.S_dbg) {
+            const float sv = head_score_any<kBf16>(trow + (uint32_t)hd.gcol, page + hd.blk_rel, hd.kind, slot);
+            if constexpr (kDbg) {
               if (valid) a.S_dbg[(row0 + hh) * a.P_ld + t] = sv;
-              continue;
+            } else {
+              // softmax statistics of the 32-token group: m = max s and P =
+              // exp2(s - m) rounded to fp16 (the value kernel sums the P it uses)
+              const float m = warp_max(valid ? sv : -FLT_MAX);
+              if (valid) *prow = __float2half_rn(ex2_approx(sv - m));
+              if (lane == 0) *mrow = m;
             }
-            // softmax statistics of the 32-token group: m = max s and P =
-            // exp2(s - m) rounded to fp16 (the value kernel sums the P it uses)
-            const float m = warp_max(valid ? sv : -FLT_MAX);
-            if (valid) *prow = __float2half_rn(ex2_approx(sv - m));
-            if (lane == 0) *mrow = m;
           }
         }
         tc::tc_fence_before();
         __syncwarp();
         if (lane == 0) {
-          tc::mbar_arrive(&acc_free[set]);
+          tc::mbar_arrive(&acc_free[stg]);
           tc::mbar_arrive(&k_empty[ks]);
         }
       }
@@ -603,7 +693,10 @@ __global__ void __launch_bounds__(512) k_qprep_tc(LayerView v, const __nv_bfloat
       if (row >= item.hcol[x] && row < item.hcol[x] + item.hr[x]) hh = x;
     row_head[row] = hh;
   }
-  if (threadIdx.x < item.nh) nhi_s[threadIdx.x] = shape_hi(heads[item.h0 + threadIdx.x].kind);
+  if (threadIdx.x < item.nh) {
+    const int k = heads[item.h0 + threadIdx.x].kind;
+    nhi_s[threadIdx.x] = kind_is_bf16(k) ? -1 : shape_hi(k);   // -1: bf16 latent, no pre-scale
+  }
   const int pos = q_pos ? q_pos[b] : seq_lens[b] - 1;
   for (int idx = threadIdx.x; idx < item.nh * 64; idx += blockDim.x) {
     const int hh = idx / 64, p = idx % 64;
@@ -630,8 +723,9 @@ __global__ void __launch_bounds__(512) k_qprep_tc(LayerView v, const __nv_bfloat
       const int h = item.h0 + hh, g = h / v.group_q, j = row - item.hcol[hh];
       // pre-scale 2^(-c B) of the channel's place c in its code tuple (see code_float)
       const int nhi = nhi_s[hh];
-      const float pre = j < nhi ? ((j % 32) % 2 ? 1.f / 16.f : 1.f)
-                                : (((j - nhi) % 32) % 3 == 0 ? 1.f : ((j - nhi) % 32) % 3 == 1 ? 1.f / 8.f : 1.f / 64.f);
+      const float pre = nhi < 0 ? 1.f
+                        : j < nhi ? ((j % 32) % 2 ? 1.f / 16.f : 1.f)
+                                  : (((j - nhi) % 32) % 3 == 0 ? 1.f : ((j - nhi) % 32) % 3 == 1 ? 1.f / 8.f : 1.f / 64.f);
       const float* B = Bk + ((size_t)key_off[g] + j) * 128 + c * 8;
       const float4 x0 = *reinterpret_cast<const float4*>(B), x1 = *reinterpret_cast<const float4*>(B + 4);
       const float4 y0 = *reinterpret_cast<const float4*>(B + 64), y1 = *reinterpret_cast<const float4*>(B + 68);
@@ -679,14 +773,19 @@ __global__ void k_rope_table(float log2_theta, int n_tiles, uint8_t* __restrict_
 bool plan_scores_tc(starkv_layer* L) {
   const LayerView& v = L->view;
   const starkv_layer_config& c = L->cfg;
-  if (c.dtype != STARKV_BF16 || c.plain || !c.rope || c.head_dim != 128 || !v.quantized) return false;
+  if (c.dtype != STARKV_BF16 || c.plain || !c.rope || c.head_dim != 128) return false;
   if (c.n_heads > kMaxHeads) return false;
   // Every key latent must have one of the compiled head shapes: NHI 4-bit
   // channels then NLO 3-bit channels, each segment cut into groups of 32 from
-  // its start.
+  // its start; or, unquantized, a bf16 latent of 8 .. 64 channels (a multiple of 8).
   std::vector<int> kv_kind(v.Hkv, -1);
   for (int g = 0; g < v.Hkv; ++g) {
     const LatentDesc& ld = L->lat[g];
+    if (!v.quantized) {
+      if (ld.n_groups != 1 || ld.width % 8 != 0 || ld.width < 8 || ld.width > 8 * kBf16Kinds) return false;
+      kv_kind[g] = kHeadShapes + ld.width / 8 - 1;
+      continue;
+    }
     if (ld.n_groups > 4) return false;
     for (int k = 0; k < kHeadShapes && kv_kind[g] < 0; ++k) {
       const int nhi = shape_hi(k), nlo = shape_lo(k);
@@ -705,6 +804,10 @@ bool plan_scores_tc(starkv_layer* L) {
   }
   L->items.clear();
   L->score_heads.assign(v.H, ScoreHead{});
+  // bf16 key latents take 2 bytes per channel and token: an item's key range
+  // is kept to 2 KB per page, so that a 16-page key stage is 32 KB and
+  // several stages fit (query heads that share a KV head share its range)
+  const int max_item_key = v.quantized ? (1 << 30) : 2048;
   int w_off = 0, max_key = 0, max_w = 0;
   int h = 0;
   while (h < v.H) {
@@ -713,7 +816,9 @@ bool plan_scores_tc(starkv_layer* L) {
     int cols = 0;
     while (h < v.H && it.nh < kMaxItemHeads) {
       const int r = L->lat[h / v.group_q].width;
-      if (cols + r > 128) break;
+      if (cols + r > kItemCols) break;
+      const int g0 = it.h0 / v.group_q, g = h / v.group_q;
+      if (it.nh > 0 && L->lat[g + 1].block_off - L->lat[g0].block_off > max_item_key) break;
       it.hr[it.nh] = r;
       it.hcol[it.nh++] = cols;
       cols += r;
@@ -745,7 +850,14 @@ bool plan_scores_tc(starkv_layer* L) {
   // dynamic shared memory: what the opt-in limit leaves beside the static
   // tables and barriers, less the alignment slack and the two RoPE tiles
   cudaFuncAttributes fa;
-  if (cudaFuncGetAttributes(&fa, k_scores_tc) != cudaSuccess) return false;
+  const void* fns[4] = {(const void*)k_scores_tc<false, false>, (const void*)k_scores_tc<true, false>,
+                        (const void*)k_scores_tc<false, true>, (const void*)k_scores_tc<true, true>};
+  fa.sharedSizeBytes = 0;
+  for (const void* fn : fns) {
+    cudaFuncAttributes f1;
+    if (cudaFuncGetAttributes(&f1, fn) != cudaSuccess) return false;
+    fa.sharedSizeBytes = std::max(fa.sharedSizeBytes, f1.sharedSizeBytes);
+  }
   const long long budget = 232448LL - (long long)fa.sharedSizeBytes - 1024 - 2LL * kETileBytes;
   // Two W'' stages (read from L2, short latency) and as many key stages as fit:
   // the key copies read HBM and need the most bytes in flight.
@@ -823,10 +935,20 @@ cudaError_t launch_scores_tc(const starkv_layer* L, const uint8_t* pool, long lo
   a.KS = L->KS;
   a.status = L->status;
   const size_t smem = 2 * kETileBytes + (size_t)a.WS * a.w_stage + (size_t)a.KS * a.k_stage + 1024;
-  e = set_smem_limit((const void*)k_scores_tc, smem);
+  const bool bf = !v.quantized;
+  const void* fn = S_dbg ? (bf ? (const void*)k_scores_tc<true, true> : (const void*)k_scores_tc<true, false>)
+                         : (bf ? (const void*)k_scores_tc<false, true> : (const void*)k_scores_tc<false, false>);
+  e = set_smem_limit(fn, smem);
   if (e != cudaSuccess) return e;
   const int G = (int)std::min<long long>(num_sms(), a.U);
-  k_scores_tc<<<G, kScoreThreads, smem, s>>>(a);
+  if (S_dbg && bf)
+    k_scores_tc<true, true><<<G, kScoreThreads, smem, s>>>(a);
+  else if (S_dbg)
+    k_scores_tc<true, false><<<G, kScoreThreads, smem, s>>>(a);
+  else if (bf)
+    k_scores_tc<false, true><<<G, kScoreThreads, smem, s>>>(a);
+  else
+    k_scores_tc<false, false><<<G, kScoreThreads, smem, s>>>(a);
   return cudaGetLastError();
 }
 

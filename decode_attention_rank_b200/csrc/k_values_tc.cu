@@ -127,9 +127,19 @@ __device__ __forceinline__ void deq_channel3(uint64_t x, __half2 sub, const uint
   }
 }
 
+// An unquantized bf16 value latent is stored channel-major too: channel j's
+// 16 tokens are 32 contiguous bytes.  Word c holds slots 2c and 2c + 1, which
+// become one fp16 pair of the A tile row (bf16 -> fp32 is exact, fp32 -> fp16
+// rounds to nearest; the latents are far inside the fp16 range).
+__device__ __forceinline__ uint32_t bf16x2_to_f16x2(uint32_t w) {
+  const __half2 h = __floats2half2_rn(__uint_as_float(w << 16), __uint_as_float(w & 0xFFFF0000u));
+  return *reinterpret_cast<const uint32_t*>(&h);
+}
+
 // NBT: 128-channel blocks per team (the value latent has 128 * nblk channels,
-// team j owns blocks j + 4 i, i < NBT).
-template <int NBT>
+// team j owns blocks j + 4 i, i < NBT).  BF16: the value latent is unquantized
+// bf16 instead of 4/3-bit codes.
+template <int NBT, bool BF16>
 __global__ void __launch_bounds__(kValThreads, 1) k_values_tc(ValArgs a) {
   extern __shared__ uint8_t smem_raw[];
   __shared__ __align__(8) uint64_t t_full[kTeams][kMaxASlots], t_free[kTeams][kMaxASlots], t_seg[kTeams],
@@ -177,7 +187,7 @@ __global__ void __launch_bounds__(kValThreads, 1) k_values_tc(ValArgs a) {
     abort_flag = 0;
     tc::fence_mbar_init();
   }
-  for (int g = threadIdx.x; g < a.rv / 32; g += blockDim.x) {
+  for (int g = threadIdx.x; g < (BF16 ? 0 : a.rv / 32); g += blockDim.x) {
     const int bits = a.vgrp[g].bits;
     const float offm = 1024.f + (float)(1 << (bits - 1));
     const __half2 sub = __floats2half2_rn(offm, offm);
@@ -266,7 +276,7 @@ __global__ void __launch_bounds__(kValThreads, 1) k_values_tc(ValArgs a) {
       for (int pg = 0; pg < n_pg; ++pg) {
         const uint32_t rsp = rsp_s[pg];
         const int rs = (int)(rsp & 127u);
-        if (!tc::mbar_wait_ab(&r_empty[rs], (rsp >> 7) ^ 1u, a.status, &abort_flag)) break;
+        if (!tc::mbar_wait_ab_lazy(&r_empty[rs], (rsp >> 7) ^ 1u, a.status, &abort_flag)) break;
         const int page = pid_s[pg >> 3][pg & 7];
         tc::mbar_expect_tx(&r_full[rs], page >= 0 ? (uint32_t)a.vblk_bytes : 0u);
         if (page >= 0)
@@ -518,6 +528,26 @@ __global__ void __launch_bounds__(kValThreads, 1) k_values_tc(ValArgs a) {
           for (int i = 0; i < NBT; ++i) {
             if (i >= nbt) break;
             const int g = (j + 4 * i) * 4 + q;
+            if constexpr (BF16) {
+#pragma unroll
+              for (int e = 0; e < 2; ++e) {
+                const uint8_t* row = R_s + (size_t)(e ? rs1 : rs0) * a.raw_stage + (size_t)(g * 32 + lane) * 32;
+                uint32_t out[8];
+                if (e ? valid1 : valid0) {
+                  const uint4 w0 = *reinterpret_cast<const uint4*>(row);
+                  const uint4 w1 = *reinterpret_cast<const uint4*>(row + 16);
+                  out[0] = bf16x2_to_f16x2(w0.x); out[1] = bf16x2_to_f16x2(w0.y);
+                  out[2] = bf16x2_to_f16x2(w0.z); out[3] = bf16x2_to_f16x2(w0.w);
+                  out[4] = bf16x2_to_f16x2(w1.x); out[5] = bf16x2_to_f16x2(w1.y);
+                  out[6] = bf16x2_to_f16x2(w1.z); out[7] = bf16x2_to_f16x2(w1.w);
+                } else {
+#pragma unroll
+                  for (int x = 0; x < 8; ++x) out[x] = 0u;
+                }
+                tc::tmem_st8(tmem + lane_base + slot_col + (uint32_t)(i * 16 + e * 8), out);
+              }
+              continue;
+            }
             const int4 vg = vg_s[g];
             const __half2 sub = *reinterpret_cast<const __half2*>(&vg.z);
 #pragma unroll
@@ -705,20 +735,27 @@ bool plan_values_tc(starkv_layer* L) {
   L->val_na = std::min(kMaxASlots, (512 - nblk * v.H) / (n_teams * nbt * 16));   // slots of two pages
   if (L->val_na < 2) return false;
   const LatentDesc& ld = L->lat[v.L - 1];
-  if (ld.n_groups * 32 != v.rv || !ld.cmajor) return false;
-  for (int g = 0; g < ld.n_groups; ++g) {
-    const GroupDesc& gd = L->grp[ld.group0 + g];
-    if (gd.n != 32 || (gd.bits != 3 && gd.bits != 4) || gd.start != g * 32) return false;
+  if (!ld.cmajor) return false;
+  size_t bytes = 0;
+  if (v.quantized) {
+    if (ld.n_groups * 32 != v.rv) return false;
+    for (int g = 0; g < ld.n_groups; ++g) {
+      const GroupDesc& gd = L->grp[ld.group0 + g];
+      if (gd.n != 32 || (gd.bits != 3 && gd.bits != 4) || gd.start != g * 32) return false;
+    }
+    // bytes of the value block: scales + code blocks
+    bytes = ld.scale_bytes;
+    for (int g = 0; g < ld.n_groups; ++g) bytes += (size_t)kPage * 32 * L->grp[ld.group0 + g].bits / 8;
+  } else {
+    if (c.dtype != STARKV_BF16 || ld.n_groups != 1) return false;
+    bytes = (size_t)kPage * v.rv * 2;   // [channel][slot] bf16
   }
-  (void)c;
+  L->val_bf16 = !v.quantized;
   L->vblk_off = ld.block_off;
-  // bytes of the value block: scales + code blocks
-  size_t bytes = ld.scale_bytes;
-  for (int g = 0; g < ld.n_groups; ++g) bytes += (size_t)kPage * 32 * L->grp[ld.group0 + g].bits / 8;
   L->vblk_bytes = (int)bytes;
   // as many raw stages as fit next to the static tables and barriers
   cudaFuncAttributes fa;
-  if (cudaFuncGetAttributes(&fa, k_values_tc<2>) != cudaSuccess) return false;
+  if (cudaFuncGetAttributes(&fa, k_values_tc<2, false>) != cudaSuccess) return false;
   const int min_raw = 4;
   L->val_raw = 0;
   for (int n_raw = kMaxRawStages; n_raw >= min_raw && !L->val_raw; --n_raw)
@@ -779,13 +816,19 @@ cudaError_t launch_values_tc(const starkv_layer* L, const uint8_t* pool, long lo
   a.status = L->status;
   const size_t smem = values_smem(v.H, L->vblk_bytes, L->val_raw);
   const bool two = v.rv / 128 > kTeams;   // two channel blocks per team
-  const void* kern = two ? (const void*)k_values_tc<2> : (const void*)k_values_tc<1>;
+  const bool bf = L->val_bf16;
+  const void* kern = two ? (bf ? (const void*)k_values_tc<2, true> : (const void*)k_values_tc<2, false>)
+                         : (bf ? (const void*)k_values_tc<1, true> : (const void*)k_values_tc<1, false>);
   cudaError_t e = set_smem_limit(kern, smem);
   if (e != cudaSuccess) return e;
-  if (two)
-    k_values_tc<2><<<G, kValThreads, smem, s>>>(a);
+  if (two && bf)
+    k_values_tc<2, true><<<G, kValThreads, smem, s>>>(a);
+  else if (two)
+    k_values_tc<2, false><<<G, kValThreads, smem, s>>>(a);
+  else if (bf)
+    k_values_tc<1, true><<<G, kValThreads, smem, s>>>(a);
   else
-    k_values_tc<1><<<G, kValThreads, smem, s>>>(a);
+    k_values_tc<1, false><<<G, kValThreads, smem, s>>>(a);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   if (ev_mid && (e = cudaEventRecord(ev_mid, s)) != cudaSuccess) return e;

@@ -30,7 +30,7 @@ struct LatentDesc {
   int group0;       // index of the first group in the group table
   int ch_off;       // offset of this latent in the concatenated latent vector
   int scale_bytes;  // bytes of the scale block (0 when unquantized)
-  int cmajor;       // 1: code blocks channel-major (the quantized value latent), see code_bit
+  int cmajor;       // 1: channel-major (the value latent of a latent layer), see code_bit and elem_index
 };
 
 constexpr int kPage = 16;
@@ -44,6 +44,14 @@ constexpr int kPage = 16;
 __host__ __device__ __forceinline__ uint32_t code_bit(int slot, int i, int n, int bits, int cmajor) {
   return cmajor ? (uint32_t)(i * kPage + (slot & 1) * (kPage / 2) + (slot >> 1)) * (uint32_t)bits
                 : (uint32_t)(slot * n + i) * (uint32_t)bits;
+}
+
+// Element index of (slot, channel j) inside an unquantized latent block of
+// `width` channels: slot-major [slot][j], or channel-major [j][slot] (the
+// value latent of a latent layer, so that one channel's 16 tokens are
+// contiguous for the value contraction).
+__host__ __device__ __forceinline__ size_t elem_index(int slot, int j, int width, int cmajor) {
+  return cmajor ? (size_t)j * kPage + slot : (size_t)slot * width + j;
 }
 
 // Device status bits (mirror of STARKV_DEV_* in the public header).
@@ -73,6 +81,28 @@ struct LayerView {
   const GroupDesc* grp;
   uint32_t* status;
 };
+
+// Stored value of channel j of latent `ld` for token slot `slot` of a page block.
+__device__ __forceinline__ float latent_value(const LayerView& v, const uint8_t* blk, const LatentDesc& ld,
+                                              int slot, int j) {
+  if (!v.quantized) {
+    const size_t o = elem_index(slot, j, ld.width, ld.cmajor);
+    return v.es == 4 ? reinterpret_cast<const float*>(blk)[o]
+                     : __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(blk)[o]);
+  }
+  int g = 0;
+  for (int k = 1; k < ld.n_groups; ++k)
+    if (j >= v.grp[ld.group0 + k].start) g = k;
+  const GroupDesc gd = v.grp[ld.group0 + g];
+  const float s = __half2float(reinterpret_cast<const __half*>(blk)[g * kPage + slot]);
+  const uint32_t bit = code_bit(slot, j - gd.start, gd.n, gd.bits, ld.cmajor);
+  const uint32_t* w = reinterpret_cast<const uint32_t*>(blk + gd.code_off) + (bit >> 5);
+  const uint32_t sh = bit & 31;
+  uint32_t u = w[0] >> sh;
+  if (sh + gd.bits > 32) u |= w[1] << (32 - sh);
+  u &= (1u << gd.bits) - 1u;
+  return (float)((int)u - (1 << (gd.bits - 1))) * s;
+}
 
 // One MMA item of the tensor-core score kernel: consecutive query heads whose
 // W'' rows (sum of ranks <= 128) form the B operand of one 128 x npad MMA.
@@ -151,6 +181,7 @@ struct starkv_layer {
   int vblk_off = 0, vblk_bytes = 0;
   int val_raw = 0;              // raw page stages of the value kernel
   int val_na = 0;               // pages of A tiles the value kernel keeps in TMEM
+  bool val_bf16 = false;        // the value latent is unquantized bf16 (channel-major)
   // optional per-kernel timing of the tensor-core decode: prof_n sets of
   // STARKV_N_PHASES + 1 events, the decode call number prof_calls picks the set
   std::vector<cudaEvent_t> prof_ev;
@@ -235,7 +266,13 @@ cudaError_t launch_gemm_tc(const uint8_t* Mt, int n_out, int K, int n_valid, con
                            void* out, bool out_f32, float* part, uint32_t* status, cudaStream_t s, int y_group = 0);
 // Rows of a bf16 matrix as fp16 swizzled tiles of nb rows x 64 columns (nb = 0: the B-tile height for `rows`).
 cudaError_t launch_pack_rows_tiles(const void* x, int rows, int K, void* tiles, cudaStream_t s, int nb = 0);
-cudaError_t launch_pack_rows_tiles_f32(const float* x, int rows, int K, void* tiles, cudaStream_t s);
+cudaError_t launch_pack_rows_tiles_f32(const float* x, int rows, int K, void* tiles, cudaStream_t s, int nb = 0);
+// Tensor-core causal prefill (k_prefill.cu): one chunk of one sequence.
+bool prefill_flash_supported(const starkv_layer* L);
+size_t prefill_flash_ws_bytes(const starkv_layer* L, int max_T, int max_q);
+cudaError_t launch_prefill_flash(const starkv_layer* L, const uint8_t* pool, long long n_pages, const int32_t* pt_row,
+                                 int q_start, int q_len, const void* q, void* out, void* ws, int max_T, int max_q,
+                                 cudaStream_t s);
 // Unfused output factors: B'_v,kv(h) per query head as 128 x 64 fp16 tiles [H][r_v / 64], and W_o^T
 // as tiles [Dp / 128][H d / 64] (built from the same inputs as M).
 cudaError_t launch_build_unfused(starkv_layer* L, const float* Bv_rot, const void* W_o, cudaStream_t s);

@@ -81,13 +81,18 @@ __device__ __forceinline__ bool mbar_test_wait(uint64_t* bar, uint32_t parity) {
 // is polled with a suspending try_wait until `limit_ns` of the global timer
 // have passed.
 static __device__ __noinline__ bool mbar_wait_slow(uint64_t* bar, uint32_t parity, uint32_t* status, volatile int* abort,
-                                                   unsigned long long limit_ns = kWaitLimitNs) {
+                                                   unsigned long long limit_ns = kWaitLimitNs, uint32_t nap_ns = 0) {
   if (mbar_try_wait(bar, parity)) return true;
   const unsigned long long t0 = global_ns();
-  for (uint32_t i = 1;; ++i) {
-    if (mbar_try_wait(bar, parity)) return true;
+  for (;;) {
+    // eight polls between checks of the abort flag and the clock
+#pragma unroll 1
+    for (int k = 0; k < 8; ++k) {
+      if (mbar_try_wait(bar, parity)) return true;
+      if (nap_ns) __nanosleep(nap_ns);
+    }
     if (abort && *abort) return false;
-    if ((i & 15u) == 0u && global_ns() - t0 > limit_ns) break;
+    if (global_ns() - t0 > limit_ns) break;
   }
   if (status) atomicOr(status, kTimeout);
   if (abort) *abort = 1;
@@ -107,6 +112,15 @@ __device__ __forceinline__ bool mbar_wait_ab(uint64_t* bar, uint32_t parity, uin
                                              volatile int* abort) {
   if (mbar_test_wait(bar, parity)) return true;
   return mbar_wait_slow(bar, parity, status, abort);
+}
+
+// The same for a role whose wait is not on the critical path (a copy warp
+// several stages ahead): it naps between polls, so it takes fewer issue
+// slots from the warps that share its scheduler.
+__device__ __forceinline__ bool mbar_wait_ab_lazy(uint64_t* bar, uint32_t parity, uint32_t* status,
+                                                  volatile int* abort) {
+  if (mbar_test_wait(bar, parity)) return true;
+  return mbar_wait_slow(bar, parity, status, abort, kWaitLimitNs, 256);
 }
 
 // ---- bulk copies (global -> shared, completion on an mbarrier) -------------

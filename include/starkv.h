@@ -218,15 +218,21 @@ STARKV_API starkv_status starkv_decode_attn(const starkv_layer* layer, const voi
  * appended).  Sequence b has q_len[b] queries at positions q_start[b] ..
  * q_start[b] + q_len[b] - 1; query i attends to slots [0, q_start[b] + i].
  *   q_start_host, q_len_host: HOST int32 arrays [batch] (they set the launch shape).
- *     The per-row table built from them is copied from pageable host memory,
- *     so this call synchronises `stream` before it returns.
  *   q: [sum q_len][H][d] in dtype, sequences one after another; out: [sum q_len][D].
  *   workspace: at least starkv_workspace_bytes(layer, batch, max_ctx, max q_len)
- *     bytes, where max_ctx >= every q_start[b] + q_len[b].  Layers that the
- *     tensor-core kernels take (bf16, RoPE, quantized, compiled head shapes)
- *     run every query row through them, 256 rows at a time, when max_ctx is the
- *     page table's capacity (max_pages * 16); a workspace sized for a shorter
- *     max_ctx runs the CUDA-core kernels instead.
+ *     bytes, where max_ctx >= every q_start[b] + q_len[b].
+ * Paths, in order of preference:
+ *   - bf16 layers with head_dim 128 (plain layers; compressed layers that the
+ *     tensor-core decode takes, with key ranks <= 64 and positions inside
+ *     the RoPE table): per sequence the chunk's keys and values are rebuilt
+ *     once (K = RoPE(Zhat_k B'_k), V = Zhat_v B'_v, section 5.3 of the
+ *     reading notes), then tiled causal attention and the output through W_o,
+ *     all on the tensor cores.  Asynchronous on `stream`.
+ *   - other tensor-core layers: every query row as a decode row, 256 rows at a
+ *     time, when max_ctx is the page table's capacity (max_pages * 16).
+ *   - the CUDA-core kernels otherwise.
+ *   The last two copy a per-row table from pageable host memory and
+ *   synchronise `stream` before returning.
  */
 STARKV_API starkv_status starkv_prefill_attn(const starkv_layer* layer, const void* pool, int64_t n_pages,
                                   const int32_t* page_table, int max_pages, int batch, const int32_t* q_start_host,

@@ -204,7 +204,10 @@ def dequantize_group(u: np.ndarray, s16: np.float16, bits: int) -> np.ndarray:
 #
 #   page = latent block 0 | latent block 1 | ... | latent block L-1 | pad to 128 B
 #   latents in order: key latent of KV head 0 .. H_kv-1, then the joint value latent
-#   unquantized block: element (slot, j) at byte (slot * r + j) * elem_size; pad to 16 B
+#   unquantized block: element (slot, j) at byte (slot * r + j) * elem_size (key
+#                      latents, and every latent of a plain layer), or at byte
+#                      (j * P + slot) * elem_size (the value latent of a latent
+#                      layer: channel-major); pad to 16 B
 #   quantized block:   scales [group][slot] fp16, pad to 16 B; then for each group g
 #                      a code block of P * n_g * b_g bits, pad to 16 B, a bitstream
 #                      written least significant bit first (stream bit k is bit
@@ -277,7 +280,8 @@ def pack_block(Z: np.ndarray, r: int, spec, channel_major: bool = False) -> np.n
 
     Rows of Z that are NaN-free are written; a slot that holds no token should
     be passed as None rows (see `pack_page`), which leaves its bytes zero.
-    channel_major selects the value latent's code order (see the page format above).
+    channel_major selects the value latent's order (see the page format above):
+    codes by `code_bit`, unquantized elements [channel][slot].
     """
     P = spec.page_size
     out = np.zeros(block_bytes(r, spec), dtype=np.uint8)
@@ -287,12 +291,18 @@ def pack_block(Z: np.ndarray, r: int, spec, channel_major: bool = False) -> np.n
         else:
             vals = bf16_round(Z).view(np.uint32) >> np.uint32(16)
             vals = vals.astype(np.uint16)
+        es = elem_size(spec)
         for slot in range(P):
             if Z[slot] is None or np.isnan(np.asarray(Z[slot], dtype=np.float64)).any():
                 continue
-            row = vals[slot].view(np.uint8)
-            o = slot * r * elem_size(spec)
-            out[o:o + row.size] = row
+            if channel_major:
+                for j in range(r):
+                    o = (j * P + slot) * es
+                    out[o:o + es] = vals[slot][j:j + 1].view(np.uint8)
+            else:
+                row = vals[slot].view(np.uint8)
+                o = slot * r * es
+                out[o:o + row.size] = row
         return out
     gs = groups(r, spec)
     scale_bytes = _ru(len(gs) * P * 2, 16)
@@ -327,7 +337,8 @@ def pack_page(latents_per_slot, spec) -> np.ndarray:
         for slot in range(P):
             if latents_per_slot[slot] is not None:
                 Z[slot] = latents_per_slot[slot][li]
-        blk = pack_block(Z, r, spec, channel_major=(li == len(spec.latent_widths) - 1))
+        last = li == len(spec.latent_widths) - 1
+        blk = pack_block(Z, r, spec, channel_major=last and not spec.plain)
         page[offs[li]:offs[li] + blk.size] = blk
     return page
 

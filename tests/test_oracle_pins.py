@@ -210,6 +210,40 @@ def test_unquantized_block_bf16_layout():
                                   torch.from_numpy(Z).to(torch.bfloat16).float().numpy())
 
 
+def test_unquantized_value_block_channel_major():
+    # The value latent of a latent layer is stored channel-major, quantized or not (page format
+    # reading): element (slot, j) of a bf16 block at index j * 16 + slot; empty slots stay zero.
+    spec = gen.config_spec(1)
+    r = 40
+    Z = np.full((16, r), np.nan, dtype=np.float32)
+    Z[:11] = (np.arange(11 * r, dtype=np.float32).reshape(11, r) - 200.0) / 7.0
+    blk = O.pack_block(Z, r, spec, channel_major=True)
+    assert blk.size == 16 * r * 2
+    vals = (blk.view(np.uint16).astype(np.uint32) << 16).view(np.float32).reshape(r, 16)
+    want = np.zeros((r, 16), dtype=np.float32)
+    want[:, :11] = torch.from_numpy(Z[:11]).to(torch.bfloat16).float().numpy().T
+    np.testing.assert_array_equal(vals, want)
+    # a whole page: only the value latent of the latent layer is channel-major
+    slots = [[z[:spec.key_ranks[0]] for _ in spec.key_ranks] + [np.resize(z, spec.value_rank)] if s < 11 else None
+             for s, z in enumerate(np.nan_to_num(Z))]
+    slots = [None if x is None else [np.resize(x[0], r_) for r_ in spec.key_ranks] + [x[-1]] for x in slots]
+    page = O.pack_page(slots, spec)
+    offs, _ = O.page_layout(spec)
+    k0 = page[offs[0]:offs[0] + 16 * spec.key_ranks[0] * 2].view(np.uint16).reshape(16, spec.key_ranks[0])
+    np.testing.assert_array_equal(k0[3], torch.from_numpy(slots[3][0]).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16))
+    v = page[offs[-1]:offs[-1] + 16 * spec.value_rank * 2].view(np.uint16).reshape(spec.value_rank, 16)
+    np.testing.assert_array_equal(v[:, 3], torch.from_numpy(slots[3][-1]).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16))
+    # a plain layer keeps its V block slot-major
+    plain = gen.LayerSpec(hidden=64, n_heads=2, n_kv_heads=2, head_dim=8, key_ranks=[], value_rank=0, plain=True)
+    rows = [gen.normals(gen.stream_key(11, 90, s), 32).astype(np.float32) for s in range(2)]
+    pslots = [[row[:8], row[8:16], row[16:]] for row in rows] + [None] * 14
+    ppage = O.pack_page(pslots, plain)
+    poffs, _ = O.page_layout(plain)
+    pv = ppage[poffs[-1]:poffs[-1] + 16 * 16 * 2].view(np.uint16).reshape(16, 16)
+    np.testing.assert_array_equal(pv[1], torch.from_numpy(rows[1][16:]).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16))
+    assert not pv[2:].any()
+
+
 def test_pool_page_table_permutation():
     spec = small_spec(quantized=True, hadamard_block=32, key_ranks=[8, 12], value_rank=40)
     T = 37

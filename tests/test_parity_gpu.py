@@ -199,10 +199,9 @@ def test_prefill_two_output_tiles():
 
 
 def test_prefill_tc_row_batches():
-    """A quantized RoPE layer's prefill runs its query rows through the
-    tensor-core decode kernels, 256 rows at a time: two sequences with
-    different history lengths, 320 rows (256 + 64), sampled rows and a
-    peaky-attention rerun against the oracle; the CUDA-core path agrees."""
+    """A quantized RoPE layer's tensor-core prefill (keys and values rebuilt per chunk, tiled causal
+    attention): two sequences with different history lengths, 320 rows, rows at the 128-query tile
+    and sequence edges and a peaky-attention rerun against the oracle; the CUDA-core path agrees."""
     c = case(2)
     s = c.spec
     starts, ns = [100, 30], [200, 120]
@@ -238,6 +237,8 @@ def test_prefill_tc_row_batches():
 @pytest.mark.parametrize("cfg,quant,lens", [
     (2, False, [600, 257, 256, 1]),
     (3, True, [300, 97]),
+    (1, False, [600, 257, 1]),
+    (3, False, [300, 97]),
 ])
 def test_tc_scores_feeding_cuda_core_values(cfg, quant, lens):
     """Tensor-core score kernel (path 2) against the oracle, with multiple and
@@ -279,9 +280,11 @@ def test_tc_long_context_runs():
     run_decode(case(2), [12000, 12000], peaky=25.0, use_hidden=False, check_pool=False)
 
 
-def test_decode_paths_agree():
-    """CUDA-core path (1), tensor-core scores (2) and all tensor-core (0) agree."""
-    outs = [run_decode(case(2), [700, 300], use_hidden=False, check_pool=False, path=p) for p in (1, 2, 0)]
+@pytest.mark.parametrize("cfg", [2, 1, 3])
+def test_decode_paths_agree(cfg):
+    """CUDA-core path (1), tensor-core scores (2) and all tensor-core (0) agree: 4/3-bit latents
+    (workload 2) and unquantized bf16 latents (workload 1; workload 3 with GQA)."""
+    outs = [run_decode(case(cfg), [700, 300], use_hidden=False, check_pool=False, path=p) for p in (1, 2, 0)]
     for o in outs[1:]:
         assert np.linalg.norm(o - outs[0]) <= 3e-3 * np.linalg.norm(outs[0])
 
@@ -380,3 +383,54 @@ def test_phase_timing_leaves_results_unchanged():
     L.profile_decode(0)
     assert L.sync_status() == 0
     np.testing.assert_array_equal(outs[0], outs[1])
+
+
+def _prefill_rows(c, L, starts, ns, peaky=1.0):
+    """Append each sequence's latents (history and chunk), run one prefill call, return
+    (outputs [sum ns][D] float64, queries, stored latents per sequence)."""
+    s = c.spec
+    cache = GpuCache(L, [a + n for a, n in zip(starts, ns)])
+    Zs = []
+    for b, (a, n) in enumerate(zip(starts, ns)):
+        T = a + n
+        Z = c.latents_from_hidden(c.hidden(b, T), np.arange(T)) if s.plain else c.latents_direct(b, T)
+        cache.append_latents(b, Z)
+        Zs.append(c.stored(Z))
+    Qall = queries(c, len(ns), peaky=peaky, n_pos=max(ns))
+    Q = np.concatenate([Qall[b][:n] for b, n in enumerate(ns)])
+    qt = torch.from_numpy(Q).cuda().to(torch.bfloat16)
+    out = torch.empty(sum(ns), s.hidden, device="cuda", dtype=torch.bfloat16)
+    ws = torch.empty(L.workspace_bytes(len(ns), cache.page_table.shape[1] * 16, max(ns)), dtype=torch.uint8,
+                     device="cuda")
+    L.prefill(cache.pool, cache.n_pages, cache.page_table, starts, ns, qt, out, ws)
+    torch.cuda.synchronize()
+    assert L.sync_status() == 0
+    return out.double().cpu().numpy(), Q, Zs
+
+
+@pytest.mark.parametrize("cfg,quant,layer", [(2, False, 2), (1, False, 2), (3, False, 2), (3, True, 2), (4, False, 0)])
+def test_prefill_tensor_core_tiles(cfg, quant, layer):
+    """Tensor-core prefill against the oracle's causal attention: 4/3-bit and bf16 latents, GQA
+    (workload 3) and an uncompressed layer (workload 4, layer 0).  Two sequences, one with history
+    and a chunk that ends inside a 128-query tile, one a prompt from position 0; rows at the tile
+    edges, the first and last rows, and a peaky rerun; all rows agree with the CUDA-core path."""
+    c = case(cfg, quantized=quant, layer=layer)
+    s = c.spec
+    starts, ns = [300, 0], [200, 131]
+    for peaky in (1.0, 25.0):
+        L = c.load()
+        got, Q, Zs = _prefill_rows(c, L, starts, ns, peaky)
+        for r in (0, 1, 127, 128, 199, 200, 327, 328, 330):
+            b = 0 if r < ns[0] else 1
+            i = r if b == 0 else r - ns[0]
+            T = starts[b] + i + 1
+            if s.plain:
+                want = O.decode_plain(s, c.f, np.concatenate(Zs[b][:-1], axis=1), Zs[b][-1], Q[r], T, T - 1)
+            else:
+                want = O.decode(s, c.f, Zs[b], Q[r], T - 1, T, c.B_rot)
+            check_close(got[r], want, f"prefill row {r} (peaky {peaky})")
+        if peaky == 1.0:
+            L1 = c.load()
+            L1.set_decode_path(1)
+            ref, _, _ = _prefill_rows(c, L1, starts, ns, peaky)
+            assert np.linalg.norm(ref - got) <= 3e-3 * np.linalg.norm(ref)

@@ -80,8 +80,9 @@ def test_cfg3_batch64_ctx8192_peaky():
 
 def test_cfg4_prefill_chunk_1024_after_3072():
     """One 1024-query chunk of the 4096-token prefill of a compressed stack layer, after 3072 tokens of
-    history (chunks of 1024, appended before their attention), through the tensor-core row batches
-    (256 rows each): rows at the batch edges checked against the oracle's causal prefill."""
+    history (chunks of 1024, appended before their attention), on the tensor cores (keys and values
+    rebuilt for the chunk, tiled causal attention, output through W_o): rows at the 128-query tile
+    edges checked against the oracle's causal prefill."""
     c = _case(4, layer=2)
     s = c.spec
     L = c.load()
