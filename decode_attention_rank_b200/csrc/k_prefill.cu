@@ -366,12 +366,15 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_gemm_full(GemmArgs a) {
 // O in columns 256 .. 383.
 //   warp 0     bulk copies: the Q tile, then K and V^T tiles into two stages
 //   warp 1     MMA issue: S(k + 1) = Q K(k + 1)^T is issued before O += P(k) V(k)
-//   warps 4-7  softmax, one query row per thread: S row from TMEM, causal
-//              mask, running maximum; O is rescaled only when the maximum
-//              grew by more than 2^8 since the last rescale (P then stays
-//              below 256, exact in fp16), P written as the fp16 A operand of
-//              the next MMA; at the end y = O / l
-constexpr int kFlashThreads = 256;
+//   warps 4-11 softmax, two warps per TMEM lane quarter: warp 4 + x + 4 w
+//              takes half x (64 key columns of S, 64 channels of O) of the
+//              rows 32 w ..; each thread one query row: S from TMEM, causal
+//              mask, the row maximum (the two halves exchange theirs through
+//              shared memory), P as the fp16 A operand of the next MMA; O is
+//              rescaled only when the maximum grew by more than 2^8 since the
+//              last rescale (P then stays below 256, exact in fp16); at the
+//              end y = O / l
+constexpr int kFlashThreads = 384;
 constexpr float kRescaleSlack = 8.f;   // log2 units
 
 struct FlashArgs {
@@ -385,6 +388,13 @@ struct FlashArgs {
   int y_ld;
   uint32_t* status;
 };
+
+// 2^x (hardware approximation; 2^x for x far below zero flushes to 0).
+__device__ __forceinline__ float ex2_approx(float x) {
+  float r;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(x));
+  return r;
+}
 
 __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float* v) {
   uint32_t r[32];
@@ -415,6 +425,7 @@ __global__ void __launch_bounds__(kFlashThreads, 1) k_flash_prefill(FlashArgs a)
   __shared__ __align__(8) uint64_t q_full, kv_full[2], kv_empty[2], s_full[2], s_free[2], p_full, o_done, fin;
   __shared__ uint32_t tmem_base;
   __shared__ volatile int abort_flag;
+  __shared__ float xch[2][kT];   // per half and row: the half-row maximum, then the half-row sum
   uint8_t* smem = smem_raw + ((1024u - (tc::smem_u32(smem_raw) & 1023u)) & 1023u);
   uint8_t* Q_s = smem;
   uint8_t* K_s = Q_s + kTileB;        // two stages
@@ -431,9 +442,9 @@ __global__ void __launch_bounds__(kFlashThreads, 1) k_flash_prefill(FlashArgs a)
       tc::mbar_init(&kv_full[s], 1);
       tc::mbar_init(&kv_empty[s], 1);
       tc::mbar_init(&s_full[s], 1);
-      tc::mbar_init(&s_free[s], 4);
+      tc::mbar_init(&s_free[s], 8);
     }
-    tc::mbar_init(&p_full, 4);
+    tc::mbar_init(&p_full, 8);
     tc::mbar_init(&o_done, 1);
     tc::mbar_init(&fin, 1);
     abort_flag = 0;
@@ -506,53 +517,62 @@ __global__ void __launch_bounds__(kFlashThreads, 1) k_flash_prefill(FlashArgs a)
     }
     __syncwarp();
   } else if (warp >= 4) {
-    const int qq = warp & 3;
+    const int qq = warp & 3;                      // TMEM lane quarter
+    const int x = (warp - 4) >> 2;                // column half
     const int r = qq * 32 + lane;                 // query row of the tile = TMEM lane
     const int pos = a.q_start + q0 + r;           // its position
     const uint32_t lane_base = (uint32_t)(qq * 32) << 16;
+    const int bar_id = 1 + qq;                    // named barrier of the two warps of this quarter
     float m_used = -FLT_MAX, l = 0.f;
     bool ok = true;
     for (int k = 0; k < n_kt; ++k) {
       const int b = k & 1;
       ok = ok && tc::mbar_wait_ab(&s_full[b], ((uint32_t)(k >> 1)) & 1u, a.status, &abort_flag);
       tc::tc_fence_after();
-      float s[128];
+      float s[64];
       if (ok) {
-#pragma unroll
-        for (int c = 0; c < 128; c += 32) tmem_ld32(tmem + lane_base + (uint32_t)(b * 128 + c), s + c);
+        tmem_ld32(tmem + lane_base + (uint32_t)(b * 128 + 64 * x), s);
+        tmem_ld32(tmem + lane_base + (uint32_t)(b * 128 + 64 * x + 32), s + 32);
         tc::tmem_ld_wait();
       } else {
 #pragma unroll
-        for (int c = 0; c < 128; ++c) s[c] = 0.f;
+        for (int c = 0; c < 64; ++c) s[c] = 0.f;
       }
       // the S buffer may be overwritten once every warp has it in registers
       tc::tc_fence_before();
       __syncwarp();
       if (lane == 0) tc::mbar_arrive(&s_free[b]);
-      // causal mask: key k * 128 + c is visible to the query at `pos` if it is not later
-      const int lim = pos - k * kT;   // columns c <= lim are visible
+      // causal mask: key k * 128 + 64 x + c is visible to the query at `pos` if it is not later
+      const int lim = pos - k * kT - 64 * x;   // columns c <= lim are visible
       float mx = -FLT_MAX;
+      if (lim < 63) {
 #pragma unroll
-      for (int c = 0; c < 128; ++c) {
-        if (c > lim) s[c] = -FLT_MAX;
-        mx = fmaxf(mx, s[c]);
+        for (int c = 0; c < 64; ++c) {
+          if (c > lim) s[c] = -FLT_MAX;
+          mx = fmaxf(mx, s[c]);
+        }
+      } else {
+#pragma unroll
+        for (int c = 0; c < 64; ++c) mx = fmaxf(mx, s[c]);
       }
-      // rescale O only when the maximum moved far enough
+      // row maximum over both halves
+      xch[x][r] = mx;
+      asm volatile("bar.sync %0, 64;" ::"r"(bar_id) : "memory");
+      mx = fmaxf(mx, xch[x ^ 1][r]);
+      asm volatile("bar.sync %0, 64;" ::"r"(bar_id) : "memory");
+      // rescale O only when the maximum moved far enough (both halves decide alike)
       float f = 1.f;
       if (mx > m_used + kRescaleSlack || k == 0) {
-        f = k == 0 ? 0.f : exp2f(m_used - mx);
+        f = k == 0 ? 0.f : ex2_approx(m_used - mx);
         m_used = mx;
       }
-      uint32_t p2[64];
+      uint32_t p2[32];
       float ls = 0.f;
 #pragma unroll
-      for (int c = 0; c < 128; c += 2) {
-        const float e0 = s[c] == -FLT_MAX ? 0.f : exp2f(s[c] - m_used);
-        const float e1 = s[c + 1] == -FLT_MAX ? 0.f : exp2f(s[c + 1] - m_used);
-        const __half2 hp = __floats2half2_rn(e0, e1);
-        const float2 back = __half22float2(hp);
-        ls += back.x + back.y;
-        p2[c / 2] = *reinterpret_cast<const uint32_t*>(&hp);
+      for (int c = 0; c < 64; c += 2) {
+        const float e0 = ex2_approx(s[c] - m_used), e1 = ex2_approx(s[c + 1] - m_used);   // masked: 2^-huge = 0
+        ls += e0 + e1;
+        p2[c / 2] = pack_half2(e0, e1);
       }
       l = l * f + ls;
       // P(k - 1) V(k - 1) must be done before O is touched and P is overwritten
@@ -561,20 +581,20 @@ __global__ void __launch_bounds__(kFlashThreads, 1) k_flash_prefill(FlashArgs a)
         tc::tc_fence_after();
         if (ok && f != 1.f) {
 #pragma unroll 1
-          for (int c = 0; c < 128; c += 32) {
+          for (int c = 0; c < 64; c += 32) {
             float o[32];
-            tmem_ld32(tmem + lane_base + o_col + (uint32_t)c, o);
+            tmem_ld32(tmem + lane_base + o_col + (uint32_t)(64 * x + c), o);
             tc::tmem_ld_wait();
 #pragma unroll
             for (int i = 0; i < 32; ++i) o[i] *= f;
-            tmem_st32(tmem + lane_base + o_col + (uint32_t)c, o);
+            tmem_st32(tmem + lane_base + o_col + (uint32_t)(64 * x + c), o);
           }
           tc::tmem_st_wait();
         }
       }
 #pragma unroll
-      for (int c8 = 0; c8 < 16; ++c8)
-        *reinterpret_cast<uint4*>(P_s + tile_off(r, c8 * 8)) =
+      for (int c8 = 0; c8 < 8; ++c8)
+        *reinterpret_cast<uint4*>(P_s + tile_off(r, 64 * x + c8 * 8)) =
             make_uint4(p2[c8 * 4], p2[c8 * 4 + 1], p2[c8 * 4 + 2], p2[c8 * 4 + 3]);
       tc::fence_proxy_async();
       tc::tc_fence_before();
@@ -583,17 +603,21 @@ __global__ void __launch_bounds__(kFlashThreads, 1) k_flash_prefill(FlashArgs a)
     }
     ok = ok && tc::mbar_wait_ab(&o_done, ((uint32_t)(n_kt - 1)) & 1u, a.status, &abort_flag);
     tc::tc_fence_after();
+    // row sum over both halves
+    xch[x][r] = l;
+    asm volatile("bar.sync %0, 64;" ::"r"(bar_id) : "memory");
+    l += xch[x ^ 1][r];
     const float inv = l > 0.f ? 1.f / l : 0.f;
     const bool row_ok = r < nq;
 #pragma unroll 1
-    for (int c = 0; c < 128; c += 32) {
+    for (int c = 0; c < 64; c += 32) {
       float o[32];
       if (ok) {
-        tmem_ld32(tmem + lane_base + o_col + (uint32_t)c, o);
+        tmem_ld32(tmem + lane_base + o_col + (uint32_t)(64 * x + c), o);
         tc::tmem_ld_wait();
       }
       if (row_ok) {
-        float* yr = a.y + (size_t)(q0 + r) * a.y_ld + (size_t)h * 128 + c;
+        float* yr = a.y + (size_t)(q0 + r) * a.y_ld + (size_t)h * 128 + 64 * x + c;
 #pragma unroll
         for (int i = 0; i < 32; i += 4)
           *reinterpret_cast<float4*>(yr + i) =

@@ -84,12 +84,13 @@ static __device__ __noinline__ bool mbar_wait_slow(uint64_t* bar, uint32_t parit
                                                    unsigned long long limit_ns = kWaitLimitNs, uint32_t nap_ns = 0) {
   if (mbar_try_wait(bar, parity)) return true;
   const unsigned long long t0 = global_ns();
-  for (;;) {
-    // eight polls between checks of the abort flag and the clock
+  for (uint32_t n = 0;; ++n) {
+    // eight polls between checks of the abort flag and the clock; with a nap
+    // time, naps between the polls after the first round
 #pragma unroll 1
     for (int k = 0; k < 8; ++k) {
       if (mbar_try_wait(bar, parity)) return true;
-      if (nap_ns) __nanosleep(nap_ns);
+      if (nap_ns && n) __nanosleep(nap_ns);
     }
     if (abort && *abort) return false;
     if (global_ns() - t0 > limit_ns) break;
@@ -120,8 +121,9 @@ __device__ __forceinline__ bool mbar_wait_ab(uint64_t* bar, uint32_t parity, uin
 __device__ __forceinline__ bool mbar_wait_ab_lazy(uint64_t* bar, uint32_t parity, uint32_t* status,
                                                   volatile int* abort) {
   if (mbar_test_wait(bar, parity)) return true;
-  return mbar_wait_slow(bar, parity, status, abort, kWaitLimitNs, 256);
+  return mbar_wait_slow(bar, parity, status, abort, kWaitLimitNs, 512);
 }
+
 
 // ---- bulk copies (global -> shared, completion on an mbarrier) -------------
 __device__ __forceinline__ void bulk_g2s(void* smem_dst, const void* gmem_src, uint32_t bytes, uint64_t* bar) {
