@@ -530,6 +530,14 @@ def run_prefill(args):
     clk = clocks.stop()
     status = L.sync_status()
     ms = e0.elapsed_time(e1) / args.steps
+    # algorithmic tensor flops of the chunk: S = QK^T and O += PV over the visible (query, key) pairs of every
+    # head, the key and value rebuild of the T cached tokens, and the output through W_o
+    d, H, Hkv = spec.head_dim, spec.n_heads, spec.n_kv_heads
+    pairs = n * (T - n) + n * (n + 1) // 2
+    flops = (4.0 * d * pairs * H + 2.0 * T * d * sum(spec.key_ranks) + 2.0 * T * spec.value_rank * Hkv * d +
+             2.0 * n * H * d * spec.hidden)
+    tpk, tsrc = measured_tensor_peak()
+    ach = flops / (ms * 1e-3) / 1e12
     return {"metric": "causal prefill query tokens/s (latent attention over the paged cache)", "value": n / (ms * 1e-3),
             "unit": "query tokens/s", "n_gpus": 1, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "u3/u4 latent codes + fp16 "
@@ -537,6 +545,8 @@ def run_prefill(args):
             "config": {"workload": f"prefill chunk of {n} queries after {T - n} tokens of history, batch 1 "
                                    "(LongChat-7B-shaped layer, 4/3-bit latents)", "batch": 1, "ctx": T,
                        "queries": n},
+            "roofline": {"bound": "tensor", "achieved": ach, "peak": tpk, "unit": "TFLOP/s", "frac": ach / tpk,
+                         "traffic": None, "peak_source": tsrc, "algorithmic_flops": flops},
             "clocks": clk, "device_status": status}
 
 

@@ -119,6 +119,8 @@ static starkv_status plan_layer(starkv_layer* L) {
         for (int k = 0; k < seg_len[s]; k += c.group_size)
           gs.push_back(GroupDesc{seg_start[s] + k, std::min(c.group_size, seg_len[s] - k), seg_bits[s], 0});
       ld.n_groups = (int)gs.size();
+      ld.n_hi = nh;
+      ld.gsize = c.group_size;
       ld.scale_bytes = (int)ru((size_t)gs.size() * kPage * 2, 16);
       size_t boff = ld.scale_bytes;
       for (auto& g : gs) {

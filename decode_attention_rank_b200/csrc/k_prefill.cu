@@ -13,9 +13,11 @@
 // is the standard one over 128 x 128 tiles:
 //
 //   k_prefill_q        Q tiles: RoPE at the query positions, softmax scale * log2(e), fp16
-//   k_prefill_keys     K tiles: dequantize, K = Zhat B'_k (CUDA cores, r <= 64 MACs per output), RoPE, fp16
+//   k_prefill_zk       the dequantized key latents as fp16 A tiles (r <= 64 channels, zero padded to 64)
+//   k_prefill_bkt      B'_k of every KV head as an fp16 B tile
 //   k_prefill_zv       the dequantized value latent as fp16 B tiles
-//   k_gemm_full        V^T tiles = (B'_v)^T Zhat_v^T on tcgen05; also out = y W_o
+//   k_gemm_full        on tcgen05: K = Zhat_k B'_k with RoPE in the epilogue (K tiles); V^T tiles =
+//                      (B'_v)^T Zhat_v^T; out = y W_o
 //   k_prefill_plain_kv plain layers: their stored K (already rotated) and V as tiles
 //   k_flash_prefill    S = Q K^T and O += P V on tcgen05, online softmax in registers
 //
@@ -33,7 +35,7 @@ namespace {
 constexpr int kT = 128;            // queries per query tile, keys per key tile
 constexpr int kTileB = 32768;      // one 128 x 128 fp16 tile
 constexpr int kAtomB = 16384;      // one 128 x 64 atom
-constexpr int kMaxPrefillRank = 64;   // key ranks the key reconstruction holds in registers
+constexpr int kMaxPrefillRank = 64;   // key ranks that fit the one 64-channel k-tile of the key rebuild
 
 // Byte offset of element (row, col) inside a tile.
 __device__ __forceinline__ uint32_t tile_off(int row, int col) {
@@ -51,56 +53,64 @@ __device__ __forceinline__ uint32_t pack_half2(float a, float b) {
 // of tile [h][i / 128].  Rows past the chunk are zero.
 __global__ void __launch_bounds__(kT) k_prefill_q(LayerView v, const __nv_bfloat16* __restrict__ q, int q_len,
                                                   int q_start, int n_qt, uint8_t* __restrict__ Qt) {
+  __shared__ double freq[64];   // theta_p
+  if (threadIdx.x < 64) freq[threadIdx.x] = exp2(-(2.0 * threadIdx.x / 128.0) * (double)v.rope_log2_theta);
+  __syncthreads();
   const int qt = blockIdx.x, h = blockIdx.y, r = threadIdx.x;
   const int i = qt * kT + r;
   uint8_t* tile = Qt + ((size_t)h * n_qt + qt) * kTileB;
-  const __nv_bfloat16* qr = q + ((size_t)i * v.H + h) * 128;
+  // the query row: 128 bf16 in 16-byte loads (zero past the chunk)
+  uint4 row[16];
+  const uint4* qr = reinterpret_cast<const uint4*>(q + ((size_t)i * v.H + h) * 128);
+#pragma unroll
+  for (int k = 0; k < 16; ++k) row[k] = i < q_len ? qr[k] : make_uint4(0, 0, 0, 0);
   const int pos = q_start + i;
   for (int c8 = 0; c8 < 8; ++c8) {   // pairs p = 8 c8 .. 8 c8 + 7 and p + 64
+    const uint32_t aw[4] = {row[c8].x, row[c8].y, row[c8].z, row[c8].w};
+    const uint32_t bw[4] = {row[8 + c8].x, row[8 + c8].y, row[8 + c8].z, row[8 + c8].w};
     uint32_t lo[4], hi[4];
 #pragma unroll
-    for (int k = 0; k < 8; k += 2) {
-      float re[2] = {0.f, 0.f}, im[2] = {0.f, 0.f};
-      if (i < q_len) {
+    for (int k = 0; k < 4; ++k) {
+      float re[2], im[2];
 #pragma unroll
-        for (int e = 0; e < 2; ++e) {
-          const int p = c8 * 8 + k + e;
-          const float a = __bfloat162float(qr[p]), b = __bfloat162float(qr[p + 64]);
-          float cs = 1.f, sn = 0.f;
-          if (v.rope) {
-            const double ang = (double)pos * exp2(-(2.0 * p / 128.0) * (double)v.rope_log2_theta);
-            const double two_pi = 6.283185307179586476925286766559;
-            sincosf((float)(ang - two_pi * rint(ang / two_pi)), &sn, &cs);
-          }
-          re[e] = (a * cs - b * sn) * v.scale_log2;
-          im[e] = (b * cs + a * sn) * v.scale_log2;
+      for (int e = 0; e < 2; ++e) {
+        const int p = c8 * 8 + 2 * k + e;
+        const float a = __uint_as_float(e ? aw[k] & 0xFFFF0000u : aw[k] << 16);
+        const float b = __uint_as_float(e ? bw[k] & 0xFFFF0000u : bw[k] << 16);
+        float cs = 1.f, sn = 0.f;
+        if (v.rope) {
+          // angle pos * theta_p reduced modulo 2 pi in double, then a float sincos
+          const double ang = (double)pos * freq[p];
+          const double two_pi = 6.283185307179586476925286766559;
+          sincosf((float)(ang - two_pi * rint(ang / two_pi)), &sn, &cs);
         }
+        re[e] = (a * cs - b * sn) * v.scale_log2;
+        im[e] = (b * cs + a * sn) * v.scale_log2;
       }
-      lo[k / 2] = pack_half2(re[0], re[1]);
-      hi[k / 2] = pack_half2(im[0], im[1]);
+      lo[k] = pack_half2(re[0], re[1]);
+      hi[k] = pack_half2(im[0], im[1]);
     }
     *reinterpret_cast<uint4*>(tile + tile_off(r, c8 * 8)) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
     *reinterpret_cast<uint4*>(tile + tile_off(r, 64 + c8 * 8)) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
   }
 }
 
-// ------------------------------------------------------------------ K tiles (latent layers)
-// Token t = kt * 128 + r of the sequence, KV head g: the dequantized key
-// latent (r_g <= 64 channels), K = zhat B'_k,g, rotated at position t with
-// the layer's RoPE table (the same fp16 cos / sin the decode scores use).
-__global__ void __launch_bounds__(kT) k_prefill_keys(LayerView v, const uint8_t* __restrict__ pool,
-                                                     long long n_pages, const int32_t* __restrict__ pt_row,
-                                                     int T, const float* __restrict__ Bk,
-                                                     const int* __restrict__ key_off, const uint8_t* __restrict__ E,
-                                                     int n_kt, uint8_t* __restrict__ Kt) {
-  __shared__ float Bs[kMaxPrefillRank][128];
-  const int kt = blockIdx.x, g = blockIdx.y, r = threadIdx.x;
+// ------------------------------------------------------------------ dequantized key latents (A tiles)
+// Tile [g][kt]: 128 tokens x 64 channels (fp16, swizzled); channels past the
+// KV head's rank r_g (<= 64) and tokens past T are zero.
+__global__ void k_prefill_zk(LayerView v, const uint8_t* __restrict__ pool, long long n_pages,
+                             const int32_t* __restrict__ pt_row, int T, int n_kt, int n_kt_l,
+                             uint8_t* __restrict__ Zk) {
+  const long long idx = (long long)blockIdx.x * blockDim.x + threadIdx.x;   // (g, tile kt, row, chunk)
+  if (idx >= (long long)v.Hkv * n_kt * kT * 8) return;
+  const int c = (int)(idx & 7);
+  const int row = (int)((idx >> 3) % kT);
+  const long long gk = (idx >> 3) / kT;
+  const int kt = (int)(gk % n_kt), g = (int)(gk / n_kt);
+  const int t = kt * kT + row;
   const LatentDesc ld = v.lat[g];
-  const int R = ld.width;
-  for (int e = threadIdx.x; e < R * 128; e += blockDim.x) Bs[e >> 7][e & 127] = Bk[(size_t)key_off[g] * 128 + e];
-  const int t = kt * kT + r;
-  float z[kMaxPrefillRank];
-  if (t < T) {
+  uint32_t o[4] = {0u, 0u, 0u, 0u};
+  if (t < T && c * 8 < ld.width) {
     int page = pt_row[t / kPage];
     if (page < 0 || page >= n_pages) {
       atomicOr(v.status, kBadPage);
@@ -108,47 +118,35 @@ __global__ void __launch_bounds__(kT) k_prefill_keys(LayerView v, const uint8_t*
     }
     const uint8_t* blk = pool + (size_t)page * v.page_bytes + ld.block_off;
 #pragma unroll
-    for (int j = 0; j < kMaxPrefillRank; ++j) z[j] = j < R ? latent_value(v, blk, ld, t % kPage, j) : 0.f;
-  } else {
-#pragma unroll
-    for (int j = 0; j < kMaxPrefillRank; ++j) z[j] = 0.f;
-  }
-  __syncthreads();
-  uint8_t* tile = Kt + ((size_t)g * n_kt + kt) * kTileB;
-  const uint8_t* Et = E + (size_t)(t / kT) * kTileB;
-  for (int c8 = 0; c8 < 8; ++c8) {
-    float re[8], im[8];
-#pragma unroll
-    for (int k = 0; k < 8; ++k) re[k] = im[k] = 0.f;
-#pragma unroll
-    for (int j = 0; j < kMaxPrefillRank; ++j) {
-      if (j >= R) break;
-#pragma unroll
-      for (int k = 0; k < 8; ++k) {
-        re[k] = fmaf(z[j], Bs[j][c8 * 8 + k], re[k]);
-        im[k] = fmaf(z[j], Bs[j][64 + c8 * 8 + k], im[k]);
-      }
+    for (int k = 0; k < 8; k += 2) {
+      const int j = c * 8 + k;
+      const float z0 = j < ld.width ? latent_value(v, blk, ld, t % kPage, j) : 0.f;
+      const float z1 = j + 1 < ld.width ? latent_value(v, blk, ld, t % kPage, j + 1) : 0.f;
+      o[k / 2] = pack_half2(z0, z1);
     }
-    uint32_t lo[4], hi[4];
+  }
+  uint8_t* tile = Zk + ((size_t)g * n_kt_l + kt) * kAtomB;
+  *reinterpret_cast<uint4*>(tile + tc::sw128((uint32_t)row, (uint32_t)c)) = make_uint4(o[0], o[1], o[2], o[3]);
+}
+
+// B'_k,g as the B operand of K = Zhat_k B'_k: tile g holds row p (channel of
+// K, 0 .. 127), column j (latent channel, 0 .. 63) = B'_k,g[j][p], zero for j >= r_g.
+__global__ void k_prefill_bkt(LayerView v, const float* __restrict__ Bk, const int* __restrict__ key_off,
+                              uint8_t* __restrict__ Bkt) {
+  const int g = blockIdx.x;
+  const int r = key_off[g + 1] - key_off[g];
+  for (int e = threadIdx.x; e < 128 * 8; e += blockDim.x) {   // (chunk c, row p): consecutive threads, consecutive p
+    const int p = e & 127, c = e >> 7;
+    uint32_t o[4];
 #pragma unroll
     for (int k = 0; k < 8; k += 2) {
-      float a[2], b[2];
-#pragma unroll
-      for (int e = 0; e < 2; ++e) {
-        const int p = c8 * 8 + k + e;
-        float cs = 1.f, sn = 0.f;
-        if (v.rope && t < T) {
-          cs = __half2float(*reinterpret_cast<const __half*>(Et + tile_off(t % kT, p)));
-          sn = __half2float(*reinterpret_cast<const __half*>(Et + tile_off(t % kT, 64 + p)));
-        }
-        a[e] = re[k + e] * cs - im[k + e] * sn;
-        b[e] = im[k + e] * cs + re[k + e] * sn;
-      }
-      lo[k / 2] = pack_half2(a[0], a[1]);
-      hi[k / 2] = pack_half2(b[0], b[1]);
+      const int j = c * 8 + k;
+      const float b0 = j < r ? Bk[((size_t)key_off[g] + j) * 128 + p] : 0.f;
+      const float b1 = j + 1 < r ? Bk[((size_t)key_off[g] + j + 1) * 128 + p] : 0.f;
+      o[k / 2] = pack_half2(b0, b1);
     }
-    *reinterpret_cast<uint4*>(tile + tile_off(r, c8 * 8)) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
-    *reinterpret_cast<uint4*>(tile + tile_off(r, 64 + c8 * 8)) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+    *reinterpret_cast<uint4*>(Bkt + (size_t)g * kAtomB + tc::sw128((uint32_t)p, (uint32_t)c)) =
+        make_uint4(o[0], o[1], o[2], o[3]);
   }
 }
 
@@ -237,24 +235,29 @@ __global__ void __launch_bounds__(256) k_prefill_plain_kv(LayerView v, const uin
 
 // ------------------------------------------------------------------ full-K GEMM on tcgen05
 // D[m][n] = sum_k A[m][k] B[n][k] for one 128 x 128 output tile, all of K in
-// one CTA.  A: 128 x 64 tiles at a_base + blockIdx.y * a_step, k-tiles 16 KB
-// apart; B: 128 x 64 tiles at b_base + blockIdx.x * b_step, likewise.
-//   EPI_VT:  the tile is V^T of KV head blockIdx.y, key tile blockIdx.x:
-//            written as a flash-attention V^T tile (fp16)
-//   EPI_OUT: out[n][m] for rows n < rows and columns m < n_valid (bf16 or fp32)
+// one CTA.  A: 128 x 64 tiles at A + blockIdx.x * a_step_x + blockIdx.y *
+// a_step_y, k-tiles 16 KB apart; B likewise.
+//   EPI_VT:    the tile is V^T of KV head blockIdx.y, key tile blockIdx.x:
+//              written as a flash-attention V^T tile (fp16)
+//   EPI_OUT:   out[n][m] for rows n < rows and columns m < n_valid (bf16 or fp32)
+//   EPI_KROPE: the tile is K of KV head blockIdx.y, key tile blockIdx.x (rows
+//              = tokens, columns = channels): rotated at each token's position
+//              with the RoPE table and written as a flash-attention K tile
 constexpr int kGemmThreads = 256;
 constexpr int kGemmStages = 4;
-enum { EPI_VT = 0, EPI_OUT_BF16 = 1, EPI_OUT_F32 = 2 };
+enum { EPI_VT = 0, EPI_OUT_BF16 = 1, EPI_OUT_F32 = 2, EPI_KROPE = 3 };
 
 struct GemmArgs {
   const uint8_t* A;
-  long long a_step;
+  long long a_step_x, a_step_y;
   const uint8_t* B;
-  long long b_step;
+  long long b_step_x, b_step_y;
   int KT;
-  void* out;            // EPI_VT: tiles [blockIdx.y][n_tiles]; EPI_OUT: row-major [rows][ld]
-  int n_tiles;          // EPI_VT
+  int stages;           // smem stages of (A, B) k-tiles, <= kGemmStages
+  void* out;            // EPI_VT / EPI_KROPE: tiles [blockIdx.y][n_tiles]; EPI_OUT: row-major [rows][ld]
+  int n_tiles;
   int rows, n_valid, ld;   // EPI_OUT
+  const uint8_t* E;        // EPI_KROPE: RoPE table (null: no rotation)
   uint32_t* status;
 };
 
@@ -266,8 +269,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_gemm_full(GemmArgs a) {
   __shared__ volatile int abort_flag;
   uint8_t* smem = smem_raw + ((1024u - (tc::smem_u32(smem_raw) & 1023u)) & 1023u);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const uint8_t* Ab = a.A + (size_t)blockIdx.y * a.a_step;
-  const uint8_t* Bb = a.B + (size_t)blockIdx.x * a.b_step;
+  const uint8_t* Ab = a.A + (size_t)blockIdx.x * a.a_step_x + (size_t)blockIdx.y * a.a_step_y;
+  const uint8_t* Bb = a.B + (size_t)blockIdx.x * a.b_step_x + (size_t)blockIdx.y * a.b_step_y;
   if (threadIdx.x == 0) {
     for (int s = 0; s < kGemmStages; ++s) {
       tc::mbar_init(&full[s], 1);
@@ -286,14 +289,14 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_gemm_full(GemmArgs a) {
     if (lane == 0) {
       int k = 0;
       for (; k < a.KT; ++k) {
-        const int s = k % kGemmStages;
-        if (!tc::mbar_wait_ab_lazy(&empty[s], (((uint32_t)(k / kGemmStages)) & 1u) ^ 1u, a.status, &abort_flag)) break;
+        const int s = k % a.stages;
+        if (!tc::mbar_wait_ab_lazy(&empty[s], (((uint32_t)(k / a.stages)) & 1u) ^ 1u, a.status, &abort_flag)) break;
         tc::mbar_expect_tx(&full[s], 2 * kAtomB);
         tc::bulk_g2s(smem + (size_t)s * 2 * kAtomB, Ab + (size_t)k * kAtomB, kAtomB, &full[s]);
         tc::bulk_g2s(smem + (size_t)s * 2 * kAtomB + kAtomB, Bb + (size_t)k * kAtomB, kAtomB, &full[s]);
       }
-      for (int j = max(0, k - kGemmStages); j < k; ++j)
-        tc::mbar_wait(&full[j % kGemmStages], ((uint32_t)(j / kGemmStages)) & 1u, a.status);
+      for (int j = max(0, k - a.stages); j < k; ++j)
+        tc::mbar_wait(&full[j % a.stages], ((uint32_t)(j / a.stages)) & 1u, a.status);
     }
     __syncwarp();
   } else if (warp == 1) {
@@ -303,8 +306,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_gemm_full(GemmArgs a) {
       const uint32_t lo0 = tc::desc_lo(d0), hi = tc::desc_hi(d0);
       int k = 0;
       for (; k < a.KT && !abort_flag; ++k) {
-        const int s = k % kGemmStages;
-        if (!tc::mbar_wait_ab(&full[s], ((uint32_t)(k / kGemmStages)) & 1u, a.status, &abort_flag)) {
+        const int s = k % a.stages;
+        if (!tc::mbar_wait_ab(&full[s], ((uint32_t)(k / a.stages)) & 1u, a.status, &abort_flag)) {
           abort_flag = 1;
           break;
         }
@@ -323,7 +326,46 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_gemm_full(GemmArgs a) {
     const int m = q * 32 + lane;   // TMEM lane = output row m
     const bool ok = tc::mbar_wait_ab(&done, 0, a.status, &abort_flag);
     tc::tc_fence_after();
-    for (int c0 = 0; c0 < 128; c0 += 16) {
+    if constexpr (EPI == EPI_KROPE) {
+      // row m = token blockIdx.x * 128 + m: pairs (p, p + 64) of K rotated at that position
+      uint8_t* tile = (uint8_t*)a.out + ((size_t)blockIdx.y * a.n_tiles + blockIdx.x) * kTileB;
+      const uint8_t* Et = a.E ? a.E + (size_t)blockIdx.x * kTileB : nullptr;
+      for (int c0 = 0; c0 < 64; c0 += 16) {
+        float re[16], im[16];
+        if (ok) {
+          tc::tmem_ld16_sync(tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)c0, re);
+          tc::tmem_ld16_sync(tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(64 + c0), im);
+        } else {
+#pragma unroll
+          for (int i = 0; i < 16; ++i) re[i] = im[i] = 0.f;
+        }
+        uint32_t lo[8], hi[8];
+#pragma unroll
+        for (int i = 0; i < 16; i += 2) {
+          float x0[2], y0[2];
+#pragma unroll
+          for (int e = 0; e < 2; ++e) {
+            float cs = 1.f, sn = 0.f;
+            if (Et) {
+              cs = __half2float(*reinterpret_cast<const __half*>(Et + tile_off(m, c0 + i + e)));
+              sn = __half2float(*reinterpret_cast<const __half*>(Et + tile_off(m, 64 + c0 + i + e)));
+            }
+            x0[e] = re[i + e] * cs - im[i + e] * sn;
+            y0[e] = im[i + e] * cs + re[i + e] * sn;
+          }
+          lo[i / 2] = pack_half2(x0[0], x0[1]);
+          hi[i / 2] = pack_half2(y0[0], y0[1]);
+        }
+#pragma unroll
+        for (int h8 = 0; h8 < 2; ++h8) {
+          *reinterpret_cast<uint4*>(tile + tile_off(m, c0 + h8 * 8)) =
+              make_uint4(lo[h8 * 4], lo[h8 * 4 + 1], lo[h8 * 4 + 2], lo[h8 * 4 + 3]);
+          *reinterpret_cast<uint4*>(tile + tile_off(m, 64 + c0 + h8 * 8)) =
+              make_uint4(hi[h8 * 4], hi[h8 * 4 + 1], hi[h8 * 4 + 2], hi[h8 * 4 + 3]);
+        }
+      }
+    }
+    for (int c0 = 0; c0 < (EPI == EPI_KROPE ? 0 : 128); c0 += 16) {
       float x[16];
       if (ok) {
         tc::tmem_ld16_sync(tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)c0, x);
@@ -362,22 +404,25 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_gemm_full(GemmArgs a) {
 }
 
 // ------------------------------------------------------------------ flash attention over the tiles
-// One CTA per (query tile, query head).  TMEM: S in two 128-column buffers,
-// O in columns 256 .. 383.
-//   warp 0     bulk copies: the Q tile, then K and V^T tiles into two stages
+// A persistent grid over (query tile, query head) items.  TMEM: S in two
+// 128-column buffers, O in columns 256 .. 383.
+//   warp 0     bulk copies: each item's Q tile, then its K and V^T tiles into two stages
 //   warp 1     MMA issue: S(k + 1) = Q K(k + 1)^T is issued before O += P(k) V(k)
-//   warps 4-11 softmax, two warps per TMEM lane quarter: warp 4 + x + 4 w
-//              takes half x (64 key columns of S, 64 channels of O) of the
-//              rows 32 w ..; each thread one query row: S from TMEM, causal
-//              mask, the row maximum (the two halves exchange theirs through
-//              shared memory), P as the fp16 A operand of the next MMA; O is
-//              rescaled only when the maximum grew by more than 2^8 since the
-//              last rescale (P then stays below 256, exact in fp16); at the
-//              end y = O / l
-constexpr int kFlashThreads = 384;
+//   warps 4 .. softmax, kSoftWarps per TMEM lane quarter: warp 4 + w + 4 x
+//              takes part x (kSoftCols key columns of S, kSoftCols channels
+//              of O) of the rows 32 w ..; each thread one query row: S from
+//              TMEM, causal mask, the row maximum (the parts exchange theirs
+//              through shared memory), P as the fp16 A operand of the next
+//              MMA; O is rescaled only when the maximum grew by more than 2^8
+//              since the last rescale (P then stays below 256, exact in
+//              fp16); at the end y = O / l
+constexpr int kSoftWarps = 2;                      // softmax warps per TMEM lane quarter
+constexpr int kSoftCols = 128 / kSoftWarps;        // key columns (and O channels) per softmax warp
+constexpr int kFlashThreads = 128 + 128 * kSoftWarps;
 constexpr float kRescaleSlack = 8.f;   // log2 units
 
 struct FlashArgs {
+  int n_qt_used, H;     // query tiles of this chunk, query heads
   const uint8_t* Q;     // [H][n_qt] tiles
   const uint8_t* K;     // [Hkv][n_kt] tiles: rows = keys, columns = channels
   const uint8_t* Vt;    // [Hkv][n_kt] tiles: rows = channels, columns = keys
@@ -420,32 +465,41 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const float* v) {
       : "memory");
 }
 
+// Work items are (query tile, head) pairs taken longest first: item it is
+// query tile n_qt - 1 - it / H (later tiles see more keys), head it % H; CTA c
+// takes items c, c + G, ... (a persistent grid, so the causal imbalance is
+// spread over all CTAs).  Barrier phases run on across items.
+__device__ __forceinline__ int flash_n_kt(const FlashArgs& a, int qt) {
+  const int nq = min(kT, a.q_len - qt * kT);
+  return (a.q_start + qt * kT + nq - 1) / kT + 1;   // key tiles holding a key visible to the tile
+}
+
 __global__ void __launch_bounds__(kFlashThreads, 1) k_flash_prefill(FlashArgs a) {
   extern __shared__ uint8_t smem_raw[];
-  __shared__ __align__(8) uint64_t q_full, kv_full[2], kv_empty[2], s_full[2], s_free[2], p_full, o_done, fin;
+  __shared__ __align__(8) uint64_t q_full, q_empty, kv_full[2], kv_empty[2], s_full[2], s_free[2], p_full, o_done,
+      o_free, fin;
   __shared__ uint32_t tmem_base;
   __shared__ volatile int abort_flag;
-  __shared__ float xch[2][kT];   // per half and row: the half-row maximum, then the half-row sum
+  __shared__ float xch[kSoftWarps][kT];   // per part and row: the part's row maximum, then its row sum
   uint8_t* smem = smem_raw + ((1024u - (tc::smem_u32(smem_raw) & 1023u)) & 1023u);
   uint8_t* Q_s = smem;
   uint8_t* K_s = Q_s + kTileB;        // two stages
   uint8_t* V_s = K_s + 2 * kTileB;    // two stages
   uint8_t* P_s = V_s + 2 * kTileB;
-  const int qt = blockIdx.x, h = blockIdx.y, g = h / a.group_q;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int q0 = qt * kT;
-  const int nq = min(kT, a.q_len - q0);
-  const int n_kt = (a.q_start + q0 + nq - 1) / kT + 1;   // key tiles holding a key visible to this tile
+  const int n_items = a.n_qt_used * a.H;
   if (threadIdx.x == 0) {
     tc::mbar_init(&q_full, 1);
+    tc::mbar_init(&q_empty, 1);
     for (int s = 0; s < 2; ++s) {
       tc::mbar_init(&kv_full[s], 1);
       tc::mbar_init(&kv_empty[s], 1);
       tc::mbar_init(&s_full[s], 1);
-      tc::mbar_init(&s_free[s], 8);
+      tc::mbar_init(&s_free[s], 4 * kSoftWarps);
     }
-    tc::mbar_init(&p_full, 8);
+    tc::mbar_init(&p_full, 4 * kSoftWarps);
     tc::mbar_init(&o_done, 1);
+    tc::mbar_init(&o_free, 4 * kSoftWarps);
     tc::mbar_init(&fin, 1);
     abort_flag = 0;
     tc::fence_mbar_init();
@@ -458,34 +512,43 @@ __global__ void __launch_bounds__(kFlashThreads, 1) k_flash_prefill(FlashArgs a)
   const uint32_t o_col = 256;
 
   if (warp == 0) {
+    // ------------------------------------------------ copies: Q once per item, K and V^T per key tile
     if (lane == 0) {
-      tc::mbar_expect_tx(&q_full, kTileB);
-      tc::bulk_g2s(Q_s, a.Q + ((size_t)h * a.n_qt + qt) * kTileB, kTileB, &q_full);
-      int k = 0;
-      for (; k < n_kt; ++k) {
-        const int s = k & 1;
-        if (!tc::mbar_wait_ab_lazy(&kv_empty[s], (((uint32_t)(k >> 1)) & 1u) ^ 1u, a.status, &abort_flag)) break;
-        tc::mbar_expect_tx(&kv_full[s], 2 * kTileB);
-        tc::bulk_g2s(K_s + (size_t)s * kTileB, a.K + ((size_t)g * a.n_kt + k) * kTileB, kTileB, &kv_full[s]);
-        tc::bulk_g2s(V_s + (size_t)s * kTileB, a.Vt + ((size_t)g * a.n_kt + k) * kTileB, kTileB, &kv_full[s]);
+      int jg = 0, n = 0;   // key tiles and items issued
+      bool ok = true;
+      for (int it = blockIdx.x; it < n_items && ok; it += gridDim.x, ++n) {
+        const int qt = a.n_qt_used - 1 - it / a.H, h = it % a.H, g = h / a.group_q;
+        const int n_kt = flash_n_kt(a, qt);
+        if (!(ok = tc::mbar_wait_ab_lazy(&q_empty, ((uint32_t)n & 1u) ^ 1u, a.status, &abort_flag))) break;
+        tc::mbar_expect_tx(&q_full, kTileB);
+        tc::bulk_g2s(Q_s, a.Q + ((size_t)h * a.n_qt + qt) * kTileB, kTileB, &q_full);
+        for (int k = 0; k < n_kt; ++k, ++jg) {
+          const int s = jg & 1;
+          if (!(ok = tc::mbar_wait_ab_lazy(&kv_empty[s], (((uint32_t)(jg >> 1)) & 1u) ^ 1u, a.status, &abort_flag)))
+            break;
+          tc::mbar_expect_tx(&kv_full[s], 2 * kTileB);
+          tc::bulk_g2s(K_s + (size_t)s * kTileB, a.K + ((size_t)g * a.n_kt + k) * kTileB, kTileB, &kv_full[s]);
+          tc::bulk_g2s(V_s + (size_t)s * kTileB, a.Vt + ((size_t)g * a.n_kt + k) * kTileB, kTileB, &kv_full[s]);
+        }
       }
-      tc::mbar_wait(&q_full, 0, a.status);
-      for (int j = max(0, k - 2); j < k; ++j) tc::mbar_wait(&kv_full[j & 1], ((uint32_t)(j >> 1)) & 1u, a.status);
+      // let copies in flight land before the CTA can exit
+      if (n > 0) tc::mbar_wait(&q_full, ((uint32_t)(n - 1)) & 1u, a.status);
+      for (int j = max(0, jg - 2); j < jg; ++j) tc::mbar_wait(&kv_full[j & 1], ((uint32_t)(j >> 1)) & 1u, a.status);
     }
     __syncwarp();
   } else if (warp == 1) {
+    // ------------------------------------------------ MMA issue
     if (lane == 0) {
       const uint32_t idesc = tc::idesc_f16(128, 128, false, false, false);
       const uint64_t d0 = tc::sdesc_sw128(tc::smem_u32(smem), 0, 1024);
       const uint32_t base_lo = tc::desc_lo(d0), hi = tc::desc_hi(d0);
       const uint32_t q_lo = base_lo, k_lo = base_lo + (kTileB >> 4), v_lo = base_lo + (3 * kTileB >> 4),
                      p_lo = base_lo + (5 * kTileB >> 4);
-      bool ok = tc::mbar_wait_ab(&q_full, 0, a.status, &abort_flag);
-      // S(k) = Q K(k)^T into S buffer k & 1
-      auto issue_s = [&](int k) -> bool {
-        const int s = k & 1;
-        if (!tc::mbar_wait_ab(&kv_full[s], ((uint32_t)(k >> 1)) & 1u, a.status, &abort_flag)) return false;
-        if (!tc::mbar_wait_ab(&s_free[s], (((uint32_t)(k >> 1)) & 1u) ^ 1u, a.status, &abort_flag)) return false;
+      // S(j) = Q K(j)^T into S buffer j & 1 (j counts key tiles over all items)
+      auto issue_s = [&](int j) -> bool {
+        const int s = j & 1;
+        if (!tc::mbar_wait_ab(&kv_full[s], ((uint32_t)(j >> 1)) & 1u, a.status, &abort_flag)) return false;
+        if (!tc::mbar_wait_ab(&s_free[s], (((uint32_t)(j >> 1)) & 1u) ^ 1u, a.status, &abort_flag)) return false;
         tc::tc_fence_after();
         const uint32_t kb = k_lo + (uint32_t)(s * kTileB >> 4);
 #pragma unroll
@@ -495,20 +558,30 @@ __global__ void __launch_bounds__(kFlashThreads, 1) k_flash_prefill(FlashArgs a)
         tc::mma_commit(&s_full[s]);
         return true;
       };
-      tc::tc_fence_after();
-      if (ok) ok = issue_s(0);
-      for (int k = 0; k < n_kt && ok; ++k) {
-        if (k + 1 < n_kt && !(ok = issue_s(k + 1))) break;
-        // O += P(k) V(k)
-        if (!(ok = tc::mbar_wait_ab(&p_full, (uint32_t)k & 1u, a.status, &abort_flag))) break;
+      bool ok = true;
+      int jg = 0, n = 0;
+      for (int it = blockIdx.x; it < n_items && ok; it += gridDim.x, ++n) {
+        const int qt = a.n_qt_used - 1 - it / a.H;
+        const int n_kt = flash_n_kt(a, qt);
+        if (!(ok = tc::mbar_wait_ab(&q_full, (uint32_t)n & 1u, a.status, &abort_flag))) break;
         tc::tc_fence_after();
-        const uint32_t vb = v_lo + (uint32_t)((k & 1) * kTileB >> 4);
+        if (!(ok = issue_s(jg))) break;
+        for (int k = 0; k < n_kt; ++k) {
+          if (k + 1 < n_kt && !(ok = issue_s(jg + k + 1))) break;
+          if (k + 1 == n_kt) tc::mma_commit(&q_empty);   // every S of this item issued: Q may be replaced
+          // O += P(k) V(k); the first of an item overwrites O once the softmax has read the last item's
+          if (k == 0 && !(ok = tc::mbar_wait_ab(&o_free, ((uint32_t)n & 1u) ^ 1u, a.status, &abort_flag))) break;
+          if (!(ok = tc::mbar_wait_ab(&p_full, (uint32_t)(jg + k) & 1u, a.status, &abort_flag))) break;
+          tc::tc_fence_after();
+          const uint32_t vb = v_lo + (uint32_t)(((jg + k) & 1) * kTileB >> 4);
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk)
-          tc::mma_f16_ss2(tmem + o_col, p_lo + (uint32_t)(kk >> 2) * (kAtomB >> 4) + 2u * (kk & 3), hi,
-                          vb + (uint32_t)(kk >> 2) * (kAtomB >> 4) + 2u * (kk & 3), hi, idesc, (k | kk) ? 1u : 0u);
-        tc::mma_commit(&o_done);
-        tc::mma_commit(&kv_empty[k & 1]);
+          for (int kk = 0; kk < 8; ++kk)
+            tc::mma_f16_ss2(tmem + o_col, p_lo + (uint32_t)(kk >> 2) * (kAtomB >> 4) + 2u * (kk & 3), hi,
+                            vb + (uint32_t)(kk >> 2) * (kAtomB >> 4) + 2u * (kk & 3), hi, idesc, (k | kk) ? 1u : 0u);
+          tc::mma_commit(&o_done);
+          tc::mma_commit(&kv_empty[(jg + k) & 1]);
+        }
+        jg += n_kt;
       }
       if (!ok) abort_flag = 1;
       // every MMA has completed before the CTA may exit
@@ -517,112 +590,130 @@ __global__ void __launch_bounds__(kFlashThreads, 1) k_flash_prefill(FlashArgs a)
     }
     __syncwarp();
   } else if (warp >= 4) {
+    // ------------------------------------------------ softmax and output
     const int qq = warp & 3;                      // TMEM lane quarter
-    const int x = (warp - 4) >> 2;                // column half
+    const int x = (warp - 4) >> 2;                // column part
     const int r = qq * 32 + lane;                 // query row of the tile = TMEM lane
-    const int pos = a.q_start + q0 + r;           // its position
     const uint32_t lane_base = (uint32_t)(qq * 32) << 16;
-    const int bar_id = 1 + qq;                    // named barrier of the two warps of this quarter
-    float m_used = -FLT_MAX, l = 0.f;
+    const int bar_id = 1 + qq;                    // named barrier of the softmax warps of this quarter
+    const uint32_t xc = (uint32_t)(kSoftCols * x);   // this warp's first S column / O channel
     bool ok = true;
-    for (int k = 0; k < n_kt; ++k) {
-      const int b = k & 1;
-      ok = ok && tc::mbar_wait_ab(&s_full[b], ((uint32_t)(k >> 1)) & 1u, a.status, &abort_flag);
-      tc::tc_fence_after();
-      float s[64];
-      if (ok) {
-        tmem_ld32(tmem + lane_base + (uint32_t)(b * 128 + 64 * x), s);
-        tmem_ld32(tmem + lane_base + (uint32_t)(b * 128 + 64 * x + 32), s + 32);
-        tc::tmem_ld_wait();
-      } else {
-#pragma unroll
-        for (int c = 0; c < 64; ++c) s[c] = 0.f;
-      }
-      // the S buffer may be overwritten once every warp has it in registers
-      tc::tc_fence_before();
-      __syncwarp();
-      if (lane == 0) tc::mbar_arrive(&s_free[b]);
-      // causal mask: key k * 128 + 64 x + c is visible to the query at `pos` if it is not later
-      const int lim = pos - k * kT - 64 * x;   // columns c <= lim are visible
-      float mx = -FLT_MAX;
-      if (lim < 63) {
-#pragma unroll
-        for (int c = 0; c < 64; ++c) {
-          if (c > lim) s[c] = -FLT_MAX;
-          mx = fmaxf(mx, s[c]);
-        }
-      } else {
-#pragma unroll
-        for (int c = 0; c < 64; ++c) mx = fmaxf(mx, s[c]);
-      }
-      // row maximum over both halves
-      xch[x][r] = mx;
-      asm volatile("bar.sync %0, 64;" ::"r"(bar_id) : "memory");
-      mx = fmaxf(mx, xch[x ^ 1][r]);
-      asm volatile("bar.sync %0, 64;" ::"r"(bar_id) : "memory");
-      // rescale O only when the maximum moved far enough (both halves decide alike)
-      float f = 1.f;
-      if (mx > m_used + kRescaleSlack || k == 0) {
-        f = k == 0 ? 0.f : ex2_approx(m_used - mx);
-        m_used = mx;
-      }
-      uint32_t p2[32];
-      float ls = 0.f;
-#pragma unroll
-      for (int c = 0; c < 64; c += 2) {
-        const float e0 = ex2_approx(s[c] - m_used), e1 = ex2_approx(s[c + 1] - m_used);   // masked: 2^-huge = 0
-        ls += e0 + e1;
-        p2[c / 2] = pack_half2(e0, e1);
-      }
-      l = l * f + ls;
-      // P(k - 1) V(k - 1) must be done before O is touched and P is overwritten
-      if (k > 0) {
-        ok = ok && tc::mbar_wait_ab(&o_done, ((uint32_t)(k - 1)) & 1u, a.status, &abort_flag);
+    int jg = 0;
+    for (int it = blockIdx.x; it < n_items; it += gridDim.x) {
+      const int qt = a.n_qt_used - 1 - it / a.H, h = it % a.H;
+      const int q0 = qt * kT;
+      const int nq = min(kT, a.q_len - q0);
+      const int n_kt = flash_n_kt(a, qt);
+      const int pos = a.q_start + q0 + r;         // this row's position
+      float m_used = -FLT_MAX, l = 0.f;
+      for (int k = 0; k < n_kt; ++k) {
+        const int j = jg + k, b = j & 1;
+        ok = ok && tc::mbar_wait_ab(&s_full[b], ((uint32_t)(j >> 1)) & 1u, a.status, &abort_flag);
         tc::tc_fence_after();
-        if (ok && f != 1.f) {
-#pragma unroll 1
-          for (int c = 0; c < 64; c += 32) {
-            float o[32];
-            tmem_ld32(tmem + lane_base + o_col + (uint32_t)(64 * x + c), o);
-            tc::tmem_ld_wait();
+        float s[kSoftCols];
+        if (ok) {
 #pragma unroll
-            for (int i = 0; i < 32; ++i) o[i] *= f;
-            tmem_st32(tmem + lane_base + o_col + (uint32_t)(64 * x + c), o);
+          for (int c = 0; c < kSoftCols; c += 32) tmem_ld32(tmem + lane_base + (uint32_t)(b * 128) + xc + c, s + c);
+          tc::tmem_ld_wait();
+        } else {
+#pragma unroll
+          for (int c = 0; c < kSoftCols; ++c) s[c] = 0.f;
+        }
+        // the S buffer may be overwritten once every warp has it in registers
+        tc::tc_fence_before();
+        __syncwarp();
+        if (lane == 0) tc::mbar_arrive(&s_free[b]);
+        // causal mask: key k * 128 + xc + c is visible to the query at `pos` if it is not later
+        const int lim = pos - k * kT - (int)xc;   // columns c <= lim are visible
+        float mx = -FLT_MAX;
+        if (lim < kSoftCols - 1) {
+#pragma unroll
+          for (int c = 0; c < kSoftCols; ++c) {
+            if (c > lim) s[c] = -FLT_MAX;
+            mx = fmaxf(mx, s[c]);
           }
-          tc::tmem_st_wait();
+        } else {
+#pragma unroll
+          for (int c = 0; c < kSoftCols; ++c) mx = fmaxf(mx, s[c]);
+        }
+        // row maximum over the parts
+        xch[x][r] = mx;
+        asm volatile("bar.sync %0, %1;" ::"r"(bar_id), "n"(32 * kSoftWarps) : "memory");
+#pragma unroll
+        for (int y = 0; y < kSoftWarps; ++y) mx = fmaxf(mx, xch[y][r]);
+        asm volatile("bar.sync %0, %1;" ::"r"(bar_id), "n"(32 * kSoftWarps) : "memory");
+        // rescale O only when the maximum moved far enough (both halves decide alike)
+        float f = 1.f;
+        if (mx > m_used + kRescaleSlack || k == 0) {
+          f = k == 0 ? 0.f : ex2_approx(m_used - mx);
+          m_used = mx;
+        }
+        uint32_t p2[kSoftCols / 2];
+        float ls = 0.f;
+#pragma unroll
+        for (int c = 0; c < kSoftCols; c += 2) {
+          const float e0 = ex2_approx(s[c] - m_used), e1 = ex2_approx(s[c + 1] - m_used);   // masked: 0
+          ls += e0 + e1;
+          p2[c / 2] = pack_half2(e0, e1);
+        }
+        l = l * f + ls;
+        // the previous PV must be done before O is touched and P is overwritten
+        // (within an item; across items the end of the last one waited for it)
+        if (k > 0) {
+          ok = ok && tc::mbar_wait_ab(&o_done, ((uint32_t)(j - 1)) & 1u, a.status, &abort_flag);
+          tc::tc_fence_after();
+          if (ok && f != 1.f) {
+#pragma unroll 1
+            for (int c = 0; c < kSoftCols; c += 32) {
+              float o[32];
+              tmem_ld32(tmem + lane_base + o_col + xc + (uint32_t)c, o);
+              tc::tmem_ld_wait();
+#pragma unroll
+              for (int i = 0; i < 32; ++i) o[i] *= f;
+              tmem_st32(tmem + lane_base + o_col + xc + (uint32_t)c, o);
+            }
+            tc::tmem_st_wait();
+          }
+        }
+#pragma unroll
+        for (int c8 = 0; c8 < kSoftCols / 8; ++c8)
+          *reinterpret_cast<uint4*>(P_s + tile_off(r, (int)xc + c8 * 8)) =
+              make_uint4(p2[c8 * 4], p2[c8 * 4 + 1], p2[c8 * 4 + 2], p2[c8 * 4 + 3]);
+        tc::fence_proxy_async();
+        tc::tc_fence_before();
+        __syncwarp();
+        if (lane == 0) tc::mbar_arrive(&p_full);
+      }
+      jg += n_kt;
+      ok = ok && tc::mbar_wait_ab(&o_done, ((uint32_t)(jg - 1)) & 1u, a.status, &abort_flag);
+      tc::tc_fence_after();
+      // row sum over the parts
+      xch[x][r] = l;
+      asm volatile("bar.sync %0, %1;" ::"r"(bar_id), "n"(32 * kSoftWarps) : "memory");
+      l = 0.f;
+#pragma unroll
+      for (int y = 0; y < kSoftWarps; ++y) l += xch[y][r];
+      const float inv = l > 0.f ? 1.f / l : 0.f;
+      const bool row_ok = r < nq;
+#pragma unroll 1
+      for (int c = 0; c < kSoftCols; c += 32) {
+        float o[32];
+        if (ok) {
+          tmem_ld32(tmem + lane_base + o_col + xc + (uint32_t)c, o);
+          tc::tmem_ld_wait();
+        }
+        if (row_ok) {
+          float* yr = a.y + (size_t)(q0 + r) * a.y_ld + (size_t)h * 128 + xc + c;
+#pragma unroll
+          for (int i = 0; i < 32; i += 4)
+            *reinterpret_cast<float4*>(yr + i) =
+                ok ? make_float4(o[i] * inv, o[i + 1] * inv, o[i + 2] * inv, o[i + 3] * inv) : make_float4(0, 0, 0, 0);
         }
       }
-#pragma unroll
-      for (int c8 = 0; c8 < 8; ++c8)
-        *reinterpret_cast<uint4*>(P_s + tile_off(r, 64 * x + c8 * 8)) =
-            make_uint4(p2[c8 * 4], p2[c8 * 4 + 1], p2[c8 * 4 + 2], p2[c8 * 4 + 3]);
-      tc::fence_proxy_async();
+      // O has been read (and xch is free for the next item)
       tc::tc_fence_before();
-      __syncwarp();
-      if (lane == 0) tc::mbar_arrive(&p_full);
-    }
-    ok = ok && tc::mbar_wait_ab(&o_done, ((uint32_t)(n_kt - 1)) & 1u, a.status, &abort_flag);
-    tc::tc_fence_after();
-    // row sum over both halves
-    xch[x][r] = l;
-    asm volatile("bar.sync %0, 64;" ::"r"(bar_id) : "memory");
-    l += xch[x ^ 1][r];
-    const float inv = l > 0.f ? 1.f / l : 0.f;
-    const bool row_ok = r < nq;
-#pragma unroll 1
-    for (int c = 0; c < 64; c += 32) {
-      float o[32];
-      if (ok) {
-        tmem_ld32(tmem + lane_base + o_col + (uint32_t)(64 * x + c), o);
-        tc::tmem_ld_wait();
-      }
-      if (row_ok) {
-        float* yr = a.y + (size_t)(q0 + r) * a.y_ld + (size_t)h * 128 + 64 * x + c;
-#pragma unroll
-        for (int i = 0; i < 32; i += 4)
-          *reinterpret_cast<float4*>(yr + i) =
-              ok ? make_float4(o[i] * inv, o[i + 1] * inv, o[i + 2] * inv, o[i + 3] * inv) : make_float4(0, 0, 0, 0);
-      }
+      asm volatile("bar.sync %0, %1;" ::"r"(bar_id), "n"(32 * kSoftWarps) : "memory");
+      if (lane == 0) tc::mbar_arrive(&o_free);
     }
   }
   tc::tc_fence_before();
@@ -634,7 +725,7 @@ __global__ void __launch_bounds__(kFlashThreads, 1) k_flash_prefill(FlashArgs a)
 size_t al256(size_t x) { return (x + 255) / 256 * 256; }
 
 struct PrefillWs {
-  uint8_t *Qt, *Kt, *Vt, *Zt, *yt;
+  uint8_t *Qt, *Kt, *Vt, *Zt, *Zk, *Bkt, *yt;
   float* y;
 };
 
@@ -651,6 +742,10 @@ PrefillWs prefill_ws_layout(const starkv_layer* L, void* ws, int max_T, int max_
   p += al256((size_t)v.Hkv * n_kt * kTileB);
   w.Zt = p;
   p += al256(v.plain ? 0 : (size_t)n_kt * (v.rv / 64) * kAtomB);
+  w.Zk = p;
+  p += al256(v.plain ? 0 : (size_t)v.Hkv * n_kt * kAtomB);
+  w.Bkt = p;
+  p += al256(v.plain ? 0 : (size_t)v.Hkv * kAtomB);
   w.y = (float*)p;
   p += al256(sizeof(float) * (size_t)n_qt * kT * v.H * 128);
   w.yt = p;
@@ -677,7 +772,8 @@ size_t prefill_flash_ws_bytes(const starkv_layer* L, int max_T, int max_q) {
   const LayerView& v = L->view;
   const int n_qt = (max_q + kT - 1) / kT, n_kt = (max_T + kT - 1) / kT;
   return al256((size_t)v.H * n_qt * kTileB) + 2 * al256((size_t)v.Hkv * n_kt * kTileB) +
-         al256(v.plain ? 0 : (size_t)n_kt * (v.rv / 64) * kAtomB) +
+         al256(v.plain ? 0 : (size_t)n_kt * (v.rv / 64) * kAtomB) + al256(v.plain ? 0 : (size_t)v.Hkv * n_kt * kAtomB) +
+         al256(v.plain ? 0 : (size_t)v.Hkv * kAtomB) +
          al256(sizeof(float) * (size_t)n_qt * kT * v.H * 128) + al256((size_t)n_qt * (v.H * 128 / 64) * kAtomB);
 }
 
@@ -701,8 +797,27 @@ cudaError_t launch_prefill_flash(const starkv_layer* L, const uint8_t* pool, lon
     k_prefill_plain_kv<<<dim3(n_kt, v.Hkv), 256, 0, s>>>(v, pool, n_pages, pt_row, T, n_kt_l, w.Kt, w.Vt);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   } else {
-    k_prefill_keys<<<dim3(n_kt, v.Hkv), kT, 0, s>>>(v, pool, n_pages, pt_row, T, L->Bk, L->d_key_off,
-                                                    (const uint8_t*)L->rope_E, n_kt_l, w.Kt);
+    // K = Zhat_k B'_k on the tensor cores, rotated in the epilogue
+    const long long nzk = (long long)v.Hkv * n_kt * kT * 8;
+    k_prefill_zk<<<(unsigned)((nzk + 255) / 256), 256, 0, s>>>(v, pool, n_pages, pt_row, T, n_kt, n_kt_l, w.Zk);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    k_prefill_bkt<<<v.Hkv, 256, 0, s>>>(v, L->Bk, L->d_key_off, w.Bkt);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    GemmArgs gk{};
+    gk.A = w.Zk;
+    gk.a_step_x = kAtomB;
+    gk.a_step_y = (long long)n_kt_l * kAtomB;
+    gk.B = w.Bkt;
+    gk.b_step_y = kAtomB;
+    gk.KT = 1;
+    gk.stages = 1;
+    gk.out = w.Kt;
+    gk.n_tiles = n_kt_l;
+    gk.E = v.rope ? (const uint8_t*)L->rope_E : nullptr;
+    gk.status = v.status;
+    const size_t smem1 = 2 * (size_t)kAtomB + 1024;
+    if ((e = set_smem_limit((const void*)k_gemm_full<EPI_KROPE>, smem1)) != cudaSuccess) return e;
+    k_gemm_full<EPI_KROPE><<<dim3(n_kt, v.Hkv), kGemmThreads, smem1, s>>>(gk);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     const long long nz = (long long)n_kt * (v.rv / 64) * kT * 8;
     k_prefill_zv<<<(unsigned)((nz + 255) / 256), 256, 0, s>>>(v, pool, n_pages, pt_row, T, n_kt, w.Zt);
@@ -710,14 +825,15 @@ cudaError_t launch_prefill_flash(const starkv_layer* L, const uint8_t* pool, lon
     // V^T of KV head g = (B'_v columns of g)^T Zhat_v^T: A = the 128 x r_v B'_v tiles of query head g * group_q
     GemmArgs ga{};
     ga.A = (const uint8_t*)L->Bv_tiles;
-    ga.a_step = (long long)v.group_q * (v.rv / 64) * kAtomB;
+    ga.a_step_y = (long long)v.group_q * (v.rv / 64) * kAtomB;
     ga.B = w.Zt;
-    ga.b_step = (long long)(v.rv / 64) * kAtomB;
+    ga.b_step_x = (long long)(v.rv / 64) * kAtomB;
     ga.KT = v.rv / 64;
+    ga.stages = std::min(3, ga.KT);   // three stages: two CTAs per SM overlap one's epilogue with the other's loads
     ga.out = w.Vt;
     ga.n_tiles = n_kt_l;
     ga.status = v.status;
-    const size_t smem = (size_t)kGemmStages * 2 * kAtomB + 1024;
+    const size_t smem = (size_t)ga.stages * 2 * kAtomB + 1024;
     if ((e = set_smem_limit((const void*)k_gemm_full<EPI_VT>, smem)) != cudaSuccess) return e;
     k_gemm_full<EPI_VT><<<dim3(n_kt, v.Hkv), kGemmThreads, smem, s>>>(ga);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
@@ -728,6 +844,8 @@ cudaError_t launch_prefill_flash(const starkv_layer* L, const uint8_t* pool, lon
   fa.Vt = w.Vt;
   fa.n_qt = n_qt_l;
   fa.n_kt = n_kt_l;
+  fa.n_qt_used = n_qt;
+  fa.H = v.H;
   fa.q_len = q_len;
   fa.q_start = q_start;
   fa.group_q = v.group_q;
@@ -736,22 +854,23 @@ cudaError_t launch_prefill_flash(const starkv_layer* L, const uint8_t* pool, lon
   fa.status = v.status;
   const size_t fsmem = 6 * (size_t)kTileB + 1024;
   if ((e = set_smem_limit((const void*)k_flash_prefill, fsmem)) != cudaSuccess) return e;
-  k_flash_prefill<<<dim3(n_qt, v.H), kFlashThreads, fsmem, s>>>(fa);
+  k_flash_prefill<<<std::min(num_sms(), n_qt * v.H), kFlashThreads, fsmem, s>>>(fa);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   // out = y W_o: y as fp16 B tiles of 128 rows, W_o as the A tiles
   if ((e = launch_pack_rows_tiles_f32(w.y, q_len, v.H * 128, w.yt, s, 128)) != cudaSuccess) return e;
   GemmArgs go{};
   go.A = (const uint8_t*)prefill_wo_tiles(L);
-  go.a_step = (long long)(v.H * 128 / 64) * kAtomB;
+  go.a_step_y = (long long)(v.H * 128 / 64) * kAtomB;
   go.B = w.yt;
-  go.b_step = (long long)(v.H * 128 / 64) * kAtomB;
+  go.b_step_x = (long long)(v.H * 128 / 64) * kAtomB;
   go.KT = v.H * 128 / 64;
+  go.stages = std::min(3, go.KT);
   go.out = out;
   go.rows = q_len;
   go.n_valid = v.D;
   go.ld = v.D;
   go.status = v.status;
-  const size_t smem = (size_t)kGemmStages * 2 * kAtomB + 1024;
+  const size_t smem = (size_t)go.stages * 2 * kAtomB + 1024;
   const void* gk = v.dtype == STARKV_F32 ? (const void*)k_gemm_full<EPI_OUT_F32> : (const void*)k_gemm_full<EPI_OUT_BF16>;
   if ((e = set_smem_limit(gk, smem)) != cudaSuccess) return e;
   const dim3 grid(n_qt, (v.D + 127) / 128);

@@ -31,6 +31,8 @@ struct LatentDesc {
   int ch_off;       // offset of this latent in the concatenated latent vector
   int scale_bytes;  // bytes of the scale block (0 when unquantized)
   int cmajor;       // 1: channel-major (the value latent of a latent layer), see code_bit and elem_index
+  int n_hi;         // quantized: channels of the first (high-precision) segment
+  int gsize;        // quantized: channels per group (groups are cut from each segment's start)
 };
 
 constexpr int kPage = 16;
@@ -90,9 +92,9 @@ __device__ __forceinline__ float latent_value(const LayerView& v, const uint8_t*
     return v.es == 4 ? reinterpret_cast<const float*>(blk)[o]
                      : __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(blk)[o]);
   }
-  int g = 0;
-  for (int k = 1; k < ld.n_groups; ++k)
-    if (j >= v.grp[ld.group0 + k].start) g = k;
+  // groups of gsize channels from the start of each segment
+  const int g = ld.gsize == 32 ? (j < ld.n_hi ? j >> 5 : ((ld.n_hi + 31) >> 5) + ((j - ld.n_hi) >> 5))
+                               : (j < ld.n_hi ? j / ld.gsize : (ld.n_hi + ld.gsize - 1) / ld.gsize + (j - ld.n_hi) / ld.gsize);
   const GroupDesc gd = v.grp[ld.group0 + g];
   const float s = __half2float(reinterpret_cast<const __half*>(blk)[g * kPage + slot]);
   const uint32_t bit = code_bit(slot, j - gd.start, gd.n, gd.bits, ld.cmajor);
