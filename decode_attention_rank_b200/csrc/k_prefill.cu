@@ -405,8 +405,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_gemm_full(GemmArgs a) {
 
 // ------------------------------------------------------------------ flash attention over the tiles
 // A persistent grid over (query tile, query head) items.  TMEM: S in two
-// 128-column buffers, O in columns 256 .. 383.
-//   warp 0     bulk copies: each item's Q tile, then its K and V^T tiles into two stages
+// 128-column buffers, O in columns 256 .. 383; P(j) (fp16 pairs, 64 columns)
+// overwrites the S buffer it came from and is the A operand of O += P V read
+// straight from TMEM (the MMAs of the issuing thread run in issue order, so
+// S(j + 2) lands in that buffer only after PV(j) has read P(j)).
+//   warp 0     bulk copies: each item's Q tile, then its K and V^T tiles into kKV stages
+//              (three: the copies run two key tiles ahead of the MMAs)
 //   warp 1     MMA issue: S(k + 1) = Q K(k + 1)^T is issued before O += P(k) V(k)
 //   warps 4 .. softmax, kSoftWarps per TMEM lane quarter: warp 4 + w + 4 x
 //              takes part x (kSoftCols key columns of S, kSoftCols channels
@@ -417,6 +421,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_gemm_full(GemmArgs a) {
 //              since the last rescale (P then stays below 256, exact in
 //              fp16); at the end y = O / l
 constexpr int kSoftWarps = 2;                      // softmax warps per TMEM lane quarter
+constexpr int kKV = 3;                             // shared-memory stages of (K, V^T) tiles
 constexpr int kSoftCols = 128 / kSoftWarps;        // key columns (and O channels) per softmax warp
 constexpr int kFlashThreads = 128 + 128 * kSoftWarps;
 constexpr float kRescaleSlack = 8.f;   // log2 units
@@ -474,26 +479,43 @@ __device__ __forceinline__ int flash_n_kt(const FlashArgs& a, int qt) {
   return (a.q_start + qt * kT + nq - 1) / kT + 1;   // key tiles holding a key visible to the tile
 }
 
+// N (16 or 32) consecutive 32-bit TMEM columns of this warp's lane quarter from registers.
+template <int N>
+__device__ __forceinline__ void tmem_st_p(uint32_t taddr, const uint32_t* v) {
+  if constexpr (N == 32) {
+    tmem_st32(taddr, reinterpret_cast<const float*>(v));
+  } else {
+    static_assert(N == 16, "16 or 32 columns");
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(
+            taddr),
+        "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]), "r"(v[8]), "r"(v[9]),
+        "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15])
+        : "memory");
+  }
+}
+
 __global__ void __launch_bounds__(kFlashThreads, 1) k_flash_prefill(FlashArgs a) {
   extern __shared__ uint8_t smem_raw[];
-  __shared__ __align__(8) uint64_t q_full, q_empty, kv_full[2], kv_empty[2], s_full[2], s_free[2], p_full, o_done,
+  __shared__ __align__(8) uint64_t q_full, q_empty, kv_full[kKV], kv_empty[kKV], s_full[2], s_free[2], p_full, o_done,
       o_free, fin;
   __shared__ uint32_t tmem_base;
   __shared__ volatile int abort_flag;
   __shared__ float xch[kSoftWarps][kT];   // per part and row: the part's row maximum, then its row sum
   uint8_t* smem = smem_raw + ((1024u - (tc::smem_u32(smem_raw) & 1023u)) & 1023u);
   uint8_t* Q_s = smem;
-  uint8_t* K_s = Q_s + kTileB;        // two stages
-  uint8_t* V_s = K_s + 2 * kTileB;    // two stages
-  uint8_t* P_s = V_s + 2 * kTileB;
+  uint8_t* K_s = Q_s + kTileB;          // kKV stages
+  uint8_t* V_s = K_s + kKV * kTileB;    // kKV stages
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int n_items = a.n_qt_used * a.H;
   if (threadIdx.x == 0) {
     tc::mbar_init(&q_full, 1);
     tc::mbar_init(&q_empty, 1);
-    for (int s = 0; s < 2; ++s) {
+    for (int s = 0; s < kKV; ++s) {
       tc::mbar_init(&kv_full[s], 1);
       tc::mbar_init(&kv_empty[s], 1);
+    }
+    for (int s = 0; s < 2; ++s) {
       tc::mbar_init(&s_full[s], 1);
       tc::mbar_init(&s_free[s], 4 * kSoftWarps);
     }
@@ -523,8 +545,8 @@ __global__ void __launch_bounds__(kFlashThreads, 1) k_flash_prefill(FlashArgs a)
         tc::mbar_expect_tx(&q_full, kTileB);
         tc::bulk_g2s(Q_s, a.Q + ((size_t)h * a.n_qt + qt) * kTileB, kTileB, &q_full);
         for (int k = 0; k < n_kt; ++k, ++jg) {
-          const int s = jg & 1;
-          if (!(ok = tc::mbar_wait_ab_lazy(&kv_empty[s], (((uint32_t)(jg >> 1)) & 1u) ^ 1u, a.status, &abort_flag)))
+          const int s = jg % kKV;
+          if (!(ok = tc::mbar_wait_ab_lazy(&kv_empty[s], (((uint32_t)(jg / kKV)) & 1u) ^ 1u, a.status, &abort_flag)))
             break;
           tc::mbar_expect_tx(&kv_full[s], 2 * kTileB);
           tc::bulk_g2s(K_s + (size_t)s * kTileB, a.K + ((size_t)g * a.n_kt + k) * kTileB, kTileB, &kv_full[s]);
@@ -533,7 +555,8 @@ __global__ void __launch_bounds__(kFlashThreads, 1) k_flash_prefill(FlashArgs a)
       }
       // let copies in flight land before the CTA can exit
       if (n > 0) tc::mbar_wait(&q_full, ((uint32_t)(n - 1)) & 1u, a.status);
-      for (int j = max(0, jg - 2); j < jg; ++j) tc::mbar_wait(&kv_full[j & 1], ((uint32_t)(j >> 1)) & 1u, a.status);
+      for (int j = max(0, jg - kKV); j < jg; ++j)
+        tc::mbar_wait(&kv_full[j % kKV], ((uint32_t)(j / kKV)) & 1u, a.status);
     }
     __syncwarp();
   } else if (warp == 1) {
@@ -542,15 +565,14 @@ __global__ void __launch_bounds__(kFlashThreads, 1) k_flash_prefill(FlashArgs a)
       const uint32_t idesc = tc::idesc_f16(128, 128, false, false, false);
       const uint64_t d0 = tc::sdesc_sw128(tc::smem_u32(smem), 0, 1024);
       const uint32_t base_lo = tc::desc_lo(d0), hi = tc::desc_hi(d0);
-      const uint32_t q_lo = base_lo, k_lo = base_lo + (kTileB >> 4), v_lo = base_lo + (3 * kTileB >> 4),
-                     p_lo = base_lo + (5 * kTileB >> 4);
-      // S(j) = Q K(j)^T into S buffer j & 1 (j counts key tiles over all items)
+      const uint32_t q_lo = base_lo, k_lo = base_lo + (kTileB >> 4), v_lo = base_lo + ((1 + kKV) * kTileB >> 4);
+      // S(j) = Q K(j)^T into S buffer j & 1 (j counts key tiles over all items; K in stage j % kKV)
       auto issue_s = [&](int j) -> bool {
-        const int s = j & 1;
-        if (!tc::mbar_wait_ab(&kv_full[s], ((uint32_t)(j >> 1)) & 1u, a.status, &abort_flag)) return false;
+        const int s = j & 1, ks = j % kKV;
+        if (!tc::mbar_wait_ab(&kv_full[ks], ((uint32_t)(j / kKV)) & 1u, a.status, &abort_flag)) return false;
         if (!tc::mbar_wait_ab(&s_free[s], (((uint32_t)(j >> 1)) & 1u) ^ 1u, a.status, &abort_flag)) return false;
         tc::tc_fence_after();
-        const uint32_t kb = k_lo + (uint32_t)(s * kTileB >> 4);
+        const uint32_t kb = k_lo + (uint32_t)(ks * kTileB >> 4);
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)
           tc::mma_f16_ss2(tmem + (uint32_t)(s * 128), q_lo + (uint32_t)(kk >> 2) * (kAtomB >> 4) + 2u * (kk & 3), hi,
@@ -573,13 +595,15 @@ __global__ void __launch_bounds__(kFlashThreads, 1) k_flash_prefill(FlashArgs a)
           if (k == 0 && !(ok = tc::mbar_wait_ab(&o_free, ((uint32_t)n & 1u) ^ 1u, a.status, &abort_flag))) break;
           if (!(ok = tc::mbar_wait_ab(&p_full, (uint32_t)(jg + k) & 1u, a.status, &abort_flag))) break;
           tc::tc_fence_after();
-          const uint32_t vb = v_lo + (uint32_t)(((jg + k) & 1) * kTileB >> 4);
+          const int pb = (jg + k) & 1;
+          const uint32_t vb = v_lo + (uint32_t)(((jg + k) % kKV) * kTileB >> 4);
+          // A = P(j) from TMEM: K = 16 keys per MMA, 8 columns of fp16 pairs
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk)
-            tc::mma_f16_ss2(tmem + o_col, p_lo + (uint32_t)(kk >> 2) * (kAtomB >> 4) + 2u * (kk & 3), hi,
-                            vb + (uint32_t)(kk >> 2) * (kAtomB >> 4) + 2u * (kk & 3), hi, idesc, (k | kk) ? 1u : 0u);
+            tc::mma_f16_ts(tmem + o_col, tmem + (uint32_t)(pb * 128 + kk * 8),
+                           vb + (uint32_t)(kk >> 2) * (kAtomB >> 4) + 2u * (kk & 3), hi, idesc, (k | kk) ? 1u : 0u);
           tc::mma_commit(&o_done);
-          tc::mma_commit(&kv_empty[(jg + k) & 1]);
+          tc::mma_commit(&kv_empty[(jg + k) % kKV]);
         }
         jg += n_kt;
       }
@@ -625,17 +649,18 @@ __global__ void __launch_bounds__(kFlashThreads, 1) k_flash_prefill(FlashArgs a)
         if (lane == 0) tc::mbar_arrive(&s_free[b]);
         // causal mask: key k * 128 + xc + c is visible to the query at `pos` if it is not later
         const int lim = pos - k * kT - (int)xc;   // columns c <= lim are visible
-        float mx = -FLT_MAX;
         if (lim < kSoftCols - 1) {
 #pragma unroll
-          for (int c = 0; c < kSoftCols; ++c) {
+          for (int c = 0; c < kSoftCols; ++c)
             if (c > lim) s[c] = -FLT_MAX;
-            mx = fmaxf(mx, s[c]);
-          }
-        } else {
-#pragma unroll
-          for (int c = 0; c < kSoftCols; ++c) mx = fmaxf(mx, s[c]);
         }
+        // maximum in eight independent chains
+        float m8[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) m8[i] = s[i];
+#pragma unroll
+        for (int c = 8; c < kSoftCols; ++c) m8[c & 7] = fmaxf(m8[c & 7], s[c]);
+        float mx = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])), fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
         // row maximum over the parts
         xch[x][r] = mx;
         asm volatile("bar.sync %0, %1;" ::"r"(bar_id), "n"(32 * kSoftWarps) : "memory");
@@ -649,20 +674,22 @@ __global__ void __launch_bounds__(kFlashThreads, 1) k_flash_prefill(FlashArgs a)
           m_used = mx;
         }
         uint32_t p2[kSoftCols / 2];
-        float ls = 0.f;
+        float l8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};   // row sum in eight independent chains
 #pragma unroll
         for (int c = 0; c < kSoftCols; c += 2) {
           const float e0 = ex2_approx(s[c] - m_used), e1 = ex2_approx(s[c + 1] - m_used);   // masked: 0
-          ls += e0 + e1;
+          l8[(c >> 1) & 7] += e0 + e1;
           p2[c / 2] = pack_half2(e0, e1);
         }
+        const float ls = ((l8[0] + l8[1]) + (l8[2] + l8[3])) + ((l8[4] + l8[5]) + (l8[6] + l8[7]));
         l = l * f + ls;
-        // the previous PV must be done before O is touched and P is overwritten
-        // (within an item; across items the end of the last one waited for it)
-        if (k > 0) {
+        // O is rescaled once the previous PV is done (rare: only when the
+        // maximum moved by more than the slack); o_done can then be at most
+        // one phase ahead of the one waited for, so skipping waits is safe
+        if (k > 0 && f != 1.f) {
           ok = ok && tc::mbar_wait_ab(&o_done, ((uint32_t)(j - 1)) & 1u, a.status, &abort_flag);
           tc::tc_fence_after();
-          if (ok && f != 1.f) {
+          if (ok) {
 #pragma unroll 1
             for (int c = 0; c < kSoftCols; c += 32) {
               float o[32];
@@ -675,11 +702,10 @@ __global__ void __launch_bounds__(kFlashThreads, 1) k_flash_prefill(FlashArgs a)
             tc::tmem_st_wait();
           }
         }
-#pragma unroll
-        for (int c8 = 0; c8 < kSoftCols / 8; ++c8)
-          *reinterpret_cast<uint4*>(P_s + tile_off(r, (int)xc + c8 * 8)) =
-              make_uint4(p2[c8 * 4], p2[c8 * 4 + 1], p2[c8 * 4 + 2], p2[c8 * 4 + 3]);
-        tc::fence_proxy_async();
+        // P into the S buffer's columns for these keys (every part has read its S:
+        // the maximum exchange above came after the loads)
+        tmem_st_p<kSoftCols / 2>(tmem + lane_base + (uint32_t)(b * 128) + xc / 2, p2);
+        tc::tmem_st_wait();
         tc::tc_fence_before();
         __syncwarp();
         if (lane == 0) tc::mbar_arrive(&p_full);
@@ -852,7 +878,7 @@ cudaError_t launch_prefill_flash(const starkv_layer* L, const uint8_t* pool, lon
   fa.y = w.y;
   fa.y_ld = v.H * 128;
   fa.status = v.status;
-  const size_t fsmem = 6 * (size_t)kTileB + 1024;
+  const size_t fsmem = (1 + 2 * kKV) * (size_t)kTileB + 1024;
   if ((e = set_smem_limit((const void*)k_flash_prefill, fsmem)) != cudaSuccess) return e;
   k_flash_prefill<<<std::min(num_sms(), n_qt * v.H), kFlashThreads, fsmem, s>>>(fa);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
