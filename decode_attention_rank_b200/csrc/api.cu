@@ -235,6 +235,7 @@ void starkv_free_layer(starkv_layer* L) {
   cudaFree(L->Bk);
   cudaFree(L->M_T);
   cudaFree(L->Bv_tiles);
+  cudaFree(L->Bk_tiles);
   cudaFree(L->Wo_tiles);
   cudaFree(L->status);
   cudaFree(L->d_items);
@@ -346,6 +347,14 @@ starkv_status starkv_load_factors(const starkv_layer_config* cfg, const void* A_
   }
   cudaError_t e = L->unfused ? launch_build_unfused(L, Bv_rot, W_o, s) : launch_fold_M(L, Bv_rot, W_o, s);
   if (e == cudaSuccess && !L->unfused && L->Bv_tiles) e = launch_build_unfused(L, Bv_rot, W_o, s);
+  // B'_k as tiles for the prefill's key rebuild (key ranks up to 64)
+  if (e == cudaSuccess && L->Bv_tiles && *std::max_element(L->key_ranks.begin(), L->key_ranks.end()) <= 64) {
+    if (cudaMalloc(&L->Bk_tiles, (size_t)v.Hkv * 16384) != cudaSuccess) {
+      if (Bv_rot) cudaFree(Bv_rot);
+      return fail(STARKV_ERR_OOM, "cudaMalloc");
+    }
+    e = launch_prefill_bk_tiles(L, L->Bk_tiles, s);
+  }
   if (Bv_rot) {
     cudaStreamSynchronize(s);
     cudaFree(Bv_rot);

@@ -12,9 +12,10 @@
 // taken through W_o after the values are rebuilt), and the attention itself
 // is the standard one over 128 x 128 tiles:
 //
+//   k_prefill_qrope    cos / sin of the chunk's query positions (shared by all heads)
 //   k_prefill_q        Q tiles: RoPE at the query positions, softmax scale * log2(e), fp16
 //   k_prefill_zk       the dequantized key latents as fp16 A tiles (r <= 64 channels, zero padded to 64)
-//   k_prefill_bkt      B'_k of every KV head as an fp16 B tile
+//   k_prefill_bkt      B'_k of every KV head as an fp16 B tile (once, at load)
 //   k_prefill_zv       the dequantized value latent as fp16 B tiles
 //   k_gemm_full        on tcgen05: K = Zhat_k B'_k with RoPE in the epilogue (K tiles); V^T tiles =
 //                      (B'_v)^T Zhat_v^T; out = y W_o
@@ -48,44 +49,46 @@ __device__ __forceinline__ uint32_t pack_half2(float a, float b) {
 }
 
 // ------------------------------------------------------------------ Q tiles
-// Query i of the chunk (position q_start + i): RoPE (rotate-half pairs, angle
-// reduced modulo 2 pi in double), times softmax scale * log2(e), as row i % 128
-// of tile [h][i / 128].  Rows past the chunk are zero.
-__global__ void __launch_bounds__(kT) k_prefill_q(LayerView v, const __nv_bfloat16* __restrict__ q, int q_len,
-                                                  int q_start, int n_qt, uint8_t* __restrict__ Qt) {
-  __shared__ double freq[64];   // theta_p
-  if (threadIdx.x < 64) freq[threadIdx.x] = exp2(-(2.0 * threadIdx.x / 128.0) * (double)v.rope_log2_theta);
-  __syncthreads();
-  const int qt = blockIdx.x, h = blockIdx.y, r = threadIdx.x;
-  const int i = qt * kT + r;
+// cos / sin of every (query, pair) of the chunk, shared by all heads: query i
+// (position q_start + i), pair p: the angle reduced modulo 2 pi in double,
+// then a float sincos.  cs[i][p] = (cos, sin).
+__global__ void k_prefill_qrope(float log2_theta, int q_len, int q_start, float2* __restrict__ cs) {
+  const int idx = blockIdx.x * blockDim.x + threadIdx.x;
+  if (idx >= q_len * 64) return;
+  const int i = idx >> 6, p = idx & 63;
+  const double ang = (double)(q_start + i) * exp2(-(2.0 * p / 128.0) * (double)log2_theta);
+  const double two_pi = 6.283185307179586476925286766559;
+  float sn, c;
+  sincosf((float)(ang - two_pi * rint(ang / two_pi)), &sn, &c);
+  cs[idx] = make_float2(c, sn);
+}
+
+// Query i of the chunk: RoPE (rotate-half pairs, cos / sin from the table;
+// none when the layer has no RoPE), times softmax scale * log2(e), as row
+// i % 128 of tile [h][i / 128].  Rows past the chunk are zero.  A thread
+// takes (row, 8-pair chunk) items of one head.
+__global__ void __launch_bounds__(256) k_prefill_q(LayerView v, const __nv_bfloat16* __restrict__ q, int q_len,
+                                                  const float2* __restrict__ cs, int n_qt, uint8_t* __restrict__ Qt) {
+  const int qt = blockIdx.x, h = blockIdx.y;
   uint8_t* tile = Qt + ((size_t)h * n_qt + qt) * kTileB;
-  // the query row: 128 bf16 in 16-byte loads (zero past the chunk)
-  uint4 row[16];
-  const uint4* qr = reinterpret_cast<const uint4*>(q + ((size_t)i * v.H + h) * 128);
-#pragma unroll
-  for (int k = 0; k < 16; ++k) row[k] = i < q_len ? qr[k] : make_uint4(0, 0, 0, 0);
-  const int pos = q_start + i;
-  for (int c8 = 0; c8 < 8; ++c8) {   // pairs p = 8 c8 .. 8 c8 + 7 and p + 64
-    const uint32_t aw[4] = {row[c8].x, row[c8].y, row[c8].z, row[c8].w};
-    const uint32_t bw[4] = {row[8 + c8].x, row[8 + c8].y, row[8 + c8].z, row[8 + c8].w};
+  for (int e = threadIdx.x; e < kT * 8; e += blockDim.x) {
+    const int r = e >> 3, c8 = e & 7;   // row, pairs p = 8 c8 .. 8 c8 + 7 (and p + 64)
+    const int i = qt * kT + r;
+    const uint4* qr = reinterpret_cast<const uint4*>(q + ((size_t)i * v.H + h) * 128);
+    const uint4 ra = i < q_len ? qr[c8] : make_uint4(0, 0, 0, 0);       // elements 8 c8 ..
+    const uint4 rb = i < q_len ? qr[8 + c8] : make_uint4(0, 0, 0, 0);   // elements 64 + 8 c8 ..
+    const uint32_t aw[4] = {ra.x, ra.y, ra.z, ra.w}, bw[4] = {rb.x, rb.y, rb.z, rb.w};
     uint32_t lo[4], hi[4];
 #pragma unroll
     for (int k = 0; k < 4; ++k) {
       float re[2], im[2];
 #pragma unroll
-      for (int e = 0; e < 2; ++e) {
-        const int p = c8 * 8 + 2 * k + e;
-        const float a = __uint_as_float(e ? aw[k] & 0xFFFF0000u : aw[k] << 16);
-        const float b = __uint_as_float(e ? bw[k] & 0xFFFF0000u : bw[k] << 16);
-        float cs = 1.f, sn = 0.f;
-        if (v.rope) {
-          // angle pos * theta_p reduced modulo 2 pi in double, then a float sincos
-          const double ang = (double)pos * freq[p];
-          const double two_pi = 6.283185307179586476925286766559;
-          sincosf((float)(ang - two_pi * rint(ang / two_pi)), &sn, &cs);
-        }
-        re[e] = (a * cs - b * sn) * v.scale_log2;
-        im[e] = (b * cs + a * sn) * v.scale_log2;
+      for (int x = 0; x < 2; ++x) {
+        const float a = __uint_as_float(x ? aw[k] & 0xFFFF0000u : aw[k] << 16);
+        const float b = __uint_as_float(x ? bw[k] & 0xFFFF0000u : bw[k] << 16);
+        const float2 t = (v.rope && i < q_len) ? cs[(size_t)i * 64 + c8 * 8 + 2 * k + x] : make_float2(1.f, 0.f);
+        re[x] = (a * t.x - b * t.y) * v.scale_log2;
+        im[x] = (b * t.x + a * t.y) * v.scale_log2;
       }
       lo[k] = pack_half2(re[0], re[1]);
       hi[k] = pack_half2(im[0], im[1]);
@@ -339,22 +342,31 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_gemm_full(GemmArgs a) {
 #pragma unroll
           for (int i = 0; i < 16; ++i) re[i] = im[i] = 0.f;
         }
+        // this row's cos / sin of channels c0 .. c0 + 15: four 16-byte loads of the table row
+        uint32_t cw[8], sw[8];
+        if (Et) {
+#pragma unroll
+          for (int h8 = 0; h8 < 2; ++h8) {
+            const uint4 c4 = *reinterpret_cast<const uint4*>(Et + tile_off(m, c0 + 8 * h8));
+            const uint4 s4 = *reinterpret_cast<const uint4*>(Et + tile_off(m, 64 + c0 + 8 * h8));
+            cw[4 * h8] = c4.x; cw[4 * h8 + 1] = c4.y; cw[4 * h8 + 2] = c4.z; cw[4 * h8 + 3] = c4.w;
+            sw[4 * h8] = s4.x; sw[4 * h8 + 1] = s4.y; sw[4 * h8 + 2] = s4.z; sw[4 * h8 + 3] = s4.w;
+          }
+        } else {
+          const __half2 one = __floats2half2_rn(1.f, 1.f), zero = __floats2half2_rn(0.f, 0.f);
+#pragma unroll
+          for (int k = 0; k < 8; ++k) {
+            cw[k] = *reinterpret_cast<const uint32_t*>(&one);
+            sw[k] = *reinterpret_cast<const uint32_t*>(&zero);
+          }
+        }
         uint32_t lo[8], hi[8];
 #pragma unroll
         for (int i = 0; i < 16; i += 2) {
-          float x0[2], y0[2];
-#pragma unroll
-          for (int e = 0; e < 2; ++e) {
-            float cs = 1.f, sn = 0.f;
-            if (Et) {
-              cs = __half2float(*reinterpret_cast<const __half*>(Et + tile_off(m, c0 + i + e)));
-              sn = __half2float(*reinterpret_cast<const __half*>(Et + tile_off(m, 64 + c0 + i + e)));
-            }
-            x0[e] = re[i + e] * cs - im[i + e] * sn;
-            y0[e] = im[i + e] * cs + re[i + e] * sn;
-          }
-          lo[i / 2] = pack_half2(x0[0], x0[1]);
-          hi[i / 2] = pack_half2(y0[0], y0[1]);
+          const float2 cs = __half22float2(*reinterpret_cast<const __half2*>(&cw[i / 2]));
+          const float2 sn = __half22float2(*reinterpret_cast<const __half2*>(&sw[i / 2]));
+          lo[i / 2] = pack_half2(re[i] * cs.x - im[i] * sn.x, re[i + 1] * cs.y - im[i + 1] * sn.y);
+          hi[i / 2] = pack_half2(im[i] * cs.x + re[i] * sn.x, im[i + 1] * cs.y + re[i + 1] * sn.y);
         }
 #pragma unroll
         for (int h8 = 0; h8 < 2; ++h8) {
@@ -751,8 +763,9 @@ __global__ void __launch_bounds__(kFlashThreads, 1) k_flash_prefill(FlashArgs a)
 size_t al256(size_t x) { return (x + 255) / 256 * 256; }
 
 struct PrefillWs {
-  uint8_t *Qt, *Kt, *Vt, *Zt, *Zk, *Bkt, *yt;
+  uint8_t *Qt, *Kt, *Vt, *Zt, *Zk, *yt;
   float* y;
+  float2* qcs;   // cos / sin per (query, pair)
 };
 
 PrefillWs prefill_ws_layout(const starkv_layer* L, void* ws, int max_T, int max_q) {
@@ -770,11 +783,11 @@ PrefillWs prefill_ws_layout(const starkv_layer* L, void* ws, int max_T, int max_
   p += al256(v.plain ? 0 : (size_t)n_kt * (v.rv / 64) * kAtomB);
   w.Zk = p;
   p += al256(v.plain ? 0 : (size_t)v.Hkv * n_kt * kAtomB);
-  w.Bkt = p;
-  p += al256(v.plain ? 0 : (size_t)v.Hkv * kAtomB);
   w.y = (float*)p;
   p += al256(sizeof(float) * (size_t)n_qt * kT * v.H * 128);
   w.yt = p;
+  p += al256((size_t)n_qt * (v.H * 128 / 64) * kAtomB);
+  w.qcs = (float2*)p;
   return w;
 }
 
@@ -784,11 +797,16 @@ PrefillWs prefill_ws_layout(const starkv_layer* L, void* ws, int max_T, int max_
 // a plain layer's output factors are W_o itself.
 static const void* prefill_wo_tiles(const starkv_layer* L) { return L->view.plain ? L->M_T : L->Wo_tiles; }
 
+cudaError_t launch_prefill_bk_tiles(const starkv_layer* L, void* tiles, cudaStream_t s) {
+  k_prefill_bkt<<<L->view.Hkv, 256, 0, s>>>(L->view, L->Bk, L->d_key_off, (uint8_t*)tiles);
+  return cudaGetLastError();
+}
+
 bool prefill_flash_supported(const starkv_layer* L) {
   const LayerView& v = L->view;
   if (v.dtype != STARKV_BF16 || v.d != 128 || !prefill_wo_tiles(L)) return false;
   if (v.plain) return true;
-  if (!L->tc_scores || !L->Bv_tiles || v.rv % 64 != 0) return false;
+  if (!L->tc_scores || !L->Bv_tiles || !L->Bk_tiles || v.rv % 64 != 0) return false;
   for (int g = 0; g < v.Hkv; ++g)
     if (L->lat[g].width > kMaxPrefillRank) return false;
   return true;
@@ -799,8 +817,8 @@ size_t prefill_flash_ws_bytes(const starkv_layer* L, int max_T, int max_q) {
   const int n_qt = (max_q + kT - 1) / kT, n_kt = (max_T + kT - 1) / kT;
   return al256((size_t)v.H * n_qt * kTileB) + 2 * al256((size_t)v.Hkv * n_kt * kTileB) +
          al256(v.plain ? 0 : (size_t)n_kt * (v.rv / 64) * kAtomB) + al256(v.plain ? 0 : (size_t)v.Hkv * n_kt * kAtomB) +
-         al256(v.plain ? 0 : (size_t)v.Hkv * kAtomB) +
-         al256(sizeof(float) * (size_t)n_qt * kT * v.H * 128) + al256((size_t)n_qt * (v.H * 128 / 64) * kAtomB);
+         al256(sizeof(float) * (size_t)n_qt * kT * v.H * 128) + al256((size_t)n_qt * (v.H * 128 / 64) * kAtomB) +
+         al256(sizeof(float2) * (size_t)n_qt * kT * 64);
 }
 
 // One chunk of q_len queries of one sequence (page table row pt_row) at
@@ -817,7 +835,11 @@ cudaError_t launch_prefill_flash(const starkv_layer* L, const uint8_t* pool, lon
   const int n_qt_l = (max_q + kT - 1) / kT, n_kt_l = (max_T + kT - 1) / kT;
   PrefillWs w = prefill_ws_layout(L, ws, max_T, max_q);
   cudaError_t e;
-  k_prefill_q<<<dim3(n_qt, v.H), kT, 0, s>>>(v, (const __nv_bfloat16*)q, q_len, q_start, n_qt_l, w.Qt);
+  if (v.rope) {
+    k_prefill_qrope<<<(q_len * 64 + 255) / 256, 256, 0, s>>>(v.rope_log2_theta, q_len, q_start, w.qcs);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  }
+  k_prefill_q<<<dim3(n_qt, v.H), 256, 0, s>>>(v, (const __nv_bfloat16*)q, q_len, w.qcs, n_qt_l, w.Qt);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   if (v.plain) {
     k_prefill_plain_kv<<<dim3(n_kt, v.Hkv), 256, 0, s>>>(v, pool, n_pages, pt_row, T, n_kt_l, w.Kt, w.Vt);
@@ -827,13 +849,11 @@ cudaError_t launch_prefill_flash(const starkv_layer* L, const uint8_t* pool, lon
     const long long nzk = (long long)v.Hkv * n_kt * kT * 8;
     k_prefill_zk<<<(unsigned)((nzk + 255) / 256), 256, 0, s>>>(v, pool, n_pages, pt_row, T, n_kt, n_kt_l, w.Zk);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    k_prefill_bkt<<<v.Hkv, 256, 0, s>>>(v, L->Bk, L->d_key_off, w.Bkt);
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
     GemmArgs gk{};
     gk.A = w.Zk;
     gk.a_step_x = kAtomB;
     gk.a_step_y = (long long)n_kt_l * kAtomB;
-    gk.B = w.Bkt;
+    gk.B = (const uint8_t*)L->Bk_tiles;
     gk.b_step_y = kAtomB;
     gk.KT = 1;
     gk.stages = 1;

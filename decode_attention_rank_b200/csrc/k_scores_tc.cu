@@ -859,10 +859,10 @@ bool plan_scores_tc(starkv_layer* L) {
     fa.sharedSizeBytes = std::max(fa.sharedSizeBytes, f1.sharedSizeBytes);
   }
   const long long budget = 232448LL - (long long)fa.sharedSizeBytes - 1024 - 2LL * kETileBytes;
-  // Two W'' stages (read from L2, short latency) and as many key stages as fit:
-  // the key copies read HBM and need the most bytes in flight.
-  L->WS = 2;
-  L->KS = (int)std::min<long long>(kMaxStages, (budget - 2LL * L->w_stage) / L->k_stage);
+  // Two or three W'' stages (read from L2) and as many key stages as fit: the
+  // key copies read HBM and need the most bytes in flight.
+  L->WS = (budget - 3LL * L->w_stage) / L->k_stage >= 3 ? 3 : 2;   // a third W'' stage when three key stages remain
+  L->KS = (int)std::min<long long>(kMaxStages, (budget - (long long)L->WS * L->w_stage) / L->k_stage);
   if (L->KS < 2) return false;
   const int mp = c.max_positions > 0 ? c.max_positions : 32768;
   L->rope_tiles = (mp + kSuper - 1) / kSuper * (kSuper / 128);

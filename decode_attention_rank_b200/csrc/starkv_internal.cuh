@@ -166,6 +166,7 @@ struct starkv_layer {
   int unfused = 0;
   void* Bv_tiles = nullptr;     // fp16 tiles [H][r_v / 64] of 128 x 64: row p, column j = B'_v[j][kv(h) d + p]
   void* Wo_tiles = nullptr;     // fp16 tiles [Dp / 128][H d / 64] of 128 x 64: row n, column k = W_o[k][n]
+  void* Bk_tiles = nullptr;     // prefill: per KV head one fp16 128 x 64 tile, row p, column j = B'_k[j][p] (j < r <= 64)
   uint32_t* status = nullptr;
   // tensor-core score kernel
   bool tc_scores = false;
@@ -271,6 +272,7 @@ cudaError_t launch_pack_rows_tiles(const void* x, int rows, int K, void* tiles, 
 cudaError_t launch_pack_rows_tiles_f32(const float* x, int rows, int K, void* tiles, cudaStream_t s, int nb = 0);
 // Tensor-core causal prefill (k_prefill.cu): one chunk of one sequence.
 bool prefill_flash_supported(const starkv_layer* L);
+cudaError_t launch_prefill_bk_tiles(const starkv_layer* L, void* tiles, cudaStream_t s);
 size_t prefill_flash_ws_bytes(const starkv_layer* L, int max_T, int max_q);
 cudaError_t launch_prefill_flash(const starkv_layer* L, const uint8_t* pool, long long n_pages, const int32_t* pt_row,
                                  int q_start, int q_len, const void* q, void* out, void* ws, int max_T, int max_q,
