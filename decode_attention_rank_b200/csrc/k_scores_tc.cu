@@ -176,6 +176,11 @@ __device__ __forceinline__ float group_dot(const uint32_t* w, uint32_t sh, float
   return scale * fmaf(kf, a - ((S0 + S1) + S2), -off);
 }
 
+template <int N, int B, int... I>
+__device__ __forceinline__ void code_floats(const uint32_t* run, uint32_t one, float* f, std::integer_sequence<int, I...>) {
+  ((f[I] = code_float<N, B, I>(run, one)), ...);
+}
+
 // TMEM -> registers: columns [C, R) of this warp's lane quarter, no wait.
 template <int C, int R>
 __device__ __forceinline__ void tmem_cols(uint32_t taddr, float* G) {
@@ -214,6 +219,58 @@ __device__ __forceinline__ void reg_fence(float* G) {
   for (int c = 0; c < R; ++c) asm volatile("" : "+f"(G[c]));
 }
 
+// The same group's part for a code run already turned into floats f[0 .. N)
+// (query heads that share a KV head share the codes: GQA decodes them once),
+// with the G columns read from TMEM 16 at a time (fewer live registers).
+template <int B, int P0, int... I>
+__device__ __forceinline__ void pairs_f(const float* f, const float* G, float2* acc, float2* ps,
+                                        std::integer_sequence<int, I...>) {
+  ((acc[I & 1] = __ffma2_rn(make_float2(f[2 * (P0 + I)], f[2 * (P0 + I) + 1]), make_float2(G[2 * I], G[2 * I + 1]),
+                            acc[I & 1]),
+    ps[place_acc<B, P0 + I>()] = __fadd2_rn(make_float2(G[2 * I], G[2 * I + 1]), ps[place_acc<B, P0 + I>()])),
+   ...);
+}
+template <int N, int B, int C = 0>
+__device__ __forceinline__ void chunks_f(const float* f, uint32_t taddr, float2* acc, float2* ps, float* tail_g) {
+  if constexpr (C < N) {
+    constexpr int n = N - C >= 16 ? 16 : N - C;
+    float G[16];
+    tmem_cols<0, n>(taddr + (uint32_t)C, G);
+    tc::tmem_ld_wait();
+    reg_fence<n>(G);
+    pairs_f<B, C / 2>(f, G, acc, ps, std::make_integer_sequence<int, n / 2>{});
+    if constexpr (n % 2) *tail_g = G[n - 1];   // the odd last channel of the group
+    chunks_f<N, B, C + 16>(f, taddr, acc, ps, tail_g);
+  }
+}
+template <int N, int B>
+__device__ __forceinline__ float group_dot_f(const float* f, float scale, uint32_t taddr) {
+  const float2 z = make_float2(0.f, 0.f);
+  float2 acc[2] = {z, z}, ps[3] = {z, z, z};
+  float gl = 0.f;
+  chunks_f<N, B>(f, taddr, acc, ps, &gl);
+  float a = (acc[0].x + acc[1].x) + (acc[0].y + acc[1].y);
+  float S0, S1, S2 = 0.f;
+  if constexpr (B == 4) {
+    S0 = ps[0].x + ps[1].x;
+    S1 = ps[0].y + ps[1].y;
+  } else {
+    S0 = ps[0].x + ps[1].y;
+    S1 = ps[0].y + ps[2].x;
+    S2 = ps[1].x + ps[2].y;
+  }
+  if constexpr (N % 2) {
+    constexpr int c = (N - 1) % tuple_len<B>();
+    a = fmaf(f[N - 1], gl, a);
+    if constexpr (c == 0) S0 += gl;
+    else if constexpr (c == 1) S1 += gl;
+    else S2 += gl;
+  }
+  constexpr float kf = (float)(1 << (tuple_len<B>() * B));
+  constexpr float h = (float)(1 << (B - 1));
+  const float off = B == 4 ? h * fmaf(16.f, S1, S0) : h * fmaf(64.f, S2, fmaf(8.f, S1, S0));
+  return scale * fmaf(kf, a - ((S0 + S1) + S2), -off);
+}
 // Groups of a segment of S channels: 32 from the segment's start, the last shorter.
 __host__ __device__ constexpr int seg_groups(int S) { return (S + 31) / 32; }
 __host__ __device__ constexpr int seg_width(int S, int g) { return (g + 1) * 32 <= S ? 32 : S - g * 32; }
@@ -262,6 +319,41 @@ __device__ __forceinline__ float segment_dot(uint32_t taddr, const uint8_t* blk,
     return group_dot<N, B, 0>(wr, bit0 & 31u, scale, G) +
            segment_dot<NHI, NLO, S, B, C0, G0, g + 1>(taddr, blk, slot);
   }
+}
+
+// segment_dot for nq (1 .. 4) consecutive query heads of one KV head: a
+// group's codes are read and turned into floats once, then dotted with each
+// head's G columns (head q at taddr + q (NHI + NLO)); sv[q] += the group's part.
+template <int NHI, int NLO, int S, int B, int C0, int G0, int g = 0>
+__device__ __forceinline__ void segment_multi(uint32_t taddr, const uint8_t* blk, int slot, int nq, float* sv) {
+  if constexpr (g < seg_groups(S)) {
+    constexpr int N = seg_width(S, g);
+    constexpr int NR = (N * B + 31) / 32;
+    constexpr int R = NHI + NLO;
+    const uint32_t bit0 = (uint32_t)slot * (uint32_t)(N * B);
+    constexpr int CO = code_block_off(NHI, NLO, G0 + g);
+    const uint32_t* w = reinterpret_cast<const uint32_t*>(blk + CO) + (bit0 >> 5);
+    constexpr int NW = (N * B) % 32 == 0 ? NR : NR + 1;
+    uint32_t wr[NR + 1];
+#pragma unroll
+    for (int k = 0; k < NW; ++k) wr[k] = w[k];
+    const float scale = __half2float(reinterpret_cast<const __half*>(blk)[(G0 + g) * kPage + slot]);
+    uint32_t run[NR];
+#pragma unroll
+    for (int k = 0; k < NR; ++k) run[k] = (N * B) % 32 == 0 ? wr[k] : __funnelshift_r(wr[k], wr[k + 1], bit0 & 31u);
+    float f[N];
+    code_floats<N, B>(run, one_bits(), f, std::make_integer_sequence<int, N>{});
+#pragma unroll
+    for (int q = 0; q < 4; ++q)
+      if (q < nq) sv[q] += group_dot_f<N, B>(f, scale, taddr + (uint32_t)(q * R + C0 + g * 32));
+    segment_multi<NHI, NLO, S, B, C0, G0, g + 1>(taddr, blk, slot, nq, sv);
+  }
+}
+
+template <int NHI, int NLO>
+__device__ __forceinline__ void head_scores_multi(uint32_t taddr, const uint8_t* blk, int slot, int nq, float* sv) {
+  segment_multi<NHI, NLO, NHI, 4, 0, 0>(taddr, blk, slot, nq, sv);
+  segment_multi<NHI, NLO, NLO, 3, NHI, seg_groups(NHI)>(taddr, blk, slot, nq, sv);
 }
 
 // The score of one token for one head whose key latent has NHI 4-bit channels
@@ -326,6 +418,73 @@ __device__ __forceinline__ float bf16_chunks(uint32_t taddr, const uint8_t* row)
   }
 }
 
+// bf16_chunks for nq consecutive query heads of one KV head (head q's G
+// columns at taddr + q R): each 16-channel chunk of the latent is loaded and
+// unpacked once.
+template <int R, int C = 0>
+__device__ __forceinline__ void bf16_chunks_multi(uint32_t taddr, const uint8_t* row, int nq, float* sv) {
+  if constexpr (C < R) {
+    constexpr int N = R - C >= 16 ? 16 : 8;
+    float z[N];
+    {
+      uint32_t w[N / 2];
+      const uint4 a = *reinterpret_cast<const uint4*>(row + 2 * C);
+      w[0] = a.x; w[1] = a.y; w[2] = a.z; w[3] = a.w;
+      if constexpr (N == 16) {
+        const uint4 b = *reinterpret_cast<const uint4*>(row + 2 * C + 16);
+        w[4] = b.x; w[5] = b.y; w[6] = b.z; w[7] = b.w;
+      }
+#pragma unroll
+      for (int k = 0; k < N / 2; ++k) {
+        z[2 * k] = __uint_as_float(w[k] << 16);
+        z[2 * k + 1] = __uint_as_float(w[k] & 0xFFFF0000u);
+      }
+    }
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      if (q < nq) {
+        float G[N];
+        tmem_cols<0, N>(taddr + (uint32_t)(q * R + C), G);
+        tc::tmem_ld_wait();
+        reg_fence<N>(G);
+        float2 acc[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+#pragma unroll
+        for (int k = 0; k < N / 2; ++k)
+          acc[k & 1] = __ffma2_rn(make_float2(z[2 * k], z[2 * k + 1]), make_float2(G[2 * k], G[2 * k + 1]), acc[k & 1]);
+        sv[q] += (acc[0].x + acc[1].x) + (acc[0].y + acc[1].y);
+      }
+    }
+    bf16_chunks_multi<R, C + N>(taddr, row, nq, sv);
+  }
+}
+
+// Scores of nq (1 .. 4) consecutive query heads sharing one KV head's latent.
+template <bool kBf16>
+__device__ __forceinline__ void head_scores_any(uint32_t taddr, const uint8_t* blk, int kind, int slot, int nq,
+                                                float* sv) {
+  if constexpr (!kBf16) {
+    switch (kind) {
+#define STARKV_CASE(i, h, l) \
+  case i: head_scores_multi<h, l>(taddr, blk, slot, nq, sv); return;
+      STARKV_HEAD_SHAPES(STARKV_CASE)
+#undef STARKV_CASE
+      default: return;
+    }
+  } else {
+    switch (kind) {
+      case kHeadShapes + 0: bf16_chunks_multi<8>(taddr, blk + slot * 16, nq, sv); return;
+      case kHeadShapes + 1: bf16_chunks_multi<16>(taddr, blk + slot * 32, nq, sv); return;
+      case kHeadShapes + 2: bf16_chunks_multi<24>(taddr, blk + slot * 48, nq, sv); return;
+      case kHeadShapes + 3: bf16_chunks_multi<32>(taddr, blk + slot * 64, nq, sv); return;
+      case kHeadShapes + 4: bf16_chunks_multi<40>(taddr, blk + slot * 80, nq, sv); return;
+      case kHeadShapes + 5: bf16_chunks_multi<48>(taddr, blk + slot * 96, nq, sv); return;
+      case kHeadShapes + 6: bf16_chunks_multi<56>(taddr, blk + slot * 112, nq, sv); return;
+      case kHeadShapes + 7: bf16_chunks_multi<64>(taddr, blk + slot * 128, nq, sv); return;
+      default: return;
+    }
+  }
+}
+
 // One layer's heads are all quantized or all bf16, so each kernel instance
 // compiles only the kinds of its format (less code for the instruction cache).
 template <bool kBf16>
@@ -374,7 +533,10 @@ constexpr int kMaxHeads = 64;
 
 
 // kDbg: write the raw scores to S_dbg instead of the softmax statistics.
-template <bool kDbg, bool kBf16>
+// kBf16: unquantized bf16 key latents.  kGqa: query heads share KV heads; the
+// heads of a run in an item that share one are scored together, the latent
+// read and decoded once.
+template <bool kDbg, bool kBf16, bool kGqa>
 __global__ void __launch_bounds__(kScoreThreads, 1) k_scores_tc(ScoreArgs a) {
   extern __shared__ uint8_t smem_raw[];
   __shared__ __align__(8) uint64_t w_full[kMaxStages], w_empty[kMaxStages], k_full[kMaxStages], k_empty[kMaxStages], e_full,
@@ -639,19 +801,43 @@ __global__ void __launch_bounds__(kScoreThreads, 1) k_scores_tc(ScoreArgs a) {
         const size_t row0 = (size_t)b * a.H + item.h0;
         __half* prow = a.P + row0 * a.P_ld + t;                          // this token's P of the item's first head
         float* mrow = a.m_st + row0 * a.n_g + (t0 >> 5) + grp32;
-        for (int hh = 0; hh < nh; ++hh, prow += a.P_ld, mrow += a.n_g) {
-          if (ok) {
-            const ScoreHead& hd = heads_s[item.h0 + hh];
-            const float sv = head_score_any<kBf16>(trow + (uint32_t)hd.gcol, page + hd.blk_rel, hd.kind, slot);
-            if constexpr (kDbg) {
-              if (valid) a.S_dbg[(row0 + hh) * a.P_ld + t] = sv;
-            } else {
-              // softmax statistics of the 32-token group: m = max s and P =
-              // exp2(s - m) rounded to fp16 (the value kernel sums the P it uses)
-              const float m = warp_max(valid ? sv : -FLT_MAX);
-              if (valid) *prow = __float2half_rn(ex2_approx(sv - m));
-              if (lane == 0) *mrow = m;
+        if constexpr (!kGqa) {
+          for (int hh = 0; hh < nh; ++hh, prow += a.P_ld, mrow += a.n_g) {
+            if (ok) {
+              const ScoreHead& hd = heads_s[item.h0 + hh];
+              const float sv = head_score_any<kBf16>(trow + (uint32_t)hd.gcol, page + hd.blk_rel, hd.kind, slot);
+              if constexpr (kDbg) {
+                if (valid) a.S_dbg[(row0 + hh) * a.P_ld + t] = sv;
+              } else {
+                // softmax statistics of the 32-token group: m = max s and P =
+                // exp2(s - m) rounded to fp16 (the value kernel sums the P it uses)
+                const float m = warp_max(valid ? sv : -FLT_MAX);
+                if (valid) *prow = __float2half_rn(ex2_approx(sv - m));
+                if (lane == 0) *mrow = m;
+              }
             }
+          }
+        } else {
+          for (int hh = 0; hh < nh;) {
+            const ScoreHead& hd = heads_s[item.h0 + hh];
+            const int nq = hd.run;
+            float sv[4] = {0.f, 0.f, 0.f, 0.f};
+            if (ok) head_scores_any<kBf16>(trow + (uint32_t)hd.gcol, page + hd.blk_rel, hd.kind, slot, nq, sv);
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              if (q < nq && ok) {
+                if constexpr (kDbg) {
+                  if (valid) a.S_dbg[(row0 + hh + q) * a.P_ld + t] = sv[q];
+                } else {
+                  const float m = warp_max(valid ? sv[q] : -FLT_MAX);
+                  if (valid) prow[(size_t)q * a.P_ld] = __float2half_rn(ex2_approx(sv[q] - m));
+                  if (lane == 0) mrow[(size_t)q * a.n_g] = m;
+                }
+              }
+            }
+            hh += nq;
+            prow += (size_t)nq * a.P_ld;
+            mrow += (size_t)nq * a.n_g;
           }
         }
         tc::tc_fence_before();
@@ -840,6 +1026,15 @@ bool plan_scores_tc(starkv_layer* L) {
       hd.gcol = it.hcol[hh];
       hd.kind = kv_kind[g];
       hd.blk_rel = ld.block_off - it.key_off;
+      hd.run = 0;
+    }
+    // runs of up to four consecutive heads of the item that share a KV head (their G columns are adjacent)
+    for (int hh = 0; hh < it.nh;) {
+      const int g = (it.h0 + hh) / v.group_q;
+      int n = 1;
+      while (hh + n < it.nh && n < 4 && (it.h0 + hh + n) / v.group_q == g) ++n;
+      L->score_heads[it.h0 + hh].run = n;
+      hh += n;
     }
     L->items.push_back(it);
   }
@@ -850,8 +1045,10 @@ bool plan_scores_tc(starkv_layer* L) {
   // dynamic shared memory: what the opt-in limit leaves beside the static
   // tables and barriers, less the alignment slack and the two RoPE tiles
   cudaFuncAttributes fa;
-  const void* fns[4] = {(const void*)k_scores_tc<false, false>, (const void*)k_scores_tc<true, false>,
-                        (const void*)k_scores_tc<false, true>, (const void*)k_scores_tc<true, true>};
+  const void* fns[8] = {(const void*)k_scores_tc<false, false, false>, (const void*)k_scores_tc<true, false, false>,
+                        (const void*)k_scores_tc<false, true, false>, (const void*)k_scores_tc<true, true, false>,
+                        (const void*)k_scores_tc<false, false, true>, (const void*)k_scores_tc<true, false, true>,
+                        (const void*)k_scores_tc<false, true, true>, (const void*)k_scores_tc<true, true, true>};
   fa.sharedSizeBytes = 0;
   for (const void* fn : fns) {
     cudaFuncAttributes f1;
@@ -935,20 +1132,25 @@ cudaError_t launch_scores_tc(const starkv_layer* L, const uint8_t* pool, long lo
   a.KS = L->KS;
   a.status = L->status;
   const size_t smem = 2 * kETileBytes + (size_t)a.WS * a.w_stage + (size_t)a.KS * a.k_stage + 1024;
-  const bool bf = !v.quantized;
-  const void* fn = S_dbg ? (bf ? (const void*)k_scores_tc<true, true> : (const void*)k_scores_tc<true, false>)
-                         : (bf ? (const void*)k_scores_tc<false, true> : (const void*)k_scores_tc<false, false>);
-  e = set_smem_limit(fn, smem);
-  if (e != cudaSuccess) return e;
   const int G = (int)std::min<long long>(num_sms(), a.U);
-  if (S_dbg && bf)
-    k_scores_tc<true, true><<<G, kScoreThreads, smem, s>>>(a);
-  else if (S_dbg)
-    k_scores_tc<true, false><<<G, kScoreThreads, smem, s>>>(a);
-  else if (bf)
-    k_scores_tc<false, true><<<G, kScoreThreads, smem, s>>>(a);
-  else
-    k_scores_tc<false, false><<<G, kScoreThreads, smem, s>>>(a);
+  const int sel = (S_dbg ? 1 : 0) | (!v.quantized ? 2 : 0) | (v.group_q > 1 ? 4 : 0);
+  switch (sel) {
+#define STARKV_SCORES_LAUNCH(k, dbg, bf, gqa)                                      \
+  case k:                                                                          \
+    e = set_smem_limit((const void*)k_scores_tc<dbg, bf, gqa>, smem);             \
+    if (e != cudaSuccess) return e;                                                \
+    k_scores_tc<dbg, bf, gqa><<<G, kScoreThreads, smem, s>>>(a);                   \
+    break;
+    STARKV_SCORES_LAUNCH(0, false, false, false)
+    STARKV_SCORES_LAUNCH(1, true, false, false)
+    STARKV_SCORES_LAUNCH(2, false, true, false)
+    STARKV_SCORES_LAUNCH(3, true, true, false)
+    STARKV_SCORES_LAUNCH(4, false, false, true)
+    STARKV_SCORES_LAUNCH(5, true, false, true)
+    STARKV_SCORES_LAUNCH(6, false, true, true)
+    STARKV_SCORES_LAUNCH(7, true, true, true)
+#undef STARKV_SCORES_LAUNCH
+  }
   return cudaGetLastError();
 }
 

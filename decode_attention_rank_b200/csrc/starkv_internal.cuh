@@ -124,7 +124,7 @@ struct ScoreHead {
   int gcol;          // G column of the head's first latent channel (item-relative)
   int kind;          // index of the compiled (hi channels, lo channels) shape
   int blk_rel;       // byte offset of the key latent block, relative to the item's key range in a page
-  int pad_;
+  int run;           // GQA: heads from this one on in the item that share its KV head (1 .. 4; 0 inside a run)
 };
 
 // Outputs of the tensor-core score kernel.
