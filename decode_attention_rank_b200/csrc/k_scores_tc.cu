@@ -25,10 +25,11 @@
 //               MMAs are issued from two schedulers (one thread issues
 //               tcgen05.mma at best every ~50 cycles); warp 1 allocates TMEM
 //   warp 2      bulk copies of the RoPE table tiles and W'' item blocks
-//   warps 3-18  epilogue, two sets of 8 warps taking alternate MMA items; in
-//               a set, warp (tile, lane quarter) owns 32 tokens of one
-//               128-token tile.  A thread scores its token for every head of
-//               the item (TMEM -> registers, dot with the 4/3-bit codes), and
+//   warps 3-18  epilogue, four sets of 4 warps, one per accumulator stage
+//               (tile 0 or 1 of the even or odd items); in a set, warp (lane
+//               quarter) owns 32 tokens of one 128-token tile.  A thread
+//               scores its token for every head of the item (TMEM ->
+//               registers, dot with the 4/3-bit codes or bf16 latent), and
 //               the warp takes the softmax statistics of its 32-token group
 //               in registers: m = max s and P = exp2(s - m) as fp16
 // Outputs per (sequence, head): P (fp16), and the maximum m of every 32-token group.
