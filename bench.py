@@ -522,10 +522,12 @@ def run_prefill(args):
     clocks.start()
     time.sleep(0.3)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.nvtx.range_push("timed")
     e0.record()
     for _ in range(args.steps):
         L.prefill(pool, n_pages, page_table, [T - n], [n], q, out, ws)
     e1.record()
+    torch.cuda.nvtx.range_pop()
     torch.cuda.synchronize()
     clk = clocks.stop()
     status = L.sync_status()
@@ -552,8 +554,8 @@ def run_prefill(args):
 
 def run_plain(args):
     """Time the decode of one uncompressed (plain) layer of the 32-layer stack
-    (K stored after RoPE and V in bf16 pages; the CUDA-core decode kernels and
-    the tensor-core output GEMM): batch and ctx from --batch/--ctx (default 16
+    (K stored after RoPE and V in bf16 pages; the streaming split-K kernel
+    k_plain_decode, the run merge and the tensor-core output GEMM): batch and ctx from --batch/--ctx (default 16
     and 4096).  Separate JSON line; not the headline metric."""
     import numpy as np
     import torch
@@ -615,10 +617,12 @@ def _time_decodes(L, pool, n_pages, page_table, lens, q, out, ws, steps, warmup)
         L.decode(pool, n_pages, page_table, lens, q, out, ws)
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.nvtx.range_push("timed")
     e0.record()
     for _ in range(steps):
         L.decode(pool, n_pages, page_table, lens, q, out, ws)
     e1.record()
+    torch.cuda.nvtx.range_pop()
     torch.cuda.synchronize()
     assert L.sync_status() == 0
     return e0.elapsed_time(e1) / steps
