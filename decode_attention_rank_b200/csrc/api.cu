@@ -68,6 +68,11 @@ using namespace starkv;
     }                                   \
   } while (0)
 
+// Buffers that kernels reach with 16-byte accesses or bulk copies (pool, q,
+// out, input, workspace) must start on a 16-byte boundary, int32 arrays on a
+// 4-byte one; a misaligned pointer is refused on the host before any launch.
+static bool aligned_to(const void* p, uintptr_t a) { return ((uintptr_t)p & (a - 1)) == 0; }
+
 #define CUDA_TRY(expr)                                                          \
   do {                                                                          \
     cudaError_t e_ = (expr);                                                    \
@@ -422,6 +427,9 @@ starkv_status starkv_append(const starkv_layer* L, void* pool, int64_t n_pages, 
   CHECK_ARG(((uintptr_t)pool & 15) == 0, "pool must be 16-byte aligned");
   CHECK_ARG(n_pages > 0 && max_pages > 0 && n_seqs > 0, "empty pool or page table");
   CHECK_ARG(max_pages <= INT_MAX / kPage, "max_pages * 16 overflows int");
+  CHECK_ARG(aligned_to(page_table, 4) && aligned_to(seq_idx, 4) && aligned_to(positions, 4),
+            "page_table, seq_idx and positions must be 4-byte aligned");
+  CHECK_ARG(aligned_to(input, 16) && aligned_to(workspace, 16), "input and workspace must be 16-byte aligned");
   cudaStream_t s = (cudaStream_t)stream;
   const float* z = (const float*)input;
   if (!input_is_latent) {
@@ -508,6 +516,10 @@ starkv_status starkv_decode_attn(const starkv_layer* L, const void* pool, int64_
   CHECK_ARG(pool && page_table && seq_lens && q && out, "NULL buffer");
   CHECK_ARG(n_pages > 0 && max_pages > 0, "empty pool or page table");
   CHECK_ARG(max_pages <= INT_MAX / kPage, "max_pages * 16 overflows int");
+  CHECK_ARG(aligned_to(pool, 16) && aligned_to(q, 16) && aligned_to(out, 16) && aligned_to(workspace, 16),
+            "pool, q, out and workspace must be 16-byte aligned");
+  CHECK_ARG(aligned_to(page_table, 4) && aligned_to(seq_lens, 4) && aligned_to(q_pos, 4),
+            "page_table, seq_lens and q_pos must be 4-byte aligned");
   const int max_len = max_pages * kPage;
   const bool tc_ok = L->tc_scores && max_len <= L->rope_tiles * 128;
   const bool use_tc_all = tc_ok && L->tc_values && L->decode_path == 0;
@@ -540,6 +552,9 @@ starkv_status starkv_prefill_attn(const starkv_layer* L, const void* pool, int64
   CHECK_ARG(pool && page_table && q_start_host && q_len_host && q && out, "NULL buffer");
   CHECK_ARG(n_pages > 0 && max_pages > 0, "empty pool or page table");
   CHECK_ARG(max_pages <= INT_MAX / kPage, "max_pages * 16 overflows int");
+  CHECK_ARG(aligned_to(pool, 16) && aligned_to(q, 16) && aligned_to(out, 16) && aligned_to(workspace, 16),
+            "pool, q, out and workspace must be 16-byte aligned");
+  CHECK_ARG(aligned_to(page_table, 4), "page_table must be 4-byte aligned");
   std::vector<int32_t> tab;
   int rows = 0, max_len = 0;
   for (int b = 0; b < batch; ++b) {

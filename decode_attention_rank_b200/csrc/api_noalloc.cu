@@ -65,6 +65,12 @@ extern "C" starkv_status starkv_decode_attn_noalloc(const starkv_layer* L, const
     set_error("max_pages * 16 overflows int");
     return STARKV_ERR_ARG;
   }
+  // the alignment rules of starkv_decode_attn, checked before the scratch lookup
+  if ((((uintptr_t)pool | (uintptr_t)q | (uintptr_t)out) & 15) != 0 ||
+      (((uintptr_t)page_table | (uintptr_t)seq_lens | (uintptr_t)q_pos) & 3) != 0) {
+    set_error("pool, q and out must be 16-byte aligned, page_table, seq_lens and q_pos 4-byte aligned");
+    return STARKV_ERR_ARG;
+  }
   const size_t need = starkv_workspace_bytes(L, batch, max_pages * kPage, 1);
   if (need > STARKV_NOALLOC_SCRATCH_BYTES) {
     set_error("decode needs " + std::to_string(need) + " bytes of scratch; the built-in array holds " +

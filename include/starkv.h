@@ -18,6 +18,10 @@
  *   - Pointers named *host* are host memory; every other buffer pointer is
  *     device memory on the current CUDA device.  The caller owns all of them.
  *   - Row-major layouts; sizes are element counts unless stated in bytes.
+ *   - Alignment: the pool, q, out, input and workspace buffers of the
+ *     append, decode and prefill calls start on a 16-byte boundary, their
+ *     int32 arrays on a 4-byte one (cudaMalloc and framework allocators give
+ *     both).  A misaligned pointer returns STARKV_ERR_ARG before any launch.
  *   - Calls are asynchronous on `stream` (a cudaStream_t; NULL = legacy
  *     default stream) and never allocate device memory, except
  *     starkv_load_factors, which allocates the layer's own folded factors.

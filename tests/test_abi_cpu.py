@@ -88,3 +88,35 @@ def test_page_table_capacity_overflow_rejected_on_the_host():
     assert "overflows" in raw.starkv_last_error().decode()
     assert raw.starkv_append(p, p, 1, p, 1, big, 1, p, p, p, 1, p, 0, None) == 1
     assert "overflows" in raw.starkv_last_error().decode()
+
+
+def test_misaligned_buffers_rejected_on_the_host():
+    # 16-byte device buffers and 4-byte int32 arrays: a pointer off its boundary is refused with
+    # STARKV_ERR_ARG before the layer is read or any CUDA call is made (dummy host pointers, never
+    # dereferenced).
+    from decode_attention_rank_b200 import starkv as lib
+    raw = lib.raw_lib()
+    dummy = ctypes.create_string_buffer(4096 + 64)
+    p = (ctypes.cast(dummy, ctypes.c_void_p).value + 15) // 16 * 16
+    for off in (2, 8):
+        m = p + off
+        assert raw.starkv_decode_attn(p, p, 1, p, 1, 1, p, None, m, p, p, 1 << 20, None) == 1     # q
+        assert "aligned" in raw.starkv_last_error().decode()
+        assert raw.starkv_decode_attn(p, p, 1, p, 1, 1, p, None, p, m, p, 1 << 20, None) == 1     # out
+        assert raw.starkv_decode_attn(p, p, 1, p, 1, 1, p, None, p, p, m, 1 << 20, None) == 1     # workspace
+        assert raw.starkv_decode_attn(p, m, 1, p, 1, 1, p, None, p, p, p, 1 << 20, None) == 1     # pool
+        assert raw.starkv_decode_attn_noalloc(p, p, 1, p, 1, 1, p, None, m, p, None) == 1         # q
+        assert "aligned" in raw.starkv_last_error().decode()
+        assert raw.starkv_prefill_attn(p, p, 1, p, 1, 1, p, p, m, p, p, 1 << 20, None) == 1       # q
+        assert "aligned" in raw.starkv_last_error().decode()
+        assert raw.starkv_append(p, p, 1, p, 1, 1, 1, p, p, m, 1, p, 0, None) == 1                # input
+        assert "aligned" in raw.starkv_last_error().decode()
+    # int32 arrays off a 4-byte boundary
+    assert raw.starkv_decode_attn(p, p, 1, p + 2, 1, 1, p, None, p, p, p, 1 << 20, None) == 1      # page_table
+    assert raw.starkv_decode_attn(p, p, 1, p, 1, 1, p + 1, None, p, p, p, 1 << 20, None) == 1      # seq_lens
+    assert raw.starkv_decode_attn(p, p, 1, p, 1, 1, p, p + 2, p, p, p, 1 << 20, None) == 1         # q_pos
+    assert raw.starkv_decode_attn_noalloc(p, p, 1, p + 2, 1, 1, p, None, p, p, None) == 1
+    assert raw.starkv_prefill_attn(p, p, 1, p + 2, 1, 1, p, p, p, p, p, 1 << 20, None) == 1
+    assert raw.starkv_append(p, p, 1, p, 1, 1, 1, p + 2, p, p, 1, p, 0, None) == 1               # seq_idx
+    assert raw.starkv_append(p, p, 1, p, 1, 1, 1, p, p + 2, p, 1, p, 0, None) == 1               # positions
+    assert "aligned" in raw.starkv_last_error().decode()
