@@ -265,3 +265,21 @@ def test_cpp_decode_plain_matches_numpy():
     K, V = Z[:, :32], Z[:, 32:]
     np.testing.assert_allclose(C.decode_plain(spec, f, K, V, q, 23, 22), O.decode_plain(spec, f, K, V, q, 23, 22),
                                rtol=1e-11, atol=1e-13)
+
+
+@pytest.mark.parametrize("top_fraction,top_bits,bottom_bits,group_size,hadamard", [
+    (0.25, 4, 3, 32, True), (0.2, 4, 3, 32, True), (1.0, 4, 3, 32, True), (0.0, 4, 3, 32, False),
+    (0.25, 8, 2, 16, True), (0.5, 5, 6, 7, False), (0.3, 2, 8, 1, False), (0.25, 4, 3, 24, True)])
+def test_cpp_matches_numpy_formats_across_bit_splits(top_fraction, top_bits, bottom_bits, group_size, hadamard):
+    # The two oracles agree on group layout, rotation and stored bytes for every bit split, group size and
+    # rank tried: the 20:80 and 25:75 splits of the pages, uniform widths, odd group sizes, ragged segments.
+    spec = _quant_spec(top_fraction=top_fraction, top_bits=top_bits, bottom_bits=bottom_bits,
+                       group_size=group_size, hadamard_block=group_size if hadamard else 0)
+    for r in (1, 2, 3, 8, 17, 31, 33, 40, 64, 97, 130):
+        assert [(g.start, g.n, g.bits) for g in O.groups(r, spec)] == C.groups(r, spec), r
+        np.testing.assert_array_equal(C.rotation(r, spec), O.rotation(r, spec))
+        Z = (gen.normals(gen.stream_key(11, r), 16 * r) * 1.5).astype(np.float32).reshape(16, r)
+        Z[3, : (r + 1) // 2] = 0.0             # an all-zero head of a token (zero scale)
+        for cm in (False, True):
+            np.testing.assert_array_equal(C.pack_block(Z, r, spec, cm), O.pack_block(Z, r, spec, cm))
+        np.testing.assert_array_equal(C.stored_values(Z, r, spec), O.stored_values(Z, r, spec))
