@@ -51,6 +51,21 @@ def workload_label(spec, B, ctx):
     return f"batch {B}, ctx ~{ctx} ({name} layer: {shape}, {store}, 16-token pages)"
 
 
+def tail_start(ctx, W, K):
+    """Tokens cached before the run: W warm-up and K timed steps then append one token each, filling the last
+    pages up to ctx."""
+    return ctx - 16 * ((W + K + 15) // 16)
+
+
+def decode_config(spec, B, ctx, W, K, ws, unfused):
+    """The `config` of the decode-step line (both arms print the same one)."""
+    T0 = tail_start(ctx, W, K)
+    return {"workload": "STAR-KV decode step: append 1 token/seq + decode, " + workload_label(spec, B, ctx)
+                        + (", unfused value output y_h B_v,h then W_o" if unfused else ""),
+            "batch": B, "ctx": ctx, "ctx_range": [T0 + W + 1, T0 + W + K], "parallelism": f"replicas x{ws}",
+            "l2": "inputs larger than L2 (the latent cache and M, read once per step)"}
+
+
 def measured_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -323,7 +338,7 @@ def run_ours(args, rank, ws, local):
     K, W = args.steps, args.warmup
     spec, f, L = build_layer(unfused=args.unfused)
     tail_pages = (W + K + 15) // 16
-    T0 = ctx - 16 * tail_pages      # each step appends one token at T0 + i and decodes T0 + i + 1 tokens
+    T0 = tail_start(ctx, W, K)      # each step appends one token at T0 + i and decodes T0 + i + 1 tokens
     pool, n_pages, page_table, page_table_e2e = fill_cache(spec, f, L, B, T0, rank, ctx, tail_pages)
     dev = torch.device("cuda", torch.cuda.current_device())
     stream = torch.cuda.current_stream()
@@ -440,11 +455,8 @@ def run_ours(args, rank, ws, local):
         "dtype": ("u3/u4 latent codes + fp16 scales, bf16 factors/q/out, fp32 accumulate" if spec.quantized
                   else "bf16 latents/factors/q/out, fp32 accumulate"),
         "data": "synthetic (seeded latents with the factor spectrum; random-init factors)",
-        "config": {"workload": "STAR-KV decode step: append 1 token/seq + decode, " + workload_label(spec, B, ctx)
-                               + (", unfused value output y_h B_v,h then W_o" if args.unfused else ""),
-                   "batch": B, "ctx": ctx, "ctx_range": [T0 + W + 1, T0 + W + K], "parallelism": f"replicas x{ws}",
-                   "l2": "inputs larger than L2 (cache %.0f MB + M %.0f MB)" % (B * ctx * L.bytes_per_token / 1e6,
-                                                                            L.factor_bytes / 1e6)},
+        "config": decode_config(spec, B, ctx, W, K, ws, args.unfused),
+        "input_bytes": {"latent_cache": B * ctx * L.bytes_per_token, "factors": L.factor_bytes, "l2": 126 << 20},
         "us_per_layer_step": ms_step * 1e3,
         "decode_us": dec_ms * 1e3,
         "roofline": {"bound": "hbm", "kernel": PHASES[dom], "achieved": kernels[dom]["GB/s"], "peak": peak,
@@ -474,7 +486,8 @@ def run_ours(args, rank, ws, local):
 
 
 def run_reference(args, rank, ws):
-    """The oracle, as it stands, on the host cores: one sequence per step."""
+    """The oracle, as it stands, on the host cores: one sequence of the workload per step, reported on the
+    decode step's own config."""
     if rank != 0:
         return None
     B, ctx = WORKLOAD["batch"], WORKLOAD["ctx"]
@@ -491,10 +504,10 @@ def run_reference(args, rank, ws):
     return {"metric": METRIC, "value": v, "unit": "tokens/s", "n_gpus": ws, "steps": K, "warmup": W,
             "ms_per_step": dt * 1e3, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "f64", "data": "synthetic", "impl": "reference",
-            "config": {"workload": f"oracle decode of 1 sequence per step at ctx {T} (sample of batch {B})",
-                       "batch": 1, "ctx": T},
+            "config": decode_config(workload_spec(), B, ctx, W, K, ws, args.unfused),
             "cpu_baseline": {"value": v, "unit": "tokens/s", "cores": cores, "kind": "oracle",
-                             "sample": f"1 of {B} sequences per step at ctx {T}"},
+                             "sample": f"1 of the {B} sequences per step, decoded at ctx {T} by the float64 C++ "
+                                       "oracle (explicit K/V reconstruction + softmax attention + W_o)"},
             "e2e": {"value": v, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
 
 
