@@ -50,8 +50,6 @@ template <>
 __device__ __forceinline__ float ldf<__nv_bfloat16>(const __nv_bfloat16* p, size_t i) {
   return __bfloat162float(p[i]);
 }
-template <>
-__device__ __forceinline__ float ldf<__half>(const __half* p, size_t i) { return __half2float(p[i]); }
 
 // qrot[row][h][p] = RoPE(q, pos)[p] * scale * log2(e)
 template <typename T>

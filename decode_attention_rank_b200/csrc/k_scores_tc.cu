@@ -391,7 +391,6 @@ __host__ __device__ constexpr int shape_lo(int k) {
 // load (a tail of 8), the bf16 pairs of a word split into two floats.
 constexpr int kBf16Kinds = 8;
 __host__ __device__ constexpr bool kind_is_bf16(int k) { return k >= kHeadShapes; }
-__host__ __device__ constexpr int bf16_kind_rank(int k) { return 8 * (k - kHeadShapes + 1); }
 
 template <int R, int C = 0>
 __device__ __forceinline__ float bf16_chunks(uint32_t taddr, const uint8_t* row) {
