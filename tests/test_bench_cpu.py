@@ -52,3 +52,16 @@ def test_phase_bytes_and_flops_by_hand():
 def test_job_throughput():
     assert bench.job_tokens_per_s(16, 1, 0.5) == pytest.approx(32000.0)
     assert bench.job_tokens_per_s(16, 8, 0.5) == pytest.approx(256000.0)
+
+
+def test_reference_arm_reports_the_decode_steps_config():
+    # Both arms print one config: the workload of the decode step (the oracle's sample is described in
+    # cpu_baseline.sample, not in config).
+    import argparse
+    args = argparse.Namespace(steps=1, warmup=0, ref_ctx=64, unfused=False)
+    res = bench.run_reference(args, 0, 1)
+    B, ctx = bench.WORKLOAD["batch"], bench.WORKLOAD["ctx"]
+    assert res["config"] == bench.decode_config(bench.workload_spec(), B, ctx, 0, 1, 1, False)
+    assert res["impl"] == "reference" and res["cpu_baseline"]["kind"] == "oracle"
+    assert res["e2e"]["h2d_bytes_per_step"] == 0 and res["value"] > 0
+    assert bench.run_reference(args, 1, 2) is None          # only rank 0 runs it
