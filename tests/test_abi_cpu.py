@@ -120,3 +120,22 @@ def test_misaligned_buffers_rejected_on_the_host():
     assert raw.starkv_append(p, p, 1, p, 1, 1, 1, p + 2, p, p, 1, p, 0, None) == 1               # seq_idx
     assert raw.starkv_append(p, p, 1, p, 1, 1, 1, p, p + 2, p, 1, p, 0, None) == 1               # positions
     assert "aligned" in raw.starkv_last_error().decode()
+
+
+def test_binding_argument_counts_match_the_header():
+    # Every entry point the binding declares argtypes for takes as many arguments as include/starkv.h says.
+    from decode_attention_rank_b200 import starkv as lib
+    text = open(os.path.join(ROOT, "include", "starkv.h")).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    sigs = dict(re.findall(r"STARKV_API\s+[\w\s\*]+?\b(starkv_\w+)\s*\(([^)]*)\)", text))
+    raw = lib.raw_lib()
+    checked = 0
+    for name, params in sigs.items():
+        argtypes = getattr(raw, name).argtypes
+        if argtypes is None:
+            continue
+        p = params.strip()
+        n = 0 if p in ("", "void") else len(p.split(","))
+        assert len(argtypes) == n, (name, len(argtypes), n)
+        checked += 1
+    assert checked >= 15
